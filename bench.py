@@ -1,0 +1,468 @@
+#!/usr/bin/env python
+"""Benchmark of the HSA hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl hsa|reference]
+
+Headline step: one ``hsa_fwd`` (pool -> select -> chunk attention + fusion)
+over the 64K-token workload (B=1, L=65536, S=64, K=8, h_q=16, h_kv=2, d=128,
+bf16, per-chunk key offsets), inputs resident in HBM, L2 flushed (256 MB
+write) before every timed step.  Prints ONE JSON line on rank 0.
+
+Also measured in the same run (keys "decode" and "train"): the decode step at
+B=16 with a 16K-token cache (median of CUDA-graph replays) and one
+forward+backward step of the B=4, L=16K training workload.
+
+Multi-GPU (torchrun): each rank runs its own sequence (the (batch, group)
+units are independent: no collective on the data path), weak scaling; time is
+the max over ranks of the device time.
+
+``--impl reference`` times the fp64 CPU oracle (the only reference this
+method has) on a bounded row sample of the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "HSA fwd tokens/s at L=64K and fraction of roofline; decode step latency at B=16"
+FLUSH_BYTES = 256 << 20
+
+
+# --------------------------------------------------------------------------- helpers
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": j["hbm_gbs"], "bf16_tflops": j["bf16_tflops"],
+                "bf16_tflops_sustained": j.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+def selected_pairs(wl) -> int:
+    """sum over (b, t, g) of min(K, eligible chunks): the (token, group, slot) triples."""
+    t = np.arange(wl.L)
+    ne = np.minimum(t // wl.S, wl.n_c)
+    return int(wl.B * wl.h_kv * np.minimum(ne, wl.K).sum())
+
+
+def eligible_pairs(wl) -> int:
+    t = np.arange(wl.L)
+    return int(wl.B * wl.h_kv * np.minimum(t // wl.S, wl.n_c).sum())
+
+
+def fwd_work(wl):
+    """Algorithmic FLOPs and compulsory bytes of one forward (selected pairs only)."""
+    G = wl.h_q // wl.h_kv
+    att_flops = selected_pairs(wl) * G * 4 * wl.S * wl.d
+    sel_flops = eligible_pairs(wl) * 2 * wl.d
+    eb = 2 if wl.dtype == "bf16" else 4
+    tok = wl.B * wl.L
+    kv = 2 * wl.B * wl.h_kv * wl.L * wl.d * eb
+    q = tok * wl.h_q * wl.d * eb
+    qs = tok * wl.h_kv * wl.d * eb
+    kbar = wl.B * wl.h_kv * wl.n_c * wl.d * 4
+    byt = q + qs + kv + q + 2 * kbar  # q, q_slc, k, v read; o written; kbar written + read
+    return att_flops, sel_flops, byt
+
+
+def source_hash(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:12]
+
+
+def read_traffic(kernel_file: str):
+    """Per-launch DRAM bytes of the dominant kernel from the committed ncu
+    summary, if it was taken on the current source (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(p):
+        return None
+    want = source_hash([kernel_file])
+    for ln in open(p):
+        m = re.match(r"\s*(\S+)\s+source=(\w+)\s+bytes_per_launch=(\d+)", ln)
+        if m and m.group(1) == os.path.basename(kernel_file) and m.group(2) == want:
+            return int(m.group(3))
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def __exit__(self, *a):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- reference arm
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    import oracle
+    from chunked_hierarchical_sparse_b200 import synth
+    wl = synth.WORKLOADS["fwd64k"]
+    x = synth.make_inputs(wl)
+    kbar = oracle.pool(x["k"], wl.S)
+    rng = np.random.default_rng(0)
+    n_rows = args.ref_rows
+    times = []
+    for i in range(args.warmup + args.steps):
+        rows = np.sort(rng.choice(wl.B * wl.L, size=n_rows, replace=False))
+        t0 = time.perf_counter()
+        oracle.fwd(x["q"], x["k"], x["v"], x["q_slc"], kbar, wl.S, wl.K, rows=rows)
+        dt = time.perf_counter() - t0
+        if i >= args.warmup:
+            times.append(dt)
+    tot = sum(times)
+    value = n_rows * len(times) / tot
+    cores = oracle.num_threads()
+    sample = f"{n_rows} uniformly sampled token rows of the 64K workload per step (pool once per run)"
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "impl": "reference",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * tot / len(times), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "fwd64k", "B": wl.B, "L": wl.L, "S": wl.S, "K": wl.K,
+                       "h_q": wl.h_q, "h_kv": wl.h_kv, "d": wl.d, "global_batch": wl.B,
+                       "seq_len": wl.L},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------- hsa arm
+def cpu_baseline(wl, x, budget_s: float):
+    """Time the oracle as it stands on a bounded row sample of the workload."""
+    import oracle
+    kbar = oracle.pool(x["k"], wl.S)
+    rng = np.random.default_rng(1)
+    probe = np.sort(rng.choice(wl.B * wl.L, size=64, replace=False))
+    t0 = time.perf_counter()
+    oracle.fwd(x["q"], x["k"], x["v"], x["q_slc"], kbar, wl.S, wl.K, rows=probe)
+    per_row = (time.perf_counter() - t0) / 64
+    n = int(min(wl.B * wl.L, max(64, budget_s / max(per_row, 1e-9))))
+    rows = np.sort(rng.choice(wl.B * wl.L, size=n, replace=False))
+    t0 = time.perf_counter()
+    oracle.fwd(x["q"], x["k"], x["v"], x["q_slc"], kbar, wl.S, wl.K, rows=rows)
+    dt = time.perf_counter() - t0
+    return {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{n} uniformly sampled token rows of the 64K workload ({dt:.1f} s)"}
+
+
+def to_dev(a, dev, bf16=True):
+    import torch
+    return torch.from_numpy(a).to(dev, torch.bfloat16 if bf16 else torch.float32)
+
+
+def bench_decode(hsa, dev, reps=1000):
+    import torch
+    from chunked_hierarchical_sparse_b200 import synth
+    wl = synth.WORKLOADS["decode16k"]
+    x = synth.make_inputs(wl)
+    q, qs, kc, vc = (to_dev(x[n], dev) for n in ("q", "q_slc", "k", "v"))
+    kbar = hsa.hsa_pool(kc)
+    o = torch.empty_like(q)
+    n = hsa.hsa_workspace_size(wl.B, wl.L, wl.h_q, wl.h_kv, wl.d, wl.S, wl.K, torch.bfloat16,
+                               hsa.OP_DECODE)
+    ws = torch.empty(n, dtype=torch.uint8, device=dev)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for _ in range(3):
+            hsa.hsa_decode(q, qs, kc, vc, kbar, wl.K, o=o, ws=ws, want_sel=False)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        hsa.hsa_decode(q, qs, kc, vc, kbar, wl.K, o=o, ws=ws, want_sel=False)
+    for _ in range(20):
+        g.replay()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for a, b in ev:
+        a.record()
+        g.replay()
+        b.record()
+    torch.cuda.synchronize()
+    warm = sorted(a.elapsed_time(b) * 1e3 for a, b in ev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    cold = []
+    for i in range(50):
+        flush.fill_(float(i))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        cold.append(a.elapsed_time(b) * 1e3)
+    cold.sort()
+    del g
+    # kernel-only time of the decode kernel (timing facility, warm)
+    hsa.hsa_timing_enable(True)
+    for _ in range(50):
+        hsa.hsa_decode(q, qs, kc, vc, kbar, wl.K, o=o, ws=ws, want_sel=False)
+    torch.cuda.synchronize()
+    kms, kn = hsa.hsa_timing_read("decode")
+    hsa.hsa_timing_enable(False)
+    eb = 2
+    sel_bytes = wl.B * wl.h_kv * wl.K * 2 * wl.S * wl.d * eb
+    byt = (x["q"].size + x["q_slc"].size) * eb + wl.B * wl.h_kv * wl.n_c * wl.d * 4 + sel_bytes + x["q"].size * eb
+    return {"workload": "decode16k", "B": wl.B, "P": wl.L, "unit": "us",
+            "median_us_warm_graph": warm[len(warm) // 2], "p10_us_warm": warm[len(warm) // 10],
+            "p90_us_warm": warm[9 * len(warm) // 10], "median_us_cold_l2": cold[len(cold) // 2],
+            "replays": reps, "kernel_us": 1e3 * kms / max(kn, 1),
+            "compulsory_bytes": int(byt), "roofline_us": byt / (load_peaks()["hbm_gbs"] * 1e9) * 1e6}
+
+
+def bench_train(hsa, dev, steps=3):
+    import torch
+    from chunked_hierarchical_sparse_b200 import synth
+    wl = synth.WORKLOADS["train16k"]
+    x = synth.make_inputs(wl)
+    t = {n: to_dev(x[n], dev) for n in ("q", "k", "v", "q_slc", "dO")}
+    del x
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def step():
+        o, lse, idx, w, kbar = hsa.hsa_fwd(t["q"], t["k"], t["v"], t["q_slc"], wl.K)
+        return hsa.hsa_bwd(t["q"], t["k"], t["v"], t["q_slc"], t["dO"], lse, idx, w, kbar, wl.K)
+
+    step()
+    torch.cuda.synchronize()
+    times = []
+    hsa.hsa_timing_enable(True)
+    for i in range(steps):
+        flush.fill_(float(i))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        step()
+        b.record()
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+    per_kernel = {k: round(hsa.hsa_timing_read(k)[0] / steps, 4) for k in
+                  ("pool", "select", "attend_simt", "attend_tc", "plan", "bwd1", "invert", "bwd2")}
+    hsa.hsa_timing_enable(False)
+    att, sel, _ = fwd_work(wl)
+    G = wl.h_q // wl.h_kv
+    bwd_flops = selected_pairs(wl) * G * 12 * wl.S * wl.d
+    ms = float(np.median(times))
+    flops = att + sel + bwd_flops
+    return {"workload": "train16k", "ms_per_step": ms, "tokens_per_s": wl.B * wl.L / (ms / 1e3),
+            "algorithmic_tflop": flops / 1e12,
+            "roofline_ms": flops / (load_peaks()["bf16_tflops"] * 1e12) * 1e3,
+            "kernel_ms_per_step": per_kernel}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="hsa", choices=["hsa", "reference"])
+    ap.add_argument("--ref-rows", type=int, default=4096)
+    ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    ap.add_argument("--no-extras", action="store_true", help="skip the decode and train measurements")
+    ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    args = ap.parse_args()
+    assert args.warmup >= 3 or args.impl == "reference", "at least 3 warm-up steps"
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+
+    import torch
+    import torch.distributed as dist
+    import chunked_hierarchical_sparse_b200 as hsa
+    from chunked_hierarchical_sparse_b200 import synth
+
+    if world > 1:
+        torch.cuda.set_device(local)
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+    dev = torch.device("cuda", local if world > 1 else 0)
+    torch.cuda.set_device(dev)
+    hsa.load_library()
+
+    base = synth.WORKLOADS["fwd64k"]
+    wl = base.scaled(seed=base.seed + 100 * rank)  # one independent sequence per rank
+    x = synth.make_inputs(wl)
+    q, k, v, qs = (to_dev(x[n], dev) for n in ("q", "k", "v", "q_slc"))
+    o = torch.empty_like(q)
+    nws = hsa.hsa_workspace_size(wl.B, wl.L, wl.h_q, wl.h_kv, wl.d, wl.S, wl.K, torch.bfloat16, hsa.OP_FWD)
+    ws = torch.empty(nws, dtype=torch.uint8, device=dev)
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def fwd():
+        hsa.hsa_fwd(q, k, v, qs, wl.K, want_lse=False, want_sel=False, o=o, ws=ws)
+
+    for i in range(args.warmup):
+        flush.fill_(float(i))
+        fwd()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    hsa.hsa_timing_enable(True)
+    with ClockSampler(dev.index) as clocks:
+        for i, (a, b) in enumerate(ev):
+            flush.fill_(float(i))
+            a.record()
+            fwd()
+            b.record()
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    kern = {name: hsa.hsa_timing_read(name) for name in hsa.KERNELS}
+    hsa.hsa_timing_enable(False)
+    assert hsa.hsa_device_status(ws) == 0, "device status set during the timed region"
+    dev_ms = sum(step_ms)
+    t = torch.tensor([dev_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+    tokens = world * wl.B * wl.L * args.steps
+    value = tokens / (max_ms / 1e3)
+
+    # dominant kernel: the chunk attention (whichever path ran)
+    att_name = "attend_tc" if kern["attend_tc"][1] > 0 else "attend_simt"
+    att_ms, att_n = kern[att_name]
+    att_flops, sel_flops, comp_bytes = fwd_work(wl)
+    peaks = load_peaks()
+    achieved = att_flops / (att_ms / att_n / 1e3) / 1e12 if att_n else 0.0
+    att_src = ("chunked_hierarchical_sparse_b200/csrc/k_attend_tc.cu" if att_name == "attend_tc"
+               else "chunked_hierarchical_sparse_b200/csrc/k_attend_simt.cu")
+    roof_us = max((att_flops + sel_flops) / (peaks["bf16_tflops"] * 1e12),
+                  comp_bytes / (peaks["hbm_gbs"] * 1e9)) * 1e6
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "fwd64k", "B": wl.B, "L": wl.L, "S": wl.S, "K": wl.K, "h_q": wl.h_q,
+                   "h_kv": wl.h_kv, "d": wl.d, "global_batch": wl.B * world, "seq_len": wl.L,
+                   "parallelism": f"dp{world} (independent sequences)",
+                   "l2": "flushed (256 MB write) before every timed step"},
+        "q_heads_per_s": value * wl.h_q,
+        "roofline_fraction_step": roof_us / (max_ms / args.steps * 1e3),
+        "roofline_step_us": roof_us,
+        "roofline": {"bound": "tensor", "kernel": att_name, "achieved": achieved,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": achieved / peaks["bf16_tflops"],
+                     "traffic": read_traffic(att_src),
+                     "peak_source": f"{peaks['source']} bf16 dense (burst)",
+                     "algorithmic_flops_per_launch": att_flops,
+                     "avg_launch_us": 1e3 * att_ms / max(att_n, 1)},
+        "kernel_us_per_step": {n: round(1e3 * ms / args.steps, 2) for n, (ms, c) in kern.items() if c},
+        "gpu_launches": int(sum(c for _, c in kern.values())),
+        "clocks": clocks.summary(),
+    }
+
+    # end to end through the public API: pinned host inputs -> device -> fwd -> host output
+    hq = {n: torch.from_numpy(x[n]).to(torch.bfloat16).pin_memory() for n in ("q", "k", "v", "q_slc")}
+    ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    e2e = []
+    for i in range(4):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        q.copy_(hq["q"], non_blocking=True)
+        k.copy_(hq["k"], non_blocking=True)
+        v.copy_(hq["v"], non_blocking=True)
+        qs.copy_(hq["q_slc"], non_blocking=True)
+        fwd()
+        ho.copy_(o, non_blocking=True)
+        b.record()
+        torch.cuda.synchronize()
+        if i:
+            e2e.append(a.elapsed_time(b))
+    h2d = sum(t_.numel() * t_.element_size() for t_ in hq.values())
+    e2e_ms = float(np.median(e2e))
+    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    line["e2e"] = {"value": world * wl.B * wl.L / (float(te.item()) / 1e3), "unit": "tokens/s",
+                   "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(ho.numel() * ho.element_size())}
+    del hq, ho
+
+    if not args.no_extras:
+        line["decode"] = bench_decode(hsa, dev)
+        line["train"] = bench_train(hsa, dev)
+    if rank == 0 and world == 1 and not args.no_cpu:
+        line["cpu_baseline"] = cpu_baseline(wl, x, args.cpu_budget_s)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,259 @@
+// hsa_api.cu -- the extern "C" entry points declared in include/hsa.h:
+// argument checks, workspace carving, and the kernel sequence of each call.
+#include <cstring>
+
+#include "hsa_internal.cuh"
+
+namespace hsa {
+
+// ------------------------------------------------------------------ checks
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static hsa_status_t check_shape(const hsa_shape_t *s, bool decode) {
+    if (!s) return HSA_ERR_INVALID_ARG;
+    if (s->B < 0 || s->L < 0 || s->h_q < 1 || s->h_kv < 1 || s->d < 1 || s->S < 1 || s->K < 1)
+        return HSA_ERR_INVALID_ARG;
+    if (s->h_q % s->h_kv != 0) return HSA_ERR_INVALID_ARG;
+    if (s->dtype != HSA_F32 && s->dtype != HSA_BF16) return HSA_ERR_INVALID_ARG;
+    if (s->S != kChunk) return HSA_ERR_UNSUPPORTED;
+    if (s->d != 64 && s->d != 128) return HSA_ERR_UNSUPPORTED;
+    if (s->K > kMaxK || s->h_q / s->h_kv > kMaxG) return HSA_ERR_UNSUPPORTED;
+    // entries pack t * 16 + slot into int32; list offsets are int32
+    if ((int64_t)s->L * 16 >= ((int64_t)1 << 31) || (int64_t)s->L * s->K >= ((int64_t)1 << 31))
+        return HSA_ERR_UNSUPPORTED;
+    if ((int64_t)s->B * s->h_kv > 65535 && !decode) return HSA_ERR_UNSUPPORTED;  // grid.y
+    return HSA_OK;
+}
+
+// all pointers in the list must be non-null and 16-byte aligned
+static bool ptrs_ok(std::initializer_list<const void *> ps) {
+    for (const void *p : ps)
+        if (!p || !aligned16(p)) return false;
+    return true;
+}
+static bool opt_ok(const void *p) { return !p || aligned16(p); }
+
+// ------------------------------------------------------------------ workspace
+struct Carver {
+    char *base;
+    size_t off = kWsHeader;
+    template <typename T> T *take(size_t count) {
+        T *p = base ? reinterpret_cast<T *>(base + off) : nullptr;
+        off += round_up((int64_t)(count * sizeof(T)), 256);
+        return p;
+    }
+};
+
+struct FwdWs {
+    float *kbar;
+    int32_t *idx;
+    float *w;
+};
+
+static FwdWs carve_fwd(const Shape &sh, void *ws, size_t *bytes) {
+    Carver c{static_cast<char *>(ws)};
+    FwdWs f;
+    f.kbar = c.take<float>((size_t)sh.B * sh.hkv * sh.nc * sh.d);
+    f.idx = c.take<int32_t>((size_t)sh.B * sh.L * sh.hkv * sh.K);
+    f.w = c.take<float>((size_t)sh.B * sh.L * sh.hkv * sh.K);
+    if (bytes) *bytes = c.off;
+    return f;
+}
+
+static BwdWs carve_bwd(const Shape &sh, void *ws, size_t *bytes) {
+    Carver c{static_cast<char *>(ws)};
+    BwdWs b;
+    const int ntb = (int)ceil_div(sh.L, kInvTokBlock);
+    b.dkbar = c.take<float>((size_t)sh.B * sh.hkv * sh.nc * sh.d);
+    b.delta = c.take<float>((size_t)sh.B * sh.L * sh.hq * sh.K);
+    b.dk_acc = c.take<float>((size_t)sh.B * sh.hkv * sh.L * sh.d);
+    b.dv_acc = c.take<float>((size_t)sh.B * sh.hkv * sh.L * sh.d);
+    b.hist = c.take<int32_t>((size_t)sh.B * sh.hkv * ntb * sh.nc);
+    b.chunk_off = c.take<int32_t>((size_t)sh.B * sh.hkv * (sh.nc + 1));
+    b.seg_off = c.take<int32_t>((size_t)sh.B * sh.hkv * (sh.nc + 1));
+    b.entries = c.take<int32_t>((size_t)sh.B * sh.hkv * sh.L * sh.K);
+    if (bytes) *bytes = c.off;
+    return b;
+}
+
+static size_t ws_size(const Shape &sh, int op) {
+    size_t bytes = kWsHeader;
+    switch (op) {
+        case HSA_OP_POOL:
+        case HSA_OP_SELECT:
+        case HSA_OP_DECODE:
+            return bytes;
+        case HSA_OP_FWD:
+            carve_fwd(sh, nullptr, &bytes);
+            return bytes;
+        case HSA_OP_BWD:
+            carve_bwd(sh, nullptr, &bytes);
+            return bytes;
+        default:
+            return 0;
+    }
+}
+
+static hsa_status_t check_ws(const Shape &sh, int op, void *ws, size_t ws_bytes) {
+    if (!ws || (reinterpret_cast<uintptr_t>(ws) & 255u)) return HSA_ERR_INVALID_ARG;
+    if (ws_bytes < ws_size(sh, op)) return HSA_ERR_WORKSPACE;
+    return HSA_OK;
+}
+
+static hsa_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? HSA_OK : HSA_ERR_CUDA; }
+
+// A problem with no tokens reads and writes nothing: its tensors may be empty
+// (null data pointers); only the workspace status word is cleared.
+static hsa_status_t empty_call(const Shape &sh, int op, void *ws, size_t ws_bytes, cudaStream_t st) {
+    hsa_status_t s = check_ws(sh, op, ws, ws_bytes);
+    if (s != HSA_OK) return s;
+    return cuda_status(cudaMemsetAsync(ws, 0, sizeof(DevStatus), st));
+}
+
+static cudaError_t clear_status(void *ws, cudaStream_t st) {
+    return cudaMemsetAsync(ws, 0, sizeof(DevStatus), st);
+}
+
+// run a launcher inside a timing bracket of `kind` covering `n` kernel launches
+template <typename F> static cudaError_t timed(int kind, int n, cudaStream_t st, F &&f) {
+    TimedLaunch tl(kind, n, st);
+    return f();
+}
+
+}  // namespace hsa
+
+using namespace hsa;
+
+extern "C" {
+
+size_t hsa_workspace_size(const hsa_shape_t *shape, int op) {
+    if (check_shape(shape, op == HSA_OP_DECODE) != HSA_OK) return 0;
+    return ws_size(make_shape(*shape), op);
+}
+
+hsa_status_t hsa_pool(const hsa_shape_t *shape, const void *k, float *kbar, void *ws, size_t ws_bytes,
+                      void *stream) {
+    hsa_status_t s = check_shape(shape, false);
+    if (s != HSA_OK) return s;
+    const Shape sh = make_shape(*shape);
+    if ((int64_t)sh.B * sh.L == 0) return empty_call(sh, HSA_OP_POOL, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+    if (!ptrs_ok({k, kbar})) return HSA_ERR_INVALID_ARG;
+    if ((s = check_ws(sh, HSA_OP_POOL, ws, ws_bytes)) != HSA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    DevStatus *ds = static_cast<DevStatus *>(ws);
+    cudaError_t e = clear_status(ws, st);
+    if (e == cudaSuccess) e = timed(HSA_K_POOL, 1, st, [&] { return launch_pool(sh, k, kbar, ds, st); });
+    return cuda_status(e);
+}
+
+hsa_status_t hsa_select(const hsa_shape_t *shape, const void *q_slc, const void *k, float *kbar,
+                        int32_t *idx, float *w, void *ws, size_t ws_bytes, void *stream) {
+    hsa_status_t s = check_shape(shape, false);
+    if (s != HSA_OK) return s;
+    const Shape sh = make_shape(*shape);
+    if ((int64_t)sh.B * sh.L == 0) return empty_call(sh, HSA_OP_SELECT, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+    if (!ptrs_ok({q_slc, k, kbar, idx, w})) return HSA_ERR_INVALID_ARG;
+    if ((s = check_ws(sh, HSA_OP_SELECT, ws, ws_bytes)) != HSA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    DevStatus *ds = static_cast<DevStatus *>(ws);
+    cudaError_t e = clear_status(ws, st);
+    if (e == cudaSuccess) e = timed(HSA_K_POOL, 1, st, [&] { return launch_pool(sh, k, kbar, ds, st); });
+    if (e == cudaSuccess) e = timed(HSA_K_SELECT, 1, st, [&] { return launch_select_simt(sh, q_slc, kbar, idx, w, ds, st); });
+    return cuda_status(e);
+}
+
+hsa_status_t hsa_fwd(const hsa_shape_t *shape, const void *q, const void *k, const void *v,
+                     const void *q_slc, void *o, float *lse, int32_t *idx, float *w, float *kbar,
+                     void *ws, size_t ws_bytes, void *stream) {
+    hsa_status_t s = check_shape(shape, false);
+    if (s != HSA_OK) return s;
+    const Shape sh = make_shape(*shape);
+    if ((int64_t)sh.B * sh.L == 0) return empty_call(sh, HSA_OP_FWD, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+    if (!ptrs_ok({q, k, v, q_slc, o}) || !opt_ok(lse) || !opt_ok(idx) || !opt_ok(w) || !opt_ok(kbar))
+        return HSA_ERR_INVALID_ARG;
+    if ((s = check_ws(sh, HSA_OP_FWD, ws, ws_bytes)) != HSA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    DevStatus *ds = static_cast<DevStatus *>(ws);
+    FwdWs f = carve_fwd(sh, ws, nullptr);
+    if (kbar) f.kbar = kbar;
+    if (idx) f.idx = idx;
+    if (w) f.w = w;
+    cudaError_t e = clear_status(ws, st);
+    if (e == cudaSuccess) e = timed(HSA_K_POOL, 1, st, [&] { return launch_pool(sh, k, f.kbar, ds, st); });
+    if (e == cudaSuccess) e = timed(HSA_K_SELECT, 1, st, [&] { return launch_select_simt(sh, q_slc, f.kbar, f.idx, f.w, ds, st); });
+    if (e == cudaSuccess) e = timed(HSA_K_ATTEND_SIMT, 1, st, [&] { return launch_attend_simt(sh, q, k, v, f.idx, f.w, o, lse, ds, st); });
+    return cuda_status(e);
+}
+
+hsa_status_t hsa_decode(const hsa_shape_t *shape, const void *q, const void *q_slc,
+                        const void *k_cache, const void *v_cache, const float *kbar, void *o,
+                        int32_t *idx, float *w, void *ws, size_t ws_bytes, void *stream) {
+    hsa_status_t s = check_shape(shape, true);
+    if (s != HSA_OK) return s;
+    const Shape sh = make_shape(*shape);
+    if (sh.B == 0) return empty_call(sh, HSA_OP_DECODE, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+    if (!ptrs_ok({q, q_slc, k_cache, v_cache, o}) || !opt_ok(idx) || !opt_ok(w)) return HSA_ERR_INVALID_ARG;
+    if (sh.nc > 0 && !ptrs_ok({kbar})) return HSA_ERR_INVALID_ARG;
+    if ((s = check_ws(sh, HSA_OP_DECODE, ws, ws_bytes)) != HSA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    DevStatus *ds = static_cast<DevStatus *>(ws);
+    cudaError_t e = clear_status(ws, st);
+    if (e == cudaSuccess) e = timed(HSA_K_DECODE, 1, st, [&] { return launch_decode_simt(sh, q, q_slc, k_cache, v_cache, kbar, o, idx, w, ds, st); });
+    return cuda_status(e);
+}
+
+hsa_status_t hsa_bwd(const hsa_shape_t *shape, const void *q, const void *k, const void *v,
+                     const void *q_slc, const void *dO, const float *lse, const int32_t *idx,
+                     const float *w, const float *kbar, void *dq, void *dk, void *dv,
+                     void *dq_slc, void *ws, size_t ws_bytes, void *stream) {
+    hsa_status_t s = check_shape(shape, false);
+    if (s != HSA_OK) return s;
+    const Shape sh = make_shape(*shape);
+    if ((int64_t)sh.B * sh.L == 0) return empty_call(sh, HSA_OP_BWD, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+    if (!ptrs_ok({q, k, v, q_slc, dO, lse, idx, w, dq, dk, dv, dq_slc})) return HSA_ERR_INVALID_ARG;
+    if (sh.nc > 0 && !ptrs_ok({kbar})) return HSA_ERR_INVALID_ARG;
+    if ((s = check_ws(sh, HSA_OP_BWD, ws, ws_bytes)) != HSA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    DevStatus *ds = static_cast<DevStatus *>(ws);
+    BwdWs b = carve_bwd(sh, ws, nullptr);
+    cudaError_t e = clear_status(ws, st);
+    const size_t acc_bytes = sizeof(float) * (size_t)sh.B * sh.hkv * sh.L * sh.d;
+    if (e == cudaSuccess && sh.nc > 0)
+        e = cudaMemsetAsync(b.dkbar, 0, sizeof(float) * (size_t)sh.B * sh.hkv * sh.nc * sh.d, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(b.dk_acc, 0, acc_bytes, st);
+    if (e == cudaSuccess) e = cudaMemsetAsync(b.dv_acc, 0, acc_bytes, st);
+    if (e == cudaSuccess)
+        e = timed(HSA_K_BWD1, 1, st, [&] {
+            return launch_bwd_phase1(sh, q, q_slc, k, v, dO, lse, idx, w, kbar, dq, dq_slc, b, ds, st);
+        });
+    if (e == cudaSuccess) e = timed(HSA_K_INVERT, sh.nc > 0 ? 3 : 0, st, [&] { return launch_invert(sh, idx, b, ds, st); });
+    if (e == cudaSuccess)
+        e = timed(HSA_K_BWD2, sh.nc > 0 ? 2 : 1, st, [&] { return launch_bwd_phase2(sh, q, k, v, dO, lse, w, dk, dv, b, ds, st); });
+    return cuda_status(e);
+}
+
+hsa_status_t hsa_device_status(const void *ws, int32_t *code_out, void *stream) {
+    if (!ws || !code_out) return HSA_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    DevStatus h;
+    cudaError_t e = cudaMemcpyAsync(&h, ws, sizeof(h), cudaMemcpyDeviceToHost, st);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return HSA_ERR_CUDA;
+    *code_out = h.code;
+    return HSA_OK;
+}
+
+const char *hsa_status_string(int32_t code) {
+    switch (code) {
+        case HSA_OK: return "ok";
+        case HSA_ERR_INVALID_ARG: return "invalid argument";
+        case HSA_ERR_UNSUPPORTED: return "unsupported shape";
+        case HSA_ERR_WORKSPACE: return "workspace too small";
+        case HSA_ERR_CUDA: return "CUDA launch or API error";
+        case HSA_ERR_TIMEOUT: return "device wait timed out";
+        case HSA_ERR_DEVICE_CHECK: return "device-side input check failed";
+        default: return "unknown status";
+    }
+}
+
+}  // extern "C"

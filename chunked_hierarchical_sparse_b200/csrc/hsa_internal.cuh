@@ -1,0 +1,135 @@
+// hsa_internal.cuh -- shared device helpers and launcher declarations of the
+// HSA CUDA library.  Nothing here is visible through the C ABI.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/hsa.h"
+
+namespace hsa {
+
+constexpr int kChunk = 64;     // S: the only chunk size built (fixed on the pages)
+constexpr int kMaxK = 16;      // top-K bound
+constexpr int kMaxG = 16;      // query heads per KV group bound
+constexpr size_t kWsHeader = 256;
+
+// ---------------------------------------------------------------- status word
+// The first bytes of every workspace: code (first error wins) and details.
+struct DevStatus {
+    int32_t code;
+    int32_t where;  // kernel id that reported
+    int32_t a, b;   // details (e.g. the offending index)
+};
+
+enum KernelId : int32_t {
+    kKPool = 1, kKSelect = 2, kKAttendSimt = 3, kKDecode = 4, kKBwd1 = 5, kKInvert = 6,
+    kKBwd2 = 7, kKAttendTc = 8, kKFinal = 9, kKSelectTc = 10
+};
+
+__device__ __forceinline__ void report(DevStatus *st, int32_t code, int32_t where, int32_t a,
+                                       int32_t b) {
+    if (atomicCAS(&st->code, 0, code) == 0) {
+        st->where = where;
+        st->a = a;
+        st->b = b;
+    }
+}
+
+// ---------------------------------------------------------------- element access
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+    __device__ __forceinline__ static float load(const float *p) { return *p; }
+    __device__ __forceinline__ static void store(float *p, float v) { *p = v; }
+};
+template <> struct Elem<__nv_bfloat16> {
+    __device__ __forceinline__ static float load(const __nv_bfloat16 *p) { return __bfloat162float(*p); }
+    __device__ __forceinline__ static void store(__nv_bfloat16 *p, float v) { *p = __float2bfloat16_rn(v); }
+};
+
+__host__ __device__ constexpr inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+__host__ __device__ constexpr inline int64_t round_up(int64_t a, int64_t b) { return ceil_div(a, b) * b; }
+
+// ---------------------------------------------------------------- shapes
+struct Shape {
+    int B, L, hq, hkv, d, S, K, G, nc;
+    bool bf16;
+};
+
+inline Shape make_shape(const hsa_shape_t &s) {
+    Shape r;
+    r.B = s.B; r.L = s.L; r.hq = s.h_q; r.hkv = s.h_kv; r.d = s.d; r.S = s.S; r.K = s.K;
+    r.G = s.h_kv > 0 ? s.h_q / s.h_kv : 0;
+    r.nc = s.S > 0 ? s.L / s.S : 0;
+    r.bf16 = s.dtype == HSA_BF16;
+    return r;
+}
+
+// ---------------------------------------------------------------- launch helpers
+// Raise a kernel's dynamic shared-memory limit to `bytes` once (cached per
+// kernel, so repeated calls -- and calls during stream capture -- make no
+// runtime API call once the limit has been set).
+cudaError_t set_smem_once(const void *func, size_t bytes);
+
+// ---------------------------------------------------------------- timing
+// RAII bracket: records a CUDA event pair around the launches made in its
+// scope when hsa_timing_enable(1) is in force (see timing.cu).
+class TimedLaunch {
+  public:
+    TimedLaunch(int kind, int nlaunch, cudaStream_t st);
+    ~TimedLaunch();
+    TimedLaunch(const TimedLaunch &) = delete;
+    TimedLaunch &operator=(const TimedLaunch &) = delete;
+
+  private:
+    int kind_, nlaunch_;
+    cudaStream_t st_;
+    cudaEvent_t a_ = nullptr, b_ = nullptr;
+    bool active_ = false;
+};
+
+// ---------------------------------------------------------------- launchers
+// All launchers enqueue on `st` and return the launch's cudaError_t.
+cudaError_t launch_pool(const Shape &sh, const void *k, float *kbar, DevStatus *ds, cudaStream_t st);
+
+cudaError_t launch_select_simt(const Shape &sh, const void *q_slc, const float *kbar, int32_t *idx,
+                               float *w, DevStatus *ds, cudaStream_t st);
+
+cudaError_t launch_attend_simt(const Shape &sh, const void *q, const void *k, const void *v,
+                               const int32_t *idx, const float *w, void *o, float *lse,
+                               DevStatus *ds, cudaStream_t st);
+
+// Decode: shape.L = P.  idx_out / w_out may point into the workspace.
+cudaError_t launch_decode_simt(const Shape &sh, const void *q, const void *q_slc, const void *kc,
+                               const void *vc, const float *kbar, void *o, int32_t *idx_out,
+                               float *w_out, DevStatus *ds, cudaStream_t st);
+
+// Backward pieces.
+struct BwdWs {
+    float *dkbar;     // [B,hkv,nc,d] fp32 accumulator (zeroed by the launcher)
+    float *delta;     // [B,L,hq,K]  dO . O_k per (token, head, slot)
+    float *dk_acc;    // [B,hkv,L,d] fp32 accumulators (zeroed by the launcher)
+    float *dv_acc;
+    int32_t *hist;    // [B,hkv,ntb,nc] per token-block counts -> offsets
+    int32_t *chunk_off;  // [B,hkv,nc+1] CSR offsets into entries (per (b,g) base)
+    int32_t *seg_off;    // [B,hkv,nc+1] phase-2 segment offsets (kBwdSeg entries each)
+    int32_t *entries;    // [B,hkv, L*K] packed t*16 + slot, sorted by t per chunk
+};
+
+cudaError_t launch_bwd_phase1(const Shape &sh, const void *q, const void *q_slc, const void *k,
+                              const void *v, const void *dO, const float *lse, const int32_t *idx,
+                              const float *w, const float *kbar, void *dq, void *dq_slc,
+                              const BwdWs &ws, DevStatus *ds, cudaStream_t st);
+
+cudaError_t launch_invert(const Shape &sh, const int32_t *idx, const BwdWs &ws, DevStatus *ds,
+                          cudaStream_t st);
+
+cudaError_t launch_bwd_phase2(const Shape &sh, const void *q, const void *k, const void *v,
+                              const void *dO, const float *lse, const float *w, void *dk, void *dv,
+                              const BwdWs &ws, DevStatus *ds, cudaStream_t st);
+
+constexpr int kInvTokBlock = 256;  // tokens per histogram block of the inversion
+constexpr int kBwdSeg = 32;        // list entries per phase-2 block
+
+}  // namespace hsa

@@ -1,0 +1,187 @@
+// k_select.cu -- chunk pooling and chunk selection on CUDA cores.
+//
+// Cited page: "Hardware-aligned Hierarchical Sparse Attention for Efficient
+// Long-term Memory Access" (paper notes), §HSA "Chunk Selection": every token
+// scores the mean-pooled key of each chunk with its selection query and each
+// query group keeps its own top-K; §HSA second stage: stick-breaking weights
+// from the sigmoid of the score.  §training/inference: the chunk index is
+// floor(L/S) x d per KV head.
+#include "hsa_internal.cuh"
+#include "topk_warp.cuh"
+
+namespace hsa {
+
+// ------------------------------------------------------------------ pooling
+// One block per (b, g, chunk).  16-byte vector loads along d; each thread sums
+// its columns over a strided set of the chunk's rows in fp64, the partial sums
+// are combined in shared memory, and the mean is rounded once to fp32.  The
+// fp64 sum of 64 bf16 values is exact, so the result does not depend on the
+// summation order.
+template <typename T>
+__global__ void __launch_bounds__(256) pool_kernel(const T *__restrict__ k, float *__restrict__ kbar,
+                                                   int L, int d, int nc) {
+    constexpr int VEC = 16 / sizeof(T);
+    __shared__ double red[256 * VEC];
+    const int64_t bgc = blockIdx.x;
+    const int c = (int)(bgc % nc);
+    const int64_t bg = bgc / nc;
+    const T *src = k + (bg * L + (int64_t)c * kChunk) * d;
+    const int lanes_per_row = d / VEC;
+    const int rows_par = blockDim.x / lanes_per_row;
+    const int lr = threadIdx.x % lanes_per_row;
+    const int r0 = threadIdx.x / lanes_per_row;
+    double acc[VEC];
+#pragma unroll
+    for (int e = 0; e < VEC; ++e) acc[e] = 0.0;
+    if (r0 < rows_par) {
+        for (int r = r0; r < kChunk; r += rows_par) {
+            const uint4 raw = *reinterpret_cast<const uint4 *>(src + (int64_t)r * d + lr * VEC);
+            const T *vals = reinterpret_cast<const T *>(&raw);
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) acc[e] += (double)Elem<T>::load(vals + e);
+        }
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) red[r0 * d + lr * VEC + e] = acc[e];
+    }
+    __syncthreads();
+    for (int j = threadIdx.x; j < d; j += blockDim.x) {
+        double s = 0.0;
+        for (int r = 0; r < rows_par; ++r) s += red[r * d + j];
+        kbar[bgc * d + j] = (float)(s / kChunk);
+    }
+}
+
+cudaError_t launch_pool(const Shape &sh, const void *k, float *kbar, DevStatus *, cudaStream_t st) {
+    const int64_t blocks = (int64_t)sh.B * sh.hkv * sh.nc;
+    if (blocks == 0) return cudaSuccess;
+    if (sh.bf16)
+        pool_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(
+            (const __nv_bfloat16 *)k, kbar, sh.L, sh.d, sh.nc);
+    else
+        pool_kernel<float><<<(unsigned)blocks, 256, 0, st>>>((const float *)k, kbar, sh.L, sh.d, sh.nc);
+    return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ selection
+// Block = 64 tokens of one (b, g); 256 threads.  Chunk tiles of 64 pooled keys
+// are scored as a 64x64 fp32 tile (4x4 per thread), then each warp merges its
+// 8 tokens' rows into running top-K lists kept in shared memory.
+constexpr int kSelTok = 64;
+constexpr int kSelCh = 64;
+
+template <typename T>
+__global__ void __launch_bounds__(256) select_simt_kernel(
+    const T *__restrict__ q_slc, const float *__restrict__ kbar, int32_t *__restrict__ idx,
+    float *__restrict__ w, int L, int hkv, int d, int nc, int K) {
+    extern __shared__ float4 smem4[];
+    float *sm = reinterpret_cast<float *>(smem4);
+    float *qT = sm;                                 // [d][64]
+    float *kT = qT + d * kSelTok;                   // [d][64]
+    float *sc = kT + d * kSelCh;                    // [64][65]
+    float *best_s = sc + kSelTok * (kSelCh + 1);    // [64][kMaxK]
+    int *best_c = reinterpret_cast<int *>(best_s + kSelTok * kMaxK);
+
+    const int bg = blockIdx.y;
+    const int b = bg / hkv, g = bg % hkv;
+    const int t0 = blockIdx.x * kSelTok;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const float scale = 1.0f / sqrtf((float)d);
+
+    for (int e = tid; e < kSelTok * d; e += blockDim.x) {
+        const int tt = e / d, j = e % d, t = t0 + tt;
+        qT[j * kSelTok + tt] = (t < L) ? Elem<T>::load(q_slc + (((int64_t)b * L + t) * hkv + g) * d + j) : 0.f;
+    }
+    for (int e = tid; e < kSelTok * kMaxK; e += blockDim.x) {
+        best_s[e] = -CUDART_INF_F;
+        best_c[e] = -1;
+    }
+    const int tlast = min(t0 + kSelTok, L) - 1;
+    const int ne_max = min(tlast / kChunk, nc);
+    const int ty = tid / 16, tx = tid % 16;
+    const float *kb = kbar + (int64_t)bg * nc * d;
+
+    for (int c0 = 0; c0 < ne_max; c0 += kSelCh) {
+        __syncthreads();
+        for (int e = tid; e < kSelCh * d; e += blockDim.x) {
+            const int cc = e / d, j = e % d;
+            kT[j * kSelCh + cc] = (c0 + cc < nc) ? kb[(int64_t)(c0 + cc) * d + j] : 0.f;
+        }
+        __syncthreads();
+        float acc[4][4];
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb) acc[a][bb] = 0.f;
+        for (int j = 0; j < d; ++j) {
+            const float4 qa = *reinterpret_cast<const float4 *>(qT + j * kSelTok + ty * 4);
+            const float4 ka = *reinterpret_cast<const float4 *>(kT + j * kSelCh + tx * 4);
+            const float qv[4] = {qa.x, qa.y, qa.z, qa.w};
+            const float kv[4] = {ka.x, ka.y, ka.z, ka.w};
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                for (int bb = 0; bb < 4; ++bb) acc[a][bb] = fmaf(qv[a], kv[bb], acc[a][bb]);
+        }
+#pragma unroll
+        for (int a = 0; a < 4; ++a)
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb) sc[(ty * 4 + a) * (kSelCh + 1) + tx * 4 + bb] = acc[a][bb] * scale;
+        __syncthreads();
+        for (int tt = warp * 8; tt < warp * 8 + 8; ++tt) {
+            const int t = t0 + tt;
+            if (t >= L) break;
+            const int ne = min(t / kChunk, nc);
+            const int ca = c0 + lane, cb = c0 + lane + 32;
+            const float sa = sc[tt * (kSelCh + 1) + lane];
+            const float sb = sc[tt * (kSelCh + 1) + lane + 32];
+            float ls = (lane < K) ? best_s[tt * kMaxK + lane] : CUDART_INF_F;
+            int lc = (lane < K) ? best_c[tt * kMaxK + lane] : 0x7fffffff;
+            topk_merge(K, sa, ca < ne ? ca : -1, sb, cb < ne ? cb : -1, ls, lc);
+            if (lane < K) {
+                best_s[tt * kMaxK + lane] = ls;
+                best_c[tt * kMaxK + lane] = lc;
+            }
+        }
+    }
+    __syncthreads();
+    for (int tt = warp * 8; tt < warp * 8 + 8; ++tt) {
+        const int t = t0 + tt;
+        if (t >= L) break;
+        const float ls = (lane < K) ? best_s[tt * kMaxK + lane] : -CUDART_INF_F;
+        const int lc = (lane < K) ? best_c[tt * kMaxK + lane] : -1;
+        int sc_; float sw, ss;
+        topk_finish(K, ls, lc, sc_, sw, ss);
+        if (lane < K) {
+            const int64_t o = (((int64_t)b * L + t) * hkv + g) * K + lane;
+            idx[o] = sc_;
+            w[o] = sw;
+        }
+    }
+}
+
+size_t select_simt_smem(int d) {
+    return sizeof(float) * ((size_t)d * kSelTok + (size_t)d * kSelCh + kSelTok * (kSelCh + 1) +
+                            kSelTok * kMaxK) + sizeof(int) * kSelTok * kMaxK;
+}
+
+cudaError_t launch_select_simt(const Shape &sh, const void *q_slc, const float *kbar, int32_t *idx,
+                               float *w, DevStatus *, cudaStream_t st) {
+    if (sh.B == 0 || sh.L == 0) return cudaSuccess;
+    dim3 grid((unsigned)ceil_div(sh.L, kSelTok), (unsigned)(sh.B * sh.hkv));
+    const size_t smem = select_simt_smem(sh.d);
+    cudaError_t e;
+    if (sh.bf16) {
+        e = set_smem_once((const void *)select_simt_kernel<__nv_bfloat16>, (size_t)(smem));
+        if (e != cudaSuccess) return e;
+        select_simt_kernel<__nv_bfloat16><<<grid, 256, smem, st>>>(
+            (const __nv_bfloat16 *)q_slc, kbar, idx, w, sh.L, sh.hkv, sh.d, sh.nc, sh.K);
+    } else {
+        e = set_smem_once((const void *)select_simt_kernel<float>, (size_t)(smem));
+        if (e != cudaSuccess) return e;
+        select_simt_kernel<float><<<grid, 256, smem, st>>>((const float *)q_slc, kbar, idx, w, sh.L,
+                                                           sh.hkv, sh.d, sh.nc, sh.K);
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace hsa

@@ -63,16 +63,14 @@ def _rng(seed: int, tensor: str, attempt: int = 0) -> np.random.Generator:
 
 
 def round_to(x: np.ndarray, dtype: str) -> np.ndarray:
-    """Round fp64 values to the workload dtype; return them widened to fp64."""
+    """Round fp64 values to the workload dtype (fp64 -> fp32 -> bf16, each step
+    round-to-nearest-even); return them widened back to fp64."""
+    import torch
     if dtype == "f32":
         return x.astype(np.float32).astype(np.float64)
     if dtype == "bf16":
-        # round-to-nearest-even on the fp32 bit pattern (fp64 -> fp32 first)
-        f = np.ascontiguousarray(x, dtype=np.float32)
-        u = f.view(np.uint32).astype(np.uint64)
-        u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16
-        out = (u.astype(np.uint32) << 16).view(np.float32)
-        return out.astype(np.float64)
+        f = torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32))
+        return f.to(torch.bfloat16).to(torch.float64).numpy()
     raise ValueError(dtype)
 
 

@@ -1,0 +1,250 @@
+"""GPU parity: the CUDA library (through the C ABI) against the fp64 oracle.
+
+Bars (fixed in advance, not tuned to results):
+  chunk indices           bit-exact (the gap rule leaves no near-ties)
+  pooled keys             bit-exact (fp64 sum of bf16/fp32 values, one fp32 rounding)
+  fp32 outputs            max |err| <= 1e-5
+  bf16 outputs            max |err| <= 2e-2 and relative L2 <= 5e-3
+  bf16 gradients          relative L2 <= 5e-3 and max |err| <= 2e-2 * max(1, max|ref|)
+                          (a bf16 rounding of a value v moves it by up to |v| 2^-9)
+  selection weights w     |err| <= 1e-5 (fp32 sigmoid products of fp32 scores)
+"""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from chunked_hierarchical_sparse_b200 import synth
+from hsa_testutil import cached_workload, gap_ruled
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda:0"
+
+
+def hsa():
+    import chunked_hierarchical_sparse_b200 as m
+    m.load_library()
+    return m
+
+
+def to_dev(a: np.ndarray, dtype: str) -> torch.Tensor:
+    t = torch.from_numpy(np.ascontiguousarray(a))
+    return t.to(device=DEV, dtype=torch.bfloat16 if dtype == "bf16" else torch.float32)
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def assert_out(got: np.ndarray, want: np.ndarray, dtype: str, what: str, grad: bool = False):
+    err = np.abs(got - want)
+    if dtype == "f32":
+        assert err.max() <= 1e-5, f"{what}: max abs err {err.max():.3e}"
+        return
+    rel = np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-30)
+    bound = 2e-2 * (max(1.0, np.abs(want).max()) if grad else 1.0)
+    assert err.max() <= bound, f"{what}: max abs err {err.max():.3e} > {bound:.3e}"
+    assert rel <= 5e-3, f"{what}: rel L2 err {rel:.3e}"
+
+
+def small(name="s", B=2, L=1000, h_q=8, h_kv=2, d=128, K=4, dtype="bf16", structure="iid",
+          seed=123, kind="fwd"):
+    return synth.Workload(name, B, L, h_q, h_kv, d, 64, K, dtype, structure, kind, seed)
+
+
+def run_fwd(wl, x):
+    m = hsa()
+    q, k, v, qs = (to_dev(x[n], wl.dtype) for n in ("q", "k", "v", "q_slc"))
+    o, lse, idx, w, kbar = m.hsa_fwd(q, k, v, qs, wl.K)
+    torch.cuda.synchronize()
+    return o, lse, idx, w, kbar
+
+
+# --------------------------------------------------------------------------- pool / select
+@pytest.mark.parametrize("wl", [small(dtype="f32", d=64), small(), small(L=64 * 40 + 17, B=1)],
+                         ids=["f32", "bf16", "ragged"])
+def test_pool_bit_exact(wl):
+    x = synth.make_inputs(wl)
+    kb = hsa().hsa_pool(to_dev(x["k"], wl.dtype))
+    assert np.array_equal(kb.cpu().numpy(), oracle.pool(x["k"], wl.S))
+
+
+@pytest.mark.parametrize("wl", [small(dtype="f32", d=64, K=3), small(K=8, L=4096),
+                                small(K=16, L=2048, h_kv=4, h_q=8), small(K=1, L=700)],
+                         ids=["f32", "bf16-k8", "k16", "k1-ragged"])
+def test_select_indices_exact(wl):
+    x, kbar, (idx, w, s, gap) = gap_ruled(wl)
+    kb, gi, gw = hsa().hsa_select(to_dev(x["q_slc"], wl.dtype), to_dev(x["k"], wl.dtype), wl.K)
+    assert np.array_equal(kb.cpu().numpy(), kbar)
+    gi = gi.cpu().numpy().reshape(idx.shape)
+    assert np.array_equal(gi, idx), f"{(gi != idx).sum()} index mismatches"
+    assert np.abs(gw.cpu().numpy().reshape(w.shape) - w).max() <= 1e-5
+
+
+# --------------------------------------------------------------------------- forward
+FWD_SMALL = [small(dtype="f32", d=64, K=4, L=1024, h_q=4, h_kv=1),
+             small(), small(L=64 * 37 + 5, K=8, h_q=16, h_kv=2),
+             small(h_q=4, h_kv=4, K=2, L=640), small(d=64, L=1500, K=5),
+             small(L=60, K=4), small(L=128, K=8)]
+
+
+@pytest.mark.parametrize("wl", FWD_SMALL, ids=["f32", "bf16", "ragged-g8", "g1", "d64", "one-chunk",
+                                               "K>n_c"])
+def test_fwd_small_full(wl):
+    x, kbar, sel = gap_ruled(wl)
+    o_ref, lse_ref, idx_ref, w_ref = oracle.fwd(x["q"], x["k"], x["v"], x["q_slc"], kbar, wl.S, wl.K)
+    o, lse, idx, w, kb = run_fwd(wl, x)
+    assert np.array_equal(idx.cpu().numpy().reshape(idx_ref.shape), idx_ref)
+    assert_out(f64(o).reshape(o_ref.shape), o_ref, wl.dtype, "o")
+    assert np.abs(f64(lse).reshape(lse_ref.shape) - lse_ref).max() <= (1e-5 if wl.dtype == "f32" else 2e-3)
+    # tokens of chunk 0 output exactly zero
+    assert not f64(o)[:, :wl.S].any()
+
+
+def test_fwd_tiny_fp32_workload():
+    """The tiny fp32 workload in full: indices exact, max |err| <= 1e-5."""
+    wl, (x, kbar, sel) = cached_workload("tiny_fp32")
+    o_ref, lse_ref, idx_ref, w_ref = oracle.fwd(x["q"], x["k"], x["v"], x["q_slc"], kbar, wl.S, wl.K)
+    o, lse, idx, w, kb = run_fwd(wl, x)
+    assert np.array_equal(idx.cpu().numpy().reshape(idx_ref.shape), idx_ref)
+    assert_out(f64(o).reshape(o_ref.shape), o_ref, "f32", "o")
+
+
+def _sample_rows(wl, n, seed=0):
+    rng = np.random.default_rng(seed)
+    rows = set(rng.integers(0, wl.B * wl.L, size=n).tolist())
+    for b in range(wl.B):  # edges: first chunk, chunk boundaries, last token
+        rows.update([b * wl.L + t for t in (0, wl.S - 1, wl.S, 2 * wl.S - 1, wl.L - 1)])
+    return np.array(sorted(rows), dtype=np.int64)
+
+
+@pytest.mark.parametrize("name", ["fwd16k", "fwd64k"])
+def test_fwd_full_size_sampled(name):
+    """Full-size workloads in the launch configuration the benchmark times: all
+    chunk indices exact; outputs on sampled rows (oracle row by row)."""
+    wl, (x, kbar, (idx_ref, w_ref, s_ref, gap)) = cached_workload(name)
+    o, lse, idx, w, kb = run_fwd(wl, x)
+    assert np.array_equal(kb.cpu().numpy(), kbar)
+    gi = idx.cpu().numpy().reshape(idx_ref.shape)
+    assert np.array_equal(gi, idx_ref), f"{(gi != idx_ref).sum()} index mismatches"
+    assert np.abs(w.cpu().numpy().reshape(w_ref.shape) - w_ref).max() <= 1e-5
+    rows = _sample_rows(wl, 384)
+    o_ref, lse_ref, _, _ = oracle.fwd(x["q"], x["k"], x["v"], x["q_slc"], kbar, wl.S, wl.K, rows=rows)
+    og = f64(o).reshape(wl.B * wl.L, wl.h_q, wl.d)[rows]
+    assert_out(og, o_ref, wl.dtype, "o")
+
+
+# --------------------------------------------------------------------------- decode
+def test_decode_workload():
+    wl, (x, kbar, (o_ref, idx_ref, w_ref, gap)) = cached_workload("decode16k")
+    m = hsa()
+    kc, vc = to_dev(x["k"], "bf16"), to_dev(x["v"], "bf16")
+    kb = m.hsa_pool(kc)
+    assert np.array_equal(kb.cpu().numpy(), kbar)
+    o, idx, w = m.hsa_decode(to_dev(x["q"], "bf16"), to_dev(x["q_slc"], "bf16"), kc, vc, kb, wl.K)
+    torch.cuda.synchronize()
+    assert np.array_equal(idx.cpu().numpy(), idx_ref)
+    assert np.abs(w.cpu().numpy() - w_ref).max() <= 1e-5
+    assert_out(f64(o), o_ref, "bf16", "o")
+
+
+@pytest.mark.parametrize("P", [0, 63, 64, 640 + 7])
+def test_decode_small_edges(P):
+    wl = synth.Workload("dec", 3, P, 8, 2, 64, 64, 4, "f32", "iid", "decode", 77 + P)
+    x, kbar, (o_ref, idx_ref, w_ref, gap) = gap_ruled(wl)
+    m = hsa()
+    kc, vc = to_dev(x["k"], "f32"), to_dev(x["v"], "f32")
+    o, idx, w = m.hsa_decode(to_dev(x["q"], "f32"), to_dev(x["q_slc"], "f32"), kc, vc,
+                             torch.from_numpy(kbar).to(DEV), wl.K)
+    torch.cuda.synchronize()
+    assert np.array_equal(idx.cpu().numpy(), idx_ref)
+    assert_out(f64(o), o_ref, "f32", "o")
+
+
+# --------------------------------------------------------------------------- backward
+def run_bwd(wl, x, kbar_np=None):
+    m = hsa()
+    q, k, v, qs, dO = (to_dev(x[n], wl.dtype) for n in ("q", "k", "v", "q_slc", "dO"))
+    o, lse, idx, w, kbar = m.hsa_fwd(q, k, v, qs, wl.K)
+    dq, dk, dv, dqs = m.hsa_bwd(q, k, v, qs, dO, lse, idx, w, kbar, wl.K)
+    torch.cuda.synchronize()
+    return dq, dk, dv, dqs
+
+
+BWD_SMALL = [small(dtype="f32", d=64, L=512, K=3, kind="train"),
+             small(L=64 * 21 + 9, K=4, kind="train"),
+             small(L=1024, K=8, h_q=16, h_kv=2, kind="train")]
+
+
+@pytest.mark.parametrize("wl", BWD_SMALL, ids=["f32", "bf16-ragged", "bf16-g8"])
+def test_bwd_small_full(wl):
+    x, kbar, sel = gap_ruled(wl)
+    ref = oracle.bwd(x["q"], x["k"], x["v"], x["q_slc"], kbar, x["dO"], wl.S, wl.K)
+    got = run_bwd(wl, x)
+    for name, g, r in zip(("dq", "dk", "dv", "dq_slc"), got, ref[:4]):
+        if wl.dtype == "f32":
+            err = np.abs(f64(g) - r).max()
+            assert err <= 1e-4 * max(1.0, np.abs(r).max()), f"{name}: {err:.3e}"
+        else:
+            assert_out(f64(g), r, "bf16", name, grad=True)
+
+
+def test_bwd_train_workload_sampled():
+    """Full-size training workload: dq / dq_slc on sampled tokens, dk / dv on
+    sampled chunks (the oracle walks every token that selected them)."""
+    wl, (x, kbar, (idx, w, s, gap)) = cached_workload("train16k")
+    dq, dk, dv, dqs = run_bwd(wl, x)
+    rng = np.random.default_rng(5)
+    chunks = [(0, 0, 1), (1, 1, wl.n_c // 2), (3, 0, wl.n_c - 2), (2, 1, 7)]
+    idx4 = idx.reshape(wl.B, wl.L, wl.h_kv, wl.K)
+    mask = np.zeros((wl.B, wl.L), dtype=bool)
+    for b, g, c in chunks:
+        mask[b] |= (idx4[b, :, g, :] == c).any(-1)
+    toks = rng.integers(0, wl.L, size=(wl.B, 16))
+    for b in range(wl.B):
+        mask[b, toks[b]] = True
+    rdq, rdk, rdv, rdqs, _ = oracle.bwd(x["q"], x["k"], x["v"], x["q_slc"], kbar, x["dO"], wl.S, wl.K,
+                                        tok_mask=mask)
+    for b in range(wl.B):
+        tt = toks[b]
+        assert_out(f64(dq)[b, tt], rdq[b, tt], "bf16", "dq", grad=True)
+        assert_out(f64(dqs)[b, tt], rdqs[b, tt], "bf16", "dq_slc", grad=True)
+    for b, g, c in chunks:
+        sl = slice(c * wl.S, (c + 1) * wl.S)
+        # dk includes the pooled path of every token selecting c: all are in the mask
+        assert_out(f64(dk)[b, g, sl], rdk[b, g, sl], "bf16", f"dk[{b},{g},{c}]", grad=True)
+        assert_out(f64(dv)[b, g, sl], rdv[b, g, sl], "bf16", f"dv[{b},{g},{c}]", grad=True)
+
+
+# --------------------------------------------------------------------------- status / errors
+def test_device_status_clean_and_bad_index_reported():
+    """A corrupted chunk index (one that is not causally eligible) is caught on
+    the device: the kernel skips it and sets HSA_ERR_DEVICE_CHECK; nothing traps."""
+    m = hsa()
+    wl = small(L=512, K=4, kind="train")
+    x, kbar, sel = gap_ruled(wl)
+    q, k, v, qs, dO = (to_dev(x[n], wl.dtype) for n in ("q", "k", "v", "q_slc", "dO"))
+    o, lse, idx, w, kb = m.hsa_fwd(q, k, v, qs, wl.K)
+    ws = torch.empty(m.hsa_workspace_size(wl.B, wl.L, wl.h_q, wl.h_kv, wl.d, 64, wl.K, torch.bfloat16,
+                                          m.OP_BWD), dtype=torch.uint8, device=DEV)
+    m.hsa_bwd(q, k, v, qs, dO, lse, idx, w, kb, wl.K, ws=ws)
+    assert m.hsa_device_status(ws) == 0
+    bad = idx.clone()
+    bad[0, 100, 0, 0] = 7   # token 100 is in chunk 1: chunk 7 is not eligible
+    m.hsa_bwd(q, k, v, qs, dO, lse, bad, w, kb, wl.K, ws=ws)
+    assert m.hsa_device_status(ws) == 6
+    m.hsa_bwd(q, k, v, qs, dO, lse, idx, w, kb, wl.K, ws=ws)   # cleared by the next call
+    assert m.hsa_device_status(ws) == 0
+
+
+def test_empty_inputs():
+    m = hsa()
+    for L in (0, 30):
+        wl = small(L=L, B=1, K=4)
+        x = synth.make_inputs(wl)
+        o, lse, idx, w, kb = run_fwd(wl, x)
+        assert not f64(o).any()
+        assert (idx.cpu().numpy() == -1).all() and not w.cpu().numpy().any()

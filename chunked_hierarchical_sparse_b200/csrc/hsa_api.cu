@@ -192,8 +192,9 @@ hsa_status_t hsa_decode(const hsa_shape_t *shape, const void *q, const void *q_s
     if (s != HSA_OK) return s;
     const Shape sh = make_shape(*shape);
     if (sh.B == 0) return empty_call(sh, HSA_OP_DECODE, ws, ws_bytes, static_cast<cudaStream_t>(stream));
-    if (!ptrs_ok({q, q_slc, k_cache, v_cache, o}) || !opt_ok(idx) || !opt_ok(w)) return HSA_ERR_INVALID_ARG;
-    if (sh.nc > 0 && !ptrs_ok({kbar})) return HSA_ERR_INVALID_ARG;
+    if (!ptrs_ok({q, q_slc, o}) || !opt_ok(idx) || !opt_ok(w)) return HSA_ERR_INVALID_ARG;
+    // with no complete cached chunk the caches and the index are never read
+    if (sh.nc > 0 && !ptrs_ok({k_cache, v_cache, kbar})) return HSA_ERR_INVALID_ARG;
     if ((s = check_ws(sh, HSA_OP_DECODE, ws, ws_bytes)) != HSA_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     DevStatus *ds = static_cast<DevStatus *>(ws);

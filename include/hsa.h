@@ -148,6 +148,24 @@ HSA_API hsa_status_t hsa_bwd(const hsa_shape_t *shape, const void *q, const void
                      const float *w, const float *kbar, void *dq, void *dk, void *dv,
                      void *dq_slc, void *ws, size_t ws_bytes, void *stream);
 
+/* hsa_fwd without a caller-provided workspace.  The source pages have no
+ * counterpart to this call; it exists for callers that cannot allocate device
+ * memory where they run the forward pass -- e.g. a plug-in inside an inference
+ * runtime that owns all device allocations and forbids cudaMalloc to its
+ * plug-ins, or a latency-critical loop where cudaMalloc/cudaFree (which may
+ * synchronise the device) is not allowed.  Inputs and outputs are passed as in
+ * hsa_fwd (o required; lse, idx, w, kbar optional).  Scratch comes from one
+ * fixed 32 MiB device array owned by the library (held by each GPU that loads
+ * it until process exit); a problem whose scratch would exceed it -- status
+ * word plus kbar, idx, w for those not supplied -- returns HSA_ERR_WORKSPACE
+ * without launching.  The first call on a device looks the array's address up
+ * (make it before any stream capture).  All calls on a device share the array:
+ * calls that may overlap on the GPU race and must not be issued.  It runs the
+ * token-major CUDA-core kernel sequence and allocates nothing. */
+HSA_API hsa_status_t hsa_fwd_noalloc(const hsa_shape_t *shape, const void *q, const void *k,
+                                     const void *v, const void *q_slc, void *o, float *lse,
+                                     int32_t *idx, float *w, float *kbar, void *stream);
+
 /* Synchronises `stream`, then reads the device status word of workspace `ws`
  * into *code_out (an hsa_status_t value; HSA_OK when nothing went wrong). */
 HSA_API hsa_status_t hsa_device_status(const void *ws, int32_t *code_out, void *stream);

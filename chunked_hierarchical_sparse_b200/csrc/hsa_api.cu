@@ -48,14 +48,37 @@ struct FwdWs {
     float *kbar;
     int32_t *idx;
     float *w;
+    bool tc;             // chunk-major tensor-core path
+    BwdWs inv;           // token->chunk lists (hist, chunk_off, seg_off, entries)
+    AttendPlan plan;
+    __nv_bfloat16 *part; // partial-output ring
 };
 
 static FwdWs carve_fwd(const Shape &sh, void *ws, size_t *bytes) {
     Carver c{static_cast<char *>(ws)};
-    FwdWs f;
+    FwdWs f{};
     f.kbar = c.take<float>((size_t)sh.B * sh.hkv * sh.nc * sh.d);
     f.idx = c.take<int32_t>((size_t)sh.B * sh.L * sh.hkv * sh.K);
     f.w = c.take<float>((size_t)sh.B * sh.L * sh.hkv * sh.K);
+    f.tc = attend_tc_supported(sh);
+    if (f.tc) {
+        const int ntb = (int)ceil_div(sh.L, kInvTokBlock);
+        f.inv.hist = c.take<int32_t>((size_t)sh.B * sh.hkv * ntb * sh.nc);
+        f.inv.chunk_off = c.take<int32_t>((size_t)sh.B * sh.hkv * (sh.nc + 1));
+        f.inv.seg_off = c.take<int32_t>((size_t)sh.B * sh.hkv * (sh.nc + 1));
+        f.inv.entries = c.take<int32_t>((size_t)sh.B * sh.hkv * sh.L * sh.K);
+        AttendPlan &P = f.plan;
+        P.B = sh.B; P.L = sh.L; P.hq = sh.hq; P.hkv = sh.hkv; P.D = sh.d; P.K = sh.K; P.G = sh.G;
+        P.nc = sh.nc; P.ntb = ntb; P.W = attend_window(sh.K, sh.G, sh.d);
+        P.nW = (int)ceil_div(sh.L, P.W); P.J = sh.B * sh.hkv * P.nW; P.TT = 128 / sh.G;
+        P.unit_prefix = c.take<int32_t>((size_t)P.J * (sh.nc + 1));
+        P.win_units = c.take<int32_t>((size_t)P.J);
+        P.win_tiles = c.take<int32_t>((size_t)P.J);
+        P.win_ncomb = c.take<int32_t>((size_t)P.J);
+        P.seg_start = c.take<int32_t>((size_t)P.J + 2);
+        P.counters = c.take<int32_t>((size_t)2 * P.J + 1);
+        f.part = c.take<__nv_bfloat16>((size_t)kRing * P.W * sh.K * sh.G * sh.d);
+    }
     if (bytes) *bytes = c.off;
     return f;
 }
@@ -181,7 +204,23 @@ hsa_status_t hsa_fwd(const hsa_shape_t *shape, const void *q, const void *k, con
     cudaError_t e = clear_status(ws, st);
     if (e == cudaSuccess) e = timed(HSA_K_POOL, 1, st, [&] { return launch_pool(sh, k, f.kbar, ds, st); });
     if (e == cudaSuccess) e = timed(HSA_K_SELECT, 1, st, [&] { return launch_select_simt(sh, q_slc, f.kbar, f.idx, f.w, ds, st); });
-    if (e == cudaSuccess) e = timed(HSA_K_ATTEND_SIMT, 1, st, [&] { return launch_attend_simt(sh, q, k, v, f.idx, f.w, o, lse, ds, st); });
+    if (!f.tc) {
+        if (e == cudaSuccess)
+            e = timed(HSA_K_ATTEND_SIMT, 1, st, [&] { return launch_attend_simt(sh, q, k, v, f.idx, f.w, o, lse, ds, st); });
+        return cuda_status(e);
+    }
+    // chunk-major tensor-core path: invert the selection, plan windows, attend
+    if (e == cudaSuccess && sh.nc > 0)
+        e = timed(HSA_K_INVERT, 3, st, [&] { return launch_invert(sh, f.idx, f.inv, ds, st); });
+    if (e == cudaSuccess) e = timed(HSA_K_PLAN, 2, st, [&] { return launch_plan(sh, f.inv, f.plan, st); });
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(f.plan.counters, 0, sizeof(int32_t) * ((size_t)2 * f.plan.J + 1), st);
+    if (e == cudaSuccess && lse)
+        e = cudaMemsetAsync(lse, 0, sizeof(float) * (size_t)sh.B * sh.L * sh.hq * sh.K, st);
+    if (e == cudaSuccess)
+        e = timed(HSA_K_ATTEND_TC, 1, st, [&] {
+            return launch_attend_tc(sh, f.plan, f.inv, q, k, v, f.idx, f.w, f.part, o, lse, ds, st);
+        });
     return cuda_status(e);
 }
 

@@ -132,4 +132,36 @@ cudaError_t launch_bwd_phase2(const Shape &sh, const void *q, const void *k, con
 constexpr int kInvTokBlock = 256;  // tokens per histogram block of the inversion
 constexpr int kBwdSeg = 32;        // list entries per phase-2 block
 
+// ---------------------------------------------------------------- chunk-major forward plan
+constexpr int kUnitTiles = 4;      // tiles of one chunk per work unit (one K/V load)
+constexpr int kCombTokens = 16;    // tokens per combine item
+constexpr int kRing = 2;           // windows whose partial outputs are live at once
+constexpr size_t kPartSlotBudget = size_t(32) << 20;  // bytes of partials per window
+
+struct AttendPlan {
+    int B, L, hq, hkv, D, K, G, nc, ntb, W, nW, J, TT;
+    int32_t *unit_prefix;  // [J][nc+1] work units per (window, chunk), exclusive prefix
+    int32_t *win_units;    // [J]
+    int32_t *win_tiles;    // [J]
+    int32_t *win_ncomb;    // [J]
+    int32_t *seg_start;    // [J+2] queue segment starts (units of s, combines of s-1)
+    int32_t *counters;     // [2J+1] tiles_done[J], comb_done[J], queue head (zeroed per call)
+};
+
+// window length (tokens) of the chunk-major forward: a multiple of 256 such that
+// one window's partials (W * K * G * d bf16) fit in kPartSlotBudget
+inline int attend_window(int K, int G, int d) {
+    const int64_t per_tok = (int64_t)K * G * d * 2;
+    int64_t w = (int64_t)(kPartSlotBudget / per_tok) / kInvTokBlock * kInvTokBlock;
+    if (w < kInvTokBlock) w = kInvTokBlock;
+    if (w > 4096) w = 4096;
+    return (int)w;
+}
+
+cudaError_t launch_plan(const Shape &sh, const BwdWs &inv, const AttendPlan &plan, cudaStream_t st);
+bool attend_tc_supported(const Shape &sh);
+cudaError_t launch_attend_tc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv, const void *q,
+                             const void *k, const void *v, const int32_t *idx, const float *w,
+                             const __nv_bfloat16 *part, void *o, float *lse, DevStatus *ds, cudaStream_t st);
+
 }  // namespace hsa

@@ -1,0 +1,684 @@
+// k_attend_tc.cu -- chunk-major softmax-off-by-one attention with
+// stick-breaking fusion on the 5th-generation tensor cores (tcgen05 + TMEM +
+// TMA), persistent, warp-specialised.
+//
+// Cited page: "Hardware-aligned Hierarchical Sparse Attention for Efficient
+// Long-term Memory Access" (paper notes), §HSA first and second stages (token-
+// level attention inside each selected chunk, stick-breaking fusion of the
+// chunk outputs) and §kernel (softmax-off-by-one; the backward's second phase
+// walks, per chunk, the tokens that selected it).  The pages' forward kernel
+// is token-major; this one is chunk-major: a tile holds TT = 128/G tokens
+// that selected the same chunk, with the G query heads of each token as rows
+// (the GQA-group idea of the NSA blog), so one 64-key K/V tile loaded by TMA
+// serves 128 query rows on the tensor cores:
+//   S[128 x 64]  = Q_tile[128 x d] . K_c^T          (tcgen05, fp32 in TMEM)
+//   p = exp(x - m) / (e^{-m} + sum exp(x - m)),  x = S / sqrt(d), m = max(0, max x)
+//   O[128 x d]   = P[128 x 64] . V_c                (tcgen05, fp32 in TMEM)
+//   partial(t, h, slot) = bf16( w_{t,g,slot} / Z * O )     -> window ring (TMA store)
+// Each window's partials are summed per token by combine items of the same
+// persistent kernel once the window's tiles are done:
+//   o[t, h] = bf16( sum_slot partial(t, h, slot) ).
+//
+// Roles (192 threads): warp 0 pulls queue items and issues TMA loads, warp 1
+// allocates TMEM and issues the MMAs (one elected lane), warps 2-5 do the
+// softmax, the epilogue (TMEM -> bf16 -> swizzled SMEM -> TMA store) and the
+// combine items.  Every wait is bounded (a wall-clock limit); on expiry the
+// kernel records HSA_ERR_TIMEOUT, unwinds, frees its TMEM and returns.
+#include "hsa_internal.cuh"
+#include "sm100.cuh"
+
+namespace hsa {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int kThreads = 192;
+constexpr int kInfo = 4;                 // tile-info ring entries
+constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s bound on any single wait
+
+enum ItemType : int { kItemTile = 0, kItemComb = 1, kItemEnd = 2 };
+
+struct TileInfo {
+    int type;
+    int j;        // window
+    int b, g, c;  // sequence, group, chunk (tile) ; c = combine index for combine items
+    int ntok;     // valid tokens in the tile
+    int kvs, kvph, unit_first, unit_last;
+    int qs, qph;
+    int tok[16];
+    int slot[16];
+};
+
+template <int D> struct Smem {
+    static constexpr int QHALF = 128 * 128;  // bytes per 64-column half of a 128-row tile
+    static constexpr int NH = D / 64;        // halves along d
+    static constexpr int QBYTES = NH * QHALF;
+    static constexpr int KVHALF = 64 * 128;
+    static constexpr int KVBYTES = NH * KVHALF;
+    static constexpr int PBYTES = 128 * 128;
+    static constexpr int STBYTES = NH * QHALF;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_K = OFF_Q + 2 * QBYTES;
+    static constexpr int OFF_V = OFF_K + 2 * KVBYTES;
+    static constexpr int OFF_P = OFF_V + 2 * KVBYTES;
+    static constexpr int OFF_ST = OFF_P + 2 * PBYTES;
+    static constexpr int OFF_INFO = OFF_ST + STBYTES;
+    static constexpr int OFF_BAR = OFF_INFO + kInfo * (int)sizeof(TileInfo);
+    static constexpr int NBAR = 2 * kInfo + 2 * 2 + 2 * 2 + 2 * 2 + 2 + 2 * 2 + 1;
+    static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+    static constexpr int BYTES = OFF_MISC + 64;
+    static constexpr int ALLOC = BYTES + 1024;  // slack for 1 KB alignment
+};
+
+struct Bars {
+    uint64_t *info_full, *info_empty;  // [kInfo]
+    uint64_t *q_full, *q_empty;        // [2]
+    uint64_t *kv_full, *kv_empty;      // [2]
+    uint64_t *s_full, *s_empty;        // [2]
+    uint64_t *p_full;                  // [2]
+    uint64_t *o_full, *o_empty;        // [2]
+};
+
+__device__ __forceinline__ int ld_acquire(const int32_t *p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// bounded spin until *p >= target; false on timeout
+__device__ bool spin_geq(const int32_t *p, int target) {
+    if (ld_acquire(p) >= target) return true;
+    const uint64_t t0 = globaltimer();
+    while (true) {
+        __nanosleep(128);
+        if (ld_acquire(p) >= target) return true;
+        if (globaltimer() - t0 > kWaitNs) return false;
+    }
+}
+
+__device__ __forceinline__ void wg_sync() {  // named barrier 1 over warps 2..5
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+}
+
+__device__ __forceinline__ uint4 ldcg_u4(const void *p) {
+    uint4 r;
+    asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+    return r;
+}
+
+struct ItemDecode {
+    int type, j, unit_or_comb;
+};
+
+__device__ ItemDecode decode_item(const AttendPlan &P, int q) {
+    // last s with seg_start[s] <= q
+    int lo = 0, hi = P.J;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (P.seg_start[mid] <= q) lo = mid; else hi = mid - 1;
+    }
+    const int s = lo;
+    const int local = q - P.seg_start[s];
+    const int units = (s < P.J) ? P.win_units[s] : 0;
+    ItemDecode d;
+    if (local < units) { d.type = kItemTile; d.j = s; d.unit_or_comb = local; }
+    else { d.type = kItemComb; d.j = s - 1; d.unit_or_comb = local - units; }
+    return d;
+}
+
+}  // namespace
+
+template <int D, int G>
+__global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
+    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_part,
+    const __grid_constant__ AttendPlan P, const int32_t *__restrict__ hist,
+    const int32_t *__restrict__ chunk_off, const int32_t *__restrict__ entries,
+    const int32_t *__restrict__ idx, const float *__restrict__ wsel, const __nv_bfloat16 *__restrict__ part,
+    __nv_bfloat16 *__restrict__ out, float *__restrict__ lse, DevStatus *ds) {
+    using L = Smem<D>;
+    constexpr int TT = 128 / G;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    TileInfo *info = reinterpret_cast<TileInfo *>(sm + L::OFF_INFO);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + L::OFF_BAR);
+    Bars B;
+    B.info_full = bar; B.info_empty = bar + kInfo;
+    B.q_full = bar + 2 * kInfo; B.q_empty = B.q_full + 2;
+    B.kv_full = B.q_empty + 2; B.kv_empty = B.kv_full + 2;
+    B.s_full = B.kv_empty + 2; B.s_empty = B.s_full + 2;
+    B.p_full = B.s_empty + 2;
+    B.o_full = B.p_full + 2; B.o_empty = B.o_full + 2;
+    uint64_t *mma_done = B.o_empty + 2;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::OFF_MISC);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 16);
+    volatile int *wg_flag = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 32);  // [2]
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < kInfo; ++i) { mbar_init(&B.info_full[i], 1); mbar_init(&B.info_empty[i], 2); }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&B.q_full[i], 1); mbar_init(&B.q_empty[i], 1);
+            mbar_init(&B.kv_full[i], 1); mbar_init(&B.kv_empty[i], 1);
+            mbar_init(&B.s_full[i], 1); mbar_init(&B.s_empty[i], 4);
+            mbar_init(&B.p_full[i], 128);
+            mbar_init(&B.o_full[i], 1); mbar_init(&B.o_empty[i], 4);
+        }
+        mbar_init(mma_done, 1);
+        *abort_flag = 0;
+        mbar_fence_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    if (warp == 0 && lane == 0) {
+        prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v); prefetch_tmap(&tm_part);
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    int32_t *tiles_done = P.counters;
+    int32_t *comb_done = P.counters + P.J;
+    int32_t *qhead = P.counters + 2 * P.J;
+    const float scale = 1.0f / sqrtf((float)D);
+
+    // lane 0 waits, the whole warp gets the verdict (warp-uniform control flow)
+    auto warp_wait = [&](uint64_t *b, uint32_t par) -> bool {
+        int r = 1;
+        if (lane == 0) r = mbar_wait(b, par, kWaitNs) ? 1 : 0;
+        return __shfl_sync(0xffffffffu, r, 0) != 0;
+    };
+
+    if (warp == 0) {
+        // ============================================================ producer
+        int it = 0, qc = 0, kvc = 0;
+        bool ok = true;
+        const int total = P.seg_start[P.J + 1];
+        while (ok) {
+            const int ii = it % kInfo;
+            if (it >= kInfo && !warp_wait(&B.info_empty[ii], ((it / kInfo) - 1) & 1)) { ok = false; break; }
+            if (*abort_flag) { ok = false; break; }
+            int q = 0;
+            if (lane == 0) q = atomicAdd(qhead, 1);
+            q = __shfl_sync(0xffffffffu, q, 0);
+            TileInfo &inf = info[ii];
+            if (q >= total) {
+                if (lane == 0) { inf.type = kItemEnd; mbar_arrive(&B.info_full[ii]); }
+                break;
+            }
+            const ItemDecode dq = decode_item(P, q);
+            const int bg = dq.j / P.nW, wwin = dq.j % P.nW;
+            const int b = bg / P.hkv, g = bg % P.hkv;
+            if (dq.type == kItemComb) {
+                if (lane == 0) {
+                    inf.type = kItemComb; inf.j = dq.j; inf.b = b; inf.g = g; inf.c = dq.unit_or_comb;
+                    mbar_arrive(&B.info_full[ii]);
+                }
+                ++it;
+                continue;
+            }
+            // ---- a work unit: chunk c, tiles [t0, t1) of its bucket in window j
+            const int32_t *up = P.unit_prefix + (int64_t)dq.j * (P.nc + 1);
+            int lo = 0, hi = P.nc - 1;
+            while (lo < hi) {
+                const int mid = (lo + hi + 1) >> 1;
+                if (up[mid] <= dq.unit_or_comb) lo = mid; else hi = mid - 1;
+            }
+            const int c = lo;
+            const int uib = dq.unit_or_comb - up[c];
+            const int tb0 = wwin * (P.W / kInvTokBlock);
+            const int tb1 = min(P.ntb, (wwin + 1) * (P.W / kInvTokBlock));
+            const int32_t *H = hist + (int64_t)bg * P.ntb * P.nc;
+            const int e0 = H[(int64_t)tb0 * P.nc + c];
+            const int e1 = (tb1 < P.ntb) ? H[(int64_t)tb1 * P.nc + c] : chunk_off[(int64_t)bg * (P.nc + 1) + c + 1];
+            const int nt = (e1 - e0 + TT - 1) / TT;
+            const int t0 = uib * kUnitTiles, t1 = min(nt, t0 + kUnitTiles);
+            // ring guard: window j's partial slot was used by window j - kRing
+            if (dq.j >= kRing) {
+                int g_ok = 1;
+                if (lane == 0) g_ok = spin_geq(&comb_done[dq.j - kRing], P.win_ncomb[dq.j - kRing]) ? 1 : 0;
+                if (!__shfl_sync(0xffffffffu, g_ok, 0)) {
+                    if (lane == 0) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 1, dq.j);
+                    ok = false;
+                    break;
+                }
+            }
+            // K/V tiles of chunk c
+            const int kvs = kvc & 1, kvph = (kvc >> 1) & 1;
+            if (kvc >= 2 && !warp_wait(&B.kv_empty[kvs], ((kvc >> 1) - 1) & 1)) { ok = false; break; }
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&B.kv_full[kvs], 2 * L::KVBYTES);
+                const int row = bg * P.L + c * kChunk;
+#pragma unroll
+                for (int h = 0; h < L::NH; ++h) {
+                    tma_load_2d(sm + L::OFF_K + kvs * L::KVBYTES + h * L::KVHALF, &tm_k, h * 64, row, &B.kv_full[kvs]);
+                    tma_load_2d(sm + L::OFF_V + kvs * L::KVBYTES + h * L::KVHALF, &tm_v, h * 64, row, &B.kv_full[kvs]);
+                }
+            }
+            ++kvc;
+            for (int tt = t0; tt < t1; ++tt) {
+                const int ti = it % kInfo;
+                if (it >= kInfo && !warp_wait(&B.info_empty[ti], ((it / kInfo) - 1) & 1)) { ok = false; break; }
+                const int qs = qc & 1, qph = (qc >> 1) & 1;
+                if (qc >= 2 && !warp_wait(&B.q_empty[qs], ((qc >> 1) - 1) & 1)) { ok = false; break; }
+                TileInfo &ti_ = info[ti];
+                const int eb = e0 + tt * TT;
+                const int ntok = min(TT, e1 - eb);
+                int ent = 0;
+                if (lane < ntok) ent = entries[(int64_t)bg * P.L * P.K + eb + lane];
+                const int t = ent >> 4, slot = ent & 15;
+                if (lane < 16) { ti_.tok[lane] = (lane < ntok) ? t : -1; ti_.slot[lane] = (lane < ntok) ? slot : 0; }
+                if (lane == 0) {
+                    ti_.type = kItemTile; ti_.j = dq.j; ti_.b = b; ti_.g = g; ti_.c = c; ti_.ntok = ntok;
+                    ti_.kvs = kvs; ti_.kvph = kvph; ti_.unit_first = (tt == t0); ti_.unit_last = (tt == t1 - 1);
+                    ti_.qs = qs; ti_.qph = qph;
+                    mbar_arrive_expect_tx(&B.q_full[qs], ntok * L::NH * G * 128);
+                }
+                __syncwarp();
+                if (lane < ntok) {
+                    const int row = (b * P.L + t) * P.hq + g * G;
+#pragma unroll
+                    for (int h = 0; h < L::NH; ++h)
+                        tma_load_2d(sm + L::OFF_Q + qs * L::QBYTES + h * L::QHALF + lane * G * 128, &tm_q, h * 64,
+                                    row, &B.q_full[qs]);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&B.info_full[ti]);
+                ++qc;
+                ++it;
+            }
+        }
+        if (!ok) {
+            *abort_flag = 1;
+            if (lane == 0) {
+                report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 2, it);
+                // let the loads already issued land before the CTA goes away (bounded)
+                for (int s2 = 0; s2 < 2; ++s2) {
+                    if (qc > s2) mbar_wait(&B.q_full[(qc - 1 - s2) & 1], ((qc - 1 - s2) >> 1) & 1, kWaitNs);
+                    if (kvc > s2) mbar_wait(&B.kv_full[(kvc - 1 - s2) & 1], ((kvc - 1 - s2) >> 1) & 1, kWaitNs);
+                }
+            }
+            __syncwarp();
+        }
+    } else if (warp == 1) {
+        // ============================================================ MMA issuer
+        constexpr uint32_t idesc1 = idesc_bf16_f32(128, 64, false, false);
+        constexpr uint32_t idesc2 = idesc_bf16_f32(128, D, false, true);
+        int it = 0, tseq = 0;
+        int pend = -1, pend_buf = 0, pend_seq = 0, pend_last = 0, pend_kvs = 0, pend_ii = 0;
+        bool ok = true;
+        auto do_mma2 = [&]() -> bool {
+            // O[pb] = P[pb] . V   (for the pending tile)
+            if (!warp_wait(&B.p_full[pend_buf], (pend_seq >> 1) & 1)) return false;
+            if (pend_seq >= 2 && !warp_wait(&B.o_empty[pend_buf], ((pend_seq >> 1) - 1) & 1)) return false;
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t pa = smem_u32(sm + L::OFF_P + pend_buf * L::PBYTES);
+                const uint32_t vb = smem_u32(sm + L::OFF_V + pend_kvs * L::KVBYTES);
+                const uint32_t dcol = tmem + 128 + pend_buf * 128;
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16_ss(dcol, smem_desc_sw128(pa + ks * 32, 16, 1024),
+                                smem_desc_sw128(vb + ks * 2048, L::KVHALF, 1024), idesc2, ks > 0);
+                mma_commit(&B.o_full[pend_buf]);
+                if (pend_last) mma_commit(&B.kv_empty[pend_kvs]);
+                mbar_arrive(&B.info_empty[pend_ii]);
+            }
+            __syncwarp();
+            pend = -1;
+            return true;
+        };
+        while (ok) {
+            const int ii = it % kInfo;
+            const uint32_t ipar = (it / kInfo) & 1;
+            // never sit on a pending PV product while the next item is not there yet
+            if (pend >= 0) {
+                int ready = 0;
+                if (lane == 0) ready = mbar_test(&B.info_full[ii], ipar) ? 1 : 0;
+                if (!__shfl_sync(0xffffffffu, ready, 0) && !do_mma2()) { ok = false; break; }
+            }
+            if (!warp_wait(&B.info_full[ii], ipar)) { ok = false; break; }
+            const TileInfo &inf = info[ii];
+            const int type = inf.type;
+            if (type == kItemEnd) break;
+            if (type == kItemComb) {
+                if (pend >= 0 && !do_mma2()) { ok = false; break; }
+                if (lane == 0) mbar_arrive(&B.info_empty[ii]);
+                ++it;
+                continue;
+            }
+            const int sb = tseq & 1;
+            if (inf.unit_first && !warp_wait(&B.kv_full[inf.kvs], inf.kvph)) { ok = false; break; }
+            if (!warp_wait(&B.q_full[inf.qs], inf.qph)) { ok = false; break; }
+            if (tseq >= 2 && !warp_wait(&B.s_empty[sb], ((tseq >> 1) - 1) & 1)) { ok = false; break; }
+            tc_fence_after();
+            if (lane == 0) {
+                const uint32_t qa = smem_u32(sm + L::OFF_Q + inf.qs * L::QBYTES);
+                const uint32_t kb = smem_u32(sm + L::OFF_K + inf.kvs * L::KVBYTES);
+                const uint32_t dcol = tmem + sb * 64;
+#pragma unroll
+                for (int ks = 0; ks < D / 16; ++ks) {
+                    const int h = ks >> 2, kk = ks & 3;
+                    mma_bf16_ss(dcol, smem_desc_sw128(qa + h * L::QHALF + kk * 32, 16, 1024),
+                                smem_desc_sw128(kb + h * L::KVHALF + kk * 32, 16, 1024), idesc1, ks > 0);
+                }
+                mma_commit(&B.s_full[sb]);
+                mma_commit(&B.q_empty[inf.qs]);
+            }
+            __syncwarp();
+            if (pend >= 0 && !do_mma2()) { ok = false; break; }
+            pend = 1; pend_buf = sb; pend_seq = tseq; pend_last = inf.unit_last; pend_kvs = inf.kvs; pend_ii = ii;
+            ++tseq;
+            ++it;
+        }
+        if (ok && pend >= 0 && !do_mma2()) ok = false;
+        if (!ok) { *abort_flag = 1; if (lane == 0) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 3, it); }
+        // drain: every MMA issued by this warp has finished before TMEM is released
+        if (lane == 0) {
+            mma_commit(mma_done);
+            mbar_wait(mma_done, 0, kWaitNs);
+        }
+        __syncwarp();
+    } else {
+        // ============================================================ softmax / epilogue / combine
+        const int wq = warp & 3;                 // TMEM lane quadrant of this warp
+        const int r = wq * 32 + lane;            // tile row = token * G + head
+        const int tid = threadIdx.x - 64;        // 0..127
+        const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
+        int it = 0, tseq = 0, wcnt = 0;
+        bool ok = true;
+        int pe = -1, pe_buf = 0, pe_seq = 0, pe_ii = 0;  // pending epilogue
+        float pe_coef = 0.f;
+        int pend_count_j = -1;  // (thread 0) window of the last stored tile not yet counted
+
+        // thread 0 decides, the whole group follows (uniform control flow at named barriers)
+        auto wg_vote = [&](int v) -> bool {
+            const int slot = (wcnt++) & 1;
+            if (tid == 0) wg_flag[slot] = v;
+            wg_sync();
+            return wg_flag[slot] != 0;
+        };
+        auto wg_wait = [&](uint64_t *b, uint32_t par) -> bool {
+            int v = 1;
+            if (tid == 0) v = mbar_wait(b, par, kWaitNs) ? 1 : 0;
+            return wg_vote(v);
+        };
+        auto flush_counts = [&]() {
+            if (tid == 0) {
+                bulk_wait<0>();
+                if (pend_count_j >= 0) {
+                    fence_proxy_async_global();
+                    __threadfence();
+                    atomicAdd(&tiles_done[pend_count_j], 1);
+                }
+                pend_count_j = -1;
+            }
+        };
+        auto epilogue = [&]() -> bool {
+            const TileInfo &inf = info[pe_ii];
+            if (tid == 0) bulk_wait_read<0>();  // the staging buffer is free again
+            if (!wg_wait(&B.o_full[pe_buf], (pe_seq >> 1) & 1)) return false;
+            tc_fence_after();
+            uint8_t *stg = sm + L::OFF_ST;
+#pragma unroll
+            for (int h = 0; h < L::NH; ++h) {
+                float v0[32], v1[32];
+                tmem_ld32(lane_base + 128 + pe_buf * 128 + h * 64, v0);
+                tmem_ld32(lane_base + 128 + pe_buf * 128 + h * 64 + 32, v1);
+                tmem_wait_ld();
+                uint8_t *rowp = stg + h * L::QHALF + r * 128;
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    const float *src = (ch < 4) ? (v0 + ch * 8) : (v1 + (ch - 4) * 8);
+                    uint4 pk;
+                    __nv_bfloat162 a0 = __floats2bfloat162_rn(src[0] * pe_coef, src[1] * pe_coef);
+                    __nv_bfloat162 a1 = __floats2bfloat162_rn(src[2] * pe_coef, src[3] * pe_coef);
+                    __nv_bfloat162 a2 = __floats2bfloat162_rn(src[4] * pe_coef, src[5] * pe_coef);
+                    __nv_bfloat162 a3 = __floats2bfloat162_rn(src[6] * pe_coef, src[7] * pe_coef);
+                    pk.x = *reinterpret_cast<uint32_t *>(&a0); pk.y = *reinterpret_cast<uint32_t *>(&a1);
+                    pk.z = *reinterpret_cast<uint32_t *>(&a2); pk.w = *reinterpret_cast<uint32_t *>(&a3);
+                    *reinterpret_cast<uint4 *>(rowp + ((ch ^ (r & 7)) << 4)) = pk;
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&B.o_empty[pe_buf]);
+            fence_proxy_async_smem();
+            wg_sync();
+            if (tid == 0) {
+                const int s = inf.j % kRing;
+                const int ws = (inf.j % P.nW) * P.W;
+                for (int i = 0; i < inf.ntok; ++i) {
+                    const int prow = ((s * P.W + (inf.tok[i] - ws)) * P.K + inf.slot[i]) * G;
+#pragma unroll
+                    for (int h = 0; h < L::NH; ++h)
+                        tma_store_2d(&tm_part, stg + h * L::QHALF + i * G * 128, h * 64, prow);
+                }
+                bulk_commit();
+                bulk_wait<1>();  // the previous group (previous tile) is complete
+                if (pend_count_j >= 0) {
+                    fence_proxy_async_global();
+                    __threadfence();
+                    atomicAdd(&tiles_done[pend_count_j], 1);
+                }
+                pend_count_j = inf.j;
+                mbar_arrive(&B.info_empty[pe_ii]);
+            }
+            pe = -1;
+            return true;
+        };
+
+        while (ok) {
+            const int ii = it % kInfo;
+            const uint32_t ipar = (it / kInfo) & 1;
+            if (pe >= 0) {  // never sit on a finished tile while the next item is not there yet
+                int ready = 1;
+                if (tid == 0) ready = mbar_test(&B.info_full[ii], ipar) ? 1 : 0;
+                if (!wg_vote(ready)) {
+                    if (!epilogue()) { ok = false; break; }
+                    flush_counts();
+                }
+            }
+            if (!wg_wait(&B.info_full[ii], ipar)) { ok = false; break; }
+            const TileInfo &inf = info[ii];
+            const int type = inf.type;
+            if (type == kItemEnd) break;
+            if (type == kItemComb) {
+                if (pe >= 0 && !epilogue()) { ok = false; break; }
+                flush_counts();
+                // every tile of window j has stored its partials
+                int gok = 1;
+                if (tid == 0) gok = spin_geq(&tiles_done[inf.j], P.win_tiles[inf.j]) ? 1 : 0;
+                if (!wg_vote(gok)) { if (tid == 0) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 4, inf.j); ok = false; break; }
+                const int j = inf.j, b = inf.b, g = inf.g;
+                const int s = j % kRing;
+                const int ws = (j % P.nW) * P.W;
+                const int we = min(P.L, ws + P.W);
+                const int ta = ws + inf.c * kCombTokens, tb = min(we, ta + kCombTokens);
+                for (int t = ta; t < tb; ++t) {
+                    const int ne = min(t / kChunk, P.nc);
+                    const int nsel = min(P.K, ne);
+                    const int32_t *ix = idx + (((int64_t)b * P.L + t) * P.hkv + g) * P.K;
+                    for (int e = tid; e < G * D / 8; e += 128) {
+                        float acc[8];
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+                        for (int k = 0; k < nsel; ++k) {
+                            const int c = ix[k];
+                            if (c < 0 || c >= ne) continue;
+                            const uint4 raw =
+                                ldcg_u4(part + ((int64_t)((s * P.W + (t - ws)) * P.K + k) * G) * D + e * 8);
+                            const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+                            for (int q = 0; q < 4; ++q) {
+                                const float2 f = __bfloat1622float2(h2[q]);
+                                acc[2 * q] += f.x;
+                                acc[2 * q + 1] += f.y;
+                            }
+                        }
+                        uint4 pk;
+                        __nv_bfloat162 a0 = __floats2bfloat162_rn(acc[0], acc[1]);
+                        __nv_bfloat162 a1 = __floats2bfloat162_rn(acc[2], acc[3]);
+                        __nv_bfloat162 a2 = __floats2bfloat162_rn(acc[4], acc[5]);
+                        __nv_bfloat162 a3 = __floats2bfloat162_rn(acc[6], acc[7]);
+                        pk.x = *reinterpret_cast<uint32_t *>(&a0); pk.y = *reinterpret_cast<uint32_t *>(&a1);
+                        pk.z = *reinterpret_cast<uint32_t *>(&a2); pk.w = *reinterpret_cast<uint32_t *>(&a3);
+                        *reinterpret_cast<uint4 *>(out + (((int64_t)b * P.L + t) * P.hq + g * G) * D + e * 8) = pk;
+                    }
+                }
+                wg_sync();
+                if (tid == 0) {
+                    __threadfence();
+                    atomicAdd(&comb_done[j], 1);
+                    mbar_arrive(&B.info_empty[ii]);
+                }
+                ++it;
+                continue;
+            }
+            // ---------------- softmax of this tile
+            const int sb = tseq & 1;
+            if (!wg_wait(&B.s_full[sb], (tseq >> 1) & 1)) { ok = false; break; }
+            tc_fence_after();
+            float x0[32], x1[32];
+            tmem_ld32(lane_base + sb * 64, x0);
+            tmem_ld32(lane_base + sb * 64 + 32, x1);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&B.s_empty[sb]);
+            const int ti = r / G, hh = r % G;
+            const bool valid = ti < inf.ntok;
+            uint8_t *prow = sm + L::OFF_P + sb * L::PBYTES + r * 128;
+            float coef = 0.f;
+            if (valid) {
+                const int t = inf.tok[ti], slot = inf.slot[ti];
+                const float L2E = 1.4426950408889634f;
+                float m = 0.f;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    x0[i] *= scale;
+                    x1[i] *= scale;
+                    m = fmaxf(m, fmaxf(x0[i], x1[i]));
+                }
+                const float mb = m * L2E;
+                float z = exp2f(-mb);
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    x0[i] = exp2f(fmaf(x0[i], L2E, -mb));
+                    x1[i] = exp2f(fmaf(x1[i], L2E, -mb));
+                    z += x0[i] + x1[i];
+                }
+                const int64_t srow = (((int64_t)inf.b * P.L + t) * P.hkv + inf.g) * P.K + slot;
+                coef = wsel[srow] / z;
+                if (lse) lse[(((int64_t)inf.b * P.L + t) * P.hq + inf.g * G + hh) * P.K + slot] = m + logf(z);
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) {
+                    const float *src = (ch < 4) ? (x0 + ch * 8) : (x1 + (ch - 4) * 8);
+                    uint4 pk;
+                    __nv_bfloat162 a0 = __floats2bfloat162_rn(src[0], src[1]);
+                    __nv_bfloat162 a1 = __floats2bfloat162_rn(src[2], src[3]);
+                    __nv_bfloat162 a2 = __floats2bfloat162_rn(src[4], src[5]);
+                    __nv_bfloat162 a3 = __floats2bfloat162_rn(src[6], src[7]);
+                    pk.x = *reinterpret_cast<uint32_t *>(&a0); pk.y = *reinterpret_cast<uint32_t *>(&a1);
+                    pk.z = *reinterpret_cast<uint32_t *>(&a2); pk.w = *reinterpret_cast<uint32_t *>(&a3);
+                    *reinterpret_cast<uint4 *>(prow + ((ch ^ (r & 7)) << 4)) = pk;
+                }
+            } else {
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch) *reinterpret_cast<uint4 *>(prow + (ch << 4)) = make_uint4(0, 0, 0, 0);
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&B.p_full[sb]);
+            // epilogue of the previous tile while this tile's O = P.V runs
+            if (pe >= 0 && !epilogue()) { ok = false; break; }
+            pe = 1; pe_buf = sb; pe_seq = tseq; pe_ii = ii; pe_coef = coef;
+            ++tseq;
+            ++it;
+        }
+        if (ok && pe >= 0 && !epilogue()) ok = false;
+        if (ok) flush_counts();
+        if (!ok) { *abort_flag = 1; if (tid == 0) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 5, it); }
+        if (tid == 0) bulk_wait<0>();
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// ------------------------------------------------------------------ host side
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+// 2D bf16 map: inner dim `cols` (contiguous), outer `rows`; box 64 x box_rows, 128B swizzle
+bool make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint32_t box_rows) {
+    EncodeTiledFn enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {cols, rows};
+    cuuint64_t strides[1] = {cols * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t es[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int D, int G>
+cudaError_t launch_tc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv, const void *q, const void *k,
+                      const void *v, const int32_t *idx, const float *w, const __nv_bfloat16 *part, void *o,
+                      float *lse, DevStatus *ds, cudaStream_t st) {
+    CUtensorMap mq, mk, mv, mp;
+    if (!make_map(&mq, q, D, (uint64_t)sh.B * sh.L * sh.hq, G) ||
+        !make_map(&mk, k, D, (uint64_t)sh.B * sh.hkv * sh.L, 64) ||
+        !make_map(&mv, v, D, (uint64_t)sh.B * sh.hkv * sh.L, 64) ||
+        !make_map(&mp, part, D, (uint64_t)kRing * plan.W * sh.K * G, G))
+        return cudaErrorInvalidValue;
+    const size_t smem = Smem<D>::ALLOC;
+    cudaError_t e = set_smem_once((const void *)attend_tc_kernel<D, G>, smem);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+    attend_tc_kernel<D, G><<<sms, kThreads, smem, st>>>(mq, mk, mv, mp, plan, inv.hist, inv.chunk_off, inv.entries,
+                                                        idx, w, part, (__nv_bfloat16 *)o, lse, ds);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+bool attend_tc_supported(const Shape &sh) {
+    return sh.bf16 && (sh.d == 64 || sh.d == 128) && (sh.G == 8 || sh.G == 16) && sh.K <= 16 &&
+           get_encode() != nullptr;
+}
+
+cudaError_t launch_attend_tc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv, const void *q,
+                             const void *k, const void *v, const int32_t *idx, const float *w,
+                             const __nv_bfloat16 *part, void *o, float *lse, DevStatus *ds, cudaStream_t st) {
+    if (sh.d == 128 && sh.G == 8) return launch_tc<128, 8>(sh, plan, inv, q, k, v, idx, w, part, o, lse, ds, st);
+    if (sh.d == 128 && sh.G == 16) return launch_tc<128, 16>(sh, plan, inv, q, k, v, idx, w, part, o, lse, ds, st);
+    if (sh.d == 64 && sh.G == 8) return launch_tc<64, 8>(sh, plan, inv, q, k, v, idx, w, part, o, lse, ds, st);
+    if (sh.d == 64 && sh.G == 16) return launch_tc<64, 16>(sh, plan, inv, q, k, v, idx, w, part, o, lse, ds, st);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace hsa

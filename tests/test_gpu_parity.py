@@ -58,8 +58,12 @@ def small(name="s", B=2, L=1000, h_q=8, h_kv=2, d=128, K=4, dtype="bf16", struct
 def run_fwd(wl, x):
     m = hsa()
     q, k, v, qs = (to_dev(x[n], wl.dtype) for n in ("q", "k", "v", "q_slc"))
-    o, lse, idx, w, kbar = m.hsa_fwd(q, k, v, qs, wl.K)
+    tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    ws = torch.empty(m.hsa_workspace_size(wl.B, wl.L, wl.h_q, wl.h_kv, wl.d, 64, wl.K, tdt, m.OP_FWD),
+                     dtype=torch.uint8, device=DEV)
+    o, lse, idx, w, kbar = m.hsa_fwd(q, k, v, qs, wl.K, ws=ws)
     torch.cuda.synchronize()
+    assert m.hsa_device_status(ws) == 0, "device status word set"
     return o, lse, idx, w, kbar
 
 
@@ -101,6 +105,30 @@ def test_fwd_small_full(wl):
     assert_out(f64(o).reshape(o_ref.shape), o_ref, wl.dtype, "o")
     assert np.abs(f64(lse).reshape(lse_ref.shape) - lse_ref).max() <= (1e-5 if wl.dtype == "f32" else 2e-3)
     # tokens of chunk 0 output exactly zero
+    assert not f64(o)[:, :wl.S].any()
+
+
+# chunk-major tensor-core path: bf16 with G = h_q / h_kv in {8, 16}
+FWD_TC = [small(h_q=16, h_kv=2, K=8, L=1000), small(h_q=16, h_kv=1, K=4, L=64 * 45 + 3, B=1),
+          small(h_q=16, h_kv=2, d=64, K=8, L=64 * 70 + 30), small(h_q=16, h_kv=2, K=16, L=2048),
+          small(h_q=16, h_kv=2, K=1, L=777, B=3),
+          small(h_q=16, h_kv=2, K=8, L=64 * 100 + 17, B=2, seed=9)]
+
+
+@pytest.mark.parametrize("wl", FWD_TC, ids=["g8", "g16-ragged", "g8-d64", "g8-k16", "g8-k1-b3",
+                                            "g8-multiwindow"])
+def test_fwd_tensor_core_path_full(wl):
+    x, kbar, sel = gap_ruled(wl)
+    o_ref, lse_ref, idx_ref, w_ref = oracle.fwd(x["q"], x["k"], x["v"], x["q_slc"], kbar, wl.S, wl.K)
+    m = hsa()
+    m.hsa_timing_enable(True)
+    o, lse, idx, w, kb = run_fwd(wl, x)
+    ms, n = m.hsa_timing_read("attend_tc")
+    m.hsa_timing_enable(False)
+    assert n == 1, "the tensor-core kernel did not run"
+    assert np.array_equal(idx.cpu().numpy().reshape(idx_ref.shape), idx_ref)
+    assert_out(f64(o).reshape(o_ref.shape), o_ref, "bf16", "o")
+    assert np.abs(f64(lse).reshape(lse_ref.shape) - lse_ref).max() <= 2e-3
     assert not f64(o)[:, :wl.S].any()
 
 

@@ -103,57 +103,51 @@ def read_traffic(kernel_file: str):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons during the timed region."""
+    """SM clocks and throttle reasons sampled through NVML every few ms while
+    the timed region runs."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
-
-    def __init__(self, index: int):
+    def __init__(self, index: int, period_s: float = 0.005):
         self.index = index
-        self.proc = None
-        self.lines = []
+        self.period = period_s
+        self.samples = []
+        self.stop = threading.Event()
+        self.err = None
+
+    def _run(self):
+        try:
+            import pynvml as nv
+            nv.nvmlInit()
+            h = nv.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            bits = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+                    "sw_power_cap": 0x4}
+            while not self.stop.is_set():
+                mhz = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+                self.samples.append((mhz, [n for n, b in bits.items() if r & b]))
+                time.sleep(self.period)
+        except Exception as e:  # pragma: no cover - reported in the JSON line
+            self.err = repr(e)
 
     def __enter__(self):
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
-                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
-            self.t.start()
-        except OSError:
-            self.proc = None
+        self.max_mhz = None
+        self.t = threading.Thread(target=self._run, daemon=True)
+        self.t.start()
+        time.sleep(0.05)
         return self
 
-    def _read(self):
-        for ln in self.proc.stdout:
-            self.lines.append(ln.strip())
-
     def __exit__(self, *a):
-        if self.proc:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
+        self.stop.set()
+        self.t.join(timeout=5)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        sm = [m for m, _ in self.samples]
+        reasons = sorted({r for _, rs in self.samples for r in rs})
+        out = {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": self.max_mhz,
+               "reasons": reasons, "samples": len(sm), "source": "nvml"}
+        if self.err:
+            out["error"] = self.err
+        return out
 
 
 # --------------------------------------------------------------------------- reference arm
@@ -162,7 +156,7 @@ def run_reference(args, rank, world):
         return
     import oracle
     from chunked_hierarchical_sparse_b200 import synth
-    wl = synth.WORKLOADS["fwd64k"]
+    wl = synth.WORKLOADS[args.workload]
     x = synth.make_inputs(wl)
     kbar = oracle.pool(x["k"], wl.S)
     rng = np.random.default_rng(0)
@@ -178,12 +172,12 @@ def run_reference(args, rank, world):
     tot = sum(times)
     value = n_rows * len(times) / tot
     cores = oracle.num_threads()
-    sample = f"{n_rows} uniformly sampled token rows of the 64K workload per step (pool once per run)"
+    sample = f"{n_rows} uniformly sampled token rows of the {args.workload} workload per step (pool once per run)"
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "impl": "reference",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * tot / len(times), "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "fwd64k", "B": wl.B, "L": wl.L, "S": wl.S, "K": wl.K,
+            "config": {"workload": args.workload, "B": wl.B, "L": wl.L, "S": wl.S, "K": wl.K,
                        "h_q": wl.h_q, "h_kv": wl.h_kv, "d": wl.d, "global_batch": wl.B,
                        "seq_len": wl.L},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
@@ -325,6 +319,8 @@ def main():
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     ap.add_argument("--no-extras", action="store_true", help="skip the decode and train measurements")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    ap.add_argument("--workload", default="fwd64k", choices=["fwd64k", "fwd16k"],
+                    help="forward workload (fwd16k: the smaller case used for ncu captures)")
     args = ap.parse_args()
     assert args.warmup >= 3 or args.impl == "reference", "at least 3 warm-up steps"
 
@@ -349,7 +345,7 @@ def main():
     torch.cuda.set_device(dev)
     hsa.load_library()
 
-    base = synth.WORKLOADS["fwd64k"]
+    base = synth.WORKLOADS[args.workload]
     wl = base.scaled(seed=base.seed + 100 * rank)  # one independent sequence per rank
     x = synth.make_inputs(wl)
     q, k, v, qs = (to_dev(x[n], dev) for n in ("q", "k", "v", "q_slc"))
@@ -407,7 +403,7 @@ def main():
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "fwd64k", "B": wl.B, "L": wl.L, "S": wl.S, "K": wl.K, "h_q": wl.h_q,
+        "config": {"workload": args.workload, "B": wl.B, "L": wl.L, "S": wl.S, "K": wl.K, "h_q": wl.h_q,
                    "h_kv": wl.h_kv, "d": wl.d, "global_batch": wl.B * world, "seq_len": wl.L,
                    "parallelism": f"dp{world} (independent sequences)",
                    "l2": "flushed (256 MB write) before every timed step"},

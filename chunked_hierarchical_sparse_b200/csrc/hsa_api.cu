@@ -1,5 +1,7 @@
 // hsa_api.cu -- the extern "C" entry points declared in include/hsa.h:
 // argument checks, workspace carving, and the kernel sequence of each call.
+#include <algorithm>
+#include <climits>
 #include <cstring>
 
 #include "hsa_internal.cuh"
@@ -77,6 +79,12 @@ static FwdWs carve_fwd(const Shape &sh, void *ws, size_t *bytes) {
         P.win_ncomb = c.take<int32_t>((size_t)P.J);
         P.seg_start = c.take<int32_t>((size_t)P.J + 2);
         P.counters = c.take<int32_t>((size_t)2 * P.J + 1);
+        // queue items: units <= tiles <= L*K/TT + nc per (b, g) window set, plus combine items
+        P.max_items = (int)std::min<int64_t>(
+            ((int64_t)sh.B * sh.hkv * ((int64_t)sh.L * sh.K / P.TT + (int64_t)P.nW * sh.nc) +
+             (int64_t)sh.B * sh.hkv * ceil_div(sh.L, kCombTokens) + P.nW * (int64_t)sh.B * sh.hkv + 16),
+            (int64_t)INT32_MAX / 4);
+        P.items = c.take<int4>((size_t)2 * P.max_items);
         f.part = c.take<__nv_bfloat16>((size_t)kRing * P.W * sh.K * sh.G * sh.d);
     }
     if (bytes) *bytes = c.off;
@@ -212,7 +220,7 @@ hsa_status_t hsa_fwd(const hsa_shape_t *shape, const void *q, const void *k, con
     // chunk-major tensor-core path: invert the selection, plan windows, attend
     if (e == cudaSuccess && sh.nc > 0)
         e = timed(HSA_K_INVERT, 3, st, [&] { return launch_invert(sh, f.idx, f.inv, ds, st); });
-    if (e == cudaSuccess) e = timed(HSA_K_PLAN, 2, st, [&] { return launch_plan(sh, f.inv, f.plan, st); });
+    if (e == cudaSuccess) e = timed(HSA_K_PLAN, 3, st, [&] { return launch_plan(sh, f.inv, f.plan, st); });
     if (e == cudaSuccess)
         e = cudaMemsetAsync(f.plan.counters, 0, sizeof(int32_t) * ((size_t)2 * f.plan.J + 1), st);
     if (e == cudaSuccess && lse)

@@ -135,7 +135,7 @@ constexpr int kBwdSeg = 32;        // list entries per phase-2 block
 // ---------------------------------------------------------------- chunk-major forward plan
 constexpr int kUnitTiles = 4;      // tiles of one chunk per work unit (one K/V load)
 constexpr int kCombTokens = 16;    // tokens per combine item
-constexpr int kRing = 2;           // windows whose partial outputs are live at once
+constexpr int kRing = 3;           // window slots of the partial-output ring
 constexpr size_t kPartSlotBudget = size_t(32) << 20;  // bytes of partials per window
 
 struct AttendPlan {
@@ -146,7 +146,13 @@ struct AttendPlan {
     int32_t *win_ncomb;    // [J]
     int32_t *seg_start;    // [J+2] queue segment starts (units of s, combines of s-1)
     int32_t *counters;     // [2J+1] tiles_done[J], comb_done[J], queue head (zeroed per call)
+    int4 *items;           // [2 per queue item] flat descriptors in queue order
+    int max_items;         // capacity of `items`
 };
+
+// queue item descriptor (two int4): {type, j, c, e0} {e1, t0, t1, 0}
+//   type 0: work unit, chunk c, entries [e0, e1) of its bucket, tiles [t0, t1)
+//   type 1: combine item c of window j
 
 // window length (tokens) of the chunk-major forward: a multiple of 256 such that
 // one window's partials (W * K * G * d bf16) fit in kPartSlotBudget

@@ -31,9 +31,29 @@ namespace hsa {
 
 using namespace sm100;
 
+#ifdef HSA_TC_PROFILE
+// Per-CTA cycle accounting of the roles' waits (development builds only).
+__device__ unsigned long long *g_tc_prof = nullptr;
+#define PROF_DECL unsigned long long prof_acc[16] = {0}; long long prof_t0 = 0;
+#define PROF_BEGIN() (prof_t0 = clock64())
+#define PROF_END(slot) (prof_acc[slot] += (unsigned long long)(clock64() - prof_t0))
+#define PROF_INC(slot) (prof_acc[slot] += 1)
+#define PROF_DUMP(base)                                                                        \
+    do {                                                                                       \
+        if (g_tc_prof)                                                                         \
+            for (int _i = 0; _i < 16; ++_i) atomicAdd(&g_tc_prof[(base) + _i], prof_acc[_i]);  \
+    } while (0)
+#else
+#define PROF_DECL
+#define PROF_BEGIN() ((void)0)
+#define PROF_END(slot) ((void)0)
+#define PROF_INC(slot) ((void)0)
+#define PROF_DUMP(base) ((void)0)
+#endif
+
 namespace {
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;  // 7 warps: producer, MMA, 4 softmax/epilogue, store
 constexpr int kInfo = 4;                 // tile-info ring entries
 constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s bound on any single wait
 
@@ -48,6 +68,7 @@ struct TileInfo {
     int qs, qph;
     int tok[16];
     int slot[16];
+    float w[16];  // stick-breaking weight of each token's slot
 };
 
 template <int D> struct Smem {
@@ -65,7 +86,7 @@ template <int D> struct Smem {
     static constexpr int OFF_ST = OFF_P + 2 * PBYTES;
     static constexpr int OFF_INFO = OFF_ST + STBYTES;
     static constexpr int OFF_BAR = OFF_INFO + kInfo * (int)sizeof(TileInfo);
-    static constexpr int NBAR = 2 * kInfo + 2 * 2 + 2 * 2 + 2 * 2 + 2 + 2 * 2 + 1;
+    static constexpr int NBAR = 2 * kInfo + 2 * 2 + 2 * 2 + 2 * 2 + 2 + 2 * 2 + 1 + 2;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_MISC + 64;
     static constexpr int ALLOC = BYTES + 1024;  // slack for 1 KB alignment
@@ -101,30 +122,14 @@ __device__ __forceinline__ void wg_sync() {  // named barrier 1 over warps 2..5
     asm volatile("bar.sync 1, 128;" ::: "memory");
 }
 
+__device__ __forceinline__ void discard_l2(const void *p) {
+    asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
+}
+
 __device__ __forceinline__ uint4 ldcg_u4(const void *p) {
     uint4 r;
     asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
     return r;
-}
-
-struct ItemDecode {
-    int type, j, unit_or_comb;
-};
-
-__device__ ItemDecode decode_item(const AttendPlan &P, int q) {
-    // last s with seg_start[s] <= q
-    int lo = 0, hi = P.J;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (P.seg_start[mid] <= q) lo = mid; else hi = mid - 1;
-    }
-    const int s = lo;
-    const int local = q - P.seg_start[s];
-    const int units = (s < P.J) ? P.win_units[s] : 0;
-    ItemDecode d;
-    if (local < units) { d.type = kItemTile; d.j = s; d.unit_or_comb = local; }
-    else { d.type = kItemComb; d.j = s - 1; d.unit_or_comb = local - units; }
-    return d;
 }
 
 }  // namespace
@@ -151,6 +156,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     B.p_full = B.s_empty + 2;
     B.o_full = B.p_full + 2; B.o_empty = B.o_full + 2;
     uint64_t *mma_done = B.o_empty + 2;
+    uint64_t *st_full = mma_done + 1;  // staging written (softmax group -> store warp)
+    uint64_t *st_free = mma_done + 2;  // staging read by the TMA engine (store warp -> softmax group)
+    volatile int *st_req = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 48);  // info index, -1 = end
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 16);
     volatile int *wg_flag = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 32);  // [2]
@@ -166,6 +174,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             mbar_init(&B.o_full[i], 1); mbar_init(&B.o_empty[i], 4);
         }
         mbar_init(mma_done, 1);
+        mbar_init(st_full, 1);
+        mbar_init(st_free, 1);
         *abort_flag = 0;
         mbar_fence_init();
     }
@@ -195,61 +205,94 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
 
     if (warp == 0) {
         // ============================================================ producer
+        PROF_DECL
+        const long long prof_start = clock64();
         int it = 0, qc = 0, kvc = 0;
         bool ok = true;
-        const int total = P.seg_start[P.J + 1];
+        const int total = min(P.seg_start[P.J + 1], P.max_items);
+        // item descriptors are fetched one ahead (queue slot + descriptor), lane 0 only
+        int4 nx0 = make_int4(kItemEnd, 0, 0, 0), nx1 = make_int4(0, 0, 0, 0);
+        int nx_ea = 0, nx_eb = 0;  // the next unit's (token, slot) entries, two per lane
+        int guard_ok_j = -1;       // highest window whose ring guard already passed
+        auto fetch = [&]() {
+            if (lane == 0) {
+                const int q = atomicAdd(qhead, 1);
+                if (q < total) { nx0 = P.items[2 * q]; nx1 = P.items[2 * q + 1]; }
+                else { nx0 = make_int4(kItemEnd, 0, 0, 0); }
+            }
+            const int ty = __shfl_sync(0xffffffffu, nx0.x, 0);
+            if (ty == kItemTile) {
+                const int jn = __shfl_sync(0xffffffffu, nx0.y, 0);
+                const int en0 = __shfl_sync(0xffffffffu, nx0.w, 0);
+                const int en1 = __shfl_sync(0xffffffffu, nx1.x, 0);
+                const int tn0 = __shfl_sync(0xffffffffu, nx1.y, 0);
+                const int tn1 = __shfl_sync(0xffffffffu, nx1.z, 0);
+                const int32_t *En = entries + (int64_t)(jn / P.nW) * P.L * P.K;
+                const int ub = en0 + tn0 * TT;
+                const int un = min(en1, en0 + tn1 * TT) - ub;
+                nx_ea = (lane < un) ? En[ub + lane] : 0;
+                nx_eb = (lane + 32 < un) ? En[ub + lane + 32] : 0;
+            }
+        };
+        fetch();
         while (ok) {
             const int ii = it % kInfo;
+            PROF_BEGIN();
             if (it >= kInfo && !warp_wait(&B.info_empty[ii], ((it / kInfo) - 1) & 1)) { ok = false; break; }
+            PROF_END(2);
             if (*abort_flag) { ok = false; break; }
-            int q = 0;
-            if (lane == 0) q = atomicAdd(qhead, 1);
-            q = __shfl_sync(0xffffffffu, q, 0);
+            PROF_BEGIN();
+            const int type = __shfl_sync(0xffffffffu, nx0.x, 0);
+            const int j = __shfl_sync(0xffffffffu, nx0.y, 0);
+            const int c = __shfl_sync(0xffffffffu, nx0.z, 0);
+            const int e0 = __shfl_sync(0xffffffffu, nx0.w, 0);
+            const int e1 = __shfl_sync(0xffffffffu, nx1.x, 0);
+            const int t0 = __shfl_sync(0xffffffffu, nx1.y, 0);
+            const int t1 = __shfl_sync(0xffffffffu, nx1.z, 0);
+            const int ent_a = nx_ea, ent_b = nx_eb;
+#ifdef HSA_TC_PROFILE
+            if (ent_a == 0x7fffffff) prof_t0 = 0;  // keeps the entry loads ordered before the timer read
+#endif
+            PROF_END(1);
             TileInfo &inf = info[ii];
-            if (q >= total) {
+            if (type == kItemEnd) {
                 if (lane == 0) { inf.type = kItemEnd; mbar_arrive(&B.info_full[ii]); }
                 break;
             }
-            const ItemDecode dq = decode_item(P, q);
-            const int bg = dq.j / P.nW, wwin = dq.j % P.nW;
+            fetch();  // next descriptor and entries in flight while this item is issued
+            const int bg = j / P.nW;
             const int b = bg / P.hkv, g = bg % P.hkv;
-            if (dq.type == kItemComb) {
+            if (type == kItemComb) {
                 if (lane == 0) {
-                    inf.type = kItemComb; inf.j = dq.j; inf.b = b; inf.g = g; inf.c = dq.unit_or_comb;
+                    inf.type = kItemComb; inf.j = j; inf.b = b; inf.g = g; inf.c = c;
                     mbar_arrive(&B.info_full[ii]);
                 }
                 ++it;
                 continue;
             }
-            // ---- a work unit: chunk c, tiles [t0, t1) of its bucket in window j
-            const int32_t *up = P.unit_prefix + (int64_t)dq.j * (P.nc + 1);
-            int lo = 0, hi = P.nc - 1;
-            while (lo < hi) {
-                const int mid = (lo + hi + 1) >> 1;
-                if (up[mid] <= dq.unit_or_comb) lo = mid; else hi = mid - 1;
-            }
-            const int c = lo;
-            const int uib = dq.unit_or_comb - up[c];
-            const int tb0 = wwin * (P.W / kInvTokBlock);
-            const int tb1 = min(P.ntb, (wwin + 1) * (P.W / kInvTokBlock));
-            const int32_t *H = hist + (int64_t)bg * P.ntb * P.nc;
-            const int e0 = H[(int64_t)tb0 * P.nc + c];
-            const int e1 = (tb1 < P.ntb) ? H[(int64_t)tb1 * P.nc + c] : chunk_off[(int64_t)bg * (P.nc + 1) + c + 1];
-            const int nt = (e1 - e0 + TT - 1) / TT;
-            const int t0 = uib * kUnitTiles, t1 = min(nt, t0 + kUnitTiles);
-            // ring guard: window j's partial slot was used by window j - kRing
-            if (dq.j >= kRing) {
+            // ---- work unit: chunk c, tiles [t0, t1) of the bucket entries [e0, e1) of window j
+            // the unit's (token, slot) entries: up to kUnitTiles * TT <= 64, two per lane
+            const int ub = e0 + t0 * TT;
+            const int un = min(e1, e0 + t1 * TT) - ub;
+            // ring guard: window j's partial slot was last used by window j - kRing
+            PROF_INC(6);
+            PROF_BEGIN();
+            if (j >= kRing && j > guard_ok_j) {
                 int g_ok = 1;
-                if (lane == 0) g_ok = spin_geq(&comb_done[dq.j - kRing], P.win_ncomb[dq.j - kRing]) ? 1 : 0;
+                if (lane == 0) g_ok = spin_geq(&comb_done[j - kRing], P.win_ncomb[j - kRing]) ? 1 : 0;
                 if (!__shfl_sync(0xffffffffu, g_ok, 0)) {
-                    if (lane == 0) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 1, dq.j);
+                    if (lane == 0) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 1, j);
                     ok = false;
                     break;
                 }
+                guard_ok_j = j;
             }
+            PROF_END(3);
             // K/V tiles of chunk c
             const int kvs = kvc & 1, kvph = (kvc >> 1) & 1;
+            PROF_BEGIN();
             if (kvc >= 2 && !warp_wait(&B.kv_empty[kvs], ((kvc >> 1) - 1) & 1)) { ok = false; break; }
+            PROF_END(4);
             if (lane == 0) {
                 mbar_arrive_expect_tx(&B.kv_full[kvs], 2 * L::KVBYTES);
                 const int row = bg * P.L + c * kChunk;
@@ -262,18 +305,30 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             ++kvc;
             for (int tt = t0; tt < t1; ++tt) {
                 const int ti = it % kInfo;
+                PROF_BEGIN();
                 if (it >= kInfo && !warp_wait(&B.info_empty[ti], ((it / kInfo) - 1) & 1)) { ok = false; break; }
+                PROF_END(2);
                 const int qs = qc & 1, qph = (qc >> 1) & 1;
+                PROF_BEGIN();
                 if (qc >= 2 && !warp_wait(&B.q_empty[qs], ((qc >> 1) - 1) & 1)) { ok = false; break; }
+                PROF_END(5);
+                PROF_INC(7);
                 TileInfo &ti_ = info[ti];
-                const int eb = e0 + tt * TT;
-                const int ntok = min(TT, e1 - eb);
-                int ent = 0;
-                if (lane < ntok) ent = entries[(int64_t)bg * P.L * P.K + eb + lane];
+                const int lo = (tt - t0) * TT;          // first entry of this tile within the unit
+                const int ntok = min(TT, un - lo);
+                // entry of token `lane` of this tile lives in lane (lo + lane) % 32 of ent_a/ent_b
+                const int src = (lo + lane) & 31;
+                const int va = __shfl_sync(0xffffffffu, ent_a, src);
+                const int vb = __shfl_sync(0xffffffffu, ent_b, src);
+                const int ent = (lo + lane < 32) ? va : vb;
                 const int t = ent >> 4, slot = ent & 15;
-                if (lane < 16) { ti_.tok[lane] = (lane < ntok) ? t : -1; ti_.slot[lane] = (lane < ntok) ? slot : 0; }
+                if (lane < 16) {
+                    ti_.tok[lane] = (lane < ntok) ? t : -1;
+                    ti_.slot[lane] = (lane < ntok) ? slot : 0;
+                    ti_.w[lane] = (lane < ntok) ? wsel[(((int64_t)b * P.L + t) * P.hkv + g) * P.K + slot] : 0.f;
+                }
                 if (lane == 0) {
-                    ti_.type = kItemTile; ti_.j = dq.j; ti_.b = b; ti_.g = g; ti_.c = c; ti_.ntok = ntok;
+                    ti_.type = kItemTile; ti_.j = j; ti_.b = b; ti_.g = g; ti_.c = c; ti_.ntok = ntok;
                     ti_.kvs = kvs; ti_.kvph = kvph; ti_.unit_first = (tt == t0); ti_.unit_last = (tt == t1 - 1);
                     ti_.qs = qs; ti_.qph = qph;
                     mbar_arrive_expect_tx(&B.q_full[qs], ntok * L::NH * G * 128);
@@ -304,17 +359,27 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             }
             __syncwarp();
         }
+#ifdef HSA_TC_PROFILE
+        prof_acc[0] = clock64() - prof_start;
+        if (lane == 0) PROF_DUMP(blockIdx.x * 48 + 0);
+#endif
     } else if (warp == 1) {
         // ============================================================ MMA issuer
         constexpr uint32_t idesc1 = idesc_bf16_f32(128, 64, false, false);
         constexpr uint32_t idesc2 = idesc_bf16_f32(128, D, false, true);
+        PROF_DECL
+        const long long prof_start = clock64();
         int it = 0, tseq = 0;
         int pend = -1, pend_buf = 0, pend_seq = 0, pend_last = 0, pend_kvs = 0, pend_ii = 0;
         bool ok = true;
         auto do_mma2 = [&]() -> bool {
             // O[pb] = P[pb] . V   (for the pending tile)
+            PROF_BEGIN();
             if (!warp_wait(&B.p_full[pend_buf], (pend_seq >> 1) & 1)) return false;
+            PROF_END(5);
+            PROF_BEGIN();
             if (pend_seq >= 2 && !warp_wait(&B.o_empty[pend_buf], ((pend_seq >> 1) - 1) & 1)) return false;
+            PROF_END(6);
             tc_fence_after();
             if (lane == 0) {
                 const uint32_t pa = smem_u32(sm + L::OFF_P + pend_buf * L::PBYTES);
@@ -341,7 +406,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 if (lane == 0) ready = mbar_test(&B.info_full[ii], ipar) ? 1 : 0;
                 if (!__shfl_sync(0xffffffffu, ready, 0) && !do_mma2()) { ok = false; break; }
             }
+            PROF_BEGIN();
             if (!warp_wait(&B.info_full[ii], ipar)) { ok = false; break; }
+            PROF_END(1);
             const TileInfo &inf = info[ii];
             const int type = inf.type;
             if (type == kItemEnd) break;
@@ -352,9 +419,15 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 continue;
             }
             const int sb = tseq & 1;
+            PROF_BEGIN();
             if (inf.unit_first && !warp_wait(&B.kv_full[inf.kvs], inf.kvph)) { ok = false; break; }
+            PROF_END(2);
+            PROF_BEGIN();
             if (!warp_wait(&B.q_full[inf.qs], inf.qph)) { ok = false; break; }
+            PROF_END(3);
+            PROF_BEGIN();
             if (tseq >= 2 && !warp_wait(&B.s_empty[sb], ((tseq >> 1) - 1) & 1)) { ok = false; break; }
+            PROF_END(4);
             tc_fence_after();
             if (lane == 0) {
                 const uint32_t qa = smem_u32(sm + L::OFF_Q + inf.qs * L::QBYTES);
@@ -383,7 +456,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             mbar_wait(mma_done, 0, kWaitNs);
         }
         __syncwarp();
-    } else {
+#ifdef HSA_TC_PROFILE
+        prof_acc[0] = clock64() - prof_start;
+        if (lane == 0) PROF_DUMP(blockIdx.x * 48 + 16);
+#endif
+    } else if (warp <= 5) {
         // ============================================================ softmax / epilogue / combine
         const int wq = warp & 3;                 // TMEM lane quadrant of this warp
         const int r = wq * 32 + lane;            // tile row = token * G + head
@@ -393,7 +470,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         bool ok = true;
         int pe = -1, pe_buf = 0, pe_seq = 0, pe_ii = 0;  // pending epilogue
         float pe_coef = 0.f;
-        int pend_count_j = -1;  // (thread 0) window of the last stored tile not yet counted
+        int nreq = 0;  // staging hand-offs to the store warp so far
+        PROF_DECL
+        const long long prof_start = clock64();
+        (void)prof_start;
 
         // thread 0 decides, the whole group follows (uniform control flow at named barriers)
         auto wg_vote = [&](int v) -> bool {
@@ -407,21 +487,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             if (tid == 0) v = mbar_wait(b, par, kWaitNs) ? 1 : 0;
             return wg_vote(v);
         };
-        auto flush_counts = [&]() {
-            if (tid == 0) {
-                bulk_wait<0>();
-                if (pend_count_j >= 0) {
-                    fence_proxy_async_global();
-                    __threadfence();
-                    atomicAdd(&tiles_done[pend_count_j], 1);
-                }
-                pend_count_j = -1;
-            }
-        };
         auto epilogue = [&]() -> bool {
-            const TileInfo &inf = info[pe_ii];
-            if (tid == 0) bulk_wait_read<0>();  // the staging buffer is free again
+            PROF_BEGIN();
+            // the staging buffer is free once the store warp's TMA stores have read it
+            if (nreq > 0 && !wg_wait(st_free, (nreq - 1) & 1)) return false;
             if (!wg_wait(&B.o_full[pe_buf], (pe_seq >> 1) & 1)) return false;
+            PROF_END(4);
+            PROF_BEGIN();
             tc_fence_after();
             uint8_t *stg = sm + L::OFF_ST;
 #pragma unroll
@@ -449,25 +521,14 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             if (lane == 0) mbar_arrive(&B.o_empty[pe_buf]);
             fence_proxy_async_smem();
             wg_sync();
+            PROF_END(5);
+            PROF_BEGIN();
             if (tid == 0) {
-                const int s = inf.j % kRing;
-                const int ws = (inf.j % P.nW) * P.W;
-                for (int i = 0; i < inf.ntok; ++i) {
-                    const int prow = ((s * P.W + (inf.tok[i] - ws)) * P.K + inf.slot[i]) * G;
-#pragma unroll
-                    for (int h = 0; h < L::NH; ++h)
-                        tma_store_2d(&tm_part, stg + h * L::QHALF + i * G * 128, h * 64, prow);
-                }
-                bulk_commit();
-                bulk_wait<1>();  // the previous group (previous tile) is complete
-                if (pend_count_j >= 0) {
-                    fence_proxy_async_global();
-                    __threadfence();
-                    atomicAdd(&tiles_done[pend_count_j], 1);
-                }
-                pend_count_j = inf.j;
-                mbar_arrive(&B.info_empty[pe_ii]);
+                *st_req = pe_ii;
+                mbar_arrive(st_full);
             }
+            ++nreq;
+            PROF_END(6);
             pe = -1;
             return true;
         };
@@ -479,55 +540,92 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 int ready = 1;
                 if (tid == 0) ready = mbar_test(&B.info_full[ii], ipar) ? 1 : 0;
                 if (!wg_vote(ready)) {
+                    PROF_INC(10);
                     if (!epilogue()) { ok = false; break; }
-                    flush_counts();
                 }
             }
+            PROF_BEGIN();
             if (!wg_wait(&B.info_full[ii], ipar)) { ok = false; break; }
+            PROF_END(1);
             const TileInfo &inf = info[ii];
             const int type = inf.type;
             if (type == kItemEnd) break;
             if (type == kItemComb) {
                 if (pe >= 0 && !epilogue()) { ok = false; break; }
-                flush_counts();
+                PROF_INC(11);
                 // every tile of window j has stored its partials
+                PROF_BEGIN();
                 int gok = 1;
                 if (tid == 0) gok = spin_geq(&tiles_done[inf.j], P.win_tiles[inf.j]) ? 1 : 0;
                 if (!wg_vote(gok)) { if (tid == 0) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 4, inf.j); ok = false; break; }
+                PROF_END(7);
+                PROF_BEGIN();
                 const int j = inf.j, b = inf.b, g = inf.g;
                 const int s = j % kRing;
                 const int ws = (j % P.nW) * P.W;
                 const int we = min(P.L, ws + P.W);
                 const int ta = ws + inf.c * kCombTokens, tb = min(we, ta + kCombTokens);
-                for (int t = ta; t < tb; ++t) {
-                    const int ne = min(t / kChunk, P.nc);
-                    const int nsel = min(P.K, ne);
-                    const int32_t *ix = idx + (((int64_t)b * P.L + t) * P.hkv + g) * P.K;
-                    for (int e = tid; e < G * D / 8; e += 128) {
-                        float acc[8];
+                constexpr int NCH = G * D / 8;  // 16-byte chunks per (token, slot) block
+                constexpr int TU = 4;           // tokens whose slot loads are in flight together
+                // each thread owns chunk e of every token of the item
+                for (int e = tid; e < NCH; e += 128) {
+                    for (int t = ta; t < tb; t += TU) {
+                        float acc[TU][8];
+                        int nsel[TU];
 #pragma unroll
-                        for (int q = 0; q < 8; ++q) acc[q] = 0.f;
-                        for (int k = 0; k < nsel; ++k) {
-                            const int c = ix[k];
-                            if (c < 0 || c >= ne) continue;
-                            const uint4 raw =
-                                ldcg_u4(part + ((int64_t)((s * P.W + (t - ws)) * P.K + k) * G) * D + e * 8);
-                            const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+                        for (int u = 0; u < TU; ++u) {
+                            nsel[u] = (t + u < tb) ? min(P.K, min((t + u) / kChunk, P.nc)) : 0;
 #pragma unroll
-                            for (int q = 0; q < 4; ++q) {
-                                const float2 f = __bfloat1622float2(h2[q]);
-                                acc[2 * q] += f.x;
-                                acc[2 * q + 1] += f.y;
-                            }
+                            for (int q = 0; q < 8; ++q) acc[u][q] = 0.f;
                         }
-                        uint4 pk;
-                        __nv_bfloat162 a0 = __floats2bfloat162_rn(acc[0], acc[1]);
-                        __nv_bfloat162 a1 = __floats2bfloat162_rn(acc[2], acc[3]);
-                        __nv_bfloat162 a2 = __floats2bfloat162_rn(acc[4], acc[5]);
-                        __nv_bfloat162 a3 = __floats2bfloat162_rn(acc[6], acc[7]);
-                        pk.x = *reinterpret_cast<uint32_t *>(&a0); pk.y = *reinterpret_cast<uint32_t *>(&a1);
-                        pk.z = *reinterpret_cast<uint32_t *>(&a2); pk.w = *reinterpret_cast<uint32_t *>(&a3);
-                        *reinterpret_cast<uint4 *>(out + (((int64_t)b * P.L + t) * P.hq + g * G) * D + e * 8) = pk;
+                        for (int k0 = 0; k0 < P.K; k0 += 8) {
+                            uint4 raw[TU][8];
+#pragma unroll
+                            for (int u = 0; u < TU; ++u) {
+                                const __nv_bfloat16 *base =
+                                    part + ((int64_t)(s * P.W + (t + u - ws)) * P.K * G) * D + e * 8;
+#pragma unroll
+                                for (int k = 0; k < 8; ++k)
+                                    if (k0 + k < nsel[u]) raw[u][k] = ldcg_u4(base + (int64_t)(k0 + k) * G * D);
+                            }
+#pragma unroll
+                            for (int u = 0; u < TU; ++u)
+#pragma unroll
+                                for (int k = 0; k < 8; ++k)
+                                    if (k0 + k < nsel[u]) {
+                                        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw[u][k]);
+#pragma unroll
+                                        for (int q = 0; q < 4; ++q) {
+                                            const float2 f = __bfloat1622float2(h2[q]);
+                                            acc[u][2 * q] += f.x;
+                                            acc[u][2 * q + 1] += f.y;
+                                        }
+                                    }
+                        }
+#pragma unroll
+                        for (int u = 0; u < TU; ++u) {
+                            if (t + u >= tb) break;
+                            uint4 pk;
+                            __nv_bfloat162 a0 = __floats2bfloat162_rn(acc[u][0], acc[u][1]);
+                            __nv_bfloat162 a1 = __floats2bfloat162_rn(acc[u][2], acc[u][3]);
+                            __nv_bfloat162 a2 = __floats2bfloat162_rn(acc[u][4], acc[u][5]);
+                            __nv_bfloat162 a3 = __floats2bfloat162_rn(acc[u][6], acc[u][7]);
+                            pk.x = *reinterpret_cast<uint32_t *>(&a0); pk.y = *reinterpret_cast<uint32_t *>(&a1);
+                            pk.z = *reinterpret_cast<uint32_t *>(&a2); pk.w = *reinterpret_cast<uint32_t *>(&a3);
+                            *reinterpret_cast<uint4 *>(out + (((int64_t)b * P.L + t + u) * P.hq + g * G) * D + e * 8) = pk;
+                        }
+                    }
+                }
+                wg_sync();
+                // the combined partials are dead: drop their L2 lines without writing them back
+                {
+                    const int64_t blk_bytes = (int64_t)G * D * 2;  // one (token, slot) block
+                    for (int t = ta; t < tb; ++t) {
+                        const int nsel = min(P.K, min(t / kChunk, P.nc));
+                        const char *base = reinterpret_cast<const char *>(part) +
+                                           (int64_t)(s * P.W + (t - ws)) * P.K * blk_bytes;
+                        const int lines = (int)(nsel * blk_bytes / 128);
+                        for (int l = tid; l < lines; l += 128) discard_l2(base + (int64_t)l * 128);
                     }
                 }
                 wg_sync();
@@ -536,12 +634,17 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                     atomicAdd(&comb_done[j], 1);
                     mbar_arrive(&B.info_empty[ii]);
                 }
+                PROF_END(8);
                 ++it;
                 continue;
             }
             // ---------------- softmax of this tile
             const int sb = tseq & 1;
+            PROF_BEGIN();
             if (!wg_wait(&B.s_full[sb], (tseq >> 1) & 1)) { ok = false; break; }
+            PROF_END(2);
+            PROF_INC(12);
+            PROF_BEGIN();
             tc_fence_after();
             float x0[32], x1[32];
             tmem_ld32(lane_base + sb * 64, x0);
@@ -572,8 +675,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                     x1[i] = exp2f(fmaf(x1[i], L2E, -mb));
                     z += x0[i] + x1[i];
                 }
-                const int64_t srow = (((int64_t)inf.b * P.L + t) * P.hkv + inf.g) * P.K + slot;
-                coef = wsel[srow] / z;
+                coef = inf.w[ti] / z;
                 if (lse) lse[(((int64_t)inf.b * P.L + t) * P.hq + inf.g * G + hh) * P.K + slot] = m + logf(z);
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) {
@@ -593,6 +695,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             }
             fence_proxy_async_smem();
             mbar_arrive(&B.p_full[sb]);
+            PROF_END(3);
             // epilogue of the previous tile while this tile's O = P.V runs
             if (pe >= 0 && !epilogue()) { ok = false; break; }
             pe = 1; pe_buf = sb; pe_seq = tseq; pe_ii = ii; pe_coef = coef;
@@ -600,9 +703,73 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             ++it;
         }
         if (ok && pe >= 0 && !epilogue()) ok = false;
-        if (ok) flush_counts();
         if (!ok) { *abort_flag = 1; if (tid == 0) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 5, it); }
-        if (tid == 0) bulk_wait<0>();
+        // tell the store warp to finish (after its last hand-off was taken)
+        if (tid == 0) {
+            if (nreq > 0) mbar_wait(st_free, (nreq - 1) & 1, kWaitNs);
+            *st_req = -1;
+            mbar_arrive(st_full);
+        }
+#ifdef HSA_TC_PROFILE
+        prof_acc[0] = clock64() - prof_start;
+        if (tid == 0) PROF_DUMP(blockIdx.x * 48 + 32);
+#endif
+    } else {
+        // ============================================================ store warp
+        // Takes the staged partial outputs of each tile, issues their TMA stores
+        // (one lane per (token, d-half) box), releases the staging buffer once
+        // the TMA engine has read it, and counts the tile into tiles_done[window]
+        // once its stores are complete (kLag hand-offs later, or when idle).
+        constexpr int kLag = 6;
+        int lagj[kLag + 1];
+        int nlag = 0;
+        int k = 0;
+        bool ok = true;
+        auto count_oldest = [&](bool all) {
+            if (all) bulk_wait<0>(); else bulk_wait<kLag>();
+            __syncwarp();
+            if (lane == 0) {
+                fence_proxy_async_global();
+                __threadfence();
+            }
+            const int n = all ? nlag : 1;
+            if (lane == 0)
+                for (int i = 0; i < n; ++i) atomicAdd(&tiles_done[lagj[i]], 1);
+            for (int i = 0; i + n < nlag; ++i) lagj[i] = lagj[i + n];
+            nlag -= n;
+        };
+        while (true) {
+            // idle: finish and count everything outstanding before blocking
+            int ready = 0;
+            if (lane == 0) ready = mbar_test(st_full, k & 1) ? 1 : 0;
+            if (!__shfl_sync(0xffffffffu, ready, 0) && nlag > 0) count_oldest(true);
+            if (!warp_wait(st_full, k & 1)) { ok = false; break; }
+            const int ii = *st_req;
+            if (ii < 0) break;
+            const TileInfo &inf = info[ii];
+            const int s = inf.j % kRing;
+            const int ws = (inf.j % P.nW) * P.W;
+            const uint8_t *stg = sm + L::OFF_ST;
+            if (lane < inf.ntok * L::NH) {
+                const int i = lane / L::NH, h = lane % L::NH;
+                const int prow = ((s * P.W + (inf.tok[i] - ws)) * P.K + inf.slot[i]) * G;
+                tma_store_2d(&tm_part, stg + h * L::QHALF + i * G * 128, h * 64, prow);
+            }
+            bulk_commit();
+            bulk_wait_read<0>();
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(st_free);
+                mbar_arrive(&B.info_empty[ii]);
+            }
+            lagj[nlag++] = inf.j;
+            if (nlag > kLag) count_oldest(false);
+            ++k;
+        }
+        if (nlag > 0) count_oldest(true);
+        if (!ok) { *abort_flag = 1; if (lane == 0) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 6, k); }
+        bulk_wait<0>();
+        __syncwarp();
     }
 
     tc_fence_before();
@@ -665,6 +832,12 @@ cudaError_t launch_tc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv,
 }
 
 }  // namespace
+
+#ifdef HSA_TC_PROFILE
+extern "C" HSA_API int hsa_debug_tc_profile(void *dev_buf) {
+    return cudaMemcpyToSymbol(g_tc_prof, &dev_buf, sizeof(void *)) == cudaSuccess ? 0 : 4;
+}
+#endif
 
 bool attend_tc_supported(const Shape &sh) {
     return sh.bf16 && (sh.d == 64 || sh.d == 128) && (sh.G == 8 || sh.G == 16) && sh.K <= 16 &&

@@ -94,6 +94,49 @@ __global__ void plan_segments_kernel(AttendPlan plan) {
     }
 }
 
+// One block per step s: writes the descriptors of window s's units and of
+// window s-1's combine items at their queue positions.
+__global__ void __launch_bounds__(256) plan_fill_kernel(const int32_t *__restrict__ hist,
+                                                        const int32_t *__restrict__ chunk_off, AttendPlan plan) {
+    const int s = blockIdx.x;
+    const int base = plan.seg_start[s];
+    const int nc = plan.nc, ntb = plan.ntb;
+    int units = 0;
+    if (s < plan.J) {
+        const int j = s;
+        units = plan.win_units[j];
+        const int bg = j / plan.nW, w = j % plan.nW;
+        const int tb0 = w * (plan.W / kInvTokBlock);
+        const int tb1 = min(ntb, (w + 1) * (plan.W / kInvTokBlock));
+        const int32_t *H = hist + (int64_t)bg * ntb * nc;
+        const int32_t *off = chunk_off + (int64_t)bg * (nc + 1);
+        const int32_t *up = plan.unit_prefix + (int64_t)j * (nc + 1);
+        for (int c = threadIdx.x; c < nc; c += blockDim.x) {
+            const int u0 = up[c], u1 = up[c + 1];
+            if (u0 == u1) continue;
+            const int e0 = H[(int64_t)tb0 * nc + c];
+            const int e1 = (tb1 < ntb) ? H[(int64_t)tb1 * nc + c] : off[c + 1];
+            const int nt = (e1 - e0 + plan.TT - 1) / plan.TT;
+            for (int u = u0; u < u1; ++u) {
+                const int t0 = (u - u0) * kUnitTiles;
+                const int q = base + u;
+                if (q >= plan.max_items) continue;
+                plan.items[2 * q] = make_int4(0, j, c, e0);
+                plan.items[2 * q + 1] = make_int4(e1, t0, min(nt, t0 + kUnitTiles), 0);
+            }
+        }
+    }
+    if (s >= 1) {
+        const int nco = plan.win_ncomb[s - 1];
+        for (int v = threadIdx.x; v < nco; v += blockDim.x) {
+            const int q = base + units + v;
+            if (q >= plan.max_items) continue;
+            plan.items[2 * q] = make_int4(1, s - 1, v, 0);
+            plan.items[2 * q + 1] = make_int4(0, 0, 0, 0);
+        }
+    }
+}
+
 cudaError_t launch_plan(const Shape &sh, const BwdWs &inv, const AttendPlan &plan, cudaStream_t st) {
     const size_t smem = sizeof(int) * (size_t)sh.nc;
     cudaError_t e = set_smem_once((const void *)plan_windows_kernel, smem);
@@ -101,6 +144,8 @@ cudaError_t launch_plan(const Shape &sh, const BwdWs &inv, const AttendPlan &pla
     plan_windows_kernel<<<plan.J, 1024, smem, st>>>(inv.hist, inv.chunk_off, plan);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     plan_segments_kernel<<<1, 32, 0, st>>>(plan);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    plan_fill_kernel<<<plan.J + 1, 256, 0, st>>>(inv.hist, inv.chunk_off, plan);
     return cudaGetLastError();
 }
 

@@ -50,6 +50,7 @@ struct FwdWs {
     float *kbar;
     int32_t *idx;
     float *w;
+    __nv_bfloat16 *kb_hi, *kb_lo;  // split pooled keys for the tensor-core scores
     bool tc;             // chunk-major tensor-core path
     BwdWs inv;           // token->chunk lists (hist, chunk_off, seg_off, entries)
     AttendPlan plan;
@@ -62,6 +63,10 @@ static FwdWs carve_fwd(const Shape &sh, void *ws, size_t *bytes) {
     f.kbar = c.take<float>((size_t)sh.B * sh.hkv * sh.nc * sh.d);
     f.idx = c.take<int32_t>((size_t)sh.B * sh.L * sh.hkv * sh.K);
     f.w = c.take<float>((size_t)sh.B * sh.L * sh.hkv * sh.K);
+    if (select_tc_supported(sh)) {
+        f.kb_hi = c.take<__nv_bfloat16>((size_t)sh.B * sh.hkv * sh.nc * sh.d);
+        f.kb_lo = c.take<__nv_bfloat16>((size_t)sh.B * sh.hkv * sh.nc * sh.d);
+    }
     f.tc = attend_tc_supported(sh);
     if (f.tc) {
         const int ntb = (int)ceil_div(sh.L, kInvTokBlock);
@@ -111,8 +116,11 @@ static size_t ws_size(const Shape &sh, int op) {
     size_t bytes = kWsHeader;
     switch (op) {
         case HSA_OP_POOL:
-        case HSA_OP_SELECT:
         case HSA_OP_DECODE:
+            return bytes;
+        case HSA_OP_SELECT:
+            if (select_tc_supported(sh))
+                bytes += 2 * round_up((int64_t)sizeof(__nv_bfloat16) * sh.B * sh.hkv * sh.nc * sh.d, 256);
             return bytes;
         case HSA_OP_FWD:
             carve_fwd(sh, nullptr, &bytes);
@@ -145,10 +153,21 @@ static cudaError_t clear_status(void *ws, cudaStream_t st) {
     return cudaMemsetAsync(ws, 0, sizeof(DevStatus), st);
 }
 
+// selection (a2-a4): tensor-core scores for bf16 inputs, CUDA cores otherwise
+static cudaError_t run_select(const Shape &sh, const void *q_slc, const float *kbar, __nv_bfloat16 *hi,
+                              __nv_bfloat16 *lo, int32_t *idx, float *w, DevStatus *ds, cudaStream_t st);
+
 // run a launcher inside a timing bracket of `kind` covering `n` kernel launches
 template <typename F> static cudaError_t timed(int kind, int n, cudaStream_t st, F &&f) {
     TimedLaunch tl(kind, n, st);
     return f();
+}
+
+static cudaError_t run_select(const Shape &sh, const void *q_slc, const float *kbar, __nv_bfloat16 *hi,
+                              __nv_bfloat16 *lo, int32_t *idx, float *w, DevStatus *ds, cudaStream_t st) {
+    TimedLaunch tl(HSA_K_SELECT, hi ? 2 : 1, st);
+    if (hi && lo) return launch_select_tc(sh, q_slc, kbar, hi, lo, idx, w, ds, st);
+    return launch_select_simt(sh, q_slc, kbar, idx, w, ds, st);
 }
 
 }  // namespace hsa
@@ -189,7 +208,13 @@ hsa_status_t hsa_select(const hsa_shape_t *shape, const void *q_slc, const void 
     DevStatus *ds = static_cast<DevStatus *>(ws);
     cudaError_t e = clear_status(ws, st);
     if (e == cudaSuccess) e = timed(HSA_K_POOL, 1, st, [&] { return launch_pool(sh, k, kbar, ds, st); });
-    if (e == cudaSuccess) e = timed(HSA_K_SELECT, 1, st, [&] { return launch_select_simt(sh, q_slc, kbar, idx, w, ds, st); });
+    __nv_bfloat16 *hi = nullptr, *lo = nullptr;
+    if (select_tc_supported(sh)) {
+        Carver c{static_cast<char *>(ws)};
+        hi = c.take<__nv_bfloat16>((size_t)sh.B * sh.hkv * sh.nc * sh.d);
+        lo = c.take<__nv_bfloat16>((size_t)sh.B * sh.hkv * sh.nc * sh.d);
+    }
+    if (e == cudaSuccess) e = run_select(sh, q_slc, kbar, hi, lo, idx, w, ds, st);
     return cuda_status(e);
 }
 
@@ -211,7 +236,7 @@ hsa_status_t hsa_fwd(const hsa_shape_t *shape, const void *q, const void *k, con
     if (w) f.w = w;
     cudaError_t e = clear_status(ws, st);
     if (e == cudaSuccess) e = timed(HSA_K_POOL, 1, st, [&] { return launch_pool(sh, k, f.kbar, ds, st); });
-    if (e == cudaSuccess) e = timed(HSA_K_SELECT, 1, st, [&] { return launch_select_simt(sh, q_slc, f.kbar, f.idx, f.w, ds, st); });
+    if (e == cudaSuccess) e = run_select(sh, q_slc, f.kbar, f.kb_hi, f.kb_lo, f.idx, f.w, ds, st);
     if (!f.tc) {
         if (e == cudaSuccess)
             e = timed(HSA_K_ATTEND_SIMT, 1, st, [&] { return launch_attend_simt(sh, q, k, v, f.idx, f.w, o, lse, ds, st); });
@@ -246,7 +271,12 @@ hsa_status_t hsa_decode(const hsa_shape_t *shape, const void *q, const void *q_s
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     DevStatus *ds = static_cast<DevStatus *>(ws);
     cudaError_t e = clear_status(ws, st);
-    if (e == cudaSuccess) e = timed(HSA_K_DECODE, 1, st, [&] { return launch_decode_simt(sh, q, q_slc, k_cache, v_cache, kbar, o, idx, w, ds, st); });
+    if (e == cudaSuccess)
+        e = timed(HSA_K_DECODE, 1, st, [&] {
+            return decode_cluster_supported(sh)
+                       ? launch_decode_cluster(sh, q, q_slc, k_cache, v_cache, kbar, o, idx, w, ds, st)
+                       : launch_decode_simt(sh, q, q_slc, k_cache, v_cache, kbar, o, idx, w, ds, st);
+        });
     return cuda_status(e);
 }
 

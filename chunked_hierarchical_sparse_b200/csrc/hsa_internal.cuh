@@ -105,6 +105,12 @@ cudaError_t launch_decode_simt(const Shape &sh, const void *q, const void *q_slc
                                const void *vc, const float *kbar, void *o, int32_t *idx_out,
                                float *w_out, DevStatus *ds, cudaStream_t st);
 
+// Decode on a thread-block cluster per (b, g) (DSMEM exchange of scores and partials).
+bool decode_cluster_supported(const Shape &sh);
+cudaError_t launch_decode_cluster(const Shape &sh, const void *q, const void *q_slc, const void *kc,
+                                  const void *vc, const float *kbar, void *o, int32_t *idx_out, float *w_out,
+                                  DevStatus *ds, cudaStream_t st);
+
 // Backward pieces.
 struct BwdWs {
     float *dkbar;     // [B,hkv,nc,d] fp32 accumulator (zeroed by the launcher)
@@ -163,6 +169,11 @@ inline int attend_window(int K, int G, int d) {
     if (w > 4096) w = 4096;
     return (int)w;
 }
+
+bool select_tc_supported(const Shape &sh);
+// Chunk selection with tensor-core scores; hi/lo: [B,hkv,nc,d] bf16 scratch.
+cudaError_t launch_select_tc(const Shape &sh, const void *q_slc, const float *kbar, __nv_bfloat16 *hi,
+                             __nv_bfloat16 *lo, int32_t *idx, float *w, DevStatus *ds, cudaStream_t st);
 
 cudaError_t launch_plan(const Shape &sh, const BwdWs &inv, const AttendPlan &plan, cudaStream_t st);
 bool attend_tc_supported(const Shape &sh);

@@ -53,9 +53,17 @@ __device__ unsigned long long *g_tc_prof = nullptr;
 
 namespace {
 
-constexpr int kThreads = 224;  // 7 warps: producer, MMA, 4 softmax/epilogue, store
+// 12 warps in three aligned warpgroups:
+//   warps 0-3 softmax / epilogue, warps 4-7 combine items,
+//   warp 8 producer, warp 9 MMA issuer, warp 10 store warp, warp 11 idle
+constexpr int kThreads = 384;
+constexpr int kWarpComb = 4, kWarpProd = 8, kWarpMma = 9, kWarpStore = 10;
+constexpr int kComb = 4;  // combine-item ring entries
 constexpr int kInfo = 4;                 // tile-info ring entries
-constexpr uint64_t kWaitNs = 2000000000ull;  // 2 s bound on any single wait
+#ifndef HSA_WAIT_NS
+#define HSA_WAIT_NS 2000000000ull
+#endif
+constexpr uint64_t kWaitNs = HSA_WAIT_NS;  // bound on any single wait (default 2 s)
 
 enum ItemType : int { kItemTile = 0, kItemComb = 1, kItemEnd = 2 };
 
@@ -85,8 +93,9 @@ template <int D> struct Smem {
     static constexpr int OFF_P = OFF_V + 2 * KVBYTES;
     static constexpr int OFF_ST = OFF_P + 2 * PBYTES;
     static constexpr int OFF_INFO = OFF_ST + STBYTES;
-    static constexpr int OFF_BAR = OFF_INFO + kInfo * (int)sizeof(TileInfo);
-    static constexpr int NBAR = 2 * kInfo + 2 * 2 + 2 * 2 + 2 * 2 + 2 + 2 * 2 + 1 + 2;
+    static constexpr int OFF_COMB = OFF_INFO + kInfo * (int)sizeof(TileInfo);
+    static constexpr int OFF_BAR = OFF_COMB + kComb * 16;
+    static constexpr int NBAR = 2 * kInfo + 2 * 2 + 2 * 2 + 2 * 2 + 2 + 2 * 2 + 1 + 2 + 2 * kComb;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_MISC + 64;
     static constexpr int ALLOC = BYTES + 1024;  // slack for 1 KB alignment
@@ -118,7 +127,7 @@ __device__ bool spin_geq(const int32_t *p, int target) {
     }
 }
 
-__device__ __forceinline__ void wg_sync() {  // named barrier 1 over warps 2..5
+__device__ __forceinline__ void wg_sync() {  // named barrier 1 over the softmax warps 0..3
     asm volatile("bar.sync 1, 128;" ::: "memory");
 }
 
@@ -161,7 +170,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     volatile int *st_req = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 48);  // info index, -1 = end
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 16);
-    volatile int *wg_flag = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 32);  // [2]
+    volatile int *wg_flag = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 32);  // [2] softmax group
+    volatile int *cg_flag = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 56);  // [2] combine group
+    int4 *comb_ring = reinterpret_cast<int4 *>(sm + L::OFF_COMB);                      // {j, b, g, item}
+    uint64_t *comb_full = st_free + 1;                                                  // [kComb]
+    uint64_t *comb_empty = comb_full + kComb;                                           // [kComb]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -176,14 +189,15 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         mbar_init(mma_done, 1);
         mbar_init(st_full, 1);
         mbar_init(st_free, 1);
+        for (int i = 0; i < kComb; ++i) { mbar_init(&comb_full[i], 1); mbar_init(&comb_empty[i], 1); }
         *abort_flag = 0;
         mbar_fence_init();
     }
-    if (warp == 1) {
+    if (warp == kWarpMma) {
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
-    if (warp == 0 && lane == 0) {
+    if (warp == kWarpProd && lane == 0) {
         prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v); prefetch_tmap(&tm_part);
     }
     tc_fence_before();
@@ -203,11 +217,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         return __shfl_sync(0xffffffffu, r, 0) != 0;
     };
 
-    if (warp == 0) {
+    if (warp == kWarpProd) {
         // ============================================================ producer
         PROF_DECL
         const long long prof_start = clock64();
-        int it = 0, qc = 0, kvc = 0;
+        int it = 0, qc = 0, kvc = 0, ncomb_sent = 0;
         bool ok = true;
         const int total = min(P.seg_start[P.J + 1], P.max_items);
         // item descriptors are fetched one ahead (queue slot + descriptor), lane 0 only
@@ -256,18 +270,30 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             PROF_END(1);
             TileInfo &inf = info[ii];
             if (type == kItemEnd) {
-                if (lane == 0) { inf.type = kItemEnd; mbar_arrive(&B.info_full[ii]); }
+                if (lane == 0) {
+                    inf.type = kItemEnd;
+                    mbar_arrive(&B.info_full[ii]);
+                    const int ci = ncomb_sent % kComb;
+                    if (ncomb_sent >= kComb) mbar_wait(&comb_empty[ci], ((ncomb_sent / kComb) - 1) & 1, kWaitNs);
+                    comb_ring[ci] = make_int4(-1, 0, 0, 0);
+                    mbar_arrive(&comb_full[ci]);
+                }
                 break;
             }
             fetch();  // next descriptor and entries in flight while this item is issued
             const int bg = j / P.nW;
             const int b = bg / P.hkv, g = bg % P.hkv;
             if (type == kItemComb) {
-                if (lane == 0) {
-                    inf.type = kItemComb; inf.j = j; inf.b = b; inf.g = g; inf.c = c;
-                    mbar_arrive(&B.info_full[ii]);
+                const int ci = ncomb_sent % kComb;
+                if (ncomb_sent >= kComb && !warp_wait(&comb_empty[ci], ((ncomb_sent / kComb) - 1) & 1)) {
+                    ok = false;
+                    break;
                 }
-                ++it;
+                if (lane == 0) {
+                    comb_ring[ci] = make_int4(j, b, g, c);
+                    mbar_arrive(&comb_full[ci]);
+                }
+                ++ncomb_sent;
                 continue;
             }
             // ---- work unit: chunk c, tiles [t0, t1) of the bucket entries [e0, e1) of window j
@@ -351,6 +377,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             *abort_flag = 1;
             if (lane == 0) {
                 report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 2, it);
+                const int ci = ncomb_sent % kComb;
+                if (ncomb_sent < kComb || mbar_wait(&comb_empty[ci], ((ncomb_sent / kComb) - 1) & 1, kWaitNs)) {
+                    comb_ring[ci] = make_int4(-1, 0, 0, 0);
+                    mbar_arrive(&comb_full[ci]);
+                }
                 // let the loads already issued land before the CTA goes away (bounded)
                 for (int s2 = 0; s2 < 2; ++s2) {
                     if (qc > s2) mbar_wait(&B.q_full[(qc - 1 - s2) & 1], ((qc - 1 - s2) >> 1) & 1, kWaitNs);
@@ -361,9 +392,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         }
 #ifdef HSA_TC_PROFILE
         prof_acc[0] = clock64() - prof_start;
-        if (lane == 0) PROF_DUMP(blockIdx.x * 48 + 0);
+        if (lane == 0) PROF_DUMP(blockIdx.x * 64 + 0);
 #endif
-    } else if (warp == 1) {
+    } else if (warp == kWarpMma) {
         // ============================================================ MMA issuer
         constexpr uint32_t idesc1 = idesc_bf16_f32(128, 64, false, false);
         constexpr uint32_t idesc2 = idesc_bf16_f32(128, D, false, true);
@@ -412,12 +443,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             const TileInfo &inf = info[ii];
             const int type = inf.type;
             if (type == kItemEnd) break;
-            if (type == kItemComb) {
-                if (pend >= 0 && !do_mma2()) { ok = false; break; }
-                if (lane == 0) mbar_arrive(&B.info_empty[ii]);
-                ++it;
-                continue;
-            }
             const int sb = tseq & 1;
             PROF_BEGIN();
             if (inf.unit_first && !warp_wait(&B.kv_full[inf.kvs], inf.kvph)) { ok = false; break; }
@@ -458,13 +483,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         __syncwarp();
 #ifdef HSA_TC_PROFILE
         prof_acc[0] = clock64() - prof_start;
-        if (lane == 0) PROF_DUMP(blockIdx.x * 48 + 16);
+        if (lane == 0) PROF_DUMP(blockIdx.x * 64 + 16);
 #endif
-    } else if (warp <= 5) {
-        // ============================================================ softmax / epilogue / combine
+    } else if (warp < kWarpComb) {
+        // ============================================================ softmax / epilogue
         const int wq = warp & 3;                 // TMEM lane quadrant of this warp
         const int r = wq * 32 + lane;            // tile row = token * G + head
-        const int tid = threadIdx.x - 64;        // 0..127
+        const int tid = threadIdx.x;             // 0..127
         const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
         int it = 0, tseq = 0, wcnt = 0;
         bool ok = true;
@@ -497,15 +522,15 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             tc_fence_after();
             uint8_t *stg = sm + L::OFF_ST;
 #pragma unroll
-            for (int h = 0; h < L::NH; ++h) {
-                float v0[32], v1[32];
-                tmem_ld32(lane_base + 128 + pe_buf * 128 + h * 64, v0);
-                tmem_ld32(lane_base + 128 + pe_buf * 128 + h * 64 + 32, v1);
+            for (int q = 0; q < 2 * L::NH; ++q) {  // 32 columns at a time
+                float v[32];
+                tmem_ld32(lane_base + 128 + pe_buf * 128 + q * 32, v);
                 tmem_wait_ld();
-                uint8_t *rowp = stg + h * L::QHALF + r * 128;
+                uint8_t *rowp = stg + (q >> 1) * L::QHALF + r * 128;
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    const float *src = (ch < 4) ? (v0 + ch * 8) : (v1 + (ch - 4) * 8);
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const int ch = (q & 1) * 4 + c4;
+                    const float *src = v + c4 * 8;
                     uint4 pk;
                     __nv_bfloat162 a0 = __floats2bfloat162_rn(src[0] * pe_coef, src[1] * pe_coef);
                     __nv_bfloat162 a1 = __floats2bfloat162_rn(src[2] * pe_coef, src[3] * pe_coef);
@@ -550,94 +575,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             const TileInfo &inf = info[ii];
             const int type = inf.type;
             if (type == kItemEnd) break;
-            if (type == kItemComb) {
-                if (pe >= 0 && !epilogue()) { ok = false; break; }
-                PROF_INC(11);
-                // every tile of window j has stored its partials
-                PROF_BEGIN();
-                int gok = 1;
-                if (tid == 0) gok = spin_geq(&tiles_done[inf.j], P.win_tiles[inf.j]) ? 1 : 0;
-                if (!wg_vote(gok)) { if (tid == 0) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 4, inf.j); ok = false; break; }
-                PROF_END(7);
-                PROF_BEGIN();
-                const int j = inf.j, b = inf.b, g = inf.g;
-                const int s = j % kRing;
-                const int ws = (j % P.nW) * P.W;
-                const int we = min(P.L, ws + P.W);
-                const int ta = ws + inf.c * kCombTokens, tb = min(we, ta + kCombTokens);
-                constexpr int NCH = G * D / 8;  // 16-byte chunks per (token, slot) block
-                constexpr int TU = 4;           // tokens whose slot loads are in flight together
-                // each thread owns chunk e of every token of the item
-                for (int e = tid; e < NCH; e += 128) {
-                    for (int t = ta; t < tb; t += TU) {
-                        float acc[TU][8];
-                        int nsel[TU];
-#pragma unroll
-                        for (int u = 0; u < TU; ++u) {
-                            nsel[u] = (t + u < tb) ? min(P.K, min((t + u) / kChunk, P.nc)) : 0;
-#pragma unroll
-                            for (int q = 0; q < 8; ++q) acc[u][q] = 0.f;
-                        }
-                        for (int k0 = 0; k0 < P.K; k0 += 8) {
-                            uint4 raw[TU][8];
-#pragma unroll
-                            for (int u = 0; u < TU; ++u) {
-                                const __nv_bfloat16 *base =
-                                    part + ((int64_t)(s * P.W + (t + u - ws)) * P.K * G) * D + e * 8;
-#pragma unroll
-                                for (int k = 0; k < 8; ++k)
-                                    if (k0 + k < nsel[u]) raw[u][k] = ldcg_u4(base + (int64_t)(k0 + k) * G * D);
-                            }
-#pragma unroll
-                            for (int u = 0; u < TU; ++u)
-#pragma unroll
-                                for (int k = 0; k < 8; ++k)
-                                    if (k0 + k < nsel[u]) {
-                                        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw[u][k]);
-#pragma unroll
-                                        for (int q = 0; q < 4; ++q) {
-                                            const float2 f = __bfloat1622float2(h2[q]);
-                                            acc[u][2 * q] += f.x;
-                                            acc[u][2 * q + 1] += f.y;
-                                        }
-                                    }
-                        }
-#pragma unroll
-                        for (int u = 0; u < TU; ++u) {
-                            if (t + u >= tb) break;
-                            uint4 pk;
-                            __nv_bfloat162 a0 = __floats2bfloat162_rn(acc[u][0], acc[u][1]);
-                            __nv_bfloat162 a1 = __floats2bfloat162_rn(acc[u][2], acc[u][3]);
-                            __nv_bfloat162 a2 = __floats2bfloat162_rn(acc[u][4], acc[u][5]);
-                            __nv_bfloat162 a3 = __floats2bfloat162_rn(acc[u][6], acc[u][7]);
-                            pk.x = *reinterpret_cast<uint32_t *>(&a0); pk.y = *reinterpret_cast<uint32_t *>(&a1);
-                            pk.z = *reinterpret_cast<uint32_t *>(&a2); pk.w = *reinterpret_cast<uint32_t *>(&a3);
-                            *reinterpret_cast<uint4 *>(out + (((int64_t)b * P.L + t + u) * P.hq + g * G) * D + e * 8) = pk;
-                        }
-                    }
-                }
-                wg_sync();
-                // the combined partials are dead: drop their L2 lines without writing them back
-                {
-                    const int64_t blk_bytes = (int64_t)G * D * 2;  // one (token, slot) block
-                    for (int t = ta; t < tb; ++t) {
-                        const int nsel = min(P.K, min(t / kChunk, P.nc));
-                        const char *base = reinterpret_cast<const char *>(part) +
-                                           (int64_t)(s * P.W + (t - ws)) * P.K * blk_bytes;
-                        const int lines = (int)(nsel * blk_bytes / 128);
-                        for (int l = tid; l < lines; l += 128) discard_l2(base + (int64_t)l * 128);
-                    }
-                }
-                wg_sync();
-                if (tid == 0) {
-                    __threadfence();
-                    atomicAdd(&comb_done[j], 1);
-                    mbar_arrive(&B.info_empty[ii]);
-                }
-                PROF_END(8);
-                ++it;
-                continue;
-            }
             // ---------------- softmax of this tile
             const int sb = tseq & 1;
             PROF_BEGIN();
@@ -712,9 +649,126 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         }
 #ifdef HSA_TC_PROFILE
         prof_acc[0] = clock64() - prof_start;
-        if (tid == 0) PROF_DUMP(blockIdx.x * 48 + 32);
+        if (tid == 0) PROF_DUMP(blockIdx.x * 64 + 32);
 #endif
-    } else {
+    } else if (warp < kWarpProd) {
+        // ============================================================ combine group
+        // Sums each window's partial outputs per token into o once every tile of
+        // the window has stored them; runs alongside the tile pipeline.
+        const int tid = threadIdx.x - kWarpComb * 32;  // 0..127
+        int ci_n = 0, vcnt = 0;
+        bool ok = true;
+        PROF_DECL
+        const long long prof_start = clock64();
+        (void)prof_start;
+        auto cg_sync = [&]() { asm volatile("bar.sync 2, 128;" ::: "memory"); };
+        auto cg_vote = [&](int v) -> bool {
+            const int slot = (vcnt++) & 1;
+            if (tid == 0) cg_flag[slot] = v;
+            cg_sync();
+            return cg_flag[slot] != 0;
+        };
+        while (true) {
+            const int ci = ci_n % kComb;
+            int v = 1;
+            PROF_BEGIN();
+            if (tid == 0) v = mbar_wait(&comb_full[ci], (ci_n / kComb) & 1, kWaitNs) ? 1 : 0;
+            if (!cg_vote(v)) { ok = false; break; }
+            PROF_END(1);
+            const int4 ce = comb_ring[ci];
+            if (ce.x < 0) break;
+            int gok = 1;
+            PROF_BEGIN();
+            if (tid == 0) gok = spin_geq(&tiles_done[ce.x], P.win_tiles[ce.x]) ? 1 : 0;
+            if (!cg_vote(gok)) { if (tid == 0) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 4, ce.x); ok = false; break; }
+            PROF_END(2);
+            PROF_INC(5);
+            PROF_BEGIN();
+            const int j = ce.x, b = ce.y, g = ce.z;
+            const int s = j % kRing;
+            const int ws = (j % P.nW) * P.W;
+            const int we = min(P.L, ws + P.W);
+            const int ta = ws + ce.w * kCombTokens, tb = min(we, ta + kCombTokens);
+            constexpr int NCH = G * D / 8;  // 16-byte chunks per (token, slot) block
+            constexpr int TU = 2;           // tokens whose slot loads are in flight together
+            // each thread owns chunk e of every token of the item
+            for (int e = tid; e < NCH; e += 128) {
+                for (int t = ta; t < tb; t += TU) {
+                    float acc[TU][8];
+                    int nsel[TU];
+#pragma unroll
+                    for (int u = 0; u < TU; ++u) {
+                        nsel[u] = (t + u < tb) ? min(P.K, min((t + u) / kChunk, P.nc)) : 0;
+#pragma unroll
+                        for (int q = 0; q < 8; ++q) acc[u][q] = 0.f;
+                    }
+                    for (int k0 = 0; k0 < P.K; k0 += 8) {
+                        uint4 raw[TU][8];
+#pragma unroll
+                        for (int u = 0; u < TU; ++u) {
+                            const __nv_bfloat16 *base =
+                                part + ((int64_t)(s * P.W + (t + u - ws)) * P.K * G) * D + e * 8;
+#pragma unroll
+                            for (int k = 0; k < 8; ++k)
+                                if (k0 + k < nsel[u]) raw[u][k] = ldcg_u4(base + (int64_t)(k0 + k) * G * D);
+                        }
+#pragma unroll
+                        for (int u = 0; u < TU; ++u)
+#pragma unroll
+                            for (int k = 0; k < 8; ++k)
+                                if (k0 + k < nsel[u]) {
+                                    const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw[u][k]);
+#pragma unroll
+                                    for (int q = 0; q < 4; ++q) {
+                                        const float2 f = __bfloat1622float2(h2[q]);
+                                        acc[u][2 * q] += f.x;
+                                        acc[u][2 * q + 1] += f.y;
+                                    }
+                                }
+                    }
+#pragma unroll
+                    for (int u = 0; u < TU; ++u) {
+                        if (t + u >= tb) break;
+                        uint4 pk;
+                        __nv_bfloat162 a0 = __floats2bfloat162_rn(acc[u][0], acc[u][1]);
+                        __nv_bfloat162 a1 = __floats2bfloat162_rn(acc[u][2], acc[u][3]);
+                        __nv_bfloat162 a2 = __floats2bfloat162_rn(acc[u][4], acc[u][5]);
+                        __nv_bfloat162 a3 = __floats2bfloat162_rn(acc[u][6], acc[u][7]);
+                        pk.x = *reinterpret_cast<uint32_t *>(&a0); pk.y = *reinterpret_cast<uint32_t *>(&a1);
+                        pk.z = *reinterpret_cast<uint32_t *>(&a2); pk.w = *reinterpret_cast<uint32_t *>(&a3);
+                        *reinterpret_cast<uint4 *>(out + (((int64_t)b * P.L + t + u) * P.hq + g * G) * D + e * 8) = pk;
+                    }
+                }
+            }
+            cg_sync();
+            PROF_END(3);
+            PROF_BEGIN();
+            // the combined partials are dead: drop their L2 lines without writing them back
+            {
+                const int64_t blk_bytes = (int64_t)G * D * 2;  // one (token, slot) block
+                for (int t = ta; t < tb; ++t) {
+                    const int nsel = min(P.K, min(t / kChunk, P.nc));
+                    const char *base = reinterpret_cast<const char *>(part) +
+                                       (int64_t)(s * P.W + (t - ws)) * P.K * blk_bytes;
+                    const int lines = (int)(nsel * blk_bytes / 128);
+                    for (int l = tid; l < lines; l += 128) discard_l2(base + (int64_t)l * 128);
+                }
+            }
+            cg_sync();
+            PROF_END(4);
+            if (tid == 0) {
+                __threadfence();
+                atomicAdd(&comb_done[j], 1);
+                mbar_arrive(&comb_empty[ci]);
+            }
+            ++ci_n;
+        }
+        if (!ok) { *abort_flag = 1; if (tid == 0) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 7, ci_n); }
+#ifdef HSA_TC_PROFILE
+        prof_acc[0] = clock64() - prof_start;
+        if (tid == 0) PROF_DUMP(blockIdx.x * 64 + 48);
+#endif
+    } else if (warp == kWarpStore) {
         // ============================================================ store warp
         // Takes the staged partial outputs of each tile, issues their TMA stores
         // (one lane per (token, d-half) box), releases the staging buffer once
@@ -775,7 +829,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, 512);
+    if (warp == kWarpMma) tmem_dealloc(tmem, 512);
 }
 
 // ------------------------------------------------------------------ host side

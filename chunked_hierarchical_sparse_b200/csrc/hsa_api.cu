@@ -54,7 +54,7 @@ struct FwdWs {
     bool tc;             // chunk-major tensor-core path
     BwdWs inv;           // token->chunk lists (hist, chunk_off, seg_off, entries)
     AttendPlan plan;
-    __nv_bfloat16 *part; // partial-output ring
+    float *acc;          // fp32 output-accumulator ring (chunk-major path)
 };
 
 static FwdWs carve_fwd(const Shape &sh, void *ws, size_t *bytes) {
@@ -76,21 +76,20 @@ static FwdWs carve_fwd(const Shape &sh, void *ws, size_t *bytes) {
         f.inv.entries = c.take<int32_t>((size_t)sh.B * sh.hkv * sh.L * sh.K);
         AttendPlan &P = f.plan;
         P.B = sh.B; P.L = sh.L; P.hq = sh.hq; P.hkv = sh.hkv; P.D = sh.d; P.K = sh.K; P.G = sh.G;
-        P.nc = sh.nc; P.ntb = ntb; P.W = attend_window(sh.K, sh.G, sh.d);
+        P.nc = sh.nc; P.ntb = ntb; P.W = (int)std::min<int64_t>(attend_window(sh.G, sh.d), round_up(std::max(sh.L, 1), kInvTokBlock));
         P.nW = (int)ceil_div(sh.L, P.W); P.J = sh.B * sh.hkv * P.nW; P.TT = 128 / sh.G;
         P.unit_prefix = c.take<int32_t>((size_t)P.J * (sh.nc + 1));
         P.win_units = c.take<int32_t>((size_t)P.J);
         P.win_tiles = c.take<int32_t>((size_t)P.J);
         P.win_ncomb = c.take<int32_t>((size_t)P.J);
-        P.seg_start = c.take<int32_t>((size_t)P.J + 2);
-        P.counters = c.take<int32_t>((size_t)2 * P.J + 1);
-        // queue items: units <= tiles <= L*K/TT + nc per (b, g) window set, plus combine items
+        P.seg_start = c.take<int32_t>((size_t)P.J + 1);
+        P.counters = c.take<int32_t>(plan_counter_count(P.J));
+        // queue items (work units): units <= tiles <= L*K/TT + nc per window, summed over (b, g)
         P.max_items = (int)std::min<int64_t>(
-            ((int64_t)sh.B * sh.hkv * ((int64_t)sh.L * sh.K / P.TT + (int64_t)P.nW * sh.nc) +
-             (int64_t)sh.B * sh.hkv * ceil_div(sh.L, kCombTokens) + P.nW * (int64_t)sh.B * sh.hkv + 16),
+            ((int64_t)sh.B * sh.hkv * ((int64_t)sh.L * sh.K / P.TT + (int64_t)P.nW * sh.nc) + 16),
             (int64_t)INT32_MAX / 4);
         P.items = c.take<int4>((size_t)2 * P.max_items);
-        f.part = c.take<__nv_bfloat16>((size_t)kRing * P.W * sh.K * sh.G * sh.d);
+        f.acc = c.take<float>(attend_acc_floats(P.W, sh.G, sh.d));
     }
     if (bytes) *bytes = c.off;
     return f;
@@ -247,12 +246,17 @@ hsa_status_t hsa_fwd(const hsa_shape_t *shape, const void *q, const void *k, con
         e = timed(HSA_K_INVERT, 3, st, [&] { return launch_invert(sh, f.idx, f.inv, ds, st); });
     if (e == cudaSuccess) e = timed(HSA_K_PLAN, 3, st, [&] { return launch_plan(sh, f.inv, f.plan, st); });
     if (e == cudaSuccess)
-        e = cudaMemsetAsync(f.plan.counters, 0, sizeof(int32_t) * ((size_t)2 * f.plan.J + 1), st);
+        e = cudaMemsetAsync(f.plan.counters, 0, sizeof(int32_t) * plan_counter_count(f.plan.J), st);
+    if (e == cudaSuccess)  // the used accumulator slots start at zero (the kernel re-zeroes them after use)
+        e = cudaMemsetAsync(f.acc, 0,
+                            sizeof(float) * std::min<size_t>(attend_acc_floats(f.plan.W, sh.G, sh.d),
+                                                             (size_t)f.plan.J * f.plan.W * sh.G * sh.d),
+                            st);
     if (e == cudaSuccess && lse)
         e = cudaMemsetAsync(lse, 0, sizeof(float) * (size_t)sh.B * sh.L * sh.hq * sh.K, st);
     if (e == cudaSuccess)
         e = timed(HSA_K_ATTEND_TC, 1, st, [&] {
-            return launch_attend_tc(sh, f.plan, f.inv, q, k, v, f.idx, f.w, f.part, o, lse, ds, st);
+            return launch_attend_tc(sh, f.plan, f.inv, q, k, v, f.idx, f.w, f.acc, o, lse, ds, st);
         });
     return cuda_status(e);
 }

@@ -141,8 +141,18 @@ constexpr int kBwdSeg = 32;        // list entries per phase-2 block
 // ---------------------------------------------------------------- chunk-major forward plan
 constexpr int kUnitTiles = 4;      // tiles of one chunk per work unit (one K/V load)
 constexpr int kCombTokens = 16;    // tokens per combine item
-constexpr int kRing = 3;           // window slots of the partial-output ring
-constexpr size_t kPartSlotBudget = size_t(32) << 20;  // bytes of partials per window
+// Output accumulators of the chunk-major forward: a ring of kRing window
+// slots, each an fp32 [W tokens][G heads][d] block that the tiles of one
+// window reduce their weighted outputs into (compile-time tunables; the ring
+// stays resident in L2 next to the K/V and query working set).
+#ifndef HSA_ACC_RING
+#define HSA_ACC_RING 3
+#endif
+#ifndef HSA_ACC_SLOT_MB
+#define HSA_ACC_SLOT_MB 16
+#endif
+constexpr int kRing = HSA_ACC_RING;
+constexpr size_t kAccSlotBudget = size_t(HSA_ACC_SLOT_MB) << 20;
 
 struct AttendPlan {
     int B, L, hq, hkv, D, K, G, nc, ntb, W, nW, J, TT;
@@ -150,25 +160,31 @@ struct AttendPlan {
     int32_t *win_units;    // [J]
     int32_t *win_tiles;    // [J]
     int32_t *win_ncomb;    // [J]
-    int32_t *seg_start;    // [J+2] queue segment starts (units of s, combines of s-1)
-    int32_t *counters;     // [2J+1] tiles_done[J], comb_done[J], queue head (zeroed per call)
+    int32_t *seg_start;    // [J+1] queue segment starts (the units of window s)
+    int32_t *counters;     // [3J+1] tiles_done[J], comb_done[J], comb_head[J], queue head (zeroed per call)
     int4 *items;           // [2 per queue item] flat descriptors in queue order
     int max_items;         // capacity of `items`
 };
 
+inline size_t plan_counter_count(int J) { return 3 * (size_t)J + 1; }
+
 // queue item descriptor (two int4): {type, j, c, e0} {e1, t0, t1, 0}
 //   type 0: work unit, chunk c, entries [e0, e1) of its bucket, tiles [t0, t1)
-//   type 1: combine item c of window j
+// Combine items are not queued: once every tile of window j is stored, the
+// combine warps of all CTAs claim window j's items from comb_head[j].
 
-// window length (tokens) of the chunk-major forward: a multiple of 256 such that
-// one window's partials (W * K * G * d bf16) fit in kPartSlotBudget
-inline int attend_window(int K, int G, int d) {
-    const int64_t per_tok = (int64_t)K * G * d * 2;
-    int64_t w = (int64_t)(kPartSlotBudget / per_tok) / kInvTokBlock * kInvTokBlock;
+// window length (tokens) of the chunk-major forward: a multiple of 256 such
+// that one window's fp32 accumulators (W * G * d * 4 bytes) fit in kAccSlotBudget
+inline int attend_window(int G, int d) {
+    const int64_t per_tok = (int64_t)G * d * 4;
+    int64_t w = (int64_t)(kAccSlotBudget / per_tok) / kInvTokBlock * kInvTokBlock;
     if (w < kInvTokBlock) w = kInvTokBlock;
-    if (w > 4096) w = 4096;
+    if (w > 8192) w = 8192;
     return (int)w;
 }
+
+// bytes of the accumulator ring of one call
+inline size_t attend_acc_floats(int W, int G, int d) { return (size_t)kRing * W * G * d; }
 
 bool select_tc_supported(const Shape &sh);
 // Chunk selection with tensor-core scores; hi/lo: [B,hkv,nc,d] bf16 scratch.
@@ -179,6 +195,6 @@ cudaError_t launch_plan(const Shape &sh, const BwdWs &inv, const AttendPlan &pla
 bool attend_tc_supported(const Shape &sh);
 cudaError_t launch_attend_tc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv, const void *q,
                              const void *k, const void *v, const int32_t *idx, const float *w,
-                             const __nv_bfloat16 *part, void *o, float *lse, DevStatus *ds, cudaStream_t st);
+                             float *acc, void *o, float *lse, DevStatus *ds, cudaStream_t st);
 
 }  // namespace hsa

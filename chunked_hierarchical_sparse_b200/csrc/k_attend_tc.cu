@@ -14,16 +14,19 @@
 //   S[128 x 64]  = Q_tile[128 x d] . K_c^T          (tcgen05, fp32 in TMEM)
 //   p = exp(x - m) / (e^{-m} + sum exp(x - m)),  x = S / sqrt(d), m = max(0, max x)
 //   O[128 x d]   = P[128 x 64] . V_c                (tcgen05, fp32 in TMEM)
-//   partial(t, h, slot) = bf16( w_{t,g,slot} / Z * O )     -> window ring (TMA store)
-// Each window's partials are summed per token by combine items of the same
-// persistent kernel once the window's tiles are done:
-//   o[t, h] = bf16( sum_slot partial(t, h, slot) ).
+//   acc[t, h] += (w_{t,g,slot} / Z) * O     (fp32 TMA reduce-add in L2 into the
+//                                             window's accumulator slot)
+// Once every tile of a window has been reduced, the convert step of the same
+// persistent kernel writes o[t, h] = bf16(acc[t, h]) and zeroes the slot for
+// the window that reuses it kRing windows later.  The slot sums each token's
+// chunk outputs in fp32, so no per-chunk partial is ever rounded or spilled.
 //
-// Roles (192 threads): warp 0 pulls queue items and issues TMA loads, warp 1
-// allocates TMEM and issues the MMAs (one elected lane), warps 2-5 do the
-// softmax, the epilogue (TMEM -> bf16 -> swizzled SMEM -> TMA store) and the
-// combine items.  Every wait is bounded (a wall-clock limit); on expiry the
-// kernel records HSA_ERR_TIMEOUT, unwinds, frees its TMEM and returns.
+// Roles (12 warps): warp 8 pulls work units and issues the TMA loads, warp 9
+// allocates TMEM and issues the MMAs (one elected lane), warps 0-3 do the
+// softmax and the epilogue (TMEM -> fp32 x coefficient -> swizzled SMEM),
+// warp 10 issues the reductions, warps 4-7 run the convert step.  Every wait
+// is bounded (a wall-clock limit); on expiry the kernel records
+// HSA_ERR_TIMEOUT, unwinds, frees its TMEM and returns.
 #include "hsa_internal.cuh"
 #include "sm100.cuh"
 
@@ -53,24 +56,23 @@ __device__ unsigned long long *g_tc_prof = nullptr;
 
 namespace {
 
-// 12 warps in three aligned warpgroups:
-//   warps 0-3 softmax / epilogue, warps 4-7 combine items,
-//   warp 8 producer, warp 9 MMA issuer, warp 10 store warp, warp 11 idle
-constexpr int kThreads = 384;
-constexpr int kWarpComb = 4, kWarpProd = 8, kWarpMma = 9, kWarpStore = 10;
-constexpr int kComb = 4;  // combine-item ring entries
+// 14 warps:
+//   warps 0-3 softmax, warps 4-7 epilogue (weighted O -> fp32 reductions into the
+//   window accumulators), warps 8-11 convert step, warp 12 producer, warp 13 MMA issuer
+constexpr int kThreads = 448;
+constexpr int kWarpEpi = 4, kWarpConv = 8, kWarpProd = 12, kWarpMma = 13;
 constexpr int kInfo = 4;                 // tile-info ring entries
 #ifndef HSA_WAIT_NS
 #define HSA_WAIT_NS 2000000000ull
 #endif
 constexpr uint64_t kWaitNs = HSA_WAIT_NS;  // bound on any single wait (default 2 s)
 
-enum ItemType : int { kItemTile = 0, kItemComb = 1, kItemEnd = 2 };
+enum ItemType : int { kItemTile = 0, kItemEnd = 2 };
 
 struct TileInfo {
     int type;
     int j;        // window
-    int b, g, c;  // sequence, group, chunk (tile) ; c = combine index for combine items
+    int b, g, c;  // sequence, group, chunk
     int ntok;     // valid tokens in the tile
     int kvs, kvph, unit_first, unit_last;
     int qs, qph;
@@ -86,20 +88,21 @@ template <int D> struct Smem {
     static constexpr int KVHALF = 64 * 128;
     static constexpr int KVBYTES = NH * KVHALF;
     static constexpr int PBYTES = 128 * 128;
-    static constexpr int STBYTES = NH * QHALF;
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + 2 * QBYTES;
     static constexpr int OFF_V = OFF_K + 2 * KVBYTES;
     static constexpr int OFF_P = OFF_V + 2 * KVBYTES;
-    static constexpr int OFF_ST = OFF_P + 2 * PBYTES;
-    static constexpr int OFF_INFO = OFF_ST + STBYTES;
-    static constexpr int OFF_COMB = OFF_INFO + kInfo * (int)sizeof(TileInfo);
-    static constexpr int OFF_BAR = OFF_COMB + kComb * 16;
-    static constexpr int NBAR = 2 * kInfo + 2 * 2 + 2 * 2 + 2 * 2 + 2 + 2 * 2 + 1 + 2 + 2 * kComb;
+    static constexpr int OFF_X = OFF_P + 2 * PBYTES;            // epilogue transpose scratch, 4 KB per warp
+    static constexpr int OFF_COEF = OFF_X + 4 * 4096;           // [kInfo][128] fp32 row coefficients w / Z
+    static constexpr int OFF_INFO = OFF_COEF + kInfo * 128 * 4;
+    static constexpr int OFF_BAR = OFF_INFO + kInfo * (int)sizeof(TileInfo);
+    static constexpr int NBAR = 3 * kInfo + 2 * 2 + 2 * 2 + 2 * 2 + 2 + 2 * 2 + 1;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_MISC + 64;
     static constexpr int ALLOC = BYTES + 1024;  // slack for 1 KB alignment
 };
+
+static_assert(Smem<128>::ALLOC <= 227 * 1024, "attention tile buffers exceed the shared memory of a CTA");
 
 struct Bars {
     uint64_t *info_full, *info_empty;  // [kInfo]
@@ -116,29 +119,29 @@ __device__ __forceinline__ int ld_acquire(const int32_t *p) {
     return v;
 }
 
-// bounded spin until *p >= target; false on timeout
-__device__ bool spin_geq(const int32_t *p, int target) {
+// 2^x with the hardware approximation (relative error about 2^-22, subnormal
+// results flushed to zero); its inputs here are <= 0 logits in base 2.
+__device__ __forceinline__ float ex2_approx(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// bounded spin until *p >= target; false on timeout or once *abort is set
+__device__ bool spin_geq_live(const int32_t *p, int target, volatile int *abort) {
     if (ld_acquire(p) >= target) return true;
     const uint64_t t0 = globaltimer();
     while (true) {
-        __nanosleep(128);
+        __nanosleep(256);
         if (ld_acquire(p) >= target) return true;
+        if (*abort) return false;
         if (globaltimer() - t0 > kWaitNs) return false;
     }
 }
 
+
 __device__ __forceinline__ void wg_sync() {  // named barrier 1 over the softmax warps 0..3
     asm volatile("bar.sync 1, 128;" ::: "memory");
-}
-
-__device__ __forceinline__ void discard_l2(const void *p) {
-    asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
-}
-
-__device__ __forceinline__ uint4 ldcg_u4(const void *p) {
-    uint4 r;
-    asm volatile("ld.global.cg.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
-    return r;
 }
 
 }  // namespace
@@ -146,10 +149,10 @@ __device__ __forceinline__ uint4 ldcg_u4(const void *p) {
 template <int D, int G>
 __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_part,
+    const __grid_constant__ CUtensorMap tm_v,
     const __grid_constant__ AttendPlan P, const int32_t *__restrict__ hist,
     const int32_t *__restrict__ chunk_off, const int32_t *__restrict__ entries,
-    const int32_t *__restrict__ idx, const float *__restrict__ wsel, const __nv_bfloat16 *__restrict__ part,
+    const int32_t *__restrict__ idx, const float *__restrict__ wsel, float *__restrict__ acc,
     __nv_bfloat16 *__restrict__ out, float *__restrict__ lse, DevStatus *ds) {
     using L = Smem<D>;
     constexpr int TT = 128 / G;
@@ -165,16 +168,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     B.p_full = B.s_empty + 2;
     B.o_full = B.p_full + 2; B.o_empty = B.o_full + 2;
     uint64_t *mma_done = B.o_empty + 2;
-    uint64_t *st_full = mma_done + 1;  // staging written (softmax group -> store warp)
-    uint64_t *st_free = mma_done + 2;  // staging read by the TMA engine (store warp -> softmax group)
-    volatile int *st_req = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 48);  // info index, -1 = end
+    uint64_t *coef_full = mma_done + 1;  // [kInfo] row coefficients written (softmax -> epilogue)
+    float *ecoef = reinterpret_cast<float *>(sm + L::OFF_COEF);
+    volatile int *eg_flag = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 48);  // [2] epilogue group
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 16);
     volatile int *wg_flag = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 32);  // [2] softmax group
-    volatile int *cg_flag = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 56);  // [2] combine group
-    int4 *comb_ring = reinterpret_cast<int4 *>(sm + L::OFF_COMB);                      // {j, b, g, item}
-    uint64_t *comb_full = st_free + 1;                                                  // [kComb]
-    uint64_t *comb_empty = comb_full + kComb;                                           // [kComb]
+    volatile int *cg_flag = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 56);  // [2] convert group
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
@@ -187,9 +187,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             mbar_init(&B.o_full[i], 1); mbar_init(&B.o_empty[i], 4);
         }
         mbar_init(mma_done, 1);
-        mbar_init(st_full, 1);
-        mbar_init(st_free, 1);
-        for (int i = 0; i < kComb; ++i) { mbar_init(&comb_full[i], 1); mbar_init(&comb_empty[i], 1); }
+        for (int i = 0; i < kInfo; ++i) mbar_init(&coef_full[i], 128);
         *abort_flag = 0;
         mbar_fence_init();
     }
@@ -198,7 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         tmem_relinquish();
     }
     if (warp == kWarpProd && lane == 0) {
-        prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v); prefetch_tmap(&tm_part);
+        prefetch_tmap(&tm_q); prefetch_tmap(&tm_k); prefetch_tmap(&tm_v);
     }
     tc_fence_before();
     __syncthreads();
@@ -207,7 +205,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
 
     int32_t *tiles_done = P.counters;
     int32_t *comb_done = P.counters + P.J;
-    int32_t *qhead = P.counters + 2 * P.J;
+    int32_t *comb_head = P.counters + 2 * P.J;
+    int32_t *qhead = P.counters + 3 * P.J;
     const float scale = 1.0f / sqrtf((float)D);
 
     // lane 0 waits, the whole warp gets the verdict (warp-uniform control flow)
@@ -221,9 +220,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         // ============================================================ producer
         PROF_DECL
         const long long prof_start = clock64();
-        int it = 0, qc = 0, kvc = 0, ncomb_sent = 0;
+        int it = 0, qc = 0, kvc = 0;
         bool ok = true;
-        const int total = min(P.seg_start[P.J + 1], P.max_items);
+        const int total = min(P.seg_start[P.J], P.max_items);
         // item descriptors are fetched one ahead (queue slot + descriptor), lane 0 only
         int4 nx0 = make_int4(kItemEnd, 0, 0, 0), nx1 = make_int4(0, 0, 0, 0);
         int nx_ea = 0, nx_eb = 0;  // the next unit's (token, slot) entries, two per lane
@@ -273,29 +272,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 if (lane == 0) {
                     inf.type = kItemEnd;
                     mbar_arrive(&B.info_full[ii]);
-                    const int ci = ncomb_sent % kComb;
-                    if (ncomb_sent >= kComb) mbar_wait(&comb_empty[ci], ((ncomb_sent / kComb) - 1) & 1, kWaitNs);
-                    comb_ring[ci] = make_int4(-1, 0, 0, 0);
-                    mbar_arrive(&comb_full[ci]);
                 }
                 break;
             }
             fetch();  // next descriptor and entries in flight while this item is issued
             const int bg = j / P.nW;
             const int b = bg / P.hkv, g = bg % P.hkv;
-            if (type == kItemComb) {
-                const int ci = ncomb_sent % kComb;
-                if (ncomb_sent >= kComb && !warp_wait(&comb_empty[ci], ((ncomb_sent / kComb) - 1) & 1)) {
-                    ok = false;
-                    break;
-                }
-                if (lane == 0) {
-                    comb_ring[ci] = make_int4(j, b, g, c);
-                    mbar_arrive(&comb_full[ci]);
-                }
-                ++ncomb_sent;
-                continue;
-            }
             // ---- work unit: chunk c, tiles [t0, t1) of the bucket entries [e0, e1) of window j
             // the unit's (token, slot) entries: up to kUnitTiles * TT <= 64, two per lane
             const int ub = e0 + t0 * TT;
@@ -305,9 +287,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             PROF_BEGIN();
             if (j >= kRing && j > guard_ok_j) {
                 int g_ok = 1;
-                if (lane == 0) g_ok = spin_geq(&comb_done[j - kRing], P.win_ncomb[j - kRing]) ? 1 : 0;
+                if (lane == 0) g_ok = spin_geq_live(&comb_done[j - kRing], P.win_ncomb[j - kRing], abort_flag) ? 1 : 0;
                 if (!__shfl_sync(0xffffffffu, g_ok, 0)) {
-                    if (lane == 0) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 1, j);
+                    if (lane == 0 && !*abort_flag) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 1, j);
                     ok = false;
                     break;
                 }
@@ -377,11 +359,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             *abort_flag = 1;
             if (lane == 0) {
                 report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 2, it);
-                const int ci = ncomb_sent % kComb;
-                if (ncomb_sent < kComb || mbar_wait(&comb_empty[ci], ((ncomb_sent / kComb) - 1) & 1, kWaitNs)) {
-                    comb_ring[ci] = make_int4(-1, 0, 0, 0);
-                    mbar_arrive(&comb_full[ci]);
-                }
                 // let the loads already issued land before the CTA goes away (bounded)
                 for (int s2 = 0; s2 < 2; ++s2) {
                     if (qc > s2) mbar_wait(&B.q_full[(qc - 1 - s2) & 1], ((qc - 1 - s2) >> 1) & 1, kWaitNs);
@@ -392,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         }
 #ifdef HSA_TC_PROFILE
         prof_acc[0] = clock64() - prof_start;
-        if (lane == 0) PROF_DUMP(blockIdx.x * 64 + 0);
+        if (lane == 0) PROF_DUMP(blockIdx.x * 80 + 0);
 #endif
     } else if (warp == kWarpMma) {
         // ============================================================ MMA issuer
@@ -483,19 +460,16 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         __syncwarp();
 #ifdef HSA_TC_PROFILE
         prof_acc[0] = clock64() - prof_start;
-        if (lane == 0) PROF_DUMP(blockIdx.x * 64 + 16);
+        if (lane == 0) PROF_DUMP(blockIdx.x * 80 + 16);
 #endif
-    } else if (warp < kWarpComb) {
-        // ============================================================ softmax / epilogue
+    } else if (warp < kWarpEpi) {
+        // ============================================================ softmax
         const int wq = warp & 3;                 // TMEM lane quadrant of this warp
         const int r = wq * 32 + lane;            // tile row = token * G + head
         const int tid = threadIdx.x;             // 0..127
         const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
         int it = 0, tseq = 0, wcnt = 0;
         bool ok = true;
-        int pe = -1, pe_buf = 0, pe_seq = 0, pe_ii = 0;  // pending epilogue
-        float pe_coef = 0.f;
-        int nreq = 0;  // staging hand-offs to the store warp so far
         PROF_DECL
         const long long prof_start = clock64();
         (void)prof_start;
@@ -512,63 +486,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             if (tid == 0) v = mbar_wait(b, par, kWaitNs) ? 1 : 0;
             return wg_vote(v);
         };
-        auto epilogue = [&]() -> bool {
-            PROF_BEGIN();
-            // the staging buffer is free once the store warp's TMA stores have read it
-            if (nreq > 0 && !wg_wait(st_free, (nreq - 1) & 1)) return false;
-            if (!wg_wait(&B.o_full[pe_buf], (pe_seq >> 1) & 1)) return false;
-            PROF_END(4);
-            PROF_BEGIN();
-            tc_fence_after();
-            uint8_t *stg = sm + L::OFF_ST;
-#pragma unroll
-            for (int q = 0; q < 2 * L::NH; ++q) {  // 32 columns at a time
-                float v[32];
-                tmem_ld32(lane_base + 128 + pe_buf * 128 + q * 32, v);
-                tmem_wait_ld();
-                uint8_t *rowp = stg + (q >> 1) * L::QHALF + r * 128;
-#pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    const int ch = (q & 1) * 4 + c4;
-                    const float *src = v + c4 * 8;
-                    uint4 pk;
-                    __nv_bfloat162 a0 = __floats2bfloat162_rn(src[0] * pe_coef, src[1] * pe_coef);
-                    __nv_bfloat162 a1 = __floats2bfloat162_rn(src[2] * pe_coef, src[3] * pe_coef);
-                    __nv_bfloat162 a2 = __floats2bfloat162_rn(src[4] * pe_coef, src[5] * pe_coef);
-                    __nv_bfloat162 a3 = __floats2bfloat162_rn(src[6] * pe_coef, src[7] * pe_coef);
-                    pk.x = *reinterpret_cast<uint32_t *>(&a0); pk.y = *reinterpret_cast<uint32_t *>(&a1);
-                    pk.z = *reinterpret_cast<uint32_t *>(&a2); pk.w = *reinterpret_cast<uint32_t *>(&a3);
-                    *reinterpret_cast<uint4 *>(rowp + ((ch ^ (r & 7)) << 4)) = pk;
-                }
-            }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&B.o_empty[pe_buf]);
-            fence_proxy_async_smem();
-            wg_sync();
-            PROF_END(5);
-            PROF_BEGIN();
-            if (tid == 0) {
-                *st_req = pe_ii;
-                mbar_arrive(st_full);
-            }
-            ++nreq;
-            PROF_END(6);
-            pe = -1;
-            return true;
-        };
 
         while (ok) {
             const int ii = it % kInfo;
             const uint32_t ipar = (it / kInfo) & 1;
-            if (pe >= 0) {  // never sit on a finished tile while the next item is not there yet
-                int ready = 1;
-                if (tid == 0) ready = mbar_test(&B.info_full[ii], ipar) ? 1 : 0;
-                if (!wg_vote(ready)) {
-                    PROF_INC(10);
-                    if (!epilogue()) { ok = false; break; }
-                }
-            }
             PROF_BEGIN();
             if (!wg_wait(&B.info_full[ii], ipar)) { ok = false; break; }
             PROF_END(1);
@@ -597,21 +518,31 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             if (valid) {
                 const int t = inf.tok[ti], slot = inf.slot[ti];
                 const float L2E = 1.4426950408889634f;
-                float m = 0.f;
+                // running maxima start at 0: the off-by-one term is a logit of 0.
+                // scale > 0, so max(scale * x) = scale * max(x) exactly.
+                float mq[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    x0[i] *= scale;
-                    x1[i] *= scale;
-                    m = fmaxf(m, fmaxf(x0[i], x1[i]));
+                for (int i = 0; i < 32; i += 2) {
+                    mq[0] = fmaxf(mq[0], x0[i]);
+                    mq[1] = fmaxf(mq[1], x0[i + 1]);
+                    mq[2] = fmaxf(mq[2], x1[i]);
+                    mq[3] = fmaxf(mq[3], x1[i + 1]);
                 }
-                const float mb = m * L2E;
-                float z = exp2f(-mb);
+                const float m = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * scale;
+                const float mb = m * L2E, sl2 = scale * L2E;
+                float zq[4] = {ex2_approx(-mb), 0.f, 0.f, 0.f};
 #pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    x0[i] = exp2f(fmaf(x0[i], L2E, -mb));
-                    x1[i] = exp2f(fmaf(x1[i], L2E, -mb));
-                    z += x0[i] + x1[i];
+                for (int i = 0; i < 32; i += 2) {
+                    x0[i] = ex2_approx(fmaf(x0[i], sl2, -mb));
+                    x0[i + 1] = ex2_approx(fmaf(x0[i + 1], sl2, -mb));
+                    x1[i] = ex2_approx(fmaf(x1[i], sl2, -mb));
+                    x1[i + 1] = ex2_approx(fmaf(x1[i + 1], sl2, -mb));
+                    zq[0] += x0[i];
+                    zq[1] += x0[i + 1];
+                    zq[2] += x1[i];
+                    zq[3] += x1[i + 1];
                 }
+                const float z = (zq[0] + zq[1]) + (zq[2] + zq[3]);
                 coef = inf.w[ti] / z;
                 if (lse) lse[(((int64_t)inf.b * P.L + t) * P.hq + inf.g * G + hh) * P.K + slot] = m + logf(z);
 #pragma unroll
@@ -633,197 +564,217 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             fence_proxy_async_smem();
             mbar_arrive(&B.p_full[sb]);
             PROF_END(3);
-            // epilogue of the previous tile while this tile's O = P.V runs
-            if (pe >= 0 && !epilogue()) { ok = false; break; }
-            pe = 1; pe_buf = sb; pe_seq = tseq; pe_ii = ii; pe_coef = coef;
+            // the row's output coefficient w / Z for the epilogue group
+            ecoef[ii * 128 + r] = coef;
+            mbar_arrive(&coef_full[ii]);
             ++tseq;
             ++it;
         }
-        if (ok && pe >= 0 && !epilogue()) ok = false;
         if (!ok) { *abort_flag = 1; if (tid == 0) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 5, it); }
-        // tell the store warp to finish (after its last hand-off was taken)
-        if (tid == 0) {
-            if (nreq > 0) mbar_wait(st_free, (nreq - 1) & 1, kWaitNs);
-            *st_req = -1;
-            mbar_arrive(st_full);
-        }
 #ifdef HSA_TC_PROFILE
         prof_acc[0] = clock64() - prof_start;
-        if (tid == 0) PROF_DUMP(blockIdx.x * 64 + 32);
+        if (tid == 0) PROF_DUMP(blockIdx.x * 80 + 32);
+#endif
+    } else if (warp < kWarpConv) {
+        // ============================================================ epilogue
+        // Per tile: O (fp32, TMEM) times the row coefficient w / Z, transposed
+        // through a 4 KB per-warp scratch so that each warp-wide vector reduction
+        // covers four whole 128-byte lines, then reduce-added into the window's
+        // accumulator slot in L2.  The tiles reduced per window are published in
+        // tiles_done[window] (after a fence) when the window changes, when the
+        // next tile is not there yet, and at the end.
+        const int wq = warp & 3;
+        const int r = wq * 32 + lane;                 // tile row of this lane's TMEM loads
+        const int tid = threadIdx.x - kWarpEpi * 32;  // 0..127
+        const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
+        float4 *xs = reinterpret_cast<float4 *>(sm + L::OFF_X + wq * 4096);  // [32 rows][8 chunks]
+        int it = 0, tseq = 0, ecnt = 0, ecnt_j = -1, vcnt = 0;
+        bool ok = true;
+        PROF_DECL
+        const long long prof_start = clock64();
+        (void)prof_start;
+        auto eg_sync = [&]() { asm volatile("bar.sync 3, 128;" ::: "memory"); };
+        auto eg_vote = [&](int v) -> bool {
+            const int slot = (vcnt++) & 1;
+            if (tid == 0) eg_flag[slot] = v;
+            eg_sync();
+            return eg_flag[slot] != 0;
+        };
+        auto eg_wait = [&](uint64_t *b, uint32_t par) -> bool {
+            int v = 1;
+            if (tid == 0) v = mbar_wait(b, par, kWaitNs) ? 1 : 0;
+            return eg_vote(v);
+        };
+        auto flush = [&]() {  // publish the reductions of the tiles counted so far
+            __threadfence();
+            eg_sync();
+            if (tid == 0) {
+                __threadfence();
+                atomicAdd(&tiles_done[ecnt_j], ecnt);
+            }
+            ecnt = 0;
+        };
+        while (ok) {
+            const int ii = it % kInfo;
+            const uint32_t ipar = (it / kInfo) & 1;
+            if (ecnt > 0) {  // never sit on unpublished tiles while the next one is not there yet
+                int ready = 1;
+                if (tid == 0) ready = mbar_test(&B.info_full[ii], ipar) ? 1 : 0;
+                if (!eg_vote(ready)) flush();
+            }
+            PROF_BEGIN();
+            if (!eg_wait(&B.info_full[ii], ipar)) { ok = false; break; }
+            PROF_END(1);
+            const TileInfo &inf = info[ii];
+            if (inf.type == kItemEnd) break;
+            if (inf.j != ecnt_j) {
+                if (ecnt > 0) flush();
+                ecnt_j = inf.j;
+            }
+            const int sb = tseq & 1;
+            PROF_BEGIN();
+            if (!eg_wait(&B.o_full[sb], (tseq >> 1) & 1)) { ok = false; break; }
+            if (!eg_wait(&coef_full[ii], ipar)) { ok = false; break; }
+            PROF_END(2);
+            PROF_BEGIN();
+            tc_fence_after();
+            const float coef = ecoef[ii * 128 + r];
+            const int s = inf.j % kRing;
+            const int ws = (inf.j % P.nW) * P.W;
+            // this lane reduces, for m = 0..7, the 16-byte chunk lane % 8 of warp row 4m + lane / 8
+            float *dst[8];
+            bool dok[8];
+#pragma unroll
+            for (int m = 0; m < 8; ++m) {
+                const int tr = wq * 32 + 4 * m + (lane >> 3);
+                const int i = tr / G;
+                dok[m] = i < inf.ntok;
+                dst[m] = acc + ((int64_t)(s * P.W + inf.tok[i] - ws) * G + tr % G) * D + (lane & 7) * 4;
+            }
+#pragma unroll
+            for (int q = 0; q < D / 32; ++q) {
+                float v[32];
+                tmem_ld32(lane_base + 128 + sb * 128 + q * 32, v);
+                tmem_wait_ld();
+#pragma unroll
+                for (int ch = 0; ch < 8; ++ch)
+                    xs[lane * 8 + (ch ^ (lane & 7))] = make_float4(v[4 * ch] * coef, v[4 * ch + 1] * coef,
+                                                                   v[4 * ch + 2] * coef, v[4 * ch + 3] * coef);
+                __syncwarp();
+#pragma unroll
+                for (int m = 0; m < 8; ++m) {
+                    const int row = 4 * m + (lane >> 3);
+                    const float4 f = xs[row * 8 + ((lane & 7) ^ (row & 7))];
+                    if (dok[m]) red_add_v4_f32(dst[m] + q * 32, f);
+                }
+                __syncwarp();
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&B.o_empty[sb]);
+            eg_sync();  // the whole group is done with this tile's info entry
+            if (tid == 0) mbar_arrive(&B.info_empty[ii]);
+            PROF_END(3);
+            ++ecnt;
+            ++tseq;
+            ++it;
+        }
+        if (ok && ecnt > 0) flush();
+        if (!ok) { *abort_flag = 1; if (tid == 0) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 6, it); }
+#ifdef HSA_TC_PROFILE
+        prof_acc[0] = clock64() - prof_start;
+        if (tid == 0) PROF_DUMP(blockIdx.x * 80 + 64);
 #endif
     } else if (warp < kWarpProd) {
-        // ============================================================ combine group
-        // Sums each window's partial outputs per token into o once every tile of
-        // the window has stored them; runs alongside the tile pipeline.
-        const int tid = threadIdx.x - kWarpComb * 32;  // 0..127
+        // ============================================================ convert group
+        // Converts each window's fp32 accumulators into o.  Every CTA's convert
+        // group walks the windows in order: it waits until all tiles of window
+        // jc are reduced, then claims jc's convert items (kCombTokens tokens
+        // each) from comb_head[jc] until none are left, so a finished window is
+        // converted by all CTAs at once while the tile pipeline moves on.
+        const int tid = threadIdx.x - kWarpConv * 32;  // 0..127
         int ci_n = 0, vcnt = 0;
         bool ok = true;
         PROF_DECL
         const long long prof_start = clock64();
         (void)prof_start;
         auto cg_sync = [&]() { asm volatile("bar.sync 2, 128;" ::: "memory"); };
-        auto cg_vote = [&](int v) -> bool {
+        auto cg_bcast = [&](int v) -> int {  // thread 0's value to the whole group
             const int slot = (vcnt++) & 1;
             if (tid == 0) cg_flag[slot] = v;
             cg_sync();
-            return cg_flag[slot] != 0;
+            return cg_flag[slot];
         };
-        while (true) {
-            const int ci = ci_n % kComb;
-            int v = 1;
-            PROF_BEGIN();
-            if (tid == 0) v = mbar_wait(&comb_full[ci], (ci_n / kComb) & 1, kWaitNs) ? 1 : 0;
-            if (!cg_vote(v)) { ok = false; break; }
-            PROF_END(1);
-            const int4 ce = comb_ring[ci];
-            if (ce.x < 0) break;
+        for (int jc = 0; jc < P.J && ok; ++jc) {
             int gok = 1;
             PROF_BEGIN();
-            if (tid == 0) gok = spin_geq(&tiles_done[ce.x], P.win_tiles[ce.x]) ? 1 : 0;
-            if (!cg_vote(gok)) { if (tid == 0) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 4, ce.x); ok = false; break; }
+            if (tid == 0) gok = spin_geq_live(&tiles_done[jc], P.win_tiles[jc], abort_flag) ? 1 : 0;
+            if (!cg_bcast(gok)) { if (tid == 0 && !*abort_flag) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 4, jc); ok = false; break; }
             PROF_END(2);
-            PROF_INC(5);
-            PROF_BEGIN();
-            const int j = ce.x, b = ce.y, g = ce.z;
-            const int s = j % kRing;
-            const int ws = (j % P.nW) * P.W;
-            const int we = min(P.L, ws + P.W);
-            const int ta = ws + ce.w * kCombTokens, tb = min(we, ta + kCombTokens);
-            constexpr int NCH = G * D / 8;  // 16-byte chunks per (token, slot) block
-            constexpr int TU = 2;           // tokens whose slot loads are in flight together
-            // each thread owns chunk e of every token of the item
-            for (int e = tid; e < NCH; e += 128) {
-                for (int t = ta; t < tb; t += TU) {
-                    float acc[TU][8];
-                    int nsel[TU];
+            const int ncomb = P.win_ncomb[jc];
+            while (true) {
+                PROF_BEGIN();
+                const int item = cg_bcast(tid == 0 ? atomicAdd(&comb_head[jc], 1) : 0);
+                PROF_END(1);
+                if (item >= ncomb) break;
+                PROF_INC(5);
+                PROF_BEGIN();
+                const int j = jc, b = (jc / P.nW) / P.hkv, g = (jc / P.nW) % P.hkv;
+                const int s = j % kRing;
+                const int ws = (j % P.nW) * P.W;
+                const int we = min(P.L, ws + P.W);
+                const int ta = ws + item * kCombTokens, tb = min(we, ta + kCombTokens);
+                // fp32 accumulators of tokens [ta, tb): G*D contiguous floats per token, and
+                // o of (token, group g): G*D contiguous bf16.  A unit is 8 floats -> 16 bytes of o.
+                constexpr int UPT = G * D / 8;  // units per token
+                constexpr int kBatch = 8;       // units in flight per thread
+                float4 *A = reinterpret_cast<float4 *>(acc + (int64_t)(s * P.W + (ta - ws)) * G * D);
+                const int nunits = (tb - ta) * UPT;
+                for (int u0 = 0; u0 < nunits; u0 += 128 * kBatch) {
+                    float4 lo[kBatch], hi[kBatch];
 #pragma unroll
-                    for (int u = 0; u < TU; ++u) {
-                        nsel[u] = (t + u < tb) ? min(P.K, min((t + u) / kChunk, P.nc)) : 0;
-#pragma unroll
-                        for (int q = 0; q < 8; ++q) acc[u][q] = 0.f;
-                    }
-                    for (int k0 = 0; k0 < P.K; k0 += 8) {
-                        uint4 raw[TU][8];
-#pragma unroll
-                        for (int u = 0; u < TU; ++u) {
-                            const __nv_bfloat16 *base =
-                                part + ((int64_t)(s * P.W + (t + u - ws)) * P.K * G) * D + e * 8;
-#pragma unroll
-                            for (int k = 0; k < 8; ++k)
-                                if (k0 + k < nsel[u]) raw[u][k] = ldcg_u4(base + (int64_t)(k0 + k) * G * D);
+                    for (int k = 0; k < kBatch; ++k) {
+                        const int u = u0 + k * 128 + tid;
+                        if (u < nunits) {
+                            lo[k] = __ldcg(A + 2 * u);
+                            hi[k] = __ldcg(A + 2 * u + 1);
                         }
-#pragma unroll
-                        for (int u = 0; u < TU; ++u)
-#pragma unroll
-                            for (int k = 0; k < 8; ++k)
-                                if (k0 + k < nsel[u]) {
-                                    const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw[u][k]);
-#pragma unroll
-                                    for (int q = 0; q < 4; ++q) {
-                                        const float2 f = __bfloat1622float2(h2[q]);
-                                        acc[u][2 * q] += f.x;
-                                        acc[u][2 * q + 1] += f.y;
-                                    }
-                                }
                     }
 #pragma unroll
-                    for (int u = 0; u < TU; ++u) {
-                        if (t + u >= tb) break;
-                        uint4 pk;
-                        __nv_bfloat162 a0 = __floats2bfloat162_rn(acc[u][0], acc[u][1]);
-                        __nv_bfloat162 a1 = __floats2bfloat162_rn(acc[u][2], acc[u][3]);
-                        __nv_bfloat162 a2 = __floats2bfloat162_rn(acc[u][4], acc[u][5]);
-                        __nv_bfloat162 a3 = __floats2bfloat162_rn(acc[u][6], acc[u][7]);
-                        pk.x = *reinterpret_cast<uint32_t *>(&a0); pk.y = *reinterpret_cast<uint32_t *>(&a1);
-                        pk.z = *reinterpret_cast<uint32_t *>(&a2); pk.w = *reinterpret_cast<uint32_t *>(&a3);
-                        *reinterpret_cast<uint4 *>(out + (((int64_t)b * P.L + t + u) * P.hq + g * G) * D + e * 8) = pk;
+                    for (int k = 0; k < kBatch; ++k) {
+                        const int u = u0 + k * 128 + tid;
+                        if (u < nunits) {
+                            const int t = ta + u / UPT, e = u % UPT;
+                            __nv_bfloat162 a0 = __floats2bfloat162_rn(lo[k].x, lo[k].y);
+                            __nv_bfloat162 a1 = __floats2bfloat162_rn(lo[k].z, lo[k].w);
+                            __nv_bfloat162 a2 = __floats2bfloat162_rn(hi[k].x, hi[k].y);
+                            __nv_bfloat162 a3 = __floats2bfloat162_rn(hi[k].z, hi[k].w);
+                            uint4 pk;
+                            pk.x = *reinterpret_cast<uint32_t *>(&a0); pk.y = *reinterpret_cast<uint32_t *>(&a1);
+                            pk.z = *reinterpret_cast<uint32_t *>(&a2); pk.w = *reinterpret_cast<uint32_t *>(&a3);
+                            // o is not read again here: streaming store
+                            __stcs(reinterpret_cast<uint4 *>(out + (((int64_t)b * P.L + t) * P.hq + g * G) * D + e * 8),
+                                   pk);
+                            // the slot starts the window kRing later at zero
+                            A[2 * u] = make_float4(0.f, 0.f, 0.f, 0.f);
+                            A[2 * u + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
+                        }
                     }
                 }
-            }
-            cg_sync();
-            PROF_END(3);
-            PROF_BEGIN();
-            // the combined partials are dead: drop their L2 lines without writing them back
-            {
-                const int64_t blk_bytes = (int64_t)G * D * 2;  // one (token, slot) block
-                for (int t = ta; t < tb; ++t) {
-                    const int nsel = min(P.K, min(t / kChunk, P.nc));
-                    const char *base = reinterpret_cast<const char *>(part) +
-                                       (int64_t)(s * P.W + (t - ws)) * P.K * blk_bytes;
-                    const int lines = (int)(nsel * blk_bytes / 128);
-                    for (int l = tid; l < lines; l += 128) discard_l2(base + (int64_t)l * 128);
+                cg_sync();
+                PROF_END(3);
+                if (tid == 0) {
+                    __threadfence();
+                    atomicAdd(&comb_done[j], 1);
                 }
+                ++ci_n;
             }
-            cg_sync();
-            PROF_END(4);
-            if (tid == 0) {
-                __threadfence();
-                atomicAdd(&comb_done[j], 1);
-                mbar_arrive(&comb_empty[ci]);
-            }
-            ++ci_n;
         }
         if (!ok) { *abort_flag = 1; if (tid == 0) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 7, ci_n); }
 #ifdef HSA_TC_PROFILE
         prof_acc[0] = clock64() - prof_start;
-        if (tid == 0) PROF_DUMP(blockIdx.x * 64 + 48);
+        if (tid == 0) PROF_DUMP(blockIdx.x * 80 + 48);
 #endif
-    } else if (warp == kWarpStore) {
-        // ============================================================ store warp
-        // Takes the staged partial outputs of each tile, issues their TMA stores
-        // (one lane per (token, d-half) box), releases the staging buffer once
-        // the TMA engine has read it, and counts the tile into tiles_done[window]
-        // once its stores are complete (kLag hand-offs later, or when idle).
-        constexpr int kLag = 6;
-        int lagj[kLag + 1];
-        int nlag = 0;
-        int k = 0;
-        bool ok = true;
-        auto count_oldest = [&](bool all) {
-            if (all) bulk_wait<0>(); else bulk_wait<kLag>();
-            __syncwarp();
-            if (lane == 0) {
-                fence_proxy_async_global();
-                __threadfence();
-            }
-            const int n = all ? nlag : 1;
-            if (lane == 0)
-                for (int i = 0; i < n; ++i) atomicAdd(&tiles_done[lagj[i]], 1);
-            for (int i = 0; i + n < nlag; ++i) lagj[i] = lagj[i + n];
-            nlag -= n;
-        };
-        while (true) {
-            // idle: finish and count everything outstanding before blocking
-            int ready = 0;
-            if (lane == 0) ready = mbar_test(st_full, k & 1) ? 1 : 0;
-            if (!__shfl_sync(0xffffffffu, ready, 0) && nlag > 0) count_oldest(true);
-            if (!warp_wait(st_full, k & 1)) { ok = false; break; }
-            const int ii = *st_req;
-            if (ii < 0) break;
-            const TileInfo &inf = info[ii];
-            const int s = inf.j % kRing;
-            const int ws = (inf.j % P.nW) * P.W;
-            const uint8_t *stg = sm + L::OFF_ST;
-            if (lane < inf.ntok * L::NH) {
-                const int i = lane / L::NH, h = lane % L::NH;
-                const int prow = ((s * P.W + (inf.tok[i] - ws)) * P.K + inf.slot[i]) * G;
-                tma_store_2d(&tm_part, stg + h * L::QHALF + i * G * 128, h * 64, prow);
-            }
-            bulk_commit();
-            bulk_wait_read<0>();
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(st_free);
-                mbar_arrive(&B.info_empty[ii]);
-            }
-            lagj[nlag++] = inf.j;
-            if (nlag > kLag) count_oldest(false);
-            ++k;
-        }
-        if (nlag > 0) count_oldest(true);
-        if (!ok) { *abort_flag = 1; if (lane == 0) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 6, k); }
-        bulk_wait<0>();
-        __syncwarp();
     }
 
     tc_fence_before();
@@ -866,13 +817,12 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, ui
 
 template <int D, int G>
 cudaError_t launch_tc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv, const void *q, const void *k,
-                      const void *v, const int32_t *idx, const float *w, const __nv_bfloat16 *part, void *o,
+                      const void *v, const int32_t *idx, const float *w, float *acc, void *o,
                       float *lse, DevStatus *ds, cudaStream_t st) {
-    CUtensorMap mq, mk, mv, mp;
+    CUtensorMap mq, mk, mv;
     if (!make_map(&mq, q, D, (uint64_t)sh.B * sh.L * sh.hq, G) ||
         !make_map(&mk, k, D, (uint64_t)sh.B * sh.hkv * sh.L, 64) ||
-        !make_map(&mv, v, D, (uint64_t)sh.B * sh.hkv * sh.L, 64) ||
-        !make_map(&mp, part, D, (uint64_t)kRing * plan.W * sh.K * G, G))
+        !make_map(&mv, v, D, (uint64_t)sh.B * sh.hkv * sh.L, 64))
         return cudaErrorInvalidValue;
     const size_t smem = Smem<D>::ALLOC;
     cudaError_t e = set_smem_once((const void *)attend_tc_kernel<D, G>, smem);
@@ -880,8 +830,8 @@ cudaError_t launch_tc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv,
     int dev = 0, sms = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    attend_tc_kernel<D, G><<<sms, kThreads, smem, st>>>(mq, mk, mv, mp, plan, inv.hist, inv.chunk_off, inv.entries,
-                                                        idx, w, part, (__nv_bfloat16 *)o, lse, ds);
+    attend_tc_kernel<D, G><<<sms, kThreads, smem, st>>>(mq, mk, mv, plan, inv.hist, inv.chunk_off, inv.entries,
+                                                        idx, w, acc, (__nv_bfloat16 *)o, lse, ds);
     return cudaGetLastError();
 }
 
@@ -900,11 +850,11 @@ bool attend_tc_supported(const Shape &sh) {
 
 cudaError_t launch_attend_tc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv, const void *q,
                              const void *k, const void *v, const int32_t *idx, const float *w,
-                             const __nv_bfloat16 *part, void *o, float *lse, DevStatus *ds, cudaStream_t st) {
-    if (sh.d == 128 && sh.G == 8) return launch_tc<128, 8>(sh, plan, inv, q, k, v, idx, w, part, o, lse, ds, st);
-    if (sh.d == 128 && sh.G == 16) return launch_tc<128, 16>(sh, plan, inv, q, k, v, idx, w, part, o, lse, ds, st);
-    if (sh.d == 64 && sh.G == 8) return launch_tc<64, 8>(sh, plan, inv, q, k, v, idx, w, part, o, lse, ds, st);
-    if (sh.d == 64 && sh.G == 16) return launch_tc<64, 16>(sh, plan, inv, q, k, v, idx, w, part, o, lse, ds, st);
+                             float *acc, void *o, float *lse, DevStatus *ds, cudaStream_t st) {
+    if (sh.d == 128 && sh.G == 8) return launch_tc<128, 8>(sh, plan, inv, q, k, v, idx, w, acc, o, lse, ds, st);
+    if (sh.d == 128 && sh.G == 16) return launch_tc<128, 16>(sh, plan, inv, q, k, v, idx, w, acc, o, lse, ds, st);
+    if (sh.d == 64 && sh.G == 8) return launch_tc<64, 8>(sh, plan, inv, q, k, v, idx, w, acc, o, lse, ds, st);
+    if (sh.d == 64 && sh.G == 16) return launch_tc<64, 16>(sh, plan, inv, q, k, v, idx, w, acc, o, lse, ds, st);
     return cudaErrorInvalidValue;
 }
 

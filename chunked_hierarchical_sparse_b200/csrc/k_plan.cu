@@ -8,10 +8,11 @@
 // TT = 128/G tokens (the tile's rows are its tokens' G query heads) and tiles
 // into work units of up to kUnitTiles tiles (one K/V load per unit).
 //
-// The persistent attention kernel pulls queue items in this order:
-//   step s = 0..J:  [units of window s (s < J)]  [combine items of window s-1 (s >= 1)]
-// so a window's partial outputs are combined right after the next window's
-// tiles were queued, while they are still in L2.
+// The persistent attention kernel pulls work units window by window (the
+// units of window s form queue segment s).  Combine items are not queued:
+// plan_windows records each window's tile and combine-item counts, and the
+// kernel's combine warps claim a window's items as soon as all its tiles are
+// stored, while its partial outputs are still in L2.
 #include "hsa_internal.cuh"
 
 namespace hsa {
@@ -82,29 +83,25 @@ __global__ void __launch_bounds__(1024) plan_windows_kernel(const int32_t *__res
     }
 }
 
-// One thread: queue segment starts over steps s = 0..J (J+2 entries).
+// One thread: queue segment starts of the windows (J+1 entries).
 __global__ void plan_segments_kernel(AttendPlan plan) {
     if (threadIdx.x != 0 || blockIdx.x != 0) return;
     int acc = 0;
     plan.seg_start[0] = 0;
-    for (int s = 0; s <= plan.J; ++s) {
-        const int len = (s < plan.J ? plan.win_units[s] : 0) + (s >= 1 ? plan.win_ncomb[s - 1] : 0);
-        acc += len;
+    for (int s = 0; s < plan.J; ++s) {
+        acc += plan.win_units[s];
         plan.seg_start[s + 1] = acc;
     }
 }
 
-// One block per step s: writes the descriptors of window s's units and of
-// window s-1's combine items at their queue positions.
+// One block per window j: writes the descriptors of its units at their queue positions.
 __global__ void __launch_bounds__(256) plan_fill_kernel(const int32_t *__restrict__ hist,
                                                         const int32_t *__restrict__ chunk_off, AttendPlan plan) {
     const int s = blockIdx.x;
     const int base = plan.seg_start[s];
     const int nc = plan.nc, ntb = plan.ntb;
-    int units = 0;
-    if (s < plan.J) {
+    {
         const int j = s;
-        units = plan.win_units[j];
         const int bg = j / plan.nW, w = j % plan.nW;
         const int tb0 = w * (plan.W / kInvTokBlock);
         const int tb1 = min(ntb, (w + 1) * (plan.W / kInvTokBlock));
@@ -126,18 +123,10 @@ __global__ void __launch_bounds__(256) plan_fill_kernel(const int32_t *__restric
             }
         }
     }
-    if (s >= 1) {
-        const int nco = plan.win_ncomb[s - 1];
-        for (int v = threadIdx.x; v < nco; v += blockDim.x) {
-            const int q = base + units + v;
-            if (q >= plan.max_items) continue;
-            plan.items[2 * q] = make_int4(1, s - 1, v, 0);
-            plan.items[2 * q + 1] = make_int4(0, 0, 0, 0);
-        }
-    }
 }
 
 cudaError_t launch_plan(const Shape &sh, const BwdWs &inv, const AttendPlan &plan, cudaStream_t st) {
+    if (plan.J == 0) return cudaSuccess;
     const size_t smem = sizeof(int) * (size_t)sh.nc;
     cudaError_t e = set_smem_once((const void *)plan_windows_kernel, smem);
     if (e != cudaSuccess) return e;
@@ -145,7 +134,7 @@ cudaError_t launch_plan(const Shape &sh, const BwdWs &inv, const AttendPlan &pla
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     plan_segments_kernel<<<1, 32, 0, st>>>(plan);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    plan_fill_kernel<<<plan.J + 1, 256, 0, st>>>(inv.hist, inv.chunk_off, plan);
+    plan_fill_kernel<<<plan.J, 256, 0, st>>>(inv.hist, inv.chunk_off, plan);
     return cudaGetLastError();
 }
 

@@ -243,7 +243,7 @@ hsa_status_t hsa_fwd(const hsa_shape_t *shape, const void *q, const void *k, con
     }
     // chunk-major tensor-core path: invert the selection, plan windows, attend
     if (e == cudaSuccess && sh.nc > 0)
-        e = timed(HSA_K_INVERT, 3, st, [&] { return launch_invert(sh, f.idx, f.inv, ds, st); });
+        e = timed(HSA_K_INVERT, 5, st, [&] { return launch_invert(sh, f.idx, f.inv, ds, st); });
     if (e == cudaSuccess) e = timed(HSA_K_PLAN, 3, st, [&] { return launch_plan(sh, f.inv, f.plan, st); });
     if (e == cudaSuccess)
         e = cudaMemsetAsync(f.plan.counters, 0, sizeof(int32_t) * plan_counter_count(f.plan.J), st);
@@ -308,7 +308,7 @@ hsa_status_t hsa_bwd(const hsa_shape_t *shape, const void *q, const void *k, con
         e = timed(HSA_K_BWD1, 1, st, [&] {
             return launch_bwd_phase1(sh, q, q_slc, k, v, dO, lse, idx, w, kbar, dq, dq_slc, b, ds, st);
         });
-    if (e == cudaSuccess) e = timed(HSA_K_INVERT, sh.nc > 0 ? 3 : 0, st, [&] { return launch_invert(sh, idx, b, ds, st); });
+    if (e == cudaSuccess) e = timed(HSA_K_INVERT, sh.nc > 0 ? 5 : 0, st, [&] { return launch_invert(sh, idx, b, ds, st); });
     if (e == cudaSuccess)
         e = timed(HSA_K_BWD2, sh.nc > 0 ? 2 : 1, st, [&] { return launch_bwd_phase2(sh, q, k, v, dO, lse, w, dk, dv, b, ds, st); });
     return cuda_status(e);

@@ -6,8 +6,9 @@
 // a stable counting sort keyed by chunk, so each chunk's entries come out in
 // increasing token order and the result is deterministic:
 //   1. per block of 256 tokens, a histogram over chunks;
-//   2. per (b, g), a prefix over token blocks for every chunk and an exclusive
-//      scan over chunks (CSR offsets);
+//   2. per (b, g), a prefix over token blocks for every chunk (column scan),
+//      an exclusive scan of the chunk totals (CSR offsets), and the offsets
+//      added to every token block's prefix;
 //   3. per token block, one warp walks its tokens in order and places each
 //      (token, slot) entry at its chunk's running cursor.
 // Entry encoding: t * 16 + slot.
@@ -76,25 +77,46 @@ __device__ int block_exclusive_scan(int *a, int n, int *wsum) {
     return total;
 }
 
-// One block (1024 threads) per (b, g): per-chunk prefix over token blocks,
-// CSR offsets over chunks, and the per-chunk segment table of phase 2.
-__global__ void __launch_bounds__(1024) inv_scan_kernel(int32_t *__restrict__ hist,
-                                                        int32_t *__restrict__ chunk_off,
-                                                        int32_t *__restrict__ seg_off, int nc,
-                                                        int ntb, int seg) {
+// Per-chunk exclusive prefix over token blocks, in place, and per-chunk totals.
+// Block (32 x 32) per (32-chunk strip, b*hkv + g): tx = chunk in the strip
+// (coalesced rows), ty = a contiguous run of token blocks.
+__global__ void __launch_bounds__(1024) inv_colscan_kernel(int32_t *__restrict__ hist,
+                                                           int32_t *__restrict__ chunk_cnt, int nc,
+                                                           int ntb) {
+    __shared__ int part[32][33];
+    const int tx = threadIdx.x, ty = threadIdx.y;
+    const int c = blockIdx.x * 32 + tx, bg = blockIdx.y;
+    const int per = (ntb + 31) / 32;
+    const int tb0 = ty * per, tb1 = min(ntb, tb0 + per);
+    int32_t *H = hist + (int64_t)bg * ntb * nc;
+    int local = 0;
+    if (c < nc)
+        for (int tb = tb0; tb < tb1; ++tb) local += H[(int64_t)tb * nc + c];
+    part[ty][tx] = local;
+    __syncthreads();
+    int run = 0;
+    for (int y = 0; y < ty; ++y) run += part[y][tx];
+    if (c < nc) {
+        for (int tb = tb0; tb < tb1; ++tb) {
+            const int v = H[(int64_t)tb * nc + c];
+            H[(int64_t)tb * nc + c] = run;
+            run += v;
+        }
+        if (ty == 31) chunk_cnt[(int64_t)bg * (nc + 1) + c] = run;
+    }
+}
+
+// One block (1024 threads) per (b, g): CSR offsets over chunks and the
+// per-chunk segment table of the backward's phase 2 (from the chunk totals).
+__global__ void __launch_bounds__(1024) inv_scan_kernel(int32_t *__restrict__ chunk_off,
+                                                        int32_t *__restrict__ seg_off, int nc, int seg) {
     extern __shared__ int sm_i[];
     int *cnt_s = sm_i;        // [nc]
     int *seg_s = sm_i + nc;   // [nc]
     __shared__ int wsum[32];
     const int bg = blockIdx.x;
-    int32_t *H = hist + (int64_t)bg * ntb * nc;
     for (int c = threadIdx.x; c < nc; c += blockDim.x) {
-        int run = 0;
-        for (int tb = 0; tb < ntb; ++tb) {
-            const int v = H[(int64_t)tb * nc + c];
-            H[(int64_t)tb * nc + c] = run;
-            run += v;
-        }
+        const int run = chunk_off[(int64_t)bg * (nc + 1) + c];  // the chunk's total, from inv_colscan
         cnt_s[c] = run;
         seg_s[c] = (run + seg - 1) / seg;
     }
@@ -104,8 +126,6 @@ __global__ void __launch_bounds__(1024) inv_scan_kernel(int32_t *__restrict__ hi
     for (int c = threadIdx.x; c < nc; c += blockDim.x) {
         chunk_off[(int64_t)bg * (nc + 1) + c] = cnt_s[c];
         seg_off[(int64_t)bg * (nc + 1) + c] = seg_s[c];
-        const int base = cnt_s[c];
-        for (int tb = 0; tb < ntb; ++tb) H[(int64_t)tb * nc + c] += base;
     }
     if (threadIdx.x == 0) {
         chunk_off[(int64_t)bg * (nc + 1) + nc] = total;
@@ -113,23 +133,38 @@ __global__ void __launch_bounds__(1024) inv_scan_kernel(int32_t *__restrict__ hi
     }
 }
 
+// hist[bg][tb][c] += chunk_off[bg][c]: per-block cursors become absolute positions.
+__global__ void __launch_bounds__(256) inv_base_kernel(int32_t *__restrict__ hist,
+                                                       const int32_t *__restrict__ chunk_off, int nc,
+                                                       int ntb) {
+    const int bg = blockIdx.y;
+    const int64_t n = (int64_t)ntb * nc;
+    int32_t *H = hist + (int64_t)bg * n;
+    const int32_t *off = chunk_off + (int64_t)bg * (nc + 1);
+    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x)
+        H[e] += off[e % nc];
+}
+
 // One warp per (token block, b*hkv + g): tokens in order, slots in parallel.
 __global__ void __launch_bounds__(32) inv_scatter_kernel(const int32_t *__restrict__ idx,
                                                          const int32_t *__restrict__ hist,
                                                          int32_t *__restrict__ entries, int L,
                                                          int hkv, int nc, int K, int ntb) {
-    extern __shared__ int cur[];  // [nc]
+    extern __shared__ int cur[];  // [nc] cursors, then [kInvTokBlock * K] the block's selections
+    int *sel = cur + nc;
     const int tb = blockIdx.x, bg = blockIdx.y, b = bg / hkv, g = bg % hkv;
     const int lane = threadIdx.x;
     const int32_t *H = hist + ((int64_t)bg * ntb + tb) * nc;
     for (int c = lane; c < nc; c += 32) cur[c] = H[c];
-    __syncwarp();
-    int32_t *E = entries + (int64_t)bg * L * K;
     const int t0 = tb * kInvTokBlock;
     const int t1 = min(t0 + kInvTokBlock, L);
+    for (int e = lane; e < (t1 - t0) * K; e += 32)
+        sel[e] = idx[(((int64_t)b * L + t0 + e / K) * hkv + g) * K + e % K];
+    __syncwarp();
+    int32_t *E = entries + (int64_t)bg * L * K;
     for (int t = t0; t < t1; ++t) {
         if (lane < K) {
-            const int c = idx[(((int64_t)b * L + t) * hkv + g) * K + lane];
+            const int c = sel[(t - t0) * K + lane];
             if (c >= 0 && c < nc && c < t / kChunk) {
                 const int pos = cur[c];
                 cur[c] = pos + 1;
@@ -146,21 +181,26 @@ cudaError_t launch_invert(const Shape &sh, const int32_t *idx, const BwdWs &ws, 
     const int ntb = (int)ceil_div(sh.L, kInvTokBlock);
     const size_t smem = sizeof(int) * (size_t)sh.nc;
     cudaError_t e;
-    if (2 * smem > 48 * 1024) {
+    const size_t ssmem = smem + sizeof(int) * (size_t)kInvTokBlock * sh.K;
+    if (2 * smem > 48 * 1024 || ssmem > 48 * 1024) {
         e = set_smem_once((const void *)inv_hist_kernel, (size_t)(smem));
         if (e != cudaSuccess) return e;
         e = set_smem_once((const void *)inv_scan_kernel, (size_t)(2 * smem));
         if (e != cudaSuccess) return e;
-        e = set_smem_once((const void *)inv_scatter_kernel, (size_t)(smem));
+        e = set_smem_once((const void *)inv_scatter_kernel, ssmem);
         if (e != cudaSuccess) return e;
     }
     dim3 grid(ntb, sh.B * sh.hkv);
     inv_hist_kernel<<<grid, 256, smem, st>>>(idx, ws.hist, sh.L, sh.hkv, sh.nc, sh.K, ntb, ds);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    inv_scan_kernel<<<sh.B * sh.hkv, 1024, 2 * smem, st>>>(ws.hist, ws.chunk_off, ws.seg_off, sh.nc,
-                                                            ntb, kBwdSeg);
+    inv_colscan_kernel<<<dim3((unsigned)ceil_div(sh.nc, 32), sh.B * sh.hkv), dim3(32, 32), 0, st>>>(
+        ws.hist, ws.chunk_off, sh.nc, ntb);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    inv_scatter_kernel<<<grid, 32, smem, st>>>(idx, ws.hist, ws.entries, sh.L, sh.hkv, sh.nc, sh.K, ntb);
+    inv_scan_kernel<<<sh.B * sh.hkv, 1024, 2 * smem, st>>>(ws.chunk_off, ws.seg_off, sh.nc, kBwdSeg);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    inv_base_kernel<<<dim3(148, sh.B * sh.hkv), 256, 0, st>>>(ws.hist, ws.chunk_off, sh.nc, ntb);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    inv_scatter_kernel<<<grid, 32, ssmem, st>>>(idx, ws.hist, ws.entries, sh.L, sh.hkv, sh.nc, sh.K, ntb);
     return cudaGetLastError();
 }
 

@@ -74,6 +74,7 @@ static FwdWs carve_fwd(const Shape &sh, void *ws, size_t *bytes) {
         f.inv.chunk_off = c.take<int32_t>((size_t)sh.B * sh.hkv * (sh.nc + 1));
         f.inv.seg_off = c.take<int32_t>((size_t)sh.B * sh.hkv * (sh.nc + 1));
         f.inv.entries = c.take<int32_t>((size_t)sh.B * sh.hkv * sh.L * sh.K);
+        f.inv.entw = c.take<float>((size_t)sh.B * sh.hkv * sh.L * sh.K);
         AttendPlan &P = f.plan;
         P.B = sh.B; P.L = sh.L; P.hq = sh.hq; P.hkv = sh.hkv; P.D = sh.d; P.K = sh.K; P.G = sh.G;
         P.nc = sh.nc; P.ntb = ntb; P.W = (int)std::min<int64_t>(attend_window(sh.G, sh.d), round_up(std::max(sh.L, 1), kInvTokBlock));
@@ -107,6 +108,7 @@ static BwdWs carve_bwd(const Shape &sh, void *ws, size_t *bytes) {
     b.chunk_off = c.take<int32_t>((size_t)sh.B * sh.hkv * (sh.nc + 1));
     b.seg_off = c.take<int32_t>((size_t)sh.B * sh.hkv * (sh.nc + 1));
     b.entries = c.take<int32_t>((size_t)sh.B * sh.hkv * sh.L * sh.K);
+    b.entw = nullptr;
     if (bytes) *bytes = c.off;
     return b;
 }
@@ -243,7 +245,7 @@ hsa_status_t hsa_fwd(const hsa_shape_t *shape, const void *q, const void *k, con
     }
     // chunk-major tensor-core path: invert the selection, plan windows, attend
     if (e == cudaSuccess && sh.nc > 0)
-        e = timed(HSA_K_INVERT, 5, st, [&] { return launch_invert(sh, f.idx, f.inv, ds, st); });
+        e = timed(HSA_K_INVERT, 5, st, [&] { return launch_invert(sh, f.idx, f.w, f.inv, ds, st); });
     if (e == cudaSuccess) e = timed(HSA_K_PLAN, 3, st, [&] { return launch_plan(sh, f.inv, f.plan, st); });
     if (e == cudaSuccess)
         e = cudaMemsetAsync(f.plan.counters, 0, sizeof(int32_t) * plan_counter_count(f.plan.J), st);
@@ -308,7 +310,7 @@ hsa_status_t hsa_bwd(const hsa_shape_t *shape, const void *q, const void *k, con
         e = timed(HSA_K_BWD1, 1, st, [&] {
             return launch_bwd_phase1(sh, q, q_slc, k, v, dO, lse, idx, w, kbar, dq, dq_slc, b, ds, st);
         });
-    if (e == cudaSuccess) e = timed(HSA_K_INVERT, sh.nc > 0 ? 5 : 0, st, [&] { return launch_invert(sh, idx, b, ds, st); });
+    if (e == cudaSuccess) e = timed(HSA_K_INVERT, sh.nc > 0 ? 5 : 0, st, [&] { return launch_invert(sh, idx, nullptr, b, ds, st); });
     if (e == cudaSuccess)
         e = timed(HSA_K_BWD2, sh.nc > 0 ? 2 : 1, st, [&] { return launch_bwd_phase2(sh, q, k, v, dO, lse, w, dk, dv, b, ds, st); });
     return cuda_status(e);

@@ -121,6 +121,7 @@ struct BwdWs {
     int32_t *chunk_off;  // [B,hkv,nc+1] CSR offsets into entries (per (b,g) base)
     int32_t *seg_off;    // [B,hkv,nc+1] phase-2 segment offsets (kBwdSeg entries each)
     int32_t *entries;    // [B,hkv, L*K] packed t*16 + slot, sorted by t per chunk
+    float *entw;         // [B,hkv, L*K] the entries' stick-breaking weights (forward only, else null)
 };
 
 cudaError_t launch_bwd_phase1(const Shape &sh, const void *q, const void *q_slc, const void *k,
@@ -128,7 +129,8 @@ cudaError_t launch_bwd_phase1(const Shape &sh, const void *q, const void *q_slc,
                               const float *w, const float *kbar, void *dq, void *dq_slc,
                               const BwdWs &ws, DevStatus *ds, cudaStream_t st);
 
-cudaError_t launch_invert(const Shape &sh, const int32_t *idx, const BwdWs &ws, DevStatus *ds,
+// w (nullable): when given, the entries' weights are gathered into ws.entw.
+cudaError_t launch_invert(const Shape &sh, const int32_t *idx, const float *w, const BwdWs &ws, DevStatus *ds,
                           cudaStream_t st);
 
 cudaError_t launch_bwd_phase2(const Shape &sh, const void *q, const void *k, const void *v,

@@ -56,12 +56,14 @@ __device__ unsigned long long *g_tc_prof = nullptr;
 
 namespace {
 
-// 14 warps:
-//   warps 0-3 softmax, warps 4-7 epilogue (weighted O -> fp32 reductions into the
-//   window accumulators), warps 8-11 convert step, warp 12 producer, warp 13 MMA issuer
-constexpr int kThreads = 448;
-constexpr int kWarpEpi = 4, kWarpConv = 8, kWarpProd = 12, kWarpMma = 13;
-constexpr int kInfo = 4;                 // tile-info ring entries
+// 16 warps:
+//   warps 0-3 softmax, warps 4-7 and 8-11 two epilogue groups (weighted O ->
+//   fp32 reductions into the window accumulators; group e takes the tiles whose
+//   O buffer is e), warps 12-13 convert step, warp 14 producer, warp 15 MMA issuer
+constexpr int kThreads = 512;
+constexpr int kWarpEpi = 4, kWarpConv = 12, kWarpProd = 14, kWarpMma = 15;
+constexpr int kConvThreads = 64;
+constexpr int kInfo = 8;                 // tile-info ring entries
 #ifndef HSA_WAIT_NS
 #define HSA_WAIT_NS 2000000000ull
 #endif
@@ -93,10 +95,10 @@ template <int D> struct Smem {
     static constexpr int OFF_V = OFF_K + 2 * KVBYTES;
     static constexpr int OFF_P = OFF_V + 2 * KVBYTES;
     static constexpr int OFF_X = OFF_P + 2 * PBYTES;            // epilogue transpose scratch, 4 KB per warp
-    static constexpr int OFF_COEF = OFF_X + 4 * 4096;           // [kInfo][128] fp32 row coefficients w / Z
+    static constexpr int OFF_COEF = OFF_X + 8 * 4096;           // [kInfo][128] fp32 row coefficients w / Z
     static constexpr int OFF_INFO = OFF_COEF + kInfo * 128 * 4;
     static constexpr int OFF_BAR = OFF_INFO + kInfo * (int)sizeof(TileInfo);
-    static constexpr int NBAR = 3 * kInfo + 2 * 2 + 2 * 2 + 2 * 2 + 2 + 2 * 2 + 1;
+    static constexpr int NBAR = 3 * kInfo + 2 * 2 + 2 * 2 + 2 * 2 + 2 + 2 * 2 + 1 + 2;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_MISC + 64;
     static constexpr int ALLOC = BYTES + 1024;  // slack for 1 KB alignment
@@ -152,7 +154,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     const __grid_constant__ CUtensorMap tm_v,
     const __grid_constant__ AttendPlan P, const int32_t *__restrict__ hist,
     const int32_t *__restrict__ chunk_off, const int32_t *__restrict__ entries,
-    const int32_t *__restrict__ idx, const float *__restrict__ wsel, float *__restrict__ acc,
+    const int32_t *__restrict__ idx, const float *__restrict__ entw, float *__restrict__ acc,
     __nv_bfloat16 *__restrict__ out, float *__restrict__ lse, DevStatus *ds) {
     using L = Smem<D>;
     constexpr int TT = 128 / G;
@@ -169,8 +171,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     B.o_full = B.p_full + 2; B.o_empty = B.o_full + 2;
     uint64_t *mma_done = B.o_empty + 2;
     uint64_t *coef_full = mma_done + 1;  // [kInfo] row coefficients written (softmax -> epilogue)
+    uint64_t *p_empty = coef_full + kInfo;  // [2] P buffer read by its O = P.V (MMA -> softmax)
     float *ecoef = reinterpret_cast<float *>(sm + L::OFF_COEF);
-    volatile int *eg_flag = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 48);  // [2] epilogue group
+    volatile int *eg_flag = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 40);  // [2][2] epilogue groups
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 16);
     volatile int *wg_flag = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 32);  // [2] softmax group
@@ -178,7 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kInfo; ++i) { mbar_init(&B.info_full[i], 1); mbar_init(&B.info_empty[i], 2); }
+        for (int i = 0; i < kInfo; ++i) { mbar_init(&B.info_full[i], 1); mbar_init(&B.info_empty[i], 3); }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&B.q_full[i], 1); mbar_init(&B.q_empty[i], 1);
             mbar_init(&B.kv_full[i], 1); mbar_init(&B.kv_empty[i], 1);
@@ -188,6 +191,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         }
         mbar_init(mma_done, 1);
         for (int i = 0; i < kInfo; ++i) mbar_init(&coef_full[i], 128);
+        for (int i = 0; i < 2; ++i) mbar_init(&p_empty[i], 1);
         *abort_flag = 0;
         mbar_fence_init();
     }
@@ -206,7 +210,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     int32_t *tiles_done = P.counters;
     int32_t *comb_done = P.counters + P.J;
     int32_t *comb_head = P.counters + 2 * P.J;
-    int32_t *qhead = P.counters + 3 * P.J;
     const float scale = 1.0f / sqrtf((float)D);
 
     // lane 0 waits, the whole warp gets the verdict (warp-uniform control flow)
@@ -218,36 +221,39 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
 
     if (warp == kWarpProd) {
         // ============================================================ producer
+        // Work units are dealt to the CTAs in queue order (unit q to CTA
+        // q mod gridDim.x), which keeps every CTA in window order.  Descriptors
+        // are loaded two units ahead and a unit's entries and weights one unit
+        // ahead, so no global-memory latency sits on the tile path.
         PROF_DECL
         const long long prof_start = clock64();
         int it = 0, qc = 0, kvc = 0;
         bool ok = true;
         const int total = min(P.seg_start[P.J], P.max_items);
-        // item descriptors are fetched one ahead (queue slot + descriptor), lane 0 only
-        int4 nx0 = make_int4(kItemEnd, 0, 0, 0), nx1 = make_int4(0, 0, 0, 0);
-        int nx_ea = 0, nx_eb = 0;  // the next unit's (token, slot) entries, two per lane
-        int guard_ok_j = -1;       // highest window whose ring guard already passed
-        auto fetch = [&]() {
-            if (lane == 0) {
-                const int q = atomicAdd(qhead, 1);
-                if (q < total) { nx0 = P.items[2 * q]; nx1 = P.items[2 * q + 1]; }
-                else { nx0 = make_int4(kItemEnd, 0, 0, 0); }
-            }
-            const int ty = __shfl_sync(0xffffffffu, nx0.x, 0);
-            if (ty == kItemTile) {
-                const int jn = __shfl_sync(0xffffffffu, nx0.y, 0);
-                const int en0 = __shfl_sync(0xffffffffu, nx0.w, 0);
-                const int en1 = __shfl_sync(0xffffffffu, nx1.x, 0);
-                const int tn0 = __shfl_sync(0xffffffffu, nx1.y, 0);
-                const int tn1 = __shfl_sync(0xffffffffu, nx1.z, 0);
-                const int32_t *En = entries + (int64_t)(jn / P.nW) * P.L * P.K;
-                const int ub = en0 + tn0 * TT;
-                const int un = min(en1, en0 + tn1 * TT) - ub;
-                nx_ea = (lane < un) ? En[ub + lane] : 0;
-                nx_eb = (lane + 32 < un) ? En[ub + lane + 32] : 0;
-            }
+        const int qstep = gridDim.x;
+        int guard_ok_j = -1;  // highest window whose ring guard already passed
+        struct Desc { int4 a, b; };
+        auto load_desc = [&](int q) -> Desc {  // every lane loads the same 32 bytes
+            Desc d;
+            if (q < total) { d.a = P.items[2 * q]; d.b = P.items[2 * q + 1]; }
+            else { d.a = make_int4(kItemEnd, 0, 0, 0); d.b = make_int4(0, 0, 0, 0); }
+            return d;
         };
-        fetch();
+        struct Pay { int ea, eb; float wa, wb; };  // a unit's (token, slot) entries and weights, two per lane
+        auto load_pay = [&](const Desc &d) -> Pay {
+            Pay p{0, 0, 0.f, 0.f};
+            if (d.a.x == kItemTile) {
+                const int64_t base = (int64_t)(d.a.y / P.nW) * P.L * P.K;
+                const int ub = d.a.w + d.b.y * TT;
+                const int un = min(d.b.x, d.a.w + d.b.z * TT) - ub;
+                if (lane < un) { p.ea = entries[base + ub + lane]; p.wa = entw[base + ub + lane]; }
+                if (lane + 32 < un) { p.eb = entries[base + ub + lane + 32]; p.wb = entw[base + ub + lane + 32]; }
+            }
+            return p;
+        };
+        int qn = blockIdx.x;  // queue index of the unit in dc
+        Desc dc = load_desc(qn), dn = load_desc(qn + qstep);
+        Pay pc = load_pay(dc);
         while (ok) {
             const int ii = it % kInfo;
             PROF_BEGIN();
@@ -255,17 +261,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             PROF_END(2);
             if (*abort_flag) { ok = false; break; }
             PROF_BEGIN();
-            const int type = __shfl_sync(0xffffffffu, nx0.x, 0);
-            const int j = __shfl_sync(0xffffffffu, nx0.y, 0);
-            const int c = __shfl_sync(0xffffffffu, nx0.z, 0);
-            const int e0 = __shfl_sync(0xffffffffu, nx0.w, 0);
-            const int e1 = __shfl_sync(0xffffffffu, nx1.x, 0);
-            const int t0 = __shfl_sync(0xffffffffu, nx1.y, 0);
-            const int t1 = __shfl_sync(0xffffffffu, nx1.z, 0);
-            const int ent_a = nx_ea, ent_b = nx_eb;
-#ifdef HSA_TC_PROFILE
-            if (ent_a == 0x7fffffff) prof_t0 = 0;  // keeps the entry loads ordered before the timer read
-#endif
+            const int type = dc.a.x, j = dc.a.y, c = dc.a.z, e0 = dc.a.w;
+            const int e1 = dc.b.x, t0 = dc.b.y, t1 = dc.b.z;
+            const int ent_a = pc.ea, ent_b = pc.eb;
+            const float w_a = pc.wa, w_b = pc.wb;
             PROF_END(1);
             TileInfo &inf = info[ii];
             if (type == kItemEnd) {
@@ -275,7 +274,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 }
                 break;
             }
-            fetch();  // next descriptor and entries in flight while this item is issued
+            {  // the next units' data in flight while this one is issued
+                const Pay pn = load_pay(dn);
+                dc = dn;
+                dn = load_desc(qn + 2 * qstep);
+                pc = pn;
+                qn += qstep;
+            }
             const int bg = j / P.nW;
             const int b = bg / P.hkv, g = bg % P.hkv;
             // ---- work unit: chunk c, tiles [t0, t1) of the bucket entries [e0, e1) of window j
@@ -321,6 +326,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 if (qc >= 2 && !warp_wait(&B.q_empty[qs], ((qc >> 1) - 1) & 1)) { ok = false; break; }
                 PROF_END(5);
                 PROF_INC(7);
+                PROF_BEGIN();
                 TileInfo &ti_ = info[ti];
                 const int lo = (tt - t0) * TT;          // first entry of this tile within the unit
                 const int ntok = min(TT, un - lo);
@@ -329,11 +335,14 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 const int va = __shfl_sync(0xffffffffu, ent_a, src);
                 const int vb = __shfl_sync(0xffffffffu, ent_b, src);
                 const int ent = (lo + lane < 32) ? va : vb;
+                const float wva = __shfl_sync(0xffffffffu, w_a, src);
+                const float wvb = __shfl_sync(0xffffffffu, w_b, src);
+                const float wgt = (lo + lane < 32) ? wva : wvb;
                 const int t = ent >> 4, slot = ent & 15;
                 if (lane < 16) {
                     ti_.tok[lane] = (lane < ntok) ? t : -1;
                     ti_.slot[lane] = (lane < ntok) ? slot : 0;
-                    ti_.w[lane] = (lane < ntok) ? wsel[(((int64_t)b * P.L + t) * P.hkv + g) * P.K + slot] : 0.f;
+                    ti_.w[lane] = (lane < ntok) ? wgt : 0.f;
                 }
                 if (lane == 0) {
                     ti_.type = kItemTile; ti_.j = j; ti_.b = b; ti_.g = g; ti_.c = c; ti_.ntok = ntok;
@@ -342,6 +351,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                     mbar_arrive_expect_tx(&B.q_full[qs], ntok * L::NH * G * 128);
                 }
                 __syncwarp();
+                PROF_END(8);
+                PROF_BEGIN();
                 if (lane < ntok) {
                     const int row = (b * P.L + t) * P.hq + g * G;
 #pragma unroll
@@ -351,6 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&B.info_full[ti]);
+                PROF_END(9);
                 ++qc;
                 ++it;
             }
@@ -369,98 +381,98 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         }
 #ifdef HSA_TC_PROFILE
         prof_acc[0] = clock64() - prof_start;
-        if (lane == 0) PROF_DUMP(blockIdx.x * 80 + 0);
+        if (lane == 0) PROF_DUMP(blockIdx.x * 96 + 0);
 #endif
     } else if (warp == kWarpMma) {
         // ============================================================ MMA issuer
+        // Two in-order streams polled by one lane: S(t) = Q_t K^T is issued as
+        // soon as the tile's Q and K are in SMEM and an S buffer is free, and
+        // O(t) = P_t V as soon as P_t is written and an O buffer is free, so a
+        // slow epilogue never holds back the scores of the following tiles.
         constexpr uint32_t idesc1 = idesc_bf16_f32(128, 64, false, false);
         constexpr uint32_t idesc2 = idesc_bf16_f32(128, D, false, true);
         PROF_DECL
         const long long prof_start = clock64();
-        int it = 0, tseq = 0;
-        int pend = -1, pend_buf = 0, pend_seq = 0, pend_last = 0, pend_kvs = 0, pend_ii = 0;
         bool ok = true;
-        auto do_mma2 = [&]() -> bool {
-            // O[pb] = P[pb] . V   (for the pending tile)
-            PROF_BEGIN();
-            if (!warp_wait(&B.p_full[pend_buf], (pend_seq >> 1) & 1)) return false;
-            PROF_END(5);
-            PROF_BEGIN();
-            if (pend_seq >= 2 && !warp_wait(&B.o_empty[pend_buf], ((pend_seq >> 1) - 1) & 1)) return false;
-            PROF_END(6);
-            tc_fence_after();
-            if (lane == 0) {
-                const uint32_t pa = smem_u32(sm + L::OFF_P + pend_buf * L::PBYTES);
-                const uint32_t vb = smem_u32(sm + L::OFF_V + pend_kvs * L::KVBYTES);
-                const uint32_t dcol = tmem + 128 + pend_buf * 128;
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ss(dcol, smem_desc_sw128(pa + ks * 32, 16, 1024),
-                                smem_desc_sw128(vb + ks * 2048, L::KVHALF, 1024), idesc2, ks > 0);
-                mma_commit(&B.o_full[pend_buf]);
-                if (pend_last) mma_commit(&B.kv_empty[pend_kvs]);
-                mbar_arrive(&B.info_empty[pend_ii]);
-            }
-            __syncwarp();
-            pend = -1;
-            return true;
-        };
-        while (ok) {
-            const int ii = it % kInfo;
-            const uint32_t ipar = (it / kInfo) & 1;
-            // never sit on a pending PV product while the next item is not there yet
-            if (pend >= 0) {
-                int ready = 0;
-                if (lane == 0) ready = mbar_test(&B.info_full[ii], ipar) ? 1 : 0;
-                if (!__shfl_sync(0xffffffffu, ready, 0) && !do_mma2()) { ok = false; break; }
-            }
-            PROF_BEGIN();
-            if (!warp_wait(&B.info_full[ii], ipar)) { ok = false; break; }
-            PROF_END(1);
-            const TileInfo &inf = info[ii];
-            const int type = inf.type;
-            if (type == kItemEnd) break;
-            const int sb = tseq & 1;
-            PROF_BEGIN();
-            if (inf.unit_first && !warp_wait(&B.kv_full[inf.kvs], inf.kvph)) { ok = false; break; }
-            PROF_END(2);
-            PROF_BEGIN();
-            if (!warp_wait(&B.q_full[inf.qs], inf.qph)) { ok = false; break; }
-            PROF_END(3);
-            PROF_BEGIN();
-            if (tseq >= 2 && !warp_wait(&B.s_empty[sb], ((tseq >> 1) - 1) & 1)) { ok = false; break; }
-            PROF_END(4);
-            tc_fence_after();
-            if (lane == 0) {
-                const uint32_t qa = smem_u32(sm + L::OFF_Q + inf.qs * L::QBYTES);
-                const uint32_t kb = smem_u32(sm + L::OFF_K + inf.kvs * L::KVBYTES);
-                const uint32_t dcol = tmem + sb * 64;
-#pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const int h = ks >> 2, kk = ks & 3;
-                    mma_bf16_ss(dcol, smem_desc_sw128(qa + h * L::QHALF + kk * 32, 16, 1024),
-                                smem_desc_sw128(kb + h * L::KVHALF + kk * 32, 16, 1024), idesc1, ks > 0);
-                }
-                mma_commit(&B.s_full[sb]);
-                mma_commit(&B.q_empty[inf.qs]);
-            }
-            __syncwarp();
-            if (pend >= 0 && !do_mma2()) { ok = false; break; }
-            pend = 1; pend_buf = sb; pend_seq = tseq; pend_last = inf.unit_last; pend_kvs = inf.kvs; pend_ii = ii;
-            ++tseq;
-            ++it;
-        }
-        if (ok && pend >= 0 && !do_mma2()) ok = false;
-        if (!ok) { *abort_flag = 1; if (lane == 0) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 3, it); }
-        // drain: every MMA issued by this warp has finished before TMEM is released
+        int ts = 0, tp = 0;
         if (lane == 0) {
+            bool s_done = false;  // the S stream has met the end item
+            uint64_t t_last = globaltimer();
+            while (true) {
+                bool prog = false;
+                if (!s_done) {
+                    const int ii = ts % kInfo;
+                    if (mbar_test(&B.info_full[ii], (ts / kInfo) & 1)) {
+                        const TileInfo &inf = info[ii];
+                        const int sb = ts & 1;
+                        if (inf.type == kItemEnd) {
+                            s_done = true;
+                            prog = true;
+                        } else if ((!inf.unit_first || mbar_test(&B.kv_full[inf.kvs], inf.kvph)) &&
+                                   mbar_test(&B.q_full[inf.qs], inf.qph) &&
+                                   (ts < 2 || mbar_test(&B.s_empty[sb], ((ts >> 1) - 1) & 1))) {
+                            tc_fence_after();
+                            const uint32_t qa = smem_u32(sm + L::OFF_Q + inf.qs * L::QBYTES);
+                            const uint32_t kb = smem_u32(sm + L::OFF_K + inf.kvs * L::KVBYTES);
+                            const uint32_t dcol = tmem + sb * 64;
+#pragma unroll
+                            for (int ks = 0; ks < D / 16; ++ks) {
+                                const int h = ks >> 2, kk = ks & 3;
+                                mma_bf16_ss(dcol, smem_desc_sw128(qa + h * L::QHALF + kk * 32, 16, 1024),
+                                            smem_desc_sw128(kb + h * L::KVHALF + kk * 32, 16, 1024), idesc1, ks > 0);
+                            }
+                            mma_commit(&B.s_full[sb]);
+                            mma_commit(&B.q_empty[inf.qs]);
+                            ++ts;
+                            prog = true;
+                        }
+                    }
+                }
+                if (tp < ts) {
+                    const int ii = tp % kInfo;
+                    const TileInfo &inf = info[ii];
+                    const int pb = tp & 1;
+                    if (mbar_test(&B.p_full[pb], (tp >> 1) & 1) &&
+                        (tp < 2 || mbar_test(&B.o_empty[pb], ((tp >> 1) - 1) & 1))) {
+                        tc_fence_after();
+                        const uint32_t pa = smem_u32(sm + L::OFF_P + pb * L::PBYTES);
+                        const uint32_t vb = smem_u32(sm + L::OFF_V + inf.kvs * L::KVBYTES);
+                        const uint32_t dcol = tmem + 128 + pb * 128;
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks)
+                            mma_bf16_ss(dcol, smem_desc_sw128(pa + ks * 32, 16, 1024),
+                                        smem_desc_sw128(vb + ks * 2048, L::KVHALF, 1024), idesc2, ks > 0);
+                        mma_commit(&B.o_full[pb]);
+                        mma_commit(&p_empty[pb]);
+                        if (inf.unit_last) mma_commit(&B.kv_empty[inf.kvs]);
+                        mbar_arrive(&B.info_empty[ii]);
+                        ++tp;
+                        prog = true;
+                    }
+                } else if (s_done) {
+                    break;
+                }
+                if (prog) {
+                    t_last = globaltimer();
+                } else {
+                    if (*abort_flag || globaltimer() - t_last > kWaitNs) { ok = false; break; }
+                    PROF_INC(1);
+                }
+            }
+            if (!ok) {
+                *abort_flag = 1;
+                report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 3, ts);
+            }
+            // drain: every MMA issued by this warp has finished before TMEM is released
             mma_commit(mma_done);
             mbar_wait(mma_done, 0, kWaitNs);
         }
         __syncwarp();
 #ifdef HSA_TC_PROFILE
         prof_acc[0] = clock64() - prof_start;
-        if (lane == 0) PROF_DUMP(blockIdx.x * 80 + 16);
+        if (lane == 0) PROF_DUMP(blockIdx.x * 96 + 16);
+#else
+        (void)prof_start;
 #endif
     } else if (warp < kWarpEpi) {
         // ============================================================ softmax
@@ -511,6 +523,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&B.s_empty[sb]);
+            // P buffer sb is free once the O = P.V of tile tseq - 2 has read it
+            if (tseq >= 2 && !wg_wait(&p_empty[sb], ((tseq >> 1) - 1) & 1)) { ok = false; break; }
             const int ti = r / G, hh = r % G;
             const bool valid = ti < inf.ntok;
             uint8_t *prow = sm + L::OFF_P + sb * L::PBYTES + r * 128;
@@ -573,7 +587,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         if (!ok) { *abort_flag = 1; if (tid == 0) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 5, it); }
 #ifdef HSA_TC_PROFILE
         prof_acc[0] = clock64() - prof_start;
-        if (tid == 0) PROF_DUMP(blockIdx.x * 80 + 32);
+        if (tid == 0) PROF_DUMP(blockIdx.x * 96 + 32);
 #endif
     } else if (warp < kWarpConv) {
         // ============================================================ epilogue
@@ -583,22 +597,24 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         // accumulator slot in L2.  The tiles reduced per window are published in
         // tiles_done[window] (after a fence) when the window changes, when the
         // next tile is not there yet, and at the end.
+        const int eg = (warp - kWarpEpi) >> 2;                    // epilogue group = its O buffer
         const int wq = warp & 3;
-        const int r = wq * 32 + lane;                 // tile row of this lane's TMEM loads
-        const int tid = threadIdx.x - kWarpEpi * 32;  // 0..127
+        const int r = wq * 32 + lane;                             // tile row of this lane's TMEM loads
+        const int tid = threadIdx.x - (kWarpEpi + 4 * eg) * 32;   // 0..127
         const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
-        float4 *xs = reinterpret_cast<float4 *>(sm + L::OFF_X + wq * 4096);  // [32 rows][8 chunks]
+        float4 *xs = reinterpret_cast<float4 *>(sm + L::OFF_X + (warp - kWarpEpi) * 4096);  // [32 rows][8 chunks]
+        volatile int *gflag = eg_flag + 2 * eg;
         int it = 0, tseq = 0, ecnt = 0, ecnt_j = -1, vcnt = 0;
         bool ok = true;
         PROF_DECL
         const long long prof_start = clock64();
         (void)prof_start;
-        auto eg_sync = [&]() { asm volatile("bar.sync 3, 128;" ::: "memory"); };
+        auto eg_sync = [&]() { asm volatile("bar.sync %0, 128;" ::"r"(3 + eg) : "memory"); };
         auto eg_vote = [&](int v) -> bool {
             const int slot = (vcnt++) & 1;
-            if (tid == 0) eg_flag[slot] = v;
+            if (tid == 0) gflag[slot] = v;
             eg_sync();
-            return eg_flag[slot] != 0;
+            return gflag[slot] != 0;
         };
         auto eg_wait = [&](uint64_t *b, uint32_t par) -> bool {
             int v = 1;
@@ -627,6 +643,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             PROF_END(1);
             const TileInfo &inf = info[ii];
             if (inf.type == kItemEnd) break;
+            if ((tseq & 1) != eg) {  // the other group's tile: acknowledge the slot and move on
+                eg_sync();
+                if (tid == 0) mbar_arrive(&B.info_empty[ii]);
+                ++tseq;
+                ++it;
+                continue;
+            }
             if (inf.j != ecnt_j) {
                 if (ecnt > 0) flush();
                 ecnt_j = inf.j;
@@ -683,7 +706,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         if (!ok) { *abort_flag = 1; if (tid == 0) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 6, it); }
 #ifdef HSA_TC_PROFILE
         prof_acc[0] = clock64() - prof_start;
-        if (tid == 0) PROF_DUMP(blockIdx.x * 80 + 64);
+        if (tid == 0) PROF_DUMP(blockIdx.x * 96 + 64 + 16 * eg);
 #endif
     } else if (warp < kWarpProd) {
         // ============================================================ convert group
@@ -692,13 +715,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         // jc are reduced, then claims jc's convert items (kCombTokens tokens
         // each) from comb_head[jc] until none are left, so a finished window is
         // converted by all CTAs at once while the tile pipeline moves on.
-        const int tid = threadIdx.x - kWarpConv * 32;  // 0..127
+        const int tid = threadIdx.x - kWarpConv * 32;  // 0..kConvThreads-1
         int ci_n = 0, vcnt = 0;
         bool ok = true;
         PROF_DECL
         const long long prof_start = clock64();
         (void)prof_start;
-        auto cg_sync = [&]() { asm volatile("bar.sync 2, 128;" ::: "memory"); };
+        auto cg_sync = [&]() { asm volatile("bar.sync 2, %0;" ::"n"(kConvThreads) : "memory"); };
         auto cg_bcast = [&](int v) -> int {  // thread 0's value to the whole group
             const int slot = (vcnt++) & 1;
             if (tid == 0) cg_flag[slot] = v;
@@ -730,11 +753,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 constexpr int kBatch = 8;       // units in flight per thread
                 float4 *A = reinterpret_cast<float4 *>(acc + (int64_t)(s * P.W + (ta - ws)) * G * D);
                 const int nunits = (tb - ta) * UPT;
-                for (int u0 = 0; u0 < nunits; u0 += 128 * kBatch) {
+                for (int u0 = 0; u0 < nunits; u0 += kConvThreads * kBatch) {
                     float4 lo[kBatch], hi[kBatch];
 #pragma unroll
                     for (int k = 0; k < kBatch; ++k) {
-                        const int u = u0 + k * 128 + tid;
+                        const int u = u0 + k * kConvThreads + tid;
                         if (u < nunits) {
                             lo[k] = __ldcg(A + 2 * u);
                             hi[k] = __ldcg(A + 2 * u + 1);
@@ -742,7 +765,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                     }
 #pragma unroll
                     for (int k = 0; k < kBatch; ++k) {
-                        const int u = u0 + k * 128 + tid;
+                        const int u = u0 + k * kConvThreads + tid;
                         if (u < nunits) {
                             const int t = ta + u / UPT, e = u % UPT;
                             __nv_bfloat162 a0 = __floats2bfloat162_rn(lo[k].x, lo[k].y);
@@ -773,7 +796,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         if (!ok) { *abort_flag = 1; if (tid == 0) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 7, ci_n); }
 #ifdef HSA_TC_PROFILE
         prof_acc[0] = clock64() - prof_start;
-        if (tid == 0) PROF_DUMP(blockIdx.x * 80 + 48);
+        if (tid == 0) PROF_DUMP(blockIdx.x * 96 + 48);
 #endif
     }
 
@@ -831,7 +854,7 @@ cudaError_t launch_tc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv,
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     attend_tc_kernel<D, G><<<sms, kThreads, smem, st>>>(mq, mk, mv, plan, inv.hist, inv.chunk_off, inv.entries,
-                                                        idx, w, acc, (__nv_bfloat16 *)o, lse, ds);
+                                                        idx, inv.entw, acc, (__nv_bfloat16 *)o, lse, ds);
     return cudaGetLastError();
 }
 

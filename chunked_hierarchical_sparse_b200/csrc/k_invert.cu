@@ -147,21 +147,28 @@ __global__ void __launch_bounds__(256) inv_base_kernel(int32_t *__restrict__ his
 
 // One warp per (token block, b*hkv + g): tokens in order, slots in parallel.
 __global__ void __launch_bounds__(32) inv_scatter_kernel(const int32_t *__restrict__ idx,
+                                                         const float *__restrict__ w,
                                                          const int32_t *__restrict__ hist,
-                                                         int32_t *__restrict__ entries, int L,
+                                                         int32_t *__restrict__ entries,
+                                                         float *__restrict__ entw, int L,
                                                          int hkv, int nc, int K, int ntb) {
-    extern __shared__ int cur[];  // [nc] cursors, then [kInvTokBlock * K] the block's selections
+    extern __shared__ int cur[];  // [nc] cursors, [kInvTokBlock * K] the block's selections and weights
     int *sel = cur + nc;
+    float *selw = reinterpret_cast<float *>(sel + kInvTokBlock * K);
     const int tb = blockIdx.x, bg = blockIdx.y, b = bg / hkv, g = bg % hkv;
     const int lane = threadIdx.x;
     const int32_t *H = hist + ((int64_t)bg * ntb + tb) * nc;
     for (int c = lane; c < nc; c += 32) cur[c] = H[c];
     const int t0 = tb * kInvTokBlock;
     const int t1 = min(t0 + kInvTokBlock, L);
-    for (int e = lane; e < (t1 - t0) * K; e += 32)
-        sel[e] = idx[(((int64_t)b * L + t0 + e / K) * hkv + g) * K + e % K];
+    for (int e = lane; e < (t1 - t0) * K; e += 32) {
+        const int64_t o = (((int64_t)b * L + t0 + e / K) * hkv + g) * K + e % K;
+        sel[e] = idx[o];
+        if (w) selw[e] = w[o];
+    }
     __syncwarp();
     int32_t *E = entries + (int64_t)bg * L * K;
+    float *EW = entw ? entw + (int64_t)bg * L * K : nullptr;
     for (int t = t0; t < t1; ++t) {
         if (lane < K) {
             const int c = sel[(t - t0) * K + lane];
@@ -169,19 +176,20 @@ __global__ void __launch_bounds__(32) inv_scatter_kernel(const int32_t *__restri
                 const int pos = cur[c];
                 cur[c] = pos + 1;
                 E[pos] = t * 16 + lane;
+                if (EW) EW[pos] = selw[(t - t0) * K + lane];
             }
         }
         __syncwarp();
     }
 }
 
-cudaError_t launch_invert(const Shape &sh, const int32_t *idx, const BwdWs &ws, DevStatus *ds,
+cudaError_t launch_invert(const Shape &sh, const int32_t *idx, const float *w, const BwdWs &ws, DevStatus *ds,
                           cudaStream_t st) {
     if (sh.B == 0 || sh.L == 0 || sh.nc == 0) return cudaSuccess;
     const int ntb = (int)ceil_div(sh.L, kInvTokBlock);
     const size_t smem = sizeof(int) * (size_t)sh.nc;
     cudaError_t e;
-    const size_t ssmem = smem + sizeof(int) * (size_t)kInvTokBlock * sh.K;
+    const size_t ssmem = smem + 2 * sizeof(int) * (size_t)kInvTokBlock * sh.K;
     if (2 * smem > 48 * 1024 || ssmem > 48 * 1024) {
         e = set_smem_once((const void *)inv_hist_kernel, (size_t)(smem));
         if (e != cudaSuccess) return e;
@@ -200,7 +208,8 @@ cudaError_t launch_invert(const Shape &sh, const int32_t *idx, const BwdWs &ws, 
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     inv_base_kernel<<<dim3(148, sh.B * sh.hkv), 256, 0, st>>>(ws.hist, ws.chunk_off, sh.nc, ntb);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    inv_scatter_kernel<<<grid, 32, ssmem, st>>>(idx, ws.hist, ws.entries, sh.L, sh.hkv, sh.nc, sh.K, ntb);
+    inv_scatter_kernel<<<grid, 32, ssmem, st>>>(idx, w, ws.hist, ws.entries, w ? ws.entw : nullptr, sh.L,
+                                                 sh.hkv, sh.nc, sh.K, ntb);
     return cudaGetLastError();
 }
 

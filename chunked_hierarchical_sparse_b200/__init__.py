@@ -30,7 +30,8 @@ OP_POOL, OP_SELECT, OP_FWD, OP_DECODE, OP_BWD = range(5)
 _F32, _BF16 = 0, 1
 # kernel kinds of hsa_timing_read (hsa_kernel_t)
 KERNELS = {"pool": 1, "select": 2, "attend_simt": 3, "decode": 4, "bwd1": 5, "invert": 6, "bwd2": 7,
-           "attend_tc": 8, "plan": 9}
+           "attend_tc": 8, "plan": 9,
+           "bwd_tc": 10, "bwd_sel": 11}
 _STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported shape", 3: "workspace too small",
            4: "CUDA launch or API error", 5: "device wait timed out",
            6: "device-side input check failed"}

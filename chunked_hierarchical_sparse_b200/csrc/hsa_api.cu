@@ -57,6 +57,36 @@ struct FwdWs {
     float *acc;          // fp32 output-accumulator ring (chunk-major path)
 };
 
+// token->chunk lists of the chunk-major passes (with the entries' weights if `weights`)
+static void carve_lists(Carver &c, const Shape &sh, BwdWs &inv, bool weights) {
+    const int ntb = (int)ceil_div(sh.L, kInvTokBlock);
+    inv.hist = c.take<int32_t>((size_t)sh.B * sh.hkv * ntb * sh.nc);
+    inv.chunk_off = c.take<int32_t>((size_t)sh.B * sh.hkv * (sh.nc + 1));
+    inv.seg_off = c.take<int32_t>((size_t)sh.B * sh.hkv * (sh.nc + 1));
+    inv.entries = c.take<int32_t>((size_t)sh.B * sh.hkv * sh.L * sh.K);
+    inv.entw = weights ? c.take<float>((size_t)sh.B * sh.hkv * sh.L * sh.K) : nullptr;
+}
+
+// work plan of the chunk-major passes: windows, units of up to `unit_tiles` tiles, queue
+static void carve_plan(Carver &c, const Shape &sh, AttendPlan &P, int unit_tiles) {
+    P.B = sh.B; P.L = sh.L; P.hq = sh.hq; P.hkv = sh.hkv; P.D = sh.d; P.K = sh.K; P.G = sh.G;
+    P.nc = sh.nc; P.ntb = (int)ceil_div(sh.L, kInvTokBlock);
+    P.W = (int)std::min<int64_t>(attend_window(sh.G, sh.d), round_up(std::max(sh.L, 1), kInvTokBlock));
+    P.nW = (int)ceil_div(sh.L, P.W); P.J = sh.B * sh.hkv * P.nW; P.TT = 128 / sh.G;
+    P.unit_tiles = unit_tiles;
+    P.unit_prefix = c.take<int32_t>((size_t)P.J * (sh.nc + 1));
+    P.win_units = c.take<int32_t>((size_t)P.J);
+    P.win_tiles = c.take<int32_t>((size_t)P.J);
+    P.win_ncomb = c.take<int32_t>((size_t)P.J);
+    P.seg_start = c.take<int32_t>((size_t)P.J + 1);
+    P.counters = c.take<int32_t>(plan_counter_count(P.J));
+    // work units <= tiles <= L*K/TT + nc per window, summed over (b, g)
+    P.max_items = (int)std::min<int64_t>(
+        ((int64_t)sh.B * sh.hkv * ((int64_t)sh.L * sh.K / P.TT + (int64_t)P.nW * sh.nc) + 16),
+        (int64_t)INT32_MAX / 4);
+    P.items = c.take<int4>((size_t)2 * P.max_items);
+}
+
 static FwdWs carve_fwd(const Shape &sh, void *ws, size_t *bytes) {
     Carver c{static_cast<char *>(ws)};
     FwdWs f{};
@@ -69,48 +99,41 @@ static FwdWs carve_fwd(const Shape &sh, void *ws, size_t *bytes) {
     }
     f.tc = attend_tc_supported(sh);
     if (f.tc) {
-        const int ntb = (int)ceil_div(sh.L, kInvTokBlock);
-        f.inv.hist = c.take<int32_t>((size_t)sh.B * sh.hkv * ntb * sh.nc);
-        f.inv.chunk_off = c.take<int32_t>((size_t)sh.B * sh.hkv * (sh.nc + 1));
-        f.inv.seg_off = c.take<int32_t>((size_t)sh.B * sh.hkv * (sh.nc + 1));
-        f.inv.entries = c.take<int32_t>((size_t)sh.B * sh.hkv * sh.L * sh.K);
-        f.inv.entw = c.take<float>((size_t)sh.B * sh.hkv * sh.L * sh.K);
-        AttendPlan &P = f.plan;
-        P.B = sh.B; P.L = sh.L; P.hq = sh.hq; P.hkv = sh.hkv; P.D = sh.d; P.K = sh.K; P.G = sh.G;
-        P.nc = sh.nc; P.ntb = ntb; P.W = (int)std::min<int64_t>(attend_window(sh.G, sh.d), round_up(std::max(sh.L, 1), kInvTokBlock));
-        P.nW = (int)ceil_div(sh.L, P.W); P.J = sh.B * sh.hkv * P.nW; P.TT = 128 / sh.G;
-        P.unit_prefix = c.take<int32_t>((size_t)P.J * (sh.nc + 1));
-        P.win_units = c.take<int32_t>((size_t)P.J);
-        P.win_tiles = c.take<int32_t>((size_t)P.J);
-        P.win_ncomb = c.take<int32_t>((size_t)P.J);
-        P.seg_start = c.take<int32_t>((size_t)P.J + 1);
-        P.counters = c.take<int32_t>(plan_counter_count(P.J));
-        // queue items (work units): units <= tiles <= L*K/TT + nc per window, summed over (b, g)
-        P.max_items = (int)std::min<int64_t>(
-            ((int64_t)sh.B * sh.hkv * ((int64_t)sh.L * sh.K / P.TT + (int64_t)P.nW * sh.nc) + 16),
-            (int64_t)INT32_MAX / 4);
-        P.items = c.take<int4>((size_t)2 * P.max_items);
-        f.acc = c.take<float>(attend_acc_floats(P.W, sh.G, sh.d));
+        carve_lists(c, sh, f.inv, true);
+        carve_plan(c, sh, f.plan, kUnitTiles);
+        f.acc = c.take<float>(attend_acc_floats(f.plan.W, sh.G, sh.d));
     }
     if (bytes) *bytes = c.off;
     return f;
 }
 
-static BwdWs carve_bwd(const Shape &sh, void *ws, size_t *bytes) {
-    Carver c{static_cast<char *>(ws)};
+struct BwdAll {
     BwdWs b;
-    const int ntb = (int)ceil_div(sh.L, kInvTokBlock);
+    bool tc;          // chunk-major tensor-core path
+    AttendPlan plan;
+    float *acc;       // fp32 dq accumulator ring (tensor-core path)
+    float *dw;        // [B,L,h_kv,K] gradients of the chunk weights (tensor-core path)
+};
+
+constexpr int kBwdUnitTiles = 16;  // backward work units: up to 16 tiles (one dK/dV flush each)
+
+static BwdAll carve_bwd(const Shape &sh, void *ws, size_t *bytes) {
+    Carver c{static_cast<char *>(ws)};
+    BwdAll r{};
+    BwdWs &b = r.b;
+    r.tc = bwd_tc_supported(sh) && sh.nc > 0;
     b.dkbar = c.take<float>((size_t)sh.B * sh.hkv * sh.nc * sh.d);
-    b.delta = c.take<float>((size_t)sh.B * sh.L * sh.hq * sh.K);
+    b.delta = r.tc ? nullptr : c.take<float>((size_t)sh.B * sh.L * sh.hq * sh.K);
     b.dk_acc = c.take<float>((size_t)sh.B * sh.hkv * sh.L * sh.d);
     b.dv_acc = c.take<float>((size_t)sh.B * sh.hkv * sh.L * sh.d);
-    b.hist = c.take<int32_t>((size_t)sh.B * sh.hkv * ntb * sh.nc);
-    b.chunk_off = c.take<int32_t>((size_t)sh.B * sh.hkv * (sh.nc + 1));
-    b.seg_off = c.take<int32_t>((size_t)sh.B * sh.hkv * (sh.nc + 1));
-    b.entries = c.take<int32_t>((size_t)sh.B * sh.hkv * sh.L * sh.K);
-    b.entw = nullptr;
+    carve_lists(c, sh, b, r.tc);
+    if (r.tc) {
+        r.dw = c.take<float>((size_t)sh.B * sh.L * sh.hkv * sh.K);
+        carve_plan(c, sh, r.plan, kBwdUnitTiles);
+        r.acc = c.take<float>(attend_acc_floats(r.plan.W, sh.G, sh.d));
+    }
     if (bytes) *bytes = c.off;
-    return b;
+    return r;
 }
 
 static size_t ws_size(const Shape &sh, int op) {
@@ -299,13 +322,37 @@ hsa_status_t hsa_bwd(const hsa_shape_t *shape, const void *q, const void *k, con
     if ((s = check_ws(sh, HSA_OP_BWD, ws, ws_bytes)) != HSA_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     DevStatus *ds = static_cast<DevStatus *>(ws);
-    BwdWs b = carve_bwd(sh, ws, nullptr);
+    BwdAll all = carve_bwd(sh, ws, nullptr);
+    BwdWs &b = all.b;
     cudaError_t e = clear_status(ws, st);
     const size_t acc_bytes = sizeof(float) * (size_t)sh.B * sh.hkv * sh.L * sh.d;
     if (e == cudaSuccess && sh.nc > 0)
         e = cudaMemsetAsync(b.dkbar, 0, sizeof(float) * (size_t)sh.B * sh.hkv * sh.nc * sh.d, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(b.dk_acc, 0, acc_bytes, st);
     if (e == cudaSuccess) e = cudaMemsetAsync(b.dv_acc, 0, acc_bytes, st);
+    if (all.tc) {
+        // one chunk-major pass on the tensor cores (dq, dw, dk, dv), then the
+        // stick-breaking backward and the finishing pass on CUDA cores
+        const AttendPlan &P = all.plan;
+        if (e == cudaSuccess) e = timed(HSA_K_INVERT, 5, st, [&] { return launch_invert(sh, idx, w, b, ds, st); });
+        if (e == cudaSuccess) e = timed(HSA_K_PLAN, 3, st, [&] { return launch_plan(sh, b, P, st); });
+        if (e == cudaSuccess) e = cudaMemsetAsync(P.counters, 0, sizeof(int32_t) * plan_counter_count(P.J), st);
+        if (e == cudaSuccess)
+            e = cudaMemsetAsync(all.acc, 0,
+                                sizeof(float) * std::min<size_t>(attend_acc_floats(P.W, sh.G, sh.d),
+                                                                 (size_t)P.J * P.W * sh.G * sh.d),
+                                st);
+        if (e == cudaSuccess)
+            e = timed(HSA_K_BWD_TC, 1, st, [&] {
+                return launch_bwd_tc(sh, P, b, q, k, v, dO, lse, all.dw, all.acc, dq, b.dk_acc, b.dv_acc, ds, st);
+            });
+        if (e == cudaSuccess)
+            e = timed(HSA_K_BWD_SEL, 2, st, [&] {
+                cudaError_t e2 = launch_bwd_select(sh, q_slc, idx, w, all.dw, kbar, dq_slc, b.dkbar, st);
+                return e2 == cudaSuccess ? launch_bwd_finish(sh, b, dk, dv, st) : e2;
+            });
+        return cuda_status(e);
+    }
     if (e == cudaSuccess)
         e = timed(HSA_K_BWD1, 1, st, [&] {
             return launch_bwd_phase1(sh, q, q_slc, k, v, dO, lse, idx, w, kbar, dq, dq_slc, b, ds, st);

@@ -25,7 +25,7 @@ struct DevStatus {
 
 enum KernelId : int32_t {
     kKPool = 1, kKSelect = 2, kKAttendSimt = 3, kKDecode = 4, kKBwd1 = 5, kKInvert = 6,
-    kKBwd2 = 7, kKAttendTc = 8, kKFinal = 9, kKSelectTc = 10
+    kKBwd2 = 7, kKAttendTc = 8, kKFinal = 9, kKSelectTc = 10, kKBwdTc = 11
 };
 
 __device__ __forceinline__ void report(DevStatus *st, int32_t code, int32_t where, int32_t a,
@@ -141,7 +141,7 @@ constexpr int kInvTokBlock = 256;  // tokens per histogram block of the inversio
 constexpr int kBwdSeg = 32;        // list entries per phase-2 block
 
 // ---------------------------------------------------------------- chunk-major forward plan
-constexpr int kUnitTiles = 4;      // tiles of one chunk per work unit (one K/V load)
+constexpr int kUnitTiles = 4;      // forward: tiles of one chunk per work unit (one K/V load)
 constexpr int kCombTokens = 16;    // tokens per combine item
 // Output accumulators of the chunk-major forward: a ring of kRing window
 // slots, each an fp32 [W tokens][G heads][d] block that the tiles of one
@@ -158,6 +158,7 @@ constexpr size_t kAccSlotBudget = size_t(HSA_ACC_SLOT_MB) << 20;
 
 struct AttendPlan {
     int B, L, hq, hkv, D, K, G, nc, ntb, W, nW, J, TT;
+    int unit_tiles;        // tiles per work unit (at most; one K/V load per unit)
     int32_t *unit_prefix;  // [J][nc+1] work units per (window, chunk), exclusive prefix
     int32_t *win_units;    // [J]
     int32_t *win_tiles;    // [J]
@@ -198,5 +199,18 @@ bool attend_tc_supported(const Shape &sh);
 cudaError_t launch_attend_tc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv, const void *q,
                              const void *k, const void *v, const int32_t *idx, const float *w,
                              float *acc, void *o, float *lse, DevStatus *ds, cudaStream_t st);
+
+// Chunk-major backward on the tensor cores (d = 128, G in {8, 16}): dq (via the
+// plan's window ring `acc`), dw [B,L,hkv,K], and dK / dV added into the fp32
+// accumulators of `inv` (dk_acc / dv_acc).  inv.entw must hold the entries' weights.
+bool bwd_tc_supported(const Shape &sh);
+cudaError_t launch_bwd_tc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv, const void *q, const void *k,
+                          const void *v, const void *dO, const float *lse, float *dw, float *acc, void *dq,
+                          float *dk_acc, float *dv_acc, DevStatus *ds, cudaStream_t st);
+// Stick-breaking backward from dw: dq_slc, and dkbar (added into, fp32).
+cudaError_t launch_bwd_select(const Shape &sh, const void *q_slc, const int32_t *idx, const float *w,
+                              const float *dw, const float *kbar, void *dq_slc, float *dkbar, cudaStream_t st);
+// dk = dk_acc + dkbar_c / S, dv = dv_acc, in the input dtype.
+cudaError_t launch_bwd_finish(const Shape &sh, const BwdWs &ws, void *dk, void *dv, cudaStream_t st);
 
 }  // namespace hsa

@@ -353,6 +353,20 @@ static cudaError_t phase2_dispatch(const Shape &sh, const void *q, const void *k
     return cudaGetLastError();
 }
 
+template <typename T>
+static cudaError_t finish_dispatch(const Shape &sh, const BwdWs &ws, void *dk, void *dv, cudaStream_t st) {
+    const int64_t total = (int64_t)sh.B * sh.hkv * sh.L * sh.d;
+    if (total == 0) return cudaSuccess;
+    const int blocks = (int)std::min<int64_t>(ceil_div(total, 256), 148 * 16);
+    bwd_finish_kernel<T><<<blocks, 256, 0, st>>>(ws.dk_acc, ws.dv_acc, ws.dkbar, (T *)dk, (T *)dv, sh.L, sh.d,
+                                                  sh.nc, total);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_finish(const Shape &sh, const BwdWs &ws, void *dk, void *dv, cudaStream_t st) {
+    return sh.bf16 ? finish_dispatch<__nv_bfloat16>(sh, ws, dk, dv, st) : finish_dispatch<float>(sh, ws, dk, dv, st);
+}
+
 cudaError_t launch_bwd_phase2(const Shape &sh, const void *q, const void *k, const void *v,
                               const void *dO, const float *lse, const float *w, void *dk, void *dv,
                               const BwdWs &ws, DevStatus *, cudaStream_t st) {

@@ -6,7 +6,7 @@
 // window sequence j = (b*h_kv + g)*nW + w is processed in order.  Inside a
 // window, the entries of chunk c form a bucket; a bucket is cut into tiles of
 // TT = 128/G tokens (the tile's rows are its tokens' G query heads) and tiles
-// into work units of up to kUnitTiles tiles (one K/V load per unit).
+// into work units of up to plan.unit_tiles tiles (one K/V load per unit).
 //
 // The persistent attention kernel pulls work units window by window (the
 // units of window s form queue segment s).  Combine items are not queued:
@@ -39,7 +39,7 @@ __global__ void __launch_bounds__(1024) plan_windows_kernel(const int32_t *__res
         const int e1 = (tb1 < ntb) ? H[(int64_t)tb1 * nc + c] : off[c + 1];
         const int nt = (e1 - e0 + plan.TT - 1) / plan.TT;
         my_tiles += nt;
-        s_units[c] = (nt + kUnitTiles - 1) / kUnitTiles;
+        s_units[c] = (nt + plan.unit_tiles - 1) / plan.unit_tiles;
     }
     atomicAdd(&s_tiles, my_tiles);
     __syncthreads();
@@ -115,11 +115,11 @@ __global__ void __launch_bounds__(256) plan_fill_kernel(const int32_t *__restric
             const int e1 = (tb1 < ntb) ? H[(int64_t)tb1 * nc + c] : off[c + 1];
             const int nt = (e1 - e0 + plan.TT - 1) / plan.TT;
             for (int u = u0; u < u1; ++u) {
-                const int t0 = (u - u0) * kUnitTiles;
+                const int t0 = (u - u0) * plan.unit_tiles;
                 const int q = base + u;
                 if (q >= plan.max_items) continue;
                 plan.items[2 * q] = make_int4(0, j, c, e0);
-                plan.items[2 * q + 1] = make_int4(e1, t0, min(nt, t0 + kUnitTiles), 0);
+                plan.items[2 * q + 1] = make_int4(e1, t0, min(nt, t0 + plan.unit_tiles), 0);
             }
         }
     }

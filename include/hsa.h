@@ -182,10 +182,12 @@ typedef enum {
     HSA_K_ATTEND_SIMT = 3, /* token-major attention (CUDA cores)             */
     HSA_K_DECODE = 4,      /* decode step                                    */
     HSA_K_BWD1 = 5,        /* backward phase 1 (per token)                   */
-    HSA_K_INVERT = 6,      /* token->chunk list inversion (3 launches)       */
+    HSA_K_INVERT = 6,      /* token->chunk list inversion (5 launches)       */
     HSA_K_BWD2 = 7,        /* backward phase 2 (per chunk) + finishing pass  */
     HSA_K_ATTEND_TC = 8,   /* chunk-major attention (tcgen05)                */
     HSA_K_PLAN = 9,        /* chunk-major work planning                      */
+    HSA_K_BWD_TC = 10,     /* chunk-major backward (tcgen05): dq, dw, dk, dv */
+    HSA_K_BWD_SEL = 11,    /* stick-breaking backward + finishing pass       */
     HSA_K_COUNT = 16
 } hsa_kernel_t;
 

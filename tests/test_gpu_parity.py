@@ -220,6 +220,27 @@ def test_bwd_small_full(wl):
             assert_out(f64(g), r, "bf16", name, grad=True)
 
 
+# chunk-major tensor-core backward: bf16, d = 128, G in {8, 16}
+BWD_TC = [small(h_q=16, h_kv=1, K=4, L=64 * 45 + 3, B=1, kind="train"),
+          small(h_q=16, h_kv=2, K=8, L=64 * 100 + 17, B=2, seed=9, kind="train"),
+          small(h_q=16, h_kv=2, K=16, L=2048, kind="train"),
+          small(h_q=16, h_kv=2, K=1, L=777, B=3, kind="train")]
+
+
+@pytest.mark.parametrize("wl", BWD_TC, ids=["g16-ragged", "g8-multiwindow", "g8-k16", "g8-k1-b3"])
+def test_bwd_tensor_core_path_full(wl):
+    x, kbar, sel = gap_ruled(wl)
+    ref = oracle.bwd(x["q"], x["k"], x["v"], x["q_slc"], kbar, x["dO"], wl.S, wl.K)
+    m = hsa()
+    m.hsa_timing_enable(True)
+    got = run_bwd(wl, x)
+    ms, n = m.hsa_timing_read("bwd_tc")
+    m.hsa_timing_enable(False)
+    assert n == 1, "the tensor-core backward did not run"
+    for name, g, r in zip(("dq", "dk", "dv", "dq_slc"), got, ref[:4]):
+        assert_out(f64(g), r, "bf16", name, grad=True)
+
+
 def test_bwd_train_workload_sampled():
     """Full-size training workload: dq / dq_slc on sampled tokens, dk / dv on
     sampled chunks (the oracle walks every token that selected them)."""

@@ -295,8 +295,8 @@ def bench_train(hsa, dev, steps=3):
         b.record()
         torch.cuda.synchronize()
         times.append(a.elapsed_time(b))
-    per_kernel = {k: round(hsa.hsa_timing_read(k)[0] / steps, 4) for k in
-                  ("pool", "select", "attend_simt", "attend_tc", "plan", "bwd1", "invert", "bwd2")}
+    per_kernel = {k: round(hsa.hsa_timing_read(k)[0] / steps, 4) for k in hsa.KERNELS
+                  if hsa.hsa_timing_read(k)[1] > 0}
     hsa.hsa_timing_enable(False)
     att, sel, _ = fwd_work(wl)
     G = wl.h_q // wl.h_kv

@@ -54,7 +54,7 @@ struct FwdWs {
     bool tc;             // chunk-major tensor-core path
     BwdWs inv;           // token->chunk lists (hist, chunk_off, seg_off, entries)
     AttendPlan plan;
-    float *acc;          // fp32 output-accumulator ring (chunk-major path)
+    __half *acc;         // fp16 output-accumulator ring, scaled (chunk-major path)
 };
 
 // token->chunk lists of the chunk-major passes (with the entries' weights if `weights`)
@@ -68,10 +68,10 @@ static void carve_lists(Carver &c, const Shape &sh, BwdWs &inv, bool weights) {
 }
 
 // work plan of the chunk-major passes: windows, units of up to `unit_tiles` tiles, queue
-static void carve_plan(Carver &c, const Shape &sh, AttendPlan &P, int unit_tiles) {
+static void carve_plan(Carver &c, const Shape &sh, AttendPlan &P, int unit_tiles, int acc_bytes) {
     P.B = sh.B; P.L = sh.L; P.hq = sh.hq; P.hkv = sh.hkv; P.D = sh.d; P.K = sh.K; P.G = sh.G;
     P.nc = sh.nc; P.ntb = (int)ceil_div(sh.L, kInvTokBlock);
-    P.W = (int)std::min<int64_t>(attend_window(sh.G, sh.d), round_up(std::max(sh.L, 1), kInvTokBlock));
+    P.W = (int)std::min<int64_t>(attend_window(sh.G, sh.d, acc_bytes), round_up(std::max(sh.L, 1), kInvTokBlock));
     P.nW = (int)ceil_div(sh.L, P.W); P.J = sh.B * sh.hkv * P.nW; P.TT = 128 / sh.G;
     P.unit_tiles = unit_tiles;
     P.unit_prefix = c.take<int32_t>((size_t)P.J * (sh.nc + 1));
@@ -100,8 +100,8 @@ static FwdWs carve_fwd(const Shape &sh, void *ws, size_t *bytes) {
     f.tc = attend_tc_supported(sh);
     if (f.tc) {
         carve_lists(c, sh, f.inv, true);
-        carve_plan(c, sh, f.plan, kUnitTiles);
-        f.acc = c.take<float>(attend_acc_floats(f.plan.W, sh.G, sh.d));
+        carve_plan(c, sh, f.plan, kUnitTiles, kFwdAccBytes);
+        f.acc = c.take<__half>(attend_acc_elems(f.plan.W, sh.G, sh.d));
     }
     if (bytes) *bytes = c.off;
     return f;
@@ -129,8 +129,8 @@ static BwdAll carve_bwd(const Shape &sh, void *ws, size_t *bytes) {
     carve_lists(c, sh, b, r.tc);
     if (r.tc) {
         r.dw = c.take<float>((size_t)sh.B * sh.L * sh.hkv * sh.K);
-        carve_plan(c, sh, r.plan, kBwdUnitTiles);
-        r.acc = c.take<float>(attend_acc_floats(r.plan.W, sh.G, sh.d));
+        carve_plan(c, sh, r.plan, kBwdUnitTiles, kBwdAccBytes);
+        r.acc = c.take<float>(attend_acc_elems(r.plan.W, sh.G, sh.d));
     }
     if (bytes) *bytes = c.off;
     return r;
@@ -274,11 +274,13 @@ hsa_status_t hsa_fwd(const hsa_shape_t *shape, const void *q, const void *k, con
         e = cudaMemsetAsync(f.plan.counters, 0, sizeof(int32_t) * plan_counter_count(f.plan.J), st);
     if (e == cudaSuccess)  // the used accumulator slots start at zero (the kernel re-zeroes them after use)
         e = cudaMemsetAsync(f.acc, 0,
-                            sizeof(float) * std::min<size_t>(attend_acc_floats(f.plan.W, sh.G, sh.d),
+                            sizeof(__half) * std::min<size_t>(attend_acc_elems(f.plan.W, sh.G, sh.d),
                                                              (size_t)f.plan.J * f.plan.W * sh.G * sh.d),
                             st);
     if (e == cudaSuccess && lse)
         e = cudaMemsetAsync(lse, 0, sizeof(float) * (size_t)sh.B * sh.L * sh.hq * sh.K, st);
+    if (e == cudaSuccess)  // the accumulators' power-of-two scale comes from max|v|
+        e = timed(HSA_K_PLAN, 1, st, [&] { return launch_vmax(sh, v, f.plan.counters + 3 * f.plan.J + 1, st); });
     if (e == cudaSuccess)
         e = timed(HSA_K_ATTEND_TC, 1, st, [&] {
             return launch_attend_tc(sh, f.plan, f.inv, q, k, v, f.idx, f.w, f.acc, o, lse, ds, st);
@@ -339,7 +341,7 @@ hsa_status_t hsa_bwd(const hsa_shape_t *shape, const void *q, const void *k, con
         if (e == cudaSuccess) e = cudaMemsetAsync(P.counters, 0, sizeof(int32_t) * plan_counter_count(P.J), st);
         if (e == cudaSuccess)
             e = cudaMemsetAsync(all.acc, 0,
-                                sizeof(float) * std::min<size_t>(attend_acc_floats(P.W, sh.G, sh.d),
+                                sizeof(float) * std::min<size_t>(attend_acc_elems(P.W, sh.G, sh.d),
                                                                  (size_t)P.J * P.W * sh.G * sh.d),
                                 st);
         if (e == cudaSuccess)

@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -169,25 +170,31 @@ struct AttendPlan {
     int max_items;         // capacity of `items`
 };
 
-inline size_t plan_counter_count(int J) { return 3 * (size_t)J + 1; }
+// tiles_done[J], comb_done[J], comb_head[J], then one word: the bits of max|v| (forward)
+inline size_t plan_counter_count(int J) { return 3 * (size_t)J + 2; }
 
 // queue item descriptor (two int4): {type, j, c, e0} {e1, t0, t1, 0}
 //   type 0: work unit, chunk c, entries [e0, e1) of its bucket, tiles [t0, t1)
 // Combine items are not queued: once every tile of window j is stored, the
 // combine warps of all CTAs claim window j's items from comb_head[j].
 
-// window length (tokens) of the chunk-major forward: a multiple of 256 such
-// that one window's fp32 accumulators (W * G * d * 4 bytes) fit in kAccSlotBudget
-inline int attend_window(int G, int d) {
-    const int64_t per_tok = (int64_t)G * d * 4;
+// window length (tokens) of the chunk-major passes: a multiple of 256 such that
+// one window's accumulators (W * G * d elements of `esize` bytes) fit in kAccSlotBudget
+inline int attend_window(int G, int d, int esize) {
+    const int64_t per_tok = (int64_t)G * d * esize;
     int64_t w = (int64_t)(kAccSlotBudget / per_tok) / kInvTokBlock * kInvTokBlock;
     if (w < kInvTokBlock) w = kInvTokBlock;
     if (w > 8192) w = 8192;
     return (int)w;
 }
 
-// bytes of the accumulator ring of one call
-inline size_t attend_acc_floats(int W, int G, int d) { return (size_t)kRing * W * G * d; }
+// elements of the accumulator ring of one call
+inline size_t attend_acc_elems(int W, int G, int d) { return (size_t)kRing * W * G * d; }
+
+// The forward's ring holds fp16 sums scaled by 2^-e, 2^e >= max|v| (every
+// partial sum of w_k * softmax-average of v is bounded by max|v|); the
+// backward's dq ring holds fp32.
+constexpr int kFwdAccBytes = 2, kBwdAccBytes = 4;
 
 bool select_tc_supported(const Shape &sh);
 // Chunk selection with tensor-core scores; hi/lo: [B,hkv,nc,d] bf16 scratch.
@@ -198,7 +205,9 @@ cudaError_t launch_plan(const Shape &sh, const BwdWs &inv, const AttendPlan &pla
 bool attend_tc_supported(const Shape &sh);
 cudaError_t launch_attend_tc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv, const void *q,
                              const void *k, const void *v, const int32_t *idx, const float *w,
-                             float *acc, void *o, float *lse, DevStatus *ds, cudaStream_t st);
+                             __half *acc, void *o, float *lse, DevStatus *ds, cudaStream_t st);
+// max|v| over the whole value tensor, as float bits, max-ed into *bits (zeroed by the caller)
+cudaError_t launch_vmax(const Shape &sh, const void *v, int32_t *bits, cudaStream_t st);
 
 // Chunk-major backward on the tensor cores (d = 128, G in {8, 16}): dq (via the
 // plan's window ring `acc`), dw [B,L,hkv,K], and dK / dV added into the fp32

@@ -14,8 +14,8 @@
 //   S[128 x 64]  = Q_tile[128 x d] . K_c^T          (tcgen05, fp32 in TMEM)
 //   p = exp(x - m) / (e^{-m} + sum exp(x - m)),  x = S / sqrt(d), m = max(0, max x)
 //   O[128 x d]   = P[128 x 64] . V_c                (tcgen05, fp32 in TMEM)
-//   acc[t, h] += (w_{t,g,slot} / Z) * O     (fp32 TMA reduce-add in L2 into the
-//                                             window's accumulator slot)
+//   acc[t, h] += (w_{t,g,slot} / Z) * O * 2^-e   (fp16 reduce-add in L2 into the
+//                                             window's accumulator slot; 2^e >= max|v|)
 // Once every tile of a window has been reduced, the convert step of the same
 // persistent kernel writes o[t, h] = bf16(acc[t, h]) and zeroes the slot for
 // the window that reuses it kRing windows later.  The slot sums each token's
@@ -27,6 +27,8 @@
 // warp 10 issues the reductions, warps 4-7 run the convert step.  Every wait
 // is bounded (a wall-clock limit); on expiry the kernel records
 // HSA_ERR_TIMEOUT, unwinds, frees its TMEM and returns.
+#include <algorithm>
+
 #include "hsa_internal.cuh"
 #include "sm100.cuh"
 
@@ -84,6 +86,8 @@ struct TileInfo {
 };
 
 template <int D> struct Smem {
+    // A query tile is 16 groups of 8 rows; a group holds its rows' 64-column halves
+    // one after the other (1 KB each), so one TMA box loads a whole group.
     static constexpr int QHALF = 128 * 128;  // bytes per 64-column half of a 128-row tile
     static constexpr int NH = D / 64;        // halves along d
     static constexpr int QBYTES = NH * QHALF;
@@ -154,7 +158,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     const __grid_constant__ CUtensorMap tm_v,
     const __grid_constant__ AttendPlan P, const int32_t *__restrict__ hist,
     const int32_t *__restrict__ chunk_off, const int32_t *__restrict__ entries,
-    const int32_t *__restrict__ idx, const float *__restrict__ entw, float *__restrict__ acc,
+    const int32_t *__restrict__ idx, const float *__restrict__ entw, __half *__restrict__ acc,
     __nv_bfloat16 *__restrict__ out, float *__restrict__ lse, DevStatus *ds) {
     using L = Smem<D>;
     constexpr int TT = 128 / G;
@@ -211,6 +215,17 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     int32_t *comb_done = P.counters + P.J;
     int32_t *comb_head = P.counters + 2 * P.J;
     const float scale = 1.0f / sqrtf((float)D);
+    // power-of-two scale of the fp16 accumulators: 2^e >= max|v| (bits written by vmax_kernel)
+    float acc_scale, acc_inv;
+    {
+        const uint32_t vb = (uint32_t)P.counters[3 * P.J + 1];
+        int ev = (int)((vb >> 23) & 0xff) - 127;
+        if (vb & 0x7fffffu) ev += 1;
+        if (vb == 0) ev = 0;
+        ev = max(-100, min(ev, 120));
+        acc_scale = __int_as_float((ev + 127) << 23);
+        acc_inv = __int_as_float((127 - ev) << 23);
+    }
 
     // lane 0 waits, the whole warp gets the verdict (warp-uniform control flow)
     auto warp_wait = [&](uint64_t *b, uint32_t par) -> bool {
@@ -353,12 +368,17 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 __syncwarp();
                 PROF_END(8);
                 PROF_BEGIN();
-                if (lane < ntok) {
+                if constexpr (L::NH == 2) {
+                    // one 3D box per 8-row group (both 64-column halves): 128 rows = 16 loads
+                    constexpr int GPT = G / 8;  // 8-row groups per token
+                    const int tq = __shfl_sync(0xffffffffu, t, lane / GPT);
+                    if (lane < ntok * GPT) {
+                        const int row = (b * P.L + tq) * P.hq + g * G + (lane % GPT) * 8;
+                        tma_load_3d(sm + L::OFF_Q + qs * L::QBYTES + lane * 2048, &tm_q, 0, row, 0, &B.q_full[qs]);
+                    }
+                } else if (lane < ntok) {
                     const int row = (b * P.L + t) * P.hq + g * G;
-#pragma unroll
-                    for (int h = 0; h < L::NH; ++h)
-                        tma_load_2d(sm + L::OFF_Q + qs * L::QBYTES + h * L::QHALF + lane * G * 128, &tm_q, h * 64,
-                                    row, &B.q_full[qs]);
+                    tma_load_2d(sm + L::OFF_Q + qs * L::QBYTES + lane * G * 128, &tm_q, 0, row, &B.q_full[qs]);
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&B.info_full[ti]);
@@ -418,7 +438,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
 #pragma unroll
                             for (int ks = 0; ks < D / 16; ++ks) {
                                 const int h = ks >> 2, kk = ks & 3;
-                                mma_bf16_ss(dcol, smem_desc_sw128(qa + h * L::QHALF + kk * 32, 16, 1024),
+                                // Q: d = 128 in 2 KB groups of 8 rows x both halves; d = 64 in 1 KB groups
+                                mma_bf16_ss(dcol, smem_desc_sw128(qa + h * 1024 + kk * 32, 16, L::NH * 1024),
                                             smem_desc_sw128(kb + h * L::KVHALF + kk * 32, 16, 1024), idesc1, ks > 0);
                             }
                             mma_commit(&B.s_full[sb]);
@@ -664,31 +685,41 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             const float coef = ecoef[ii * 128 + r];
             const int s = inf.j % kRing;
             const int ws = (inf.j % P.nW) * P.W;
-            // this lane reduces, for m = 0..7, the 16-byte chunk lane % 8 of warp row 4m + lane / 8
-            float *dst[8];
+            // this lane reduces, for m = 0..7, the 16-byte chunk lane % 8 (8 halves) of warp row 4m + lane / 8
+            const float cf = coef * acc_inv;
+            __half *dst[8];
             bool dok[8];
 #pragma unroll
             for (int m = 0; m < 8; ++m) {
                 const int tr = wq * 32 + 4 * m + (lane >> 3);
                 const int i = tr / G;
                 dok[m] = i < inf.ntok;
-                dst[m] = acc + ((int64_t)(s * P.W + inf.tok[i] - ws) * G + tr % G) * D + (lane & 7) * 4;
+                dst[m] = acc + ((int64_t)(s * P.W + inf.tok[i] - ws) * G + tr % G) * D + (lane & 7) * 8;
             }
+            uint4 *xs4 = reinterpret_cast<uint4 *>(xs);
 #pragma unroll
-            for (int q = 0; q < D / 32; ++q) {
-                float v[32];
-                tmem_ld32(lane_base + 128 + sb * 128 + q * 32, v);
-                tmem_wait_ld();
+            for (int q = 0; q < D / 64; ++q) {  // 64 columns = one 128-byte fp16 line per row
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch)
-                    xs[lane * 8 + (ch ^ (lane & 7))] = make_float4(v[4 * ch] * coef, v[4 * ch + 1] * coef,
-                                                                   v[4 * ch + 2] * coef, v[4 * ch + 3] * coef);
+                for (int hv = 0; hv < 2; ++hv) {  // 32 columns at a time: 4 chunks of 8 halves
+                    float v[32];
+                    tmem_ld32(lane_base + 128 + sb * 128 + q * 64 + hv * 32, v);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        const int ch = hv * 4 + c4;
+                        __half2 h[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            h[e] = __floats2half2_rn(v[c4 * 8 + 2 * e] * cf, v[c4 * 8 + 2 * e + 1] * cf);
+                        xs4[lane * 8 + (ch ^ (lane & 7))] = *reinterpret_cast<uint4 *>(h);
+                    }
+                }
                 __syncwarp();
 #pragma unroll
                 for (int m = 0; m < 8; ++m) {
                     const int row = 4 * m + (lane >> 3);
-                    const float4 f = xs[row * 8 + ((lane & 7) ^ (row & 7))];
-                    if (dok[m]) red_add_v4_f32(dst[m] + q * 32, f);
+                    const uint4 f = xs4[row * 8 + ((lane & 7) ^ (row & 7))];
+                    if (dok[m]) red_add_v4_f16x2(dst[m] + q * 64, f);
                 }
                 __syncwarp();
             }
@@ -747,40 +778,36 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 const int ws = (j % P.nW) * P.W;
                 const int we = min(P.L, ws + P.W);
                 const int ta = ws + item * kCombTokens, tb = min(we, ta + kCombTokens);
-                // fp32 accumulators of tokens [ta, tb): G*D contiguous floats per token, and
-                // o of (token, group g): G*D contiguous bf16.  A unit is 8 floats -> 16 bytes of o.
+                // fp16 accumulators of tokens [ta, tb): G*D contiguous values per token, and
+                // o of (token, group g): G*D contiguous bf16.  A unit is 8 values -> 16 bytes of o.
                 constexpr int UPT = G * D / 8;  // units per token
                 constexpr int kBatch = 8;       // units in flight per thread
-                float4 *A = reinterpret_cast<float4 *>(acc + (int64_t)(s * P.W + (ta - ws)) * G * D);
+                uint4 *A = reinterpret_cast<uint4 *>(acc + (int64_t)(s * P.W + (ta - ws)) * G * D);
                 const int nunits = (tb - ta) * UPT;
                 for (int u0 = 0; u0 < nunits; u0 += kConvThreads * kBatch) {
-                    float4 lo[kBatch], hi[kBatch];
+                    uint4 raw[kBatch];
 #pragma unroll
                     for (int k = 0; k < kBatch; ++k) {
                         const int u = u0 + k * kConvThreads + tid;
-                        if (u < nunits) {
-                            lo[k] = __ldcg(A + 2 * u);
-                            hi[k] = __ldcg(A + 2 * u + 1);
-                        }
+                        if (u < nunits) raw[k] = __ldcg(A + u);
                     }
 #pragma unroll
                     for (int k = 0; k < kBatch; ++k) {
                         const int u = u0 + k * kConvThreads + tid;
                         if (u < nunits) {
                             const int t = ta + u / UPT, e = u % UPT;
-                            __nv_bfloat162 a0 = __floats2bfloat162_rn(lo[k].x, lo[k].y);
-                            __nv_bfloat162 a1 = __floats2bfloat162_rn(lo[k].z, lo[k].w);
-                            __nv_bfloat162 a2 = __floats2bfloat162_rn(hi[k].x, hi[k].y);
-                            __nv_bfloat162 a3 = __floats2bfloat162_rn(hi[k].z, hi[k].w);
-                            uint4 pk;
-                            pk.x = *reinterpret_cast<uint32_t *>(&a0); pk.y = *reinterpret_cast<uint32_t *>(&a1);
-                            pk.z = *reinterpret_cast<uint32_t *>(&a2); pk.w = *reinterpret_cast<uint32_t *>(&a3);
+                            const __half2 *h2 = reinterpret_cast<const __half2 *>(&raw[k]);
+                            __nv_bfloat162 o2[4];
+#pragma unroll
+                            for (int x = 0; x < 4; ++x) {
+                                const float2 f = __half22float2(h2[x]);
+                                o2[x] = __floats2bfloat162_rn(f.x * acc_scale, f.y * acc_scale);
+                            }
                             // o is not read again here: streaming store
                             __stcs(reinterpret_cast<uint4 *>(out + (((int64_t)b * P.L + t) * P.hq + g * G) * D + e * 8),
-                                   pk);
+                                   *reinterpret_cast<uint4 *>(o2));
                             // the slot starts the window kRing later at zero
-                            A[2 * u] = make_float4(0.f, 0.f, 0.f, 0.f);
-                            A[2 * u + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
+                            A[u] = make_uint4(0, 0, 0, 0);
                         }
                     }
                 }
@@ -838,12 +865,28 @@ bool make_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, ui
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// query rows of d = 128 as a 3D view (64 columns, rows, 2 halves of 128 bytes);
+// box = 8 rows x both halves, stored half after half (2 KB, 128B swizzle)
+bool make_map_q3(CUtensorMap *m, const void *base, uint64_t rows) {
+    EncodeTiledFn enc = get_encode();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {64, rows, 2};
+    cuuint64_t strides[2] = {256, 128};
+    cuuint32_t box[3] = {64, 8, 2};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int D, int G>
 cudaError_t launch_tc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv, const void *q, const void *k,
-                      const void *v, const int32_t *idx, const float *w, float *acc, void *o,
+                      const void *v, const int32_t *idx, const float *w, __half *acc, void *o,
                       float *lse, DevStatus *ds, cudaStream_t st) {
     CUtensorMap mq, mk, mv;
-    if (!make_map(&mq, q, D, (uint64_t)sh.B * sh.L * sh.hq, G) ||
+    const bool qok = D == 128 ? make_map_q3(&mq, q, (uint64_t)sh.B * sh.L * sh.hq)
+                              : make_map(&mq, q, D, (uint64_t)sh.B * sh.L * sh.hq, G);
+    if (!qok ||
         !make_map(&mk, k, D, (uint64_t)sh.B * sh.hkv * sh.L, 64) ||
         !make_map(&mv, v, D, (uint64_t)sh.B * sh.hkv * sh.L, 64))
         return cudaErrorInvalidValue;
@@ -866,6 +909,33 @@ extern "C" HSA_API int hsa_debug_tc_profile(void *dev_buf) {
 }
 #endif
 
+// max|v| over the value tensor (bf16, length a multiple of 8), as float bits
+// max-ed into *bits: non-negative floats order like their bit patterns.
+__global__ void __launch_bounds__(256) vmax_kernel(const __nv_bfloat16 *__restrict__ v, int64_t n8,
+                                                   int32_t *__restrict__ bits) {
+    float m = 0.f;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8; i += (int64_t)gridDim.x * blockDim.x) {
+        const uint4 raw = __ldcs(reinterpret_cast<const uint4 *>(v) + i);
+        const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(h[e]);
+            m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if ((threadIdx.x & 31) == 0) atomicMax(bits, __float_as_int(m));
+}
+
+cudaError_t launch_vmax(const Shape &sh, const void *v, int32_t *bits, cudaStream_t st) {
+    const int64_t n8 = (int64_t)sh.B * sh.hkv * sh.L * sh.d / 8;
+    if (n8 == 0) return cudaSuccess;
+    const int blocks = (int)std::min<int64_t>(ceil_div(n8, 256), 148 * 4);
+    vmax_kernel<<<blocks, 256, 0, st>>>((const __nv_bfloat16 *)v, n8, bits);
+    return cudaGetLastError();
+}
+
 bool attend_tc_supported(const Shape &sh) {
     return sh.bf16 && (sh.d == 64 || sh.d == 128) && (sh.G == 8 || sh.G == 16) && sh.K <= 16 &&
            get_encode() != nullptr;
@@ -873,7 +943,7 @@ bool attend_tc_supported(const Shape &sh) {
 
 cudaError_t launch_attend_tc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv, const void *q,
                              const void *k, const void *v, const int32_t *idx, const float *w,
-                             float *acc, void *o, float *lse, DevStatus *ds, cudaStream_t st) {
+                             __half *acc, void *o, float *lse, DevStatus *ds, cudaStream_t st) {
     if (sh.d == 128 && sh.G == 8) return launch_tc<128, 8>(sh, plan, inv, q, k, v, idx, w, acc, o, lse, ds, st);
     if (sh.d == 128 && sh.G == 16) return launch_tc<128, 16>(sh, plan, inv, q, k, v, idx, w, acc, o, lse, ds, st);
     if (sh.d == 64 && sh.G == 8) return launch_tc<64, 8>(sh, plan, inv, q, k, v, idx, w, acc, o, lse, ds, st);

@@ -84,6 +84,12 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap *map, const void 
                  "r"(smem_u32(smem_src)), "r"(x), "r"(y)
                  : "memory");
 }
+// Element-wise add of 8 fp16 values (16 bytes, no flush of subnormals), performed in L2.
+__device__ __forceinline__ void red_add_v4_f16x2(void *p, uint4 v) {
+    asm volatile("red.relaxed.gpu.global.add.noftz.v4.f16x2 [%0], {%1, %2, %3, %4};" ::"l"(p), "r"(v.x), "r"(v.y),
+                 "r"(v.z), "r"(v.w)
+                 : "memory");
+}
 // Element-wise fp32 add of 16 bytes into global memory, performed in L2 (no return value).
 __device__ __forceinline__ void red_add_v4_f32(float *p, float4 v) {
     asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(v.x), "f"(v.y), "f"(v.z),

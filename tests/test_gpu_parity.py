@@ -132,6 +132,21 @@ def test_fwd_tensor_core_path_full(wl):
     assert not f64(o)[:, :wl.S].any()
 
 
+@pytest.mark.parametrize("factor", [2.0 ** 12, 2.0 ** -12], ids=["v-x4096", "v-x1/4096"])
+def test_fwd_tensor_core_value_scale(factor):
+    """The chunk-major forward sums chunk outputs in fp16 scaled by a power of two
+    >= max|v|.  Scaling v by an exact power of two scales o exactly, so o / factor
+    must match the unscaled oracle at the same bar."""
+    wl = FWD_TC[0]
+    x, kbar, sel = gap_ruled(wl)
+    o_ref, lse_ref, idx_ref, w_ref = oracle.fwd(x["q"], x["k"], x["v"], x["q_slc"], kbar, wl.S, wl.K)
+    xs = dict(x)
+    xs["v"] = x["v"] * factor
+    o, lse, idx, w, kb = run_fwd(wl, xs)
+    assert np.array_equal(idx.cpu().numpy().reshape(idx_ref.shape), idx_ref)
+    assert_out(f64(o).reshape(o_ref.shape) / factor, o_ref, "bf16", "o")
+
+
 def test_fwd_tiny_fp32_workload():
     """The tiny fp32 workload in full: indices exact, max |err| <= 1e-5."""
     wl, (x, kbar, sel) = cached_workload("tiny_fp32")

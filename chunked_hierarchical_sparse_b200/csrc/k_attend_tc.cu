@@ -146,10 +146,6 @@ __device__ bool spin_geq_live(const int32_t *p, int target, volatile int *abort)
 }
 
 
-__device__ __forceinline__ void wg_sync() {  // named barrier 1 over the softmax warps 0..3
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-}
-
 }  // namespace
 
 template <int D, int G>
@@ -177,24 +173,22 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     uint64_t *coef_full = mma_done + 1;  // [kInfo] row coefficients written (softmax -> epilogue)
     uint64_t *p_empty = coef_full + kInfo;  // [2] P buffer read by its O = P.V (MMA -> softmax)
     float *ecoef = reinterpret_cast<float *>(sm + L::OFF_COEF);
-    volatile int *eg_flag = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 40);  // [2][2] epilogue groups
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 16);
-    volatile int *wg_flag = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 32);  // [2] softmax group
     volatile int *cg_flag = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 56);  // [2] convert group
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kInfo; ++i) { mbar_init(&B.info_full[i], 1); mbar_init(&B.info_empty[i], 3); }
+        for (int i = 0; i < kInfo; ++i) { mbar_init(&B.info_full[i], 1); mbar_init(&B.info_empty[i], 1 + 8); }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&B.q_full[i], 1); mbar_init(&B.q_empty[i], 1);
             mbar_init(&B.kv_full[i], 1); mbar_init(&B.kv_empty[i], 1);
             mbar_init(&B.s_full[i], 1); mbar_init(&B.s_empty[i], 4);
-            mbar_init(&B.p_full[i], 128);
+            mbar_init(&B.p_full[i], 4);
             mbar_init(&B.o_full[i], 1); mbar_init(&B.o_empty[i], 4);
         }
         mbar_init(mma_done, 1);
-        for (int i = 0; i < kInfo; ++i) mbar_init(&coef_full[i], 128);
+        for (int i = 0; i < kInfo; ++i) mbar_init(&coef_full[i], 4);
         for (int i = 0; i < 2; ++i) mbar_init(&p_empty[i], 1);
         *abort_flag = 0;
         mbar_fence_init();
@@ -499,32 +493,20 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         // ============================================================ softmax
         const int wq = warp & 3;                 // TMEM lane quadrant of this warp
         const int r = wq * 32 + lane;            // tile row = token * G + head
-        const int tid = threadIdx.x;             // 0..127
         const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
-        int it = 0, tseq = 0, wcnt = 0;
+        int it = 0, tseq = 0;
         bool ok = true;
         PROF_DECL
         const long long prof_start = clock64();
         (void)prof_start;
 
-        // thread 0 decides, the whole group follows (uniform control flow at named barriers)
-        auto wg_vote = [&](int v) -> bool {
-            const int slot = (wcnt++) & 1;
-            if (tid == 0) wg_flag[slot] = v;
-            wg_sync();
-            return wg_flag[slot] != 0;
-        };
-        auto wg_wait = [&](uint64_t *b, uint32_t par) -> bool {
-            int v = 1;
-            if (tid == 0) v = mbar_wait(b, par, kWaitNs) ? 1 : 0;
-            return wg_vote(v);
-        };
-
+        // every warp waits for itself (lane 0 polls, the warp gets the verdict): the four
+        // warps only meet at the mbarriers they arrive on
         while (ok) {
             const int ii = it % kInfo;
             const uint32_t ipar = (it / kInfo) & 1;
             PROF_BEGIN();
-            if (!wg_wait(&B.info_full[ii], ipar)) { ok = false; break; }
+            if (!warp_wait(&B.info_full[ii], ipar)) { ok = false; break; }
             PROF_END(1);
             const TileInfo &inf = info[ii];
             const int type = inf.type;
@@ -532,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             // ---------------- softmax of this tile
             const int sb = tseq & 1;
             PROF_BEGIN();
-            if (!wg_wait(&B.s_full[sb], (tseq >> 1) & 1)) { ok = false; break; }
+            if (!warp_wait(&B.s_full[sb], (tseq >> 1) & 1)) { ok = false; break; }
             PROF_END(2);
             PROF_INC(12);
             PROF_BEGIN();
@@ -545,7 +527,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             __syncwarp();
             if (lane == 0) mbar_arrive(&B.s_empty[sb]);
             // P buffer sb is free once the O = P.V of tile tseq - 2 has read it
-            if (tseq >= 2 && !wg_wait(&p_empty[sb], ((tseq >> 1) - 1) & 1)) { ok = false; break; }
+            PROF_END(3);
+            PROF_BEGIN();
+            if (tseq >= 2 && !warp_wait(&p_empty[sb], ((tseq >> 1) - 1) & 1)) { ok = false; break; }
+            PROF_END(4);
+            PROF_BEGIN();
             const int ti = r / G, hh = r % G;
             const bool valid = ti < inf.ntok;
             uint8_t *prow = sm + L::OFF_P + sb * L::PBYTES + r * 128;
@@ -596,19 +582,21 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch) *reinterpret_cast<uint4 *>(prow + (ch << 4)) = make_uint4(0, 0, 0, 0);
             }
-            fence_proxy_async_smem();
-            mbar_arrive(&B.p_full[sb]);
+            fence_proxy_async_smem();  // each writer orders its P rows before the MMA's reads
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&B.p_full[sb]);  // one arrival per warp
             PROF_END(3);
             // the row's output coefficient w / Z for the epilogue group
             ecoef[ii * 128 + r] = coef;
-            mbar_arrive(&coef_full[ii]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&coef_full[ii]);
             ++tseq;
             ++it;
         }
-        if (!ok) { *abort_flag = 1; if (tid == 0) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 5, it); }
+        if (!ok) { *abort_flag = 1; if (lane == 0) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 5, it); }
 #ifdef HSA_TC_PROFILE
         prof_acc[0] = clock64() - prof_start;
-        if (tid == 0) PROF_DUMP(blockIdx.x * 96 + 32);
+        if (threadIdx.x == 0) PROF_DUMP(blockIdx.x * 96 + 32);
 #endif
     } else if (warp < kWarpConv) {
         // ============================================================ epilogue
@@ -621,31 +609,20 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         const int eg = (warp - kWarpEpi) >> 2;                    // epilogue group = its O buffer
         const int wq = warp & 3;
         const int r = wq * 32 + lane;                             // tile row of this lane's TMEM loads
-        const int tid = threadIdx.x - (kWarpEpi + 4 * eg) * 32;   // 0..127
         const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
         float4 *xs = reinterpret_cast<float4 *>(sm + L::OFF_X + (warp - kWarpEpi) * 4096);  // [32 rows][8 chunks]
-        volatile int *gflag = eg_flag + 2 * eg;
-        int it = 0, tseq = 0, ecnt = 0, ecnt_j = -1, vcnt = 0;
+        int it = 0, tseq = 0, ecnt = 0, ecnt_j = -1;
         bool ok = true;
         PROF_DECL
         const long long prof_start = clock64();
         (void)prof_start;
-        auto eg_sync = [&]() { asm volatile("bar.sync %0, 128;" ::"r"(3 + eg) : "memory"); };
-        auto eg_vote = [&](int v) -> bool {
-            const int slot = (vcnt++) & 1;
-            if (tid == 0) gflag[slot] = v;
-            eg_sync();
-            return gflag[slot] != 0;
-        };
-        auto eg_wait = [&](uint64_t *b, uint32_t par) -> bool {
-            int v = 1;
-            if (tid == 0) v = mbar_wait(b, par, kWaitNs) ? 1 : 0;
-            return eg_vote(v);
-        };
-        auto flush = [&]() {  // publish the reductions of the tiles counted so far
+        // Each warp runs on its own: it waits for itself, acknowledges each info slot
+        // itself and publishes its own reduced rows per window (a window is complete
+        // when its tiles are counted by all four warps of their group).
+        auto flush = [&]() {  // publish this warp's reductions of the tiles counted so far
             __threadfence();
-            eg_sync();
-            if (tid == 0) {
+            __syncwarp();
+            if (lane == 0) {
                 __threadfence();
                 atomicAdd(&tiles_done[ecnt_j], ecnt);
             }
@@ -656,17 +633,17 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             const uint32_t ipar = (it / kInfo) & 1;
             if (ecnt > 0) {  // never sit on unpublished tiles while the next one is not there yet
                 int ready = 1;
-                if (tid == 0) ready = mbar_test(&B.info_full[ii], ipar) ? 1 : 0;
-                if (!eg_vote(ready)) flush();
+                if (lane == 0) ready = mbar_test(&B.info_full[ii], ipar) ? 1 : 0;
+                if (!__shfl_sync(0xffffffffu, ready, 0)) flush();
             }
             PROF_BEGIN();
-            if (!eg_wait(&B.info_full[ii], ipar)) { ok = false; break; }
+            if (!warp_wait(&B.info_full[ii], ipar)) { ok = false; break; }
             PROF_END(1);
             const TileInfo &inf = info[ii];
             if (inf.type == kItemEnd) break;
             if ((tseq & 1) != eg) {  // the other group's tile: acknowledge the slot and move on
-                eg_sync();
-                if (tid == 0) mbar_arrive(&B.info_empty[ii]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&B.info_empty[ii]);
                 ++tseq;
                 ++it;
                 continue;
@@ -677,8 +654,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             }
             const int sb = tseq & 1;
             PROF_BEGIN();
-            if (!eg_wait(&B.o_full[sb], (tseq >> 1) & 1)) { ok = false; break; }
-            if (!eg_wait(&coef_full[ii], ipar)) { ok = false; break; }
+            if (!warp_wait(&B.o_full[sb], (tseq >> 1) & 1)) { ok = false; break; }
+            if (!warp_wait(&coef_full[ii], ipar)) { ok = false; break; }
             PROF_END(2);
             PROF_BEGIN();
             tc_fence_after();
@@ -725,19 +702,20 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&B.o_empty[sb]);
-            eg_sync();  // the whole group is done with this tile's info entry
-            if (tid == 0) mbar_arrive(&B.info_empty[ii]);
+            if (lane == 0) {
+                mbar_arrive(&B.o_empty[sb]);
+                mbar_arrive(&B.info_empty[ii]);  // this warp is done with the tile's info entry
+            }
             PROF_END(3);
             ++ecnt;
             ++tseq;
             ++it;
         }
         if (ok && ecnt > 0) flush();
-        if (!ok) { *abort_flag = 1; if (tid == 0) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 6, it); }
+        if (!ok) { *abort_flag = 1; if (lane == 0) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 6, it); }
 #ifdef HSA_TC_PROFILE
         prof_acc[0] = clock64() - prof_start;
-        if (tid == 0) PROF_DUMP(blockIdx.x * 96 + 64 + 16 * eg);
+        if (lane == 0 && wq == 0) PROF_DUMP(blockIdx.x * 96 + 64 + 16 * eg);
 #endif
     } else if (warp < kWarpProd) {
         // ============================================================ convert group
@@ -762,7 +740,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         for (int jc = 0; jc < P.J && ok; ++jc) {
             int gok = 1;
             PROF_BEGIN();
-            if (tid == 0) gok = spin_geq_live(&tiles_done[jc], P.win_tiles[jc], abort_flag) ? 1 : 0;
+            // every tile is counted by the four warps of its epilogue group
+            if (tid == 0) gok = spin_geq_live(&tiles_done[jc], 4 * P.win_tiles[jc], abort_flag) ? 1 : 0;
             if (!cg_bcast(gok)) { if (tid == 0 && !*abort_flag) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 4, jc); ok = false; break; }
             PROF_END(2);
             const int ncomb = P.win_ncomb[jc];

@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
             mbar_init(&sd_full[i], 1); mbar_init(&sd_empty[i], 4);
         }
         mbar_init(kv_full, 1); mbar_init(kv_empty, 1);
-        mbar_init(ds_full, 128); mbar_init(ds_empty, 1);
+        mbar_init(ds_full, 4); mbar_init(ds_empty, 1);
         mbar_init(dq_full, 1); mbar_init(dq_empty, 4);
         mbar_init(dkv_full, 1); mbar_init(dkv_empty, 4);
         mbar_init(mma_done, 1);
@@ -513,8 +513,9 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
                     *reinterpret_cast<uint4 *>(wprow + (ch << 4)) = make_uint4(0, 0, 0, 0);
                 }
             }
-            fence_proxy_async_smem();
-            mbar_arrive(ds_full);
+            fence_proxy_async_smem();  // each writer orders its dS / wP rows before the MMA's reads
+            __syncwarp();
+            if (lane == 0) mbar_arrive(ds_full);  // one arrival per warp
             ++it;
         }
         if (!ok) { *abort_flag = 1; if (tid == 0) report(ds, HSA_ERR_TIMEOUT, kKBwdTc, 5, it); }

@@ -11,15 +11,18 @@
 // the work is spread over the cluster and exchanged through distributed
 // shared memory instead of global memory:
 //   1. CTA r scores its slice of the chunk index (coalesced 512 B rows).
-//   2. cluster barrier; every CTA reads all scores over DSMEM and keeps the
-//      same top-K (warp 0), orders it most-recent-first, forms the
-//      stick-breaking weights.
+//   2. cluster barrier; every CTA reads all scores over DSMEM and selects
+//      the same top-K with all its threads: a threshold (the K-th best of the
+//      per-thread bests) leaves a few survivors, which are ranked pairwise;
+//      warp 0 orders the K most-recent-first and forms the stick-breaking
+//      weights.
 //   3. CTA r attends the group's G query heads to the chunk of slot r (and
 //      r + kDecCta, ...), softmax-off-by-one, and scales by w / Z.
 //   4. cluster barrier; CTA r sums its share of the output columns over all
 //      CTAs' partial outputs (DSMEM) and writes o; a last barrier keeps every
 //      CTA's shared memory alive until all remote reads are done.
 #include <cooperative_groups.h>
+#include <type_traits>
 #include <math_constants.h>
 
 #include "hsa_internal.cuh"
@@ -29,8 +32,193 @@ namespace cg = cooperative_groups;
 
 namespace hsa {
 
+#ifdef HSA_TC_PROFILE
+// Phase timestamps of the decode step (development builds only).
+__device__ unsigned long long *g_dec_prof = nullptr;
+#define DEC_STAMP(i)                                                                                 \
+    do {                                                                                             \
+        if (g_dec_prof && threadIdx.x == 0) {                                                        \
+            unsigned long long t_;                                                                   \
+            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                                  \
+            g_dec_prof[blockIdx.x * 8 + (i)] = t_;                                                   \
+        }                                                                                            \
+    } while (0)
+#else
+#define DEC_STAMP(i) ((void)0)
+#endif
+
 constexpr int kDecCta = 8;
 constexpr int kDecThreads = 128;
+
+// The chunk's K (to a padded [64][D+1] fp32 tile) and V (to [64][D] fp32): every
+// thread issues all of its 16-byte loads before the first store.
+template <typename T, int D>
+__device__ __forceinline__ void load_chunk(const T *__restrict__ kc, const T *__restrict__ vc, float *Ks, float *Vs,
+                                           int tid) {
+    constexpr int EPV = 16 / sizeof(T);                  // elements per 16-byte vector
+    constexpr int NV = kChunk * D / EPV / kDecThreads;   // vectors per thread and tensor
+    constexpr int NB = NV < 8 ? NV : 8;                  // vectors in flight per batch
+#pragma unroll 1
+    for (int u0 = 0; u0 < NV; u0 += NB) {
+    uint4 rk[NB], rv[NB];
+#pragma unroll
+    for (int u = 0; u < NB; ++u) {
+        rk[u] = __ldcs(reinterpret_cast<const uint4 *>(kc) + tid + (u0 + u) * kDecThreads);
+        rv[u] = __ldcs(reinterpret_cast<const uint4 *>(vc) + tid + (u0 + u) * kDecThreads);
+    }
+#pragma unroll
+    for (int u = 0; u < NB; ++u) {
+        const int e = (tid + (u0 + u) * kDecThreads) * EPV;  // first element; the vector stays in one row
+        const int i = e / D, j = e % D;
+        const T *pk = reinterpret_cast<const T *>(&rk[u]);
+        const T *pv = reinterpret_cast<const T *>(&rv[u]);
+#pragma unroll
+        for (int x = 0; x < EPV; ++x) {
+            Ks[i * (D + 1) + j + x] = Elem<T>::load(pk + x);
+            Vs[e + x] = Elem<T>::load(pv + x);
+        }
+    }
+    }
+}
+
+// ---------------------------------------------------------------- bf16 tensor-core tile
+// Pitches (bf16 elements) of the shared tiles of the bf16 path, padded so that the
+// fragment loads of a warp hit 32 different banks.
+template <int D> struct DecTile {
+    static constexpr int QP = D + 8;   // Q16 [16][QP]: the G query heads (rows >= G zero)
+    static constexpr int KP = D + 8;   // K16 [64][KP]
+    static constexpr int VP = D + 8;   // V16 [64][VP] (row-major; read transposed by ldmatrix)
+};
+
+__device__ __forceinline__ uint32_t ld_b32(const __nv_bfloat16 *p) { return *reinterpret_cast<const uint32_t *>(p); }
+
+// D[16x8] += A[16x16] B[16x8], bf16 operands, fp32 accumulators (one warp)
+__device__ __forceinline__ void mma_16816(float (&c)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// The chunk's K and V to K16 / V16 (row-major, padded rows), 16-byte loads issued first.
+template <int D>
+__device__ __forceinline__ void load_chunk16(const __nv_bfloat16 *__restrict__ kc, const __nv_bfloat16 *__restrict__ vc,
+                                             __nv_bfloat16 *K16, __nv_bfloat16 *V16, int tid) {
+    using DT = DecTile<D>;
+    constexpr int NV = kChunk * D / 8 / kDecThreads;  // 16-byte vectors per thread and tensor
+    uint4 rk[NV], rv[NV];
+#pragma unroll
+    for (int u = 0; u < NV; ++u) {
+        rk[u] = __ldcs(reinterpret_cast<const uint4 *>(kc) + tid + u * kDecThreads);
+        rv[u] = __ldcs(reinterpret_cast<const uint4 *>(vc) + tid + u * kDecThreads);
+    }
+#pragma unroll
+    for (int u = 0; u < NV; ++u) {
+        const int e = (tid + u * kDecThreads) * 8;
+        const int i = e / D, j = e % D;
+        *reinterpret_cast<uint4 *>(K16 + i * DT::KP + j) = rk[u];
+        *reinterpret_cast<uint4 *>(V16 + i * DT::VP + j) = rv[u];
+    }
+}
+
+// One selected chunk on the tensor cores: every warp computes the G x 64 scores
+// (heads padded to 16 rows), applies softmax-off-by-one in registers, and adds
+// w / Z * P V for its quarter of the d columns into part[G][D].
+template <int D>
+__device__ __forceinline__ void attend_chunk16(const __nv_bfloat16 *Q16, const __nv_bfloat16 *K16,
+                                               const __nv_bfloat16 *V16, float *part, int G, float wk,
+                                               float scale, int warp, int lane) {
+    using DT = DecTile<D>;
+    const int g = lane >> 2, t = lane & 3;
+    float sacc[8][4];
+#pragma unroll
+    for (int n = 0; n < 8; ++n) sacc[n][0] = sacc[n][1] = sacc[n][2] = sacc[n][3] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+        uint32_t a[4];
+        a[0] = ld_b32(Q16 + g * DT::QP + kk * 16 + 2 * t);
+        a[1] = ld_b32(Q16 + (g + 8) * DT::QP + kk * 16 + 2 * t);
+        a[2] = ld_b32(Q16 + g * DT::QP + kk * 16 + 2 * t + 8);
+        a[3] = ld_b32(Q16 + (g + 8) * DT::QP + kk * 16 + 2 * t + 8);
+#pragma unroll
+        for (int n = 0; n < 8; ++n) {
+            uint32_t bb[2];
+            bb[0] = ld_b32(K16 + (n * 8 + g) * DT::KP + kk * 16 + 2 * t);
+            bb[1] = ld_b32(K16 + (n * 8 + g) * DT::KP + kk * 16 + 2 * t + 8);
+            mma_16816(sacc[n], a, bb);
+        }
+    }
+    // rows g (elements 0, 1) and g + 8 (elements 2, 3); a row's 64 keys live in the 4 lanes of equal g
+    float m0 = 0.f, m1 = 0.f;  // the off-by-one term is a logit of 0
+#pragma unroll
+    for (int n = 0; n < 8; ++n) {
+        m0 = fmaxf(m0, fmaxf(sacc[n][0], sacc[n][1]) * scale);
+        m1 = fmaxf(m1, fmaxf(sacc[n][2], sacc[n][3]) * scale);
+    }
+#pragma unroll
+    for (int off = 1; off < 4; off <<= 1) {
+        m0 = fmaxf(m0, __shfl_xor_sync(0xffffffffu, m0, off));
+        m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, off));
+    }
+    float z0 = 0.f, z1 = 0.f;
+#pragma unroll
+    for (int n = 0; n < 8; ++n) {
+        sacc[n][0] = expf(sacc[n][0] * scale - m0);
+        sacc[n][1] = expf(sacc[n][1] * scale - m0);
+        sacc[n][2] = expf(sacc[n][2] * scale - m1);
+        sacc[n][3] = expf(sacc[n][3] * scale - m1);
+        z0 += sacc[n][0] + sacc[n][1];
+        z1 += sacc[n][2] + sacc[n][3];
+    }
+#pragma unroll
+    for (int off = 1; off < 4; off <<= 1) {
+        z0 += __shfl_xor_sync(0xffffffffu, z0, off);
+        z1 += __shfl_xor_sync(0xffffffffu, z1, off);
+    }
+    const float cf0 = wk / (z0 + expf(-m0)), cf1 = wk / (z1 + expf(-m1));
+    // O = P V for this warp's D/4 columns; P's fragments come straight from the scores'
+    constexpr int NT = D / 32;
+    float oacc[NT][4];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) oacc[n][0] = oacc[n][1] = oacc[n][2] = oacc[n][3] = 0.f;
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+        uint32_t a[4];
+        a[0] = pack_bf16(sacc[2 * kk][0], sacc[2 * kk][1]);
+        a[1] = pack_bf16(sacc[2 * kk][2], sacc[2 * kk][3]);
+        a[2] = pack_bf16(sacc[2 * kk + 1][0], sacc[2 * kk + 1][1]);
+        a[3] = pack_bf16(sacc[2 * kk + 1][2], sacc[2 * kk + 1][3]);
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+            const int d0 = warp * (D / 4) + n * 8;
+            // B fragment of V[keys 16kk.., columns d0..d0+7]: two 8x8 tiles read transposed
+            // (lanes 0-7 address the rows of the first tile, lanes 8-15 those of the second)
+            uint32_t bb[2];
+            const uint32_t addr = (uint32_t)__cvta_generic_to_shared(V16 + (kk * 16 + (lane & 15)) * DT::VP + d0);
+            asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0, %1}, [%2];"
+                         : "=r"(bb[0]), "=r"(bb[1]) : "r"(addr));
+            mma_16816(oacc[n], a, bb);
+        }
+    }
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+        const int d0 = warp * (D / 4) + n * 8 + 2 * t;
+        if (g < G) {
+            part[g * D + d0] += cf0 * oacc[n][0];
+            part[g * D + d0 + 1] += cf0 * oacc[n][1];
+        }
+        if (g + 8 < G) {
+            part[(g + 8) * D + d0] += cf1 * oacc[n][2];
+            part[(g + 8) * D + d0 + 1] += cf1 * oacc[n][3];
+        }
+    }
+}
 
 template <typename T, int D>
 __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
@@ -38,6 +226,7 @@ __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
                           const T *__restrict__ vc, const float *__restrict__ kbar, T *__restrict__ o,
                           int32_t *__restrict__ idx_out, float *__restrict__ w_out, int P, int hq, int hkv,
                           int nc, int K, int G) {
+    DEC_STAMP(0);
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
     const int bg = blockIdx.x / kDecCta, b = bg / hkv, g = bg % hkv;
@@ -53,6 +242,16 @@ __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
     float *Ks = Qs + kMaxG * D;                       // [64][D+1]
     float *Vs = Ks + kChunk * (D + 1);                // [64][D]
     float *Pm = Vs + kChunk * D;                      // [G][64]
+    const int ncr = (nc + 3) & ~3;
+    float *allsc = Pm + kMaxG * kChunk;               // [nc] every chunk's score (top-K stage)
+    float *surv_s = allsc + ncr;                      // [nc] candidates not beaten by the threshold
+    int *surv_c = reinterpret_cast<int *>(surv_s + ncr);
+    __shared__ float tmax_s[kDecThreads];
+    __shared__ int tmax_c[kDecThreads];
+    __shared__ float top_s[kMaxK];
+    __shared__ int top_c[kMaxK];
+    __shared__ float thr_s;
+    __shared__ int thr_c, n_surv;
     __shared__ int slot_c[kMaxK];
     __shared__ float slot_w[kMaxK];
     __shared__ float coef[kMaxG];
@@ -63,31 +262,96 @@ __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
     float qv[D / 32];
 #pragma unroll
     for (int e = 0; e < D / 32; ++e) qv[e] = Elem<T>::load(q_slc + (int64_t)bg * D + lane + 32 * e);
-    for (int c = c_lo + warp; c < c_hi; c += kDecThreads / 32) {
-        float acc = 0.f;
+    // each warp takes 8 chunks at a time: all 8 rows of k-bar are loaded before any is used
+    constexpr int kCB = 8;
+    for (int c0 = c_lo + warp * kCB; c0 < c_hi; c0 += kDecThreads / 32 * kCB) {
+        float kv[kCB][D / 32];
 #pragma unroll
-        for (int e = 0; e < D / 32; ++e) acc = fmaf(qv[e], kb[(int64_t)c * D + lane + 32 * e], acc);
+        for (int u = 0; u < kCB; ++u)
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-        if (lane == 0) scores[c - c_lo] = acc * scale;
-    }
-    for (int e = tid; e < G * D; e += kDecThreads)
-        Qs[e] = Elem<T>::load(q + ((int64_t)b * hq + (int64_t)g * G) * D + e);
-    for (int e = tid; e < kMaxG * D; e += kDecThreads) part[e] = 0.f;
-    cluster.sync();
-
-    // ---- 2. top-K over all chunks (every CTA, warp 0), read over DSMEM
-    if (warp == 0) {
-        float ls = (lane < K) ? -CUDART_INF_F : CUDART_INF_F;
-        int lc = (lane < K) ? -1 : 0x7fffffff;
-        for (int c0 = 0; c0 < nc; c0 += 64) {
-            const int ca = c0 + lane, cb = c0 + lane + 32;
-            float sa = 0.f, sb = 0.f;
-            if (ca < nc) sa = cluster.map_shared_rank(scores, ca / per)[ca % per];
-            if (cb < nc) sb = cluster.map_shared_rank(scores, cb / per)[cb % per];
-            topk_merge(K, sa, ca < nc ? ca : -1, sb, cb < nc ? cb : -1, ls, lc);
+            for (int e = 0; e < D / 32; ++e)
+                kv[u][e] = (c0 + u < c_hi) ? kb[(int64_t)(c0 + u) * D + lane + 32 * e] : 0.f;
+#pragma unroll
+        for (int u = 0; u < kCB; ++u) {
+            float acc = 0.f;
+#pragma unroll
+            for (int e = 0; e < D / 32; ++e) acc = fmaf(qv[e], kv[u][e], acc);
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+            if (lane == 0 && c0 + u < c_hi) scores[c0 + u - c_lo] = acc * scale;
         }
-        if (lane >= K) { ls = -CUDART_INF_F; lc = -1; }
+    }
+    constexpr bool kTc = std::is_same<T, __nv_bfloat16>::value;  // bf16: tensor-core chunk tiles
+    __nv_bfloat16 *Q16 = reinterpret_cast<__nv_bfloat16 *>(Qs);
+    __nv_bfloat16 *K16 = reinterpret_cast<__nv_bfloat16 *>(Ks);
+    __nv_bfloat16 *V16 = reinterpret_cast<__nv_bfloat16 *>(Vs);
+    if constexpr (kTc) {
+        for (int e = tid; e < 16 * D / 8; e += kDecThreads) {  // heads padded to the MMA's 16 rows
+            const int h = e / (D / 8), j = (e % (D / 8)) * 8;
+            *reinterpret_cast<uint4 *>(Q16 + h * DecTile<D>::QP + j) =
+                (h < G) ? *reinterpret_cast<const uint4 *>(q + ((int64_t)b * hq + (int64_t)g * G + h) * D + j)
+                        : make_uint4(0, 0, 0, 0);
+        }
+    } else {
+        for (int e = tid; e < G * D; e += kDecThreads)  // a few 2-byte loads per thread, all independent
+            Qs[e] = Elem<T>::load(q + ((int64_t)b * hq + (int64_t)g * G) * D + e);
+    }
+    for (int e = tid; e < kMaxG * D; e += kDecThreads) part[e] = 0.f;
+    DEC_STAMP(1);
+    cluster.sync();
+    DEC_STAMP(2);
+
+    // ---- 2. top-K over all chunks (every CTA, all threads), scores read over DSMEM.
+    // Order: (s1, c1) beats (s2, c2) iff s1 > s2, or s1 == s2 and c1 > c2.
+    // 2a. stage every score; each thread keeps the best of its candidates
+    float bs = -CUDART_INF_F;
+    int bc = -1;
+    for (int c = tid; c < nc; c += kDecThreads) {
+        const float sc = cluster.map_shared_rank(scores, c / per)[c % per];
+        allsc[c] = sc;
+        if (beats(sc, c, bs, bc)) { bs = sc; bc = c; }
+    }
+    tmax_s[tid] = bs;
+    tmax_c[tid] = bc;
+    if (tid == 0) { thr_s = -CUDART_INF_F; thr_c = -1; n_surv = 0; }
+    __syncthreads();
+    // 2b. threshold: the K-th best of the per-thread bests, a lower bound of the K-th best
+    //     score (the K best per-thread bests are K distinct candidates)
+    if (bc >= 0) {
+        int rk = 0;
+        for (int j = 0; j < kDecThreads; ++j) rk += beats(tmax_s[j], tmax_c[j], bs, bc) ? 1 : 0;
+        if (rk == K - 1) { thr_s = bs; thr_c = bc; }
+    }
+    __syncthreads();
+    // 2c. survivors: the candidates that the threshold does not beat
+    {
+        const float ts = thr_s;
+        const int tc = thr_c;
+        for (int c = tid; c < nc; c += kDecThreads) {
+            const float sc = allsc[c];
+            if (!beats(ts, tc, sc, c)) {
+                const int i = atomicAdd(&n_surv, 1);
+                surv_s[i] = sc;
+                surv_c[i] = c;
+            }
+        }
+    }
+    __syncthreads();
+    // 2d. rank the survivors; the K best take their place by rank
+    const int ns = n_surv;
+    for (int i = tid; i < ns; i += kDecThreads) {
+        const float si = surv_s[i];
+        const int ci = surv_c[i];
+        int rk = 0;
+        for (int j = 0; j < ns; ++j) rk += beats(surv_s[j], surv_c[j], si, ci) ? 1 : 0;
+        if (rk < K) { top_s[rk] = si; top_c[rk] = ci; }
+    }
+    __syncthreads();
+    // 2e. warp 0: most-recent-first order and the stick-breaking weights
+    if (warp == 0) {
+        const int nsel = min(K, ns);
+        float ls = (lane < nsel) ? top_s[lane] : -CUDART_INF_F;
+        int lc = (lane < nsel) ? top_c[lane] : -1;
         int sc_; float sw, ss;
         topk_finish(K, ls, lc, sc_, sw, ss);
         if (lane < K) {
@@ -100,6 +364,7 @@ __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
         }
     }
     __syncthreads();
+    DEC_STAMP(3);
 
     // ---- 3. attention to the chunks of this CTA's slots
     const T *kbase = kc + (int64_t)bg * P * D;
@@ -109,15 +374,13 @@ __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
         if (c < 0) break;  // valid slots form a prefix
         const float wk = slot_w[kk];
         __syncthreads();
-        for (int e = tid * 4; e < kChunk * D; e += kDecThreads * 4) {
-            // 4 consecutive elements of one row (D is a multiple of 4)
-            const int i = e / D, j = e % D;
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                Ks[i * (D + 1) + j + u] = Elem<T>::load(kbase + (int64_t)c * kChunk * D + e + u);
-                Vs[e + u] = Elem<T>::load(vbase + (int64_t)c * kChunk * D + e + u);
-            }
+        if constexpr (kTc) {
+            load_chunk16<D>(kbase + (int64_t)c * kChunk * D, vbase + (int64_t)c * kChunk * D, K16, V16, tid);
+            __syncthreads();
+            attend_chunk16<D>(Q16, K16, V16, part, G, wk, scale, warp, lane);
+            continue;
         }
+        load_chunk<T, D>(kbase + (int64_t)c * kChunk * D, vbase + (int64_t)c * kChunk * D, Ks, Vs, tid);
         __syncthreads();
         for (int e = tid; e < G * kChunk; e += kDecThreads) {
             const int h = e / kChunk, i = e % kChunk;
@@ -153,7 +416,9 @@ __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
             part[e] = fmaf(coef[h], acc, part[e]);
         }
     }
+    DEC_STAMP(4);
     cluster.sync();
+    DEC_STAMP(5);
 
     // ---- 4. sum the partial outputs of the cluster (DSMEM), this CTA's column share
     const int ncol = G * D;
@@ -164,13 +429,22 @@ __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
         for (int r = 0; r < kDecCta; ++r) acc += cluster.map_shared_rank(part, r)[e];
         Elem<T>::store(o + ((int64_t)b * hq + (int64_t)g * G) * D + e, acc);
     }
+    DEC_STAMP(6);
     cluster.sync();
+    DEC_STAMP(7);
 }
+
+#ifdef HSA_TC_PROFILE
+extern "C" HSA_API int hsa_debug_dec_profile(void *dev_buf) {
+    return cudaMemcpyToSymbol(g_dec_prof, &dev_buf, sizeof(void *)) == cudaSuccess ? 0 : 4;
+}
+#endif
 
 size_t decode_cluster_smem(int nc, int d) {
     const int per = (nc + kDecCta - 1) / kDecCta;
+    const size_t ncr = (size_t)((nc + 3) & ~3);
     return sizeof(float) * ((size_t)((per + 3) & ~3) + 2 * (size_t)kMaxG * d + (size_t)kChunk * (d + 1) +
-                            (size_t)kChunk * d + (size_t)kMaxG * kChunk);
+                            (size_t)kChunk * d + (size_t)kMaxG * kChunk + 3 * ncr);
 }
 
 template <typename T, int D>

@@ -33,6 +33,28 @@ namespace hsa {
 
 using namespace sm100;
 
+#ifdef HSA_TC_PROFILE
+// Per-CTA cycle accounting of the roles (development builds only).
+__device__ unsigned long long *g_btc_prof = nullptr;
+extern "C" HSA_API int hsa_debug_btc_profile(void *dev_buf) {
+    return cudaMemcpyToSymbol(g_btc_prof, &dev_buf, sizeof(void *)) == cudaSuccess ? 0 : 4;
+}
+#define BP_DECL unsigned long long bp_acc[16] = {0}; long long bp_t0 = 0; const long long bp_start = clock64();
+#define BP_BEGIN() (bp_t0 = clock64())
+#define BP_END(slot) (bp_acc[slot] += (unsigned long long)(clock64() - bp_t0))
+#define BP_DUMP(base)                                                                            \
+    do {                                                                                         \
+        bp_acc[0] = clock64() - bp_start;                                                        \
+        if (g_btc_prof)                                                                          \
+            for (int _i = 0; _i < 16; ++_i) atomicAdd(&g_btc_prof[blockIdx.x * 80 + (base) + _i], bp_acc[_i]); \
+    } while (0)
+#else
+#define BP_DECL
+#define BP_BEGIN() ((void)0)
+#define BP_END(slot) ((void)0)
+#define BP_DUMP(base) ((void)0)
+#endif
+
 namespace {
 
 #ifndef HSA_WAIT_NS
@@ -60,7 +82,9 @@ struct BTileInfo {
 };
 
 struct BSmem {
-    static constexpr int QHALF = 128 * 128;  // bytes per 64-column half of a 128-row tile
+    // a 128-row Q / dO tile: 16 groups of 8 rows, each group's two 64-column halves one
+    // after the other (1 KB each), so one TMA box loads a group
+    static constexpr int QHALF = 128 * 128;  // bytes of one 64-column half of a 128-row tile
     static constexpr int QBYTES = 2 * QHALF;
     static constexpr int KVHALF = 64 * 128;
     static constexpr int KVBYTES = 2 * KVHALF;
@@ -81,8 +105,9 @@ struct BSmem {
 };
 static_assert(BSmem::ALLOC <= 227 * 1024, "backward tile buffers exceed the shared memory of a CTA");
 
-// TMEM columns: S[2] 0..127, dP[2] 128..255, dQ 256..383, dK^T 384..447, dV^T 448..511
-constexpr uint32_t kColS = 0, kColDP = 128, kColDQ = 256, kColDK = 384, kColDV = 448;
+// TMEM columns: S 0..63, dP 64..127, dQ[2] 128..383, dK^T 384..447, dV^T 448..511 (the gradient
+// warps copy S and dP out at once, so one buffer each; the dQ drain overlaps the next dQ)
+constexpr uint32_t kColS = 0, kColDP = 64, kColDQ = 128, kColDK = 384, kColDV = 448;
 
 __device__ __forceinline__ float bex2(float x) {
     float y;
@@ -139,10 +164,10 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
     uint64_t *info_full = bar, *info_empty = bar + kBInfo;
     uint64_t *qd_full = bar + 2 * kBInfo, *qd_empty = qd_full + 2;  // [2] Q + dO tiles
     uint64_t *kv_full = qd_empty + 2, *kv_empty = kv_full + 1;      // the unit's K/V
-    uint64_t *sd_full = kv_empty + 1, *sd_empty = sd_full + 2;      // [2] S and dP in TMEM
-    uint64_t *ds_full = sd_empty + 2, *ds_empty = ds_full + 1;      // dS / wP in SMEM
-    uint64_t *dq_full = ds_empty + 1, *dq_empty = dq_full + 1;      // dQ in TMEM
-    uint64_t *dkv_full = dq_empty + 1, *dkv_empty = dkv_full + 1;   // dK^T / dV^T in TMEM
+    uint64_t *sd_full = kv_empty + 1, *sd_empty = sd_full + 1;      // S and dP in TMEM
+    uint64_t *ds_full = sd_empty + 1, *ds_empty = ds_full + 1;      // dS / wP in SMEM
+    uint64_t *dq_full = ds_empty + 1, *dq_empty = dq_full + 2;      // [2] dQ in TMEM
+    uint64_t *dkv_full = dq_empty + 2, *dkv_empty = dkv_full + 1;   // dK^T / dV^T in TMEM
     uint64_t *mma_done = dkv_empty + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 16);
@@ -155,11 +180,11 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
         for (int i = 0; i < kBInfo; ++i) { mbar_init(&info_full[i], 1); mbar_init(&info_empty[i], 2); }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&qd_full[i], 1); mbar_init(&qd_empty[i], 1);
-            mbar_init(&sd_full[i], 1); mbar_init(&sd_empty[i], 4);
+            mbar_init(&dq_full[i], 1); mbar_init(&dq_empty[i], 4);
         }
         mbar_init(kv_full, 1); mbar_init(kv_empty, 1);
         mbar_init(ds_full, 4); mbar_init(ds_empty, 1);
-        mbar_init(dq_full, 1); mbar_init(dq_empty, 4);
+        mbar_init(sd_full, 1); mbar_init(sd_empty, 4);
         mbar_init(dkv_full, 1); mbar_init(dkv_empty, 4);
         mbar_init(mma_done, 1);
         *abort_flag = 0;
@@ -201,6 +226,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
         // and weights one tile ahead.
         int it = 0, qc = 0, useq = 0;
         bool ok = true;
+        BP_DECL
         const int total = min(P.seg_start[P.J], P.max_items);
         const int qstep = gridDim.x;
         int guard_ok_j = -1;
@@ -251,7 +277,9 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
                 guard_ok_j = j;
             }
             // K/V of chunk c (single buffer: free once the previous unit's last dQ is done)
+            BP_BEGIN();
             if (useq >= 1 && !warp_wait(kv_empty, (useq - 1) & 1)) { ok = false; break; }
+            BP_END(1);
             if (lane == 0) {
                 mbar_arrive_expect_tx(kv_full, 2 * L::KVBYTES);
                 const int row = bg * P.L + c * kChunk;
@@ -264,9 +292,13 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
             for (int tt = t0; tt < t1 && ok; ++tt) {
                 const Pay pn = (tt + 1 < t1) ? tile_pay(dc, tt + 1) : tile_pay(dn, dn.b.y);
                 const int ii = it % kBInfo;
+                BP_BEGIN();
                 if (it >= kBInfo && !warp_wait(&info_empty[ii], ((it / kBInfo) - 1) & 1)) { ok = false; break; }
+                BP_END(2);
                 const int qs = qc & 1, qph = (qc >> 1) & 1;
+                BP_BEGIN();
                 if (qc >= 2 && !warp_wait(&qd_empty[qs], ((qc >> 1) - 1) & 1)) { ok = false; break; }
+                BP_END(3);
                 BTileInfo &ti_ = info[ii];
                 const int ntok = min(TT, e1 - (e0 + tt * TT));
                 const int t = pc.e >> 4, slot = pc.e & 15;
@@ -283,14 +315,13 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
                     mbar_arrive_expect_tx(&qd_full[qs], 2 * ntok * 2 * G * 128);
                 }
                 __syncwarp();
-                if (lane < ntok) {
-                    const int row = (b * P.L + t) * P.hq + g * G;
-#pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        tma_load_2d(sm + L::OFF_Q + qs * L::QBYTES + h * L::QHALF + lane * G * 128, &tm_q, h * 64,
-                                    row, &qd_full[qs]);
-                        tma_load_2d(sm + L::OFF_DO + qs * L::QBYTES + h * L::QHALF + lane * G * 128, &tm_do, h * 64,
-                                    row, &qd_full[qs]);
+                {  // one 3D box per 8-row group (both 64-column halves, 2 KB) for Q and for dO
+                    constexpr int GPT = G / 8;  // 8-row groups per token
+                    const int tq = __shfl_sync(0xffffffffu, t, lane / GPT);
+                    if (lane < ntok * GPT) {
+                        const int row = (b * P.L + tq) * P.hq + g * G + (lane % GPT) * 8;
+                        tma_load_3d(sm + L::OFF_Q + qs * L::QBYTES + lane * 2048, &tm_q, 0, row, 0, &qd_full[qs]);
+                        tma_load_3d(sm + L::OFF_DO + qs * L::QBYTES + lane * 2048, &tm_do, 0, row, 0, &qd_full[qs]);
                     }
                 }
                 __syncwarp();
@@ -316,6 +347,9 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
             }
             __syncwarp();
         }
+#ifdef HSA_TC_PROFILE
+        if (lane == 0) BP_DUMP(0);
+#endif
     } else if (warp == kBWarpMma) {
         // ============================================================ MMA issuer
         // Two in-order streams polled by one lane:
@@ -327,6 +361,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
         constexpr uint32_t id_dkv = idesc_bf16_f32(D, 64, true, true);
         bool ok = true;
         int ts = 0, tg = 0;
+        BP_DECL
         if (lane == 0) {
             bool s_done = false;
             uint64_t t_last = globaltimer();
@@ -336,13 +371,12 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
                     const int ii = ts % kBInfo;
                     if (mbar_test(&info_full[ii], (ts / kBInfo) & 1)) {
                         const BTileInfo &inf = info[ii];
-                        const int sb = ts & 1;
                         if (inf.type == kBItemEnd) {
                             s_done = true;
                             prog = true;
                         } else if ((!inf.unit_first || mbar_test(kv_full, inf.kvph)) &&
                                    mbar_test(&qd_full[inf.qs], inf.qph) &&
-                                   (ts < 2 || mbar_test(&sd_empty[sb], ((ts >> 1) - 1) & 1))) {
+                                   (ts < 1 || mbar_test(sd_empty, (ts - 1) & 1))) {
                             tc_fence_after();
                             const uint32_t qa = smem_u32(sm + L::OFF_Q + inf.qs * L::QBYTES);
                             const uint32_t oa = smem_u32(sm + L::OFF_DO + inf.qs * L::QBYTES);
@@ -351,16 +385,16 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
 #pragma unroll
                             for (int ks = 0; ks < D / 16; ++ks) {
                                 const int h = ks >> 2, kk = ks & 3;
-                                mma_bf16_ss(tmem + kColS + sb * 64, smem_desc_sw128(qa + h * L::QHALF + kk * 32, 16, 1024),
+                                mma_bf16_ss(tmem + kColS, smem_desc_sw128(qa + h * 1024 + kk * 32, 16, 2048),
                                             smem_desc_sw128(kb + h * L::KVHALF + kk * 32, 16, 1024), id_s, ks > 0);
                             }
 #pragma unroll
                             for (int ks = 0; ks < D / 16; ++ks) {
                                 const int h = ks >> 2, kk = ks & 3;
-                                mma_bf16_ss(tmem + kColDP + sb * 64, smem_desc_sw128(oa + h * L::QHALF + kk * 32, 16, 1024),
+                                mma_bf16_ss(tmem + kColDP, smem_desc_sw128(oa + h * 1024 + kk * 32, 16, 2048),
                                             smem_desc_sw128(vb + h * L::KVHALF + kk * 32, 16, 1024), id_s, ks > 0);
                             }
-                            mma_commit(&sd_full[sb]);
+                            mma_commit(sd_full);
                             ++ts;
                             prog = true;
                         }
@@ -369,7 +403,8 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
                 if (tg < ts) {
                     const int ii = tg % kBInfo;
                     const BTileInfo &inf = info[ii];
-                    if (mbar_test(ds_full, tg & 1) && (tg < 1 || mbar_test(dq_empty, (tg - 1) & 1)) &&
+                    const int qb = tg & 1;  // dQ buffer
+                    if (mbar_test(ds_full, tg & 1) && (tg < 2 || mbar_test(&dq_empty[qb], ((tg >> 1) - 1) & 1)) &&
                         (!inf.unit_first || inf.useq < 1 || mbar_test(dkv_empty, (inf.useq - 1) & 1))) {
                         tc_fence_after();
                         const uint32_t qa = smem_u32(sm + L::OFF_Q + inf.qs * L::QBYTES);
@@ -380,18 +415,18 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
                         // dQ = dS K  (K = the chunk's 64 keys)
 #pragma unroll
                         for (int ks = 0; ks < 4; ++ks)
-                            mma_bf16_ss(tmem + kColDQ, smem_desc_sw128(dsa + ks * 32, 16, 1024),
+                            mma_bf16_ss(tmem + kColDQ + qb * 128, smem_desc_sw128(dsa + ks * 32, 16, 1024),
                                         smem_desc_sw128(kb + ks * 2048, L::KVHALF, 1024), id_dq, ks > 0);
-                        mma_commit(dq_full);
+                        mma_commit(&dq_full[qb]);
                         // dK^T += Q^T dS,  dV^T += dO^T wP  (K = the tile's 128 rows)
                         const bool first = inf.unit_first != 0;
 #pragma unroll
                         for (int ks = 0; ks < 8; ++ks)
-                            mma_bf16_ss(tmem + kColDK, smem_desc_sw128(qa + ks * 2048, L::QHALF, 1024),
+                            mma_bf16_ss(tmem + kColDK, smem_desc_sw128(qa + ks * 4096, 1024, 2048),
                                         smem_desc_sw128(dsa + ks * 2048, L::PB, 1024), id_dkv, ks > 0 || !first);
 #pragma unroll
                         for (int ks = 0; ks < 8; ++ks)
-                            mma_bf16_ss(tmem + kColDV, smem_desc_sw128(oa + ks * 2048, L::QHALF, 1024),
+                            mma_bf16_ss(tmem + kColDV, smem_desc_sw128(oa + ks * 4096, 1024, 2048),
                                         smem_desc_sw128(wpa + ks * 2048, L::PB, 1024), id_dkv, ks > 0 || !first);
                         mma_commit(ds_empty);
                         mma_commit(&qd_empty[inf.qs]);
@@ -408,6 +443,9 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
                 }
                 if (prog) t_last = globaltimer();
                 else if (*abort_flag || globaltimer() - t_last > kBWaitNs) { ok = false; break; }
+#ifdef HSA_TC_PROFILE
+                if (!prog) ++bp_acc[1];
+#endif
             }
             if (!ok) {
                 *abort_flag = 1;
@@ -416,6 +454,9 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
             // drain: every MMA issued by this warp has finished before TMEM is released
             mma_commit(mma_done);
             mbar_wait(mma_done, 0, kBWaitNs);
+#ifdef HSA_TC_PROFILE
+            BP_DUMP(16);
+#endif
         }
         __syncwarp();
     } else if (warp < kBWarpEpi) {
@@ -428,6 +469,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
         const float sl2 = scale * L2E;
         int it = 0, wcnt = 0;
         bool ok = true;
+        BP_DECL
         auto wg_sync = [&]() { asm volatile("bar.sync 1, 128;" ::: "memory"); };
         auto wg_vote = [&](int v) -> bool {  // thread 0 decides, the whole group follows
             const int slot = (wcnt++) & 1;
@@ -442,10 +484,11 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
         };
         while (ok) {
             const int ii = it % kBInfo;
+            BP_BEGIN();
             if (!wg_wait(&info_full[ii], (it / kBInfo) & 1)) { ok = false; break; }
+            BP_END(1);
             const BTileInfo &inf = info[ii];
             if (inf.type == kBItemEnd) break;
-            const int sb = it & 1;
             const int ti = r / G, hh = r % G;
             const bool valid = ti < inf.ntok;
             const int t = valid ? inf.tok[ti] : 0, slot = valid ? inf.slot[ti] : 0;
@@ -453,17 +496,20 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
             // the row's log-normaliser from the forward, loaded before the scores are waited for
             const float lrow =
                 valid ? lse[(((int64_t)inf.b * P.L + t) * P.hq + inf.g * G + hh) * P.K + slot] : 0.f;
-            if (!wg_wait(&sd_full[sb], (it >> 1) & 1)) { ok = false; break; }
+            BP_BEGIN();
+            if (!wg_wait(sd_full, it & 1)) { ok = false; break; }
+            BP_END(2);
+            BP_BEGIN();
             tc_fence_after();
             float x0[32], x1[32], d0[32], d1[32];
-            tmem_ld32(lane_base + kColS + sb * 64, x0);
-            tmem_ld32(lane_base + kColS + sb * 64 + 32, x1);
-            tmem_ld32(lane_base + kColDP + sb * 64, d0);
-            tmem_ld32(lane_base + kColDP + sb * 64 + 32, d1);
+            tmem_ld32(lane_base + kColS, x0);
+            tmem_ld32(lane_base + kColS + 32, x1);
+            tmem_ld32(lane_base + kColDP, d0);
+            tmem_ld32(lane_base + kColDP + 32, d1);
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sd_empty[sb]);
+            if (lane == 0) mbar_arrive(sd_empty);
             float delta = 0.f;
             if (valid) {
                 // p = exp(x - lse), x = S / sqrt(d);  Delta = sum_i p_i dP_i
@@ -495,8 +541,11 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
 #pragma unroll
             for (int off = 1; off < G; off <<= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, off);
             if (valid && hh == 0) dw[(((int64_t)inf.b * P.L + t) * P.hkv + inf.g) * P.K + slot] = dsum;
+            BP_END(3);
             // the dS / wP buffer is free once the previous tile's gradient MMAs have read it
+            BP_BEGIN();
             if (it >= 1 && !wg_wait(ds_empty, (it - 1) & 1)) { ok = false; break; }
+            BP_END(4);
             uint8_t *dsrow = sm + L::OFF_DS + r * 128;
             uint8_t *wprow = sm + L::OFF_WP + r * 128;
             if (valid) {
@@ -519,6 +568,9 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
             ++it;
         }
         if (!ok) { *abort_flag = 1; if (tid == 0) report(ds, HSA_ERR_TIMEOUT, kKBwdTc, 5, it); }
+#ifdef HSA_TC_PROFILE
+        if (tid == 0) BP_DUMP(32);
+#endif
     } else if (warp < kBWarpConv) {
         // ============================================================ dQ epilogue + dK/dV flush
         // dQ rows (times 1/sqrt(d)) are transposed through a 4 KB per-warp
@@ -534,6 +586,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
         float4 *xs = reinterpret_cast<float4 *>(sm + L::OFF_X + wq * 4096);  // [32 rows][8 chunks]
         int it = 0, ecnt = 0, ecnt_j = -1, vcnt = 0;
         bool ok = true;
+        BP_DECL
         auto eg_sync = [&]() { asm volatile("bar.sync 2, 128;" ::: "memory"); };
         auto eg_vote = [&](int v) -> bool {
             const int slot = (vcnt++) & 1;
@@ -570,7 +623,11 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
                 if (ecnt > 0) flush();
                 ecnt_j = inf.j;
             }
-            if (!eg_wait(dq_full, it & 1)) { ok = false; break; }
+            BP_BEGIN();
+            const int qb = it & 1;  // dQ buffer of this tile
+            if (!eg_wait(&dq_full[qb], (it >> 1) & 1)) { ok = false; break; }
+            BP_END(1);
+            BP_BEGIN();
             tc_fence_after();
             const int s = inf.j % kRing;
             const int ws = (inf.j % P.nW) * P.W;
@@ -586,7 +643,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
 #pragma unroll
             for (int q = 0; q < D / 32; ++q) {
                 float v[32];
-                tmem_ld32(lane_base + kColDQ + q * 32, v);
+                tmem_ld32(lane_base + kColDQ + qb * 128 + q * 32, v);
                 tmem_wait_ld();
 #pragma unroll
                 for (int ch = 0; ch < 8; ++ch)
@@ -603,9 +660,13 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(dq_empty);
+            if (lane == 0) mbar_arrive(&dq_empty[qb]);
+            BP_END(2);
             if (inf.unit_last) {
+                BP_BEGIN();
                 if (!eg_wait(dkv_full, inf.useq & 1)) { ok = false; break; }
+                BP_END(3);
+                BP_BEGIN();
                 tc_fence_after();
                 const int64_t krow = ((int64_t)(inf.b * P.hkv + inf.g) * P.L + (int64_t)inf.c * kChunk) * D + r;
 #pragma unroll
@@ -623,6 +684,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(dkv_empty);
+                BP_END(4);
             }
             eg_sync();  // the whole group is done with this tile's info entry
             if (tid == 0) mbar_arrive(&info_empty[ii]);
@@ -631,6 +693,9 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
         }
         if (ok && ecnt > 0) flush();
         if (!ok) { *abort_flag = 1; if (tid == 0) report(ds, HSA_ERR_TIMEOUT, kKBwdTc, 6, it); }
+#ifdef HSA_TC_PROFILE
+        if (tid == 0) BP_DUMP(48);
+#endif
     } else if (warp < kBWarpProd) {
         // ============================================================ convert group
         // Converts each window's fp32 dq slot into dq (bf16) and re-zeroes it,
@@ -805,12 +870,26 @@ bool b_map(CUtensorMap *m, const void *base, uint64_t cols, uint64_t rows, uint3
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// token rows of d = 128 as a 3D view (64 columns, rows, 2 halves of 128 bytes); box =
+// 8 rows x both halves, stored half after half (2 KB per 8-row group, 128B swizzle)
+bool b_map_q3(CUtensorMap *m, const void *base, uint64_t rows) {
+    BEncodeFn enc = b_encode();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {64, rows, 2};
+    cuuint64_t strides[2] = {256, 128};
+    cuuint32_t box[3] = {64, 8, 2};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int G>
 cudaError_t launch_btc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv, const void *q, const void *k,
                        const void *v, const void *dO, const float *lse, float *dw, float *acc, void *dq,
                        float *dk_acc, float *dv_acc, DevStatus *ds, cudaStream_t st) {
     CUtensorMap mq, mo, mk, mv;
-    if (!b_map(&mq, q, kBD, (uint64_t)sh.B * sh.L * sh.hq, G) || !b_map(&mo, dO, kBD, (uint64_t)sh.B * sh.L * sh.hq, G) ||
+    if (!b_map_q3(&mq, q, (uint64_t)sh.B * sh.L * sh.hq) || !b_map_q3(&mo, dO, (uint64_t)sh.B * sh.L * sh.hq) ||
         !b_map(&mk, k, kBD, (uint64_t)sh.B * sh.hkv * sh.L, 64) || !b_map(&mv, v, kBD, (uint64_t)sh.B * sh.hkv * sh.L, 64))
         return cudaErrorInvalidValue;
     const size_t smem = BSmem::ALLOC;

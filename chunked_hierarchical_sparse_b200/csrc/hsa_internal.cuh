@@ -149,10 +149,13 @@ constexpr int kCombTokens = 16;    // tokens per combine item
 // window reduce their weighted outputs into (compile-time tunables; the ring
 // stays resident in L2 next to the K/V and query working set).
 #ifndef HSA_ACC_RING
-#define HSA_ACC_RING 3
+#define HSA_ACC_RING 2
 #endif
 #ifndef HSA_ACC_SLOT_MB
-#define HSA_ACC_SLOT_MB 16
+#define HSA_ACC_SLOT_MB 32
+#endif
+#ifndef HSA_MAX_WINDOW
+#define HSA_MAX_WINDOW 16384
 #endif
 constexpr int kRing = HSA_ACC_RING;
 constexpr size_t kAccSlotBudget = size_t(HSA_ACC_SLOT_MB) << 20;
@@ -184,7 +187,7 @@ inline int attend_window(int G, int d, int esize) {
     const int64_t per_tok = (int64_t)G * d * esize;
     int64_t w = (int64_t)(kAccSlotBudget / per_tok) / kInvTokBlock * kInvTokBlock;
     if (w < kInvTokBlock) w = kInvTokBlock;
-    if (w > 8192) w = 8192;
+    if (w > HSA_MAX_WINDOW) w = HSA_MAX_WINDOW;
     return (int)w;
 }
 

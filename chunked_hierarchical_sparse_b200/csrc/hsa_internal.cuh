@@ -138,7 +138,12 @@ cudaError_t launch_bwd_phase2(const Shape &sh, const void *q, const void *k, con
                               const void *dO, const float *lse, const float *w, void *dk, void *dv,
                               const BwdWs &ws, DevStatus *ds, cudaStream_t st);
 
-constexpr int kInvTokBlock = 256;  // tokens per histogram block of the inversion
+#ifndef HSA_INV_BLOCK
+#define HSA_INV_BLOCK 128
+#endif
+// tokens per histogram block of the inversion: the scatter walks a block's tokens
+// in order (one warp); the histogram holds ceil(L / block) x n_c counts per (b, g)
+constexpr int kInvTokBlock = HSA_INV_BLOCK;
 constexpr int kBwdSeg = 32;        // list entries per phase-2 block
 
 // ---------------------------------------------------------------- chunk-major forward plan

@@ -58,6 +58,14 @@ __device__ unsigned long long *g_tc_prof = nullptr;
 
 namespace {
 
+#ifndef HSA_EPI_UNROLL
+#define HSA_EPI_UNROLL 1
+#endif
+#ifndef HSA_CONV_BATCH
+#define HSA_CONV_BATCH 8
+#endif
+constexpr int kEpiUnroll = HSA_EPI_UNROLL;  // unrolling of the epilogue's column loops (1 keeps its code small)
+
 // 16 warps:
 //   warps 0-3 softmax, warps 4-7 and 8-11 two epilogue groups (weighted O ->
 //   fp32 reductions into the window accumulators; group e takes the tiles whose
@@ -674,9 +682,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 dst[m] = acc + ((int64_t)(s * P.W + inf.tok[i] - ws) * G + tr % G) * D + (lane & 7) * 8;
             }
             uint4 *xs4 = reinterpret_cast<uint4 *>(xs);
-#pragma unroll
+#pragma unroll kEpiUnroll
             for (int q = 0; q < D / 64; ++q) {  // 64 columns = one 128-byte fp16 line per row
-#pragma unroll
+#pragma unroll kEpiUnroll
                 for (int hv = 0; hv < 2; ++hv) {  // 32 columns at a time: 4 chunks of 8 halves
                     float v[32];
                     tmem_ld32(lane_base + 128 + sb * 128 + q * 64 + hv * 32, v);
@@ -760,7 +768,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 // fp16 accumulators of tokens [ta, tb): G*D contiguous values per token, and
                 // o of (token, group g): G*D contiguous bf16.  A unit is 8 values -> 16 bytes of o.
                 constexpr int UPT = G * D / 8;  // units per token
-                constexpr int kBatch = 8;       // units in flight per thread
+                constexpr int kBatch = HSA_CONV_BATCH;  // units in flight per thread
                 uint4 *A = reinterpret_cast<uint4 *>(acc + (int64_t)(s * P.W + (ta - ws)) * G * D);
                 const int nunits = (tb - ta) * UPT;
                 for (int u0 = 0; u0 < nunits; u0 += kConvThreads * kBatch) {

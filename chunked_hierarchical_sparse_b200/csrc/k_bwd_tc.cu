@@ -62,6 +62,12 @@ namespace {
 #endif
 constexpr uint64_t kBWaitNs = HSA_WAIT_NS;  // bound on any single wait (default 2 s)
 
+#ifndef HSA_BEPI_UNROLL
+#define HSA_BEPI_UNROLL 1
+#endif
+// unrolling of the epilogue's column loops: rolled, the roles' hot code fits the instruction cache
+constexpr int kBEpiUnroll = HSA_BEPI_UNROLL;
+
 constexpr int kBThreads = 384;
 constexpr int kBWarpEpi = 4, kBWarpConv = 8, kBWarpProd = 10, kBWarpMma = 11;
 constexpr int kBConvThreads = 64;
@@ -640,7 +646,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
                 dok[m] = i < inf.ntok;
                 dst[m] = acc + ((int64_t)(s * P.W + inf.tok[i] - ws) * G + tr % G) * D + (lane & 7) * 4;
             }
-#pragma unroll
+#pragma unroll kBEpiUnroll
             for (int q = 0; q < D / 32; ++q) {
                 float v[32];
                 tmem_ld32(lane_base + kColDQ + qb * 128 + q * 32, v);
@@ -669,7 +675,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
                 BP_BEGIN();
                 tc_fence_after();
                 const int64_t krow = ((int64_t)(inf.b * P.hkv + inf.g) * P.L + (int64_t)inf.c * kChunk) * D + r;
-#pragma unroll
+#pragma unroll kBEpiUnroll
                 for (int hk = 0; hk < 2; ++hk) {
                     float v[32];
                     tmem_ld32(lane_base + kColDK + hk * 32, v);

@@ -111,7 +111,7 @@ struct BwdAll {
     BwdWs b;
     bool tc;          // chunk-major tensor-core path
     AttendPlan plan;
-    float *acc;       // fp32 dq accumulator ring (tensor-core path)
+    __half *acc;      // fp16 dq accumulator ring, scaled (tensor-core path)
     float *dw;        // [B,L,h_kv,K] gradients of the chunk weights (tensor-core path)
 };
 
@@ -130,7 +130,7 @@ static BwdAll carve_bwd(const Shape &sh, void *ws, size_t *bytes) {
     if (r.tc) {
         r.dw = c.take<float>((size_t)sh.B * sh.L * sh.hkv * sh.K);
         carve_plan(c, sh, r.plan, kBwdUnitTiles, kBwdAccBytes);
-        r.acc = c.take<float>(attend_acc_elems(r.plan.W, sh.G, sh.d));
+        r.acc = c.take<__half>(attend_acc_elems(r.plan.W, sh.G, sh.d));
     }
     if (bytes) *bytes = c.off;
     return r;
@@ -341,9 +341,17 @@ hsa_status_t hsa_bwd(const hsa_shape_t *shape, const void *q, const void *k, con
         if (e == cudaSuccess) e = cudaMemsetAsync(P.counters, 0, sizeof(int32_t) * plan_counter_count(P.J), st);
         if (e == cudaSuccess)
             e = cudaMemsetAsync(all.acc, 0,
-                                sizeof(float) * std::min<size_t>(attend_acc_elems(P.W, sh.G, sh.d),
+                                sizeof(__half) * std::min<size_t>(attend_acc_elems(P.W, sh.G, sh.d),
                                                                  (size_t)P.J * P.W * sh.G * sh.d),
                                 st);
+        if (e == cudaSuccess)  // magnitude bounds for the dq accumulators' power-of-two scale
+            e = timed(HSA_K_PLAN, 3, st, [&] {
+                int32_t *mb = P.counters + 3 * P.J + 1;
+                cudaError_t e2 = launch_rownorm_max(v, (int64_t)sh.B * sh.hkv * sh.L, sh.d, mb, st);
+                if (e2 == cudaSuccess) e2 = launch_rownorm_max(dO, (int64_t)sh.B * sh.L * sh.hq, sh.d, mb + 1, st);
+                if (e2 == cudaSuccess) e2 = launch_vmax(sh, k, mb + 2, st);
+                return e2;
+            });
         if (e == cudaSuccess)
             e = timed(HSA_K_BWD_TC, 1, st, [&] {
                 return launch_bwd_tc(sh, P, b, q, k, v, dO, lse, all.dw, all.acc, dq, b.dk_acc, b.dv_acc, ds, st);

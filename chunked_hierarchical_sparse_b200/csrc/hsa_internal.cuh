@@ -178,8 +178,9 @@ struct AttendPlan {
     int max_items;         // capacity of `items`
 };
 
-// tiles_done[J], comb_done[J], comb_head[J], then one word: the bits of max|v| (forward)
-inline size_t plan_counter_count(int J) { return 3 * (size_t)J + 2; }
+// tiles_done[J], comb_done[J], comb_head[J], then three words of magnitude bounds as
+// float bits: forward max|v|; backward max row norm of v, of dO, and max|k|
+inline size_t plan_counter_count(int J) { return 3 * (size_t)J + 4; }
 
 // queue item descriptor (two int4): {type, j, c, e0} {e1, t0, t1, 0}
 //   type 0: work unit, chunk c, entries [e0, e1) of its bucket, tiles [t0, t1)
@@ -199,10 +200,10 @@ inline int attend_window(int G, int d, int esize) {
 // elements of the accumulator ring of one call
 inline size_t attend_acc_elems(int W, int G, int d) { return (size_t)kRing * W * G * d; }
 
-// The forward's ring holds fp16 sums scaled by 2^-e, 2^e >= max|v| (every
-// partial sum of w_k * softmax-average of v is bounded by max|v|); the
-// backward's dq ring holds fp32.
-constexpr int kFwdAccBytes = 2, kBwdAccBytes = 4;
+// Both rings hold fp16 sums scaled by a power of two 2^-e at or above a bound of
+// every partial sum: the forward's by max|v| (a partial sum of w_k * softmax-
+// averages of v), the backward's dq by 2 max||dO_row|| max||v_row|| max|k| / sqrt(d).
+constexpr int kFwdAccBytes = 2, kBwdAccBytes = 2;
 
 bool select_tc_supported(const Shape &sh);
 // Chunk selection with tensor-core scores; hi/lo: [B,hkv,nc,d] bf16 scratch.
@@ -222,8 +223,10 @@ cudaError_t launch_vmax(const Shape &sh, const void *v, int32_t *bits, cudaStrea
 // accumulators of `inv` (dk_acc / dv_acc).  inv.entw must hold the entries' weights.
 bool bwd_tc_supported(const Shape &sh);
 cudaError_t launch_bwd_tc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv, const void *q, const void *k,
-                          const void *v, const void *dO, const float *lse, float *dw, float *acc, void *dq,
+                          const void *v, const void *dO, const float *lse, float *dw, __half *acc, void *dq,
                           float *dk_acc, float *dv_acc, DevStatus *ds, cudaStream_t st);
+// max L2 norm over the rows (of d bf16 values) of x, as float bits max-ed into *bits
+cudaError_t launch_rownorm_max(const void *x, int64_t rows, int d, int32_t *bits, cudaStream_t st);
 // Stick-breaking backward from dw: dq_slc, and dkbar (added into, fp32).
 cudaError_t launch_bwd_select(const Shape &sh, const void *q_slc, const int32_t *idx, const float *w,
                               const float *dw, const float *kbar, void *dq_slc, float *dkbar, cudaStream_t st);

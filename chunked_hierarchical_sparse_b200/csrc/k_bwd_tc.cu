@@ -158,7 +158,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
     const __grid_constant__ AttendPlan P, const int32_t *__restrict__ entries, const float *__restrict__ entw,
-    const float *__restrict__ lse, float *__restrict__ dw, float *__restrict__ acc, __nv_bfloat16 *__restrict__ dq,
+    const float *__restrict__ lse, float *__restrict__ dw, __half *__restrict__ acc, __nv_bfloat16 *__restrict__ dq,
     float *__restrict__ dk_acc, float *__restrict__ dv_acc, DevStatus *ds) {
     using L = BSmem;
     constexpr int D = kBD;
@@ -218,6 +218,24 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
     int32_t *comb_done = P.counters + P.J;
     int32_t *comb_head = P.counters + 2 * P.J;
     const float scale = 1.0f / sqrtf((float)D);
+    // power-of-two scale of the fp16 dq accumulators: 2^e >= 2 max||v_row|| max||dO_row|| max|k| / sqrt(d),
+    // a bound of every partial dq sum (|dS_i| <= 2 w p_i ||dO|| max||v||, sum_i p_i < 1, sum_k w_k <= 1)
+    float acc_scale, acc_inv;
+    {
+        const float nv = __int_as_float(P.counters[3 * P.J + 1]);
+        const float ndo = __int_as_float(P.counters[3 * P.J + 2]);
+        const float mk = __int_as_float(P.counters[3 * P.J + 3]);
+        const float bound = 2.f * nv * ndo * mk * scale;
+        int ev = 0;
+        if (bound > 0.f) {
+            const uint32_t vb = __float_as_uint(bound);
+            ev = (int)((vb >> 23) & 0xff) - 127;
+            if (vb & 0x7fffffu) ev += 1;
+        }
+        ev = max(-100, min(ev, 120));
+        acc_scale = __int_as_float((ev + 127) << 23);
+        acc_inv = __int_as_float((127 - ev) << 23);
+    }
 
     auto warp_wait = [&](uint64_t *b, uint32_t par) -> bool {  // lane 0 waits, the warp gets the verdict
         int r = 1;
@@ -637,30 +655,41 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
             tc_fence_after();
             const int s = inf.j % kRing;
             const int ws = (inf.j % P.nW) * P.W;
-            float *dst[8];
+            // this lane reduces, for m = 0..7, the 16-byte chunk lane % 8 (8 halves) of warp row 4m + lane / 8
+            const float cf = scale * acc_inv;
+            __half *dst[8];
             bool dok[8];
 #pragma unroll
             for (int m = 0; m < 8; ++m) {
                 const int tr = wq * 32 + 4 * m + (lane >> 3);
                 const int i = tr / G;
                 dok[m] = i < inf.ntok;
-                dst[m] = acc + ((int64_t)(s * P.W + inf.tok[i] - ws) * G + tr % G) * D + (lane & 7) * 4;
+                dst[m] = acc + ((int64_t)(s * P.W + inf.tok[i] - ws) * G + tr % G) * D + (lane & 7) * 8;
             }
+            uint4 *xs4 = reinterpret_cast<uint4 *>(xs);
 #pragma unroll kBEpiUnroll
-            for (int q = 0; q < D / 32; ++q) {
-                float v[32];
-                tmem_ld32(lane_base + kColDQ + qb * 128 + q * 32, v);
-                tmem_wait_ld();
+            for (int q = 0; q < D / 64; ++q) {  // 64 columns = one 128-byte fp16 line per row
+#pragma unroll kBEpiUnroll
+                for (int hv = 0; hv < 2; ++hv) {  // 32 columns at a time: 4 chunks of 8 halves
+                    float v[32];
+                    tmem_ld32(lane_base + kColDQ + qb * 128 + q * 64 + hv * 32, v);
+                    tmem_wait_ld();
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch)
-                    xs[lane * 8 + (ch ^ (lane & 7))] = make_float4(v[4 * ch] * scale, v[4 * ch + 1] * scale,
-                                                                   v[4 * ch + 2] * scale, v[4 * ch + 3] * scale);
+                    for (int c4 = 0; c4 < 4; ++c4) {
+                        const int ch = hv * 4 + c4;
+                        __half2 h[4];
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            h[e] = __floats2half2_rn(v[c4 * 8 + 2 * e] * cf, v[c4 * 8 + 2 * e + 1] * cf);
+                        xs4[lane * 8 + (ch ^ (lane & 7))] = *reinterpret_cast<uint4 *>(h);
+                    }
+                }
                 __syncwarp();
 #pragma unroll
                 for (int m = 0; m < 8; ++m) {
                     const int row = 4 * m + (lane >> 3);
-                    const float4 f = xs[row * 8 + ((lane & 7) ^ (row & 7))];
-                    if (dok[m]) red_add_v4_f32(dst[m] + q * 32, f);
+                    const uint4 f = xs4[row * 8 + ((lane & 7) ^ (row & 7))];
+                    if (dok[m]) red_add_v4_f16x2(dst[m] + q * 64, f);
                 }
                 __syncwarp();
             }
@@ -733,27 +762,33 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
                 const int item = cg_bcast(tid == 0 ? atomicAdd(&comb_head[jc], 1) : 0);
                 if (item >= ncomb) break;
                 const int ta = ws + item * kCombTokens, tb = min(we, ta + kCombTokens);
-                constexpr int UPT = G * D / 8;  // 8-float units per token
+                constexpr int UPT = G * D / 8;  // 8-value units per token
                 constexpr int kBatch = 8;
-                float4 *A = reinterpret_cast<float4 *>(acc + (int64_t)(s * P.W + (ta - ws)) * G * D);
+                uint4 *A = reinterpret_cast<uint4 *>(acc + (int64_t)(s * P.W + (ta - ws)) * G * D);
                 const int nunits = (tb - ta) * UPT;
                 for (int u0 = 0; u0 < nunits; u0 += kBConvThreads * kBatch) {
-                    float4 lo[kBatch], hi[kBatch];
+                    uint4 raw[kBatch];
 #pragma unroll
                     for (int k = 0; k < kBatch; ++k) {
                         const int u = u0 + k * kBConvThreads + tid;
-                        if (u < nunits) { lo[k] = __ldcg(A + 2 * u); hi[k] = __ldcg(A + 2 * u + 1); }
+                        if (u < nunits) raw[k] = __ldcg(A + u);
                     }
 #pragma unroll
                     for (int k = 0; k < kBatch; ++k) {
                         const int u = u0 + k * kBConvThreads + tid;
                         if (u < nunits) {
                             const int t = ta + u / UPT, e = u % UPT;
-                            const float f[8] = {lo[k].x, lo[k].y, lo[k].z, lo[k].w, hi[k].x, hi[k].y, hi[k].z, hi[k].w};
+                            const __half2 *h2 = reinterpret_cast<const __half2 *>(&raw[k]);
+                            float f[8];
+#pragma unroll
+                            for (int x = 0; x < 4; ++x) {
+                                const float2 g2 = __half22float2(h2[x]);
+                                f[2 * x] = g2.x * acc_scale;
+                                f[2 * x + 1] = g2.y * acc_scale;
+                            }
                             __stcs(reinterpret_cast<uint4 *>(dq + (((int64_t)b * P.L + t) * P.hq + g * G) * D + e * 8),
                                    pack8(f));
-                            A[2 * u] = make_float4(0.f, 0.f, 0.f, 0.f);
-                            A[2 * u + 1] = make_float4(0.f, 0.f, 0.f, 0.f);
+                            A[u] = make_uint4(0, 0, 0, 0);
                         }
                     }
                 }
@@ -847,6 +882,50 @@ __global__ void __launch_bounds__(256) bwd_select_kernel(const __nv_bfloat16 *__
     *reinterpret_cast<uint2 *>(dq_slc + gw * D + lane * 4) = pk;
 }
 
+// ------------------------------------------------------------------ magnitude bound
+// max over rows of the L2 norm of a row of d = 128 bf16 values, as float bits max-ed into
+// *bits.  A row is 16 lanes x 16 bytes; every thread keeps 4 rows' loads in flight.
+__global__ void __launch_bounds__(256) rownorm_max_kernel(const __nv_bfloat16 *__restrict__ x, int64_t rows,
+                                                          int32_t *__restrict__ bits) {
+    constexpr int kU = 4;
+    const int64_t nvec = rows * 16;  // 16-byte vectors
+    const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+    float m = 0.f;
+    for (int64_t v0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v0 - (int64_t)(threadIdx.x & 31) < nvec;
+         v0 += kU * stride) {
+        uint4 raw[kU];
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const int64_t vi = v0 + u * stride;
+            raw[u] = vi < nvec ? __ldcs(reinterpret_cast<const uint4 *>(x) + vi) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int u = 0; u < kU; ++u) {
+            const __nv_bfloat162 *h = reinterpret_cast<const __nv_bfloat162 *>(&raw[u]);
+            float ss = 0.f;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(h[e]);
+                ss += f.x * f.x + f.y * f.y;
+            }
+#pragma unroll
+            for (int off = 8; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);  // 16-lane row
+            m = fmaxf(m, sqrtf(ss));
+        }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if ((threadIdx.x & 31) == 0) atomicMax(bits, __float_as_int(m));
+}
+
+cudaError_t launch_rownorm_max(const void *x, int64_t rows, int d, int32_t *bits, cudaStream_t st) {
+    if (rows == 0) return cudaSuccess;
+    if (d != kBD) return cudaErrorInvalidValue;
+    const int blocks = (int)std::min<int64_t>(ceil_div(rows * 16, 256 * 4), 148 * 8);
+    rownorm_max_kernel<<<blocks, 256, 0, st>>>((const __nv_bfloat16 *)x, rows, bits);
+    return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ host side
 namespace {
 typedef CUresult (*BEncodeFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -892,7 +971,7 @@ bool b_map_q3(CUtensorMap *m, const void *base, uint64_t rows) {
 
 template <int G>
 cudaError_t launch_btc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv, const void *q, const void *k,
-                       const void *v, const void *dO, const float *lse, float *dw, float *acc, void *dq,
+                       const void *v, const void *dO, const float *lse, float *dw, __half *acc, void *dq,
                        float *dk_acc, float *dv_acc, DevStatus *ds, cudaStream_t st) {
     CUtensorMap mq, mo, mk, mv;
     if (!b_map_q3(&mq, q, (uint64_t)sh.B * sh.L * sh.hq) || !b_map_q3(&mo, dO, (uint64_t)sh.B * sh.L * sh.hq) ||
@@ -915,7 +994,7 @@ bool bwd_tc_supported(const Shape &sh) {
 }
 
 cudaError_t launch_bwd_tc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv, const void *q, const void *k,
-                          const void *v, const void *dO, const float *lse, float *dw, float *acc, void *dq,
+                          const void *v, const void *dO, const float *lse, float *dw, __half *acc, void *dq,
                           float *dk_acc, float *dv_acc, DevStatus *ds, cudaStream_t st) {
     if (sh.G == 8) return launch_btc<8>(sh, plan, inv, q, k, v, dO, lse, dw, acc, dq, dk_acc, dv_acc, ds, st);
     if (sh.G == 16) return launch_btc<16>(sh, plan, inv, q, k, v, dO, lse, dw, acc, dq, dk_acc, dv_acc, ds, st);

@@ -256,6 +256,22 @@ def test_bwd_tensor_core_path_full(wl):
         assert_out(f64(g), r, "bf16", name, grad=True)
 
 
+@pytest.mark.parametrize("factor", [2.0 ** 12, 2.0 ** -12], ids=["dO-x4096", "dO-x1/4096"])
+def test_bwd_tensor_core_grad_scale(factor):
+    """The tensor-core backward sums dq in fp16 scaled by a power of two at or above a
+    bound computed from max row norms of dO and v and max|k|.  Every gradient is
+    linear in dO and scaling dO by a power of two is exact, so grads / factor must
+    match the unscaled oracle at the same bar."""
+    wl = BWD_TC[0]
+    x, kbar, sel = gap_ruled(wl)
+    ref = oracle.bwd(x["q"], x["k"], x["v"], x["q_slc"], kbar, x["dO"], wl.S, wl.K)
+    xs = dict(x)
+    xs["dO"] = x["dO"] * factor
+    got = run_bwd(wl, xs)
+    for name, g, r in zip(("dq", "dk", "dv", "dq_slc"), got, ref[:4]):
+        assert_out(f64(g) / factor, r, "bf16", name, grad=True)
+
+
 def test_bwd_train_workload_sampled():
     """Full-size training workload: dq / dq_slc on sampled tokens, dk / dv on
     sampled chunks (the oracle walks every token that selected them)."""

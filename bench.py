@@ -325,29 +325,26 @@ def main():
     args = ap.parse_args()
     assert args.warmup >= 3 or args.impl == "reference", "at least 3 warm-up steps"
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from chunked_hierarchical_sparse_b200 import dist_util
+    world, rank, local = dist_util.env_ranks()
 
     if args.impl == "reference":
         run_reference(args, rank, world)
         return
 
     import torch
-    import torch.distributed as dist
     import chunked_hierarchical_sparse_b200 as hsa
     from chunked_hierarchical_sparse_b200 import synth
 
     if world > 1:
         torch.cuda.set_device(local)
-        from datetime import timedelta
-        dist.init_process_group("nccl", timeout=timedelta(seconds=120))
+        dist_util.init(world, "nccl")
     dev = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(dev)
     hsa.load_library()
 
     base = synth.WORKLOADS[args.workload]
-    wl = base.scaled(seed=base.seed + 100 * rank)  # one independent sequence per rank
+    wl = base.scaled(seed=dist_util.rank_seed(base.seed, rank))  # one independent sequence per rank
     x = synth.make_inputs(wl)
     q, k, v, qs = (to_dev(x[n], dev) for n in ("q", "k", "v", "q_slc"))
     o = torch.empty_like(q)
@@ -364,8 +361,7 @@ def main():
     torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
-    if world > 1:
-        dist.barrier()
+    dist_util.barrier(world)
     torch.cuda.synchronize()
     hsa.hsa_timing_enable(True)
     with ClockSampler(dev.index) as clocks:
@@ -375,20 +371,14 @@ def main():
             fwd()
             b.record()
         torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
+    dist_util.barrier(world)
     torch.cuda.synchronize()
     step_ms = [a.elapsed_time(b) for a, b in ev]
     kern = {name: hsa.hsa_timing_read(name) for name in hsa.KERNELS}
     hsa.hsa_timing_enable(False)
     assert hsa.hsa_device_status(ws) == 0, "device status set during the timed region"
-    dev_ms = sum(step_ms)
-    t = torch.tensor([dev_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
-    tokens = world * wl.B * wl.L * args.steps
-    value = tokens / (max_ms / 1e3)
+    max_ms = dist_util.max_over_ranks(sum(step_ms), world, dev)
+    value = dist_util.job_throughput(wl.B * wl.L, world, args.steps, max_ms)
 
     # dominant kernel: the chunk attention (whichever path ran)
     att_name = "attend_tc" if kern["attend_tc"][1] > 0 else "attend_simt"
@@ -441,11 +431,8 @@ def main():
         if i:
             e2e.append(a.elapsed_time(b))
     h2d = sum(t_.numel() * t_.element_size() for t_ in hq.values())
-    e2e_ms = float(np.median(e2e))
-    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    line["e2e"] = {"value": world * wl.B * wl.L / (float(te.item()) / 1e3), "unit": "tokens/s",
+    e2e_max = dist_util.max_over_ranks(float(np.median(e2e)), world, dev)
+    line["e2e"] = {"value": dist_util.job_throughput(wl.B * wl.L, world, 1, e2e_max), "unit": "tokens/s",
                    "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(ho.numel() * ho.element_size())}
     del hq, ho
 
@@ -454,9 +441,7 @@ def main():
         line["train"] = bench_train(hsa, dev)
     if rank == 0 and world == 1 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(wl, x, args.cpu_budget_s)
-    if world > 1:
-        dist.barrier()
-        dist.destroy_process_group()
+    dist_util.finish(world)
     if rank == 0:
         print(json.dumps(line), flush=True)
 

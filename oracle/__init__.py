@@ -40,9 +40,10 @@ def lib():
         L.or_pool.argtypes = [i, i, i, i, i, p, p]
         L.or_select.argtypes = [i, i, i, i, i, i, p, p, p, i64, p, p, p, p]
         L.or_fwd.argtypes = [i, i, i, i, i, i, i, p, p, p, p, p, p, i64, p, p, p, p]
+        L.or_attend.argtypes = [i, i, i, i, i, i, i, p, p, p, p, p, p, i64, p, p]
         L.or_decode.argtypes = [i, i, i, i, i, i, i, p, p, p, p, p, p, p, p, p]
         L.or_bwd.argtypes = [i, i, i, i, i, i, i, p, p, p, p, p, p, p, p, p, p, p, p]
-        for f in (L.or_pool, L.or_select, L.or_fwd, L.or_decode, L.or_bwd):
+        for f in (L.or_pool, L.or_select, L.or_fwd, L.or_attend, L.or_decode, L.or_bwd):
             f.restype = ctypes.c_int
         L.or_num_threads.restype = ctypes.c_int
         _lib = L
@@ -112,6 +113,23 @@ def fwd(q, k, v, q_slc, kbar, S: int, K: int, rows=None):
     _check(lib().or_fwd(B, L, h_q, h_kv, d, S, K, _ptr(q), _ptr(k), _ptr(v), _ptr(q_slc),
                         _ptr(kbar), _ptr(rows_a), n, _ptr(o), _ptr(lse), _ptr(idx), _ptr(w)), "fwd")
     return o, lse, idx, w
+
+
+def attend(q, k, v, idx, w, S: int, rows=None):
+    """Attention and fusion for a given selection idx, w [n, h_kv, K] (one
+    entry per listed row).  Returns o [n, h_q, d], lse [n, h_q, K]."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, L, h_q, d = q.shape
+    h_kv, K = k.shape[1], idx.shape[-1]
+    rows_a = None if rows is None else np.ascontiguousarray(rows, dtype=np.int64)
+    n = B * L if rows_a is None else rows_a.shape[0]
+    idx = np.ascontiguousarray(np.asarray(idx).reshape(n, h_kv, K), dtype=np.int32)
+    w = _f64(np.asarray(w).reshape(n, h_kv, K))
+    o = np.zeros((n, h_q, d))
+    lse = np.zeros((n, h_q, K))
+    _check(lib().or_attend(B, L, h_q, h_kv, d, S, K, _ptr(q), _ptr(k), _ptr(v), _ptr(idx), _ptr(w),
+                           _ptr(rows_a), n, _ptr(o), _ptr(lse)), "attend")
+    return o, lse
 
 
 def decode(q, q_slc, k_cache, v_cache, kbar, S: int, K: int):

@@ -223,23 +223,14 @@ static double chunk_attend(int d, int S, const double *qh, const double *kc, con
     return m + log(Z);
 }
 
-/* One token row of the forward pass: selection per group, then attention and
-   fusion per query head.  [P1 §kernel]: per token, the output accumulator
-   starts at zero and each selected chunk adds w times its chunk output.  */
-static void fwd_row(int L, int h_q, int h_kv, int d, int S, int K, int b, int t, int n_c,
-                    const double *q_row /* [h_q,d] */, const double *k, const double *v,
-                    const double *qs_row /* [h_kv,d] */, const float *kbar, cand_t *cand,
-                    double *x, double *Ok, double *o_row /* [h_q,d] */, double *lse_row /* [h_q,K] */,
-                    int32_t *idx_row /* [h_kv,K] */, double *w_row /* [h_kv,K] */,
-                    double *gap_row /* [h_kv] or NULL */)
+/* Attention and fusion of one token row for a given selection (idx_row, w_row
+   per group).  [P1 §kernel]: per token, the output accumulator starts at zero
+   and each selected chunk adds w times its chunk output.  */
+static void attend_row(int L, int h_q, int h_kv, int d, int S, int K, int b, const double *q_row,
+                       const double *k, const double *v, const int32_t *idx_row, const double *w_row,
+                       double *x, double *Ok, double *o_row, double *lse_row)
 {
     const int G = h_q / h_kv; /* C7 */
-    int n_elig = t / S;       /* C1 */
-    if (n_elig > n_c) n_elig = n_c;
-    double s_tmp[OR_MAX_K], gp;
-    for (int g = 0; g < h_kv; ++g)
-        select_row(d, K, qs_row + (int64_t)g * d, kbar + ((int64_t)b * h_kv + g) * n_c * d, n_elig,
-                   cand, idx_row + g * K, w_row + g * K, s_tmp, gap_row ? gap_row + g : &gp);
     for (int h = 0; h < h_q; ++h) {
         const int g = h / G;
         double *oh = o_row + (int64_t)h * d;
@@ -257,6 +248,24 @@ static void fwd_row(int L, int h_q, int h_kv, int d, int S, int K, int b, int t,
             for (int j = 0; j < d; ++j) oh[j] += wk * Ok[j];
         }
     }
+}
+
+/* One token row of the forward pass: selection per group, then attention and
+   fusion per query head.  */
+static void fwd_row(int L, int h_q, int h_kv, int d, int S, int K, int b, int t, int n_c,
+                    const double *q_row /* [h_q,d] */, const double *k, const double *v,
+                    const double *qs_row /* [h_kv,d] */, const float *kbar, cand_t *cand,
+                    double *x, double *Ok, double *o_row /* [h_q,d] */, double *lse_row /* [h_q,K] */,
+                    int32_t *idx_row /* [h_kv,K] */, double *w_row /* [h_kv,K] */,
+                    double *gap_row /* [h_kv] or NULL */)
+{
+    int n_elig = t / S;       /* C1 */
+    if (n_elig > n_c) n_elig = n_c;
+    double s_tmp[OR_MAX_K], gp;
+    for (int g = 0; g < h_kv; ++g)
+        select_row(d, K, qs_row + (int64_t)g * d, kbar + ((int64_t)b * h_kv + g) * n_c * d, n_elig,
+                   cand, idx_row + g * K, w_row + g * K, s_tmp, gap_row ? gap_row + g : &gp);
+    attend_row(L, h_q, h_kv, d, S, K, b, q_row, k, v, idx_row, w_row, x, Ok, o_row, lse_row);
 }
 
 int or_fwd(int B, int L, int h_q, int h_kv, int d, int S, int K, const double *q, const double *k,
@@ -291,6 +300,53 @@ int or_fwd(int B, int L, int h_q, int h_kv, int d, int S, int K, const double *q
             }
         }
         free(cand);
+        free(x);
+        free(Ok);
+    }
+    return err;
+}
+
+/* Attention and fusion for a caller-given selection.  [P1 §training/inference]:
+   one chunk retrieval per step is shared by all HSA layers, so a later layer
+   attends with its own q, k, v over the chunks (and weights) that the shared
+   selection chose.  idx, w [nrows, h_kv, K] hold the selection of each listed
+   row; -1 marks an empty slot.  An entry outside 0 <= c < min(t/S, n_c) is
+   not a causal complete chunk and makes the call fail (-4). */
+int or_attend(int B, int L, int h_q, int h_kv, int d, int S, int K, const double *q, const double *k,
+              const double *v, const int32_t *idx, const double *w, const int64_t *rows, int64_t nrows,
+              double *o, double *lse)
+{
+    if (B < 0 || L < 0 || h_q < 1 || h_kv < 1 || h_q % h_kv || d < 1 || S < 1 || K < 1 || !idx ||
+        !w || !o)
+        return -1;
+    if (!rows) nrows = (int64_t)B * L;
+    const int n_c = L / S;
+    for (int64_t i = 0; i < nrows; ++i) {
+        const int r = row_of(rows, i);
+        if (r < 0 || r >= B * L) return -2;
+        const int n_elig = (r % L) / S < n_c ? (r % L) / S : n_c;
+        for (int e = 0; e < h_kv * K; ++e) {
+            const int c = idx[i * h_kv * K + e];
+            if (c < -1 || c >= n_elig) return -4;
+        }
+    }
+    int err = 0;
+#pragma omp parallel
+    {
+        double *x = (double *)malloc(sizeof(double) * (size_t)S);
+        double *Ok = (double *)malloc(sizeof(double) * (size_t)d);
+        if (!x || !Ok) {
+#pragma omp atomic write
+            err = -3;
+        } else {
+#pragma omp for schedule(dynamic, 8)
+            for (int64_t i = 0; i < nrows; ++i) {
+                const int r = row_of(rows, i);
+                attend_row(L, h_q, h_kv, d, S, K, r / L, q + (int64_t)r * h_q * d, k, v,
+                           idx + i * h_kv * K, w + i * h_kv * K, x, Ok, o + i * h_q * d,
+                           lse ? lse + i * h_q * K : NULL);
+            }
+        }
         free(x);
         free(Ok);
     }

@@ -285,6 +285,72 @@ def test_dense_masked_bruteforce(S):
             np.testing.assert_allclose(o[b, :, h], want, atol=1e-12, rtol=1e-12)
 
 
+# --------------------------------------------------------------------------- shared selection
+def _random_causal_selection(rng, B, L, h_kv, K, S):
+    """Any causal selection: complete past chunks, empty slots (-1), repeats, any weights."""
+    idx = np.full((B * L, h_kv, K), -1, dtype=np.int32)
+    for r in range(B * L):
+        ne = min((r % L) // S, L // S)
+        if ne:
+            idx[r] = rng.integers(0, ne, size=(h_kv, K))
+    idx[rng.random(idx.shape) < 0.2] = -1
+    w = rng.normal(size=idx.shape)
+    return idx, w
+
+
+def test_attend_given_selection_dense_masked_bruteforce():
+    """attend(idx, w) for an arbitrary causal selection against the dense L x L
+    logit matrix (library matmul) with a block mask per listed chunk."""
+    wl = tiny(B=2, L=96, h_q=4, h_kv=2, d=8, S=8, K=4, seed=41)
+    x = synth.make_inputs(wl)
+    idx, w = _random_causal_selection(np.random.default_rng(5), wl.B, wl.L, wl.h_kv, wl.K, wl.S)
+    idx[3 * wl.S + 1, 0, :2] = 1  # a chunk listed twice for one row
+    o, lse = oracle.attend(x["q"], x["k"], x["v"], idx, w, wl.S)
+    o = o.reshape(wl.B, wl.L, wl.h_q, wl.d)
+    idx4, w4 = idx.reshape(wl.B, wl.L, wl.h_kv, wl.K), w.reshape(wl.B, wl.L, wl.h_kv, wl.K)
+    G = wl.h_q // wl.h_kv
+    chunk_of = np.arange(wl.L) // wl.S
+    for b in range(wl.B):
+        for h in range(wl.h_q):
+            g = h // G
+            E = np.exp(x["q"][b, :, h, :] @ x["k"][b, g].T / math.sqrt(wl.d))
+            want = np.zeros((wl.L, wl.d))
+            for t in range(wl.L):
+                for j in range(wl.K):
+                    c = idx4[b, t, g, j]
+                    if c < 0:
+                        continue
+                    m = chunk_of == c
+                    want[t] += w4[b, t, g, j] * (E[t, m] @ x["v"][b, g][m]) / (1.0 + E[t, m].sum())
+            np.testing.assert_allclose(o[b, :, h], want, atol=1e-12, rtol=1e-12)
+
+
+def test_attend_with_own_selection_is_forward():
+    """attend over select's (idx, w) is the forward pass exactly (same rows, bit for bit)."""
+    wl = tiny(B=1, L=128, h_q=4, h_kv=2, d=8, S=8, K=3, seed=42)
+    x = synth.make_inputs(wl)
+    kbar = oracle.pool(x["k"], wl.S)
+    o, lse, idx, w = oracle.fwd(x["q"], x["k"], x["v"], x["q_slc"], kbar, wl.S, wl.K)
+    o2, lse2 = oracle.attend(x["q"], x["k"], x["v"], idx, w, wl.S)
+    assert np.array_equal(o, o2) and np.array_equal(lse, lse2)
+    rows = np.array([5, 64, 127])
+    o3, _ = oracle.attend(x["q"], x["k"], x["v"], idx[rows], w[rows], wl.S, rows=rows)
+    assert np.array_equal(o3, o[rows])
+
+
+def test_attend_rejects_non_causal_entries():
+    wl = tiny(B=1, L=64, h_q=2, h_kv=1, d=8, S=8, K=2, seed=43)
+    x = synth.make_inputs(wl)
+    idx = np.full((wl.L, 1, wl.K), -1, dtype=np.int32)
+    w = np.ones(idx.shape)
+    idx[20, 0, 0] = 2  # token 20 sees chunks 0, 1 only
+    with pytest.raises(RuntimeError, match="code -4"):
+        oracle.attend(x["q"], x["k"], x["v"], idx, w, wl.S)
+    idx[20, 0, 0] = -2
+    with pytest.raises(RuntimeError, match="code -4"):
+        oracle.attend(x["q"], x["k"], x["v"], idx, w, wl.S)
+
+
 # --------------------------------------------------------------------------- decode
 def test_decode_equals_forward_last_row():
     """The decode step at position P is forward row t = P of the prompt plus one token."""

@@ -19,7 +19,7 @@ import os
 
 import torch
 
-__all__ = ["hsa_timing_enable", "hsa_timing_read", "KERNELS", "hsa_workspace_size", "hsa_pool", "hsa_select", "hsa_fwd", "hsa_decode", "hsa_bwd",
+__all__ = ["hsa_timing_enable", "hsa_timing_read", "KERNELS", "hsa_workspace_size", "hsa_pool", "hsa_select", "hsa_fwd", "hsa_attend", "hsa_decode", "hsa_bwd",
            "hsa_device_status", "HsaError", "lib_path", "load_library", "OP_POOL", "OP_SELECT",
            "OP_FWD", "OP_DECODE", "OP_BWD"]
 
@@ -65,6 +65,7 @@ def load_library():
         L.hsa_pool.argtypes = [sp, P, P, P, Z, P]
         L.hsa_select.argtypes = [sp, P, P, P, P, P, P, Z, P]
         L.hsa_fwd.argtypes = [sp, P, P, P, P, P, P, P, P, P, P, Z, P]
+        L.hsa_attend.argtypes = [sp, P, P, P, P, P, P, P, P, Z, P]
         L.hsa_decode.argtypes = [sp, P, P, P, P, P, P, P, P, P, Z, P]
         L.hsa_bwd.argtypes = [sp, P, P, P, P, P, P, P, P, P, P, P, P, P, P, Z, P]
         L.hsa_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_int32), P]
@@ -74,7 +75,7 @@ def load_library():
         L.hsa_timing_read.restype = ctypes.c_int
         L.hsa_status_string.argtypes = [ctypes.c_int32]
         L.hsa_status_string.restype = ctypes.c_char_p
-        for f in ("hsa_pool", "hsa_select", "hsa_fwd", "hsa_decode", "hsa_bwd", "hsa_device_status"):
+        for f in ("hsa_pool", "hsa_select", "hsa_fwd", "hsa_attend", "hsa_decode", "hsa_bwd", "hsa_device_status"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -193,6 +194,28 @@ def hsa_fwd(q, k, v, q_slc, K: int, S: int = 64, want_lse: bool = True, want_sel
     _check(load_library().hsa_fwd(ctypes.byref(sh), _p(q), _p(k), _p(v), _p(q_slc), _p(o), _p(lse),
                                   _p(idx), _p(w), _p(kbar), _p(w_), n, _stream(stream)), "hsa_fwd")
     return o, lse, idx, w, kbar
+
+
+def hsa_attend(q, k, v, idx, w, S: int = 64, want_lse: bool = True, o=None, ws=None, stream=None):
+    """Attention and fusion for a given selection (idx, w from hsa_select or
+    hsa_fwd), e.g. one selection shared by several layers.  Returns (o, lse)."""
+    B, L, h_q, d = q.shape
+    h_kv, K = k.shape[1], idx.shape[-1]
+    dt, dev = _dtype_code(q), q.device
+    _need(q, "q", q.shape, q.dtype)
+    _need(k, "k", (B, h_kv, L, d), q.dtype, dev)
+    _need(v, "v", (B, h_kv, L, d), q.dtype, dev)
+    _need(idx, "idx", (B, L, h_kv, K), torch.int32, dev)
+    _need(w, "w", (B, L, h_kv, K), torch.float32, dev)
+    if o is None:
+        o = torch.empty_like(q)
+    _need(o, "o", q.shape, q.dtype, dev)
+    lse = torch.empty(B, L, h_q, K, dtype=torch.float32, device=dev) if want_lse else None
+    sh = HsaShape(B, L, h_q, h_kv, d, S, K, dt)
+    w_, n = _workspace(sh, OP_FWD, dev, ws)
+    _check(load_library().hsa_attend(ctypes.byref(sh), _p(q), _p(k), _p(v), _p(idx), _p(w), _p(o),
+                                     _p(lse), _p(w_), n, _stream(stream)), "hsa_attend")
+    return o, lse
 
 
 def hsa_decode(q, q_slc, k_cache, v_cache, kbar, K: int, S: int = 64, o=None, want_sel=True,

@@ -242,6 +242,40 @@ hsa_status_t hsa_select(const hsa_shape_t *shape, const void *q_slc, const void 
     return cuda_status(e);
 }
 
+// attention + fusion (a5-a6) for a given selection f.idx / f.w: tensor-core chunk-major
+// path (inversion, plan, attend) for the shapes it takes, CUDA cores otherwise
+static cudaError_t run_attend(const Shape &sh, const void *q, const void *k, const void *v, FwdWs &f, void *o,
+                              float *lse, bool given_sel, DevStatus *ds, cudaStream_t st) {
+    cudaError_t e = cudaSuccess;
+    if (!f.tc) {
+        if (e == cudaSuccess)
+            e = timed(HSA_K_ATTEND_SIMT, 1, st, [&] { return launch_attend_simt(sh, q, k, v, f.idx, f.w, o, lse, ds, st); });
+        return e;
+    }
+    // chunk-major tensor-core path: invert the selection, plan windows, attend
+    if (e == cudaSuccess && sh.nc > 0)
+        e = timed(HSA_K_INVERT, 5, st, [&] { return launch_invert(sh, f.idx, f.w, f.inv, ds, st); });
+    if (e == cudaSuccess) e = timed(HSA_K_PLAN, 3, st, [&] { return launch_plan(sh, f.inv, f.plan, st); });
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(f.plan.counters, 0, sizeof(int32_t) * plan_counter_count(f.plan.J), st);
+    if (e == cudaSuccess)  // the used accumulator slots start at zero (the kernel re-zeroes them after use)
+        e = cudaMemsetAsync(f.acc, 0,
+                            sizeof(__half) * std::min<size_t>(attend_acc_elems(f.plan.W, sh.G, sh.d),
+                                                             (size_t)f.plan.J * f.plan.W * sh.G * sh.d),
+                            st);
+    if (e == cudaSuccess && lse)
+        e = cudaMemsetAsync(lse, 0, sizeof(float) * (size_t)sh.B * sh.L * sh.hq * sh.K, st);
+    if (e == cudaSuccess)  // the accumulators' power-of-two scale comes from max|v|
+        e = timed(HSA_K_PLAN, 1, st, [&] { return launch_vmax(sh, v, f.plan.counters + 3 * f.plan.J + 1, st); });
+    if (e == cudaSuccess && given_sel)  // weights not from stick-breaking: their row sums may exceed 1
+        e = timed(HSA_K_PLAN, 1, st, [&] { return launch_wsum(sh, f.idx, f.w, f.plan.counters + 3 * f.plan.J + 2, st); });
+    if (e == cudaSuccess)
+        e = timed(HSA_K_ATTEND_TC, 1, st, [&] {
+            return launch_attend_tc(sh, f.plan, f.inv, q, k, v, f.idx, f.w, f.acc, o, lse, ds, st);
+        });
+    return e;
+}
+
 hsa_status_t hsa_fwd(const hsa_shape_t *shape, const void *q, const void *k, const void *v,
                      const void *q_slc, void *o, float *lse, int32_t *idx, float *w, float *kbar,
                      void *ws, size_t ws_bytes, void *stream) {
@@ -261,30 +295,26 @@ hsa_status_t hsa_fwd(const hsa_shape_t *shape, const void *q, const void *k, con
     cudaError_t e = clear_status(ws, st);
     if (e == cudaSuccess) e = timed(HSA_K_POOL, 1, st, [&] { return launch_pool(sh, k, f.kbar, ds, st); });
     if (e == cudaSuccess) e = run_select(sh, q_slc, f.kbar, f.kb_hi, f.kb_lo, f.idx, f.w, ds, st);
-    if (!f.tc) {
-        if (e == cudaSuccess)
-            e = timed(HSA_K_ATTEND_SIMT, 1, st, [&] { return launch_attend_simt(sh, q, k, v, f.idx, f.w, o, lse, ds, st); });
-        return cuda_status(e);
-    }
-    // chunk-major tensor-core path: invert the selection, plan windows, attend
-    if (e == cudaSuccess && sh.nc > 0)
-        e = timed(HSA_K_INVERT, 5, st, [&] { return launch_invert(sh, f.idx, f.w, f.inv, ds, st); });
-    if (e == cudaSuccess) e = timed(HSA_K_PLAN, 3, st, [&] { return launch_plan(sh, f.inv, f.plan, st); });
-    if (e == cudaSuccess)
-        e = cudaMemsetAsync(f.plan.counters, 0, sizeof(int32_t) * plan_counter_count(f.plan.J), st);
-    if (e == cudaSuccess)  // the used accumulator slots start at zero (the kernel re-zeroes them after use)
-        e = cudaMemsetAsync(f.acc, 0,
-                            sizeof(__half) * std::min<size_t>(attend_acc_elems(f.plan.W, sh.G, sh.d),
-                                                             (size_t)f.plan.J * f.plan.W * sh.G * sh.d),
-                            st);
-    if (e == cudaSuccess && lse)
-        e = cudaMemsetAsync(lse, 0, sizeof(float) * (size_t)sh.B * sh.L * sh.hq * sh.K, st);
-    if (e == cudaSuccess)  // the accumulators' power-of-two scale comes from max|v|
-        e = timed(HSA_K_PLAN, 1, st, [&] { return launch_vmax(sh, v, f.plan.counters + 3 * f.plan.J + 1, st); });
-    if (e == cudaSuccess)
-        e = timed(HSA_K_ATTEND_TC, 1, st, [&] {
-            return launch_attend_tc(sh, f.plan, f.inv, q, k, v, f.idx, f.w, f.acc, o, lse, ds, st);
-        });
+    if (e == cudaSuccess) e = run_attend(sh, q, k, v, f, o, lse, false, ds, st);
+    return cuda_status(e);
+}
+
+hsa_status_t hsa_attend(const hsa_shape_t *shape, const void *q, const void *k, const void *v,
+                        const int32_t *idx, const float *w, void *o, float *lse, void *ws, size_t ws_bytes,
+                        void *stream) {
+    hsa_status_t s = check_shape(shape, false);
+    if (s != HSA_OK) return s;
+    const Shape sh = make_shape(*shape);
+    if ((int64_t)sh.B * sh.L == 0) return empty_call(sh, HSA_OP_FWD, ws, ws_bytes, static_cast<cudaStream_t>(stream));
+    if (!ptrs_ok({q, k, v, idx, w, o}) || !opt_ok(lse)) return HSA_ERR_INVALID_ARG;
+    if ((s = check_ws(sh, HSA_OP_FWD, ws, ws_bytes)) != HSA_OK) return s;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    DevStatus *ds = static_cast<DevStatus *>(ws);
+    FwdWs f = carve_fwd(sh, ws, nullptr);
+    f.idx = const_cast<int32_t *>(idx);  // read only from here on
+    f.w = const_cast<float *>(w);
+    cudaError_t e = clear_status(ws, st);
+    if (e == cudaSuccess) e = run_attend(sh, q, k, v, f, o, lse, true, ds, st);
     return cuda_status(e);
 }
 

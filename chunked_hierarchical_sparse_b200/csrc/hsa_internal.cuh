@@ -217,6 +217,7 @@ cudaError_t launch_attend_tc(const Shape &sh, const AttendPlan &plan, const BwdW
                              __half *acc, void *o, float *lse, DevStatus *ds, cudaStream_t st);
 // max|v| over the whole value tensor, as float bits, max-ed into *bits (zeroed by the caller)
 cudaError_t launch_vmax(const Shape &sh, const void *v, int32_t *bits, cudaStream_t st);
+cudaError_t launch_wsum(const Shape &sh, const int32_t *idx, const float *w, int32_t *bits, cudaStream_t st);
 
 // Chunk-major backward on the tensor cores (d = 128, G in {8, 16}): dq (via the
 // plan's window ring `acc`), dw [B,L,hkv,K], and dK / dV added into the fp32

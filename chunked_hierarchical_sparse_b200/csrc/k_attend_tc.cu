@@ -217,10 +217,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     int32_t *comb_done = P.counters + P.J;
     int32_t *comb_head = P.counters + 2 * P.J;
     const float scale = 1.0f / sqrtf((float)D);
-    // power-of-two scale of the fp16 accumulators: 2^e >= max|v| (bits written by vmax_kernel)
+    // power-of-two scale of the fp16 accumulators: 2^e >= max|v| * max(1, max_row sum|w|)
+    // (bits written by vmax_kernel and, for a caller-given selection, wsum_kernel)
     float acc_scale, acc_inv;
     {
-        const uint32_t vb = (uint32_t)P.counters[3 * P.J + 1];
+        const float wsum = __int_as_float(P.counters[3 * P.J + 2]);
+        const uint32_t vb = (uint32_t)__float_as_int(__int_as_float(P.counters[3 * P.J + 1]) * fmaxf(1.f, wsum));
         int ev = (int)((vb >> 23) & 0xff) - 127;
         if (vb & 0x7fffffu) ev += 1;
         if (vb == 0) ev = 0;
@@ -920,6 +922,31 @@ cudaError_t launch_vmax(const Shape &sh, const void *v, int32_t *bits, cudaStrea
     if (n8 == 0) return cudaSuccess;
     const int blocks = (int)std::min<int64_t>(ceil_div(n8, 256), 148 * 4);
     vmax_kernel<<<blocks, 256, 0, st>>>((const __nv_bfloat16 *)v, n8, bits);
+    return cudaGetLastError();
+}
+
+// max over (token, group) rows of sum_k |w_k| over the row's non-empty slots,
+// as float bits max-ed into *bits.  Stick-breaking weights sum to at most 1;
+// a caller-given selection may not, and the accumulators' scale takes it in.
+__global__ void __launch_bounds__(256) wsum_kernel(const int32_t *__restrict__ idx, const float *__restrict__ w,
+                                                   int64_t rows, int K, int32_t *__restrict__ bits) {
+    float m = 0.f;
+    for (int64_t r = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; r < rows; r += (int64_t)gridDim.x * blockDim.x) {
+        float s = 0.f;
+        for (int kk = 0; kk < K; ++kk)
+            if (idx[r * K + kk] >= 0) s += fabsf(w[r * K + kk]);
+        m = fmaxf(m, s);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if ((threadIdx.x & 31) == 0) atomicMax(bits, __float_as_int(m));
+}
+
+cudaError_t launch_wsum(const Shape &sh, const int32_t *idx, const float *w, int32_t *bits, cudaStream_t st) {
+    const int64_t rows = (int64_t)sh.B * sh.L * sh.hkv;
+    if (rows == 0) return cudaSuccess;
+    const int blocks = (int)std::min<int64_t>(ceil_div(rows, 256), 148 * 4);
+    wsum_kernel<<<blocks, 256, 0, st>>>(idx, w, rows, sh.K, bits);
     return cudaGetLastError();
 }
 

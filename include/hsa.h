@@ -132,6 +132,22 @@ HSA_API hsa_status_t hsa_fwd(const hsa_shape_t *shape, const void *q, const void
                      const void *q_slc, void *o, float *lse, int32_t *idx, float *w, float *kbar,
                      void *ws, size_t ws_bytes, void *stream);
 
+/* Steps a5-a6 for a given selection: one chunk selection shared by several
+ * HSA layers [P1 §training/inference: one retrieval per step serves all HSA
+ * layers].  Run hsa_select (or hsa_fwd) once, then hsa_attend per layer with
+ * that layer's q, k, v.  idx [B,L,h_kv,K] int32 and w [B,L,h_kv,K] fp32 are
+ * inputs in hsa_select's layout.  A negative entry is an empty slot (its
+ * weight is ignored); an entry c >= 0 must satisfy c < n_c and c < t/S for
+ * token t (a causal, complete chunk) -- one that does not is skipped and
+ * reported as HSA_ERR_DEVICE_CHECK in the status word.  A chunk listed twice
+ * for one token contributes twice.  Weights are any finite values (the fp16
+ * cross-chunk sums are scaled by max|v| times the largest per-row sum of |w|).
+ * o is required, lse optional (as in hsa_fwd).
+ * Workspace: hsa_workspace_size(shape, HSA_OP_FWD). */
+HSA_API hsa_status_t hsa_attend(const hsa_shape_t *shape, const void *q, const void *k, const void *v,
+                        const int32_t *idx, const float *w, void *o, float *lse, void *ws,
+                        size_t ws_bytes, void *stream);
+
 /* Step a7: one decode step per sequence against the chunk-level index
  * [P1 §training/inference]: shape.L = P (cached tokens); the new token sits at
  * position P, so all floor(P/S) cached chunks are eligible.  kbar is an input

@@ -26,7 +26,7 @@ def declared_symbols():
 
 def test_header_declares_the_boundary():
     names = set(declared_symbols())
-    assert {"hsa_pool", "hsa_select", "hsa_fwd", "hsa_decode", "hsa_bwd", "hsa_workspace_size",
+    assert {"hsa_pool", "hsa_select", "hsa_fwd", "hsa_attend", "hsa_decode", "hsa_bwd", "hsa_workspace_size",
             "hsa_device_status", "hsa_status_string"} <= names
 
 
@@ -89,6 +89,9 @@ def test_host_validation_without_gpu(lib):
     # bwd needs every gradient output
     assert lib.hsa_bwd(ctypes.byref(sh), good, good, good, good, good, good, good, good, good, None,
                        good, good, good, ws, 1 << 30, None) == 1
+    # shared-selection attend needs idx and w; workspace is the forward's
+    assert lib.hsa_attend(ctypes.byref(sh), good, good, good, None, good, good, None, ws, 1 << 30, None) == 1
+    assert lib.hsa_attend(ctypes.byref(sh), good, good, good, good, good, good, None, ws, 300, None) == 3
     assert lib.hsa_device_status(None, None, None) == 1
     assert lib.hsa_status_string(3) == b"workspace too small"
 

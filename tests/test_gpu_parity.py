@@ -147,6 +147,109 @@ def test_fwd_tensor_core_value_scale(factor):
     assert_out(f64(o).reshape(o_ref.shape) / factor, o_ref, "bf16", "o")
 
 
+# --------------------------------------------------------------------------- shared selection
+def run_attend(wl, x, idx, w):
+    """hsa_attend with the given selection (device tensors); returns (o, lse, status)."""
+    m = hsa()
+    q, k, v = (to_dev(x[n], wl.dtype) for n in ("q", "k", "v"))
+    tdt = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+    ws = torch.empty(m.hsa_workspace_size(wl.B, wl.L, wl.h_q, wl.h_kv, wl.d, 64, wl.K, tdt, m.OP_FWD),
+                     dtype=torch.uint8, device=DEV)
+    o, lse = m.hsa_attend(q, k, v, idx, w, ws=ws)
+    torch.cuda.synchronize()
+    return o, lse, m.hsa_device_status(ws)
+
+
+def random_selection(wl, seed, w_scale=1.0):
+    """Any causal selection (not a top-K): past complete chunks, empty slots,
+    repeated chunks and weights of either sign; [B, L, h_kv, K]."""
+    rng = np.random.default_rng(seed)
+    t = np.arange(wl.L)
+    ne = np.minimum(t // wl.S, wl.L // wl.S)[None, :, None, None]
+    shape = (wl.B, wl.L, wl.h_kv, wl.K)
+    idx = np.floor(rng.random(shape) * ne).astype(np.int32)
+    idx[(ne == 0) | (rng.random(shape) < 0.15)] = -1
+    w = (rng.normal(size=shape) * w_scale).astype(np.float32)
+    return idx, w
+
+
+ATTEND = [small(dtype="f32", d=64, K=4, L=1024, h_q=4, h_kv=1), small(L=64 * 37 + 5, K=8, h_q=8, h_kv=2),
+          small(h_q=16, h_kv=2, K=8, L=1000), small(h_q=16, h_kv=1, K=4, L=64 * 45 + 3, B=1)]
+ATTEND_IDS = ["f32-simt", "bf16-g4-simt", "g8-tc", "g16-tc-ragged"]
+
+
+def tc_ran(wl):
+    return wl.dtype == "bf16" and wl.h_q // wl.h_kv in (8, 16)
+
+
+@pytest.mark.parametrize("wl", ATTEND, ids=ATTEND_IDS)
+def test_shared_selection_across_layers(wl):
+    """Layer 1 selects (hsa_select on its q_slc, k); layer 2 attends with its own
+    q, k, v over layer 1's chunks.  The oracle's forward with layer 2's q, k, v and
+    layer 1's q_slc, kbar is the same computation."""
+    x1, kbar1, (idx_ref, w_ref, s_ref, gap) = gap_ruled(wl)
+    x2 = synth.make_inputs(wl.scaled(seed=wl.seed + 7))
+    o_ref, lse_ref, i2, _ = oracle.fwd(x2["q"], x2["k"], x2["v"], x1["q_slc"], kbar1, wl.S, wl.K)
+    assert np.array_equal(i2, idx_ref)
+    m = hsa()
+    kb, idx, w = m.hsa_select(to_dev(x1["q_slc"], wl.dtype), to_dev(x1["k"], wl.dtype), wl.K)
+    assert np.array_equal(idx.cpu().numpy().reshape(idx_ref.shape), idx_ref)
+    m.hsa_timing_enable(True)
+    o, lse, status = run_attend(wl, x2, idx, w)
+    _, n_tc = m.hsa_timing_read("attend_tc")
+    m.hsa_timing_enable(False)
+    assert status == 0
+    assert n_tc == (1 if tc_ran(wl) else 0)
+    assert_out(f64(o).reshape(o_ref.shape), o_ref, wl.dtype, "o")
+    assert np.abs(f64(lse).reshape(lse_ref.shape) - lse_ref).max() <= (1e-5 if wl.dtype == "f32" else 2e-3)
+
+
+@pytest.mark.parametrize("wl", ATTEND, ids=ATTEND_IDS)
+def test_attend_arbitrary_selection(wl):
+    """Any causal selection with empty slots, repeats and signed weights."""
+    x = synth.make_inputs(wl)
+    idx, w = random_selection(wl, wl.seed)
+    o_ref, lse_ref = oracle.attend(x["q"], x["k"], x["v"], idx, w, wl.S)
+    o, lse, status = run_attend(wl, x, torch.from_numpy(idx).to(DEV), torch.from_numpy(w).to(DEV))
+    assert status == 0
+    scale = max(1.0, np.abs(o_ref).max())
+    got = f64(o).reshape(o_ref.shape)
+    assert_out(got / scale, o_ref / scale, wl.dtype, "o")
+    assert np.abs(f64(lse).reshape(lse_ref.shape) - lse_ref).max() <= (1e-5 if wl.dtype == "f32" else 2e-3)
+
+
+def test_attend_large_weights_scale_the_accumulators():
+    """Weights of size 2^16 would overflow fp16 cross-chunk sums scaled by max|v|
+    alone; the scale takes the row sums of |w| in, so o / 2^16 matches."""
+    wl = ATTEND[2]
+    x = synth.make_inputs(wl)
+    idx, w = random_selection(wl, wl.seed + 1)
+    o_ref, _ = oracle.attend(x["q"], x["k"], x["v"], idx, w, wl.S)
+    big = torch.from_numpy(w * np.float32(2.0 ** 16)).to(DEV)
+    o, _, status = run_attend(wl, x, torch.from_numpy(idx).to(DEV), big)
+    assert status == 0
+    got = f64(o).reshape(o_ref.shape) / 2.0 ** 16
+    assert np.isfinite(got).all()
+    scale = max(1.0, np.abs(o_ref).max())
+    assert_out(got / scale, o_ref / scale, "bf16", "o")
+
+
+@pytest.mark.parametrize("wl", [ATTEND[0], ATTEND[2]], ids=["simt", "tc"])
+def test_attend_reports_non_causal_index(wl):
+    """An entry that is not a causal complete chunk is skipped and reported in the
+    status word; every other entry is still attended."""
+    x = synth.make_inputs(wl)
+    idx, w = random_selection(wl, wl.seed + 2)
+    t_bad = 3 * wl.S + 5
+    idx[0, t_bad, 0, 0] = 3  # token t_bad sees chunks 0, 1, 2 only
+    o, _, status = run_attend(wl, x, torch.from_numpy(idx).to(DEV), torch.from_numpy(w).to(DEV))
+    assert status == 6  # HSA_ERR_DEVICE_CHECK
+    idx[0, t_bad, 0, 0] = -1
+    o_ref, _ = oracle.attend(x["q"], x["k"], x["v"], idx, w, wl.S)
+    scale = max(1.0, np.abs(o_ref).max())
+    assert_out(f64(o).reshape(o_ref.shape) / scale, o_ref / scale, wl.dtype, "o")
+
+
 def test_fwd_tiny_fp32_workload():
     """The tiny fp32 workload in full: indices exact, max |err| <= 1e-5."""
     wl, (x, kbar, sel) = cached_workload("tiny_fp32")

@@ -327,7 +327,7 @@ int or_attend(int B, int L, int h_q, int h_kv, int d, int S, int K, const double
         const int n_elig = (r % L) / S < n_c ? (r % L) / S : n_c;
         for (int e = 0; e < h_kv * K; ++e) {
             const int c = idx[i * h_kv * K + e];
-            if (c < -1 || c >= n_elig) return -4;
+            if (c >= n_elig) return -4;
         }
     }
     int err = 0;

@@ -271,6 +271,62 @@ def bench_decode(hsa, dev, reps=1000):
             "compulsory_bytes": int(byt), "roofline_us": byt / (load_peaks()["hbm_gbs"] * 1e9) * 1e6}
 
 
+def _median_us(fn, reps):
+    import torch
+    for _ in range(5):
+        fn()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+    for a, b in ev:
+        a.record()
+        fn()
+        b.record()
+    torch.cuda.synchronize()
+    t = sorted(a.elapsed_time(b) * 1e3 for a, b in ev)
+    return t[len(t) // 2]
+
+
+def bench_decode_offload(hsa, dev, layers=(1, 4), reps=200):
+    """The decode16k step with the KV cache in page-locked host memory: only the
+    K selected chunks per (sequence, group) cross the host link.  For n_layers
+    layers sharing one selection (hsa_decode_multi) against n_layers separate
+    hsa_decode calls (each selecting and reading its chunks again)."""
+    import torch
+    from chunked_hierarchical_sparse_b200 import synth
+    wl = synth.WORKLOADS["decode16k"]
+    x = synth.make_inputs(wl)
+    qs = to_dev(x["q_slc"], dev)
+    kh = torch.from_numpy(x["k"]).to(torch.bfloat16).pin_memory()
+    vh = torch.from_numpy(x["v"]).to(torch.bfloat16).pin_memory()
+    kbar = hsa.hsa_pool(kh.to(dev))
+    n = hsa.hsa_workspace_size(wl.B, wl.L, wl.h_q, wl.h_kv, wl.d, wl.S, wl.K, torch.bfloat16, hsa.OP_DECODE)
+    ws = torch.empty(n, dtype=torch.uint8, device=dev)
+    # host-to-device copy bandwidth of this box's link (the bound of the offloaded step)
+    dst = torch.empty(kh.numel(), dtype=torch.bfloat16, device=dev)
+    link_us = _median_us(lambda: dst.copy_(kh.view(-1), non_blocking=True), 10)
+    link_gbs = kh.numel() * 2 / (link_us * 1e-6) / 1e9
+    del dst
+    sel_bytes = wl.B * wl.h_kv * wl.K * 2 * wl.S * wl.d * 2
+    out = {"workload": "decode16k, KV cache in page-locked host memory", "unit": "us",
+           "host_link_h2d_gbs": link_gbs, "selected_bytes_per_step": sel_bytes,
+           "link_bound_us": sel_bytes / (link_gbs * 1e9) * 1e6}
+    for NL in layers:
+        q = to_dev(synth.layer_queries(wl, NL), dev)
+        o = torch.empty_like(q)
+        shared = _median_us(lambda: hsa.hsa_decode_multi(q, qs, kh, vh, kbar, wl.K, o=o, ws=ws, want_sel=False),
+                            reps)
+        ol = [torch.empty_like(q[l]) for l in range(NL)]
+        ql = [q[l].contiguous() for l in range(NL)]
+
+        def separate():
+            for l in range(NL):
+                hsa.hsa_decode(ql[l], qs, kh, vh, kbar, wl.K, o=ol[l], ws=ws, want_sel=False)
+        sep = _median_us(separate, reps)
+        out[f"layers{NL}"] = {"shared_us": shared, "separate_us": sep,
+                              "achieved_link_gbs": sel_bytes / (shared * 1e-6) / 1e9}
+    return out
+
+
 def bench_train(hsa, dev, steps=3):
     import torch
     from chunked_hierarchical_sparse_b200 import synth
@@ -438,6 +494,7 @@ def main():
 
     if not args.no_extras:
         line["decode"] = bench_decode(hsa, dev)
+        line["decode_offload"] = bench_decode_offload(hsa, dev)
         line["train"] = bench_train(hsa, dev)
     if rank == 0 and world == 1 and not args.no_cpu:
         line["cpu_baseline"] = cpu_baseline(wl, x, args.cpu_budget_s)

@@ -19,7 +19,7 @@ import os
 
 import torch
 
-__all__ = ["hsa_timing_enable", "hsa_timing_read", "KERNELS", "hsa_workspace_size", "hsa_pool", "hsa_select", "hsa_fwd", "hsa_attend", "hsa_decode", "hsa_bwd",
+__all__ = ["hsa_timing_enable", "hsa_timing_read", "KERNELS", "hsa_workspace_size", "hsa_pool", "hsa_select", "hsa_fwd", "hsa_attend", "hsa_decode", "hsa_decode_multi", "hsa_bwd",
            "hsa_device_status", "HsaError", "lib_path", "load_library", "OP_POOL", "OP_SELECT",
            "OP_FWD", "OP_DECODE", "OP_BWD"]
 
@@ -67,6 +67,7 @@ def load_library():
         L.hsa_fwd.argtypes = [sp, P, P, P, P, P, P, P, P, P, P, Z, P]
         L.hsa_attend.argtypes = [sp, P, P, P, P, P, P, P, P, Z, P]
         L.hsa_decode.argtypes = [sp, P, P, P, P, P, P, P, P, P, Z, P]
+        L.hsa_decode_multi.argtypes = [sp, ctypes.c_int32, P, P, P, P, P, P, P, P, P, Z, P]
         L.hsa_bwd.argtypes = [sp, P, P, P, P, P, P, P, P, P, P, P, P, P, P, Z, P]
         L.hsa_device_status.argtypes = [P, ctypes.POINTER(ctypes.c_int32), P]
         L.hsa_timing_enable.argtypes = [I]
@@ -75,7 +76,7 @@ def load_library():
         L.hsa_timing_read.restype = ctypes.c_int
         L.hsa_status_string.argtypes = [ctypes.c_int32]
         L.hsa_status_string.restype = ctypes.c_char_p
-        for f in ("hsa_pool", "hsa_select", "hsa_fwd", "hsa_attend", "hsa_decode", "hsa_bwd", "hsa_device_status"):
+        for f in ("hsa_pool", "hsa_select", "hsa_fwd", "hsa_attend", "hsa_decode", "hsa_decode_multi", "hsa_bwd", "hsa_device_status"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -90,7 +91,7 @@ def _dtype_code(t: torch.Tensor) -> int:
     raise TypeError(f"token tensors must be float32 or bfloat16, got {t.dtype}")
 
 
-def _need(t: torch.Tensor, name: str, shape, dtype=None, device=None):
+def _need(t: torch.Tensor, name: str, shape, dtype=None, device=None, host_ok=False):
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
     if tuple(t.shape) != tuple(shape):
@@ -99,6 +100,10 @@ def _need(t: torch.Tensor, name: str, shape, dtype=None, device=None):
         raise TypeError(f"{name}: expected {dtype}, got {t.dtype}")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+    if host_ok and not t.is_cuda:  # an offloaded cache: page-locked host memory the GPU reads directly
+        if not t.is_pinned():
+            raise ValueError(f"{name}: a host tensor must be page-locked (pin_memory())")
+        return
     if device is not None and t.device != device:
         raise ValueError(f"{name} must be on {device}")
     if not t.is_cuda:
@@ -227,8 +232,8 @@ def hsa_decode(q, q_slc, k_cache, v_cache, kbar, K: int, S: int = 64, o=None, wa
     dt, dev = _dtype_code(q), q.device
     _need(q, "q", q.shape, q.dtype)
     _need(q_slc, "q_slc", (B, h_kv, d), q.dtype, dev)
-    _need(k_cache, "k_cache", (B, h_kv, P, d), q.dtype, dev)
-    _need(v_cache, "v_cache", (B, h_kv, P, d), q.dtype, dev)
+    _need(k_cache, "k_cache", (B, h_kv, P, d), q.dtype, dev, host_ok=True)
+    _need(v_cache, "v_cache", (B, h_kv, P, d), q.dtype, dev, host_ok=True)
     _need(kbar, "kbar", (B, h_kv, P // S, d), torch.float32, dev)
     if o is None:
         o = torch.empty_like(q)
@@ -240,6 +245,32 @@ def hsa_decode(q, q_slc, k_cache, v_cache, kbar, K: int, S: int = 64, o=None, wa
     _check(load_library().hsa_decode(ctypes.byref(sh), _p(q), _p(q_slc), _p(k_cache), _p(v_cache),
                                      _p(kbar), _p(o), _p(idx), _p(w), _p(w_), n, _stream(stream)),
            "hsa_decode")
+    return o, idx, w
+
+
+def hsa_decode_multi(q, q_slc, k_cache, v_cache, kbar, K: int, S: int = 64, o=None, want_sel=True,
+                     ws=None, stream=None):
+    """One decode step for several HSA layers sharing the selection and the KV
+    cache.  q [n_layers,B,h_q,d]; the rest as in hsa_decode (the caches may be
+    page-locked host tensors).  Returns (o [n_layers,B,h_q,d], idx, w)."""
+    NL, B, h_q, d = q.shape
+    h_kv, P = k_cache.shape[1], k_cache.shape[2]
+    dt, dev = _dtype_code(q), q.device
+    _need(q, "q", q.shape, q.dtype)
+    _need(q_slc, "q_slc", (B, h_kv, d), q.dtype, dev)
+    _need(k_cache, "k_cache", (B, h_kv, P, d), q.dtype, dev, host_ok=True)
+    _need(v_cache, "v_cache", (B, h_kv, P, d), q.dtype, dev, host_ok=True)
+    _need(kbar, "kbar", (B, h_kv, P // S, d), torch.float32, dev)
+    if o is None:
+        o = torch.empty_like(q)
+    _need(o, "o", q.shape, q.dtype, dev)
+    idx = torch.empty(B, h_kv, K, dtype=torch.int32, device=dev) if want_sel else None
+    w = torch.empty(B, h_kv, K, dtype=torch.float32, device=dev) if want_sel else None
+    sh = HsaShape(B, P, h_q, h_kv, d, S, K, dt)
+    w_, n = _workspace(sh, OP_DECODE, dev, ws)
+    _check(load_library().hsa_decode_multi(ctypes.byref(sh), NL, _p(q), _p(q_slc), _p(k_cache), _p(v_cache),
+                                           _p(kbar), _p(o), _p(idx), _p(w), _p(w_), n, _stream(stream)),
+           "hsa_decode_multi")
     return o, idx, w
 
 

@@ -318,27 +318,63 @@ hsa_status_t hsa_attend(const hsa_shape_t *shape, const void *q, const void *k, 
     return cuda_status(e);
 }
 
-hsa_status_t hsa_decode(const hsa_shape_t *shape, const void *q, const void *q_slc,
-                        const void *k_cache, const void *v_cache, const float *kbar, void *o,
-                        int32_t *idx, float *w, void *ws, size_t ws_bytes, void *stream) {
+// The address a kernel reads `p` through: device (or managed) memory as is,
+// page-locked host memory through its mapped device address.  Pageable host
+// memory has no such address and is refused before any launch.
+static bool device_view(const void *p, const void **dp) {
+    cudaPointerAttributes a{};
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        (void)cudaGetLastError();  // a plain host pointer: clear the sticky-free error state
+        return false;
+    }
+    if (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) {
+        *dp = p;
+        return true;
+    }
+    if (a.type == cudaMemoryTypeHost && a.devicePointer) {
+        *dp = a.devicePointer;
+        return aligned16(*dp);
+    }
+    return false;
+}
+
+hsa_status_t hsa_decode_multi(const hsa_shape_t *shape, int32_t n_layers, const void *q, const void *q_slc,
+                              const void *k_cache, const void *v_cache, const float *kbar, void *o,
+                              int32_t *idx, float *w, void *ws, size_t ws_bytes, void *stream) {
     hsa_status_t s = check_shape(shape, true);
     if (s != HSA_OK) return s;
+    if (n_layers < 1 || n_layers > HSA_MAX_LAYERS) return HSA_ERR_INVALID_ARG;
     const Shape sh = make_shape(*shape);
     if (sh.B == 0) return empty_call(sh, HSA_OP_DECODE, ws, ws_bytes, static_cast<cudaStream_t>(stream));
     if (!ptrs_ok({q, q_slc, o}) || !opt_ok(idx) || !opt_ok(w)) return HSA_ERR_INVALID_ARG;
     // with no complete cached chunk the caches and the index are never read
     if (sh.nc > 0 && !ptrs_ok({k_cache, v_cache, kbar})) return HSA_ERR_INVALID_ARG;
     if ((s = check_ws(sh, HSA_OP_DECODE, ws, ws_bytes)) != HSA_OK) return s;
+    const void *kc = k_cache, *vc = v_cache;
+    if (sh.nc > 0 && (!device_view(k_cache, &kc) || !device_view(v_cache, &vc))) return HSA_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     DevStatus *ds = static_cast<DevStatus *>(ws);
+    const bool cluster = decode_cluster_supported(sh, n_layers);
     cudaError_t e = clear_status(ws, st);
     if (e == cudaSuccess)
-        e = timed(HSA_K_DECODE, 1, st, [&] {
-            return decode_cluster_supported(sh)
-                       ? launch_decode_cluster(sh, q, q_slc, k_cache, v_cache, kbar, o, idx, w, ds, st)
-                       : launch_decode_simt(sh, q, q_slc, k_cache, v_cache, kbar, o, idx, w, ds, st);
+        e = timed(HSA_K_DECODE, cluster ? 1 : n_layers, st, [&] {
+            if (cluster)
+                return launch_decode_cluster(sh, n_layers, q, q_slc, kc, vc, kbar, o, idx, w, ds, st);
+            // very long caches: token-major kernel, one launch per layer (each repeats the selection)
+            const size_t lbytes = (size_t)sh.B * sh.hq * sh.d * (sh.bf16 ? 2 : 4);
+            cudaError_t r = cudaSuccess;
+            for (int l = 0; l < n_layers && r == cudaSuccess; ++l)
+                r = launch_decode_simt(sh, static_cast<const char *>(q) + l * lbytes, q_slc, kc, vc, kbar,
+                                       static_cast<char *>(o) + l * lbytes, idx, w, ds, st);
+            return r;
         });
     return cuda_status(e);
+}
+
+hsa_status_t hsa_decode(const hsa_shape_t *shape, const void *q, const void *q_slc,
+                        const void *k_cache, const void *v_cache, const float *kbar, void *o,
+                        int32_t *idx, float *w, void *ws, size_t ws_bytes, void *stream) {
+    return hsa_decode_multi(shape, 1, q, q_slc, k_cache, v_cache, kbar, o, idx, w, ws, ws_bytes, stream);
 }
 
 hsa_status_t hsa_bwd(const hsa_shape_t *shape, const void *q, const void *k, const void *v,

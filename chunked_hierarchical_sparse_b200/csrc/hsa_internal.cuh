@@ -107,8 +107,9 @@ cudaError_t launch_decode_simt(const Shape &sh, const void *q, const void *q_slc
                                float *w_out, DevStatus *ds, cudaStream_t st);
 
 // Decode on a thread-block cluster per (b, g) (DSMEM exchange of scores and partials).
-bool decode_cluster_supported(const Shape &sh);
-cudaError_t launch_decode_cluster(const Shape &sh, const void *q, const void *q_slc, const void *kc,
+// NL layers' queries q [NL,B,h_q,d] share the step's selection and chunk reads; o [NL,B,h_q,d].
+bool decode_cluster_supported(const Shape &sh, int NL);
+cudaError_t launch_decode_cluster(const Shape &sh, int NL, const void *q, const void *q_slc, const void *kc,
                                   const void *vc, const float *kbar, void *o, int32_t *idx_out, float *w_out,
                                   DevStatus *ds, cudaStream_t st);
 

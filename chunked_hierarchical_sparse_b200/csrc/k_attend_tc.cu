@@ -357,11 +357,16 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 const float wva = __shfl_sync(0xffffffffu, w_a, src);
                 const float wvb = __shfl_sync(0xffffffffu, w_b, src);
                 const float wgt = (lo + lane < 32) ? wva : wvb;
-                const int t = ent >> 4, slot = ent & 15;
-                if (lane < 16) {
-                    ti_.tok[lane] = (lane < ntok) ? t : -1;
-                    ti_.slot[lane] = (lane < ntok) ? slot : 0;
-                    ti_.w[lane] = (lane < ntok) ? wgt : 0.f;
+                int t = ent >> 4, slot = ent & 15;
+                {  // an entry outside its window (inconsistent lists) is reported and made harmless
+                    const int wsv = (j % P.nW) * P.W;
+                    const bool bad = lane < ntok && (t < wsv || t >= min(P.L, wsv + P.W) || slot >= P.K);
+                    if (bad) { report(ds, HSA_ERR_DEVICE_CHECK, kKAttendTc, t, c); t = wsv; slot = 0; }
+                    if (lane < 16) {
+                        ti_.tok[lane] = (lane < ntok) ? t : -1;
+                        ti_.slot[lane] = (lane < ntok) ? slot : 0;
+                        ti_.w[lane] = (lane < ntok && !bad) ? wgt : 0.f;
+                    }
                 }
                 if (lane == 0) {
                     ti_.type = kItemTile; ti_.j = j; ti_.b = b; ti_.g = g; ti_.c = c; ti_.ntok = ntok;

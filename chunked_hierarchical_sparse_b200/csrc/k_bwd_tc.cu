@@ -325,11 +325,16 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
                 BP_END(3);
                 BTileInfo &ti_ = info[ii];
                 const int ntok = min(TT, e1 - (e0 + tt * TT));
-                const int t = pc.e >> 4, slot = pc.e & 15;
-                if (lane < 16) {
-                    ti_.tok[lane] = (lane < ntok) ? t : -1;
-                    ti_.slot[lane] = (lane < ntok) ? slot : 0;
-                    ti_.w[lane] = (lane < ntok) ? pc.w : 0.f;
+                int t = pc.e >> 4, slot = pc.e & 15;
+                {  // an entry outside its window (inconsistent lists) is reported and made harmless
+                    const int wsv = (j % P.nW) * P.W;
+                    const bool bad = lane < ntok && (t < wsv || t >= min(P.L, wsv + P.W) || slot >= P.K);
+                    if (bad) { report(ds, HSA_ERR_DEVICE_CHECK, kKBwdTc, t, c); t = wsv; slot = 0; }
+                    if (lane < 16) {
+                        ti_.tok[lane] = (lane < ntok) ? t : -1;
+                        ti_.slot[lane] = (lane < ntok) ? slot : 0;
+                        ti_.w[lane] = (lane < ntok && !bad) ? pc.w : 0.f;
+                    }
                 }
                 if (lane == 0) {
                     ti_.type = kBItemTile; ti_.j = j; ti_.b = b; ti_.g = g; ti_.c = c; ti_.ntok = ntok;

@@ -225,7 +225,7 @@ __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
     decode_cluster_kernel(const T *__restrict__ q, const T *__restrict__ q_slc, const T *__restrict__ kc,
                           const T *__restrict__ vc, const float *__restrict__ kbar, T *__restrict__ o,
                           int32_t *__restrict__ idx_out, float *__restrict__ w_out, int P, int hq, int hkv,
-                          int nc, int K, int G) {
+                          int nc, int K, int G, int NL, int64_t lstride) {
     DEC_STAMP(0);
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
@@ -237,8 +237,8 @@ __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
     float *sm = reinterpret_cast<float *>(dsm4);
     const int per = (nc + kDecCta - 1) / kDecCta;     // chunks scored by each CTA
     float *scores = sm;                               // [per]
-    float *part = scores + ((per + 3) & ~3);          // [G][D] partial output of this CTA's slots
-    float *Qs = part + kMaxG * D;                     // [G][D]
+    float *part = scores + ((per + 3) & ~3);          // [NL][G][D] partial outputs of this CTA's slots
+    float *Qs = part + NL * kMaxG * D;                // [G][D] one layer's queries
     float *Ks = Qs + kMaxG * D;                       // [64][D+1]
     float *Vs = Ks + kChunk * (D + 1);                // [64][D]
     float *Pm = Vs + kChunk * D;                      // [G][64]
@@ -285,18 +285,23 @@ __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
     __nv_bfloat16 *Q16 = reinterpret_cast<__nv_bfloat16 *>(Qs);
     __nv_bfloat16 *K16 = reinterpret_cast<__nv_bfloat16 *>(Ks);
     __nv_bfloat16 *V16 = reinterpret_cast<__nv_bfloat16 *>(Vs);
-    if constexpr (kTc) {
-        for (int e = tid; e < 16 * D / 8; e += kDecThreads) {  // heads padded to the MMA's 16 rows
-            const int h = e / (D / 8), j = (e % (D / 8)) * 8;
-            *reinterpret_cast<uint4 *>(Q16 + h * DecTile<D>::QP + j) =
-                (h < G) ? *reinterpret_cast<const uint4 *>(q + ((int64_t)b * hq + (int64_t)g * G + h) * D + j)
-                        : make_uint4(0, 0, 0, 0);
+    // queries of layer l (all layers share this step's selection and chunks)
+    auto load_q = [&](int l) {
+        const T *ql = q + (int64_t)l * lstride + ((int64_t)b * hq + (int64_t)g * G) * D;
+        if constexpr (kTc) {
+            for (int e = tid; e < 16 * D / 8; e += kDecThreads) {  // heads padded to the MMA's 16 rows
+                const int h = e / (D / 8), j = (e % (D / 8)) * 8;
+                *reinterpret_cast<uint4 *>(Q16 + h * DecTile<D>::QP + j) =
+                    (h < G) ? *reinterpret_cast<const uint4 *>(ql + (int64_t)h * D + j) : make_uint4(0, 0, 0, 0);
+            }
+        } else {
+            for (int e = tid; e < G * D; e += kDecThreads)  // a few 2-byte loads per thread, all independent
+                Qs[e] = Elem<T>::load(ql + e);
         }
-    } else {
-        for (int e = tid; e < G * D; e += kDecThreads)  // a few 2-byte loads per thread, all independent
-            Qs[e] = Elem<T>::load(q + ((int64_t)b * hq + (int64_t)g * G) * D + e);
-    }
-    for (int e = tid; e < kMaxG * D; e += kDecThreads) part[e] = 0.f;
+    };
+    load_q(0);
+    int q_cur = 0;  // the layer whose queries Qs / Q16 hold (block-uniform)
+    for (int e = tid; e < NL * kMaxG * D; e += kDecThreads) part[e] = 0.f;
     DEC_STAMP(1);
     cluster.sync();
     DEC_STAMP(2);
@@ -377,11 +382,26 @@ __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
         if constexpr (kTc) {
             load_chunk16<D>(kbase + (int64_t)c * kChunk * D, vbase + (int64_t)c * kChunk * D, K16, V16, tid);
             __syncthreads();
-            attend_chunk16<D>(Q16, K16, V16, part, G, wk, scale, warp, lane);
+            for (int l = 0; l < NL; ++l) {  // the chunk is read once and serves every layer
+                if (l != q_cur) {
+                    __syncthreads();
+                    load_q(l);
+                    q_cur = l;
+                    __syncthreads();
+                }
+                attend_chunk16<D>(Q16, K16, V16, part + l * kMaxG * D, G, wk, scale, warp, lane);
+            }
             continue;
         }
         load_chunk<T, D>(kbase + (int64_t)c * kChunk * D, vbase + (int64_t)c * kChunk * D, Ks, Vs, tid);
         __syncthreads();
+        for (int l = 0; l < NL; ++l) {
+        if (l != q_cur) {
+            load_q(l);
+            q_cur = l;
+            __syncthreads();
+        }
+        float *pl = part + l * kMaxG * D;
         for (int e = tid; e < G * kChunk; e += kDecThreads) {
             const int h = e / kChunk, i = e % kChunk;
             const float *qh = Qs + h * D;
@@ -413,7 +433,9 @@ __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
             float acc = 0.f;
 #pragma unroll 8
             for (int i = 0; i < kChunk; ++i) acc = fmaf(ph[i], Vs[i * D + j], acc);
-            part[e] = fmaf(coef[h], acc, part[e]);
+            pl[e] = fmaf(coef[h], acc, pl[e]);
+        }
+        __syncthreads();  // Qs, Pm and coef are rewritten for the next layer
         }
     }
     DEC_STAMP(4);
@@ -421,13 +443,14 @@ __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
     DEC_STAMP(5);
 
     // ---- 4. sum the partial outputs of the cluster (DSMEM), this CTA's column share
-    const int ncol = G * D;
-    const int cper = (ncol + kDecCta - 1) / kDecCta;
-    for (int e = rank * cper + tid; e < min(ncol, (rank + 1) * cper); e += kDecThreads) {
+    const int ncol = G * D, tot = NL * ncol;
+    const int cper = (tot + kDecCta - 1) / kDecCta;
+    for (int e = rank * cper + tid; e < min(tot, (rank + 1) * cper); e += kDecThreads) {
+        const int l = e / ncol, col = e - l * ncol;
         float acc = 0.f;
 #pragma unroll
-        for (int r = 0; r < kDecCta; ++r) acc += cluster.map_shared_rank(part, r)[e];
-        Elem<T>::store(o + ((int64_t)b * hq + (int64_t)g * G) * D + e, acc);
+        for (int r = 0; r < kDecCta; ++r) acc += cluster.map_shared_rank(part, r)[l * kMaxG * D + col];
+        Elem<T>::store(o + (int64_t)l * lstride + ((int64_t)b * hq + (int64_t)g * G) * D + col, acc);
     }
     DEC_STAMP(6);
     cluster.sync();
@@ -440,39 +463,40 @@ extern "C" HSA_API int hsa_debug_dec_profile(void *dev_buf) {
 }
 #endif
 
-size_t decode_cluster_smem(int nc, int d) {
+size_t decode_cluster_smem(int nc, int d, int NL) {
     const int per = (nc + kDecCta - 1) / kDecCta;
     const size_t ncr = (size_t)((nc + 3) & ~3);
-    return sizeof(float) * ((size_t)((per + 3) & ~3) + 2 * (size_t)kMaxG * d + (size_t)kChunk * (d + 1) +
+    return sizeof(float) * ((size_t)((per + 3) & ~3) + (size_t)(NL + 1) * kMaxG * d + (size_t)kChunk * (d + 1) +
                             (size_t)kChunk * d + (size_t)kMaxG * kChunk + 3 * ncr);
 }
 
 template <typename T, int D>
-static cudaError_t decode_launch(const Shape &sh, const void *q, const void *q_slc, const void *kc, const void *vc,
-                                 const float *kbar, void *o, int32_t *idx_out, float *w_out, cudaStream_t st) {
-    const size_t smem = decode_cluster_smem(sh.nc, D);
+static cudaError_t decode_launch(const Shape &sh, int NL, const void *q, const void *q_slc, const void *kc,
+                                 const void *vc, const float *kbar, void *o, int32_t *idx_out, float *w_out,
+                                 cudaStream_t st) {
+    const size_t smem = decode_cluster_smem(sh.nc, D, NL);
     cudaError_t e = set_smem_once((const void *)decode_cluster_kernel<T, D>, smem);
     if (e != cudaSuccess) return e;
     decode_cluster_kernel<T, D><<<(unsigned)(sh.B * sh.hkv * kDecCta), kDecThreads, smem, st>>>(
         (const T *)q, (const T *)q_slc, (const T *)kc, (const T *)vc, kbar, (T *)o, idx_out, w_out, sh.L, sh.hq,
-        sh.hkv, sh.nc, sh.K, sh.G);
+        sh.hkv, sh.nc, sh.K, sh.G, NL, (int64_t)sh.B * sh.hq * D);
     return cudaGetLastError();
 }
 
-bool decode_cluster_supported(const Shape &sh) {
-    return (sh.d == 64 || sh.d == 128) && sh.G <= kMaxG && sh.K <= kMaxK &&
-           decode_cluster_smem(sh.nc, sh.d) <= 200 * 1024;
+bool decode_cluster_supported(const Shape &sh, int NL) {
+    return (sh.d == 64 || sh.d == 128) && sh.G <= kMaxG && sh.K <= kMaxK && NL >= 1 &&
+           decode_cluster_smem(sh.nc, sh.d, NL) <= 200 * 1024;
 }
 
-cudaError_t launch_decode_cluster(const Shape &sh, const void *q, const void *q_slc, const void *kc,
+cudaError_t launch_decode_cluster(const Shape &sh, int NL, const void *q, const void *q_slc, const void *kc,
                                   const void *vc, const float *kbar, void *o, int32_t *idx_out, float *w_out,
                                   DevStatus *, cudaStream_t st) {
     if (sh.B == 0) return cudaSuccess;
     if (sh.bf16)
-        return sh.d == 128 ? decode_launch<__nv_bfloat16, 128>(sh, q, q_slc, kc, vc, kbar, o, idx_out, w_out, st)
-                           : decode_launch<__nv_bfloat16, 64>(sh, q, q_slc, kc, vc, kbar, o, idx_out, w_out, st);
-    return sh.d == 128 ? decode_launch<float, 128>(sh, q, q_slc, kc, vc, kbar, o, idx_out, w_out, st)
-                       : decode_launch<float, 64>(sh, q, q_slc, kc, vc, kbar, o, idx_out, w_out, st);
+        return sh.d == 128 ? decode_launch<__nv_bfloat16, 128>(sh, NL, q, q_slc, kc, vc, kbar, o, idx_out, w_out, st)
+                           : decode_launch<__nv_bfloat16, 64>(sh, NL, q, q_slc, kc, vc, kbar, o, idx_out, w_out, st);
+    return sh.d == 128 ? decode_launch<float, 128>(sh, NL, q, q_slc, kc, vc, kbar, o, idx_out, w_out, st)
+                       : decode_launch<float, 64>(sh, NL, q, q_slc, kc, vc, kbar, o, idx_out, w_out, st);
 }
 
 }  // namespace hsa

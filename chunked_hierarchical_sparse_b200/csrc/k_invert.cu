@@ -145,7 +145,7 @@ __global__ void __launch_bounds__(256) inv_base_kernel(int32_t *__restrict__ his
         H[e] += off[e % nc];
 }
 
-// One warp per (token block, b*hkv + g): tokens in order, slots in parallel.
+// One warp per (token block, b*hkv + g): entries placed in token order.
 __global__ void __launch_bounds__(32) inv_scatter_kernel(const int32_t *__restrict__ idx,
                                                          const float *__restrict__ w,
                                                          const int32_t *__restrict__ hist,
@@ -169,16 +169,23 @@ __global__ void __launch_bounds__(32) inv_scatter_kernel(const int32_t *__restri
     __syncwarp();
     int32_t *E = entries + (int64_t)bg * L * K;
     float *EW = entw ? entw + (int64_t)bg * L * K : nullptr;
-    for (int t = t0; t < t1; ++t) {
-        if (lane < K) {
-            const int c = sel[(t - t0) * K + lane];
-            if (c >= 0 && c < nc && c < t / kChunk) {
-                const int pos = cur[c];
-                cur[c] = pos + 1;
-                E[pos] = t * 16 + lane;
-                if (EW) EW[pos] = selw[(t - t0) * K + lane];
-            }
+    // 32 / K tokens per step, lane = (token - step start) * K + slot.  Lanes that
+    // hold the same chunk take consecutive positions in lane order, i.e. by token,
+    // then slot (a caller-given selection may list a chunk in several slots).
+    const int tpi = 32 / K;
+    for (int tb = t0; tb < t1; tb += tpi) {
+        const int t = tb + lane / K, kk = lane % K;
+        int c = -1;
+        if (lane < tpi * K && t < t1) c = sel[(t - t0) * K + kk];
+        const bool ok = c >= 0 && c < nc && c < t / kChunk;
+        const unsigned peers = __match_any_sync(0xffffffffu, ok ? c : -1 - lane);
+        if (ok) {
+            const int pos = cur[c] + __popc(peers & ((1u << lane) - 1u));
+            E[pos] = t * 16 + kk;
+            if (EW) EW[pos] = selw[(t - t0) * K + kk];
         }
+        __syncwarp();
+        if (ok && lane == 31 - __clz(peers)) cur[c] += __popc(peers);
         __syncwarp();
     }
 }

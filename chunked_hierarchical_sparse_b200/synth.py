@@ -23,7 +23,7 @@ import numpy as np
 
 # tensor ids for the generator key
 _TID = {"q": 1, "k": 2, "v": 3, "q_slc": 4, "dO": 5, "plant": 6, "offset": 7,
-        "q_dec": 8, "q_slc_dec": 9}
+        "q_dec": 8, "q_slc_dec": 9, "q_layer": 10}
 
 
 @dataclass(frozen=True)
@@ -112,6 +112,16 @@ def make_inputs(wl: Workload, with_dO: bool | None = None) -> dict:
     if with_dO or (with_dO is None and wl.kind == "train"):
         out["dO"] = round_to(normal(wl.seed, "dO", (B, L, hq, d)), wl.dtype)
     return out
+
+
+def layer_queries(wl: Workload, n_layers: int) -> np.ndarray:
+    """Decode queries of n_layers HSA layers that share one selection and KV
+    cache: [n_layers, B, h_q, d]; layer 0 is make_inputs' q, layer l >= 1 is
+    drawn from its own stream."""
+    shape = (wl.B, wl.h_q, wl.d)
+    qs = [round_to(normal(wl.seed, "q_dec", shape), wl.dtype)]
+    qs += [round_to(normal(wl.seed, "q_layer", shape, attempt=l), wl.dtype) for l in range(1, n_layers)]
+    return np.stack(qs)
 
 
 def redraw_q_slc(wl: Workload, q_slc: np.ndarray, rows_bg: np.ndarray, attempt: int) -> None:

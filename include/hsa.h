@@ -151,10 +151,33 @@ HSA_API hsa_status_t hsa_attend(const hsa_shape_t *shape, const void *q, const v
 /* Step a7: one decode step per sequence against the chunk-level index
  * [P1 §training/inference]: shape.L = P (cached tokens); the new token sits at
  * position P, so all floor(P/S) cached chunks are eligible.  kbar is an input
- * (e.g. from hsa_pool over the cache).  idx and w are optional outputs. */
+ * (e.g. from hsa_pool over the cache) and stays in device memory.  idx and w
+ * are optional outputs.
+ * KV cache offloading [P1 §training/inference "KV Cache Offloading"]:
+ * k_cache and v_cache may be device memory or page-locked host memory
+ * (cudaHostAlloc / cudaHostRegister, mapped).  In host memory only the K
+ * selected chunks per (sequence, group) cross the host link, each read once,
+ * straight into the attending thread block's shared memory.  Pageable host
+ * memory is refused with HSA_ERR_INVALID_ARG before any launch. */
 HSA_API hsa_status_t hsa_decode(const hsa_shape_t *shape, const void *q, const void *q_slc,
                         const void *k_cache, const void *v_cache, const float *kbar, void *o,
                         int32_t *idx, float *w, void *ws, size_t ws_bytes, void *stream);
+
+/* Most layers one hsa_decode_multi call serves. */
+#define HSA_MAX_LAYERS 8
+
+/* hsa_decode for n_layers HSA layers that share one chunk selection and one
+ * KV cache [P1 §training/inference: all HSA layers share the retrieval and the
+ * single host-device exchange of a step; P3 "Measured effects" reports the
+ * cost of not sharing].  q and o are [n_layers, B, h_q, d] (layer-major); the
+ * selection comes from q_slc, k_cache, v_cache and kbar as in hsa_decode and
+ * each selected chunk is read once for all layers.  1 <= n_layers <=
+ * HSA_MAX_LAYERS, else HSA_ERR_INVALID_ARG.  hsa_decode is n_layers = 1.
+ * Workspace: hsa_workspace_size(shape, HSA_OP_DECODE). */
+HSA_API hsa_status_t hsa_decode_multi(const hsa_shape_t *shape, int32_t n_layers, const void *q,
+                              const void *q_slc, const void *k_cache, const void *v_cache,
+                              const float *kbar, void *o, int32_t *idx, float *w, void *ws,
+                              size_t ws_bytes, void *stream);
 
 /* Steps a8-a10: backward of hsa_fwd [P1 §kernel, §HSA "end-to-end"].
  * Inputs: the forward's inputs, its lse, idx, w and kbar outputs, and dO.

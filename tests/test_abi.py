@@ -92,6 +92,11 @@ def test_host_validation_without_gpu(lib):
     # shared-selection attend needs idx and w; workspace is the forward's
     assert lib.hsa_attend(ctypes.byref(sh), good, good, good, None, good, good, None, ws, 1 << 30, None) == 1
     assert lib.hsa_attend(ctypes.byref(sh), good, good, good, good, good, good, None, ws, 300, None) == 3
+    # decode for several layers: 1 <= n_layers <= HSA_MAX_LAYERS
+    dsh = _shape()
+    for nl in (0, 9):
+        assert lib.hsa_decode_multi(ctypes.byref(dsh), nl, good, good, good, good, good, good, None, None,
+                                    ws, 1 << 30, None) == 1
     assert lib.hsa_device_status(None, None, None) == 1
     assert lib.hsa_status_string(3) == b"workspace too small"
 

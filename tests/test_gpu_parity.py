@@ -310,6 +310,99 @@ def test_decode_small_edges(P):
     assert_out(f64(o), o_ref, "f32", "o")
 
 
+def test_decode_offloaded_cache_workload():
+    """KV cache in page-locked host memory: only the selected chunks cross the host
+    link.  Same kernel and data as the device-cache run, so the same bits."""
+    wl, (x, kbar, (o_ref, idx_ref, w_ref, gap)) = cached_workload("decode16k")
+    m = hsa()
+    kh = torch.from_numpy(x["k"]).to(torch.bfloat16).pin_memory()
+    vh = torch.from_numpy(x["v"]).to(torch.bfloat16).pin_memory()
+    kb = torch.from_numpy(kbar).to(DEV)
+    q, qs = to_dev(x["q"], "bf16"), to_dev(x["q_slc"], "bf16")
+    o, idx, w = m.hsa_decode(q, qs, kh, vh, kb, wl.K)
+    o_dev, _, _ = m.hsa_decode(q, qs, kh.to(DEV), vh.to(DEV), kb, wl.K)
+    torch.cuda.synchronize()
+    assert np.array_equal(idx.cpu().numpy(), idx_ref)
+    assert_out(f64(o), o_ref, "bf16", "o")
+    assert torch.equal(o, o_dev)
+
+
+def test_decode_refuses_pageable_host_cache():
+    """Pageable host memory has no device address: the binding and the C ABI
+    both refuse it before any launch."""
+    import ctypes
+    wl = synth.Workload("dec", 2, 640, 8, 2, 64, 64, 4, "f32", "iid", "decode", 5)
+    x = synth.make_inputs(wl)
+    m = hsa()
+    kh = torch.from_numpy(x["k"]).float()  # ordinary (pageable) host memory
+    vh = kh.clone()
+    q, qs = to_dev(x["q"], "f32"), to_dev(x["q_slc"], "f32")
+    kb = torch.from_numpy(oracle.pool(x["k"], 64)).to(DEV)
+    with pytest.raises(ValueError, match="page-locked"):
+        m.hsa_decode(q, qs, kh, vh, kb, wl.K)
+    o = torch.empty_like(q)
+    sh = m.HsaShape(wl.B, wl.L, wl.h_q, wl.h_kv, wl.d, 64, wl.K, 0)
+    n = m.hsa_workspace_size(wl.B, wl.L, wl.h_q, wl.h_kv, wl.d, 64, wl.K, torch.float32, m.OP_DECODE)
+    ws = torch.empty(n, dtype=torch.uint8, device=DEV)
+    P = ctypes.c_void_p
+    rc = m.load_library().hsa_decode(ctypes.byref(sh), P(q.data_ptr()), P(qs.data_ptr()), P(kh.data_ptr()),
+                                     P(vh.data_ptr()), P(kb.data_ptr()), P(o.data_ptr()), None, None,
+                                     P(ws.data_ptr()), n, None)
+    assert rc == 1  # HSA_ERR_INVALID_ARG
+    torch.cuda.synchronize()
+
+
+DEC_MULTI = [("decode16k", 3, "dev"), ("decode16k", 4, "host"),
+             (synth.Workload("decf32", 3, 64 * 50 + 9, 8, 2, 128, 64, 16, "f32", "iid", "decode", 31), 8, "dev"),
+             (synth.Workload("decbig", 1, 64 * 5200, 8, 1, 128, 64, 8, "f32", "iid", "decode", 32), 8, "dev")]
+
+
+@pytest.mark.parametrize("case", DEC_MULTI, ids=["bf16-3-dev", "bf16-4-host", "f32-k16-8", "f32-long-8"])
+def test_decode_multi_layer_shared_selection(case):
+    """n_layers queries share one selection and one read of each selected chunk.
+    Each layer matches the oracle's decode with that layer's query, and equals
+    (bit for bit) a single-layer call with the same query."""
+    name, NL, where = case
+    if isinstance(name, str):
+        wl, (x, kbar, (o_ref0, idx_ref, w_ref, gap)) = cached_workload(name)
+    else:
+        wl = name
+        x, kbar, (o_ref0, idx_ref, w_ref, gap) = gap_ruled(wl)
+    qs_np = synth.layer_queries(wl, NL)
+    m = hsa()
+    kc, vc = to_dev(x["k"], wl.dtype), to_dev(x["v"], wl.dtype)
+    if where == "host":
+        kc, vc = kc.cpu().pin_memory(), vc.cpu().pin_memory()
+    kb = torch.from_numpy(kbar).to(DEV)
+    qsl = to_dev(x["q_slc"], wl.dtype)
+    q = to_dev(qs_np, wl.dtype)
+    m.hsa_timing_enable(True)
+    o, idx, w = m.hsa_decode_multi(q, qsl, kc, vc, kb, wl.K)
+    _, n_launch = m.hsa_timing_read("decode")
+    m.hsa_timing_enable(False)
+    torch.cuda.synchronize()
+    assert n_launch == (NL if wl.L >= 64 * 5000 else 1)
+    assert np.array_equal(idx.cpu().numpy(), idx_ref)
+    for l in range(NL):
+        o_ref, i_l, _, _ = oracle.decode(qs_np[l], x["q_slc"], x["k"], x["v"], kbar, wl.S, wl.K)
+        assert np.array_equal(i_l, idx_ref)
+        assert_out(f64(o[l]), o_ref, wl.dtype, f"o[layer {l}]")
+        if n_launch == 1:  # the cluster kernel for both calls: identical arithmetic per layer
+            o1, _, _ = m.hsa_decode(q[l].contiguous(), qsl, kc, vc, kb, wl.K)
+            assert torch.equal(o[l], o1), f"layer {l} differs from its single-layer call"
+
+
+def test_decode_multi_layer_count_bounds():
+    wl = synth.Workload("dec", 1, 640, 8, 2, 64, 64, 4, "f32", "iid", "decode", 6)
+    x = synth.make_inputs(wl)
+    m = hsa()
+    kc, vc = to_dev(x["k"], "f32"), to_dev(x["v"], "f32")
+    kb = torch.from_numpy(oracle.pool(x["k"], 64)).to(DEV)
+    q9 = to_dev(np.stack([x["q"]] * 9), "f32")
+    with pytest.raises(m.HsaError):
+        m.hsa_decode_multi(q9, to_dev(x["q_slc"], "f32"), kc, vc, kb, wl.K)
+
+
 # --------------------------------------------------------------------------- backward
 def run_bwd(wl, x, kbar_np=None):
     m = hsa()

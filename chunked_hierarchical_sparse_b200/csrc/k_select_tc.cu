@@ -26,6 +26,17 @@ namespace hsa {
 
 using namespace sm100;
 
+#ifdef HSA_TC_PROFILE
+__device__ unsigned long long *g_sel_prof = nullptr;  // [4]: total, wait, filter, insert (epilogue thread 0)
+#define SP_DECL unsigned long long sp_acc[4] = {0, 0, 0, 0}; long long sp_t0 = 0;
+#define SP_BEGIN() (sp_t0 = clock64())
+#define SP_END(k) (sp_acc[k] += (unsigned long long)(clock64() - sp_t0))
+#else
+#define SP_DECL
+#define SP_BEGIN() ((void)0)
+#define SP_END(k) ((void)0)
+#endif
+
 namespace {
 
 constexpr int kSelThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue
@@ -80,8 +91,10 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_tc_kernel(
     volatile int *wg_flag = reinterpret_cast<volatile int *>(sm + SL::OFF_BAR + 16 * 8 + 16);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int bg = blockIdx.y, b = bg / hkv, g = bg % hkv;
-    const int t0 = blockIdx.x * 128;
+    // token blocks late in the sequence score the most chunks: they are issued first
+    const int nbg = gridDim.x / ((L + 127) / 128);
+    const int bg = blockIdx.x % nbg, b = bg / hkv, g = bg % hkv;
+    const int t0 = ((L + 127) / 128 - 1 - (int)blockIdx.x / nbg) * 128;
     const int tlast = min(t0 + 128, L) - 1;
     const int ne_max = min(tlast / kChunk, nc);
     const int ntiles = (ne_max + kSelN - 1) / kSelN;
@@ -131,7 +144,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_tc_kernel(
             }
             __syncwarp();
         }
-        if (!ok && lane == 0) report(ds, HSA_ERR_TIMEOUT, kKSelectTc, 1, blockIdx.x);
+        if (!ok && lane == 0) report(ds, HSA_ERR_TIMEOUT, kKSelectTc, 1, t0);
     } else if (warp == 1) {
         // -------------------------------------------------- MMA issuer
         constexpr uint32_t idesc = idesc_bf16_f32(128, kSelN, false, false);
@@ -160,7 +173,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_tc_kernel(
             }
             __syncwarp();
         }
-        if (!ok && lane == 0) report(ds, HSA_ERR_TIMEOUT, kKSelectTc, 2, blockIdx.x);
+        if (!ok && lane == 0) report(ds, HSA_ERR_TIMEOUT, kKSelectTc, 2, t0);
         if (lane == 0) { mma_commit(mma_done); mbar_wait(mma_done, 0, kSelWaitNs); }
         __syncwarp();
     } else {
@@ -185,14 +198,19 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_tc_kernel(
         }
         int wcnt = 0;
         bool ok = true;
+        SP_DECL
+        const long long sp_start = clock64();
+        (void)sp_start;
         for (int i = 0; i < ntiles; ++i) {
             const int s = i & 1;
+            SP_BEGIN();
             int v = 1;
             if (tid == 0) v = mbar_wait(&a_full[s], (i >> 1) & 1, kSelWaitNs) ? 1 : 0;
             const int slot = (wcnt++) & 1;
             if (tid == 0) wg_flag[slot] = v;
             asm volatile("bar.sync 1, 128;" ::: "memory");
             if (!wg_flag[slot]) { ok = false; break; }
+            SP_END(1);
             tc_fence_after();
             const int cbase = i * kSelN;
             for (int q4 = 0; q4 < kSelN / 32; ++q4) {
@@ -200,13 +218,39 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_tc_kernel(
                 tmem_ld32(lane_base + s * kSelN + q4 * 32, sc);
                 tmem_wait_ld();
                 const int c0 = cbase + q4 * 32;
+                if (c0 == 0) {
+                    // the first 32 chunks: nearly all of them enter the (still filling)
+                    // list, so take them in order, without extracting each one
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        const float x = sc[e] * scale;
+                        if (e < ne && sel_beats(x, e, bs[KM - 1], bc[KM - 1])) {
+                            float cs = x;
+                            int cc = e;
+#pragma unroll
+                            for (int k = 0; k < KM; ++k) {
+                                const bool sw = sel_beats(cs, cc, bs[k], bc[k]);
+                                const float ts = bs[k];
+                                const int tc = bc[k];
+                                bs[k] = sw ? cs : ts;
+                                bc[k] = sw ? cc : tc;
+                                cs = sw ? ts : cs;
+                                cc = sw ? tc : cc;
+                            }
+                        }
+                    }
+                    continue;
+                }
                 // cheap pass: which of the 32 candidates beat the current K-th best?
+                SP_BEGIN();
                 uint32_t m = 0;
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                     sc[e] *= scale;
                     if (c0 + e < ne && sel_beats(sc[e], c0 + e, bs[KM - 1], bc[KM - 1])) m |= 1u << e;
                 }
+                SP_END(2);
+                SP_BEGIN();
                 // rare pass: insert them one by one (candidate picked by a select tree on
                 // the bits of its position, so everything stays in registers)
                 while (m) {
@@ -237,12 +281,18 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_tc_kernel(
                         cc = sw ? tc : cc;
                     }
                 }
+                SP_END(3);
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&a_empty[s]);
         }
-        if (!ok && tid == 0) report(ds, HSA_ERR_TIMEOUT, kKSelectTc, 3, blockIdx.x);
+        if (!ok && tid == 0) report(ds, HSA_ERR_TIMEOUT, kKSelectTc, 3, t0);
+#ifdef HSA_TC_PROFILE
+        sp_acc[0] = clock64() - sp_start;
+        if (tid == 0 && g_sel_prof)
+            for (int k = 0; k < 4; ++k) atomicAdd(&g_sel_prof[k], sp_acc[k]);
+#endif
         if (t < L) {
             // most-recent-first: order the chosen chunks by descending index (invalid = -1 last)
 #pragma unroll
@@ -281,6 +331,12 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_tc_kernel(
     tc_fence_after();
     if (warp == 1) tmem_dealloc(tmem, 2 * kSelN);
 }
+
+#ifdef HSA_TC_PROFILE
+extern "C" HSA_API int hsa_debug_sel_profile(void *dev_buf) {
+    return cudaMemcpyToSymbol(g_sel_prof, &dev_buf, sizeof(void *)) == cudaSuccess ? 0 : 4;
+}
+#endif
 
 namespace {
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
@@ -328,7 +384,7 @@ cudaError_t launch_sel(const Shape &sh, const void *q_slc, const float *kbar, __
         !map_bf16(&ml, lo, 2, kd, ksd, kb))
         return cudaErrorInvalidValue;
     const size_t smem = SelSmem<D>::ALLOC;
-    dim3 grid((unsigned)ceil_div(sh.L, 128), (unsigned)(sh.B * sh.hkv));
+    const unsigned grid = (unsigned)(ceil_div(sh.L, 128) * sh.B * sh.hkv);  // 1D: (token block desc, b*hkv + g)
     cudaError_t e;
     if (sh.K <= 8) {
         if ((e = set_smem_once((const void *)select_tc_kernel<D, 8>, smem)) != cudaSuccess) return e;

@@ -231,11 +231,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         acc_inv = __int_as_float((127 - ev) << 23);
     }
 
-    // lane 0 waits, the whole warp gets the verdict (warp-uniform control flow)
+    // every lane waits (converged, sleeping in try_wait); the warp's verdict is a vote
     auto warp_wait = [&](uint64_t *b, uint32_t par) -> bool {
-        int r = 1;
-        if (lane == 0) r = mbar_wait(b, par, kWaitNs) ? 1 : 0;
-        return __shfl_sync(0xffffffffu, r, 0) != 0;
+        return __all_sync(0xffffffffu, mbar_wait(b, par, kWaitNs));
     };
 
     if (warp == kWarpProd) {
@@ -390,7 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                     tma_load_2d(sm + L::OFF_Q + qs * L::QBYTES + lane * G * 128, &tm_q, 0, row, &B.q_full[qs]);
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&B.info_full[ti]);
+                mbar_arrive_lane0(&B.info_full[ti], lane);
                 PROF_END(9);
                 ++qc;
                 ++it;
@@ -487,6 +485,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 } else {
                     if (*abort_flag || globaltimer() - t_last > kWaitNs) { ok = false; break; }
                     PROF_INC(1);
+                    __nanosleep(32);  // leave the issue slots to the working warps meanwhile
                 }
             }
             if (!ok) {
@@ -540,7 +539,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&B.s_empty[sb]);
+            mbar_arrive_lane0(&B.s_empty[sb], lane);
             // P buffer sb is free once the O = P.V of tile tseq - 2 has read it
             PROF_END(3);
             PROF_BEGIN();
@@ -599,12 +598,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             }
             fence_proxy_async_smem();  // each writer orders its P rows before the MMA's reads
             __syncwarp();
-            if (lane == 0) mbar_arrive(&B.p_full[sb]);  // one arrival per warp
+            mbar_arrive_lane0(&B.p_full[sb], lane);  // one arrival per warp
             PROF_END(3);
             // the row's output coefficient w / Z for the epilogue group
             ecoef[ii * 128 + r] = coef;
             __syncwarp();
-            if (lane == 0) mbar_arrive(&coef_full[ii]);
+            mbar_arrive_lane0(&coef_full[ii], lane);
             ++tseq;
             ++it;
         }
@@ -646,11 +645,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         while (ok) {
             const int ii = it % kInfo;
             const uint32_t ipar = (it / kInfo) & 1;
-            if (ecnt > 0) {  // never sit on unpublished tiles while the next one is not there yet
-                int ready = 1;
-                if (lane == 0) ready = mbar_test(&B.info_full[ii], ipar) ? 1 : 0;
-                if (!__shfl_sync(0xffffffffu, ready, 0)) flush();
-            }
+            if (ecnt > 0 && !__all_sync(0xffffffffu, mbar_test(&B.info_full[ii], ipar)))
+                flush();  // never sit on unpublished tiles while the next one is not there yet
             PROF_BEGIN();
             if (!warp_wait(&B.info_full[ii], ipar)) { ok = false; break; }
             PROF_END(1);
@@ -658,7 +654,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             if (inf.type == kItemEnd) break;
             if ((tseq & 1) != eg) {  // the other group's tile: acknowledge the slot and move on
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&B.info_empty[ii]);
+                mbar_arrive_lane0(&B.info_empty[ii], lane);
                 ++tseq;
                 ++it;
                 continue;
@@ -717,10 +713,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&B.o_empty[sb]);
-                mbar_arrive(&B.info_empty[ii]);  // this warp is done with the tile's info entry
-            }
+            mbar_arrive_lane0(&B.o_empty[sb], lane);
+            mbar_arrive_lane0(&B.info_empty[ii], lane);  // this warp is done with the tile's info entry
             PROF_END(3);
             ++ecnt;
             ++tseq;

@@ -26,6 +26,13 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
     asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar))
                  : "memory");
 }
+// One arrival on behalf of the warp: lane 0 arrives, by predication (no branch).
+__device__ __forceinline__ void mbar_arrive_lane0(uint64_t *bar, uint32_t lane) {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.eq.u32 p, %1, 0;\n\t@p mbarrier.arrive.shared::cta.b64 _, [%0];\n\t}" ::"r"(
+                     smem_u32(bar)),
+                 "r"(lane)
+                 : "memory");
+}
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
     asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(
                      smem_u32(bar)),
@@ -48,17 +55,28 @@ __device__ __forceinline__ uint64_t globaltimer() {
     return t;
 }
 
+// Potentially blocking test: the thread may be suspended (issuing nothing) until
+// the phase completes or a hardware time limit passes.
+__device__ __forceinline__ bool mbar_try(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 // Wait for phase `parity` of `bar` to complete, for at most `limit_ns` of wall
 // time.  Returns false when the wait ran out (the caller reports and unwinds).
+// The waiting thread sleeps in try_wait instead of spinning, so a waiting warp
+// leaves the issue slots to the warps that work.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, uint64_t limit_ns) {
-    if (mbar_test(bar, parity)) return true;
+    if (mbar_try(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
-    for (uint32_t it = 1;; ++it) {
-        if (mbar_test(bar, parity)) return true;
-        if ((it & 63) == 0) {
-            if (globaltimer() - t0 > limit_ns) return false;
-            __nanosleep(64);
-        }
+    while (true) {
+        if (mbar_try(bar, parity)) return true;
+        if (globaltimer() - t0 > limit_ns) return false;
     }
 }
 

@@ -237,10 +237,8 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
         acc_inv = __int_as_float((127 - ev) << 23);
     }
 
-    auto warp_wait = [&](uint64_t *b, uint32_t par) -> bool {  // lane 0 waits, the warp gets the verdict
-        int r = 1;
-        if (lane == 0) r = mbar_wait(b, par, kBWaitNs) ? 1 : 0;
-        return __shfl_sync(0xffffffffu, r, 0) != 0;
+    auto warp_wait = [&](uint64_t *b, uint32_t par) -> bool {  // every lane waits; the verdict is a vote
+        return __all_sync(0xffffffffu, mbar_wait(b, par, kBWaitNs));
     };
 
     if (warp == kBWarpProd) {
@@ -354,7 +352,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
                     }
                 }
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&info_full[ii]);
+                mbar_arrive_lane0(&info_full[ii], lane);
                 pc = pn;
                 ++qc;
                 ++it;
@@ -470,8 +468,12 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
                 } else if (s_done) {
                     break;
                 }
-                if (prog) t_last = globaltimer();
-                else if (*abort_flag || globaltimer() - t_last > kBWaitNs) { ok = false; break; }
+                if (prog) {
+                    t_last = globaltimer();
+                } else {
+                    if (*abort_flag || globaltimer() - t_last > kBWaitNs) { ok = false; break; }
+                    __nanosleep(32);  // leave the issue slots to the working warps meanwhile
+                }
 #ifdef HSA_TC_PROFILE
                 if (!prog) ++bp_acc[1];
 #endif
@@ -538,7 +540,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(sd_empty);
+            mbar_arrive_lane0(sd_empty, lane);
             float delta = 0.f;
             if (valid) {
                 // p = exp(x - lse), x = S / sqrt(d);  Delta = sum_i p_i dP_i
@@ -593,7 +595,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
             }
             fence_proxy_async_smem();  // each writer orders its dS / wP rows before the MMA's reads
             __syncwarp();
-            if (lane == 0) mbar_arrive(ds_full);  // one arrival per warp
+            mbar_arrive_lane0(ds_full, lane);  // one arrival per warp
             ++it;
         }
         if (!ok) { *abort_flag = 1; if (tid == 0) report(ds, HSA_ERR_TIMEOUT, kKBwdTc, 5, it); }
@@ -700,7 +702,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&dq_empty[qb]);
+            mbar_arrive_lane0(&dq_empty[qb], lane);
             BP_END(2);
             if (inf.unit_last) {
                 BP_BEGIN();
@@ -723,7 +725,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
                 }
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(dkv_empty);
+                mbar_arrive_lane0(dkv_empty, lane);
                 BP_END(4);
             }
             eg_sync();  // the whole group is done with this tile's info entry

@@ -94,8 +94,9 @@ def read_traffic(kernel_file: str):
     p = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(p):
         return None
-    # the kernel's behaviour also depends on the library's shared configuration header
-    want = source_hash([kernel_file, "chunked_hierarchical_sparse_b200/csrc/hsa_internal.cuh"])
+    # the kernel's behaviour also depends on the library's shared headers
+    want = source_hash([kernel_file, "chunked_hierarchical_sparse_b200/csrc/hsa_internal.cuh",
+                        "chunked_hierarchical_sparse_b200/csrc/sm100.cuh"])
     for ln in open(p):
         m = re.match(r"\s*(\S+)\s+source=(\w+)\s+bytes_per_launch=(\d+)", ln)
         if m and m.group(1) == os.path.basename(kernel_file) and m.group(2) == want:

@@ -366,15 +366,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                         ti_.w[lane] = (lane < ntok && !bad) ? wgt : 0.f;
                     }
                 }
-                if (lane == 0) {
-                    ti_.type = kItemTile; ti_.j = j; ti_.b = b; ti_.g = g; ti_.c = c; ti_.ntok = ntok;
-                    ti_.kvs = kvs; ti_.kvph = kvph; ti_.unit_first = (tt == t0); ti_.unit_last = (tt == t1 - 1);
-                    ti_.qs = qs; ti_.qph = qph;
-                    mbar_arrive_expect_tx(&B.q_full[qs], ntok * L::NH * G * 128);
-                }
+                // the query rows first (their gathers fly while the tile info is written)
+                if (lane == 0) mbar_arrive_expect_tx(&B.q_full[qs], ntok * L::NH * G * 128);
                 __syncwarp();
-                PROF_END(8);
-                PROF_BEGIN();
                 if constexpr (L::NH == 2) {
                     // one 3D box per 8-row group (both 64-column halves): 128 rows = 16 loads
                     constexpr int GPT = G / 8;  // 8-row groups per token
@@ -387,6 +381,14 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                     const int row = (b * P.L + t) * P.hq + g * G;
                     tma_load_2d(sm + L::OFF_Q + qs * L::QBYTES + lane * G * 128, &tm_q, 0, row, &B.q_full[qs]);
                 }
+                if (lane == 0) {
+                    ti_.type = kItemTile; ti_.j = j; ti_.b = b; ti_.g = g; ti_.c = c; ti_.ntok = ntok;
+                    ti_.kvs = kvs; ti_.kvph = kvph; ti_.unit_first = (tt == t0); ti_.unit_last = (tt == t1 - 1);
+                    ti_.qs = qs; ti_.qph = qph;
+                }
+                __syncwarp();
+                PROF_END(8);
+                PROF_BEGIN();
                 __syncwarp();
                 mbar_arrive_lane0(&B.info_full[ti], lane);
                 PROF_END(9);

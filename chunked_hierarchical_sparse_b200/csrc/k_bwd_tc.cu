@@ -177,7 +177,6 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
     uint64_t *mma_done = dkv_empty + 1;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + L::OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 16);
-    volatile int *wg_flag = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 32);  // [2] gradient group
     volatile int *eg_flag = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 40);  // [2] epilogue group
     volatile int *cg_flag = reinterpret_cast<volatile int *>(sm + L::OFF_MISC + 48);  // [2] convert group
 
@@ -498,20 +497,13 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
         const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
         const float L2E = 1.4426950408889634f;
         const float sl2 = scale * L2E;
-        int it = 0, wcnt = 0;
+        int it = 0;
         bool ok = true;
         BP_DECL
-        auto wg_sync = [&]() { asm volatile("bar.sync 1, 128;" ::: "memory"); };
-        auto wg_vote = [&](int v) -> bool {  // thread 0 decides, the whole group follows
-            const int slot = (wcnt++) & 1;
-            if (tid == 0) wg_flag[slot] = v;
-            wg_sync();
-            return wg_flag[slot] != 0;
-        };
+        // every warp of the group waits for itself (converged, sleeping in try_wait);
+        // the warps only meet at the mbarriers they arrive on
         auto wg_wait = [&](uint64_t *b, uint32_t par) -> bool {
-            int v = 1;
-            if (tid == 0) v = mbar_wait(b, par, kBWaitNs) ? 1 : 0;
-            return wg_vote(v);
+            return __all_sync(0xffffffffu, mbar_wait(b, par, kBWaitNs));
         };
         while (ok) {
             const int ii = it % kBInfo;

@@ -12,53 +12,61 @@
 namespace hsa {
 
 // ------------------------------------------------------------------ pooling
-// One block per (b, g, chunk).  16-byte vector loads along d; each thread sums
-// its columns over a strided set of the chunk's rows in fp64, the partial sums
-// are combined in shared memory, and the mean is rounded once to fp32.  The
-// fp64 sum of 64 bf16 values is exact, so the result does not depend on the
-// summation order.
+// One warp per (b, g, chunk).  A lane owns VEC = 16 / sizeof(T) columns (one
+// 16-byte load per row) and 64 / RS of the chunk's rows (RS = 32 / (d / VEC)
+// row parts per warp); it sums them in fp64 with eight loads in flight, the row
+// parts are combined by shuffles, and the mean is rounded once to fp32.  The
+// fp64 sum of 64 bf16 (or fp32) values of one tensor is exact, so the result
+// does not depend on the summation order.
 template <typename T>
 __global__ void __launch_bounds__(256) pool_kernel(const T *__restrict__ k, float *__restrict__ kbar,
-                                                   int L, int d, int nc) {
+                                                   int L, int d, int nc, int64_t nchunks) {
     constexpr int VEC = 16 / sizeof(T);
-    __shared__ double red[256 * VEC];
-    const int64_t bgc = blockIdx.x;
+    const int lane = threadIdx.x & 31;
+    const int64_t bgc = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;  // this warp's chunk
+    if (bgc >= nchunks) return;
+    const int tpc = d / VEC;      // lanes per row (8, 16 or 32)
+    const int rs = 32 / tpc;      // row parts
+    const int lr = lane % tpc, part = lane / tpc;
+    const int rows = kChunk / rs;
     const int c = (int)(bgc % nc);
     const int64_t bg = bgc / nc;
-    const T *src = k + (bg * L + (int64_t)c * kChunk) * d;
-    const int lanes_per_row = d / VEC;
-    const int rows_par = blockDim.x / lanes_per_row;
-    const int lr = threadIdx.x % lanes_per_row;
-    const int r0 = threadIdx.x / lanes_per_row;
+    const T *src = k + ((bg * L + (int64_t)c * kChunk + (int64_t)part * rows) * d) + lr * VEC;
     double acc[VEC];
 #pragma unroll
     for (int e = 0; e < VEC; ++e) acc[e] = 0.0;
-    if (r0 < rows_par) {
-        for (int r = r0; r < kChunk; r += rows_par) {
-            const uint4 raw = *reinterpret_cast<const uint4 *>(src + (int64_t)r * d + lr * VEC);
-            const T *vals = reinterpret_cast<const T *>(&raw);
+    for (int r0 = 0; r0 < rows; r0 += 8) {
+        uint4 raw[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) raw[u] = __ldcs(reinterpret_cast<const uint4 *>(src + (int64_t)(r0 + u) * d));
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const T *vals = reinterpret_cast<const T *>(&raw[u]);
 #pragma unroll
             for (int e = 0; e < VEC; ++e) acc[e] += (double)Elem<T>::load(vals + e);
         }
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) red[r0 * d + lr * VEC + e] = acc[e];
     }
-    __syncthreads();
-    for (int j = threadIdx.x; j < d; j += blockDim.x) {
-        double s = 0.0;
-        for (int r = 0; r < rows_par; ++r) s += red[r * d + j];
-        kbar[bgc * d + j] = (float)(s / kChunk);
+    for (int off = tpc; off < 32; off <<= 1)
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+    if (part == 0) {
+        float out[VEC];
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) out[e] = (float)(acc[e] / kChunk);
+        float4 *dst = reinterpret_cast<float4 *>(kbar + bgc * d + lr * VEC);
+#pragma unroll
+        for (int e = 0; e < VEC / 4; ++e) dst[e] = make_float4(out[4 * e], out[4 * e + 1], out[4 * e + 2], out[4 * e + 3]);
     }
 }
 
 cudaError_t launch_pool(const Shape &sh, const void *k, float *kbar, DevStatus *, cudaStream_t st) {
-    const int64_t blocks = (int64_t)sh.B * sh.hkv * sh.nc;
-    if (blocks == 0) return cudaSuccess;
+    const int64_t chunks = (int64_t)sh.B * sh.hkv * sh.nc;
+    if (chunks == 0) return cudaSuccess;
+    const unsigned blocks = (unsigned)ceil_div(chunks, 8);  // 8 warps = 8 chunks per block
     if (sh.bf16)
-        pool_kernel<__nv_bfloat16><<<(unsigned)blocks, 256, 0, st>>>(
-            (const __nv_bfloat16 *)k, kbar, sh.L, sh.d, sh.nc);
+        pool_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>((const __nv_bfloat16 *)k, kbar, sh.L, sh.d, sh.nc, chunks);
     else
-        pool_kernel<float><<<(unsigned)blocks, 256, 0, st>>>((const float *)k, kbar, sh.L, sh.d, sh.nc);
+        pool_kernel<float><<<blocks, 256, 0, st>>>((const float *)k, kbar, sh.L, sh.d, sh.nc, chunks);
     return cudaGetLastError();
 }
 

@@ -668,18 +668,19 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
             uint4 *xs4 = reinterpret_cast<uint4 *>(xs);
 #pragma unroll kBEpiUnroll
             for (int q = 0; q < D / 64; ++q) {  // 64 columns = one 128-byte fp16 line per row
-#pragma unroll kBEpiUnroll
-                for (int hv = 0; hv < 2; ++hv) {  // 32 columns at a time: 4 chunks of 8 halves
-                    float v[32];
-                    tmem_ld32(lane_base + kColDQ + qb * 128 + q * 64 + hv * 32, v);
-                    tmem_wait_ld();
+                float v[2][32];                   // both 32-column loads in flight, one wait
+                tmem_ld32(lane_base + kColDQ + qb * 128 + q * 64, v[0]);
+                tmem_ld32(lane_base + kColDQ + qb * 128 + q * 64 + 32, v[1]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int hv = 0; hv < 2; ++hv) {  // 4 chunks of 8 halves each
 #pragma unroll
                     for (int c4 = 0; c4 < 4; ++c4) {
                         const int ch = hv * 4 + c4;
                         __half2 h[4];
 #pragma unroll
                         for (int e = 0; e < 4; ++e)
-                            h[e] = __floats2half2_rn(v[c4 * 8 + 2 * e] * cf, v[c4 * 8 + 2 * e + 1] * cf);
+                            h[e] = __floats2half2_rn(v[hv][c4 * 8 + 2 * e] * cf, v[hv][c4 * 8 + 2 * e + 1] * cf);
                         xs4[lane * 8 + (ch ^ (lane & 7))] = *reinterpret_cast<uint4 *>(h);
                     }
                 }

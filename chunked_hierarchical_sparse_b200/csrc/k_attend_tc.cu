@@ -704,6 +704,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                         xs4[lane * 8 + (ch ^ (lane & 7))] = *reinterpret_cast<uint4 *>(h);
                     }
                 }
+                if (q == D / 64 - 1) {  // O read completely: hand the buffer back before the last reductions
+                    tc_fence_before();
+                    __syncwarp();
+                    mbar_arrive_lane0(&B.o_empty[sb], lane);
+                }
                 __syncwarp();
 #pragma unroll
                 for (int m = 0; m < 8; ++m) {
@@ -713,9 +718,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 }
                 __syncwarp();
             }
-            tc_fence_before();
-            __syncwarp();
-            mbar_arrive_lane0(&B.o_empty[sb], lane);
             mbar_arrive_lane0(&B.info_empty[ii], lane);  // this warp is done with the tile's info entry
             PROF_END(3);
             ++ecnt;

@@ -684,6 +684,11 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
                         xs4[lane * 8 + (ch ^ (lane & 7))] = *reinterpret_cast<uint4 *>(h);
                     }
                 }
+                if (q == D / 64 - 1) {  // dQ read completely: hand the buffer back before the last reductions
+                    tc_fence_before();
+                    __syncwarp();
+                    mbar_arrive_lane0(&dq_empty[qb], lane);
+                }
                 __syncwarp();
 #pragma unroll
                 for (int m = 0; m < 8; ++m) {
@@ -693,9 +698,6 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
                 }
                 __syncwarp();
             }
-            tc_fence_before();
-            __syncwarp();
-            mbar_arrive_lane0(&dq_empty[qb], lane);
             BP_END(2);
             if (inf.unit_last) {
                 BP_BEGIN();

@@ -74,6 +74,9 @@ constexpr int kThreads = 512;
 constexpr int kWarpEpi = 4, kWarpConv = 12, kWarpProd = 14, kWarpMma = 15;
 constexpr int kConvThreads = 64;
 constexpr int kInfo = 8;                 // tile-info ring entries
+constexpr int kQStages = 3;              // query-tile buffers (P lives in TMEM, not SMEM)
+// TMEM columns: S[2] 0..127 (fp32), O[2] 128..383 (fp32), P[2] 384..447 (bf16 pairs)
+constexpr uint32_t kColO = 128, kColP = 384;
 #ifndef HSA_WAIT_NS
 #define HSA_WAIT_NS 2000000000ull
 #endif
@@ -101,16 +104,14 @@ template <int D> struct Smem {
     static constexpr int QBYTES = NH * QHALF;
     static constexpr int KVHALF = 64 * 128;
     static constexpr int KVBYTES = NH * KVHALF;
-    static constexpr int PBYTES = 128 * 128;
     static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = OFF_Q + 2 * QBYTES;
+    static constexpr int OFF_K = OFF_Q + kQStages * QBYTES;
     static constexpr int OFF_V = OFF_K + 2 * KVBYTES;
-    static constexpr int OFF_P = OFF_V + 2 * KVBYTES;
-    static constexpr int OFF_X = OFF_P + 2 * PBYTES;            // epilogue transpose scratch, 4 KB per warp
+    static constexpr int OFF_X = OFF_V + 2 * KVBYTES;           // epilogue transpose scratch, 4 KB per warp
     static constexpr int OFF_COEF = OFF_X + 8 * 4096;           // [kInfo][128] fp32 row coefficients w / Z
     static constexpr int OFF_INFO = OFF_COEF + kInfo * 128 * 4;
     static constexpr int OFF_BAR = OFF_INFO + kInfo * (int)sizeof(TileInfo);
-    static constexpr int NBAR = 3 * kInfo + 2 * 2 + 2 * 2 + 2 * 2 + 2 + 2 * 2 + 1 + 2;
+    static constexpr int NBAR = 3 * kInfo + 2 * kQStages + 2 * 2 + 2 * 2 + 2 + 2 * 2 + 1 + 2;
     static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
     static constexpr int BYTES = OFF_MISC + 64;
     static constexpr int ALLOC = BYTES + 1024;  // slack for 1 KB alignment
@@ -120,7 +121,7 @@ static_assert(Smem<128>::ALLOC <= 227 * 1024, "attention tile buffers exceed the
 
 struct Bars {
     uint64_t *info_full, *info_empty;  // [kInfo]
-    uint64_t *q_full, *q_empty;        // [2]
+    uint64_t *q_full, *q_empty;        // [kQStages]
     uint64_t *kv_full, *kv_empty;      // [2]
     uint64_t *s_full, *s_empty;        // [2]
     uint64_t *p_full;                  // [2]
@@ -172,8 +173,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + L::OFF_BAR);
     Bars B;
     B.info_full = bar; B.info_empty = bar + kInfo;
-    B.q_full = bar + 2 * kInfo; B.q_empty = B.q_full + 2;
-    B.kv_full = B.q_empty + 2; B.kv_empty = B.kv_full + 2;
+    B.q_full = bar + 2 * kInfo; B.q_empty = B.q_full + kQStages;
+    B.kv_full = B.q_empty + kQStages; B.kv_empty = B.kv_full + 2;
     B.s_full = B.kv_empty + 2; B.s_empty = B.s_full + 2;
     B.p_full = B.s_empty + 2;
     B.o_full = B.p_full + 2; B.o_empty = B.o_full + 2;
@@ -188,8 +189,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if (threadIdx.x == 0) {
         for (int i = 0; i < kInfo; ++i) { mbar_init(&B.info_full[i], 1); mbar_init(&B.info_empty[i], 1 + 8); }
+        for (int i = 0; i < kQStages; ++i) { mbar_init(&B.q_full[i], 1); mbar_init(&B.q_empty[i], 1); }
         for (int i = 0; i < 2; ++i) {
-            mbar_init(&B.q_full[i], 1); mbar_init(&B.q_empty[i], 1);
             mbar_init(&B.kv_full[i], 1); mbar_init(&B.kv_empty[i], 1);
             mbar_init(&B.s_full[i], 1); mbar_init(&B.s_empty[i], 4);
             mbar_init(&B.p_full[i], 4);
@@ -338,9 +339,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 PROF_BEGIN();
                 if (it >= kInfo && !warp_wait(&B.info_empty[ti], ((it / kInfo) - 1) & 1)) { ok = false; break; }
                 PROF_END(2);
-                const int qs = qc & 1, qph = (qc >> 1) & 1;
+                const int qs = qc % kQStages, qph = (qc / kQStages) & 1;
                 PROF_BEGIN();
-                if (qc >= 2 && !warp_wait(&B.q_empty[qs], ((qc >> 1) - 1) & 1)) { ok = false; break; }
+                if (qc >= kQStages && !warp_wait(&B.q_empty[qs], ((qc / kQStages) - 1) & 1)) { ok = false; break; }
                 PROF_END(5);
                 PROF_INC(7);
                 PROF_BEGIN();
@@ -401,9 +402,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             if (lane == 0) {
                 report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 2, it);
                 // let the loads already issued land before the CTA goes away (bounded)
-                for (int s2 = 0; s2 < 2; ++s2) {
-                    if (qc > s2) mbar_wait(&B.q_full[(qc - 1 - s2) & 1], ((qc - 1 - s2) >> 1) & 1, kWaitNs);
-                    if (kvc > s2) mbar_wait(&B.kv_full[(kvc - 1 - s2) & 1], ((kvc - 1 - s2) >> 1) & 1, kWaitNs);
+                for (int s2 = 0; s2 < kQStages; ++s2) {
+                    if (qc > s2) mbar_wait(&B.q_full[(qc - 1 - s2) % kQStages], ((qc - 1 - s2) / kQStages) & 1, kWaitNs);
+                    if (s2 < 2 && kvc > s2) mbar_wait(&B.kv_full[(kvc - 1 - s2) & 1], ((kvc - 1 - s2) >> 1) & 1, kWaitNs);
                 }
             }
             __syncwarp();
@@ -465,13 +466,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                     if (mbar_test(&B.p_full[pb], (tp >> 1) & 1) &&
                         (tp < 2 || mbar_test(&B.o_empty[pb], ((tp >> 1) - 1) & 1))) {
                         tc_fence_after();
-                        const uint32_t pa = smem_u32(sm + L::OFF_P + pb * L::PBYTES);
+                        const uint32_t pa = tmem + kColP + pb * 32;  // P: 64 keys as 32 bf16 pairs per row
                         const uint32_t vb = smem_u32(sm + L::OFF_V + inf.kvs * L::KVBYTES);
-                        const uint32_t dcol = tmem + 128 + pb * 128;
+                        const uint32_t dcol = tmem + kColO + pb * 128;
 #pragma unroll
-                        for (int ks = 0; ks < 4; ++ks)
-                            mma_bf16_ss(dcol, smem_desc_sw128(pa + ks * 32, 16, 1024),
-                                        smem_desc_sw128(vb + ks * 2048, L::KVHALF, 1024), idesc2, ks > 0);
+                        for (int ks = 0; ks < 4; ++ks)  // 16 keys = 8 TMEM columns per step
+                            mma_bf16_ts(dcol, pa + ks * 8, smem_desc_sw128(vb + ks * 2048, L::KVHALF, 1024), idesc2,
+                                        ks > 0);
                         mma_commit(&B.o_full[pb]);
                         mma_commit(&p_empty[pb]);
                         if (inf.unit_last) mma_commit(&B.kv_empty[inf.kvs]);
@@ -550,7 +551,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             PROF_BEGIN();
             const int ti = r / G, hh = r % G;
             const bool valid = ti < inf.ntok;
-            uint8_t *prow = sm + L::OFF_P + sb * L::PBYTES + r * 128;
+            uint32_t pr[32];  // this row's P: key pairs (2j, 2j+1) as bf16x2, the lower key in the low half
             float coef = 0.f;
             if (valid) {
                 const int t = inf.tok[ti], slot = inf.slot[ti];
@@ -583,22 +584,20 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 coef = inf.w[ti] / z;
                 if (lse) lse[(((int64_t)inf.b * P.L + t) * P.hq + inf.g * G + hh) * P.K + slot] = m + logf(z);
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) {
-                    const float *src = (ch < 4) ? (x0 + ch * 8) : (x1 + (ch - 4) * 8);
-                    uint4 pk;
-                    __nv_bfloat162 a0 = __floats2bfloat162_rn(src[0], src[1]);
-                    __nv_bfloat162 a1 = __floats2bfloat162_rn(src[2], src[3]);
-                    __nv_bfloat162 a2 = __floats2bfloat162_rn(src[4], src[5]);
-                    __nv_bfloat162 a3 = __floats2bfloat162_rn(src[6], src[7]);
-                    pk.x = *reinterpret_cast<uint32_t *>(&a0); pk.y = *reinterpret_cast<uint32_t *>(&a1);
-                    pk.z = *reinterpret_cast<uint32_t *>(&a2); pk.w = *reinterpret_cast<uint32_t *>(&a3);
-                    *reinterpret_cast<uint4 *>(prow + ((ch ^ (r & 7)) << 4)) = pk;
+                for (int j = 0; j < 16; ++j) {
+                    const __nv_bfloat162 a = __floats2bfloat162_rn(x0[2 * j], x0[2 * j + 1]);
+                    const __nv_bfloat162 c = __floats2bfloat162_rn(x1[2 * j], x1[2 * j + 1]);
+                    pr[j] = *reinterpret_cast<const uint32_t *>(&a);
+                    pr[16 + j] = *reinterpret_cast<const uint32_t *>(&c);
                 }
             } else {
 #pragma unroll
-                for (int ch = 0; ch < 8; ++ch) *reinterpret_cast<uint4 *>(prow + (ch << 4)) = make_uint4(0, 0, 0, 0);
+                for (int j = 0; j < 32; ++j) pr[j] = 0u;
             }
-            fence_proxy_async_smem();  // each writer orders its P rows before the MMA's reads
+            // P into its TMEM buffer (the A operand of O = P.V), then handed to the MMA issuer
+            tmem_st32(lane_base + kColP + sb * 32, pr);
+            tmem_wait_st();
+            tc_fence_before();
             __syncwarp();
             mbar_arrive_lane0(&B.p_full[sb], lane);  // one arrival per warp
             PROF_END(3);
@@ -692,7 +691,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
 #pragma unroll kEpiUnroll
                 for (int hv = 0; hv < 2; ++hv) {  // 32 columns at a time: 4 chunks of 8 halves
                     float v[32];
-                    tmem_ld32(lane_base + 128 + sb * 128 + q * 64 + hv * 32, v);
+                    tmem_ld32(lane_base + kColO + sb * 128 + q * 64 + hv * 32, v);
                     tmem_wait_ld();
 #pragma unroll
                     for (int c4 = 0; c4 < 4; ++c4) {

@@ -250,8 +250,7 @@ __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
     __shared__ int tmax_c[kDecThreads];
     __shared__ float top_s[kMaxK];
     __shared__ int top_c[kMaxK];
-    __shared__ float thr_s;
-    __shared__ int thr_c, n_surv;
+    __shared__ int n_surv;
     __shared__ int slot_c[kMaxK];
     __shared__ float slot_w[kMaxK];
     __shared__ float coef[kMaxG];
@@ -316,22 +315,33 @@ __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
         allsc[c] = sc;
         if (beats(sc, c, bs, bc)) { bs = sc; bc = c; }
     }
-    tmax_s[tid] = bs;
-    tmax_c[tid] = bc;
-    if (tid == 0) { thr_s = -CUDART_INF_F; thr_c = -1; n_surv = 0; }
-    __syncthreads();
-    // 2b. threshold: the K-th best of the per-thread bests, a lower bound of the K-th best
-    //     score (the K best per-thread bests are K distinct candidates)
-    if (bc >= 0) {
-        int rk = 0;
-        for (int j = 0; j < kDecThreads; ++j) rk += beats(tmax_s[j], tmax_c[j], bs, bc) ? 1 : 0;
-        if (rk == K - 1) { thr_s = bs; thr_c = bc; }
+    // 2b. threshold: each warp sorts its 32 per-thread bests, best first (bitonic network
+    //     over the lanes); its K-th is a lower bound of the overall K-th best score (the
+    //     warp holds K distinct candidates at least as good), and the threshold is the
+    //     best of the warps' bounds
+    {
+        float s = bs;
+        int c = bc;
+#pragma unroll
+        for (int k = 2; k <= 32; k <<= 1)
+#pragma unroll
+            for (int j = k >> 1; j > 0; j >>= 1) {
+                const float os = __shfl_xor_sync(0xffffffffu, s, j);
+                const int oc = __shfl_xor_sync(0xffffffffu, c, j);
+                const bool keep_better = ((lane & j) == 0) == ((lane & k) == 0);
+                if (keep_better == beats(os, oc, s, c)) { s = os; c = oc; }
+            }
+        if (lane == K - 1) { tmax_s[warp] = s; tmax_c[warp] = c; }
     }
+    if (tid == 0) n_surv = 0;
     __syncthreads();
     // 2c. survivors: the candidates that the threshold does not beat
     {
-        const float ts = thr_s;
-        const int tc = thr_c;
+        float ts = tmax_s[0];
+        int tc = tmax_c[0];
+#pragma unroll
+        for (int q = 1; q < kDecThreads / 32; ++q)
+            if (beats(tmax_s[q], tmax_c[q], ts, tc)) { ts = tmax_s[q]; tc = tmax_c[q]; }
         for (int c = tid; c < nc; c += kDecThreads) {
             const float sc = allsc[c];
             if (!beats(ts, tc, sc, c)) {

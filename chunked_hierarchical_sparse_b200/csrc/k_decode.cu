@@ -220,6 +220,20 @@ __device__ __forceinline__ void attend_chunk16(const __nv_bfloat16 *Q16, const _
     }
 }
 
+// Sorts one (score, chunk) pair per lane across the warp, best first under `beats`
+// (bitonic network over the 32 lanes).
+__device__ __forceinline__ void warp_sort_best_first(float &s, int &c, int lane) {
+#pragma unroll
+    for (int k = 2; k <= 32; k <<= 1)
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            const float os = __shfl_xor_sync(0xffffffffu, s, j);
+            const int oc = __shfl_xor_sync(0xffffffffu, c, j);
+            const bool keep_better = ((lane & j) == 0) == ((lane & k) == 0);
+            if (keep_better == beats(os, oc, s, c)) { s = os; c = oc; }
+        }
+}
+
 template <typename T, int D>
 __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
     decode_cluster_kernel(const T *__restrict__ q, const T *__restrict__ q_slc, const T *__restrict__ kc,
@@ -310,10 +324,16 @@ __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
     // 2a. stage every score; each thread keeps the best of its candidates
     float bs = -CUDART_INF_F;
     int bc = -1;
-    for (int c = tid; c < nc; c += kDecThreads) {
-        const float sc = cluster.map_shared_rank(scores, c / per)[c % per];
-        allsc[c] = sc;
-        if (beats(sc, c, bs, bc)) { bs = sc; bc = c; }
+    for (int c = tid; c < nc; c += 2 * kDecThreads) {  // two remote reads in flight at a time
+        const int c2 = c + kDecThreads;
+        const float s1 = cluster.map_shared_rank(scores, c / per)[c % per];
+        const float s2 = (c2 < nc) ? cluster.map_shared_rank(scores, c2 / per)[c2 % per] : -CUDART_INF_F;
+        allsc[c] = s1;
+        if (beats(s1, c, bs, bc)) { bs = s1; bc = c; }
+        if (c2 < nc) {
+            allsc[c2] = s2;
+            if (beats(s2, c2, bs, bc)) { bs = s2; bc = c2; }
+        }
     }
     // 2b. threshold: each warp sorts its 32 per-thread bests, best first (bitonic network
     //     over the lanes); its K-th is a lower bound of the overall K-th best score (the
@@ -322,15 +342,7 @@ __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
     {
         float s = bs;
         int c = bc;
-#pragma unroll
-        for (int k = 2; k <= 32; k <<= 1)
-#pragma unroll
-            for (int j = k >> 1; j > 0; j >>= 1) {
-                const float os = __shfl_xor_sync(0xffffffffu, s, j);
-                const int oc = __shfl_xor_sync(0xffffffffu, c, j);
-                const bool keep_better = ((lane & j) == 0) == ((lane & k) == 0);
-                if (keep_better == beats(os, oc, s, c)) { s = os; c = oc; }
-            }
+        warp_sort_best_first(s, c, lane);
         if (lane == K - 1) { tmax_s[warp] = s; tmax_c[warp] = c; }
     }
     if (tid == 0) n_surv = 0;
@@ -352,21 +364,34 @@ __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
         }
     }
     __syncthreads();
-    // 2d. rank the survivors; the K best take their place by rank
+    // 2d. the K best survivors, best first: with at most 32 survivors (the usual case)
+    //     warp 0 sorts them in registers; otherwise every survivor is ranked pairwise
     const int ns = n_surv;
-    for (int i = tid; i < ns; i += kDecThreads) {
-        const float si = surv_s[i];
-        const int ci = surv_c[i];
-        int rk = 0;
-        for (int j = 0; j < ns; ++j) rk += beats(surv_s[j], surv_c[j], si, ci) ? 1 : 0;
-        if (rk < K) { top_s[rk] = si; top_c[rk] = ci; }
+    if (ns > 32) {
+        for (int i = tid; i < ns; i += kDecThreads) {
+            const float si = surv_s[i];
+            const int ci = surv_c[i];
+            int rk = 0;
+            for (int j = 0; j < ns; ++j) rk += beats(surv_s[j], surv_c[j], si, ci) ? 1 : 0;
+            if (rk < K) { top_s[rk] = si; top_c[rk] = ci; }
+        }
+        __syncthreads();
     }
-    __syncthreads();
     // 2e. warp 0: most-recent-first order and the stick-breaking weights
     if (warp == 0) {
         const int nsel = min(K, ns);
-        float ls = (lane < nsel) ? top_s[lane] : -CUDART_INF_F;
-        int lc = (lane < nsel) ? top_c[lane] : -1;
+        float ls, lc_s;
+        int lc;
+        if (ns > 32) {
+            ls = (lane < nsel) ? top_s[lane] : -CUDART_INF_F;
+            lc = (lane < nsel) ? top_c[lane] : -1;
+        } else {
+            lc_s = (lane < ns) ? surv_s[lane] : -CUDART_INF_F;
+            lc = (lane < ns) ? surv_c[lane] : -1;
+            warp_sort_best_first(lc_s, lc, lane);
+            ls = (lane < nsel) ? lc_s : -CUDART_INF_F;
+            if (lane >= nsel) lc = -1;
+        }
         int sc_; float sw, ss;
         topk_finish(K, ls, lc, sc_, sw, ss);
         if (lane < K) {

@@ -271,7 +271,7 @@ static cudaError_t run_attend(const Shape &sh, const void *q, const void *k, con
         e = timed(HSA_K_PLAN, 1, st, [&] { return launch_wsum(sh, f.idx, f.w, f.plan.counters + 3 * f.plan.J + 2, st); });
     if (e == cudaSuccess)
         e = timed(HSA_K_ATTEND_TC, 1, st, [&] {
-            return launch_attend_tc(sh, f.plan, f.inv, q, k, v, f.idx, f.w, f.acc, o, lse, ds, st);
+            return launch_attend_tc(sh, f.plan, f.inv, q, k, v, f.acc, o, lse, ds, st);
         });
     return e;
 }

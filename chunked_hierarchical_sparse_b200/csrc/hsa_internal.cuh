@@ -214,8 +214,8 @@ cudaError_t launch_select_tc(const Shape &sh, const void *q_slc, const float *kb
 cudaError_t launch_plan(const Shape &sh, const BwdWs &inv, const AttendPlan &plan, cudaStream_t st);
 bool attend_tc_supported(const Shape &sh);
 cudaError_t launch_attend_tc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv, const void *q,
-                             const void *k, const void *v, const int32_t *idx, const float *w,
-                             __half *acc, void *o, float *lse, DevStatus *ds, cudaStream_t st);
+                             const void *k, const void *v, __half *acc, void *o, float *lse, DevStatus *ds,
+                             cudaStream_t st);
 // max|v| over the whole value tensor, as float bits, max-ed into *bits (zeroed by the caller)
 cudaError_t launch_vmax(const Shape &sh, const void *v, int32_t *bits, cudaStream_t st);
 cudaError_t launch_wsum(const Shape &sh, const int32_t *idx, const float *w, int32_t *bits, cudaStream_t st);

@@ -161,9 +161,8 @@ template <int D, int G>
 __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
     const __grid_constant__ CUtensorMap tm_v,
-    const __grid_constant__ AttendPlan P, const int32_t *__restrict__ hist,
-    const int32_t *__restrict__ chunk_off, const int32_t *__restrict__ entries,
-    const int32_t *__restrict__ idx, const float *__restrict__ entw, __half *__restrict__ acc,
+    const __grid_constant__ AttendPlan P, const int32_t *__restrict__ entries,
+    const float *__restrict__ entw, __half *__restrict__ acc,
     __nv_bfloat16 *__restrict__ out, float *__restrict__ lse, DevStatus *ds) {
     using L = Smem<D>;
     constexpr int TT = 128 / G;
@@ -870,8 +869,7 @@ bool make_map_q3(CUtensorMap *m, const void *base, uint64_t rows) {
 
 template <int D, int G>
 cudaError_t launch_tc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv, const void *q, const void *k,
-                      const void *v, const int32_t *idx, const float *w, __half *acc, void *o,
-                      float *lse, DevStatus *ds, cudaStream_t st) {
+                      const void *v, __half *acc, void *o, float *lse, DevStatus *ds, cudaStream_t st) {
     CUtensorMap mq, mk, mv;
     const bool qok = D == 128 ? make_map_q3(&mq, q, (uint64_t)sh.B * sh.L * sh.hq)
                               : make_map(&mq, q, D, (uint64_t)sh.B * sh.L * sh.hq, G);
@@ -885,8 +883,8 @@ cudaError_t launch_tc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv,
     int dev = 0, sms = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    attend_tc_kernel<D, G><<<sms, kThreads, smem, st>>>(mq, mk, mv, plan, inv.hist, inv.chunk_off, inv.entries,
-                                                        idx, inv.entw, acc, (__nv_bfloat16 *)o, lse, ds);
+    attend_tc_kernel<D, G><<<sms, kThreads, smem, st>>>(mq, mk, mv, plan, inv.entries, inv.entw, acc,
+                                                        (__nv_bfloat16 *)o, lse, ds);
     return cudaGetLastError();
 }
 
@@ -956,12 +954,12 @@ bool attend_tc_supported(const Shape &sh) {
 }
 
 cudaError_t launch_attend_tc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv, const void *q,
-                             const void *k, const void *v, const int32_t *idx, const float *w,
-                             __half *acc, void *o, float *lse, DevStatus *ds, cudaStream_t st) {
-    if (sh.d == 128 && sh.G == 8) return launch_tc<128, 8>(sh, plan, inv, q, k, v, idx, w, acc, o, lse, ds, st);
-    if (sh.d == 128 && sh.G == 16) return launch_tc<128, 16>(sh, plan, inv, q, k, v, idx, w, acc, o, lse, ds, st);
-    if (sh.d == 64 && sh.G == 8) return launch_tc<64, 8>(sh, plan, inv, q, k, v, idx, w, acc, o, lse, ds, st);
-    if (sh.d == 64 && sh.G == 16) return launch_tc<64, 16>(sh, plan, inv, q, k, v, idx, w, acc, o, lse, ds, st);
+                             const void *k, const void *v, __half *acc, void *o, float *lse,
+                             DevStatus *ds, cudaStream_t st) {
+    if (sh.d == 128 && sh.G == 8) return launch_tc<128, 8>(sh, plan, inv, q, k, v, acc, o, lse, ds, st);
+    if (sh.d == 128 && sh.G == 16) return launch_tc<128, 16>(sh, plan, inv, q, k, v, acc, o, lse, ds, st);
+    if (sh.d == 64 && sh.G == 8) return launch_tc<64, 8>(sh, plan, inv, q, k, v, acc, o, lse, ds, st);
+    if (sh.d == 64 && sh.G == 16) return launch_tc<64, 16>(sh, plan, inv, q, k, v, acc, o, lse, ds, st);
     return cudaErrorInvalidValue;
 }
 

@@ -423,8 +423,8 @@ hsa_status_t hsa_bwd(const hsa_shape_t *shape, const void *q, const void *k, con
                 return launch_bwd_tc(sh, P, b, q, k, v, dO, lse, all.dw, all.acc, dq, b.dk_acc, b.dv_acc, ds, st);
             });
         if (e == cudaSuccess)
-            e = timed(HSA_K_BWD_SEL, 2, st, [&] {
-                cudaError_t e2 = launch_bwd_select(sh, q_slc, idx, w, all.dw, kbar, dq_slc, b.dkbar, st);
+            e = timed(HSA_K_BWD_SEL, 3, st, [&] {
+                cudaError_t e2 = launch_bwd_select(sh, q_slc, idx, w, all.dw, kbar, dq_slc, b.dkbar, b, st);
                 return e2 == cudaSuccess ? launch_bwd_finish(sh, b, dk, dv, st) : e2;
             });
         return cuda_status(e);

@@ -230,8 +230,8 @@ cudaError_t launch_bwd_tc(const Shape &sh, const AttendPlan &plan, const BwdWs &
 // max L2 norm over the rows (of d bf16 values) of x, as float bits max-ed into *bits
 cudaError_t launch_rownorm_max(const void *x, int64_t rows, int d, int32_t *bits, cudaStream_t st);
 // Stick-breaking backward from dw: dq_slc, and dkbar (added into, fp32).
-cudaError_t launch_bwd_select(const Shape &sh, const void *q_slc, const int32_t *idx, const float *w,
-                              const float *dw, const float *kbar, void *dq_slc, float *dkbar, cudaStream_t st);
+cudaError_t launch_bwd_select(const Shape &sh, const void *q_slc, const int32_t *idx, const float *w, float *dw,
+                              const float *kbar, void *dq_slc, float *dkbar, const BwdWs &inv, cudaStream_t st);
 // dk = dk_acc + dkbar_c / S, dv = dv_acc, in the input dtype.
 cudaError_t launch_bwd_finish(const Shape &sh, const BwdWs &ws, void *dk, void *dv, cudaStream_t st);
 

@@ -820,8 +820,8 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
 // "end-to-end learning" (the chunk weight's gradient reaches the scores).
 __global__ void __launch_bounds__(256) bwd_select_kernel(const __nv_bfloat16 *__restrict__ q_slc,
                                                          const int32_t *__restrict__ idx, const float *__restrict__ w,
-                                                         const float *__restrict__ dw, const float *__restrict__ kbar,
-                                                         __nv_bfloat16 *__restrict__ dq_slc, float *__restrict__ dkbar,
+                                                         float *dw_ds, const float *__restrict__ kbar,
+                                                         __nv_bfloat16 *__restrict__ dq_slc,
                                                          int64_t rows, int L, int hkv, int nc, int K) {
     const int lane = threadIdx.x & 31;
     const int64_t gw = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
@@ -845,11 +845,11 @@ __global__ void __launch_bounds__(256) bwd_select_kernel(const __nv_bfloat16 *__
     int ck = (lane < K) ? idx[gw * K + lane] : -1;
     if (ck >= min(nc, t / kChunk)) ck = -1;
     const float wk = (ck >= 0) ? w[gw * K + lane] : 0.f;
-    const float dwk = (ck >= 0) ? dw[gw * K + lane] : 0.f;
+    const float dwk = (ck >= 0) ? dw_ds[gw * K + lane] : 0.f;
     float sk = 0.f;
     for (int k = 0; k < K; ++k) {
         const int c = __shfl_sync(0xffffffffu, ck, k);
-        if (c < 0) continue;  // valid slots form a prefix; uniform over the warp
+        if (c < 0) continue;  // an empty or ineligible slot: score and gradient stay 0
         const float4 kb = *reinterpret_cast<const float4 *>(kbar + (bg * nc + c) * D + lane * 4);
         float a = qv[0] * kb.x + qv[1] * kb.y + qv[2] * kb.z + qv[3] * kb.w;
 #pragma unroll
@@ -874,14 +874,62 @@ __global__ void __launch_bounds__(256) bwd_select_kernel(const __nv_bfloat16 *__
         const float4 kb = *reinterpret_cast<const float4 *>(kbar + (bg * nc + c) * D + lane * 4);
         dq4[0] = fmaf(dsj, kb.x, dq4[0]); dq4[1] = fmaf(dsj, kb.y, dq4[1]);
         dq4[2] = fmaf(dsj, kb.z, dq4[2]); dq4[3] = fmaf(dsj, kb.w, dq4[3]);
-        red_add_v4_f32(dkbar + (bg * nc + c) * D + lane * 4,
-                       make_float4(dsj * qv[0], dsj * qv[1], dsj * qv[2], dsj * qv[3]));
     }
+    // the slot's score gradient (times 1/sqrt(d)) replaces its weight gradient in place (each
+    // lane read its own entry above); bwd_dkbar_kernel sums it into the pooled-key gradient
+    if (lane < K) dw_ds[gw * K + lane] = dsk * scale;
     __nv_bfloat162 o0 = __floats2bfloat162_rn(dq4[0], dq4[1]), o1 = __floats2bfloat162_rn(dq4[2], dq4[3]);
     uint2 pk;
     pk.x = *reinterpret_cast<uint32_t *>(&o0);
     pk.y = *reinterpret_cast<uint32_t *>(&o1);
     *reinterpret_cast<uint2 *>(dq_slc + gw * D + lane * 4) = pk;
+}
+
+// Gradient of the pooled keys, chunk-major: dkbar[c] = sum over the (token, slot) entries
+// of chunk c's list of ds(token, slot) * q_slc[token].  One warp per list segment of
+// kBwdSeg entries (segment z of (b, g) belongs to the chunk c with seg_off[c] <= z <
+// seg_off[c+1]); a lane owns 4 of the 128 columns; one reduction per segment.
+__global__ void __launch_bounds__(256) bwd_dkbar_kernel(const __nv_bfloat16 *__restrict__ q_slc,
+                                                        const float *__restrict__ ds, const int32_t *__restrict__ chunk_off,
+                                                        const int32_t *__restrict__ seg_off,
+                                                        const int32_t *__restrict__ entries, float *__restrict__ dkbar,
+                                                        int L, int hkv, int nc, int K) {
+    constexpr int D = kBD;
+    const int lane = threadIdx.x & 31;
+    const int z = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int bg = blockIdx.y, b = bg / hkv, g = bg % hkv;
+    const int32_t *so = seg_off + (int64_t)bg * (nc + 1);
+    if (z >= so[nc]) return;
+    int lo = 0, hi = nc - 1;  // last c with so[c] <= z
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (so[mid] <= z) lo = mid; else hi = mid - 1;
+    }
+    const int c = lo;
+    const int32_t *off = chunk_off + (int64_t)bg * (nc + 1);
+    const int beg = off[c] + (z - so[c]) * kBwdSeg;
+    const int n = min(off[c + 1], beg + kBwdSeg) - beg;
+    if (n <= 0) return;
+    const int32_t *E = entries + (int64_t)bg * L * K;
+    int64_t qrow = 0;  // this lane's entry: its selection-query row and score gradient
+    float dsv = 0.f;
+    if (lane < n) {
+        const int ent = E[beg + lane];
+        const int64_t row = ((int64_t)b * L + (ent >> 4)) * hkv + g;
+        qrow = row * D;
+        dsv = ds[row * K + (ent & 15)];
+    }
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int i = 0; i < n; ++i) {
+        const int64_t qr = __shfl_sync(0xffffffffu, qrow, i);
+        const float d = __shfl_sync(0xffffffffu, dsv, i);
+        const uint2 raw = *reinterpret_cast<const uint2 *>(q_slc + qr + lane * 4);
+        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+        const float2 f0 = __bfloat1622float2(h2[0]), f1 = __bfloat1622float2(h2[1]);
+        acc[0] = fmaf(d, f0.x, acc[0]); acc[1] = fmaf(d, f0.y, acc[1]);
+        acc[2] = fmaf(d, f1.x, acc[2]); acc[3] = fmaf(d, f1.y, acc[3]);
+    }
+    red_add_v4_f32(dkbar + ((int64_t)bg * nc + c) * D + lane * 4, make_float4(acc[0], acc[1], acc[2], acc[3]));
 }
 
 // ------------------------------------------------------------------ magnitude bound
@@ -1003,13 +1051,19 @@ cudaError_t launch_bwd_tc(const Shape &sh, const AttendPlan &plan, const BwdWs &
     return cudaErrorInvalidValue;
 }
 
-cudaError_t launch_bwd_select(const Shape &sh, const void *q_slc, const int32_t *idx, const float *w,
-                              const float *dw, const float *kbar, void *dq_slc, float *dkbar, cudaStream_t st) {
+cudaError_t launch_bwd_select(const Shape &sh, const void *q_slc, const int32_t *idx, const float *w, float *dw,
+                              const float *kbar, void *dq_slc, float *dkbar, const BwdWs &inv, cudaStream_t st) {
     const int64_t rows = (int64_t)sh.B * sh.L * sh.hkv;
     if (rows == 0) return cudaSuccess;
-    bwd_select_kernel<<<(unsigned)ceil_div(rows, 8), 256, 0, st>>>(
-        (const __nv_bfloat16 *)q_slc, idx, w, dw, kbar, (__nv_bfloat16 *)dq_slc, dkbar, rows, sh.L, sh.hkv,
-        std::max(sh.nc, 1), sh.K);
+    bwd_select_kernel<<<(unsigned)ceil_div(rows, 8), 256, 0, st>>>((const __nv_bfloat16 *)q_slc, idx, w, dw, kbar,
+                                                                   (__nv_bfloat16 *)dq_slc, rows, sh.L, sh.hkv,
+                                                                   std::max(sh.nc, 1), sh.K);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess || sh.nc == 0) return e;
+    // segments of kBwdSeg list entries: at most L*K/kBwdSeg + nc per (b, g); 8 per block
+    const int64_t maxseg = ceil_div((int64_t)sh.L * sh.K, kBwdSeg) + sh.nc;
+    bwd_dkbar_kernel<<<dim3((unsigned)ceil_div(maxseg, 8), (unsigned)(sh.B * sh.hkv)), 256, 0, st>>>(
+        (const __nv_bfloat16 *)q_slc, dw, inv.chunk_off, inv.seg_off, inv.entries, dkbar, sh.L, sh.hkv, sh.nc, sh.K);
     return cudaGetLastError();
 }
 

@@ -254,7 +254,7 @@ static cudaError_t run_attend(const Shape &sh, const void *q, const void *k, con
     }
     // chunk-major tensor-core path: invert the selection, plan windows, attend
     if (e == cudaSuccess && sh.nc > 0)
-        e = timed(HSA_K_INVERT, 5, st, [&] { return launch_invert(sh, f.idx, f.w, f.inv, ds, st); });
+        e = timed(HSA_K_INVERT, 4, st, [&] { return launch_invert(sh, f.idx, f.w, f.inv, ds, st); });
     if (e == cudaSuccess) e = timed(HSA_K_PLAN, 3, st, [&] { return launch_plan(sh, f.inv, f.plan, st); });
     if (e == cudaSuccess)
         e = cudaMemsetAsync(f.plan.counters, 0, sizeof(int32_t) * plan_counter_count(f.plan.J), st);
@@ -402,7 +402,7 @@ hsa_status_t hsa_bwd(const hsa_shape_t *shape, const void *q, const void *k, con
         // one chunk-major pass on the tensor cores (dq, dw, dk, dv), then the
         // stick-breaking backward and the finishing pass on CUDA cores
         const AttendPlan &P = all.plan;
-        if (e == cudaSuccess) e = timed(HSA_K_INVERT, 5, st, [&] { return launch_invert(sh, idx, w, b, ds, st); });
+        if (e == cudaSuccess) e = timed(HSA_K_INVERT, 4, st, [&] { return launch_invert(sh, idx, w, b, ds, st); });
         if (e == cudaSuccess) e = timed(HSA_K_PLAN, 3, st, [&] { return launch_plan(sh, b, P, st); });
         if (e == cudaSuccess) e = cudaMemsetAsync(P.counters, 0, sizeof(int32_t) * plan_counter_count(P.J), st);
         if (e == cudaSuccess)
@@ -433,7 +433,7 @@ hsa_status_t hsa_bwd(const hsa_shape_t *shape, const void *q, const void *k, con
         e = timed(HSA_K_BWD1, 1, st, [&] {
             return launch_bwd_phase1(sh, q, q_slc, k, v, dO, lse, idx, w, kbar, dq, dq_slc, b, ds, st);
         });
-    if (e == cudaSuccess) e = timed(HSA_K_INVERT, sh.nc > 0 ? 5 : 0, st, [&] { return launch_invert(sh, idx, nullptr, b, ds, st); });
+    if (e == cudaSuccess) e = timed(HSA_K_INVERT, sh.nc > 0 ? 4 : 0, st, [&] { return launch_invert(sh, idx, nullptr, b, ds, st); });
     if (e == cudaSuccess)
         e = timed(HSA_K_BWD2, sh.nc > 0 ? 2 : 1, st, [&] { return launch_bwd_phase2(sh, q, k, v, dO, lse, w, dk, dv, b, ds, st); });
     return cuda_status(e);

@@ -5,10 +5,10 @@
 // walks, for each chunk, all tokens that selected it.  The lists are built as
 // a stable counting sort keyed by chunk, so each chunk's entries come out in
 // increasing token order and the result is deterministic:
-//   1. per block of 256 tokens, a histogram over chunks;
-//   2. per (b, g), a prefix over token blocks for every chunk (column scan),
-//      an exclusive scan of the chunk totals (CSR offsets), and the offsets
-//      added to every token block's prefix;
+//   1. per block of 128 tokens, a histogram over chunks;
+//   2. per (b, g), a prefix over token blocks for every chunk (column scan) and
+//      an exclusive scan of the chunk totals (CSR offsets); a token block's first
+//      position in chunk c's list is then chunk_off[c] + its prefix;
 //   3. per token block, one warp walks its tokens in order and places each
 //      (token, slot) entry at its chunk's running cursor.
 // Entry encoding: t * 16 + slot.
@@ -133,22 +133,12 @@ __global__ void __launch_bounds__(1024) inv_scan_kernel(int32_t *__restrict__ ch
     }
 }
 
-// hist[bg][tb][c] += chunk_off[bg][c]: per-block cursors become absolute positions.
-__global__ void __launch_bounds__(256) inv_base_kernel(int32_t *__restrict__ hist,
-                                                       const int32_t *__restrict__ chunk_off, int nc,
-                                                       int ntb) {
-    const int bg = blockIdx.y;
-    const int64_t n = (int64_t)ntb * nc;
-    int32_t *H = hist + (int64_t)bg * n;
-    const int32_t *off = chunk_off + (int64_t)bg * (nc + 1);
-    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x)
-        H[e] += off[e % nc];
-}
 
 // One warp per (token block, b*hkv + g): entries placed in token order.
 __global__ void __launch_bounds__(32) inv_scatter_kernel(const int32_t *__restrict__ idx,
                                                          const float *__restrict__ w,
                                                          const int32_t *__restrict__ hist,
+                                                         const int32_t *__restrict__ chunk_off,
                                                          int32_t *__restrict__ entries,
                                                          float *__restrict__ entw, int L,
                                                          int hkv, int nc, int K, int ntb) {
@@ -158,7 +148,8 @@ __global__ void __launch_bounds__(32) inv_scatter_kernel(const int32_t *__restri
     const int tb = blockIdx.x, bg = blockIdx.y, b = bg / hkv, g = bg % hkv;
     const int lane = threadIdx.x;
     const int32_t *H = hist + ((int64_t)bg * ntb + tb) * nc;
-    for (int c = lane; c < nc; c += 32) cur[c] = H[c];
+    const int32_t *off = chunk_off + (int64_t)bg * (nc + 1);
+    for (int c = lane; c < nc; c += 32) cur[c] = off[c] + H[c];  // the block's first position in each list
     const int t0 = tb * kInvTokBlock;
     const int t1 = min(t0 + kInvTokBlock, L);
     for (int e = lane; e < (t1 - t0) * K; e += 32) {
@@ -213,10 +204,8 @@ cudaError_t launch_invert(const Shape &sh, const int32_t *idx, const float *w, c
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     inv_scan_kernel<<<sh.B * sh.hkv, 1024, 2 * smem, st>>>(ws.chunk_off, ws.seg_off, sh.nc, kBwdSeg);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    inv_base_kernel<<<dim3(148, sh.B * sh.hkv), 256, 0, st>>>(ws.hist, ws.chunk_off, sh.nc, ntb);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    inv_scatter_kernel<<<grid, 32, ssmem, st>>>(idx, w, ws.hist, ws.entries, w ? ws.entw : nullptr, sh.L,
-                                                 sh.hkv, sh.nc, sh.K, ntb);
+    inv_scatter_kernel<<<grid, 32, ssmem, st>>>(idx, w, ws.hist, ws.chunk_off, ws.entries, w ? ws.entw : nullptr,
+                                                 sh.L, sh.hkv, sh.nc, sh.K, ntb);
     return cudaGetLastError();
 }
 

@@ -35,8 +35,9 @@ __global__ void __launch_bounds__(1024) plan_windows_kernel(const int32_t *__res
     __syncthreads();
     int my_tiles = 0;
     for (int c = threadIdx.x; c < nc; c += blockDim.x) {
-        const int e0 = H[(int64_t)tb0 * nc + c];
-        const int e1 = (tb1 < ntb) ? H[(int64_t)tb1 * nc + c] : off[c + 1];
+        // hist holds each chunk's per-block offsets within the chunk's list; off[c] is the list's start
+        const int e0 = off[c] + H[(int64_t)tb0 * nc + c];
+        const int e1 = (tb1 < ntb) ? off[c] + H[(int64_t)tb1 * nc + c] : off[c + 1];
         const int nt = (e1 - e0 + plan.TT - 1) / plan.TT;
         my_tiles += nt;
         s_units[c] = (nt + plan.unit_tiles - 1) / plan.unit_tiles;
@@ -111,8 +112,8 @@ __global__ void __launch_bounds__(256) plan_fill_kernel(const int32_t *__restric
         for (int c = threadIdx.x; c < nc; c += blockDim.x) {
             const int u0 = up[c], u1 = up[c + 1];
             if (u0 == u1) continue;
-            const int e0 = H[(int64_t)tb0 * nc + c];
-            const int e1 = (tb1 < ntb) ? H[(int64_t)tb1 * nc + c] : off[c + 1];
+            const int e0 = off[c] + H[(int64_t)tb0 * nc + c];
+            const int e1 = (tb1 < ntb) ? off[c] + H[(int64_t)tb1 * nc + c] : off[c + 1];
             const int nt = (e1 - e0 + plan.TT - 1) / plan.TT;
             for (int u = u0; u < u1; ++u) {
                 const int t0 = (u - u0) * plan.unit_tiles;

@@ -221,7 +221,7 @@ typedef enum {
     HSA_K_ATTEND_SIMT = 3, /* token-major attention (CUDA cores)             */
     HSA_K_DECODE = 4,      /* decode step                                    */
     HSA_K_BWD1 = 5,        /* backward phase 1 (per token)                   */
-    HSA_K_INVERT = 6,      /* token->chunk list inversion (5 launches)       */
+    HSA_K_INVERT = 6,      /* token->chunk list inversion (4 launches)       */
     HSA_K_BWD2 = 7,        /* backward phase 2 (per chunk) + finishing pass  */
     HSA_K_ATTEND_TC = 8,   /* chunk-major attention (tcgen05)                */
     HSA_K_PLAN = 9,        /* chunk-major work planning                      */

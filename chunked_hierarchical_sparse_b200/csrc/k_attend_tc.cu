@@ -414,57 +414,87 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
 #endif
     } else if (warp == kWarpMma) {
         // ============================================================ MMA issuer
-        // S(t) = Q_t K^T, in tile order, as soon as the tile's info, Q and K are there and
-        // its S buffer is free (the whole warp waits, sleeping; lane 0 issues).  O = P V is
-        // issued by the epilogue group that owns the tile's O buffer.
+        // Two in-order streams polled by one lane: S(t) = Q_t K^T is issued as
+        // soon as the tile's Q and K are in SMEM and an S buffer is free, and
+        // O(t) = P_t V as soon as P_t is written and an O buffer is free, so a
+        // slow epilogue never holds back the scores of the following tiles.
         constexpr uint32_t idesc1 = idesc_bf16_f32(128, 64, false, false);
+        constexpr uint32_t idesc2 = idesc_bf16_f32(128, D, false, true);
         PROF_DECL
         const long long prof_start = clock64();
         bool ok = true;
-        int ts = 0;
-        while (true) {
-            const int ii = ts % kInfo;
-            PROF_BEGIN();
-            if (!warp_wait(&B.info_full[ii], (ts / kInfo) & 1)) { ok = false; break; }
-            PROF_END(5);
-            const TileInfo &inf = info[ii];
-            if (inf.type == kItemEnd) break;
-            const int sb = ts & 1;
-            PROF_BEGIN();
-            if (inf.unit_first && !warp_wait(&B.kv_full[inf.kvs], inf.kvph)) { ok = false; break; }
-            PROF_END(2);
-            PROF_BEGIN();
-            if (!warp_wait(&B.q_full[inf.qs], inf.qph)) { ok = false; break; }
-            PROF_END(3);
-            PROF_BEGIN();
-            if (ts >= 2 && !warp_wait(&B.s_empty[sb], ((ts >> 1) - 1) & 1)) { ok = false; break; }
-            PROF_END(4);
-            PROF_BEGIN();
-            if (lane == 0) {
-                tc_fence_after();
-                const uint32_t qa = smem_u32(sm + L::OFF_Q + inf.qs * L::QBYTES);
-                const uint32_t kb = smem_u32(sm + L::OFF_K + inf.kvs * L::KVBYTES);
-                const uint32_t dcol = tmem + sb * 64;
+        int ts = 0, tp = 0;
+        if (lane == 0) {
+            bool s_done = false;  // the S stream has met the end item
+            uint64_t t_last = globaltimer();
+            while (true) {
+                bool prog = false;
+                if (!s_done) {
+                    const int ii = ts % kInfo;
+                    if (mbar_test(&B.info_full[ii], (ts / kInfo) & 1)) {
+                        const TileInfo &inf = info[ii];
+                        const int sb = ts & 1;
+                        if (inf.type == kItemEnd) {
+                            s_done = true;
+                            prog = true;
+                        } else if ((!inf.unit_first || mbar_test(&B.kv_full[inf.kvs], inf.kvph)) &&
+                                   mbar_test(&B.q_full[inf.qs], inf.qph) &&
+                                   (ts < 2 || mbar_test(&B.s_empty[sb], ((ts >> 1) - 1) & 1))) {
+                            tc_fence_after();
+                            const uint32_t qa = smem_u32(sm + L::OFF_Q + inf.qs * L::QBYTES);
+                            const uint32_t kb = smem_u32(sm + L::OFF_K + inf.kvs * L::KVBYTES);
+                            const uint32_t dcol = tmem + sb * 64;
 #pragma unroll
-                for (int ks = 0; ks < D / 16; ++ks) {
-                    const int h = ks >> 2, kk = ks & 3;
-                    // Q: d = 128 in 2 KB groups of 8 rows x both halves; d = 64 in 1 KB groups
-                    mma_bf16_ss(dcol, smem_desc_sw128(qa + h * 1024 + kk * 32, 16, L::NH * 1024),
-                                smem_desc_sw128(kb + h * L::KVHALF + kk * 32, 16, 1024), idesc1, ks > 0);
+                            for (int ks = 0; ks < D / 16; ++ks) {
+                                const int h = ks >> 2, kk = ks & 3;
+                                // Q: d = 128 in 2 KB groups of 8 rows x both halves; d = 64 in 1 KB groups
+                                mma_bf16_ss(dcol, smem_desc_sw128(qa + h * 1024 + kk * 32, 16, L::NH * 1024),
+                                            smem_desc_sw128(kb + h * L::KVHALF + kk * 32, 16, 1024), idesc1, ks > 0);
+                            }
+                            mma_commit(&B.s_full[sb]);
+                            mma_commit(&B.q_empty[inf.qs]);
+                            ++ts;
+                            prog = true;
+                        }
+                    }
                 }
-                mma_commit(&B.s_full[sb]);
-                mma_commit(&B.q_empty[inf.qs]);
+                if (tp < ts) {
+                    const int ii = tp % kInfo;
+                    const TileInfo &inf = info[ii];
+                    const int pb = tp & 1;
+                    if (mbar_test(&B.p_full[pb], (tp >> 1) & 1) &&
+                        (tp < 2 || mbar_test(&B.o_empty[pb], ((tp >> 1) - 1) & 1))) {
+                        tc_fence_after();
+                        const uint32_t pa = tmem + kColP + pb * 32;  // P: 64 keys as 32 bf16 pairs per row
+                        const uint32_t vb = smem_u32(sm + L::OFF_V + inf.kvs * L::KVBYTES);
+                        const uint32_t dcol = tmem + kColO + pb * 128;
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks)  // 16 keys = 8 TMEM columns per step
+                            mma_bf16_ts(dcol, pa + ks * 8, smem_desc_sw128(vb + ks * 2048, L::KVHALF, 1024), idesc2,
+                                        ks > 0);
+                        mma_commit(&B.o_full[pb]);
+                        mma_commit(&p_empty[pb]);
+                        if (inf.unit_last) mma_commit(&B.kv_empty[inf.kvs]);
+                        mbar_arrive(&B.info_empty[ii]);
+                        ++tp;
+                        prog = true;
+                    }
+                } else if (s_done) {
+                    break;
+                }
+                if (prog) {
+                    t_last = globaltimer();
+                } else {
+                    if (*abort_flag || globaltimer() - t_last > kWaitNs) { ok = false; break; }
+                    PROF_INC(1);
+                    __nanosleep(32);  // leave the issue slots to the working warps meanwhile
+                }
             }
-            __syncwarp();
-            mbar_arrive_lane0(&B.info_empty[ii], lane);  // done with the tile's info entry
-            PROF_END(8);
-            ++ts;
-        }
-        if (!ok) {
-            *abort_flag = 1;
-            if (lane == 0) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 3, ts);
-        }
-        if (lane == 0) {  // drain: every MMA this warp issued has finished before TMEM is released
+            if (!ok) {
+                *abort_flag = 1;
+                report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 3, ts);
+            }
+            // drain: every MMA issued by this warp has finished before TMEM is released
             mma_commit(mma_done);
             mbar_wait(mma_done, 0, kWaitNs);
         }
@@ -595,7 +625,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         const int r = wq * 32 + lane;                             // tile row of this lane's TMEM loads
         const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
         float4 *xs = reinterpret_cast<float4 *>(sm + L::OFF_X + (warp - kWarpEpi) * 4096);  // [32 rows][8 chunks]
-        int it = 0, tseq = 0, ecnt = 0, ecnt_j = -1, pv_last = -1;
+        int it = 0, tseq = 0, ecnt = 0, ecnt_j = -1;
         bool ok = true;
         PROF_DECL
         const long long prof_start = clock64();
@@ -634,26 +664,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 ecnt_j = inf.j;
             }
             const int sb = tseq & 1;
-            if (wq == 0) {  // the group's O buffer: issue the tile's O = P V into it
-                if (!warp_wait(&B.p_full[sb], (tseq >> 1) & 1)) { ok = false; break; }
-                if (tseq >= 2 && !warp_wait(&B.o_empty[sb], ((tseq >> 1) - 1) & 1)) { ok = false; break; }
-                if (lane == 0) {
-                    constexpr uint32_t idesc2 = idesc_bf16_f32(128, D, false, true);
-                    tc_fence_after();
-                    const uint32_t pa = tmem + kColP + sb * 32;  // P: 64 keys as 32 bf16 pairs per row
-                    const uint32_t vb = smem_u32(sm + L::OFF_V + inf.kvs * L::KVBYTES);
-                    const uint32_t dcol = tmem + kColO + sb * 128;
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)  // 16 keys = 8 TMEM columns per step
-                        mma_bf16_ts(dcol, pa + ks * 8, smem_desc_sw128(vb + ks * 2048, L::KVHALF, 1024), idesc2,
-                                    ks > 0);
-                    mma_commit(&B.o_full[sb]);
-                    mma_commit(&p_empty[sb]);
-                    if (inf.unit_last) mma_commit(&B.kv_empty[inf.kvs]);  // S and P.V of the unit are done
-                }
-                pv_last = tseq;
-                __syncwarp();
-            }
             PROF_BEGIN();
             if (!warp_wait(&B.o_full[sb], (tseq >> 1) & 1)) { ok = false; break; }
             if (!warp_wait(&coef_full[ii], ipar)) { ok = false; break; }
@@ -713,15 +723,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             ++it;
         }
         if (ok && ecnt > 0) flush();
-        if (!ok) {
-            *abort_flag = 1;
-            if (lane == 0) {
-                report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 6, it);
-                // the last O = P V this warp issued has finished before TMEM is released (bounded)
-                if (pv_last >= 0) mbar_wait(&B.o_full[pv_last & 1], (pv_last >> 1) & 1, kWaitNs);
-            }
-            __syncwarp();
-        }
+        if (!ok) { *abort_flag = 1; if (lane == 0) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 6, it); }
 #ifdef HSA_TC_PROFILE
         prof_acc[0] = clock64() - prof_start;
         if (lane == 0 && wq == 0) PROF_DUMP(blockIdx.x * 96 + 64 + 16 * eg);

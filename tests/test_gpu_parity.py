@@ -283,6 +283,42 @@ def test_fwd_full_size_sampled(name):
     assert_out(og, o_ref, wl.dtype, "o")
 
 
+@pytest.mark.parametrize("name", ["fwd64k"])
+def test_fwd_repeated_runs_agree(name):
+    """The persistent attention kernel hands buffers between roles and CTAs through
+    barriers and counters; a missed hand-off shows up as a run that differs from the
+    others by far more than the fp16 summation-order noise.  Five runs on the full-size
+    workload, compared on every output element (sampled rows against the oracle are
+    covered above)."""
+    wl, (x, kbar, _) = cached_workload(name)
+    m = hsa()
+    q, k, v, qs = (to_dev(x[n], wl.dtype) for n in ("q", "k", "v", "q_slc"))
+    ws = torch.empty(m.hsa_workspace_size(wl.B, wl.L, wl.h_q, wl.h_kv, wl.d, 64, wl.K, torch.bfloat16, m.OP_FWD),
+                     dtype=torch.uint8, device=DEV)
+    outs = []
+    for _ in range(5):
+        o, _, _, _, _ = m.hsa_fwd(q, k, v, qs, wl.K, want_lse=False, want_sel=False, ws=ws)
+        torch.cuda.synchronize()
+        assert m.hsa_device_status(ws) == 0
+        outs.append(o.float())
+    scale = max(1.0, float(outs[0].abs().max()))
+    for i in range(1, len(outs)):
+        diff = float((outs[i] - outs[0]).abs().max())
+        assert diff <= 2e-2 * scale, f"run {i} differs from run 0 by {diff:.3e}"
+
+
+def test_bwd_repeated_runs_agree():
+    """The same for the backward's persistent kernel (three runs, every gradient element)."""
+    wl = BWD_TC[1]
+    x = synth.make_inputs(wl)
+    runs = [run_bwd(wl, x) for _ in range(3)]
+    for i in range(1, len(runs)):
+        for name, a, b in zip(("dq", "dk", "dv", "dq_slc"), runs[i], runs[0]):
+            scale = max(1.0, float(b.float().abs().max()))
+            diff = float((a.float() - b.float()).abs().max())
+            assert diff <= 2e-2 * scale, f"{name}: run {i} differs from run 0 by {diff:.3e}"
+
+
 # --------------------------------------------------------------------------- decode
 def test_decode_workload():
     wl, (x, kbar, (o_ref, idx_ref, w_ref, gap)) = cached_workload("decode16k")

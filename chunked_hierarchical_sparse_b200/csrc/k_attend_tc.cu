@@ -516,8 +516,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         const long long prof_start = clock64();
         (void)prof_start;
 
-        // every warp waits for itself (lane 0 polls, the warp gets the verdict): the four
-        // warps only meet at the mbarriers they arrive on
+        // every warp waits for itself (all lanes, sleeping in try_wait): the four warps
+        // only meet at the mbarriers they arrive on
         while (ok) {
             const int ii = it % kInfo;
             const uint32_t ipar = (it / kInfo) & 1;

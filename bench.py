@@ -81,10 +81,16 @@ def fwd_work(wl):
 
 
 def source_hash(files):
+    """sha256 prefix of the files' code: comments, trailing blanks and empty lines removed,
+    so an edit to comments alone leaves the key of a measurement in place."""
     h = hashlib.sha256()
     for f in files:
-        with open(os.path.join(ROOT, f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, f), encoding="utf-8") as fh:
+            src = fh.read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", "", src)
+        code = "\n".join(ln.rstrip() for ln in src.splitlines() if ln.strip())
+        h.update(code.encode())
     return h.hexdigest()[:12]
 
 

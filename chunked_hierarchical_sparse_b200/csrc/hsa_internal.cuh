@@ -150,10 +150,11 @@ constexpr int kBwdSeg = 32;        // list entries per phase-2 block
 // ---------------------------------------------------------------- chunk-major forward plan
 constexpr int kUnitTiles = 4;      // forward: tiles of one chunk per work unit (one K/V load)
 constexpr int kCombTokens = 16;    // tokens per combine item
-// Output accumulators of the chunk-major forward: a ring of kRing window
-// slots, each an fp32 [W tokens][G heads][d] block that the tiles of one
-// window reduce their weighted outputs into (compile-time tunables; the ring
-// stays resident in L2 next to the K/V and query working set).
+// Accumulators of the chunk-major passes: a ring of kRing window slots, each
+// a [W tokens][G heads][d] block of scaled fp16 sums that the tiles of one
+// window reduce their weighted outputs (forward) or dq rows (backward) into
+// (compile-time tunables; the ring stays resident in L2 next to the K/V and
+// query working set).
 #ifndef HSA_ACC_RING
 #define HSA_ACC_RING 2
 #endif

@@ -114,9 +114,15 @@ def _p(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _stream(stream):
-    s = torch.cuda.current_stream() if stream is None else stream
-    return ctypes.c_void_p(s.cuda_stream)
+def _run(name: str, dev, stream, *args):
+    """Call a C entry point with the tensors' device current, on the given stream or
+    else that device's current stream (the library launches on the current device)."""
+    if stream is not None and stream.device != dev:
+        raise ValueError(f"{name}: the stream is on {stream.device}, the tensors on {dev}")
+    fn = getattr(load_library(), name)
+    with torch.cuda.device(dev):
+        s = torch.cuda.current_stream(dev) if stream is None else stream
+        _check(fn(*args, ctypes.c_void_p(s.cuda_stream)), name)
 
 
 def _check(code: int, where: str):
@@ -137,6 +143,8 @@ def _workspace(sh: HsaShape, op: int, device, ws):
     if n == 0:
         raise HsaError(1, "hsa_workspace_size")
     if ws is not None:
+        if not isinstance(ws, torch.Tensor) or ws.device != device or not ws.is_contiguous():
+            raise ValueError(f"workspace: a contiguous tensor on {device} is required")
         if ws.numel() * ws.element_size() < n:
             raise HsaError(3, "workspace")
         return ws, ws.numel() * ws.element_size()
@@ -154,8 +162,7 @@ def hsa_pool(k: torch.Tensor, S: int = 64, kbar=None, ws=None, stream=None) -> t
         kbar = torch.empty(B, h_kv, L // S, d, dtype=torch.float32, device=k.device)
     _need(kbar, "kbar", (B, h_kv, L // S, d), torch.float32, k.device)
     w_, n = _workspace(sh, OP_POOL, k.device, ws)
-    _check(load_library().hsa_pool(ctypes.byref(sh), _p(k), _p(kbar), _p(w_), n, _stream(stream)),
-           "hsa_pool")
+    _run("hsa_pool", k.device, stream, ctypes.byref(sh), _p(k), _p(kbar), _p(w_), n)
     return kbar
 
 
@@ -171,8 +178,8 @@ def hsa_select(q_slc: torch.Tensor, k: torch.Tensor, K: int, S: int = 64, ws=Non
     w = torch.empty(B, L, h_kv, K, dtype=torch.float32, device=dev)
     sh = HsaShape(B, L, h_kv, h_kv, d, S, K, dt)
     w_, n = _workspace(sh, OP_SELECT, dev, ws)
-    _check(load_library().hsa_select(ctypes.byref(sh), _p(q_slc), _p(k), _p(kbar), _p(idx), _p(w),
-                                     _p(w_), n, _stream(stream)), "hsa_select")
+    _run("hsa_select", dev, stream, ctypes.byref(sh), _p(q_slc), _p(k), _p(kbar), _p(idx), _p(w),
+         _p(w_), n)
     return kbar, idx, w
 
 
@@ -196,8 +203,8 @@ def hsa_fwd(q, k, v, q_slc, K: int, S: int = 64, want_lse: bool = True, want_sel
     kbar = torch.empty(B, h_kv, L // S, d, dtype=torch.float32, device=dev) if want_sel else None
     sh = HsaShape(B, L, h_q, h_kv, d, S, K, dt)
     w_, n = _workspace(sh, OP_FWD, dev, ws)
-    _check(load_library().hsa_fwd(ctypes.byref(sh), _p(q), _p(k), _p(v), _p(q_slc), _p(o), _p(lse),
-                                  _p(idx), _p(w), _p(kbar), _p(w_), n, _stream(stream)), "hsa_fwd")
+    _run("hsa_fwd", dev, stream, ctypes.byref(sh), _p(q), _p(k), _p(v), _p(q_slc), _p(o), _p(lse),
+         _p(idx), _p(w), _p(kbar), _p(w_), n)
     return o, lse, idx, w, kbar
 
 
@@ -218,8 +225,8 @@ def hsa_attend(q, k, v, idx, w, S: int = 64, want_lse: bool = True, o=None, ws=N
     lse = torch.empty(B, L, h_q, K, dtype=torch.float32, device=dev) if want_lse else None
     sh = HsaShape(B, L, h_q, h_kv, d, S, K, dt)
     w_, n = _workspace(sh, OP_FWD, dev, ws)
-    _check(load_library().hsa_attend(ctypes.byref(sh), _p(q), _p(k), _p(v), _p(idx), _p(w), _p(o),
-                                     _p(lse), _p(w_), n, _stream(stream)), "hsa_attend")
+    _run("hsa_attend", dev, stream, ctypes.byref(sh), _p(q), _p(k), _p(v), _p(idx), _p(w), _p(o),
+         _p(lse), _p(w_), n)
     return o, lse
 
 
@@ -242,9 +249,8 @@ def hsa_decode(q, q_slc, k_cache, v_cache, kbar, K: int, S: int = 64, o=None, wa
     w = torch.empty(B, h_kv, K, dtype=torch.float32, device=dev) if want_sel else None
     sh = HsaShape(B, P, h_q, h_kv, d, S, K, dt)
     w_, n = _workspace(sh, OP_DECODE, dev, ws)
-    _check(load_library().hsa_decode(ctypes.byref(sh), _p(q), _p(q_slc), _p(k_cache), _p(v_cache),
-                                     _p(kbar), _p(o), _p(idx), _p(w), _p(w_), n, _stream(stream)),
-           "hsa_decode")
+    _run("hsa_decode", dev, stream, ctypes.byref(sh), _p(q), _p(q_slc), _p(k_cache), _p(v_cache),
+         _p(kbar), _p(o), _p(idx), _p(w), _p(w_), n)
     return o, idx, w
 
 
@@ -268,9 +274,8 @@ def hsa_decode_multi(q, q_slc, k_cache, v_cache, kbar, K: int, S: int = 64, o=No
     w = torch.empty(B, h_kv, K, dtype=torch.float32, device=dev) if want_sel else None
     sh = HsaShape(B, P, h_q, h_kv, d, S, K, dt)
     w_, n = _workspace(sh, OP_DECODE, dev, ws)
-    _check(load_library().hsa_decode_multi(ctypes.byref(sh), NL, _p(q), _p(q_slc), _p(k_cache), _p(v_cache),
-                                           _p(kbar), _p(o), _p(idx), _p(w), _p(w_), n, _stream(stream)),
-           "hsa_decode_multi")
+    _run("hsa_decode_multi", dev, stream, ctypes.byref(sh), NL, _p(q), _p(q_slc), _p(k_cache),
+         _p(v_cache), _p(kbar), _p(o), _p(idx), _p(w), _p(w_), n)
     return o, idx, w
 
 
@@ -291,16 +296,14 @@ def hsa_bwd(q, k, v, q_slc, dO, lse, idx, w, kbar, K: int, S: int = 64, ws=None,
                        torch.empty_like(q_slc))
     sh = HsaShape(B, L, h_q, h_kv, d, S, K, dt)
     w_, n = _workspace(sh, OP_BWD, dev, ws)
-    _check(load_library().hsa_bwd(ctypes.byref(sh), _p(q), _p(k), _p(v), _p(q_slc), _p(dO), _p(lse),
-                                  _p(idx), _p(w), _p(kbar), _p(dq), _p(dk), _p(dv), _p(dqs), _p(w_),
-                                  n, _stream(stream)), "hsa_bwd")
+    _run("hsa_bwd", dev, stream, ctypes.byref(sh), _p(q), _p(k), _p(v), _p(q_slc), _p(dO), _p(lse),
+         _p(idx), _p(w), _p(kbar), _p(dq), _p(dk), _p(dv), _p(dqs), _p(w_), n)
     return dq, dk, dv, dqs
 
 
 def hsa_device_status(ws: torch.Tensor, stream=None) -> int:
     code = ctypes.c_int32(0)
-    _check(load_library().hsa_device_status(_p(ws), ctypes.byref(code), _stream(stream)),
-           "hsa_device_status")
+    _run("hsa_device_status", ws.device, stream, _p(ws), ctypes.byref(code))
     return int(code.value)
 
 

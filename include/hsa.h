@@ -54,7 +54,9 @@
  * Ownership: the caller owns every buffer (inputs, outputs, workspace); the
  * library never allocates, frees or synchronises -- each call only enqueues
  * kernels on `stream` (a cudaStream_t; NULL = legacy default stream) and
- * returns.  Device pointers everywhere except where a name says "host".
+ * returns.  Device pointers everywhere except where a name says "host"; they
+ * and `stream` belong to the calling thread's current CUDA device, which is
+ * where the kernels are launched.
  *
  * Errors: arguments are checked on the host before any launch (INVALID_ARG,
  * UNSUPPORTED, WORKSPACE); a failed launch returns HSA_ERR_CUDA.  Kernels never

@@ -107,3 +107,49 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(hsa, "lib_path", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         hsa.load_library()
+
+
+def _prototypes():
+    """name -> (return type, [parameter declarations]) for every HSA_API prototype."""
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    out = {}
+    for m in re.finditer(r"HSA_API\s+([\w\s\*]*?)\b(hsa_\w+)\s*\(([^)]*)\)\s*;", text):
+        params = [p.strip() for p in m.group(3).split(",") if p.strip() and p.strip() != "void"]
+        out[m.group(2)] = (" ".join(m.group(1).split()), params)
+    return out
+
+
+def _ctype_kind(t):
+    if t is None:
+        return None
+    if t in (ctypes.c_void_p, ctypes.c_char_p) or hasattr(t, "_type_") and isinstance(t._type_, type):
+        return "ptr"
+    if t is ctypes.c_size_t:
+        return "size"
+    if t in (ctypes.c_int, ctypes.c_int32):
+        return "int32"
+    return repr(t)
+
+
+def _decl_kind(decl):
+    if "*" in decl:
+        return "ptr"
+    if decl.split()[0] == "size_t":
+        return "size"
+    if decl.split()[0] in ("int", "int32_t", "hsa_status_t"):
+        return "int32"
+    return decl
+
+
+def test_binding_signatures_match_the_header(lib):
+    protos = _prototypes()
+    assert set(protos) == set(declared_symbols())
+    checked = 0
+    for name, (ret, params) in protos.items():
+        fn = getattr(lib, name)
+        if fn.argtypes is None:  # not bound in Python (C callers only)
+            continue
+        assert [_ctype_kind(t) for t in fn.argtypes] == [_decl_kind(p) for p in params], name
+        assert _ctype_kind(fn.restype) == _decl_kind(ret), name
+        checked += 1
+    assert checked >= 10

@@ -11,7 +11,7 @@ namespace hsa {
 // ------------------------------------------------------------------ checks
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-static hsa_status_t check_shape(const hsa_shape_t *s, bool decode) {
+hsa_status_t check_shape(const hsa_shape_t *s, bool decode) {
     if (!s) return HSA_ERR_INVALID_ARG;
     if (s->B < 0 || s->L < 0 || s->h_q < 1 || s->h_kv < 1 || s->d < 1 || s->S < 1 || s->K < 1)
         return HSA_ERR_INVALID_ARG;

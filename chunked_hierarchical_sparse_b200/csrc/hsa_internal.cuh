@@ -67,6 +67,10 @@ inline Shape make_shape(const hsa_shape_t &s) {
     return r;
 }
 
+// Host-side validation of a problem shape shared by every entry point: INVALID_ARG
+// for inconsistent values, UNSUPPORTED for valid shapes that are not built.
+hsa_status_t check_shape(const hsa_shape_t *s, bool decode);
+
 // ---------------------------------------------------------------- launch helpers
 // Raise a kernel's dynamic shared-memory limit to `bytes` once (cached per
 // kernel, so repeated calls -- and calls during stream capture -- make no

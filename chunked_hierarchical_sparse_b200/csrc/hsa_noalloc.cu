@@ -20,7 +20,11 @@
 // behind.  Calls that overlap on the GPU (different streams, or different host
 // threads, without ordering between them) race on it and must not be issued.
 // Each call clears the status word at the start of the array; the other
-// scratch regions are written in full before they are read.
+// scratch regions are written in full before they are read.  No caller can
+// read that status word (hsa_device_status takes a caller's workspace), and
+// none of this sequence's device-side checks can fire: the chunk indices the
+// attention checks are the ones the same call's selection just wrote, and
+// these kernels contain no bounded waits.
 //
 // Kernel sequence: the same launchers as the forward pass -- pooling, chunk
 // selection, token-major chunk attention with stick-breaking fusion -- with
@@ -71,14 +75,9 @@ extern "C" HSA_API hsa_status_t hsa_fwd_noalloc(const hsa_shape_t *shape, const 
                                                 void *o, float *lse, int32_t *idx, float *w,
                                                 float *kbar, void *stream) {
     using namespace hsa;
-    if (!shape) return HSA_ERR_INVALID_ARG;
+    const hsa_status_t chk = check_shape(shape, false);  // the same validation as hsa_fwd
+    if (chk != HSA_OK) return chk;
     const hsa_shape_t &s = *shape;
-    if (s.B < 0 || s.L < 0 || s.h_q < 1 || s.h_kv < 1 || s.d < 1 || s.S < 1 || s.K < 1 ||
-        s.h_q % s.h_kv != 0 || (s.dtype != HSA_F32 && s.dtype != HSA_BF16))
-        return HSA_ERR_INVALID_ARG;
-    if (s.S != kChunk || (s.d != 64 && s.d != 128) || s.K > kMaxK || s.h_q / s.h_kv > kMaxG ||
-        (int64_t)s.B * s.h_kv > 65535 || (int64_t)s.L * 16 >= ((int64_t)1 << 31))
-        return HSA_ERR_UNSUPPORTED;
     const Shape sh = make_shape(s);
     // scratch needed: status word, plus each intermediate the caller did not ask for
     const size_t kbar_b = r256(sizeof(float) * (size_t)sh.B * sh.hkv * sh.nc * sh.d);
@@ -104,8 +103,17 @@ extern "C" HSA_API hsa_status_t hsa_fwd_noalloc(const hsa_shape_t *shape, const 
     if (!ix) { ix = reinterpret_cast<int32_t *>(p); p += sel_b; }
     float *wt = w;
     if (!wt) { wt = reinterpret_cast<float *>(p); p += sel_b; }
-    e = launch_pool(sh, k, kb, ds, st);
-    if (e == cudaSuccess) e = launch_select_simt(sh, q_slc, kb, ix, wt, ds, st);
-    if (e == cudaSuccess) e = launch_attend_simt(sh, q, k, v, ix, wt, o, lse, ds, st);
+    {
+        TimedLaunch tl(HSA_K_POOL, 1, st);
+        e = launch_pool(sh, k, kb, ds, st);
+    }
+    if (e == cudaSuccess) {
+        TimedLaunch tl(HSA_K_SELECT, 1, st);
+        e = launch_select_simt(sh, q_slc, kb, ix, wt, ds, st);
+    }
+    if (e == cudaSuccess) {
+        TimedLaunch tl(HSA_K_ATTEND_SIMT, 1, st);
+        e = launch_attend_simt(sh, q, k, v, ix, wt, o, lse, ds, st);
+    }
     return e == cudaSuccess ? HSA_OK : HSA_ERR_CUDA;
 }

@@ -36,35 +36,10 @@ namespace hsa {
 
 using namespace sm100;
 
-#ifdef HSA_TC_PROFILE
-// Per-CTA cycle accounting of the roles' waits (development builds only).
-__device__ unsigned long long *g_tc_prof = nullptr;
-#define PROF_DECL unsigned long long prof_acc[16] = {0}; long long prof_t0 = 0;
-#define PROF_BEGIN() (prof_t0 = clock64())
-#define PROF_END(slot) (prof_acc[slot] += (unsigned long long)(clock64() - prof_t0))
-#define PROF_INC(slot) (prof_acc[slot] += 1)
-#define PROF_DUMP(base)                                                                        \
-    do {                                                                                       \
-        if (g_tc_prof)                                                                         \
-            for (int _i = 0; _i < 16; ++_i) atomicAdd(&g_tc_prof[(base) + _i], prof_acc[_i]);  \
-    } while (0)
-#else
-#define PROF_DECL
-#define PROF_BEGIN() ((void)0)
-#define PROF_END(slot) ((void)0)
-#define PROF_INC(slot) ((void)0)
-#define PROF_DUMP(base) ((void)0)
-#endif
 
 namespace {
 
-#ifndef HSA_EPI_UNROLL
-#define HSA_EPI_UNROLL 1
-#endif
-#ifndef HSA_CONV_BATCH
-#define HSA_CONV_BATCH 8
-#endif
-constexpr int kEpiUnroll = HSA_EPI_UNROLL;  // unrolling of the epilogue's column loops (1 keeps its code small)
+constexpr int kConvBatch = 8;  // 16-byte accumulator loads in flight per convert thread
 
 // 16 warps:
 //   warps 0-3 softmax, warps 4-7 and 8-11 two epilogue groups (weighted O ->
@@ -242,8 +217,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         // q mod gridDim.x), which keeps every CTA in window order.  Descriptors
         // are loaded two units ahead and a unit's entries and weights one unit
         // ahead, so no global-memory latency sits on the tile path.
-        PROF_DECL
-        const long long prof_start = clock64();
         int it = 0, qc = 0, kvc = 0;
         bool ok = true;
         const int total = min(P.seg_start[P.J], P.max_items);
@@ -273,16 +246,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         Pay pc = load_pay(dc);
         while (ok) {
             const int ii = it % kInfo;
-            PROF_BEGIN();
             if (it >= kInfo && !warp_wait(&B.info_empty[ii], ((it / kInfo) - 1) & 1)) { ok = false; break; }
-            PROF_END(2);
             if (*abort_flag) { ok = false; break; }
-            PROF_BEGIN();
             const int type = dc.a.x, j = dc.a.y, c = dc.a.z, e0 = dc.a.w;
             const int e1 = dc.b.x, t0 = dc.b.y, t1 = dc.b.z;
             const int ent_a = pc.ea, ent_b = pc.eb;
             const float w_a = pc.wa, w_b = pc.wb;
-            PROF_END(1);
             TileInfo &inf = info[ii];
             if (type == kItemEnd) {
                 if (lane == 0) {
@@ -305,8 +274,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             const int ub = e0 + t0 * TT;
             const int un = min(e1, e0 + t1 * TT) - ub;
             // ring guard: window j's partial slot was last used by window j - kRing
-            PROF_INC(6);
-            PROF_BEGIN();
             if (j >= kRing && j > guard_ok_j) {
                 int g_ok = 1;
                 if (lane == 0) g_ok = spin_geq_live(&comb_done[j - kRing], P.win_ncomb[j - kRing], abort_flag) ? 1 : 0;
@@ -317,12 +284,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 }
                 guard_ok_j = j;
             }
-            PROF_END(3);
             // K/V tiles of chunk c
             const int kvs = kvc & 1, kvph = (kvc >> 1) & 1;
-            PROF_BEGIN();
             if (kvc >= 2 && !warp_wait(&B.kv_empty[kvs], ((kvc >> 1) - 1) & 1)) { ok = false; break; }
-            PROF_END(4);
             if (lane == 0) {
                 mbar_arrive_expect_tx(&B.kv_full[kvs], 2 * L::KVBYTES);
                 const int row = bg * P.L + c * kChunk;
@@ -335,15 +299,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             ++kvc;
             for (int tt = t0; tt < t1; ++tt) {
                 const int ti = it % kInfo;
-                PROF_BEGIN();
                 if (it >= kInfo && !warp_wait(&B.info_empty[ti], ((it / kInfo) - 1) & 1)) { ok = false; break; }
-                PROF_END(2);
                 const int qs = qc % kQStages, qph = (qc / kQStages) & 1;
-                PROF_BEGIN();
                 if (qc >= kQStages && !warp_wait(&B.q_empty[qs], ((qc / kQStages) - 1) & 1)) { ok = false; break; }
-                PROF_END(5);
-                PROF_INC(7);
-                PROF_BEGIN();
                 TileInfo &ti_ = info[ti];
                 const int lo = (tt - t0) * TT;          // first entry of this tile within the unit
                 const int ntok = min(TT, un - lo);
@@ -387,11 +345,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                     ti_.qs = qs; ti_.qph = qph;
                 }
                 __syncwarp();
-                PROF_END(8);
-                PROF_BEGIN();
                 __syncwarp();
                 mbar_arrive_lane0(&B.info_full[ti], lane);
-                PROF_END(9);
                 ++qc;
                 ++it;
             }
@@ -408,10 +363,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             }
             __syncwarp();
         }
-#ifdef HSA_TC_PROFILE
-        prof_acc[0] = clock64() - prof_start;
-        if (lane == 0) PROF_DUMP(blockIdx.x * 96 + 0);
-#endif
     } else if (warp == kWarpMma) {
         // ============================================================ MMA issuer
         // Two in-order streams polled by one lane: S(t) = Q_t K^T is issued as
@@ -420,8 +371,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         // slow epilogue never holds back the scores of the following tiles.
         constexpr uint32_t idesc1 = idesc_bf16_f32(128, 64, false, false);
         constexpr uint32_t idesc2 = idesc_bf16_f32(128, D, false, true);
-        PROF_DECL
-        const long long prof_start = clock64();
         bool ok = true;
         int ts = 0, tp = 0;
         if (lane == 0) {
@@ -486,7 +435,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                     t_last = globaltimer();
                 } else {
                     if (*abort_flag || globaltimer() - t_last > kWaitNs) { ok = false; break; }
-                    PROF_INC(1);
                     __nanosleep(32);  // leave the issue slots to the working warps meanwhile
                 }
             }
@@ -499,12 +447,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             mbar_wait(mma_done, 0, kWaitNs);
         }
         __syncwarp();
-#ifdef HSA_TC_PROFILE
-        prof_acc[0] = clock64() - prof_start;
-        if (lane == 0) PROF_DUMP(blockIdx.x * 96 + 16);
-#else
-        (void)prof_start;
-#endif
     } else if (warp < kWarpEpi) {
         // ============================================================ softmax
         const int wq = warp & 3;                 // TMEM lane quadrant of this warp
@@ -512,28 +454,19 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
         int it = 0, tseq = 0;
         bool ok = true;
-        PROF_DECL
-        const long long prof_start = clock64();
-        (void)prof_start;
 
         // every warp waits for itself (all lanes, sleeping in try_wait): the four warps
         // only meet at the mbarriers they arrive on
         while (ok) {
             const int ii = it % kInfo;
             const uint32_t ipar = (it / kInfo) & 1;
-            PROF_BEGIN();
             if (!warp_wait(&B.info_full[ii], ipar)) { ok = false; break; }
-            PROF_END(1);
             const TileInfo &inf = info[ii];
             const int type = inf.type;
             if (type == kItemEnd) break;
             // ---------------- softmax of this tile
             const int sb = tseq & 1;
-            PROF_BEGIN();
             if (!warp_wait(&B.s_full[sb], (tseq >> 1) & 1)) { ok = false; break; }
-            PROF_END(2);
-            PROF_INC(12);
-            PROF_BEGIN();
             tc_fence_after();
             float x0[32], x1[32];
             tmem_ld32(lane_base + sb * 64, x0);
@@ -543,11 +476,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             __syncwarp();
             mbar_arrive_lane0(&B.s_empty[sb], lane);
             // P buffer sb is free once the O = P.V of tile tseq - 2 has read it
-            PROF_END(3);
-            PROF_BEGIN();
             if (tseq >= 2 && !warp_wait(&p_empty[sb], ((tseq >> 1) - 1) & 1)) { ok = false; break; }
-            PROF_END(4);
-            PROF_BEGIN();
             const int ti = r / G, hh = r % G;
             const bool valid = ti < inf.ntok;
             uint32_t pr[32];  // this row's P: key pairs (2j, 2j+1) as bf16x2, the lower key in the low half
@@ -599,7 +528,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             tc_fence_before();
             __syncwarp();
             mbar_arrive_lane0(&B.p_full[sb], lane);  // one arrival per warp
-            PROF_END(3);
             // the row's output coefficient w / Z for the epilogue group
             ecoef[ii * 128 + r] = coef;
             __syncwarp();
@@ -608,10 +536,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             ++it;
         }
         if (!ok) { *abort_flag = 1; if (lane == 0) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 5, it); }
-#ifdef HSA_TC_PROFILE
-        prof_acc[0] = clock64() - prof_start;
-        if (threadIdx.x == 0) PROF_DUMP(blockIdx.x * 96 + 32);
-#endif
     } else if (warp < kWarpConv) {
         // ============================================================ epilogue
         // Per tile: O (fp32, TMEM) times the row coefficient w / Z, transposed
@@ -627,9 +551,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         float4 *xs = reinterpret_cast<float4 *>(sm + L::OFF_X + (warp - kWarpEpi) * 4096);  // [32 rows][8 chunks]
         int it = 0, tseq = 0, ecnt = 0, ecnt_j = -1;
         bool ok = true;
-        PROF_DECL
-        const long long prof_start = clock64();
-        (void)prof_start;
         // Each warp runs on its own: it waits for itself, acknowledges each info slot
         // itself and publishes its own reduced rows per window (a window is complete
         // when its tiles are counted by all four warps of their group).
@@ -647,9 +568,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             const uint32_t ipar = (it / kInfo) & 1;
             if (ecnt > 0 && !__all_sync(0xffffffffu, mbar_test(&B.info_full[ii], ipar)))
                 flush();  // never sit on unpublished tiles while the next one is not there yet
-            PROF_BEGIN();
             if (!warp_wait(&B.info_full[ii], ipar)) { ok = false; break; }
-            PROF_END(1);
             const TileInfo &inf = info[ii];
             if (inf.type == kItemEnd) break;
             if ((tseq & 1) != eg) {  // the other group's tile: acknowledge the slot and move on
@@ -664,11 +583,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 ecnt_j = inf.j;
             }
             const int sb = tseq & 1;
-            PROF_BEGIN();
             if (!warp_wait(&B.o_full[sb], (tseq >> 1) & 1)) { ok = false; break; }
             if (!warp_wait(&coef_full[ii], ipar)) { ok = false; break; }
-            PROF_END(2);
-            PROF_BEGIN();
             tc_fence_after();
             const float coef = ecoef[ii * 128 + r];
             const int s = inf.j % kRing;
@@ -685,9 +601,9 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 dst[m] = acc + ((int64_t)(s * P.W + inf.tok[i] - ws) * G + tr % G) * D + (lane & 7) * 8;
             }
             uint4 *xs4 = reinterpret_cast<uint4 *>(xs);
-#pragma unroll kEpiUnroll
+#pragma unroll 1
             for (int q = 0; q < D / 64; ++q) {  // 64 columns = one 128-byte fp16 line per row
-#pragma unroll kEpiUnroll
+#pragma unroll 1
                 for (int hv = 0; hv < 2; ++hv) {  // 32 columns at a time: 4 chunks of 8 halves
                     float v[32];
                     tmem_ld32(lane_base + kColO + sb * 128 + q * 64 + hv * 32, v);
@@ -717,17 +633,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 __syncwarp();
             }
             mbar_arrive_lane0(&B.info_empty[ii], lane);  // this warp is done with the tile's info entry
-            PROF_END(3);
             ++ecnt;
             ++tseq;
             ++it;
         }
         if (ok && ecnt > 0) flush();
         if (!ok) { *abort_flag = 1; if (lane == 0) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 6, it); }
-#ifdef HSA_TC_PROFILE
-        prof_acc[0] = clock64() - prof_start;
-        if (lane == 0 && wq == 0) PROF_DUMP(blockIdx.x * 96 + 64 + 16 * eg);
-#endif
     } else if (warp < kWarpProd) {
         // ============================================================ convert group
         // Converts each window's fp32 accumulators into o.  Every CTA's convert
@@ -738,9 +649,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         const int tid = threadIdx.x - kWarpConv * 32;  // 0..kConvThreads-1
         int ci_n = 0, vcnt = 0;
         bool ok = true;
-        PROF_DECL
-        const long long prof_start = clock64();
-        (void)prof_start;
         auto cg_sync = [&]() { asm volatile("bar.sync 2, %0;" ::"n"(kConvThreads) : "memory"); };
         auto cg_bcast = [&](int v) -> int {  // thread 0's value to the whole group
             const int slot = (vcnt++) & 1;
@@ -750,19 +658,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         };
         for (int jc = 0; jc < P.J && ok; ++jc) {
             int gok = 1;
-            PROF_BEGIN();
             // every tile is counted by the four warps of its epilogue group
             if (tid == 0) gok = spin_geq_live(&tiles_done[jc], 4 * P.win_tiles[jc], abort_flag) ? 1 : 0;
             if (!cg_bcast(gok)) { if (tid == 0 && !*abort_flag) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 4, jc); ok = false; break; }
-            PROF_END(2);
             const int ncomb = P.win_ncomb[jc];
             while (true) {
-                PROF_BEGIN();
                 const int item = cg_bcast(tid == 0 ? atomicAdd(&comb_head[jc], 1) : 0);
-                PROF_END(1);
                 if (item >= ncomb) break;
-                PROF_INC(5);
-                PROF_BEGIN();
                 const int j = jc, b = (jc / P.nW) / P.hkv, g = (jc / P.nW) % P.hkv;
                 const int s = j % kRing;
                 const int ws = (j % P.nW) * P.W;
@@ -771,7 +673,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 // fp16 accumulators of tokens [ta, tb): G*D contiguous values per token, and
                 // o of (token, group g): G*D contiguous bf16.  A unit is 8 values -> 16 bytes of o.
                 constexpr int UPT = G * D / 8;  // units per token
-                constexpr int kBatch = HSA_CONV_BATCH;  // units in flight per thread
+                constexpr int kBatch = kConvBatch;  // units in flight per thread
                 uint4 *A = reinterpret_cast<uint4 *>(acc + (int64_t)(s * P.W + (ta - ws)) * G * D);
                 const int nunits = (tb - ta) * UPT;
                 for (int u0 = 0; u0 < nunits; u0 += kConvThreads * kBatch) {
@@ -802,7 +704,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                     }
                 }
                 cg_sync();
-                PROF_END(3);
                 if (tid == 0) {
                     __threadfence();
                     atomicAdd(&comb_done[j], 1);
@@ -811,10 +712,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             }
         }
         if (!ok) { *abort_flag = 1; if (tid == 0) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 7, ci_n); }
-#ifdef HSA_TC_PROFILE
-        prof_acc[0] = clock64() - prof_start;
-        if (tid == 0) PROF_DUMP(blockIdx.x * 96 + 48);
-#endif
     }
 
     tc_fence_before();
@@ -892,11 +789,6 @@ cudaError_t launch_tc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv,
 
 }  // namespace
 
-#ifdef HSA_TC_PROFILE
-extern "C" HSA_API int hsa_debug_tc_profile(void *dev_buf) {
-    return cudaMemcpyToSymbol(g_tc_prof, &dev_buf, sizeof(void *)) == cudaSuccess ? 0 : 4;
-}
-#endif
 
 // max|v| over the value tensor (bf16, length a multiple of 8), as float bits
 // max-ed into *bits: non-negative floats order like their bit patterns.

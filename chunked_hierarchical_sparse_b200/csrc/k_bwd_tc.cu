@@ -33,27 +33,6 @@ namespace hsa {
 
 using namespace sm100;
 
-#ifdef HSA_TC_PROFILE
-// Per-CTA cycle accounting of the roles (development builds only).
-__device__ unsigned long long *g_btc_prof = nullptr;
-extern "C" HSA_API int hsa_debug_btc_profile(void *dev_buf) {
-    return cudaMemcpyToSymbol(g_btc_prof, &dev_buf, sizeof(void *)) == cudaSuccess ? 0 : 4;
-}
-#define BP_DECL unsigned long long bp_acc[16] = {0}; long long bp_t0 = 0; const long long bp_start = clock64();
-#define BP_BEGIN() (bp_t0 = clock64())
-#define BP_END(slot) (bp_acc[slot] += (unsigned long long)(clock64() - bp_t0))
-#define BP_DUMP(base)                                                                            \
-    do {                                                                                         \
-        bp_acc[0] = clock64() - bp_start;                                                        \
-        if (g_btc_prof)                                                                          \
-            for (int _i = 0; _i < 16; ++_i) atomicAdd(&g_btc_prof[blockIdx.x * 80 + (base) + _i], bp_acc[_i]); \
-    } while (0)
-#else
-#define BP_DECL
-#define BP_BEGIN() ((void)0)
-#define BP_END(slot) ((void)0)
-#define BP_DUMP(base) ((void)0)
-#endif
 
 namespace {
 
@@ -247,7 +226,6 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
         // and weights one tile ahead.
         int it = 0, qc = 0, useq = 0;
         bool ok = true;
-        BP_DECL
         const int total = min(P.seg_start[P.J], P.max_items);
         const int qstep = gridDim.x;
         int guard_ok_j = -1;
@@ -298,9 +276,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
                 guard_ok_j = j;
             }
             // K/V of chunk c (single buffer: free once the previous unit's last dQ is done)
-            BP_BEGIN();
             if (useq >= 1 && !warp_wait(kv_empty, (useq - 1) & 1)) { ok = false; break; }
-            BP_END(1);
             if (lane == 0) {
                 mbar_arrive_expect_tx(kv_full, 2 * L::KVBYTES);
                 const int row = bg * P.L + c * kChunk;
@@ -313,13 +289,9 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
             for (int tt = t0; tt < t1 && ok; ++tt) {
                 const Pay pn = (tt + 1 < t1) ? tile_pay(dc, tt + 1) : tile_pay(dn, dn.b.y);
                 const int ii = it % kBInfo;
-                BP_BEGIN();
                 if (it >= kBInfo && !warp_wait(&info_empty[ii], ((it / kBInfo) - 1) & 1)) { ok = false; break; }
-                BP_END(2);
                 const int qs = qc & 1, qph = (qc >> 1) & 1;
-                BP_BEGIN();
                 if (qc >= 2 && !warp_wait(&qd_empty[qs], ((qc >> 1) - 1) & 1)) { ok = false; break; }
-                BP_END(3);
                 BTileInfo &ti_ = info[ii];
                 const int ntok = min(TT, e1 - (e0 + tt * TT));
                 int t = pc.e >> 4, slot = pc.e & 15;
@@ -373,9 +345,6 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
             }
             __syncwarp();
         }
-#ifdef HSA_TC_PROFILE
-        if (lane == 0) BP_DUMP(0);
-#endif
     } else if (warp == kBWarpMma) {
         // ============================================================ MMA issuer
         // Two in-order streams polled by one lane:
@@ -387,7 +356,6 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
         constexpr uint32_t id_dkv = idesc_bf16_f32(D, 64, true, true);
         bool ok = true;
         int ts = 0, tg = 0;
-        BP_DECL
         if (lane == 0) {
             bool s_done = false;
             uint64_t t_last = globaltimer();
@@ -473,9 +441,6 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
                     if (*abort_flag || globaltimer() - t_last > kBWaitNs) { ok = false; break; }
                     __nanosleep(32);  // leave the issue slots to the working warps meanwhile
                 }
-#ifdef HSA_TC_PROFILE
-                if (!prog) ++bp_acc[1];
-#endif
             }
             if (!ok) {
                 *abort_flag = 1;
@@ -484,9 +449,6 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
             // drain: every MMA issued by this warp has finished before TMEM is released
             mma_commit(mma_done);
             mbar_wait(mma_done, 0, kBWaitNs);
-#ifdef HSA_TC_PROFILE
-            BP_DUMP(16);
-#endif
         }
         __syncwarp();
     } else if (warp < kBWarpEpi) {
@@ -499,7 +461,6 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
         const float sl2 = scale * L2E;
         int it = 0;
         bool ok = true;
-        BP_DECL
         // every warp of the group waits for itself (converged, sleeping in try_wait);
         // the warps only meet at the mbarriers they arrive on
         auto wg_wait = [&](uint64_t *b, uint32_t par) -> bool {
@@ -507,9 +468,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
         };
         while (ok) {
             const int ii = it % kBInfo;
-            BP_BEGIN();
             if (!wg_wait(&info_full[ii], (it / kBInfo) & 1)) { ok = false; break; }
-            BP_END(1);
             const BTileInfo &inf = info[ii];
             if (inf.type == kBItemEnd) break;
             const int ti = r / G, hh = r % G;
@@ -519,10 +478,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
             // the row's log-normaliser from the forward, loaded before the scores are waited for
             const float lrow =
                 valid ? lse[(((int64_t)inf.b * P.L + t) * P.hq + inf.g * G + hh) * P.K + slot] : 0.f;
-            BP_BEGIN();
             if (!wg_wait(sd_full, it & 1)) { ok = false; break; }
-            BP_END(2);
-            BP_BEGIN();
             tc_fence_after();
             float x0[32], x1[32], d0[32], d1[32];
             tmem_ld32(lane_base + kColS, x0);
@@ -564,11 +520,8 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
 #pragma unroll
             for (int off = 1; off < G; off <<= 1) dsum += __shfl_xor_sync(0xffffffffu, dsum, off);
             if (valid && hh == 0) dw[(((int64_t)inf.b * P.L + t) * P.hkv + inf.g) * P.K + slot] = dsum;
-            BP_END(3);
             // the dS / wP buffer is free once the previous tile's gradient MMAs have read it
-            BP_BEGIN();
             if (it >= 1 && !wg_wait(ds_empty, (it - 1) & 1)) { ok = false; break; }
-            BP_END(4);
             uint8_t *dsrow = sm + L::OFF_DS + r * 128;
             uint8_t *wprow = sm + L::OFF_WP + r * 128;
             if (valid) {
@@ -591,9 +544,6 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
             ++it;
         }
         if (!ok) { *abort_flag = 1; if (tid == 0) report(ds, HSA_ERR_TIMEOUT, kKBwdTc, 5, it); }
-#ifdef HSA_TC_PROFILE
-        if (tid == 0) BP_DUMP(32);
-#endif
     } else if (warp < kBWarpConv) {
         // ============================================================ dQ epilogue + dK/dV flush
         // dQ rows (times 1/sqrt(d)) are transposed through a 4 KB per-warp
@@ -609,7 +559,6 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
         float4 *xs = reinterpret_cast<float4 *>(sm + L::OFF_X + wq * 4096);  // [32 rows][8 chunks]
         int it = 0, ecnt = 0, ecnt_j = -1, vcnt = 0;
         bool ok = true;
-        BP_DECL
         auto eg_sync = [&]() { asm volatile("bar.sync 2, 128;" ::: "memory"); };
         auto eg_vote = [&](int v) -> bool {
             const int slot = (vcnt++) & 1;
@@ -646,11 +595,8 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
                 if (ecnt > 0) flush();
                 ecnt_j = inf.j;
             }
-            BP_BEGIN();
             const int qb = it & 1;  // dQ buffer of this tile
             if (!eg_wait(&dq_full[qb], (it >> 1) & 1)) { ok = false; break; }
-            BP_END(1);
-            BP_BEGIN();
             tc_fence_after();
             const int s = inf.j % kRing;
             const int ws = (inf.j % P.nW) * P.W;
@@ -698,12 +644,8 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
                 }
                 __syncwarp();
             }
-            BP_END(2);
             if (inf.unit_last) {
-                BP_BEGIN();
                 if (!eg_wait(dkv_full, inf.useq & 1)) { ok = false; break; }
-                BP_END(3);
-                BP_BEGIN();
                 tc_fence_after();
                 const int64_t krow = ((int64_t)(inf.b * P.hkv + inf.g) * P.L + (int64_t)inf.c * kChunk) * D + r;
 #pragma unroll kBEpiUnroll
@@ -721,7 +663,6 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
                 tc_fence_before();
                 __syncwarp();
                 mbar_arrive_lane0(dkv_empty, lane);
-                BP_END(4);
             }
             eg_sync();  // the whole group is done with this tile's info entry
             if (tid == 0) mbar_arrive(&info_empty[ii]);
@@ -730,9 +671,6 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
         }
         if (ok && ecnt > 0) flush();
         if (!ok) { *abort_flag = 1; if (tid == 0) report(ds, HSA_ERR_TIMEOUT, kKBwdTc, 6, it); }
-#ifdef HSA_TC_PROFILE
-        if (tid == 0) BP_DUMP(48);
-#endif
     } else if (warp < kBWarpProd) {
         // ============================================================ convert group
         // Converts each window's fp32 dq slot into dq (bf16) and re-zeroes it,

@@ -32,20 +32,6 @@ namespace cg = cooperative_groups;
 
 namespace hsa {
 
-#ifdef HSA_TC_PROFILE
-// Phase timestamps of the decode step (development builds only).
-__device__ unsigned long long *g_dec_prof = nullptr;
-#define DEC_STAMP(i)                                                                                 \
-    do {                                                                                             \
-        if (g_dec_prof && threadIdx.x == 0) {                                                        \
-            unsigned long long t_;                                                                   \
-            asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                                  \
-            g_dec_prof[blockIdx.x * 8 + (i)] = t_;                                                   \
-        }                                                                                            \
-    } while (0)
-#else
-#define DEC_STAMP(i) ((void)0)
-#endif
 
 constexpr int kDecCta = 8;
 constexpr int kDecThreads = 128;
@@ -240,7 +226,6 @@ __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
                           const T *__restrict__ vc, const float *__restrict__ kbar, T *__restrict__ o,
                           int32_t *__restrict__ idx_out, float *__restrict__ w_out, int P, int hq, int hkv,
                           int nc, int K, int G, int NL, int64_t lstride) {
-    DEC_STAMP(0);
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
     const int bg = blockIdx.x / kDecCta, b = bg / hkv, g = bg % hkv;
@@ -315,9 +300,7 @@ __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
     load_q(0);
     int q_cur = 0;  // the layer whose queries Qs / Q16 hold (block-uniform)
     for (int e = tid; e < NL * kMaxG * D; e += kDecThreads) part[e] = 0.f;
-    DEC_STAMP(1);
     cluster.sync();
-    DEC_STAMP(2);
 
     // ---- 2. top-K over all chunks (every CTA, all threads), scores read over DSMEM.
     // Order: (s1, c1) beats (s2, c2) iff s1 > s2, or s1 == s2 and c1 > c2.
@@ -404,7 +387,6 @@ __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
         }
     }
     __syncthreads();
-    DEC_STAMP(3);
 
     // ---- 3. attention to the chunks of this CTA's slots
     const T *kbase = kc + (int64_t)bg * P * D;
@@ -473,9 +455,7 @@ __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
         __syncthreads();  // Qs, Pm and coef are rewritten for the next layer
         }
     }
-    DEC_STAMP(4);
     cluster.sync();
-    DEC_STAMP(5);
 
     // ---- 4. sum the partial outputs of the cluster (DSMEM), this CTA's column share
     const int ncol = G * D, tot = NL * ncol;
@@ -487,16 +467,9 @@ __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
         for (int r = 0; r < kDecCta; ++r) acc += cluster.map_shared_rank(part, r)[l * kMaxG * D + col];
         Elem<T>::store(o + (int64_t)l * lstride + ((int64_t)b * hq + (int64_t)g * G) * D + col, acc);
     }
-    DEC_STAMP(6);
     cluster.sync();
-    DEC_STAMP(7);
 }
 
-#ifdef HSA_TC_PROFILE
-extern "C" HSA_API int hsa_debug_dec_profile(void *dev_buf) {
-    return cudaMemcpyToSymbol(g_dec_prof, &dev_buf, sizeof(void *)) == cudaSuccess ? 0 : 4;
-}
-#endif
 
 size_t decode_cluster_smem(int nc, int d, int NL) {
     const int per = (nc + kDecCta - 1) / kDecCta;

@@ -26,16 +26,6 @@ namespace hsa {
 
 using namespace sm100;
 
-#ifdef HSA_TC_PROFILE
-__device__ unsigned long long *g_sel_prof = nullptr;  // [4]: total, wait, filter, insert (epilogue thread 0)
-#define SP_DECL unsigned long long sp_acc[4] = {0, 0, 0, 0}; long long sp_t0 = 0;
-#define SP_BEGIN() (sp_t0 = clock64())
-#define SP_END(k) (sp_acc[k] += (unsigned long long)(clock64() - sp_t0))
-#else
-#define SP_DECL
-#define SP_BEGIN() ((void)0)
-#define SP_END(k) ((void)0)
-#endif
 
 namespace {
 
@@ -198,19 +188,14 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_tc_kernel(
         }
         int wcnt = 0;
         bool ok = true;
-        SP_DECL
-        const long long sp_start = clock64();
-        (void)sp_start;
         for (int i = 0; i < ntiles; ++i) {
             const int s = i & 1;
-            SP_BEGIN();
             int v = 1;
             if (tid == 0) v = mbar_wait(&a_full[s], (i >> 1) & 1, kSelWaitNs) ? 1 : 0;
             const int slot = (wcnt++) & 1;
             if (tid == 0) wg_flag[slot] = v;
             asm volatile("bar.sync 1, 128;" ::: "memory");
             if (!wg_flag[slot]) { ok = false; break; }
-            SP_END(1);
             tc_fence_after();
             const int cbase = i * kSelN;
             for (int q4 = 0; q4 < kSelN / 32; ++q4) {
@@ -242,15 +227,12 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_tc_kernel(
                     continue;
                 }
                 // cheap pass: which of the 32 candidates beat the current K-th best?
-                SP_BEGIN();
                 uint32_t m = 0;
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                     sc[e] *= scale;
                     if (c0 + e < ne && sel_beats(sc[e], c0 + e, bs[KM - 1], bc[KM - 1])) m |= 1u << e;
                 }
-                SP_END(2);
-                SP_BEGIN();
                 // rare pass: insert them one by one (candidate picked by a select tree on
                 // the bits of its position, so everything stays in registers)
                 while (m) {
@@ -281,18 +263,12 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_tc_kernel(
                         cc = sw ? tc : cc;
                     }
                 }
-                SP_END(3);
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&a_empty[s]);
         }
         if (!ok && tid == 0) report(ds, HSA_ERR_TIMEOUT, kKSelectTc, 3, t0);
-#ifdef HSA_TC_PROFILE
-        sp_acc[0] = clock64() - sp_start;
-        if (tid == 0 && g_sel_prof)
-            for (int k = 0; k < 4; ++k) atomicAdd(&g_sel_prof[k], sp_acc[k]);
-#endif
         if (t < L) {
             // most-recent-first: order the chosen chunks by descending index (invalid = -1 last)
 #pragma unroll
@@ -332,11 +308,6 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_tc_kernel(
     if (warp == 1) tmem_dealloc(tmem, 2 * kSelN);
 }
 
-#ifdef HSA_TC_PROFILE
-extern "C" HSA_API int hsa_debug_sel_profile(void *dev_buf) {
-    return cudaMemcpyToSymbol(g_sel_prof, &dev_buf, sizeof(void *)) == cudaSuccess ? 0 : 4;
-}
-#endif
 
 namespace {
 typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,

@@ -202,7 +202,10 @@ HSA_API hsa_status_t hsa_bwd(const hsa_shape_t *shape, const void *q, const void
  * without launching.  The first call on a device looks the array's address up
  * (make it before any stream capture).  All calls on a device share the array:
  * calls that may overlap on the GPU race and must not be issued.  It runs the
- * token-major CUDA-core kernel sequence and allocates nothing. */
+ * token-major CUDA-core kernel sequence and allocates nothing.  Its status
+ * word lives in the library's array, which hsa_device_status cannot read; no
+ * device-side check of this sequence can fire (the indices it checks are the
+ * ones its own selection wrote, and its kernels have no bounded waits). */
 HSA_API hsa_status_t hsa_fwd_noalloc(const hsa_shape_t *shape, const void *q, const void *k,
                                      const void *v, const void *q_slc, void *o, float *lse,
                                      int32_t *idx, float *w, float *kbar, void *stream);

@@ -3,11 +3,17 @@
 Bars (fixed in advance, not tuned to results):
   chunk indices           bit-exact (the gap rule leaves no near-ties)
   pooled keys             bit-exact (fp64 sum of bf16/fp32 values, one fp32 rounding)
-  fp32 outputs            max |err| <= 1e-5
+  fp32 outputs            max |err| <= 1e-5 (forward and gradients)
   bf16 outputs            max |err| <= 2e-2 and relative L2 <= 5e-3
-  bf16 gradients          relative L2 <= 5e-3 and max |err| <= 2e-2 * max(1, max|ref|)
-                          (a bf16 rounding of a value v moves it by up to |v| 2^-9)
+  bf16 gradients          relative L2 <= 5e-3 and, element by element,
+                          |err| <= 2e-2 + 2^-8 |ref|: the stated 2e-2 bounds the
+                          arithmetic; rounding an element x to bf16 (8 significant
+                          bits) moves it by up to 2^-8 |x| on top, and gradients
+                          reach magnitudes where that alone exceeds 2e-2 (for
+                          |x| >= 8 the bf16 spacing is 2^-4)
   selection weights w     |err| <= 1e-5 (fp32 sigmoid products of fp32 scores)
+
+Every comparison prints its achieved max |err| and relative L2 error.
 """
 from __future__ import annotations
 
@@ -39,14 +45,32 @@ def f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu", torch.float64).numpy()
 
 
+def _errors(got: np.ndarray, want: np.ndarray, block: int = 1 << 24):
+    """max |got - want|, relative L2 error, and for the gradient bar the largest
+    |got - want| - 2^-8 |want| (computed in blocks: full-size arrays are large)."""
+    g, w = got.reshape(-1), want.reshape(-1)
+    mx, ex, num, den = 0.0, -np.inf, 0.0, 0.0
+    for i in range(0, g.size, block):
+        d = g[i:i + block] - w[i:i + block]
+        a = np.abs(d)
+        mx = max(mx, float(a.max()))
+        ex = max(ex, float((a - 2.0 ** -8 * np.abs(w[i:i + block])).max()))
+        num += float(np.dot(d, d))
+        den += float(np.dot(w[i:i + block], w[i:i + block]))
+    return mx, np.sqrt(num) / max(np.sqrt(den), 1e-30), ex
+
+
 def assert_out(got: np.ndarray, want: np.ndarray, dtype: str, what: str, grad: bool = False):
-    err = np.abs(got - want)
+    mx, rel, ex = _errors(np.asarray(got, dtype=np.float64), np.asarray(want, dtype=np.float64))
+    print(f"[parity] {what} ({dtype}{', gradient' if grad else ''}, {want.size} elements): "
+          f"max|err| {mx:.3e}  rel L2 {rel:.3e}" + (f"  max(|err| - 2^-8|ref|) {ex:.3e}" if grad else ""))
     if dtype == "f32":
-        assert err.max() <= 1e-5, f"{what}: max abs err {err.max():.3e}"
+        assert mx <= 1e-5, f"{what}: max abs err {mx:.3e} > 1e-5"
         return
-    rel = np.linalg.norm(got - want) / max(np.linalg.norm(want), 1e-30)
-    bound = 2e-2 * (max(1.0, np.abs(want).max()) if grad else 1.0)
-    assert err.max() <= bound, f"{what}: max abs err {err.max():.3e} > {bound:.3e}"
+    if grad:
+        assert ex <= 2e-2, f"{what}: |err| - 2^-8 |ref| reaches {ex:.3e} > 2e-2"
+    else:
+        assert mx <= 2e-2, f"{what}: max abs err {mx:.3e} > 2e-2"
     assert rel <= 5e-3, f"{what}: rel L2 err {rel:.3e}"
 
 
@@ -259,28 +283,24 @@ def test_fwd_tiny_fp32_workload():
     assert_out(f64(o).reshape(o_ref.shape), o_ref, "f32", "o")
 
 
-def _sample_rows(wl, n, seed=0):
-    rng = np.random.default_rng(seed)
-    rows = set(rng.integers(0, wl.B * wl.L, size=n).tolist())
-    for b in range(wl.B):  # edges: first chunk, chunk boundaries, last token
-        rows.update([b * wl.L + t for t in (0, wl.S - 1, wl.S, 2 * wl.S - 1, wl.L - 1)])
-    return np.array(sorted(rows), dtype=np.int64)
-
-
 @pytest.mark.parametrize("name", ["fwd16k", "fwd64k"])
-def test_fwd_full_size_sampled(name):
-    """Full-size workloads in the launch configuration the benchmark times: all
-    chunk indices exact; outputs on sampled rows (oracle row by row)."""
+def test_fwd_full_size(name):
+    """Full-size workloads in the launch configuration the benchmark times: the
+    pooled keys and every chunk index exact, every element of o and lse against
+    the oracle's forward over all rows."""
     wl, (x, kbar, (idx_ref, w_ref, s_ref, gap)) = cached_workload(name)
     o, lse, idx, w, kb = run_fwd(wl, x)
     assert np.array_equal(kb.cpu().numpy(), kbar)
     gi = idx.cpu().numpy().reshape(idx_ref.shape)
     assert np.array_equal(gi, idx_ref), f"{(gi != idx_ref).sum()} index mismatches"
     assert np.abs(w.cpu().numpy().reshape(w_ref.shape) - w_ref).max() <= 1e-5
-    rows = _sample_rows(wl, 384)
-    o_ref, lse_ref, _, _ = oracle.fwd(x["q"], x["k"], x["v"], x["q_slc"], kbar, wl.S, wl.K, rows=rows)
-    og = f64(o).reshape(wl.B * wl.L, wl.h_q, wl.d)[rows]
-    assert_out(og, o_ref, wl.dtype, "o")
+    o_ref, lse_ref, i2, _ = oracle.fwd(x["q"], x["k"], x["v"], x["q_slc"], kbar, wl.S, wl.K)
+    assert np.array_equal(i2, idx_ref)
+    assert_out(f64(o).reshape(o_ref.shape), o_ref, wl.dtype, f"o[{name}]")
+    del o_ref
+    lerr = np.abs(f64(lse).reshape(lse_ref.shape) - lse_ref).max()
+    print(f"[parity] lse[{name}]: max|err| {lerr:.3e}")
+    assert lerr <= 2e-3
 
 
 @pytest.mark.parametrize("name", ["fwd64k"])
@@ -460,11 +480,7 @@ def test_bwd_small_full(wl):
     ref = oracle.bwd(x["q"], x["k"], x["v"], x["q_slc"], kbar, x["dO"], wl.S, wl.K)
     got = run_bwd(wl, x)
     for name, g, r in zip(("dq", "dk", "dv", "dq_slc"), got, ref[:4]):
-        if wl.dtype == "f32":
-            err = np.abs(f64(g) - r).max()
-            assert err <= 1e-4 * max(1.0, np.abs(r).max()), f"{name}: {err:.3e}"
-        else:
-            assert_out(f64(g), r, "bf16", name, grad=True)
+        assert_out(f64(g), r, wl.dtype, name, grad=True)
 
 
 # chunk-major tensor-core backward: bf16, d = 128, G in {8, 16}
@@ -504,31 +520,14 @@ def test_bwd_tensor_core_grad_scale(factor):
         assert_out(f64(g) / factor, r, "bf16", name, grad=True)
 
 
-def test_bwd_train_workload_sampled():
-    """Full-size training workload: dq / dq_slc on sampled tokens, dk / dv on
-    sampled chunks (the oracle walks every token that selected them)."""
+def test_bwd_train_workload_full():
+    """Full-size training workload: every element of dq, dk, dv and dq_slc against
+    the oracle's backward over all tokens."""
     wl, (x, kbar, (idx, w, s, gap)) = cached_workload("train16k")
-    dq, dk, dv, dqs = run_bwd(wl, x)
-    rng = np.random.default_rng(5)
-    chunks = [(0, 0, 1), (1, 1, wl.n_c // 2), (3, 0, wl.n_c - 2), (2, 1, 7)]
-    idx4 = idx.reshape(wl.B, wl.L, wl.h_kv, wl.K)
-    mask = np.zeros((wl.B, wl.L), dtype=bool)
-    for b, g, c in chunks:
-        mask[b] |= (idx4[b, :, g, :] == c).any(-1)
-    toks = rng.integers(0, wl.L, size=(wl.B, 16))
-    for b in range(wl.B):
-        mask[b, toks[b]] = True
-    rdq, rdk, rdv, rdqs, _ = oracle.bwd(x["q"], x["k"], x["v"], x["q_slc"], kbar, x["dO"], wl.S, wl.K,
-                                        tok_mask=mask)
-    for b in range(wl.B):
-        tt = toks[b]
-        assert_out(f64(dq)[b, tt], rdq[b, tt], "bf16", "dq", grad=True)
-        assert_out(f64(dqs)[b, tt], rdqs[b, tt], "bf16", "dq_slc", grad=True)
-    for b, g, c in chunks:
-        sl = slice(c * wl.S, (c + 1) * wl.S)
-        # dk includes the pooled path of every token selecting c: all are in the mask
-        assert_out(f64(dk)[b, g, sl], rdk[b, g, sl], "bf16", f"dk[{b},{g},{c}]", grad=True)
-        assert_out(f64(dv)[b, g, sl], rdv[b, g, sl], "bf16", f"dv[{b},{g},{c}]", grad=True)
+    got = run_bwd(wl, x)
+    ref = oracle.bwd(x["q"], x["k"], x["v"], x["q_slc"], kbar, x["dO"], wl.S, wl.K)
+    for name, g, r in zip(("dq", "dk", "dv", "dq_slc"), got, ref[:4]):
+        assert_out(f64(g), r, "bf16", f"{name}[train16k]", grad=True)
 
 
 # --------------------------------------------------------------------------- status / errors

@@ -189,7 +189,7 @@ template <typename F> static cudaError_t timed(int kind, int n, cudaStream_t st,
 
 static cudaError_t run_select(const Shape &sh, const void *q_slc, const float *kbar, __nv_bfloat16 *hi,
                               __nv_bfloat16 *lo, int32_t *idx, float *w, DevStatus *ds, cudaStream_t st) {
-    TimedLaunch tl(HSA_K_SELECT, hi ? 2 : 1, st);
+    TimedLaunch tl(HSA_K_SELECT, 1, st);
     if (hi && lo) return launch_select_tc(sh, q_slc, kbar, hi, lo, idx, w, ds, st);
     return launch_select_simt(sh, q_slc, kbar, idx, w, ds, st);
 }
@@ -230,20 +230,25 @@ hsa_status_t hsa_select(const hsa_shape_t *shape, const void *q_slc, const void 
     if ((s = check_ws(sh, HSA_OP_SELECT, ws, ws_bytes)) != HSA_OK) return s;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     DevStatus *ds = static_cast<DevStatus *>(ws);
-    cudaError_t e = clear_status(ws, st);
-    if (e == cudaSuccess) e = timed(HSA_K_POOL, 1, st, [&] { return launch_pool(sh, k, kbar, ds, st); });
     __nv_bfloat16 *hi = nullptr, *lo = nullptr;
     if (select_tc_supported(sh)) {
         Carver c{static_cast<char *>(ws)};
         hi = c.take<__nv_bfloat16>((size_t)sh.B * sh.hkv * sh.nc * sh.d);
         lo = c.take<__nv_bfloat16>((size_t)sh.B * sh.hkv * sh.nc * sh.d);
     }
+    cudaError_t e = clear_status(ws, st);
+    PoolExtras px;  // the pooling pass also writes the bf16 split the tensor-core scores use
+    px.hi = hi;
+    px.lo = lo;
+    if (e == cudaSuccess) e = timed(HSA_K_POOL, 1, st, [&] { return launch_pool(sh, k, kbar, ds, st, px); });
     if (e == cudaSuccess) e = run_select(sh, q_slc, kbar, hi, lo, idx, w, ds, st);
     return cuda_status(e);
 }
 
 // attention + fusion (a5-a6) for a given selection f.idx / f.w: tensor-core chunk-major
 // path (inversion, plan, attend) for the shapes it takes, CUDA cores otherwise
+// given_sel: a caller-given selection (hsa_attend); otherwise the forward's own,
+// whose pooling pass has already cleared the plan counters and written max|v|
 static cudaError_t run_attend(const Shape &sh, const void *q, const void *k, const void *v, FwdWs &f, void *o,
                               float *lse, bool given_sel, DevStatus *ds, cudaStream_t st) {
     cudaError_t e = cudaSuccess;
@@ -256,7 +261,7 @@ static cudaError_t run_attend(const Shape &sh, const void *q, const void *k, con
     if (e == cudaSuccess && sh.nc > 0)
         e = timed(HSA_K_INVERT, 4, st, [&] { return launch_invert(sh, f.idx, f.w, f.inv, ds, st); });
     if (e == cudaSuccess) e = timed(HSA_K_PLAN, 3, st, [&] { return launch_plan(sh, f.inv, f.plan, st); });
-    if (e == cudaSuccess)
+    if (e == cudaSuccess && given_sel)
         e = cudaMemsetAsync(f.plan.counters, 0, sizeof(int32_t) * plan_counter_count(f.plan.J), st);
     if (e == cudaSuccess)  // the used accumulator slots start at zero (the kernel re-zeroes them after use)
         e = cudaMemsetAsync(f.acc, 0,
@@ -265,7 +270,7 @@ static cudaError_t run_attend(const Shape &sh, const void *q, const void *k, con
                             st);
     if (e == cudaSuccess && lse)
         e = cudaMemsetAsync(lse, 0, sizeof(float) * (size_t)sh.B * sh.L * sh.hq * sh.K, st);
-    if (e == cudaSuccess)  // the accumulators' power-of-two scale comes from max|v|
+    if (e == cudaSuccess && given_sel)  // the accumulators' power-of-two scale comes from max|v|
         e = timed(HSA_K_PLAN, 1, st, [&] { return launch_vmax(sh, v, f.plan.counters + 3 * f.plan.J + 1, st); });
     if (e == cudaSuccess && given_sel)  // weights not from stick-breaking: their row sums may exceed 1
         e = timed(HSA_K_PLAN, 1, st, [&] { return launch_wsum(sh, f.idx, f.w, f.plan.counters + 3 * f.plan.J + 2, st); });
@@ -293,7 +298,16 @@ hsa_status_t hsa_fwd(const hsa_shape_t *shape, const void *q, const void *k, con
     if (idx) f.idx = idx;
     if (w) f.w = w;
     cudaError_t e = clear_status(ws, st);
-    if (e == cudaSuccess) e = timed(HSA_K_POOL, 1, st, [&] { return launch_pool(sh, k, f.kbar, ds, st); });
+    PoolExtras px;  // the bf16 split for the tensor-core scores, max|v| for the accumulators' scale
+    px.hi = f.kb_hi;
+    px.lo = f.kb_lo;
+    if (f.tc) {
+        if (e == cudaSuccess)
+            e = cudaMemsetAsync(f.plan.counters, 0, sizeof(int32_t) * plan_counter_count(f.plan.J), st);
+        px.v = v;
+        px.vmax_bits = f.plan.counters + 3 * f.plan.J + 1;
+    }
+    if (e == cudaSuccess) e = timed(HSA_K_POOL, 1, st, [&] { return launch_pool(sh, k, f.kbar, ds, st, px); });
     if (e == cudaSuccess) e = run_select(sh, q_slc, f.kbar, f.kb_hi, f.kb_lo, f.idx, f.w, ds, st);
     if (e == cudaSuccess) e = run_attend(sh, q, k, v, f, o, lse, false, ds, st);
     return cuda_status(e);

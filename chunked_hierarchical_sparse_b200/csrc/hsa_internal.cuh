@@ -96,7 +96,15 @@ class TimedLaunch {
 
 // ---------------------------------------------------------------- launchers
 // All launchers enqueue on `st` and return the launch's cudaError_t.
-cudaError_t launch_pool(const Shape &sh, const void *k, float *kbar, DevStatus *ds, cudaStream_t st);
+// Optional outputs of the pooling pass (bf16 inputs): the bf16 hi/lo split of the
+// pooled keys, and max|v| over the complete chunks of v max-ed into *vmax_bits.
+struct PoolExtras {
+    __nv_bfloat16 *hi = nullptr, *lo = nullptr;
+    const void *v = nullptr;
+    int32_t *vmax_bits = nullptr;
+};
+cudaError_t launch_pool(const Shape &sh, const void *k, float *kbar, DevStatus *ds, cudaStream_t st,
+                        const PoolExtras &x = PoolExtras{});
 
 cudaError_t launch_select_simt(const Shape &sh, const void *q_slc, const float *kbar, int32_t *idx,
                                float *w, DevStatus *ds, cudaStream_t st);
@@ -212,7 +220,8 @@ inline size_t attend_acc_elems(int W, int G, int d) { return (size_t)kRing * W *
 constexpr int kFwdAccBytes = 2, kBwdAccBytes = 2;
 
 bool select_tc_supported(const Shape &sh);
-// Chunk selection with tensor-core scores; hi/lo: [B,hkv,nc,d] bf16 scratch.
+// Chunk selection with tensor-core scores; hi/lo: [B,hkv,nc,d] the bf16 split of
+// kbar written by the pooling pass.
 cudaError_t launch_select_tc(const Shape &sh, const void *q_slc, const float *kbar, __nv_bfloat16 *hi,
                              __nv_bfloat16 *lo, int32_t *idx, float *w, DevStatus *ds, cudaStream_t st);
 

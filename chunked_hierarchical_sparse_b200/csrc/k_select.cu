@@ -12,43 +12,70 @@
 namespace hsa {
 
 // ------------------------------------------------------------------ pooling
-// One warp per (b, g, chunk).  A lane owns VEC = 16 / sizeof(T) columns (one
-// 16-byte load per row) and 64 / RS of the chunk's rows (RS = 32 / (d / VEC)
-// row parts per warp); it sums them in fp64 with eight loads in flight, the row
-// parts are combined by shuffles, and the mean is rounded once to fp32.  The
-// fp64 sum of 64 bf16 (or fp32) values of one tensor is exact, so the result
-// does not depend on the summation order.
+// One warp per (b, g, chunk), four warps per block.  A lane owns VEC = 16 /
+// sizeof(T) columns (one 16-byte load per row) and 64 / RS of the chunk's rows
+// (RS = 32 / (d / VEC) row parts per warp); it sums them in fp64 with sixteen
+// loads in flight, the row parts are combined by shuffles, and the mean is
+// rounded once to fp32.  The fp64 sum of 64 bf16 (or fp32) values of one tensor
+// is exact, so the result does not depend on the summation order.
+//
+// With x.hi set (bf16 inputs) the same pass also writes the two-term bf16 split
+// of each pooled key (hi = bf16(kbar), lo = bf16(kbar - hi)) that the tensor-core
+// selection scores with, and, with x.vmax_bits set, reads the chunk's values too
+// and max-es max|v| (float bits; non-negative floats order like their bit
+// patterns) into *x.vmax_bits: the scale of the chunk-major attention's fp16
+// accumulators, which only ever sum values of complete chunks.
 template <typename T>
-__global__ void __launch_bounds__(256) pool_kernel(const T *__restrict__ k, float *__restrict__ kbar,
-                                                   int L, int d, int nc, int64_t nchunks) {
+__global__ void __launch_bounds__(128) pool_kernel(const T *__restrict__ k, float *__restrict__ kbar,
+                                                   int L, int d, int nc, int64_t nchunks, PoolExtras x) {
     constexpr int VEC = 16 / sizeof(T);
+    constexpr int NB = 16;  // loads in flight per lane
     const int lane = threadIdx.x & 31;
     const int64_t bgc = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;  // this warp's chunk
     if (bgc >= nchunks) return;
     const int tpc = d / VEC;      // lanes per row (8, 16 or 32)
     const int rs = 32 / tpc;      // row parts
     const int lr = lane % tpc, part = lane / tpc;
-    const int rows = kChunk / rs;
+    const int rows = kChunk / rs;  // 16, 32 or 64: a multiple of NB
     const int c = (int)(bgc % nc);
     const int64_t bg = bgc / nc;
-    const T *src = k + ((bg * L + (int64_t)c * kChunk + (int64_t)part * rows) * d) + lr * VEC;
+    const int64_t off = ((bg * L + (int64_t)c * kChunk + (int64_t)part * rows) * d) + lr * VEC;
+    const T *src = k + off;
     double acc[VEC];
 #pragma unroll
     for (int e = 0; e < VEC; ++e) acc[e] = 0.0;
-    for (int r0 = 0; r0 < rows; r0 += 8) {
-        uint4 raw[8];
+    for (int r0 = 0; r0 < rows; r0 += NB) {
+        uint4 raw[NB];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) raw[u] = __ldcs(reinterpret_cast<const uint4 *>(src + (int64_t)(r0 + u) * d));
+        for (int u = 0; u < NB; ++u) raw[u] = __ldcs(reinterpret_cast<const uint4 *>(src + (int64_t)(r0 + u) * d));
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
+        for (int u = 0; u < NB; ++u) {
             const T *vals = reinterpret_cast<const T *>(&raw[u]);
 #pragma unroll
             for (int e = 0; e < VEC; ++e) acc[e] += (double)Elem<T>::load(vals + e);
         }
     }
-    for (int off = tpc; off < 32; off <<= 1)
+    if (x.vmax_bits) {  // bf16 values of the same chunk
+        const T *vsrc = static_cast<const T *>(x.v) + off;
+        float m = 0.f;
+        for (int r0 = 0; r0 < rows; r0 += NB) {
+            uint4 raw[NB];
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
+            for (int u = 0; u < NB; ++u) raw[u] = __ldcs(reinterpret_cast<const uint4 *>(vsrc + (int64_t)(r0 + u) * d));
+#pragma unroll
+            for (int u = 0; u < NB; ++u) {
+                const T *vals = reinterpret_cast<const T *>(&raw[u]);
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) m = fmaxf(m, fabsf(Elem<T>::load(vals + e)));
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) atomicMax(x.vmax_bits, __float_as_int(m));
+    }
+    for (int o = tpc; o < 32; o <<= 1)
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], o);
     if (part == 0) {
         float out[VEC];
 #pragma unroll
@@ -56,17 +83,33 @@ __global__ void __launch_bounds__(256) pool_kernel(const T *__restrict__ k, floa
         float4 *dst = reinterpret_cast<float4 *>(kbar + bgc * d + lr * VEC);
 #pragma unroll
         for (int e = 0; e < VEC / 4; ++e) dst[e] = make_float4(out[4 * e], out[4 * e + 1], out[4 * e + 2], out[4 * e + 3]);
+        if (x.hi) {
+            __align__(16) __nv_bfloat16 h[VEC], l[VEC];
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) {
+                h[e] = __float2bfloat16_rn(out[e]);
+                l[e] = __float2bfloat16_rn(out[e] - __bfloat162float(h[e]));
+            }
+            const int64_t o2 = bgc * d + lr * VEC;
+#pragma unroll
+            for (int e = 0; e < VEC / 8; ++e) {
+                reinterpret_cast<uint4 *>(x.hi + o2)[e] = reinterpret_cast<const uint4 *>(h)[e];
+                reinterpret_cast<uint4 *>(x.lo + o2)[e] = reinterpret_cast<const uint4 *>(l)[e];
+            }
+        }
     }
 }
 
-cudaError_t launch_pool(const Shape &sh, const void *k, float *kbar, DevStatus *, cudaStream_t st) {
+cudaError_t launch_pool(const Shape &sh, const void *k, float *kbar, DevStatus *, cudaStream_t st,
+                        const PoolExtras &x) {
     const int64_t chunks = (int64_t)sh.B * sh.hkv * sh.nc;
     if (chunks == 0) return cudaSuccess;
-    const unsigned blocks = (unsigned)ceil_div(chunks, 8);  // 8 warps = 8 chunks per block
+    const unsigned blocks = (unsigned)ceil_div(chunks, 4);  // 4 warps = 4 chunks per block
     if (sh.bf16)
-        pool_kernel<__nv_bfloat16><<<blocks, 256, 0, st>>>((const __nv_bfloat16 *)k, kbar, sh.L, sh.d, sh.nc, chunks);
+        pool_kernel<__nv_bfloat16><<<blocks, 128, 0, st>>>((const __nv_bfloat16 *)k, kbar, sh.L, sh.d, sh.nc, chunks, x);
     else
-        pool_kernel<float><<<blocks, 256, 0, st>>>((const float *)k, kbar, sh.L, sh.d, sh.nc, chunks);
+        pool_kernel<float><<<blocks, 128, 0, st>>>((const float *)k, kbar, sh.L, sh.d, sh.nc, chunks,
+                                                   PoolExtras{});  // split and max|v| serve bf16 paths only
     return cudaGetLastError();
 }
 

@@ -52,9 +52,12 @@ struct FwdWs {
     float *w;
     __nv_bfloat16 *kb_hi, *kb_lo;  // split pooled keys for the tensor-core scores
     bool tc;             // chunk-major tensor-core path
-    BwdWs inv;           // token->chunk lists (hist, chunk_off, seg_off, entries)
+    int32_t *entries;    // per (b, g): nW windows x W*K (token, slot) entries, bucket by bucket
+    float *entw;         //   and their weights
+    int32_t *bucket_cnt, *bucket_cur;  // [J][nc] entries per bucket, scatter cursors
     AttendPlan plan;
     __half *acc;         // fp16 output-accumulator ring, scaled (chunk-major path)
+    size_t zero_bytes;   // plan counters .. bucket counts: cleared by one memset per call
 };
 
 // token->chunk lists of the chunk-major passes (with the entries' weights if `weights`)
@@ -85,6 +88,8 @@ static void carve_plan(Carver &c, const Shape &sh, AttendPlan &P, int unit_tiles
         ((int64_t)sh.B * sh.hkv * ((int64_t)sh.L * sh.K / P.TT + (int64_t)P.nW * sh.nc) + 16),
         (int64_t)INT32_MAX / 4);
     P.items = c.take<int4>((size_t)2 * P.max_items);
+    P.win_cap = 0;
+    P.ent_stride = (int64_t)sh.L * sh.K;
 }
 
 static FwdWs carve_fwd(const Shape &sh, void *ws, size_t *bytes) {
@@ -99,9 +104,31 @@ static FwdWs carve_fwd(const Shape &sh, void *ws, size_t *bytes) {
     }
     f.tc = attend_tc_supported(sh);
     if (f.tc) {
-        carve_lists(c, sh, f.inv, true);
-        carve_plan(c, sh, f.plan, kUnitTiles, kFwdAccBytes);
-        f.acc = c.take<__half>(attend_acc_elems(f.plan.W, sh.G, sh.d));
+        // bucket plan: each window owns a fixed slice of the entries and of the queue
+        AttendPlan &P = f.plan;
+        P.B = sh.B; P.L = sh.L; P.hq = sh.hq; P.hkv = sh.hkv; P.D = sh.d; P.K = sh.K; P.G = sh.G;
+        P.nc = sh.nc; P.ntb = (int)ceil_div(sh.L, kInvTokBlock);
+        P.W = (int)std::min<int64_t>(attend_window(sh.G, sh.d, kFwdAccBytes), round_up(std::max(sh.L, 1), kInvTokBlock));
+        P.nW = (int)ceil_div(sh.L, P.W); P.J = sh.B * sh.hkv * P.nW; P.TT = 128 / sh.G;
+        P.unit_tiles = kUnitTiles;
+        P.ent_stride = (int64_t)P.nW * P.W * sh.K;
+        // units of a window <= its tiles <= W*K/TT + nc (one ragged tile per bucket)
+        P.win_cap = (int)std::min<int64_t>((int64_t)P.W * sh.K / P.TT + sh.nc, INT32_MAX / 4);
+        P.max_items = (int)std::min<int64_t>((int64_t)P.J * P.win_cap, INT32_MAX / 4);
+        f.entries = c.take<int32_t>((size_t)sh.B * sh.hkv * P.ent_stride);
+        f.entw = c.take<float>((size_t)sh.B * sh.hkv * P.ent_stride);
+        P.unit_prefix = nullptr;
+        P.win_units = c.take<int32_t>((size_t)P.J);
+        P.win_tiles = c.take<int32_t>((size_t)P.J);
+        P.win_ncomb = c.take<int32_t>((size_t)P.J);
+        P.seg_start = c.take<int32_t>((size_t)P.J + 1);
+        P.items = c.take<int4>((size_t)2 * P.J * P.win_cap);
+        f.bucket_cur = c.take<int32_t>((size_t)P.J * sh.nc);
+        const size_t z0 = c.off;
+        P.counters = c.take<int32_t>(plan_counter_count(P.J));
+        f.bucket_cnt = c.take<int32_t>((size_t)P.J * sh.nc);
+        f.zero_bytes = c.off - z0;
+        f.acc = c.take<__half>(attend_acc_elems(P.W, sh.G, sh.d));
     }
     if (bytes) *bytes = c.off;
     return f;
@@ -257,12 +284,14 @@ static cudaError_t run_attend(const Shape &sh, const void *q, const void *k, con
             e = timed(HSA_K_ATTEND_SIMT, 1, st, [&] { return launch_attend_simt(sh, q, k, v, f.idx, f.w, o, lse, ds, st); });
         return e;
     }
-    // chunk-major tensor-core path: invert the selection, plan windows, attend
-    if (e == cudaSuccess && sh.nc > 0)
-        e = timed(HSA_K_INVERT, 4, st, [&] { return launch_invert(sh, f.idx, f.w, f.inv, ds, st); });
-    if (e == cudaSuccess) e = timed(HSA_K_PLAN, 3, st, [&] { return launch_plan(sh, f.inv, f.plan, st); });
-    if (e == cudaSuccess && given_sel)
-        e = cudaMemsetAsync(f.plan.counters, 0, sizeof(int32_t) * plan_counter_count(f.plan.J), st);
+    // chunk-major tensor-core path: bucket the selection by (window, chunk), queue the
+    // work units, attend.  The forward's pooling pass has cleared the plan counters and
+    // bucket counts already (and written max|v|); a caller-given selection clears them here.
+    if (e == cudaSuccess && given_sel) e = cudaMemsetAsync(f.plan.counters, 0, f.zero_bytes, st);
+    if (e == cudaSuccess)
+        e = timed(HSA_K_INVERT, sh.nc > 0 ? 3 : 1, st, [&] {
+            return launch_bucket_plan(sh, f.idx, f.w, f.plan, f.bucket_cnt, f.bucket_cur, f.entries, f.entw, ds, st);
+        });
     if (e == cudaSuccess)  // the used accumulator slots start at zero (the kernel re-zeroes them after use)
         e = cudaMemsetAsync(f.acc, 0,
                             sizeof(__half) * std::min<size_t>(attend_acc_elems(f.plan.W, sh.G, sh.d),
@@ -276,7 +305,7 @@ static cudaError_t run_attend(const Shape &sh, const void *q, const void *k, con
         e = timed(HSA_K_PLAN, 1, st, [&] { return launch_wsum(sh, f.idx, f.w, f.plan.counters + 3 * f.plan.J + 2, st); });
     if (e == cudaSuccess)
         e = timed(HSA_K_ATTEND_TC, 1, st, [&] {
-            return launch_attend_tc(sh, f.plan, f.inv, q, k, v, f.acc, o, lse, ds, st);
+            return launch_attend_tc(sh, f.plan, f.entries, f.entw, q, k, v, f.acc, o, lse, ds, st);
         });
     return e;
 }
@@ -302,8 +331,7 @@ hsa_status_t hsa_fwd(const hsa_shape_t *shape, const void *q, const void *k, con
     px.hi = f.kb_hi;
     px.lo = f.kb_lo;
     if (f.tc) {
-        if (e == cudaSuccess)
-            e = cudaMemsetAsync(f.plan.counters, 0, sizeof(int32_t) * plan_counter_count(f.plan.J), st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(f.plan.counters, 0, f.zero_bytes, st);
         px.v = v;
         px.vmax_bits = f.plan.counters + 3 * f.plan.J + 1;
     }

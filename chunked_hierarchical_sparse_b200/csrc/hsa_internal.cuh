@@ -187,10 +187,24 @@ struct AttendPlan {
     int32_t *win_tiles;    // [J]
     int32_t *win_ncomb;    // [J]
     int32_t *seg_start;    // [J+1] queue segment starts (the units of window s)
-    int32_t *counters;     // [3J+1] tiles_done[J], comb_done[J], comb_head[J], queue head (zeroed per call)
-    int4 *items;           // [2 per queue item] flat descriptors in queue order
+    int32_t *counters;     // [3J+4] tiles_done[J], comb_done[J], comb_head[J], a done count, bounds (zeroed per call)
+    int4 *items;           // [2 per queue item] descriptors
     int max_items;         // capacity of `items`
+    // Layout of the lists and the queue.  win_cap == 0: the queue is contiguous in
+    // queue order and each (b, g) owns L*K entries.  win_cap > 0 (the forward's
+    // bucket plan): window j's units sit at items[j*win_cap ...], queue position q
+    // of window j is seg_start[j] + its unit index, and each window owns W*K
+    // entries of its (b, g), ent_stride = nW*W*K entries per (b, g).
+    int win_cap;
+    int64_t ent_stride;
 };
+
+// Forward bucket plan (k_bucket.cu): entries/entw [B*h_kv][nW*W*K], counts and
+// cursors [J][nc]; fills the plan's queue (win_cap layout), per-window counts and
+// seg_start.  cnt and the plan counters must be zero on entry.
+cudaError_t launch_bucket_plan(const Shape &sh, const int32_t *idx, const float *w, const AttendPlan &P,
+                               int32_t *cnt, int32_t *cursor, int32_t *entries, float *entw, DevStatus *ds,
+                               cudaStream_t st);
 
 // tiles_done[J], comb_done[J], comb_head[J], then three words of magnitude bounds as
 // float bits: forward max|v|; backward max row norm of v, of dO, and max|k|
@@ -227,9 +241,10 @@ cudaError_t launch_select_tc(const Shape &sh, const void *q_slc, const float *kb
 
 cudaError_t launch_plan(const Shape &sh, const BwdWs &inv, const AttendPlan &plan, cudaStream_t st);
 bool attend_tc_supported(const Shape &sh);
-cudaError_t launch_attend_tc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv, const void *q,
-                             const void *k, const void *v, __half *acc, void *o, float *lse, DevStatus *ds,
-                             cudaStream_t st);
+// entries/entw: the bucket plan's lists (plan.ent_stride entries per (b, g))
+cudaError_t launch_attend_tc(const Shape &sh, const AttendPlan &plan, const int32_t *entries, const float *entw,
+                             const void *q, const void *k, const void *v, __half *acc, void *o, float *lse,
+                             DevStatus *ds, cudaStream_t st);
 // max|v| over the whole value tensor, as float bits, max-ed into *bits (zeroed by the caller)
 cudaError_t launch_vmax(const Shape &sh, const void *v, int32_t *bits, cudaStream_t st);
 cudaError_t launch_wsum(const Shape &sh, const int32_t *idx, const float *w, int32_t *bits, cudaStream_t st);

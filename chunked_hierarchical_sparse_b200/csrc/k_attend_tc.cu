@@ -223,17 +223,27 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         const int qstep = gridDim.x;
         int guard_ok_j = -1;  // highest window whose ring guard already passed
         struct Desc { int4 a, b; };
+        // queue position q of window jw is unit q - seg_start[jw] of jw's slice of the
+        // queue; the positions looked up only grow, so the window only moves forward
+        int jw = 0;
         auto load_desc = [&](int q) -> Desc {  // every lane loads the same 32 bytes
             Desc d;
-            if (q < total) { d.a = P.items[2 * q]; d.b = P.items[2 * q + 1]; }
-            else { d.a = make_int4(kItemEnd, 0, 0, 0); d.b = make_int4(0, 0, 0, 0); }
+            if (q < total) {
+                while (jw + 1 < P.J && q >= P.seg_start[jw + 1]) ++jw;
+                const int64_t u = (int64_t)jw * P.win_cap + (q - P.seg_start[jw]);
+                d.a = P.items[2 * u];
+                d.b = P.items[2 * u + 1];
+            } else {
+                d.a = make_int4(kItemEnd, 0, 0, 0);
+                d.b = make_int4(0, 0, 0, 0);
+            }
             return d;
         };
         struct Pay { int ea, eb; float wa, wb; };  // a unit's (token, slot) entries and weights, two per lane
         auto load_pay = [&](const Desc &d) -> Pay {
             Pay p{0, 0, 0.f, 0.f};
             if (d.a.x == kItemTile) {
-                const int64_t base = (int64_t)(d.a.y / P.nW) * P.L * P.K;
+                const int64_t base = (int64_t)(d.a.y / P.nW) * P.ent_stride;
                 const int ub = d.a.w + d.b.y * TT;
                 const int un = min(d.b.x, d.a.w + d.b.z * TT) - ub;
                 if (lane < un) { p.ea = entries[base + ub + lane]; p.wa = entw[base + ub + lane]; }
@@ -767,8 +777,9 @@ bool make_map_q3(CUtensorMap *m, const void *base, uint64_t rows) {
 }
 
 template <int D, int G>
-cudaError_t launch_tc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv, const void *q, const void *k,
-                      const void *v, __half *acc, void *o, float *lse, DevStatus *ds, cudaStream_t st) {
+cudaError_t launch_tc(const Shape &sh, const AttendPlan &plan, const int32_t *entries, const float *entw,
+                      const void *q, const void *k, const void *v, __half *acc, void *o, float *lse, DevStatus *ds,
+                      cudaStream_t st) {
     CUtensorMap mq, mk, mv;
     const bool qok = D == 128 ? make_map_q3(&mq, q, (uint64_t)sh.B * sh.L * sh.hq)
                               : make_map(&mq, q, D, (uint64_t)sh.B * sh.L * sh.hq, G);
@@ -782,7 +793,7 @@ cudaError_t launch_tc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv,
     int dev = 0, sms = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    attend_tc_kernel<D, G><<<sms, kThreads, smem, st>>>(mq, mk, mv, plan, inv.entries, inv.entw, acc,
+    attend_tc_kernel<D, G><<<sms, kThreads, smem, st>>>(mq, mk, mv, plan, entries, entw, acc,
                                                         (__nv_bfloat16 *)o, lse, ds);
     return cudaGetLastError();
 }
@@ -847,13 +858,13 @@ bool attend_tc_supported(const Shape &sh) {
            get_encode() != nullptr;
 }
 
-cudaError_t launch_attend_tc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv, const void *q,
-                             const void *k, const void *v, __half *acc, void *o, float *lse,
+cudaError_t launch_attend_tc(const Shape &sh, const AttendPlan &plan, const int32_t *entries, const float *entw,
+                             const void *q, const void *k, const void *v, __half *acc, void *o, float *lse,
                              DevStatus *ds, cudaStream_t st) {
-    if (sh.d == 128 && sh.G == 8) return launch_tc<128, 8>(sh, plan, inv, q, k, v, acc, o, lse, ds, st);
-    if (sh.d == 128 && sh.G == 16) return launch_tc<128, 16>(sh, plan, inv, q, k, v, acc, o, lse, ds, st);
-    if (sh.d == 64 && sh.G == 8) return launch_tc<64, 8>(sh, plan, inv, q, k, v, acc, o, lse, ds, st);
-    if (sh.d == 64 && sh.G == 16) return launch_tc<64, 16>(sh, plan, inv, q, k, v, acc, o, lse, ds, st);
+    if (sh.d == 128 && sh.G == 8) return launch_tc<128, 8>(sh, plan, entries, entw, q, k, v, acc, o, lse, ds, st);
+    if (sh.d == 128 && sh.G == 16) return launch_tc<128, 16>(sh, plan, entries, entw, q, k, v, acc, o, lse, ds, st);
+    if (sh.d == 64 && sh.G == 8) return launch_tc<64, 8>(sh, plan, entries, entw, q, k, v, acc, o, lse, ds, st);
+    if (sh.d == 64 && sh.G == 16) return launch_tc<64, 16>(sh, plan, entries, entw, q, k, v, acc, o, lse, ds, st);
     return cudaErrorInvalidValue;
 }
 

@@ -10,21 +10,24 @@
 // terms, kbar = hi + lo with hi = bf16(kbar), lo = bf16(kbar - hi), so
 //   q . kbar  ~=  q . hi + q . lo      (two tcgen05 MMAs into one fp32 TMEM tile)
 // with a residual of ~2^-16 of |kbar| per element -- far below the score gaps
-// that decide the top-K.  Chunk tiles of 64 pooled keys are streamed by TMA
-// into two stages; tile i is scored into TMEM buffer i % 2.
+// that decide the top-K.  Chunk tiles of 64 pooled keys are streamed by TMA;
+// two tiles form a block of 128 scores per token, held in one of two TMEM
+// buffers.
 //
-// Top-K: two epilogue warpgroups, one per TMEM buffer, so group e sees the
-// tiles i = e, e + 2, ... in increasing chunk order.  A thread owns one token
-// row and keeps a descending list of its group's best chunks in registers.
-// Because the chunks reach a group in increasing index order, a new chunk
-// beats an equal score already listed (ties go to the higher index), so the
-// filter against the current K-th best theta is one compare, x >= theta, and
-// a 32-chunk slice whose maximum is below theta is skipped after one warp vote.
-// A surviving chunk is inserted at its position (a popcount of parallel
-// compares) with a predicated shift.  At the end group 1 hands its list to
-// group 0 through shared memory, group 0 merges it (full score-then-index
-// order), lists the K chunks most-recent-first and forms the stick-breaking
-// weights.
+// Top-K (one token row per epilogue thread, one sorted list per row), block by
+// block, two passes over the block's scores in TMEM:
+//   pass 1  the maximum of each of KS column stripes (chunk index mod KS).  K of
+//           the stripes hold a score at least as large as the K-th largest stripe
+//           maximum tau, so the block's -- and the row's -- K-th best is >= tau;
+//   pass 2  every score >= max(tau, theta) (theta: the list's current K-th best,
+//           also a lower bound) is appended, branch-free, to the row's small
+//           candidate buffer in shared memory.
+// After pass 2 the buffered candidates are inserted into the list.  They come in
+// increasing chunk order, after every chunk already listed, so a candidate beats
+// an equal listed score (ties go to the higher index) and the insertion compares
+// scores only.  A buffer that would overflow is inserted early and the threshold
+// raised.  At the end the K chunks are listed most-recent-first and the
+// stick-breaking weights are formed.
 #include <math_constants.h>
 
 #include <algorithm>
@@ -38,8 +41,10 @@ using namespace sm100;
 
 namespace {
 
-constexpr int kSelThreads = 320;  // warp 0 TMA, warp 1 MMA, warps 2-5 and 6-9 the two epilogue groups
-constexpr int kSelN = 64;         // chunks per tile (two CTAs fit per SM)
+constexpr int kSelThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue (one TMEM lane quadrant each)
+constexpr int kSelN = 64;         // chunks per tile
+constexpr int kBlkTiles = 2;      // tiles per block (one TMEM buffer: 128 columns)
+constexpr int kCap = 12;          // candidate buffer entries per row
 constexpr uint64_t kSelWaitNs = 2000000000ull;
 
 template <int D> struct SelSmem {
@@ -48,12 +53,14 @@ template <int D> struct SelSmem {
     static constexpr int BHALF = kSelN * 128;         // kSelN chunks x 64 bf16
     static constexpr int BBYTES = 2 * NH * BHALF;     // hi + lo
     static constexpr int OFF_Q = 0;
-    static constexpr int OFF_B = OFF_Q + QBYTES;      // 2 stages; group 1's lists after the last tile
-    static constexpr int OFF_BAR = OFF_B + 2 * BBYTES;
+    static constexpr int OFF_B = OFF_Q + QBYTES;      // 2 stages
+    static constexpr int OFF_CS = OFF_B + 2 * BBYTES; // [kCap][128] candidate scores
+    static constexpr int OFF_CC = OFF_CS + kCap * 128 * 4;  // [kCap][128] candidate chunks
+    static constexpr int OFF_BAR = OFF_CC + kCap * 128 * 4;
     static constexpr int BYTES = OFF_BAR + 16 * 8 + 64;
     static constexpr int ALLOC = BYTES + 1024;
 };
-static_assert(2 * SelSmem<64>::BBYTES >= 128 * 16 * 8, "group lists do not fit in the tile stages");
+static_assert(2 * (SelSmem<128>::ALLOC + 1024) <= 228 * 1024, "two selection CTAs must fit one SM");
 
 // The sorted list: KM (score, chunk) slots, best first.  The first KM - K slots
 // hold +inf sentinels that nothing displaces, so slot KM - 1 is always the
@@ -71,91 +78,59 @@ template <int KM> struct TopList {
         }
     }
     __device__ __forceinline__ float theta() const { return s[KM - 1]; }
-
-    // place (x, cx) at slot p, shifting slots p.. down by one (the last falls off)
-    __device__ __forceinline__ void put(int p, float x, int cx) {
-#pragma unroll
-        for (int k = KM - 1; k >= 1; --k) {
-            const bool sh = k > p, eq = k == p;
-            s[k] = sh ? s[k - 1] : (eq ? x : s[k]);
-            c[k] = sh ? c[k - 1] : (eq ? cx : c[k]);
-        }
-        s[0] = (p == 0) ? x : s[0];
-        c[0] = (p == 0) ? cx : c[0];
-    }
-    // a chunk with a higher index than every listed one, x >= theta()
+    // a chunk with a higher index than every listed one: it beats equal scores.
+    // Top-down pass: the element being placed moves down while it beats the slot.
     __device__ __forceinline__ void insert_newest(float x, int cx) {
-        int p = 0;
 #pragma unroll
-        for (int k = 0; k < KM; ++k) p += s[k] > x ? 1 : 0;
-        put(p, x, cx);
-    }
-    // any chunk: score first, then the higher index
-    __device__ __forceinline__ void insert_any(float x, int cx) {
-        if (!(x > s[KM - 1] || (x == s[KM - 1] && cx > c[KM - 1]))) return;
-        int p = 0;
-#pragma unroll
-        for (int k = 0; k < KM; ++k) p += (s[k] > x || (s[k] == x && c[k] > cx)) ? 1 : 0;
-        put(p, x, cx);
+        for (int k = 0; k < KM; ++k) {
+            const bool sw = x >= s[k];
+            const float ts = s[k];
+            const int tc = c[k];
+            s[k] = sw ? x : ts;
+            c[k] = sw ? cx : tc;
+            x = sw ? ts : x;
+            cx = sw ? tc : cx;
+        }
     }
 };
 
-// v[e] for a lane-varying e in [0, 32), by a select tree on e's bits (stays in registers)
-__device__ __forceinline__ float pick32(const float (&v)[32], int e) {
-    float t16[16], t8[8], t4[4];
+// ascending sort of KS floats (bitonic network, static indices)
+template <int KS> __device__ __forceinline__ void sort_asc(float (&a)[KS]) {
 #pragma unroll
-    for (int i = 0; i < 16; ++i) t16[i] = (e & 1) ? v[2 * i + 1] : v[2 * i];
+    for (int k = 2; k <= KS; k <<= 1)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) t8[i] = (e & 2) ? t16[2 * i + 1] : t16[2 * i];
+        for (int j = k >> 1; j > 0; j >>= 1)
 #pragma unroll
-    for (int i = 0; i < 4; ++i) t4[i] = (e & 4) ? t8[2 * i + 1] : t8[2 * i];
-    const float t2a = (e & 8) ? t4[1] : t4[0], t2b = (e & 8) ? t4[3] : t4[2];
-    return (e & 16) ? t2b : t2a;
-}
-
-// one 32-chunk slice [c0, c0 + 32) of this row's raw scores v (chunks < ne eligible)
-template <int KM>
-__device__ __forceinline__ void scan_slice(TopList<KM> &tl, const float (&v)[32], int c0, int ne) {
-    float m8[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) m8[i] = fmaxf(fmaxf(v[4 * i], v[4 * i + 1]), fmaxf(v[4 * i + 2], v[4 * i + 3]));
-    const float vmax = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])), fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
-    const bool any = c0 < ne && vmax >= tl.theta();
-    if (!__any_sync(0xffffffffu, any)) return;
-    uint32_t m = 0;
-    if (any) {
-        const float th = tl.theta();
-        const int nel = ne - c0;  // eligible chunks in the slice (may exceed 32)
-#pragma unroll
-        for (int e = 0; e < 32; ++e) m |= (v[e] >= th && e < nel) ? (1u << e) : 0u;
-    }
-    while (m) {
-        const int e = __ffs(m) - 1;
-        m &= m - 1;
-        const float x = pick32(v, e);
-        if (x >= tl.theta()) tl.insert_newest(x, c0 + e);
-    }
+            for (int i = 0; i < KS; ++i) {
+                const int l = i ^ j;
+                if (l > i) {
+                    const bool up = (i & k) == 0;
+                    const float lo = fminf(a[i], a[l]), hi = fmaxf(a[i], a[l]);
+                    a[i] = up ? lo : hi;
+                    a[l] = up ? hi : lo;
+                }
+            }
 }
 
 }  // namespace
 
 template <int D, int KM>
-__global__ void __launch_bounds__(kSelThreads, KM <= 8 ? 2 : 1) select_tc_kernel(
+__global__ void __launch_bounds__(kSelThreads, 2) select_tc_kernel(
     const __grid_constant__ CUtensorMap tm_qs, const __grid_constant__ CUtensorMap tm_hi,
     const __grid_constant__ CUtensorMap tm_lo, int32_t *__restrict__ idx, float *__restrict__ wout,
     int L, int hkv, int nc, int K, DevStatus *ds) {
     using SL = SelSmem<D>;
+    constexpr int KS = KM;  // column stripes of pass 1 (K <= KM of them hold the threshold)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + SL::OFF_BAR);
     uint64_t *q_full = bar;
-    uint64_t *b_full = bar + 1;     // [2]
-    uint64_t *b_empty = bar + 3;    // [2]
-    uint64_t *a_full = bar + 5;     // [2]  TMEM buffer e scored (MMA -> group e)
-    uint64_t *a_empty = bar + 7;    // [2]  TMEM buffer e read (group e -> MMA)
+    uint64_t *b_full = bar + 1;     // [2]  tile stage loaded (TMA -> MMA)
+    uint64_t *b_empty = bar + 3;    // [2]  tile stage read (MMA -> TMA)
+    uint64_t *a_full = bar + 5;     // [2]  TMEM buffer holds a scored block (MMA -> epilogue)
+    uint64_t *a_empty = bar + 7;    // [2]  TMEM buffer read (epilogue -> MMA)
     uint64_t *mma_done = bar + 9;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + SL::OFF_BAR + 16 * 8);
-    volatile int *fail = reinterpret_cast<volatile int *>(sm + SL::OFF_BAR + 16 * 8 + 16);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // token blocks late in the sequence score the most chunks: they are issued first
@@ -165,6 +140,7 @@ __global__ void __launch_bounds__(kSelThreads, KM <= 8 ? 2 : 1) select_tc_kernel
     const int tlast = min(t0 + 128, L) - 1;
     const int ne_max = min(tlast / kChunk, nc);
     const int ntiles = (ne_max + kSelN - 1) / kSelN;
+    const int nblk = (ntiles + kBlkTiles - 1) / kBlkTiles;
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
@@ -173,10 +149,9 @@ __global__ void __launch_bounds__(kSelThreads, KM <= 8 ? 2 : 1) select_tc_kernel
             mbar_init(&a_full[i], 1); mbar_init(&a_empty[i], 4);
         }
         mbar_init(mma_done, 1);
-        *fail = 0;
         mbar_fence_init();
     }
-    if (warp == 1) { tmem_alloc(tmem_slot, 2 * kSelN); tmem_relinquish(); }
+    if (warp == 1) { tmem_alloc(tmem_slot, 2 * kBlkTiles * kSelN); tmem_relinquish(); }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -196,6 +171,7 @@ __global__ void __launch_bounds__(kSelThreads, KM <= 8 ? 2 : 1) select_tc_kernel
             for (int h = 0; h < SL::NH; ++h)
                 tma_load_3d(sm + SL::OFF_Q + h * 128 * 128, &tm_qs, h * 64, g, b * L + t0, q_full);
         }
+        int issued = 0;
         for (int i = 0; i < ntiles && ok; ++i) {
             const int s = i & 1;
             if (i >= 2 && !warp_wait(&b_empty[s], ((i >> 1) - 1) & 1)) { ok = false; break; }
@@ -209,13 +185,13 @@ __global__ void __launch_bounds__(kSelThreads, KM <= 8 ? 2 : 1) select_tc_kernel
                     tma_load_2d(dst + (SL::NH + h) * SL::BHALF, &tm_lo, h * 64, row, &b_full[s]);
                 }
             }
+            issued = i + 1;
             __syncwarp();
         }
         if (!ok && lane == 0) {
-            *fail = 1;
             report(ds, HSA_ERR_TIMEOUT, kKSelectTc, 1, t0);
             // let the loads already issued land before the CTA can go away (bounded)
-            for (int i = max(0, ntiles - 2); i < ntiles; ++i) mbar_wait(&b_full[i & 1], (i >> 1) & 1, kSelWaitNs);
+            for (int i = max(0, issued - 2); i < issued; ++i) mbar_wait(&b_full[i & 1], (i >> 1) & 1, kSelWaitNs);
         }
     } else if (warp == 1) {
         // -------------------------------------------------- MMA issuer
@@ -224,13 +200,15 @@ __global__ void __launch_bounds__(kSelThreads, KM <= 8 ? 2 : 1) select_tc_kernel
         if (ntiles > 0 && !warp_wait(q_full, 0)) ok = false;
         for (int i = 0; i < ntiles && ok; ++i) {
             const int s = i & 1;
+            const int blk = i / kBlkTiles, buf = blk & 1, ti = i % kBlkTiles;
             if (!warp_wait(&b_full[s], (i >> 1) & 1)) { ok = false; break; }
-            if (i >= 2 && !warp_wait(&a_empty[s], ((i >> 1) - 1) & 1)) { ok = false; break; }
+            // the block's TMEM buffer is free once the epilogue has read block blk - 2
+            if (ti == 0 && blk >= 2 && !warp_wait(&a_empty[buf], ((blk >> 1) - 1) & 1)) { ok = false; break; }
             tc_fence_after();
             if (lane == 0) {
                 const uint32_t qa = smem_u32(sm + SL::OFF_Q);
                 const uint32_t bb = smem_u32(sm + SL::OFF_B + s * SL::BBYTES);
-                const uint32_t dcol = tmem + s * kSelN;
+                const uint32_t dcol = tmem + buf * (kBlkTiles * kSelN) + ti * kSelN;
 #pragma unroll
                 for (int part = 0; part < 2; ++part)  // hi then lo
 #pragma unroll
@@ -240,55 +218,126 @@ __global__ void __launch_bounds__(kSelThreads, KM <= 8 ? 2 : 1) select_tc_kernel
                                     smem_desc_sw128(bb + (part * SL::NH + h) * SL::BHALF + kk * 32, 16, 1024), idesc,
                                     (part | ks) != 0);
                     }
-                mma_commit(&a_full[s]);
                 mma_commit(&b_empty[s]);
+                if (ti == kBlkTiles - 1 || i == ntiles - 1) mma_commit(&a_full[buf]);
             }
             __syncwarp();
         }
-        if (!ok && lane == 0) { *fail = 1; report(ds, HSA_ERR_TIMEOUT, kKSelectTc, 2, t0); }
+        if (!ok && lane == 0) report(ds, HSA_ERR_TIMEOUT, kKSelectTc, 2, t0);
         if (lane == 0) { mma_commit(mma_done); mbar_wait(mma_done, 0, kSelWaitNs); }
         __syncwarp();
     } else {
-        // -------------------------------------------------- two epilogue groups, one token row per thread
-        const int eg = (warp - 2) >> 2;   // group = TMEM buffer = tile parity
+        // -------------------------------------------------- epilogue: one token row per thread
         const int wq = warp & 3;          // TMEM lane quadrant of this warp
         const int r = wq * 32 + lane;
         const int t = t0 + r;
         const int ne = (t < L) ? min(t / kChunk, nc) : 0;
-        const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16) + eg * kSelN;
+        const int ne_warp = __reduce_min_sync(0xffffffffu, (unsigned)ne);  // every lane: chunks < ne_warp eligible
+        float *cs = reinterpret_cast<float *>(sm + SL::OFF_CS) + r;  // candidate i at cs[i * 128]
+        int *cc = reinterpret_cast<int *>(sm + SL::OFF_CC) + r;
         TopList<KM> tl;
         tl.init(K);
+        int n = 0;  // buffered candidates
+        auto flush = [&]() {
+            for (int i = 0; i < n; ++i) {
+                const float x = cs[i * 128];
+                if (x >= tl.theta()) tl.insert_newest(x, cc[i * 128]);
+            }
+            n = 0;
+        };
         bool ok = true;
-        for (int i = eg; i < ntiles; i += 2) {
-            if (!warp_wait(&a_full[eg], (i >> 1) & 1)) { ok = false; break; }
+        for (int blk = 0; blk < nblk; ++blk) {
+            const int buf = blk & 1;
+            const int c0 = blk * kBlkTiles * kSelN;
+            const int ntb = min(kBlkTiles, ntiles - blk * kBlkTiles);
+            const uint32_t base = tmem + ((uint32_t)(wq * 32) << 16) + buf * (kBlkTiles * kSelN);
+            if (!warp_wait(&a_full[buf], (blk >> 1) & 1)) { ok = false; break; }
             tc_fence_after();
-            float v0[32], v1[32];
-            tmem_ld32(lane_base, v0);
-            tmem_ld32(lane_base + 32, v1);
-            tmem_wait_ld();
+            // every chunk of the block is eligible for every row of the warp, or masking is needed
+            const bool full = c0 + kBlkTiles * kSelN <= ne_warp;
+            // ---- pass 1: stripe maxima -> tau
+            float st[KS];
+#pragma unroll
+            for (int j = 0; j < KS; ++j) st[j] = -CUDART_INF_F;
+            for (int ti = 0; ti < ntb; ++ti) {
+                float v0[32], v1[32];
+                tmem_ld32(base + ti * kSelN, v0);
+                tmem_ld32(base + ti * kSelN + 32, v1);
+                tmem_wait_ld();
+                const int cb = c0 + ti * kSelN;
+                if (full) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        st[e % KS] = fmaxf(st[e % KS], v0[e]);
+                        st[(e + 32) % KS] = fmaxf(st[(e + 32) % KS], v1[e]);
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        st[e % KS] = fmaxf(st[e % KS], cb + e < ne ? v0[e] : -CUDART_INF_F);
+                        st[(e + 32) % KS] = fmaxf(st[(e + 32) % KS], cb + 32 + e < ne ? v1[e] : -CUDART_INF_F);
+                    }
+                }
+            }
+            float tau;
+            if (K == KS) {  // the smallest stripe maximum
+                tau = st[0];
+#pragma unroll
+                for (int j = 1; j < KS; ++j) tau = fminf(tau, st[j]);
+            } else {        // the K-th largest stripe maximum
+                sort_asc<KS>(st);
+                tau = st[0];
+#pragma unroll
+                for (int j = 1; j < KS; ++j) tau = (j == KS - K) ? st[j] : tau;
+            }
+            float thr = fmaxf(tau, tl.theta());
+            // ---- pass 2: buffer every eligible score >= thr
+            for (int ti = 0; ti < ntb; ++ti) {
+                float v[64];
+                tmem_ld32(base + ti * kSelN, *reinterpret_cast<float(*)[32]>(&v[0]));
+                tmem_ld32(base + ti * kSelN + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
+                tmem_wait_ld();
+                const int cb = c0 + ti * kSelN;
+                const int nel = full ? 64 : max(0, min(64, ne - cb));
+#pragma unroll
+                for (int hf = 0; hf < 2; ++hf) {
+                    uint32_t m = 0;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) m |= (v[hf * 32 + e] >= thr) ? (1u << e) : 0u;
+                    const int el = nel - hf * 32;
+                    m &= el >= 32 ? 0xffffffffu : (el <= 0 ? 0u : ((1u << el) - 1u));
+                    if (n + __popc(m) > kCap) {  // rare: make room, raise the threshold
+                        flush();
+                        thr = fmaxf(thr, tl.theta());
+#pragma unroll
+                        for (int e = 0; e < 32; ++e) m &= (v[hf * 32 + e] >= thr) ? 0xffffffffu : ~(1u << e);
+                        if (__popc(m) > kCap) {  // still too many: insert them directly
+#pragma unroll
+                            for (int e = 0; e < 32; ++e)
+                                if ((m >> e) & 1u) {
+                                    if (v[hf * 32 + e] >= tl.theta()) tl.insert_newest(v[hf * 32 + e], cb + hf * 32 + e);
+                                }
+                            m = 0;
+                            thr = fmaxf(thr, tl.theta());
+                        }
+                    }
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) {
+                        if ((m >> e) & 1u) {
+                            cs[n * 128] = v[hf * 32 + e];
+                            cc[n * 128] = cb + hf * 32 + e;
+                            ++n;
+                        }
+                    }
+                }
+            }
             tc_fence_before();
             __syncwarp();
-            mbar_arrive_lane0(&a_empty[eg], lane);  // the buffer is free for tile i + 2
-            scan_slice(tl, v0, i * kSelN, ne);
-            scan_slice(tl, v1, i * kSelN + 32, ne);
+            mbar_arrive_lane0(&a_empty[buf], lane);  // the buffer is free for block blk + 2
+            flush();
         }
-        if (!ok) { *fail = 1; if (lane == 0) report(ds, HSA_ERR_TIMEOUT, kKSelectTc, 3, t0); }
-        // group 1 hands its list over in the tile stages, once the MMA warp's final
-        // commit shows that every MMA (and so every tile load) has completed
-        float *ls = reinterpret_cast<float *>(sm + SL::OFF_B);
-        int *lc = reinterpret_cast<int *>(sm + SL::OFF_B) + 128 * KM;
-        if (eg == 1) {
-            if (!warp_wait(mma_done, 0)) { *fail = 1; if (lane == 0) report(ds, HSA_ERR_TIMEOUT, kKSelectTc, 4, t0); }
-#pragma unroll
-            for (int k = 0; k < KM; ++k) { ls[k * 128 + r] = tl.s[k]; lc[k * 128 + r] = tl.c[k]; }
-        }
-        asm volatile("bar.sync 1, 256;" ::: "memory");
-        if (eg == 0 && !*fail && t < L) {
-#pragma unroll
-            for (int k = 0; k < KM; ++k) {
-                const int c1 = lc[k * 128 + r];
-                if (c1 >= 0 && c1 != 0x7fffffff) tl.insert_any(ls[k * 128 + r], c1);
-            }
+        if (!ok && lane == 0) report(ds, HSA_ERR_TIMEOUT, kKSelectTc, 3, t0);
+        if (ok && t < L) {
             // most-recent-first: order the chosen chunks by descending index (empty = -1 last)
 #pragma unroll
             for (int k = 0; k < KM; ++k)
@@ -325,7 +374,7 @@ __global__ void __launch_bounds__(kSelThreads, KM <= 8 ? 2 : 1) select_tc_kernel
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, 2 * kSelN);
+    if (warp == 1) tmem_dealloc(tmem, 2 * kBlkTiles * kSelN);
 }
 
 namespace {

@@ -54,10 +54,10 @@ struct FwdWs {
     bool tc;             // chunk-major tensor-core path
     int32_t *entries;    // per (b, g): nW windows x W*K (token, slot) entries, bucket by bucket
     float *entw;         //   and their weights
-    int32_t *bucket_cnt, *bucket_cur;  // [J][nc] entries per bucket, scatter cursors
+    int32_t *bucket_hist;  // [J][blocks][nc] per token block chunk counts -> positions
     AttendPlan plan;
     __half *acc;         // fp16 output-accumulator ring, scaled (chunk-major path)
-    size_t zero_bytes;   // plan counters .. bucket counts: cleared by one memset per call
+    size_t zero_bytes;   // the plan counters: cleared by one memset per call
 };
 
 // token->chunk lists of the chunk-major passes (with the entries' weights if `weights`)
@@ -123,10 +123,9 @@ static FwdWs carve_fwd(const Shape &sh, void *ws, size_t *bytes) {
         P.win_ncomb = c.take<int32_t>((size_t)P.J);
         P.seg_start = c.take<int32_t>((size_t)P.J + 1);
         P.items = c.take<int4>((size_t)2 * P.J * P.win_cap);
-        f.bucket_cur = c.take<int32_t>((size_t)P.J * sh.nc);
+        f.bucket_hist = c.take<int32_t>(bucket_hist_elems(P));
         const size_t z0 = c.off;
         P.counters = c.take<int32_t>(plan_counter_count(P.J));
-        f.bucket_cnt = c.take<int32_t>((size_t)P.J * sh.nc);
         f.zero_bytes = c.off - z0;
         f.acc = c.take<__half>(attend_acc_elems(P.W, sh.G, sh.d));
     }
@@ -285,12 +284,12 @@ static cudaError_t run_attend(const Shape &sh, const void *q, const void *k, con
         return e;
     }
     // chunk-major tensor-core path: bucket the selection by (window, chunk), queue the
-    // work units, attend.  The forward's pooling pass has cleared the plan counters and
-    // bucket counts already (and written max|v|); a caller-given selection clears them here.
+    // work units, attend.  The forward's pooling pass has cleared the plan counters
+    // already (and written max|v|); a caller-given selection clears them here.
     if (e == cudaSuccess && given_sel) e = cudaMemsetAsync(f.plan.counters, 0, f.zero_bytes, st);
     if (e == cudaSuccess)
         e = timed(HSA_K_INVERT, sh.nc > 0 ? 3 : 1, st, [&] {
-            return launch_bucket_plan(sh, f.idx, f.w, f.plan, f.bucket_cnt, f.bucket_cur, f.entries, f.entw, ds, st);
+            return launch_bucket_plan(sh, f.idx, f.w, f.plan, f.bucket_hist, f.entries, f.entw, ds, st);
         });
     if (e == cudaSuccess)  // the used accumulator slots start at zero (the kernel re-zeroes them after use)
         e = cudaMemsetAsync(f.acc, 0,

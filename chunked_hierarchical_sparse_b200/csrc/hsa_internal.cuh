@@ -199,12 +199,12 @@ struct AttendPlan {
     int64_t ent_stride;
 };
 
-// Forward bucket plan (k_bucket.cu): entries/entw [B*h_kv][nW*W*K], counts and
-// cursors [J][nc]; fills the plan's queue (win_cap layout), per-window counts and
-// seg_start.  cnt and the plan counters must be zero on entry.
+// Forward bucket plan (k_bucket.cu): entries/entw [B*h_kv][nW*W*K], per-block
+// chunk histograms hist [bucket_hist_elems(P)]; fills the plan's queue (win_cap
+// layout), per-window counts and seg_start.  The plan counters must be zero on entry.
+size_t bucket_hist_elems(const AttendPlan &P);
 cudaError_t launch_bucket_plan(const Shape &sh, const int32_t *idx, const float *w, const AttendPlan &P,
-                               int32_t *cnt, int32_t *cursor, int32_t *entries, float *entw, DevStatus *ds,
-                               cudaStream_t st);
+                               int32_t *hist, int32_t *entries, float *entw, DevStatus *ds, cudaStream_t st);
 
 // tiles_done[J], comb_done[J], comb_head[J], then three words of magnitude bounds as
 // float bits: forward max|v|; backward max row norm of v, of dO, and max|k|

@@ -8,34 +8,40 @@
 //
 // The tokens of each (b, g) are cut into windows of W tokens; window
 // j = (b*h_kv + g)*nW + w.  Inside a window, the entries of chunk c form the
-// bucket (j, c).  Three launches:
-//   1. count:   per bucket, the number of entries (shared-memory histogram of a
-//               block of tokens, flushed with one global atomic per chunk seen);
-//   2. scan:    one block per window: bucket starts (exclusive scan of the
-//               counts), each bucket cut into tiles of TT = 128/G tokens and
-//               tiles into work units of up to unit_tiles tiles (one K/V load),
-//               the units' descriptors written into the window's slice of the
-//               queue, and the window's unit, tile and convert-item counts;
-//   3. scatter: every entry takes the next position of its bucket (an atomic
-//               cursor) and stores t * 16 + slot and its weight there.
+// bucket (j, c).  A window's tokens are processed in blocks of kCountRows.
+// Three launches:
+//   1. count:   per token block, a histogram over chunks (shared memory),
+//               written as one row of hist[j][block][c];
+//   2. scan:    one CTA per window: per chunk, the exclusive prefix of its
+//               counts over the window's blocks (in place: each block's first
+//               position inside the bucket), the bucket starts (an exclusive
+//               scan of the bucket sizes), each bucket cut into tiles of
+//               TT = 128/G tokens and tiles into work units of up to
+//               unit_tiles tiles (one K/V load), the units' descriptors written
+//               into the window's slice of the queue, and the window's unit,
+//               tile and convert-item counts; the last CTA to finish turns the
+//               unit counts into queue positions (seg_start);
+//   3. scatter: per token block, shared-memory cursors start at the block's
+//               positions; each (token, slot) entry takes the next position of
+//               its bucket and stores t * 16 + slot and its weight there.
 // Window w of (b, g) owns the fixed slice [w*W*K, (w+1)*W*K) of that (b, g)'s
-// entries and the slice [j*cap, (j+1)*cap) of the queue, so no step needs a
-// scan across windows; the attention kernel turns the per-window unit counts
-// into queue positions itself.  The order of the entries inside a bucket is
-// the order in which the atomics land: it changes only the order in which a
-// token's chunk outputs are summed.
+// entries and the slice [j*cap, (j+1)*cap) of the queue.  Inside a bucket the
+// entries of one block come in the order its shared-memory atomics land; the
+// blocks are in token order.
 #include "hsa_internal.cuh"
 
 namespace hsa {
 
 namespace {
-constexpr int kCountRows = 1024;  // (token, group) rows per counting block: one window, one (b, g)
+constexpr int kCountRows = 512;  // (token, group) rows per counting block: one window, one (b, g)
 }
 
 // Block: kCountRows consecutive tokens of one (b, g), all in one window (W is a
-// multiple of kCountRows or the block is the window's tail).
+// multiple of kCountRows or the block is the window's tail).  A thread takes
+// whole (token, group) rows: their K indices arrive in two 16-byte loads, all
+// issued before any of the shared-memory counts.
 __global__ void __launch_bounds__(256) bucket_count_kernel(const int32_t *__restrict__ idx, AttendPlan P,
-                                                           int32_t *__restrict__ cnt, DevStatus *ds) {
+                                                           int32_t *__restrict__ hist, DevStatus *ds) {
     extern __shared__ int h_s[];  // [nc]
     const int nc = P.nc, K = P.K;
     const int blocks_per_win = (P.W + kCountRows - 1) / kCountRows;
@@ -46,20 +52,35 @@ __global__ void __launch_bounds__(256) bucket_count_kernel(const int32_t *__rest
     const int t1 = min(min(t0 + kCountRows, (w + 1) * P.W), P.L);
     for (int c = threadIdx.x; c < nc; c += blockDim.x) h_s[c] = 0;
     __syncthreads();
-    for (int e = threadIdx.x; e < (t1 - t0) * K; e += blockDim.x) {
-        const int t = t0 + e / K, kk = e % K;
-        const int c = idx[(((int64_t)b * P.L + t) * P.hkv + g) * K + kk];
-        if (c < 0) continue;  // an empty slot
-        if (c >= nc || c >= t / kChunk) {  // not a causal complete chunk: skipped and reported
-            report(ds, HSA_ERR_DEVICE_CHECK, kKInvert, t, c);
-            continue;
-        }
-        atomicAdd(&h_s[c], 1);
+    constexpr int kRowsPerThread = kCountRows / 256;
+    int sel[kRowsPerThread][kMaxK];
+#pragma unroll
+    for (int u = 0; u < kRowsPerThread; ++u) {  // all loads first
+        const int t = t0 + u * 256 + threadIdx.x;
+        const int32_t *row = idx + (((int64_t)b * P.L + t) * P.hkv + g) * K;
+#pragma unroll
+        for (int kk = 0; kk < kMaxK; ++kk) sel[u][kk] = (t < t1 && kk < K) ? row[kk] : -1;
     }
+    int bad_t = -1, bad_c = 0;  // an entry that is not a causal complete chunk: skipped and reported
+#pragma unroll
+    for (int u = 0; u < kRowsPerThread; ++u) {
+        const int t = t0 + u * 256 + threadIdx.x;
+#pragma unroll
+        for (int kk = 0; kk < kMaxK; ++kk) {
+            const int c = sel[u][kk];
+            if (c < 0) continue;  // an empty slot (or no such token / slot)
+            if (c >= nc || c >= t / kChunk) {
+                bad_t = t;
+                bad_c = c;
+                continue;
+            }
+            atomicAdd(&h_s[c], 1);
+        }
+    }
+    if (bad_t >= 0) report(ds, HSA_ERR_DEVICE_CHECK, kKInvert, bad_t, bad_c);
     __syncthreads();
-    int32_t *out = cnt + (int64_t)j * nc;
-    for (int c = threadIdx.x; c < nc; c += blockDim.x)
-        if (h_s[c]) atomicAdd(&out[c], h_s[c]);
+    int32_t *out = hist + (int64_t)blockIdx.x * nc;  // row (j, block) = blockIdx.x
+    for (int c = threadIdx.x; c < nc; c += blockDim.x) out[c] = h_s[c];
 }
 
 // In-place exclusive scan of a[0..n) by one block; returns the total.
@@ -100,18 +121,28 @@ __device__ int bucket_block_scan(int *a, int n, int *wsum) {
 }
 
 // One block (1024 threads) per window j.
-__global__ void __launch_bounds__(1024) bucket_scan_kernel(AttendPlan P, const int32_t *__restrict__ cnt,
-                                                          int32_t *__restrict__ cursor) {
+__global__ void __launch_bounds__(1024) bucket_scan_kernel(AttendPlan P, int32_t *__restrict__ hist) {
     extern __shared__ int sm_b[];
-    int *start = sm_b;         // [nc] bucket starts within the window's slice
-    int *units = sm_b + P.nc;  // [nc] work units per bucket -> their first queue slot
+    int *start = sm_b;             // [nc] bucket starts within the window's slice
+    int *units = sm_b + P.nc;      // [nc] work units per bucket -> their first queue slot
+    int *bcnt = sm_b + 2 * P.nc;   // [nc] bucket sizes
     __shared__ int wsum[32];
     const int j = blockIdx.x, nc = P.nc, TT = P.TT, UT = P.unit_tiles;
     const int w = j % P.nW;
-    const int32_t *cj = cnt + (int64_t)j * nc;
+    const int nblk = (P.W + kCountRows - 1) / kCountRows;
+    int32_t *hj = hist + (int64_t)j * nblk * nc;
+    // per chunk: the bucket size (sum over the window's blocks; the loads of a
+    // column are independent and all in flight together)
+    for (int c = threadIdx.x; c < nc; c += blockDim.x) {
+        int run = 0;
+#pragma unroll 8
+        for (int k = 0; k < nblk; ++k) run += __ldcg(hj + (int64_t)k * nc + c);
+        bcnt[c] = run;
+    }
+    __syncthreads();
     int my_tiles = 0;
     for (int c = threadIdx.x; c < nc; c += blockDim.x) {
-        const int n = cj[c];
+        const int n = bcnt[c];
         const int nt = (n + TT - 1) / TT;
         start[c] = n;
         units[c] = (nt + UT - 1) / UT;
@@ -128,9 +159,22 @@ __global__ void __launch_bounds__(1024) bucket_scan_kernel(AttendPlan P, const i
     const int64_t ebase = (int64_t)w * P.W * P.K;  // the window's slice of its (b, g) entries
     int4 *items = P.items + (int64_t)2 * j * P.win_cap;
     for (int c = threadIdx.x; c < nc; c += blockDim.x) {
-        const int n = cj[c];
+        const int n = bcnt[c];
         const int e0 = (int)(ebase + start[c]);
-        cursor[(int64_t)j * nc + c] = e0;
+        // each block's first position in the bucket: e0 + the counts of the blocks before it
+        // (loads issued in groups of 8 ahead of the dependent stores)
+        int run = e0;
+        for (int k0 = 0; k0 < nblk; k0 += 8) {
+            int v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = k0 + u < nblk ? __ldcg(hj + (int64_t)(k0 + u) * nc + c) : 0;
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+                if (k0 + u < nblk) {
+                    hj[(int64_t)(k0 + u) * nc + c] = run;
+                    run += v[u];
+                }
+        }
         if (n == 0) continue;
         const int nt = (n + TT - 1) / TT;
         for (int u = units[c], t0 = 0; t0 < nt; ++u, t0 += UT) {
@@ -184,49 +228,76 @@ __global__ void __launch_bounds__(1024) bucket_scan_kernel(AttendPlan P, const i
     }
 }
 
-// One thread per (b, t, g) row: its entries go to the next positions of their buckets.
+// Block: the same kCountRows tokens as the counting block; shared-memory cursors
+// start at the block's first position in each bucket.  A thread takes whole
+// (token, group) rows; all loads are issued before any cursor update.
 __global__ void __launch_bounds__(256) bucket_scatter_kernel(const int32_t *__restrict__ idx, const float *__restrict__ w,
-                                                             AttendPlan P, int32_t *__restrict__ cursor,
+                                                             AttendPlan P, const int32_t *__restrict__ hist,
                                                              int32_t *__restrict__ entries, float *__restrict__ entw) {
-    const int64_t rows = (int64_t)P.B * P.L * P.hkv;
-    const int64_t r = blockIdx.x * (int64_t)blockDim.x + threadIdx.x;
-    if (r >= rows) return;
-    const int g = (int)(r % P.hkv);
-    const int64_t bt = r / P.hkv;
-    const int t = (int)(bt % P.L), b = (int)(bt / P.L);
-    const int bg = b * P.hkv + g;
-    const int j = bg * P.nW + t / P.W;
-    const int64_t ebase = (int64_t)bg * P.nW * P.W * P.K;  // the (b, g) entries
-    for (int kk = 0; kk < P.K; ++kk) {
-        const int c = idx[r * P.K + kk];
-        if (c < 0 || c >= P.nc || c >= t / kChunk) continue;  // empty or reported by the count
-        const int pos = atomicAdd(&cursor[(int64_t)j * P.nc + c], 1);
-        entries[ebase + pos] = t * 16 + kk;
-        entw[ebase + pos] = w[r * P.K + kk];
+    extern __shared__ int cur[];  // [nc]
+    const int nc = P.nc, K = P.K;
+    const int blocks_per_win = (P.W + kCountRows - 1) / kCountRows;
+    const int j = blockIdx.x / blocks_per_win;
+    const int bg = j / P.nW, wi = j % P.nW;
+    const int b = bg / P.hkv, g = bg % P.hkv;
+    const int t0 = wi * P.W + (blockIdx.x % blocks_per_win) * kCountRows;
+    const int t1 = min(min(t0 + kCountRows, (wi + 1) * P.W), P.L);
+    const int32_t *hrow = hist + (int64_t)blockIdx.x * nc;
+    for (int c = threadIdx.x; c < nc; c += blockDim.x) cur[c] = hrow[c];
+    constexpr int kRowsPerThread = kCountRows / 256;
+    int sel[kRowsPerThread][kMaxK];
+    float wt[kRowsPerThread][kMaxK];
+#pragma unroll
+    for (int u = 0; u < kRowsPerThread; ++u) {
+        const int t = t0 + u * 256 + threadIdx.x;
+        const int64_t row = (((int64_t)b * P.L + t) * P.hkv + g) * K;
+#pragma unroll
+        for (int kk = 0; kk < kMaxK; ++kk) {
+            const bool in = t < t1 && kk < K;
+            sel[u][kk] = in ? idx[row + kk] : -1;
+            wt[u][kk] = in ? w[row + kk] : 0.f;
+        }
+    }
+    __syncthreads();
+    const int64_t ebase = (int64_t)bg * P.ent_stride;  // the (b, g) entries
+#pragma unroll
+    for (int u = 0; u < kRowsPerThread; ++u) {
+        const int t = t0 + u * 256 + threadIdx.x;
+#pragma unroll
+        for (int kk = 0; kk < kMaxK; ++kk) {
+            const int c = sel[u][kk];
+            if (c < 0 || c >= nc || c >= t / kChunk) continue;  // empty, or reported by the count
+            const int pos = atomicAdd(&cur[c], 1);
+            entries[ebase + pos] = t * 16 + kk;
+            entw[ebase + pos] = wt[u][kk];
+        }
     }
 }
 
 cudaError_t launch_bucket_plan(const Shape &sh, const int32_t *idx, const float *w, const AttendPlan &P,
-                               int32_t *cnt, int32_t *cursor, int32_t *entries, float *entw, DevStatus *ds,
-                               cudaStream_t st) {
+                               int32_t *hist, int32_t *entries, float *entw, DevStatus *ds, cudaStream_t st) {
     if (P.J == 0) return cudaSuccess;
     cudaError_t e;
     const size_t hsmem = sizeof(int) * (size_t)sh.nc;
     if ((e = set_smem_once((const void *)bucket_count_kernel, hsmem)) != cudaSuccess) return e;
-    if ((e = set_smem_once((const void *)bucket_scan_kernel, 2 * hsmem)) != cudaSuccess) return e;
-    const int blocks_per_win = (P.W + kCountRows - 1) / kCountRows;
+    if ((e = set_smem_once((const void *)bucket_scan_kernel, 3 * hsmem)) != cudaSuccess) return e;
+    if ((e = set_smem_once((const void *)bucket_scatter_kernel, hsmem)) != cudaSuccess) return e;
+    const int blocks = P.J * ((P.W + kCountRows - 1) / kCountRows);
     if (sh.nc > 0) {
-        bucket_count_kernel<<<P.J * blocks_per_win, 256, hsmem, st>>>(idx, P, cnt, ds);
+        bucket_count_kernel<<<blocks, 256, hsmem, st>>>(idx, P, hist, ds);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
-    bucket_scan_kernel<<<P.J, 1024, 2 * hsmem, st>>>(P, cnt, cursor);
+    bucket_scan_kernel<<<P.J, 1024, 3 * hsmem, st>>>(P, hist);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    const int64_t rows = (int64_t)sh.B * sh.L * sh.hkv;
     if (sh.nc > 0) {
-        bucket_scatter_kernel<<<(unsigned)ceil_div(rows, 256), 256, 0, st>>>(idx, w, P, cursor, entries, entw);
+        bucket_scatter_kernel<<<blocks, 256, hsmem, st>>>(idx, w, P, hist, entries, entw);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
     return cudaSuccess;
+}
+
+size_t bucket_hist_elems(const AttendPlan &P) {
+    return (size_t)P.J * ((P.W + kCountRows - 1) / kCountRows) * P.nc;
 }
 
 }  // namespace hsa

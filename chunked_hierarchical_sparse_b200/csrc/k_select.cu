@@ -44,31 +44,33 @@ __global__ void __launch_bounds__(128) pool_kernel(const T *__restrict__ k, floa
     double acc[VEC];
 #pragma unroll
     for (int e = 0; e < VEC; ++e) acc[e] = 0.0;
+    const T *vsrc = x.vmax_bits ? static_cast<const T *>(x.v) + off : nullptr;  // bf16 values of the same chunk
+    float m = 0.f;
     for (int r0 = 0; r0 < rows; r0 += NB) {
-        uint4 raw[NB];
+        // the round's key rows and value rows are all in flight together
+        uint4 raw[NB], rv[NB];
 #pragma unroll
         for (int u = 0; u < NB; ++u) raw[u] = __ldcs(reinterpret_cast<const uint4 *>(src + (int64_t)(r0 + u) * d));
+        if (vsrc) {
+#pragma unroll
+            for (int u = 0; u < NB; ++u) rv[u] = __ldcs(reinterpret_cast<const uint4 *>(vsrc + (int64_t)(r0 + u) * d));
+        }
 #pragma unroll
         for (int u = 0; u < NB; ++u) {
             const T *vals = reinterpret_cast<const T *>(&raw[u]);
 #pragma unroll
             for (int e = 0; e < VEC; ++e) acc[e] += (double)Elem<T>::load(vals + e);
         }
-    }
-    if (x.vmax_bits) {  // bf16 values of the same chunk
-        const T *vsrc = static_cast<const T *>(x.v) + off;
-        float m = 0.f;
-        for (int r0 = 0; r0 < rows; r0 += NB) {
-            uint4 raw[NB];
-#pragma unroll
-            for (int u = 0; u < NB; ++u) raw[u] = __ldcs(reinterpret_cast<const uint4 *>(vsrc + (int64_t)(r0 + u) * d));
+        if (vsrc) {
 #pragma unroll
             for (int u = 0; u < NB; ++u) {
-                const T *vals = reinterpret_cast<const T *>(&raw[u]);
+                const T *vals = reinterpret_cast<const T *>(&rv[u]);
 #pragma unroll
                 for (int e = 0; e < VEC; ++e) m = fmaxf(m, fabsf(Elem<T>::load(vals + e)));
             }
         }
+    }
+    if (vsrc) {
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         if (lane == 0) atomicMax(x.vmax_bits, __float_as_int(m));

@@ -10,24 +10,25 @@
 // terms, kbar = hi + lo with hi = bf16(kbar), lo = bf16(kbar - hi), so
 //   q . kbar  ~=  q . hi + q . lo      (two tcgen05 MMAs into one fp32 TMEM tile)
 // with a residual of ~2^-16 of |kbar| per element -- far below the score gaps
-// that decide the top-K.  Chunk tiles of 64 pooled keys are streamed by TMA;
-// two tiles form a block of 128 scores per token, held in one of two TMEM
-// buffers.
+// that decide the top-K.  Chunk tiles of 64 pooled keys are streamed by TMA
+// into two stages and scored into two TMEM buffers.
 //
-// Top-K (one token row per epilogue thread, one sorted list per row), block by
-// block, two passes over the block's scores in TMEM:
-//   pass 1  the maximum of each of KS column stripes (chunk index mod KS).  K of
-//           the stripes hold a score at least as large as the K-th largest stripe
-//           maximum tau, so the block's -- and the row's -- K-th best is >= tau;
-//   pass 2  every score >= max(tau, theta) (theta: the list's current K-th best,
-//           also a lower bound) is appended, branch-free, to the row's small
-//           candidate buffer in shared memory.
-// After pass 2 the buffered candidates are inserted into the list.  They come in
-// increasing chunk order, after every chunk already listed, so a candidate beats
-// an equal listed score (ties go to the higher index) and the insertion compares
-// scores only.  A buffer that would overflow is inserted early and the threshold
-// raised.  At the end the K chunks are listed most-recent-first and the
+// Top-K, one token row per epilogue thread, in two passes over the row: the
+// tiles are scored twice (the tensor cores have time to spare; the CUDA-core
+// work per score is what bounds this kernel).
+//   pass 1  the maximum of each of 16 column stripes (chunk index mod 16) over
+//           the whole row.  K of the stripes hold a score at least as large as
+//           the K-th largest stripe maximum tau, so the row's K-th best is >= tau;
+//           for these inputs only ~2% of the scores reach tau;
+//   pass 2  the scores >= tau are appended to the row's candidate buffer in
+//           shared memory; they arrive in increasing chunk order.
+// The buffer is then inserted into a sorted list.  A candidate always has a
+// higher index than everything listed, so it beats an equal listed score
+// (ties go to the higher index) and the insertion compares scores only.  A
+// buffer that fills is inserted early and the threshold raised to the list's
+// K-th best.  At the end the K chunks are listed most-recent-first and the
 // stick-breaking weights are formed.
+#include <float.h>
 #include <math_constants.h>
 
 #include <algorithm>
@@ -43,7 +44,7 @@ namespace {
 
 constexpr int kSelThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue (one TMEM lane quadrant each)
 constexpr int kSelN = 64;         // chunks per tile
-constexpr int kBlkTiles = 2;      // tiles per block (one TMEM buffer: 128 columns)
+constexpr int kStripes = 16;      // column stripes of pass 1 (>= K)
 constexpr int kCap = 12;          // candidate buffer entries per row
 constexpr uint64_t kSelWaitNs = 2000000000ull;
 
@@ -112,6 +113,19 @@ template <int KS> __device__ __forceinline__ void sort_asc(float (&a)[KS]) {
             }
 }
 
+// v[e] for a lane-varying e in [0, 32), by a select tree on e's bits (stays in registers)
+__device__ __forceinline__ float pick32(const float *v, int e) {
+    float t16[16], t8[8], t4[4];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) t16[i] = (e & 1) ? v[2 * i + 1] : v[2 * i];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) t8[i] = (e & 2) ? t16[2 * i + 1] : t16[2 * i];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) t4[i] = (e & 4) ? t8[2 * i + 1] : t8[2 * i];
+    const float ta = (e & 8) ? t4[1] : t4[0], tb = (e & 8) ? t4[3] : t4[2];
+    return (e & 16) ? tb : ta;
+}
+
 }  // namespace
 
 template <int D, int KM>
@@ -120,14 +134,13 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_tc_kernel(
     const __grid_constant__ CUtensorMap tm_lo, int32_t *__restrict__ idx, float *__restrict__ wout,
     int L, int hkv, int nc, int K, DevStatus *ds) {
     using SL = SelSmem<D>;
-    constexpr int KS = KM;  // column stripes of pass 1 (K <= KM of them hold the threshold)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + SL::OFF_BAR);
     uint64_t *q_full = bar;
     uint64_t *b_full = bar + 1;     // [2]  tile stage loaded (TMA -> MMA)
     uint64_t *b_empty = bar + 3;    // [2]  tile stage read (MMA -> TMA)
-    uint64_t *a_full = bar + 5;     // [2]  TMEM buffer holds a scored block (MMA -> epilogue)
+    uint64_t *a_full = bar + 5;     // [2]  TMEM buffer holds a scored tile (MMA -> epilogue)
     uint64_t *a_empty = bar + 7;    // [2]  TMEM buffer read (epilogue -> MMA)
     uint64_t *mma_done = bar + 9;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + SL::OFF_BAR + 16 * 8);
@@ -140,7 +153,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_tc_kernel(
     const int tlast = min(t0 + 128, L) - 1;
     const int ne_max = min(tlast / kChunk, nc);
     const int ntiles = (ne_max + kSelN - 1) / kSelN;
-    const int nblk = (ntiles + kBlkTiles - 1) / kBlkTiles;
+    const int nsteps = 2 * ntiles;  // every tile scored twice: pass 1, then pass 2
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
@@ -151,7 +164,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_tc_kernel(
         mbar_init(mma_done, 1);
         mbar_fence_init();
     }
-    if (warp == 1) { tmem_alloc(tmem_slot, 2 * kBlkTiles * kSelN); tmem_relinquish(); }
+    if (warp == 1) { tmem_alloc(tmem_slot, 2 * kSelN); tmem_relinquish(); }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -172,12 +185,12 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_tc_kernel(
                 tma_load_3d(sm + SL::OFF_Q + h * 128 * 128, &tm_qs, h * 64, g, b * L + t0, q_full);
         }
         int issued = 0;
-        for (int i = 0; i < ntiles && ok; ++i) {
+        for (int i = 0; i < nsteps && ok; ++i) {
             const int s = i & 1;
             if (i >= 2 && !warp_wait(&b_empty[s], ((i >> 1) - 1) & 1)) { ok = false; break; }
             if (lane == 0) {
                 mbar_arrive_expect_tx(&b_full[s], SL::BBYTES);
-                const int row = bg * nc + i * kSelN;
+                const int row = bg * nc + (i % ntiles) * kSelN;
                 uint8_t *dst = sm + SL::OFF_B + s * SL::BBYTES;
 #pragma unroll
                 for (int h = 0; h < SL::NH; ++h) {
@@ -198,17 +211,15 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_tc_kernel(
         constexpr uint32_t idesc = idesc_bf16_f32(128, kSelN, false, false);
         bool ok = true;
         if (ntiles > 0 && !warp_wait(q_full, 0)) ok = false;
-        for (int i = 0; i < ntiles && ok; ++i) {
+        for (int i = 0; i < nsteps && ok; ++i) {
             const int s = i & 1;
-            const int blk = i / kBlkTiles, buf = blk & 1, ti = i % kBlkTiles;
             if (!warp_wait(&b_full[s], (i >> 1) & 1)) { ok = false; break; }
-            // the block's TMEM buffer is free once the epilogue has read block blk - 2
-            if (ti == 0 && blk >= 2 && !warp_wait(&a_empty[buf], ((blk >> 1) - 1) & 1)) { ok = false; break; }
+            if (i >= 2 && !warp_wait(&a_empty[s], ((i >> 1) - 1) & 1)) { ok = false; break; }
             tc_fence_after();
             if (lane == 0) {
                 const uint32_t qa = smem_u32(sm + SL::OFF_Q);
                 const uint32_t bb = smem_u32(sm + SL::OFF_B + s * SL::BBYTES);
-                const uint32_t dcol = tmem + buf * (kBlkTiles * kSelN) + ti * kSelN;
+                const uint32_t dcol = tmem + s * kSelN;
 #pragma unroll
                 for (int part = 0; part < 2; ++part)  // hi then lo
 #pragma unroll
@@ -218,8 +229,8 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_tc_kernel(
                                     smem_desc_sw128(bb + (part * SL::NH + h) * SL::BHALF + kk * 32, 16, 1024), idesc,
                                     (part | ks) != 0);
                     }
+                mma_commit(&a_full[s]);
                 mma_commit(&b_empty[s]);
-                if (ti == kBlkTiles - 1 || i == ntiles - 1) mma_commit(&a_full[buf]);
             }
             __syncwarp();
         }
@@ -232,7 +243,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_tc_kernel(
         const int r = wq * 32 + lane;
         const int t = t0 + r;
         const int ne = (t < L) ? min(t / kChunk, nc) : 0;
-        const int ne_warp = __reduce_min_sync(0xffffffffu, (unsigned)ne);  // every lane: chunks < ne_warp eligible
+        const int ne_warp = __reduce_min_sync(0xffffffffu, (unsigned)ne);  // chunks < ne_warp: eligible in every lane
         float *cs = reinterpret_cast<float *>(sm + SL::OFF_CS) + r;  // candidate i at cs[i * 128]
         int *cc = reinterpret_cast<int *>(sm + SL::OFF_CC) + r;
         TopList<KM> tl;
@@ -245,99 +256,73 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_tc_kernel(
             }
             n = 0;
         };
+        float st[kStripes];
+#pragma unroll
+        for (int j = 0; j < kStripes; ++j) st[j] = -CUDART_INF_F;
+        float thr = CUDART_INF_F;
         bool ok = true;
-        for (int blk = 0; blk < nblk; ++blk) {
-            const int buf = blk & 1;
-            const int c0 = blk * kBlkTiles * kSelN;
-            const int ntb = min(kBlkTiles, ntiles - blk * kBlkTiles);
-            const uint32_t base = tmem + ((uint32_t)(wq * 32) << 16) + buf * (kBlkTiles * kSelN);
-            if (!warp_wait(&a_full[buf], (blk >> 1) & 1)) { ok = false; break; }
+        for (int i = 0; i < nsteps; ++i) {
+            const int s = i & 1;
+            const int cb = (i % ntiles) * kSelN;
+            const bool full = cb + kSelN <= ne_warp;  // every chunk of the tile eligible in every lane
+            if (!warp_wait(&a_full[s], (i >> 1) & 1)) { ok = false; break; }
             tc_fence_after();
-            // every chunk of the block is eligible for every row of the warp, or masking is needed
-            const bool full = c0 + kBlkTiles * kSelN <= ne_warp;
-            // ---- pass 1: stripe maxima -> tau
-            float st[KS];
+            float v[64];
+            tmem_ld32(tmem + ((uint32_t)(wq * 32) << 16) + s * kSelN, *reinterpret_cast<float(*)[32]>(&v[0]));
+            tmem_ld32(tmem + ((uint32_t)(wq * 32) << 16) + s * kSelN + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            mbar_arrive_lane0(&a_empty[s], lane);  // the buffer is free for step i + 2
+            if (!full) {
 #pragma unroll
-            for (int j = 0; j < KS; ++j) st[j] = -CUDART_INF_F;
-            for (int ti = 0; ti < ntb; ++ti) {
-                float v0[32], v1[32];
-                tmem_ld32(base + ti * kSelN, v0);
-                tmem_ld32(base + ti * kSelN + 32, v1);
-                tmem_wait_ld();
-                const int cb = c0 + ti * kSelN;
-                if (full) {
+                for (int e = 0; e < 64; ++e) v[e] = cb + e < ne ? v[e] : -CUDART_INF_F;
+            }
+            if (i < ntiles) {
+                // ---- pass 1: stripe maxima
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        st[e % KS] = fmaxf(st[e % KS], v0[e]);
-                        st[(e + 32) % KS] = fmaxf(st[(e + 32) % KS], v1[e]);
-                    }
-                } else {
+                for (int e = 0; e < 64; ++e) st[e % kStripes] = fmaxf(st[e % kStripes], v[e]);
+                if (i == ntiles - 1) {  // tau: the K-th largest stripe maximum = the least of the top K
+                    sort_asc<kStripes>(st);
+                    thr = CUDART_INF_F;
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        st[e % KS] = fmaxf(st[e % KS], cb + e < ne ? v0[e] : -CUDART_INF_F);
-                        st[(e + 32) % KS] = fmaxf(st[(e + 32) % KS], cb + 32 + e < ne ? v1[e] : -CUDART_INF_F);
-                    }
+                    for (int j = 0; j < kStripes; ++j) thr = fminf(thr, j >= kStripes - K ? st[j] : CUDART_INF_F);
+                    // fewer than K eligible chunks leave tau = -inf: every finite (eligible)
+                    // score is a candidate, the masked -inf ones are not
+                    thr = fmaxf(thr, -FLT_MAX);
                 }
-            }
-            float tau;
-            if (K == KS) {  // the smallest stripe maximum
-                tau = st[0];
-#pragma unroll
-                for (int j = 1; j < KS; ++j) tau = fminf(tau, st[j]);
-            } else {        // the K-th largest stripe maximum
-                sort_asc<KS>(st);
-                tau = st[0];
-#pragma unroll
-                for (int j = 1; j < KS; ++j) tau = (j == KS - K) ? st[j] : tau;
-            }
-            float thr = fmaxf(tau, tl.theta());
-            // ---- pass 2: buffer every eligible score >= thr
-            for (int ti = 0; ti < ntb; ++ti) {
-                float v[64];
-                tmem_ld32(base + ti * kSelN, *reinterpret_cast<float(*)[32]>(&v[0]));
-                tmem_ld32(base + ti * kSelN + 32, *reinterpret_cast<float(*)[32]>(&v[32]));
-                tmem_wait_ld();
-                const int cb = c0 + ti * kSelN;
-                const int nel = full ? 64 : max(0, min(64, ne - cb));
+            } else {
+                // ---- pass 2: buffer every score >= thr (ineligible ones are -inf)
 #pragma unroll
                 for (int hf = 0; hf < 2; ++hf) {
                     uint32_t m = 0;
 #pragma unroll
                     for (int e = 0; e < 32; ++e) m |= (v[hf * 32 + e] >= thr) ? (1u << e) : 0u;
-                    const int el = nel - hf * 32;
-                    m &= el >= 32 ? 0xffffffffu : (el <= 0 ? 0u : ((1u << el) - 1u));
-                    if (n + __popc(m) > kCap) {  // rare: make room, raise the threshold
+                    if (n + __popc(m) > kCap) {  // rare: insert the buffer, raise the threshold
                         flush();
                         thr = fmaxf(thr, tl.theta());
 #pragma unroll
                         for (int e = 0; e < 32; ++e) m &= (v[hf * 32 + e] >= thr) ? 0xffffffffu : ~(1u << e);
-                        if (__popc(m) > kCap) {  // still too many: insert them directly
-#pragma unroll
-                            for (int e = 0; e < 32; ++e)
-                                if ((m >> e) & 1u) {
-                                    if (v[hf * 32 + e] >= tl.theta()) tl.insert_newest(v[hf * 32 + e], cb + hf * 32 + e);
-                                }
-                            m = 0;
-                            thr = fmaxf(thr, tl.theta());
+                        while (__popc(m) > kCap) {  // still too many: insert directly, lowest chunks first
+                            const int e = __ffs(m) - 1;
+                            m &= m - 1;
+                            const float x = pick32(v + hf * 32, e);
+                            if (x >= tl.theta()) tl.insert_newest(x, cb + hf * 32 + e);
                         }
                     }
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) {
-                        if ((m >> e) & 1u) {
-                            cs[n * 128] = v[hf * 32 + e];
-                            cc[n * 128] = cb + hf * 32 + e;
-                            ++n;
-                        }
+                    while (m) {
+                        const int e = __ffs(m) - 1;
+                        m &= m - 1;
+                        cs[n * 128] = pick32(v + hf * 32, e);
+                        cc[n * 128] = cb + hf * 32 + e;
+                        ++n;
                     }
                 }
             }
-            tc_fence_before();
-            __syncwarp();
-            mbar_arrive_lane0(&a_empty[buf], lane);  // the buffer is free for block blk + 2
-            flush();
         }
         if (!ok && lane == 0) report(ds, HSA_ERR_TIMEOUT, kKSelectTc, 3, t0);
         if (ok && t < L) {
+            flush();
             // most-recent-first: order the chosen chunks by descending index (empty = -1 last)
 #pragma unroll
             for (int k = 0; k < KM; ++k)
@@ -374,7 +359,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_tc_kernel(
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, 2 * kBlkTiles * kSelN);
+    if (warp == 1) tmem_dealloc(tmem, 2 * kSelN);
 }
 
 namespace {

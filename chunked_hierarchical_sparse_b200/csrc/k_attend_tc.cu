@@ -224,13 +224,18 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         int guard_ok_j = -1;  // highest window whose ring guard already passed
         struct Desc { int4 a, b; };
         // queue position q of window jw is unit q - seg_start[jw] of jw's slice of the
-        // queue; the positions looked up only grow, so the window only moves forward
-        int jw = 0;
+        // queue; the positions looked up only grow, so the window only moves forward and
+        // its bounds stay in registers (a load only when a window boundary is crossed)
+        int jw = 0, seg_lo = 0, seg_hi = P.J > 1 ? P.seg_start[1] : total;
         auto load_desc = [&](int q) -> Desc {  // every lane loads the same 32 bytes
             Desc d;
             if (q < total) {
-                while (jw + 1 < P.J && q >= P.seg_start[jw + 1]) ++jw;
-                const int64_t u = (int64_t)jw * P.win_cap + (q - P.seg_start[jw]);
+                while (q >= seg_hi && jw + 1 < P.J) {
+                    ++jw;
+                    seg_lo = seg_hi;
+                    seg_hi = jw + 1 < P.J ? P.seg_start[jw + 1] : total;
+                }
+                const int64_t u = (int64_t)jw * P.win_cap + (q - seg_lo);
                 d.a = P.items[2 * u];
                 d.b = P.items[2 * u + 1];
             } else {

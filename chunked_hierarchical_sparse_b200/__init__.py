@@ -19,7 +19,7 @@ import os
 
 import torch
 
-__all__ = ["hsa_timing_enable", "hsa_timing_read", "KERNELS", "hsa_workspace_size", "hsa_pool", "hsa_select", "hsa_fwd", "hsa_attend", "hsa_decode", "hsa_decode_multi", "hsa_bwd",
+__all__ = ["hsa_set_wait_limit_ns", "hsa_timing_enable", "hsa_timing_read", "KERNELS", "hsa_workspace_size", "hsa_pool", "hsa_select", "hsa_fwd", "hsa_attend", "hsa_decode", "hsa_decode_multi", "hsa_bwd",
            "hsa_device_status", "HsaError", "lib_path", "load_library", "OP_POOL", "OP_SELECT",
            "OP_FWD", "OP_DECODE", "OP_BWD"]
 
@@ -76,6 +76,8 @@ def load_library():
         L.hsa_timing_read.restype = ctypes.c_int
         L.hsa_status_string.argtypes = [ctypes.c_int32]
         L.hsa_status_string.restype = ctypes.c_char_p
+        L.hsa_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+        L.hsa_set_wait_limit_ns.restype = ctypes.c_int
         for f in ("hsa_pool", "hsa_select", "hsa_fwd", "hsa_attend", "hsa_decode", "hsa_decode_multi", "hsa_bwd", "hsa_device_status"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
@@ -305,6 +307,12 @@ def hsa_device_status(ws: torch.Tensor, stream=None) -> int:
     code = ctypes.c_int32(0)
     _run("hsa_device_status", ws.device, stream, _p(ws), ctypes.byref(code))
     return int(code.value)
+
+
+def hsa_set_wait_limit_ns(ns: int) -> None:
+    """Bound every wait inside the persistent kernels at `ns` nanoseconds (0: the
+    default of 2 s) -- a testing aid that makes a wait run out on purpose."""
+    _check(load_library().hsa_set_wait_limit_ns(int(ns)), "hsa_set_wait_limit_ns")
 
 
 def hsa_timing_enable(on: bool = True) -> None:

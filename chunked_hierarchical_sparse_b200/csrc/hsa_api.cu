@@ -1,12 +1,21 @@
 // hsa_api.cu -- the extern "C" entry points declared in include/hsa.h:
 // argument checks, workspace carving, and the kernel sequence of each call.
 #include <algorithm>
+#include <atomic>
 #include <climits>
 #include <cstring>
 
 #include "hsa_internal.cuh"
 
 namespace hsa {
+
+// ------------------------------------------------------------------ wait limit
+static std::atomic<uint64_t> g_wait_ns{0};  // 0: the default
+
+uint64_t wait_limit_ns() {
+    const uint64_t v = g_wait_ns.load(std::memory_order_relaxed);
+    return v ? v : kDefaultWaitNs;
+}
 
 // ------------------------------------------------------------------ checks
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
@@ -478,6 +487,11 @@ hsa_status_t hsa_bwd(const hsa_shape_t *shape, const void *q, const void *k, con
     if (e == cudaSuccess)
         e = timed(HSA_K_BWD2, sh.nc > 0 ? 2 : 1, st, [&] { return launch_bwd_phase2(sh, q, k, v, dO, lse, w, dk, dv, b, ds, st); });
     return cuda_status(e);
+}
+
+hsa_status_t hsa_set_wait_limit_ns(uint64_t ns) {
+    g_wait_ns.store(ns, std::memory_order_relaxed);
+    return HSA_OK;
 }
 
 hsa_status_t hsa_device_status(const void *ws, int32_t *code_out, void *stream) {

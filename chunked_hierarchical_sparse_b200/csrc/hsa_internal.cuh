@@ -71,6 +71,14 @@ inline Shape make_shape(const hsa_shape_t &s) {
 // for inconsistent values, UNSUPPORTED for valid shapes that are not built.
 hsa_status_t check_shape(const hsa_shape_t *s, bool decode);
 
+// Bound on one wait inside the persistent kernels (attention, selection, backward), in
+// nanoseconds of wall-clock time: 2 s unless hsa_set_wait_limit_ns changed it (a
+// testing aid for the failure path).  Passed to the kernels as an argument; the waits
+// that let a CTA's own copies and MMAs finish before it exits keep kDrainWaitNs.
+uint64_t wait_limit_ns();
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;
+constexpr uint64_t kDrainWaitNs = 2000000000ull;
+
 // ---------------------------------------------------------------- launch helpers
 // Raise a kernel's dynamic shared-memory limit to `bytes` once (cached per
 // kernel, so repeated calls -- and calls during stream capture -- make no

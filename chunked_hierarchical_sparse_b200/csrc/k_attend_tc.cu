@@ -52,10 +52,6 @@ constexpr int kInfo = 8;                 // tile-info ring entries
 constexpr int kQStages = 3;              // query-tile buffers (P lives in TMEM, not SMEM)
 // TMEM columns: S[2] 0..127 (fp32), O[2] 128..383 (fp32), P[2] 384..447 (bf16 pairs)
 constexpr uint32_t kColO = 128, kColP = 384;
-#ifndef HSA_WAIT_NS
-#define HSA_WAIT_NS 2000000000ull
-#endif
-constexpr uint64_t kWaitNs = HSA_WAIT_NS;  // bound on any single wait (default 2 s)
 
 enum ItemType : int { kItemTile = 0, kItemEnd = 2 };
 
@@ -118,14 +114,14 @@ __device__ __forceinline__ float ex2_approx(float x) {
 }
 
 // bounded spin until *p >= target; false on timeout or once *abort is set
-__device__ bool spin_geq_live(const int32_t *p, int target, volatile int *abort) {
+__device__ bool spin_geq_live(const int32_t *p, int target, volatile int *abort, uint64_t wait_ns) {
     if (ld_acquire(p) >= target) return true;
     const uint64_t t0 = globaltimer();
     while (true) {
         __nanosleep(256);
         if (ld_acquire(p) >= target) return true;
         if (*abort) return false;
-        if (globaltimer() - t0 > kWaitNs) return false;
+        if (globaltimer() - t0 > wait_ns) return false;
     }
 }
 
@@ -138,7 +134,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
     const __grid_constant__ CUtensorMap tm_v,
     const __grid_constant__ AttendPlan P, const int32_t *__restrict__ entries,
     const float *__restrict__ entw, __half *__restrict__ acc,
-    __nv_bfloat16 *__restrict__ out, float *__restrict__ lse, DevStatus *ds) {
+    __nv_bfloat16 *__restrict__ out, float *__restrict__ lse, DevStatus *ds, uint64_t wait_ns) {
     using L = Smem<D>;
     constexpr int TT = 128 / G;
     extern __shared__ uint8_t smem_raw[];
@@ -208,7 +204,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
 
     // every lane waits (converged, sleeping in try_wait); the warp's verdict is a vote
     auto warp_wait = [&](uint64_t *b, uint32_t par) -> bool {
-        return __all_sync(0xffffffffu, mbar_wait(b, par, kWaitNs));
+        return __all_sync(0xffffffffu, mbar_wait(b, par, wait_ns));
     };
 
     if (warp == kWarpProd) {
@@ -291,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             // ring guard: window j's partial slot was last used by window j - kRing
             if (j >= kRing && j > guard_ok_j) {
                 int g_ok = 1;
-                if (lane == 0) g_ok = spin_geq_live(&comb_done[j - kRing], P.win_ncomb[j - kRing], abort_flag) ? 1 : 0;
+                if (lane == 0) g_ok = spin_geq_live(&comb_done[j - kRing], P.win_ncomb[j - kRing], abort_flag, wait_ns) ? 1 : 0;
                 if (!__shfl_sync(0xffffffffu, g_ok, 0)) {
                     if (lane == 0 && !*abort_flag) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 1, j);
                     ok = false;
@@ -372,8 +368,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 2, it);
                 // let the loads already issued land before the CTA goes away (bounded)
                 for (int s2 = 0; s2 < kQStages; ++s2) {
-                    if (qc > s2) mbar_wait(&B.q_full[(qc - 1 - s2) % kQStages], ((qc - 1 - s2) / kQStages) & 1, kWaitNs);
-                    if (s2 < 2 && kvc > s2) mbar_wait(&B.kv_full[(kvc - 1 - s2) & 1], ((kvc - 1 - s2) >> 1) & 1, kWaitNs);
+                    if (qc > s2) mbar_wait(&B.q_full[(qc - 1 - s2) % kQStages], ((qc - 1 - s2) / kQStages) & 1, kDrainWaitNs);
+                    if (s2 < 2 && kvc > s2) mbar_wait(&B.kv_full[(kvc - 1 - s2) & 1], ((kvc - 1 - s2) >> 1) & 1, kDrainWaitNs);
                 }
             }
             __syncwarp();
@@ -449,7 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
                 if (prog) {
                     t_last = globaltimer();
                 } else {
-                    if (*abort_flag || globaltimer() - t_last > kWaitNs) { ok = false; break; }
+                    if (*abort_flag || globaltimer() - t_last > wait_ns) { ok = false; break; }
                     __nanosleep(32);  // leave the issue slots to the working warps meanwhile
                 }
             }
@@ -459,7 +455,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             }
             // drain: every MMA issued by this warp has finished before TMEM is released
             mma_commit(mma_done);
-            mbar_wait(mma_done, 0, kWaitNs);
+            mbar_wait(mma_done, 0, kDrainWaitNs);
         }
         __syncwarp();
     } else if (warp < kWarpEpi) {
@@ -674,7 +670,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         for (int jc = 0; jc < P.J && ok; ++jc) {
             int gok = 1;
             // every tile is counted by the four warps of its epilogue group
-            if (tid == 0) gok = spin_geq_live(&tiles_done[jc], 4 * P.win_tiles[jc], abort_flag) ? 1 : 0;
+            if (tid == 0) gok = spin_geq_live(&tiles_done[jc], 4 * P.win_tiles[jc], abort_flag, wait_ns) ? 1 : 0;
             if (!cg_bcast(gok)) { if (tid == 0 && !*abort_flag) report(ds, HSA_ERR_TIMEOUT, kKAttendTc, 4, jc); ok = false; break; }
             const int ncomb = P.win_ncomb[jc];
             while (true) {
@@ -799,7 +795,7 @@ cudaError_t launch_tc(const Shape &sh, const AttendPlan &plan, const int32_t *en
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     attend_tc_kernel<D, G><<<sms, kThreads, smem, st>>>(mq, mk, mv, plan, entries, entw, acc,
-                                                        (__nv_bfloat16 *)o, lse, ds);
+                                                        (__nv_bfloat16 *)o, lse, ds, wait_limit_ns());
     return cudaGetLastError();
 }
 

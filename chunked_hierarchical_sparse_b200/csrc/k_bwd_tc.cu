@@ -36,10 +36,6 @@ using namespace sm100;
 
 namespace {
 
-#ifndef HSA_WAIT_NS
-#define HSA_WAIT_NS 2000000000ull
-#endif
-constexpr uint64_t kBWaitNs = HSA_WAIT_NS;  // bound on any single wait (default 2 s)
 
 #ifndef HSA_BEPI_UNROLL
 #define HSA_BEPI_UNROLL 1
@@ -107,14 +103,14 @@ __device__ __forceinline__ int bld_acquire(const int32_t *p) {
 }
 
 // bounded spin until *p >= target; false on timeout or once *abort is set
-__device__ bool bspin_geq(const int32_t *p, int target, volatile int *abort) {
+__device__ bool bspin_geq(const int32_t *p, int target, volatile int *abort, uint64_t wait_ns) {
     if (bld_acquire(p) >= target) return true;
     const uint64_t t0 = globaltimer();
     while (true) {
         __nanosleep(256);
         if (bld_acquire(p) >= target) return true;
         if (*abort) return false;
-        if (globaltimer() - t0 > kBWaitNs) return false;
+        if (globaltimer() - t0 > wait_ns) return false;
     }
 }
 
@@ -138,7 +134,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
     const __grid_constant__ AttendPlan P, const int32_t *__restrict__ entries, const float *__restrict__ entw,
     const float *__restrict__ lse, float *__restrict__ dw, __half *__restrict__ acc, __nv_bfloat16 *__restrict__ dq,
-    float *__restrict__ dk_acc, float *__restrict__ dv_acc, DevStatus *ds) {
+    float *__restrict__ dk_acc, float *__restrict__ dv_acc, DevStatus *ds, uint64_t wait_ns) {
     using L = BSmem;
     constexpr int D = kBD;
     constexpr int TT = 128 / G;
@@ -216,7 +212,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
     }
 
     auto warp_wait = [&](uint64_t *b, uint32_t par) -> bool {  // every lane waits; the verdict is a vote
-        return __all_sync(0xffffffffu, mbar_wait(b, par, kBWaitNs));
+        return __all_sync(0xffffffffu, mbar_wait(b, par, wait_ns));
     };
 
     if (warp == kBWarpProd) {
@@ -267,7 +263,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
             // ring guard: window j's dq slot was last used by window j - kRing
             if (j >= kRing && j > guard_ok_j) {
                 int g_ok = 1;
-                if (lane == 0) g_ok = bspin_geq(&comb_done[j - kRing], P.win_ncomb[j - kRing], abort_flag) ? 1 : 0;
+                if (lane == 0) g_ok = bspin_geq(&comb_done[j - kRing], P.win_ncomb[j - kRing], abort_flag, wait_ns) ? 1 : 0;
                 if (!__shfl_sync(0xffffffffu, g_ok, 0)) {
                     if (lane == 0 && !*abort_flag) report(ds, HSA_ERR_TIMEOUT, kKBwdTc, 1, j);
                     ok = false;
@@ -340,8 +336,8 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
                 report(ds, HSA_ERR_TIMEOUT, kKBwdTc, 2, it);
                 // let the loads already issued land before the CTA goes away (bounded)
                 for (int s2 = 0; s2 < 2; ++s2)
-                    if (qc > s2) mbar_wait(&qd_full[(qc - 1 - s2) & 1], ((qc - 1 - s2) >> 1) & 1, kBWaitNs);
-                if (useq > 0) mbar_wait(kv_full, (useq - 1) & 1, kBWaitNs);
+                    if (qc > s2) mbar_wait(&qd_full[(qc - 1 - s2) & 1], ((qc - 1 - s2) >> 1) & 1, kDrainWaitNs);
+                if (useq > 0) mbar_wait(kv_full, (useq - 1) & 1, kDrainWaitNs);
             }
             __syncwarp();
         }
@@ -438,7 +434,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
                 if (prog) {
                     t_last = globaltimer();
                 } else {
-                    if (*abort_flag || globaltimer() - t_last > kBWaitNs) { ok = false; break; }
+                    if (*abort_flag || globaltimer() - t_last > wait_ns) { ok = false; break; }
                     __nanosleep(32);  // leave the issue slots to the working warps meanwhile
                 }
             }
@@ -448,7 +444,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
             }
             // drain: every MMA issued by this warp has finished before TMEM is released
             mma_commit(mma_done);
-            mbar_wait(mma_done, 0, kBWaitNs);
+            mbar_wait(mma_done, 0, kDrainWaitNs);
         }
         __syncwarp();
     } else if (warp < kBWarpEpi) {
@@ -464,7 +460,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
         // every warp of the group waits for itself (converged, sleeping in try_wait);
         // the warps only meet at the mbarriers they arrive on
         auto wg_wait = [&](uint64_t *b, uint32_t par) -> bool {
-            return __all_sync(0xffffffffu, mbar_wait(b, par, kBWaitNs));
+            return __all_sync(0xffffffffu, mbar_wait(b, par, wait_ns));
         };
         while (ok) {
             const int ii = it % kBInfo;
@@ -568,7 +564,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
         };
         auto eg_wait = [&](uint64_t *b, uint32_t par) -> bool {
             int v = 1;
-            if (tid == 0) v = mbar_wait(b, par, kBWaitNs) ? 1 : 0;
+            if (tid == 0) v = mbar_wait(b, par, wait_ns) ? 1 : 0;
             return eg_vote(v);
         };
         auto flush = [&]() {  // publish the reductions of the tiles counted so far
@@ -687,7 +683,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
         };
         for (int jc = 0; jc < P.J && ok; ++jc) {
             int gok = 1;
-            if (tid == 0) gok = bspin_geq(&tiles_done[jc], P.win_tiles[jc], abort_flag) ? 1 : 0;
+            if (tid == 0) gok = bspin_geq(&tiles_done[jc], P.win_tiles[jc], abort_flag, wait_ns) ? 1 : 0;
             if (!cg_bcast(gok)) {
                 if (tid == 0 && !*abort_flag) report(ds, HSA_ERR_TIMEOUT, kKBwdTc, 4, jc);
                 ok = false;
@@ -972,7 +968,7 @@ cudaError_t launch_btc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     bwd_tc_kernel<G><<<sms, kBThreads, smem, st>>>(mq, mo, mk, mv, plan, inv.entries, inv.entw, lse, dw, acc,
-                                                   (__nv_bfloat16 *)dq, dk_acc, dv_acc, ds);
+                                                   (__nv_bfloat16 *)dq, dk_acc, dv_acc, ds, wait_limit_ns());
     return cudaGetLastError();
 }
 }  // namespace

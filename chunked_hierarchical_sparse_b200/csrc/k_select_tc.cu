@@ -46,7 +46,6 @@ constexpr int kSelThreads = 192;  // warp 0 TMA, warp 1 MMA, warps 2-5 epilogue 
 constexpr int kSelN = 64;         // chunks per tile
 constexpr int kStripes = 16;      // column stripes of pass 1 (>= K)
 constexpr int kCap = 12;          // candidate buffer entries per row
-constexpr uint64_t kSelWaitNs = 2000000000ull;
 
 template <int D> struct SelSmem {
     static constexpr int NH = D / 64;
@@ -132,7 +131,7 @@ template <int D, int KM>
 __global__ void __launch_bounds__(kSelThreads, 2) select_tc_kernel(
     const __grid_constant__ CUtensorMap tm_qs, const __grid_constant__ CUtensorMap tm_hi,
     const __grid_constant__ CUtensorMap tm_lo, int32_t *__restrict__ idx, float *__restrict__ wout,
-    int L, int hkv, int nc, int K, DevStatus *ds) {
+    int L, int hkv, int nc, int K, DevStatus *ds, uint64_t wait_ns) {
     using SL = SelSmem<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -172,7 +171,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_tc_kernel(
 
     // every lane waits (converged, sleeping in try_wait); the warp's verdict is a vote
     auto warp_wait = [&](uint64_t *bb, uint32_t par) -> bool {
-        return __all_sync(0xffffffffu, mbar_wait(bb, par, kSelWaitNs));
+        return __all_sync(0xffffffffu, mbar_wait(bb, par, wait_ns));
     };
 
     if (warp == 0) {
@@ -204,7 +203,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_tc_kernel(
         if (!ok && lane == 0) {
             report(ds, HSA_ERR_TIMEOUT, kKSelectTc, 1, t0);
             // let the loads already issued land before the CTA can go away (bounded)
-            for (int i = max(0, issued - 2); i < issued; ++i) mbar_wait(&b_full[i & 1], (i >> 1) & 1, kSelWaitNs);
+            for (int i = max(0, issued - 2); i < issued; ++i) mbar_wait(&b_full[i & 1], (i >> 1) & 1, kDrainWaitNs);
         }
     } else if (warp == 1) {
         // -------------------------------------------------- MMA issuer
@@ -235,7 +234,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_tc_kernel(
             __syncwarp();
         }
         if (!ok && lane == 0) report(ds, HSA_ERR_TIMEOUT, kKSelectTc, 2, t0);
-        if (lane == 0) { mma_commit(mma_done); mbar_wait(mma_done, 0, kSelWaitNs); }
+        if (lane == 0) { mma_commit(mma_done); mbar_wait(mma_done, 0, kDrainWaitNs); }
         __syncwarp();
     } else {
         // -------------------------------------------------- epilogue: one token row per thread
@@ -406,10 +405,12 @@ cudaError_t launch_sel(const Shape &sh, const void *q_slc, const float *kbar, __
     cudaError_t e;
     if (sh.K <= 8) {
         if ((e = set_smem_once((const void *)select_tc_kernel<D, 8>, smem)) != cudaSuccess) return e;
-        select_tc_kernel<D, 8><<<grid, kSelThreads, smem, st>>>(mq, mh, ml, idx, w, sh.L, sh.hkv, sh.nc, sh.K, ds);
+        select_tc_kernel<D, 8><<<grid, kSelThreads, smem, st>>>(mq, mh, ml, idx, w, sh.L, sh.hkv, sh.nc, sh.K, ds,
+                                                                wait_limit_ns());
     } else {
         if ((e = set_smem_once((const void *)select_tc_kernel<D, 16>, smem)) != cudaSuccess) return e;
-        select_tc_kernel<D, 16><<<grid, kSelThreads, smem, st>>>(mq, mh, ml, idx, w, sh.L, sh.hkv, sh.nc, sh.K, ds);
+        select_tc_kernel<D, 16><<<grid, kSelThreads, smem, st>>>(mq, mh, ml, idx, w, sh.L, sh.hkv, sh.nc, sh.K, ds,
+                                                                 wait_limit_ns());
     }
     return cudaGetLastError();
 }

@@ -214,6 +214,18 @@ HSA_API hsa_status_t hsa_fwd_noalloc(const hsa_shape_t *shape, const void *q, co
  * into *code_out (an hsa_status_t value; HSA_OK when nothing went wrong). */
 HSA_API hsa_status_t hsa_device_status(const void *ws, int32_t *code_out, void *stream);
 
+/* Testing aid for the failure path.  Every wait inside the library's persistent
+ * kernels (the chunk-major attention, the tensor-core selection and the
+ * tensor-core backward) is bounded by `ns` nanoseconds of wall-clock time; 0
+ * restores the default bound of 2 s.  A wait that runs out makes the kernel
+ * record HSA_ERR_TIMEOUT in the status word, stop its work, let the copies and
+ * MMAs it has issued finish (these waits keep the 2 s bound), free its tensor
+ * memory and return: nothing traps and the device stays usable.  The outputs
+ * of that call are undefined; the next call starts clean.  The value is
+ * process-wide (all threads and devices) and read when a kernel is launched;
+ * it returns HSA_OK. */
+HSA_API hsa_status_t hsa_set_wait_limit_ns(uint64_t ns);
+
 /* Kernel timing, a profiling aid.  While enabled, each kernel (or fixed group
  * of kernels) this library launches is bracketed by a pair of CUDA events
  * recorded on the launching stream; hsa_timing_read waits for the recorded

@@ -124,8 +124,8 @@ def _ctype_kind(t):
         return None
     if t in (ctypes.c_void_p, ctypes.c_char_p) or hasattr(t, "_type_") and isinstance(t._type_, type):
         return "ptr"
-    if t is ctypes.c_size_t:
-        return "size"
+    if t is ctypes.c_size_t:  # on LP64 also c_uint64
+        return "u64"
     if t in (ctypes.c_int, ctypes.c_int32):
         return "int32"
     return repr(t)
@@ -134,8 +134,8 @@ def _ctype_kind(t):
 def _decl_kind(decl):
     if "*" in decl:
         return "ptr"
-    if decl.split()[0] == "size_t":
-        return "size"
+    if decl.split()[0] in ("size_t", "uint64_t"):
+        return "u64"
     if decl.split()[0] in ("int", "int32_t", "hsa_status_t"):
         return "int32"
     return decl

@@ -551,6 +551,51 @@ def test_device_status_clean_and_bad_index_reported():
     assert m.hsa_device_status(ws) == 0
 
 
+@pytest.mark.parametrize("what", ["fwd", "bwd"])
+def test_wait_limit_runs_out_is_reported_and_the_next_call_is_clean(what):
+    """The failure path of the persistent kernels, exercised on purpose: with every wait
+    bounded at 1 ns some wait runs out, the kernel records HSA_ERR_TIMEOUT in the status
+    word, unwinds (its issued copies and MMAs finish, its tensor memory is freed) and
+    returns.  The next call with the default bound runs normally and matches the oracle."""
+    m = hsa()
+    wl = small(h_q=16, h_kv=2, K=8, L=64 * 40 + 7, B=2, kind="train")
+    x, kbar, sel = gap_ruled(wl)
+    q, k, v, qs, dO = (to_dev(x[n], wl.dtype) for n in ("q", "k", "v", "q_slc", "dO"))
+    nf = m.hsa_workspace_size(wl.B, wl.L, wl.h_q, wl.h_kv, wl.d, 64, wl.K, torch.bfloat16, m.OP_FWD)
+    nb = m.hsa_workspace_size(wl.B, wl.L, wl.h_q, wl.h_kv, wl.d, 64, wl.K, torch.bfloat16, m.OP_BWD)
+    wsf = torch.empty(nf, dtype=torch.uint8, device=DEV)
+    wsb = torch.empty(nb, dtype=torch.uint8, device=DEV)
+    o, lse, idx, w, kb = m.hsa_fwd(q, k, v, qs, wl.K, ws=wsf)
+    torch.cuda.synchronize()
+    assert m.hsa_device_status(wsf) == 0
+    m.hsa_set_wait_limit_ns(1)
+    try:
+        if what == "fwd":
+            m.hsa_fwd(q, k, v, qs, wl.K, ws=wsf)
+            code = m.hsa_device_status(wsf)
+        else:
+            m.hsa_bwd(q, k, v, qs, dO, lse, idx, w, kb, wl.K, ws=wsb)
+            code = m.hsa_device_status(wsb)
+    finally:
+        m.hsa_set_wait_limit_ns(0)
+    torch.cuda.synchronize()
+    assert code == 5, f"expected HSA_ERR_TIMEOUT, got {code}"
+    if what == "fwd":
+        o, lse, idx, w, kb = m.hsa_fwd(q, k, v, qs, wl.K, ws=wsf)
+        torch.cuda.synchronize()
+        assert m.hsa_device_status(wsf) == 0
+        o_ref, _, idx_ref, _ = oracle.fwd(x["q"], x["k"], x["v"], x["q_slc"], kbar, wl.S, wl.K)
+        assert np.array_equal(idx.cpu().numpy().reshape(idx_ref.shape), idx_ref)
+        assert_out(f64(o).reshape(o_ref.shape), o_ref, "bf16", "o after a timed-out call")
+    else:
+        dq, dk, dv, dqs = m.hsa_bwd(q, k, v, qs, dO, lse, idx, w, kb, wl.K, ws=wsb)
+        torch.cuda.synchronize()
+        assert m.hsa_device_status(wsb) == 0
+        ref = oracle.bwd(x["q"], x["k"], x["v"], x["q_slc"], kbar, x["dO"], wl.S, wl.K)
+        for name, g, r in zip(("dq", "dk", "dv", "dq_slc"), (dq, dk, dv, dqs), ref[:4]):
+            assert_out(f64(g), r, "bf16", f"{name} after a timed-out call", grad=True)
+
+
 def test_empty_inputs():
     m = hsa()
     for L in (0, 30):

@@ -78,8 +78,8 @@ template <int D> struct Smem {
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_K = OFF_Q + kQStages * QBYTES;
     static constexpr int OFF_V = OFF_K + 2 * KVBYTES;
-    static constexpr int OFF_X = OFF_V + 2 * KVBYTES;           // epilogue transpose scratch, 4 KB per warp
-    static constexpr int OFF_COEF = OFF_X + 8 * 4096;           // [kInfo][128] fp32 row coefficients w / Z
+    static constexpr int OFF_X = OFF_V + 2 * KVBYTES;           // epilogue transpose scratch, 2 KB per warp
+    static constexpr int OFF_COEF = OFF_X + 8 * 2048;           // [kInfo][128] fp32 row coefficients w / Z
     static constexpr int OFF_INFO = OFF_COEF + kInfo * 128 * 4;
     static constexpr int OFF_BAR = OFF_INFO + kInfo * (int)sizeof(TileInfo);
     static constexpr int NBAR = 3 * kInfo + 2 * kQStages + 2 * 2 + 2 * 2 + 2 + 2 * 2 + 1 + 2;
@@ -559,7 +559,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         const int wq = warp & 3;
         const int r = wq * 32 + lane;                             // tile row of this lane's TMEM loads
         const uint32_t lane_base = tmem + ((uint32_t)(wq * 32) << 16);
-        float4 *xs = reinterpret_cast<float4 *>(sm + L::OFF_X + (warp - kWarpEpi) * 4096);  // [32 rows][8 chunks]
+        float4 *xs = reinterpret_cast<float4 *>(sm + L::OFF_X + (warp - kWarpEpi) * 2048);  // [32 rows][4 chunks]
         int it = 0, tseq = 0, ecnt = 0, ecnt_j = -1;
         bool ok = true;
         // Each warp runs on its own: it waits for itself, acknowledges each info slot
@@ -600,46 +600,43 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
             const float coef = ecoef[ii * 128 + r];
             const int s = inf.j % kRing;
             const int ws = (inf.j % P.nW) * P.W;
-            // this lane reduces, for m = 0..7, the 16-byte chunk lane % 8 (8 halves) of warp row 4m + lane / 8
+            // this lane reduces, for m = 0..3, the 16-byte chunk lane % 4 (8 halves) of warp row 8m + lane / 4
+            // of each 32-column slice: one warp-wide reduction covers 8 rows x 64 contiguous bytes
             const float cf = coef * acc_inv;
-            __half *dst[8];
-            bool dok[8];
+            __half *dst[4];
+            bool dok[4];
 #pragma unroll
-            for (int m = 0; m < 8; ++m) {
-                const int tr = wq * 32 + 4 * m + (lane >> 3);
+            for (int m = 0; m < 4; ++m) {
+                const int tr = wq * 32 + 8 * m + (lane >> 2);
                 const int i = tr / G;
                 dok[m] = i < inf.ntok;
-                dst[m] = acc + ((int64_t)(s * P.W + inf.tok[i] - ws) * G + tr % G) * D + (lane & 7) * 8;
+                dst[m] = acc + ((int64_t)(s * P.W + inf.tok[i] - ws) * G + tr % G) * D + (lane & 3) * 8;
             }
             uint4 *xs4 = reinterpret_cast<uint4 *>(xs);
 #pragma unroll 1
-            for (int q = 0; q < D / 64; ++q) {  // 64 columns = one 128-byte fp16 line per row
-#pragma unroll 1
-                for (int hv = 0; hv < 2; ++hv) {  // 32 columns at a time: 4 chunks of 8 halves
-                    float v[32];
-                    tmem_ld32(lane_base + kColO + sb * 128 + q * 64 + hv * 32, v);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int c4 = 0; c4 < 4; ++c4) {
-                        const int ch = hv * 4 + c4;
-                        __half2 h[4];
-#pragma unroll
-                        for (int e = 0; e < 4; ++e)
-                            h[e] = __floats2half2_rn(v[c4 * 8 + 2 * e] * cf, v[c4 * 8 + 2 * e + 1] * cf);
-                        xs4[lane * 8 + (ch ^ (lane & 7))] = *reinterpret_cast<uint4 *>(h);
-                    }
-                }
-                if (q == D / 64 - 1) {  // O read completely: hand the buffer back before the last reductions
+            for (int q = 0; q < D / 32; ++q) {  // 32 columns = 64 fp16 bytes per row
+                float v[32];
+                tmem_ld32(lane_base + kColO + sb * 128 + q * 32, v);
+                tmem_wait_ld();
+                if (q == D / 32 - 1) {  // O read completely: hand the buffer back before the last reductions
                     tc_fence_before();
                     __syncwarp();
                     mbar_arrive_lane0(&B.o_empty[sb], lane);
                 }
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    __half2 h[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        h[e] = __floats2half2_rn(v[c4 * 8 + 2 * e] * cf, v[c4 * 8 + 2 * e + 1] * cf);
+                    xs4[lane * 4 + (c4 ^ ((lane >> 1) & 3))] = *reinterpret_cast<uint4 *>(h);
+                }
                 __syncwarp();
 #pragma unroll
-                for (int m = 0; m < 8; ++m) {
-                    const int row = 4 * m + (lane >> 3);
-                    const uint4 f = xs4[row * 8 + ((lane & 7) ^ (row & 7))];
-                    if (dok[m]) red_add_v4_f16x2(dst[m] + q * 64, f);
+                for (int m = 0; m < 4; ++m) {
+                    const int row = 8 * m + (lane >> 2);
+                    const uint4 f = xs4[row * 4 + ((lane & 3) ^ ((row >> 1) & 3))];
+                    if (dok[m]) red_add_v4_f16x2(dst[m] + q * 32, f);
                 }
                 __syncwarp();
             }

@@ -10,17 +10,21 @@
 // One cluster of kDecCta CTAs per (b, g); the whole step is latency-bound, so
 // the work is spread over the cluster and exchanged through distributed
 // shared memory instead of global memory:
-//   1. CTA r scores its slice of the chunk index (coalesced 512 B rows).
-//   2. cluster barrier; every CTA reads all scores over DSMEM and selects
-//      the same top-K with all its threads: a threshold (the K-th best of the
-//      per-thread bests) leaves a few survivors, which are ranked pairwise;
-//      warp 0 orders the K most-recent-first and forms the stick-breaking
-//      weights.
+//   1. CTA r scores its slice of the chunk index (coalesced 512 B rows) and
+//      takes the slice's own top-K (a bitonic sort in one warp's registers; a
+//      long slice is first cut down by a threshold), then stores that list into
+//      every CTA of the cluster (remote shared-memory stores).  The K/V of its
+//      two best chunks are prefetched into L2 (caches in device memory): most
+//      of the step's chunks are among them.
+//   2. cluster barrier; warp 0 of every CTA sorts the kDecCta lists (the
+//      overall top-K is among them) in registers, orders the best K
+//      most-recent-first and forms the stick-breaking weights.
 //   3. CTA r attends the group's G query heads to the chunk of slot r (and
 //      r + kDecCta, ...), softmax-off-by-one, and scales by w / Z.
-//   4. cluster barrier; CTA r sums its share of the output columns over all
-//      CTAs' partial outputs (DSMEM) and writes o; a last barrier keeps every
-//      CTA's shared memory alive until all remote reads are done.
+//   4. CTA r stores its partial output into its own slot of the owner CTA of
+//      each output column (remote shared-memory stores); cluster barrier; each
+//      CTA sums its columns' slots in rank order (the result does not depend
+//      on timing) and writes them.
 #include <cooperative_groups.h>
 #include <type_traits>
 #include <math_constants.h>
@@ -35,6 +39,27 @@ namespace hsa {
 
 constexpr int kDecCta = 8;
 constexpr int kDecThreads = 128;
+
+// shared::cluster address of `p` (this CTA's shared memory) in the CTA of cluster rank `rank`
+__device__ __forceinline__ uint32_t dsmem_addr(const void *p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"((uint32_t)__cvta_generic_to_shared(p)), "r"(rank));
+    return r;
+}
+// 8-byte store into another cluster CTA's shared memory
+__device__ __forceinline__ void dsmem_st2(uint32_t addr, float x, float y) {
+    asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(x), "f"(y) : "memory");
+}
+// 16-byte store into another cluster CTA's shared memory
+__device__ __forceinline__ void dsmem_st4(uint32_t addr, float4 v) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z),
+                 "f"(v.w)
+                 : "memory");
+}
+// hint: bring `bytes` (a multiple of 16) at `p` into L2
+__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
 
 // The chunk's K (to a padded [64][D+1] fp32 tile) and V (to [64][D] fp32): every
 // thread issues all of its 16-byte loads before the first store.
@@ -206,18 +231,72 @@ __device__ __forceinline__ void attend_chunk16(const __nv_bfloat16 *Q16, const _
     }
 }
 
-// Sorts one (score, chunk) pair per lane across the warp, best first under `beats`
-// (bitonic network over the 32 lanes).
-__device__ __forceinline__ void warp_sort_best_first(float &s, int &c, int lane) {
+// Sorts the 32 E (score, chunk) pairs a warp holds, best first under `beats`:
+// element i = 32 e + lane sits in lane `lane`, register e.  Bitonic network: a
+// pair that is 32 or more apart lies in one lane, a closer one across lanes.
+template <int E>
+__device__ __forceinline__ void warp_sort_best_first(float (&s)[E], int (&c)[E], int lane) {
 #pragma unroll
-    for (int k = 2; k <= 32; k <<= 1)
+    for (int k = 2; k <= 32 * E; k <<= 1)
 #pragma unroll
         for (int j = k >> 1; j > 0; j >>= 1) {
-            const float os = __shfl_xor_sync(0xffffffffu, s, j);
-            const int oc = __shfl_xor_sync(0xffffffffu, c, j);
-            const bool keep_better = ((lane & j) == 0) == ((lane & k) == 0);
-            if (keep_better == beats(os, oc, s, c)) { s = os; c = oc; }
+            if (j >= 32) {
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    const int p = e ^ (j >> 5);
+                    if (p <= e) continue;
+                    // the lower position keeps the better entry in a block sorted best first
+                    const bool up = ((e * 32 + lane) & k) == 0;
+                    if (up == beats(s[p], c[p], s[e], c[e])) {
+                        const float ts = s[e]; s[e] = s[p]; s[p] = ts;
+                        const int tc = c[e]; c[e] = c[p]; c[p] = tc;
+                    }
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < E; ++e) {
+                    const float os = __shfl_xor_sync(0xffffffffu, s[e], j);
+                    const int oc = __shfl_xor_sync(0xffffffffu, c[e], j);
+                    const int i = e * 32 + lane;
+                    const bool keep_better = ((i & j) == 0) == ((i & k) == 0);
+                    if (keep_better == beats(os, oc, s[e], c[e])) { s[e] = os; c[e] = oc; }
+                }
+            }
         }
+}
+
+// The best K (<= 32) of the n entries (s_i, c_i) = (src_s[i], c0 + i), i < n <= 32 E,
+// sorted in one warp: lane r < K receives the r-th best ((-inf, -1) past n).
+template <int E>
+__device__ __forceinline__ void warp_top_of_scores(const float *src_s, int c0, int n, int lane, float &ls, int &lc) {
+    float s[E];
+    int c[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const int i = e * 32 + lane;
+        s[e] = i < n ? src_s[i] : -CUDART_INF_F;
+        c[e] = i < n ? c0 + i : -1;
+    }
+    warp_sort_best_first<E>(s, c, lane);
+    ls = s[0];
+    lc = c[0];
+}
+
+// The same for n <= 32 E entries given as (score, chunk bits) pairs.
+template <int E>
+__device__ __forceinline__ void warp_top_of_pairs(const float2 *src, int n, int lane, float &ls, int &lc) {
+    float s[E];
+    int c[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+        const int i = e * 32 + lane;
+        const float2 v = i < n ? src[i] : make_float2(-CUDART_INF_F, __int_as_float(-1));
+        s[e] = v.x;
+        c[e] = __float_as_int(v.y);
+    }
+    warp_sort_best_first<E>(s, c, lane);
+    ls = s[0];
+    lc = c[0];
 }
 
 template <typename T, int D>
@@ -225,7 +304,7 @@ __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
     decode_cluster_kernel(const T *__restrict__ q, const T *__restrict__ q_slc, const T *__restrict__ kc,
                           const T *__restrict__ vc, const float *__restrict__ kbar, T *__restrict__ o,
                           int32_t *__restrict__ idx_out, float *__restrict__ w_out, int P, int hq, int hkv,
-                          int nc, int K, int G, int NL, int64_t lstride) {
+                          int nc, int K, int G, int NL, int64_t lstride, int kv_prefetch) {
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
     const int bg = blockIdx.x / kDecCta, b = bg / hkv, g = bg % hkv;
@@ -235,24 +314,32 @@ __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
     extern __shared__ float4 dsm4[];
     float *sm = reinterpret_cast<float *>(dsm4);
     const int per = (nc + kDecCta - 1) / kDecCta;     // chunks scored by each CTA
+    const int per4 = (per + 3) & ~3;
+    const int tot = NL * G * D;                       // output values of the step (a multiple of 64)
+    const int cper = tot / kDecCta;                   // columns owned by each CTA (a multiple of 8)
+    // every region below is a multiple of 16 bytes long
     float *scores = sm;                               // [per]
-    float *part = scores + ((per + 3) & ~3);          // [NL][G][D] partial outputs of this CTA's slots
-    float *Qs = part + NL * kMaxG * D;                // [G][D] one layer's queries
+    float *part = scores + per4;                      // [NL][G][D] partial outputs of this CTA's slots
+    float *Qs = part + tot;                           // [16][D] one layer's queries
     float *Ks = Qs + kMaxG * D;                       // [64][D+1]
     float *Vs = Ks + kChunk * (D + 1);                // [64][D]
     float *Pm = Vs + kChunk * D;                      // [G][64]
-    const int ncr = (nc + 3) & ~3;
-    float *allsc = Pm + kMaxG * kChunk;               // [nc] every chunk's score (top-K stage)
-    float *surv_s = allsc + ncr;                      // [nc] candidates not beaten by the threshold
-    int *surv_c = reinterpret_cast<int *>(surv_s + ncr);
-    __shared__ float tmax_s[kDecThreads];
-    __shared__ int tmax_c[kDecThreads];
-    __shared__ float top_s[kMaxK];
-    __shared__ int top_c[kMaxK];
+    float *surv_s = Pm + kMaxG * kChunk;              // [per] slice entries not beaten by the threshold
+    int *surv_c = reinterpret_cast<int *>(surv_s + per4);
+    float *stage = reinterpret_cast<float *>(surv_c + per4);  // [kDecCta][cper] every source's part of my columns
+    __shared__ float tmax_s[kDecThreads / 32];
+    __shared__ int tmax_c[kDecThreads / 32];
+    __shared__ float loc_s[kMaxK];               // a long slice's top-K, best first
+    __shared__ int loc_c[kMaxK];
+    __shared__ float2 cand[kDecCta * kMaxK];     // every slice's list: (score, chunk bits), written by its CTA
     __shared__ int n_surv;
     __shared__ int slot_c[kMaxK];
     __shared__ float slot_w[kMaxK];
     __shared__ float coef[kMaxG];
+
+    // every CTA of the cluster must be running before its shared memory is written
+    // from another: arrive now, wait before the first remote store (after the scores)
+    asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 
     // ---- 1. scores of this CTA's chunk slice
     const int c_lo = rank * per, c_hi = min(nc, c_lo + per);
@@ -299,84 +386,87 @@ __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
     };
     load_q(0);
     int q_cur = 0;  // the layer whose queries Qs / Q16 hold (block-uniform)
-    for (int e = tid; e < NL * kMaxG * D; e += kDecThreads) part[e] = 0.f;
-    cluster.sync();
+    for (int e = tid; e < tot; e += kDecThreads) part[e] = 0.f;
 
-    // ---- 2. top-K over all chunks (every CTA, all threads), scores read over DSMEM.
-    // Order: (s1, c1) beats (s2, c2) iff s1 > s2, or s1 == s2 and c1 > c2.
-    // 2a. stage every score; each thread keeps the best of its candidates
-    float bs = -CUDART_INF_F;
-    int bc = -1;
-    for (int c = tid; c < nc; c += 2 * kDecThreads) {  // two remote reads in flight at a time
-        const int c2 = c + kDecThreads;
-        const float s1 = cluster.map_shared_rank(scores, c / per)[c % per];
-        const float s2 = (c2 < nc) ? cluster.map_shared_rank(scores, c2 / per)[c2 % per] : -CUDART_INF_F;
-        allsc[c] = s1;
-        if (beats(s1, c, bs, bc)) { bs = s1; bc = c; }
-        if (c2 < nc) {
-            allsc[c2] = s2;
-            if (beats(s2, c2, bs, bc)) { bs = s2; bc = c2; }
+    // ---- 1b. this slice's top-K, into every CTA's candidate list.  Order: (s1, c1)
+    // beats (s2, c2) iff s1 > s2, or s1 == s2 and c1 > c2.  A slice of up to 128
+    // chunks is sorted by warp 0 in registers.  A longer one is first cut down: each
+    // thread keeps the best of its entries and each warp sorts its 32 bests; a warp's
+    // K-th is a lower bound of the slice's K-th best score (the warp holds K distinct
+    // entries at least as good), the best of the warps' bounds is the threshold, and
+    // the entries it does not beat are ranked pairwise.
+    __syncthreads();  // scores[] written
+    const int nloc = c_hi - c_lo;
+    float ls = -CUDART_INF_F;  // warp 0, lane r < K: the slice's r-th best
+    int lc = -1;
+    if (nloc <= 128) {
+        if (warp == 0) {
+            if (nloc <= 32) warp_top_of_scores<1>(scores, c_lo, nloc, lane, ls, lc);
+            else if (nloc <= 64) warp_top_of_scores<2>(scores, c_lo, nloc, lane, ls, lc);
+            else warp_top_of_scores<4>(scores, c_lo, nloc, lane, ls, lc);
         }
-    }
-    // 2b. threshold: each warp sorts its 32 per-thread bests, best first (bitonic network
-    //     over the lanes); its K-th is a lower bound of the overall K-th best score (the
-    //     warp holds K distinct candidates at least as good), and the threshold is the
-    //     best of the warps' bounds
-    {
-        float s = bs;
-        int c = bc;
-        warp_sort_best_first(s, c, lane);
-        if (lane == K - 1) { tmax_s[warp] = s; tmax_c[warp] = c; }
-    }
-    if (tid == 0) n_surv = 0;
-    __syncthreads();
-    // 2c. survivors: the candidates that the threshold does not beat
-    {
-        float ts = tmax_s[0];
-        int tc = tmax_c[0];
+    } else {
+        {
+            float bs[1] = {-CUDART_INF_F};
+            int bc[1] = {-1};
+            for (int i = tid; i < nloc; i += kDecThreads)
+                if (beats(scores[i], c_lo + i, bs[0], bc[0])) { bs[0] = scores[i]; bc[0] = c_lo + i; }
+            warp_sort_best_first<1>(bs, bc, lane);
+            if (lane == K - 1) { tmax_s[warp] = bs[0]; tmax_c[warp] = bc[0]; }
+        }
+        if (tid == 0) n_surv = 0;
+        __syncthreads();
+        {
+            float ts = tmax_s[0];
+            int tc = tmax_c[0];
 #pragma unroll
-        for (int q = 1; q < kDecThreads / 32; ++q)
-            if (beats(tmax_s[q], tmax_c[q], ts, tc)) { ts = tmax_s[q]; tc = tmax_c[q]; }
-        for (int c = tid; c < nc; c += kDecThreads) {
-            const float sc = allsc[c];
-            if (!beats(ts, tc, sc, c)) {
-                const int i = atomicAdd(&n_surv, 1);
-                surv_s[i] = sc;
-                surv_c[i] = c;
-            }
-        }
-    }
-    __syncthreads();
-    // 2d. the K best survivors, best first: with at most 32 survivors (the usual case)
-    //     warp 0 sorts them in registers; otherwise every survivor is ranked pairwise
-    const int ns = n_surv;
-    if (ns > 32) {
-        for (int i = tid; i < ns; i += kDecThreads) {
-            const float si = surv_s[i];
-            const int ci = surv_c[i];
-            int rk = 0;
-            for (int j = 0; j < ns; ++j) rk += beats(surv_s[j], surv_c[j], si, ci) ? 1 : 0;
-            if (rk < K) { top_s[rk] = si; top_c[rk] = ci; }
+            for (int w = 1; w < kDecThreads / 32; ++w)
+                if (beats(tmax_s[w], tmax_c[w], ts, tc)) { ts = tmax_s[w]; tc = tmax_c[w]; }
+            for (int i = tid; i < nloc; i += kDecThreads)
+                if (!beats(ts, tc, scores[i], c_lo + i)) {
+                    const int j = atomicAdd(&n_surv, 1);
+                    surv_s[j] = scores[i];
+                    surv_c[j] = c_lo + i;
+                }
+            if (tid < K) { loc_s[tid] = -CUDART_INF_F; loc_c[tid] = -1; }  // fewer than K entries in the slice
         }
         __syncthreads();
-    }
-    // 2e. warp 0: most-recent-first order and the stick-breaking weights
-    if (warp == 0) {
-        const int nsel = min(K, ns);
-        float ls, lc_s;
-        int lc;
-        if (ns > 32) {
-            ls = (lane < nsel) ? top_s[lane] : -CUDART_INF_F;
-            lc = (lane < nsel) ? top_c[lane] : -1;
-        } else {
-            lc_s = (lane < ns) ? surv_s[lane] : -CUDART_INF_F;
-            lc = (lane < ns) ? surv_c[lane] : -1;
-            warp_sort_best_first(lc_s, lc, lane);
-            ls = (lane < nsel) ? lc_s : -CUDART_INF_F;
-            if (lane >= nsel) lc = -1;
+        {
+            const int ns = n_surv;
+            for (int i = tid; i < ns; i += kDecThreads) {
+                const float si = surv_s[i];
+                const int ci = surv_c[i];
+                int rk = 0;
+                for (int j = 0; j < ns; ++j) rk += beats(surv_s[j], surv_c[j], si, ci) ? 1 : 0;
+                if (rk < K) { loc_s[rk] = si; loc_c[rk] = ci; }
+            }
         }
+        __syncthreads();
+        if (warp == 0 && lane < K) { ls = loc_s[lane]; lc = loc_c[lane]; }
+    }
+    asm volatile("barrier.cluster.wait.aligned;" ::: "memory");
+    if (warp == 0 && lane < K) {
+#pragma unroll
+        for (int r = 0; r < kDecCta; ++r) dsmem_st2(dsmem_addr(&cand[rank * K + lane], (uint32_t)r), ls, __int_as_float(lc));
+        if (kv_prefetch && lane < 2 && lc >= 0) {  // the slice's two best chunks: K and V into L2
+            const int64_t off = ((int64_t)bg * P + (int64_t)lc * kChunk) * D;
+            prefetch_l2(kc + off, kChunk * D * sizeof(T));
+            prefetch_l2(vc + off, kChunk * D * sizeof(T));
+        }
+    }
+    cluster.sync();
+
+    // ---- 2. the overall top-K: the best K of the kDecCta slice lists (every CTA
+    // sorts the same candidates, so all take the same selection); most-recent-first
+    // order and the stick-breaking weights
+    if (warp == 0) {
+        float ms;
+        int mc;
+        if (K <= 4) warp_top_of_pairs<1>(cand, kDecCta * K, lane, ms, mc);
+        else if (K <= 8) warp_top_of_pairs<2>(cand, kDecCta * K, lane, ms, mc);
+        else warp_top_of_pairs<4>(cand, kDecCta * K, lane, ms, mc);
         int sc_; float sw, ss;
-        topk_finish(K, ls, lc, sc_, sw, ss);
+        topk_finish(K, ms, mc, sc_, sw, ss);
         if (lane < K) {
             slot_c[lane] = sc_;
             slot_w[lane] = sw;
@@ -406,7 +496,7 @@ __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
                     q_cur = l;
                     __syncthreads();
                 }
-                attend_chunk16<D>(Q16, K16, V16, part + l * kMaxG * D, G, wk, scale, warp, lane);
+                attend_chunk16<D>(Q16, K16, V16, part + l * G * D, G, wk, scale, warp, lane);
             }
             continue;
         }
@@ -418,7 +508,7 @@ __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
             q_cur = l;
             __syncthreads();
         }
-        float *pl = part + l * kMaxG * D;
+        float *pl = part + l * G * D;
         for (int e = tid; e < G * kChunk; e += kDecThreads) {
             const int h = e / kChunk, i = e % kChunk;
             const float *qh = Qs + h * D;
@@ -455,56 +545,67 @@ __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
         __syncthreads();  // Qs, Pm and coef are rewritten for the next layer
         }
     }
-    cluster.sync();
-
-    // ---- 4. sum the partial outputs of the cluster (DSMEM), this CTA's column share
-    const int ncol = G * D, tot = NL * ncol;
-    const int cper = (tot + kDecCta - 1) / kDecCta;
-    for (int e = rank * cper + tid; e < min(tot, (rank + 1) * cper); e += kDecThreads) {
-        const int l = e / ncol, col = e - l * ncol;
-        float acc = 0.f;
-#pragma unroll
-        for (int r = 0; r < kDecCta; ++r) acc += cluster.map_shared_rank(part, r)[l * kMaxG * D + col];
-        Elem<T>::store(o + (int64_t)l * lstride + ((int64_t)b * hq + (int64_t)g * G) * D + col, acc);
+    // ---- 4. this CTA's partial output stored into its slot at the owners of its
+    // columns (the CTAs with a selected chunk are the ranks below n_src; the others
+    // hold zeros and send nothing); after the barrier every owner holds all the
+    // parts of its columns, and no CTA touches another's shared memory any more
+    int n_src = 0;
+    while (n_src < kDecCta && n_src < K && slot_c[n_src] >= 0) ++n_src;
+    if (rank < n_src) {
+        for (int e = 4 * tid; e < tot; e += 4 * kDecThreads) {  // cper is a multiple of 4: one owner per vector
+            const int ow = e / cper;
+            dsmem_st4(dsmem_addr(stage + rank * cper + (e - ow * cper), (uint32_t)ow),
+                      *reinterpret_cast<const float4 *>(part + e));
+        }
     }
     cluster.sync();
+    const int ncol = G * D;
+    for (int i = tid; i < cper; i += kDecThreads) {
+        float acc = 0.f;
+        for (int r = 0; r < n_src; ++r) acc += stage[r * cper + i];  // rank order
+        const int e = rank * cper + i, l = e / ncol, col = e - l * ncol;
+        Elem<T>::store(o + (int64_t)l * lstride + ((int64_t)b * hq + (int64_t)g * G) * D + col, acc);
+    }
 }
 
 
-size_t decode_cluster_smem(int nc, int d, int NL) {
-    const int per = (nc + kDecCta - 1) / kDecCta;
-    const size_t ncr = (size_t)((nc + 3) & ~3);
-    return sizeof(float) * ((size_t)((per + 3) & ~3) + (size_t)(NL + 1) * kMaxG * d + (size_t)kChunk * (d + 1) +
-                            (size_t)kChunk * d + (size_t)kMaxG * kChunk + 3 * ncr);
+size_t decode_cluster_smem(int nc, int d, int NL, int G) {
+    const size_t per4 = (size_t)(((nc + kDecCta - 1) / kDecCta + 3) & ~3);
+    const size_t tot = (size_t)NL * G * d;
+    // scores, survivors (2), part and stage, Q, K, V, P
+    return sizeof(float) * (3 * per4 + 2 * tot + (size_t)kMaxG * d + (size_t)kChunk * (d + 1) + (size_t)kChunk * d +
+                            (size_t)kMaxG * kChunk);
 }
 
 template <typename T, int D>
 static cudaError_t decode_launch(const Shape &sh, int NL, const void *q, const void *q_slc, const void *kc,
                                  const void *vc, const float *kbar, void *o, int32_t *idx_out, float *w_out,
-                                 cudaStream_t st) {
-    const size_t smem = decode_cluster_smem(sh.nc, D, NL);
+                                 bool kv_device, cudaStream_t st) {
+    const size_t smem = decode_cluster_smem(sh.nc, D, NL, sh.G);
     cudaError_t e = set_smem_once((const void *)decode_cluster_kernel<T, D>, smem);
     if (e != cudaSuccess) return e;
     decode_cluster_kernel<T, D><<<(unsigned)(sh.B * sh.hkv * kDecCta), kDecThreads, smem, st>>>(
         (const T *)q, (const T *)q_slc, (const T *)kc, (const T *)vc, kbar, (T *)o, idx_out, w_out, sh.L, sh.hq,
-        sh.hkv, sh.nc, sh.K, sh.G, NL, (int64_t)sh.B * sh.hq * D);
+        sh.hkv, sh.nc, sh.K, sh.G, NL, (int64_t)sh.B * sh.hq * D, kv_device ? 1 : 0);
     return cudaGetLastError();
 }
 
 bool decode_cluster_supported(const Shape &sh, int NL) {
     return (sh.d == 64 || sh.d == 128) && sh.G <= kMaxG && sh.K <= kMaxK && NL >= 1 &&
-           decode_cluster_smem(sh.nc, sh.d, NL) <= 200 * 1024;
+           decode_cluster_smem(sh.nc, sh.d, NL, sh.G) <= 200 * 1024;
 }
 
 cudaError_t launch_decode_cluster(const Shape &sh, int NL, const void *q, const void *q_slc, const void *kc,
                                   const void *vc, const float *kbar, void *o, int32_t *idx_out, float *w_out,
-                                  DevStatus *, cudaStream_t st) {
+                                  bool kv_device, DevStatus *, cudaStream_t st) {
     if (sh.B == 0) return cudaSuccess;
     if (sh.bf16)
-        return sh.d == 128 ? decode_launch<__nv_bfloat16, 128>(sh, NL, q, q_slc, kc, vc, kbar, o, idx_out, w_out, st)
-                           : decode_launch<__nv_bfloat16, 64>(sh, NL, q, q_slc, kc, vc, kbar, o, idx_out, w_out, st);
-    return sh.d == 128 ? decode_launch<float, 128>(sh, NL, q, q_slc, kc, vc, kbar, o, idx_out, w_out, st)
-                       : decode_launch<float, 64>(sh, NL, q, q_slc, kc, vc, kbar, o, idx_out, w_out, st);
+        return sh.d == 128 ? decode_launch<__nv_bfloat16, 128>(sh, NL, q, q_slc, kc, vc, kbar, o, idx_out, w_out,
+                                                               kv_device, st)
+                           : decode_launch<__nv_bfloat16, 64>(sh, NL, q, q_slc, kc, vc, kbar, o, idx_out, w_out,
+                                                              kv_device, st);
+    return sh.d == 128 ? decode_launch<float, 128>(sh, NL, q, q_slc, kc, vc, kbar, o, idx_out, w_out, kv_device, st)
+                       : decode_launch<float, 64>(sh, NL, q, q_slc, kc, vc, kbar, o, idx_out, w_out, kv_device, st);
 }
 
 }  // namespace hsa

@@ -26,10 +26,10 @@ namespace hsa {
 // patterns) into *x.vmax_bits: the scale of the chunk-major attention's fp16
 // accumulators, which only ever sum values of complete chunks.
 template <typename T>
-__global__ void __launch_bounds__(128) pool_kernel(const T *__restrict__ k, float *__restrict__ kbar,
+__global__ void __launch_bounds__(128, 4) pool_kernel(const T *__restrict__ k, float *__restrict__ kbar,
                                                    int L, int d, int nc, int64_t nchunks, PoolExtras x) {
     constexpr int VEC = 16 / sizeof(T);
-    constexpr int NB = 16;  // loads in flight per lane
+    constexpr int NB = 8;  // rows in flight per lane and tensor (4 blocks per SM stay resident)
     const int lane = threadIdx.x & 31;
     const int64_t bgc = (blockIdx.x * (int64_t)blockDim.x + threadIdx.x) >> 5;  // this warp's chunk
     if (bgc >= nchunks) return;

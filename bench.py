@@ -402,6 +402,8 @@ def main():
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     ap.add_argument("--no-extras", action="store_true", help="skip the decode and train measurements")
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="time only the decode16k step (one GPU; the case used for ncu captures of the decode kernel)")
     ap.add_argument("--workload", default="fwd64k", choices=["fwd64k", "fwd16k"],
                     help="forward workload (fwd16k: the smaller case used for ncu captures)")
     args = ap.parse_args()
@@ -424,6 +426,11 @@ def main():
     dev = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(dev)
     hsa.load_library()
+    if args.decode_only:
+        if rank == 0:
+            print(json.dumps({"decode": bench_decode(hsa, dev)}), flush=True)
+        dist_util.finish(world)
+        return
 
     base = synth.WORKLOADS[args.workload]
     wl = base.scaled(seed=dist_util.rank_seed(base.seed, rank))  # one independent sequence per rank

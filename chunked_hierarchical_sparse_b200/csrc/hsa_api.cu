@@ -371,7 +371,7 @@ hsa_status_t hsa_attend(const hsa_shape_t *shape, const void *q, const void *k, 
 // The address a kernel reads `p` through: device (or managed) memory as is,
 // page-locked host memory through its mapped device address.  Pageable host
 // memory has no such address and is refused before any launch.
-static bool device_view(const void *p, const void **dp, bool *on_device = nullptr) {
+static bool device_view(const void *p, const void **dp) {
     cudaPointerAttributes a{};
     if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
         (void)cudaGetLastError();  // a plain host pointer: clear the sticky-free error state
@@ -379,7 +379,6 @@ static bool device_view(const void *p, const void **dp, bool *on_device = nullpt
     }
     if (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) {
         *dp = p;
-        if (on_device) *on_device = a.type == cudaMemoryTypeDevice;
         return true;
     }
     if (a.type == cudaMemoryTypeHost && a.devicePointer) {
@@ -402,8 +401,7 @@ hsa_status_t hsa_decode_multi(const hsa_shape_t *shape, int32_t n_layers, const 
     if (sh.nc > 0 && !ptrs_ok({k_cache, v_cache, kbar})) return HSA_ERR_INVALID_ARG;
     if ((s = check_ws(sh, HSA_OP_DECODE, ws, ws_bytes)) != HSA_OK) return s;
     const void *kc = k_cache, *vc = v_cache;
-    bool k_dev = false, v_dev = false;
-    if (sh.nc > 0 && (!device_view(k_cache, &kc, &k_dev) || !device_view(v_cache, &vc, &v_dev))) return HSA_ERR_INVALID_ARG;
+    if (sh.nc > 0 && (!device_view(k_cache, &kc) || !device_view(v_cache, &vc))) return HSA_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     DevStatus *ds = static_cast<DevStatus *>(ws);
     const bool cluster = decode_cluster_supported(sh, n_layers);
@@ -411,7 +409,7 @@ hsa_status_t hsa_decode_multi(const hsa_shape_t *shape, int32_t n_layers, const 
     if (e == cudaSuccess)
         e = timed(HSA_K_DECODE, cluster ? 1 : n_layers, st, [&] {
             if (cluster)
-                return launch_decode_cluster(sh, n_layers, q, q_slc, kc, vc, kbar, o, idx, w, k_dev && v_dev, ds, st);
+                return launch_decode_cluster(sh, n_layers, q, q_slc, kc, vc, kbar, o, idx, w, ds, st);
             // very long caches, or more layers x heads than the cluster's shared memory holds:
             // token-major kernel, one launch per layer (each repeats the selection)
             const size_t lbytes = (size_t)sh.B * sh.hq * sh.d * (sh.bf16 ? 2 : 4);

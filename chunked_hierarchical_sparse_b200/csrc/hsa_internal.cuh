@@ -129,11 +129,9 @@ cudaError_t launch_decode_simt(const Shape &sh, const void *q, const void *q_slc
 // Decode on a thread-block cluster per (b, g) (DSMEM exchange of scores and partials).
 // NL layers' queries q [NL,B,h_q,d] share the step's selection and chunk reads; o [NL,B,h_q,d].
 bool decode_cluster_supported(const Shape &sh, int NL);
-// kv_device: both caches are device memory (their likely chunks may be prefetched into L2;
-// caches in page-locked host memory are read only where selected)
 cudaError_t launch_decode_cluster(const Shape &sh, int NL, const void *q, const void *q_slc, const void *kc,
                                   const void *vc, const float *kbar, void *o, int32_t *idx_out, float *w_out,
-                                  bool kv_device, DevStatus *ds, cudaStream_t st);
+                                  DevStatus *ds, cudaStream_t st);
 
 // Backward pieces.
 struct BwdWs {

@@ -13,9 +13,7 @@
 //   1. CTA r scores its slice of the chunk index (coalesced 512 B rows) and
 //      takes the slice's own top-K (a bitonic sort in one warp's registers; a
 //      long slice is first cut down by a threshold), then stores that list into
-//      every CTA of the cluster (remote shared-memory stores).  The K/V of its
-//      two best chunks are prefetched into L2 (caches in device memory): most
-//      of the step's chunks are among them.
+//      every CTA of the cluster (remote shared-memory stores).
 //   2. cluster barrier; warp 0 of every CTA sorts the kDecCta lists (the
 //      overall top-K is among them) in registers, orders the best K
 //      most-recent-first and forms the stick-breaking weights.
@@ -55,10 +53,6 @@ __device__ __forceinline__ void dsmem_st4(uint32_t addr, float4 v) {
     asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z),
                  "f"(v.w)
                  : "memory");
-}
-// hint: bring `bytes` (a multiple of 16) at `p` into L2
-__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes) {
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
 }
 
 // The chunk's K (to a padded [64][D+1] fp32 tile) and V (to [64][D] fp32): every
@@ -304,7 +298,7 @@ __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
     decode_cluster_kernel(const T *__restrict__ q, const T *__restrict__ q_slc, const T *__restrict__ kc,
                           const T *__restrict__ vc, const float *__restrict__ kbar, T *__restrict__ o,
                           int32_t *__restrict__ idx_out, float *__restrict__ w_out, int P, int hq, int hkv,
-                          int nc, int K, int G, int NL, int64_t lstride, int kv_prefetch) {
+                          int nc, int K, int G, int NL, int64_t lstride) {
     cg::cluster_group cluster = cg::this_cluster();
     const int rank = (int)cluster.block_rank();
     const int bg = blockIdx.x / kDecCta, b = bg / hkv, g = bg % hkv;
@@ -448,11 +442,6 @@ __global__ void __cluster_dims__(kDecCta, 1, 1) __launch_bounds__(kDecThreads)
     if (warp == 0 && lane < K) {
 #pragma unroll
         for (int r = 0; r < kDecCta; ++r) dsmem_st2(dsmem_addr(&cand[rank * K + lane], (uint32_t)r), ls, __int_as_float(lc));
-        if (kv_prefetch && lane < 2 && lc >= 0) {  // the slice's two best chunks: K and V into L2
-            const int64_t off = ((int64_t)bg * P + (int64_t)lc * kChunk) * D;
-            prefetch_l2(kc + off, kChunk * D * sizeof(T));
-            prefetch_l2(vc + off, kChunk * D * sizeof(T));
-        }
     }
     cluster.sync();
 
@@ -580,13 +569,13 @@ size_t decode_cluster_smem(int nc, int d, int NL, int G) {
 template <typename T, int D>
 static cudaError_t decode_launch(const Shape &sh, int NL, const void *q, const void *q_slc, const void *kc,
                                  const void *vc, const float *kbar, void *o, int32_t *idx_out, float *w_out,
-                                 bool kv_device, cudaStream_t st) {
+                                 cudaStream_t st) {
     const size_t smem = decode_cluster_smem(sh.nc, D, NL, sh.G);
     cudaError_t e = set_smem_once((const void *)decode_cluster_kernel<T, D>, smem);
     if (e != cudaSuccess) return e;
     decode_cluster_kernel<T, D><<<(unsigned)(sh.B * sh.hkv * kDecCta), kDecThreads, smem, st>>>(
         (const T *)q, (const T *)q_slc, (const T *)kc, (const T *)vc, kbar, (T *)o, idx_out, w_out, sh.L, sh.hq,
-        sh.hkv, sh.nc, sh.K, sh.G, NL, (int64_t)sh.B * sh.hq * D, kv_device ? 1 : 0);
+        sh.hkv, sh.nc, sh.K, sh.G, NL, (int64_t)sh.B * sh.hq * D);
     return cudaGetLastError();
 }
 
@@ -597,15 +586,13 @@ bool decode_cluster_supported(const Shape &sh, int NL) {
 
 cudaError_t launch_decode_cluster(const Shape &sh, int NL, const void *q, const void *q_slc, const void *kc,
                                   const void *vc, const float *kbar, void *o, int32_t *idx_out, float *w_out,
-                                  bool kv_device, DevStatus *, cudaStream_t st) {
+                                  DevStatus *, cudaStream_t st) {
     if (sh.B == 0) return cudaSuccess;
     if (sh.bf16)
-        return sh.d == 128 ? decode_launch<__nv_bfloat16, 128>(sh, NL, q, q_slc, kc, vc, kbar, o, idx_out, w_out,
-                                                               kv_device, st)
-                           : decode_launch<__nv_bfloat16, 64>(sh, NL, q, q_slc, kc, vc, kbar, o, idx_out, w_out,
-                                                              kv_device, st);
-    return sh.d == 128 ? decode_launch<float, 128>(sh, NL, q, q_slc, kc, vc, kbar, o, idx_out, w_out, kv_device, st)
-                       : decode_launch<float, 64>(sh, NL, q, q_slc, kc, vc, kbar, o, idx_out, w_out, kv_device, st);
+        return sh.d == 128 ? decode_launch<__nv_bfloat16, 128>(sh, NL, q, q_slc, kc, vc, kbar, o, idx_out, w_out, st)
+                           : decode_launch<__nv_bfloat16, 64>(sh, NL, q, q_slc, kc, vc, kbar, o, idx_out, w_out, st);
+    return sh.d == 128 ? decode_launch<float, 128>(sh, NL, q, q_slc, kc, vc, kbar, o, idx_out, w_out, st)
+                       : decode_launch<float, 64>(sh, NL, q, q_slc, kc, vc, kbar, o, idx_out, w_out, st);
 }
 
 }  // namespace hsa

@@ -24,6 +24,14 @@
 // dK/dV flush, warps 8-9 convert step, warp 10 producer (TMA), warp 11 MMA
 // issuer.  Every wait is bounded; on expiry the kernel records HSA_ERR_TIMEOUT
 // and returns.
+//
+// Head dims 128 and 64.  For d = 64 every MMA keeps M = 128: a tile's Q and dO
+// rows share one buffer, each 8-row group holding its Q rows then its dO rows,
+// which is the d = 128 layout of Q with dO in place of the second 64-column
+// half.  Read as an MN-major operand of 128 rows that buffer is [Q^T; dO^T], so
+//   [Q^T; dO^T] dS = [dK^T; dO^T dS]   (TMEM lanes 0-63 hold dK^T)
+//   [Q^T; dO^T] wP = [Q^T wP; dV^T]    (TMEM lanes 64-127 hold dV^T)
+// and the flush reads the lanes that hold the gradients.
 #include <algorithm>
 
 #include "hsa_internal.cuh"
@@ -48,7 +56,6 @@ constexpr int kBWarpEpi = 4, kBWarpConv = 8, kBWarpProd = 10, kBWarpMma = 11;
 constexpr int kBConvThreads = 64;
 constexpr int kBInfo = 8;  // tile-info ring entries
 constexpr int kBItemTile = 0, kBItemEnd = 2;
-constexpr int kBD = 128;   // head dim of the tensor-core backward
 
 struct BTileInfo {
     int type;
@@ -62,17 +69,21 @@ struct BTileInfo {
     float w[16];  // stick-breaking weight of each token's slot
 };
 
-struct BSmem {
-    // a 128-row Q / dO tile: 16 groups of 8 rows, each group's two 64-column halves one
-    // after the other (1 KB each), so one TMA box loads a group
+template <int D> struct BSmem {
+    // d = 128: a 128-row Q (or dO) tile is 16 groups of 8 rows, each group's two 64-column
+    // halves one after the other (1 KB each), so one TMA box loads a group.
+    // d = 64: one 32 KB buffer per stage holds the Q and the dO rows of a tile, each
+    // group's Q rows (1 KB) then its dO rows (1 KB).
+    static constexpr bool kStack = D == 64;
     static constexpr int QHALF = 128 * 128;  // bytes of one 64-column half of a 128-row tile
     static constexpr int QBYTES = 2 * QHALF;
+    static constexpr int NQBUF = kStack ? 2 : 4;  // 32 KB buffers: [2] Q and [2] dO, or [2] Q|dO
     static constexpr int KVHALF = 64 * 128;
-    static constexpr int KVBYTES = 2 * KVHALF;
+    static constexpr int KVBYTES = (D / 64) * KVHALF;
     static constexpr int PB = 128 * 128;     // 128 rows x 64 keys bf16
     static constexpr int OFF_Q = 0;                      // [2] query tiles
-    static constexpr int OFF_DO = OFF_Q + 2 * QBYTES;    // [2] output-gradient tiles
-    static constexpr int OFF_K = OFF_DO + 2 * QBYTES;
+    static constexpr int OFF_DO = kStack ? OFF_Q + 1024 : OFF_Q + 2 * QBYTES;  // [2] output-gradient tiles
+    static constexpr int OFF_K = OFF_Q + NQBUF * QBYTES;
     static constexpr int OFF_V = OFF_K + KVBYTES;
     static constexpr int OFF_DS = OFF_V + KVBYTES;       // dS (bf16, swizzled rows)
     static constexpr int OFF_WP = OFF_DS + PB;           // w p (bf16, swizzled rows)
@@ -84,7 +95,7 @@ struct BSmem {
     static constexpr int BYTES = OFF_MISC + 64;
     static constexpr int ALLOC = BYTES + 1024;  // slack for 1 KB alignment
 };
-static_assert(BSmem::ALLOC <= 227 * 1024, "backward tile buffers exceed the shared memory of a CTA");
+static_assert(BSmem<128>::ALLOC <= 227 * 1024, "backward tile buffers exceed the shared memory of a CTA");
 
 // TMEM columns: S 0..63, dP 64..127, dQ[2] 128..383, dK^T 384..447, dV^T 448..511 (the gradient
 // warps copy S and dP out at once, so one buffer each; the dQ drain overlaps the next dQ)
@@ -128,15 +139,14 @@ __device__ __forceinline__ uint4 pack8(const float *f) {
 
 }  // namespace
 
-template <int G>
+template <int G, int D>
 __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
     const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
     const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
     const __grid_constant__ AttendPlan P, const int32_t *__restrict__ entries, const float *__restrict__ entw,
     const float *__restrict__ lse, float *__restrict__ dw, __half *__restrict__ acc, __nv_bfloat16 *__restrict__ dq,
     float *__restrict__ dk_acc, float *__restrict__ dv_acc, DevStatus *ds, uint64_t wait_ns) {
-    using L = BSmem;
-    constexpr int D = kBD;
+    using L = BSmem<D>;
     constexpr int TT = 128 / G;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -173,7 +183,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
     // Q / dO rows of a ragged tile's missing tokens are never loaded; dK^T and dV^T
     // contract over all 128 rows, so the buffers start at zero and only ever hold
     // finite input rows afterwards (their dS / wP rows are zero).
-    for (int e = threadIdx.x; e < 4 * L::QBYTES / 16; e += kBThreads)
+    for (int e = threadIdx.x; e < L::NQBUF * L::QBYTES / 16; e += kBThreads)
         reinterpret_cast<uint4 *>(sm + L::OFF_Q)[e] = make_uint4(0, 0, 0, 0);
     fence_proxy_async_smem();
     if (warp == kBWarpMma) {
@@ -277,7 +287,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
                 mbar_arrive_expect_tx(kv_full, 2 * L::KVBYTES);
                 const int row = bg * P.L + c * kChunk;
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
+                for (int h = 0; h < D / 64; ++h) {
                     tma_load_2d(sm + L::OFF_K + h * L::KVHALF, &tm_k, h * 64, row, kv_full);
                     tma_load_2d(sm + L::OFF_V + h * L::KVHALF, &tm_v, h * 64, row, kv_full);
                 }
@@ -306,16 +316,22 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
                     ti_.kvph = useq & 1; ti_.useq = useq;
                     ti_.unit_first = (tt == t0); ti_.unit_last = (tt == t1 - 1);
                     ti_.qs = qs; ti_.qph = qph;
-                    mbar_arrive_expect_tx(&qd_full[qs], 2 * ntok * 2 * G * 128);
+                    mbar_arrive_expect_tx(&qd_full[qs], 2 * ntok * G * D * 2);  // Q and dO rows, bf16
                 }
                 __syncwarp();
-                {  // one 3D box per 8-row group (both 64-column halves, 2 KB) for Q and for dO
+                {  // per 8-row group: d = 128, one 3D box (both 64-column halves, 2 KB) for Q and
+                   // for dO; d = 64, one 2D box (1 KB) each, side by side in the group's 2 KB
                     constexpr int GPT = G / 8;  // 8-row groups per token
                     const int tq = __shfl_sync(0xffffffffu, t, lane / GPT);
                     if (lane < ntok * GPT) {
                         const int row = (b * P.L + tq) * P.hq + g * G + (lane % GPT) * 8;
-                        tma_load_3d(sm + L::OFF_Q + qs * L::QBYTES + lane * 2048, &tm_q, 0, row, 0, &qd_full[qs]);
-                        tma_load_3d(sm + L::OFF_DO + qs * L::QBYTES + lane * 2048, &tm_do, 0, row, 0, &qd_full[qs]);
+                        if constexpr (D == 128) {
+                            tma_load_3d(sm + L::OFF_Q + qs * L::QBYTES + lane * 2048, &tm_q, 0, row, 0, &qd_full[qs]);
+                            tma_load_3d(sm + L::OFF_DO + qs * L::QBYTES + lane * 2048, &tm_do, 0, row, 0, &qd_full[qs]);
+                        } else {
+                            tma_load_2d(sm + L::OFF_Q + qs * L::QBYTES + lane * 2048, &tm_q, 0, row, &qd_full[qs]);
+                            tma_load_2d(sm + L::OFF_DO + qs * L::QBYTES + lane * 2048, &tm_do, 0, row, &qd_full[qs]);
+                        }
                     }
                 }
                 __syncwarp();
@@ -347,9 +363,11 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
         //   scores:    S = Q K^T and dP = dO V^T of tile ts (needs Q, dO, K, V and a free S/dP buffer)
         //   gradients: dQ = dS K, dK^T += Q^T dS, dV^T += dO^T wP of tile tg (needs dS / wP, a free
         //              dQ buffer and, at a unit's first tile, the previous unit's dK/dV flushed)
+        // dK^T / dV^T have M = 128: the d = 128 rows of Q^T / dO^T, or for d = 64 the stacked
+        // [Q^T; dO^T] of the shared buffer (both MMAs read it; see the file comment)
         constexpr uint32_t id_s = idesc_bf16_f32(128, 64, false, false);
         constexpr uint32_t id_dq = idesc_bf16_f32(128, D, false, true);
-        constexpr uint32_t id_dkv = idesc_bf16_f32(D, 64, true, true);
+        constexpr uint32_t id_dkv = idesc_bf16_f32(128, 64, true, true);
         bool ok = true;
         int ts = 0, tg = 0;
         if (lane == 0) {
@@ -398,7 +416,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
                         (!inf.unit_first || inf.useq < 1 || mbar_test(dkv_empty, (inf.useq - 1) & 1))) {
                         tc_fence_after();
                         const uint32_t qa = smem_u32(sm + L::OFF_Q + inf.qs * L::QBYTES);
-                        const uint32_t oa = smem_u32(sm + L::OFF_DO + inf.qs * L::QBYTES);
+                        const uint32_t oa = L::kStack ? qa : smem_u32(sm + L::OFF_DO + inf.qs * L::QBYTES);
                         const uint32_t kb = smem_u32(sm + L::OFF_K);
                         const uint32_t dsa = smem_u32(sm + L::OFF_DS);
                         const uint32_t wpa = smem_u32(sm + L::OFF_WP);
@@ -643,18 +661,36 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
             if (inf.unit_last) {
                 if (!eg_wait(dkv_full, inf.useq & 1)) { ok = false; break; }
                 tc_fence_after();
-                const int64_t krow = ((int64_t)(inf.b * P.hkv + inf.g) * P.L + (int64_t)inf.c * kChunk) * D + r;
+                const int64_t kbase = ((int64_t)(inf.b * P.hkv + inf.g) * P.L + (int64_t)inf.c * kChunk) * D;
+                if constexpr (D == 128) {
+                    const int64_t krow = kbase + r;
 #pragma unroll kBEpiUnroll
-                for (int hk = 0; hk < 2; ++hk) {
-                    float v[32];
-                    tmem_ld32(lane_base + kColDK + hk * 32, v);
-                    tmem_wait_ld();
+                    for (int hk = 0; hk < 2; ++hk) {
+                        float v[32];
+                        tmem_ld32(lane_base + kColDK + hk * 32, v);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) atomicAdd(dk_acc + krow + (int64_t)(hk * 32 + i) * D, v[i] * scale);
-                    tmem_ld32(lane_base + kColDV + hk * 32, v);
-                    tmem_wait_ld();
+                        for (int i = 0; i < 32; ++i) atomicAdd(dk_acc + krow + (int64_t)(hk * 32 + i) * D, v[i] * scale);
+                        tmem_ld32(lane_base + kColDV + hk * 32, v);
+                        tmem_wait_ld();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) atomicAdd(dv_acc + krow + (int64_t)(hk * 32 + i) * D, v[i]);
+                        for (int i = 0; i < 32; ++i) atomicAdd(dv_acc + krow + (int64_t)(hk * 32 + i) * D, v[i]);
+                    }
+                } else {
+                    // d = 64: warps 0-1 hold dK^T (lanes 0-63 of its columns), warps 2-3 dV^T
+                    // (lanes 64-127 of its columns); lane r is column r mod 64 of d
+                    const bool isk = wq < 2;
+                    float *dst = (isk ? dk_acc : dv_acc) + kbase + (r & 63);
+                    const float sc = isk ? scale : 1.f;
+                    const uint32_t col = isk ? kColDK : kColDV;
+#pragma unroll kBEpiUnroll
+                    for (int hk = 0; hk < 2; ++hk) {
+                        float v[32];
+                        tmem_ld32(lane_base + col + hk * 32, v);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) atomicAdd(dst + (int64_t)(hk * 32 + i) * D, v[i] * sc);
+                    }
                 }
                 tc_fence_before();
                 __syncwarp();
@@ -745,13 +781,28 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
 }
 
 // ------------------------------------------------------------------ stick-breaking backward
-// One warp per (b, t, g), d = 128 (four columns per lane).  With the chunk
+// The D / 32 consecutive bf16 values of lane `lane` of a d = D row, as floats.
+template <int D>
+__device__ __forceinline__ void lane_cols(const __nv_bfloat16 *row, int lane, float (&f)[D / 32]) {
+    if constexpr (D == 128) {
+        const uint2 raw = *reinterpret_cast<const uint2 *>(row + lane * 4);
+        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
+        const float2 f0 = __bfloat1622float2(h2[0]), f1 = __bfloat1622float2(h2[1]);
+        f[0] = f0.x; f[1] = f0.y; f[2] = f1.x; f[3] = f1.y;
+    } else {
+        const float2 f0 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(row + lane * 2));
+        f[0] = f0.x; f[1] = f0.y;
+    }
+}
+
+// One warp per (b, t, g), d = D (D / 32 columns per lane).  With the chunk
 // weights' gradients dw from the attention pass, recompute the selected
 // chunks' scores s_j = q_slc . kbar_{c_j} / sqrt(d) and sig_j = sigmoid(s_j):
 //   ds_j   = dw_j w_j (1 - sig_j) - sig_j sum_{k>j} dw_k w_k
 //   dq_slc = sum_j ds_j kbar_{c_j} / sqrt(d),   dkbar_{c_j} += ds_j q_slc / sqrt(d)
 // Cited page: "Hardware-aligned Hierarchical Sparse Attention ..." §HSA
 // "end-to-end learning" (the chunk weight's gradient reaches the scores).
+template <int D>
 __global__ void __launch_bounds__(256) bwd_select_kernel(const __nv_bfloat16 *__restrict__ q_slc,
                                                          const int32_t *__restrict__ idx, const float *__restrict__ w,
                                                          float *dw_ds, const float *__restrict__ kbar,
@@ -764,15 +815,10 @@ __global__ void __launch_bounds__(256) bwd_select_kernel(const __nv_bfloat16 *__
     const int64_t bt = gw / hkv;  // b * L + t
     const int b = (int)(bt / L);
     const int64_t bg = (int64_t)b * hkv + g;
-    constexpr int D = kBD;
+    constexpr int NC = D / 32;  // columns per lane
     const float scale = 1.0f / sqrtf((float)D);
-    float qv[4];
-    {
-        const uint2 raw = *reinterpret_cast<const uint2 *>(q_slc + gw * D + lane * 4);
-        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-        const float2 f0 = __bfloat1622float2(h2[0]), f1 = __bfloat1622float2(h2[1]);
-        qv[0] = f0.x; qv[1] = f0.y; qv[2] = f1.x; qv[3] = f1.y;
-    }
+    float qv[NC];
+    lane_cols<D>(q_slc + gw * D, lane, qv);
     // lane k < K: the slot's chunk, weight, weight gradient and score; an index
     // that is not causally eligible is skipped (the inversion reports it)
     const int t = (int)(bt % L);
@@ -784,8 +830,10 @@ __global__ void __launch_bounds__(256) bwd_select_kernel(const __nv_bfloat16 *__
     for (int k = 0; k < K; ++k) {
         const int c = __shfl_sync(0xffffffffu, ck, k);
         if (c < 0) continue;  // an empty or ineligible slot: score and gradient stay 0
-        const float4 kb = *reinterpret_cast<const float4 *>(kbar + (bg * nc + c) * D + lane * 4);
-        float a = qv[0] * kb.x + qv[1] * kb.y + qv[2] * kb.z + qv[3] * kb.w;
+        const float *kr = kbar + (bg * nc + c) * D + lane * NC;
+        float a = 0.f;
+#pragma unroll
+        for (int e = 0; e < NC; ++e) a = fmaf(qv[e], kr[e], a);
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) a += __shfl_xor_sync(0xffffffffu, a, off);
         if (lane == k) sk = a * scale;
@@ -800,35 +848,42 @@ __global__ void __launch_bounds__(256) bwd_select_kernel(const __nv_bfloat16 *__
         if (lane + off < 32) incl += y;
     }
     const float dsk = (ck >= 0) ? prod * (1.f - sg) - sg * (incl - prod) : 0.f;
-    float dq4[4] = {0.f, 0.f, 0.f, 0.f};
+    float dqv[NC];
+#pragma unroll
+    for (int e = 0; e < NC; ++e) dqv[e] = 0.f;
     for (int k = 0; k < K; ++k) {
         const int c = __shfl_sync(0xffffffffu, ck, k);
         if (c < 0) continue;
         const float dsj = __shfl_sync(0xffffffffu, dsk, k) * scale;
-        const float4 kb = *reinterpret_cast<const float4 *>(kbar + (bg * nc + c) * D + lane * 4);
-        dq4[0] = fmaf(dsj, kb.x, dq4[0]); dq4[1] = fmaf(dsj, kb.y, dq4[1]);
-        dq4[2] = fmaf(dsj, kb.z, dq4[2]); dq4[3] = fmaf(dsj, kb.w, dq4[3]);
+        const float *kr = kbar + (bg * nc + c) * D + lane * NC;
+#pragma unroll
+        for (int e = 0; e < NC; ++e) dqv[e] = fmaf(dsj, kr[e], dqv[e]);
     }
     // the slot's score gradient (times 1/sqrt(d)) replaces its weight gradient in place (each
     // lane read its own entry above); bwd_dkbar_kernel sums it into the pooled-key gradient
     if (lane < K) dw_ds[gw * K + lane] = dsk * scale;
-    __nv_bfloat162 o0 = __floats2bfloat162_rn(dq4[0], dq4[1]), o1 = __floats2bfloat162_rn(dq4[2], dq4[3]);
-    uint2 pk;
-    pk.x = *reinterpret_cast<uint32_t *>(&o0);
-    pk.y = *reinterpret_cast<uint32_t *>(&o1);
-    *reinterpret_cast<uint2 *>(dq_slc + gw * D + lane * 4) = pk;
+    if constexpr (NC == 4) {
+        __nv_bfloat162 o0 = __floats2bfloat162_rn(dqv[0], dqv[1]), o1 = __floats2bfloat162_rn(dqv[2], dqv[3]);
+        uint2 pk;
+        pk.x = *reinterpret_cast<uint32_t *>(&o0);
+        pk.y = *reinterpret_cast<uint32_t *>(&o1);
+        *reinterpret_cast<uint2 *>(dq_slc + gw * D + lane * 4) = pk;
+    } else {
+        *reinterpret_cast<__nv_bfloat162 *>(dq_slc + gw * D + lane * 2) = __floats2bfloat162_rn(dqv[0], dqv[1]);
+    }
 }
 
 // Gradient of the pooled keys, chunk-major: dkbar[c] = sum over the (token, slot) entries
 // of chunk c's list of ds(token, slot) * q_slc[token].  One warp per list segment of
 // kBwdSeg entries (segment z of (b, g) belongs to the chunk c with seg_off[c] <= z <
-// seg_off[c+1]); a lane owns 4 of the 128 columns; one reduction per segment.
+// seg_off[c+1]); a lane owns D / 32 of the D columns; one reduction per segment.
+template <int D>
 __global__ void __launch_bounds__(256) bwd_dkbar_kernel(const __nv_bfloat16 *__restrict__ q_slc,
                                                         const float *__restrict__ ds, const int32_t *__restrict__ chunk_off,
                                                         const int32_t *__restrict__ seg_off,
                                                         const int32_t *__restrict__ entries, float *__restrict__ dkbar,
                                                         int L, int hkv, int nc, int K) {
-    constexpr int D = kBD;
+    constexpr int NC = D / 32;
     const int lane = threadIdx.x & 31;
     const int z = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int bg = blockIdx.y, b = bg / hkv, g = bg % hkv;
@@ -853,26 +908,35 @@ __global__ void __launch_bounds__(256) bwd_dkbar_kernel(const __nv_bfloat16 *__r
         qrow = row * D;
         dsv = ds[row * K + (ent & 15)];
     }
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+    float acc[NC];
+#pragma unroll
+    for (int e = 0; e < NC; ++e) acc[e] = 0.f;
     for (int i = 0; i < n; ++i) {
         const int64_t qr = __shfl_sync(0xffffffffu, qrow, i);
         const float d = __shfl_sync(0xffffffffu, dsv, i);
-        const uint2 raw = *reinterpret_cast<const uint2 *>(q_slc + qr + lane * 4);
-        const __nv_bfloat162 *h2 = reinterpret_cast<const __nv_bfloat162 *>(&raw);
-        const float2 f0 = __bfloat1622float2(h2[0]), f1 = __bfloat1622float2(h2[1]);
-        acc[0] = fmaf(d, f0.x, acc[0]); acc[1] = fmaf(d, f0.y, acc[1]);
-        acc[2] = fmaf(d, f1.x, acc[2]); acc[3] = fmaf(d, f1.y, acc[3]);
+        float f[NC];
+        lane_cols<D>(q_slc + qr, lane, f);
+#pragma unroll
+        for (int e = 0; e < NC; ++e) acc[e] = fmaf(d, f[e], acc[e]);
     }
-    red_add_v4_f32(dkbar + ((int64_t)bg * nc + c) * D + lane * 4, make_float4(acc[0], acc[1], acc[2], acc[3]));
+    float *dst = dkbar + ((int64_t)bg * nc + c) * D + lane * NC;
+    if constexpr (NC == 4) {
+        red_add_v4_f32(dst, make_float4(acc[0], acc[1], acc[2], acc[3]));
+    } else {
+        atomicAdd(dst, acc[0]);
+        atomicAdd(dst + 1, acc[1]);
+    }
 }
 
 // ------------------------------------------------------------------ magnitude bound
-// max over rows of the L2 norm of a row of d = 128 bf16 values, as float bits max-ed into
-// *bits.  A row is 16 lanes x 16 bytes; every thread keeps 4 rows' loads in flight.
+// max over rows of the L2 norm of a row of d = D bf16 values, as float bits max-ed into
+// *bits.  A row is D / 8 lanes x 16 bytes; every thread keeps 4 rows' loads in flight.
+template <int D>
 __global__ void __launch_bounds__(256) rownorm_max_kernel(const __nv_bfloat16 *__restrict__ x, int64_t rows,
                                                           int32_t *__restrict__ bits) {
     constexpr int kU = 4;
-    const int64_t nvec = rows * 16;  // 16-byte vectors
+    constexpr int LPR = D / 8;  // lanes per row
+    const int64_t nvec = rows * LPR;  // 16-byte vectors
     const int64_t stride = (int64_t)gridDim.x * blockDim.x;
     float m = 0.f;
     for (int64_t v0 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; v0 - (int64_t)(threadIdx.x & 31) < nvec;
@@ -893,7 +957,7 @@ __global__ void __launch_bounds__(256) rownorm_max_kernel(const __nv_bfloat16 *_
                 ss += f.x * f.x + f.y * f.y;
             }
 #pragma unroll
-            for (int off = 8; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);  // 16-lane row
+            for (int off = LPR / 2; off > 0; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);  // one row
             m = fmaxf(m, sqrtf(ss));
         }
     }
@@ -904,9 +968,12 @@ __global__ void __launch_bounds__(256) rownorm_max_kernel(const __nv_bfloat16 *_
 
 cudaError_t launch_rownorm_max(const void *x, int64_t rows, int d, int32_t *bits, cudaStream_t st) {
     if (rows == 0) return cudaSuccess;
-    if (d != kBD) return cudaErrorInvalidValue;
-    const int blocks = (int)std::min<int64_t>(ceil_div(rows * 16, 256 * 4), 148 * 8);
-    rownorm_max_kernel<<<blocks, 256, 0, st>>>((const __nv_bfloat16 *)x, rows, bits);
+    if (d != 64 && d != 128) return cudaErrorInvalidValue;
+    const int blocks = (int)std::min<int64_t>(ceil_div(rows * (d / 8), 256 * 4), 148 * 8);
+    if (d == 128)
+        rownorm_max_kernel<128><<<blocks, 256, 0, st>>>((const __nv_bfloat16 *)x, rows, bits);
+    else
+        rownorm_max_kernel<64><<<blocks, 256, 0, st>>>((const __nv_bfloat16 *)x, rows, bits);
     return cudaGetLastError();
 }
 
@@ -953,35 +1020,44 @@ bool b_map_q3(CUtensorMap *m, const void *base, uint64_t rows) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int G>
+template <int G, int D>
 cudaError_t launch_btc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv, const void *q, const void *k,
                        const void *v, const void *dO, const float *lse, float *dw, __half *acc, void *dq,
                        float *dk_acc, float *dv_acc, DevStatus *ds, cudaStream_t st) {
     CUtensorMap mq, mo, mk, mv;
-    if (!b_map_q3(&mq, q, (uint64_t)sh.B * sh.L * sh.hq) || !b_map_q3(&mo, dO, (uint64_t)sh.B * sh.L * sh.hq) ||
-        !b_map(&mk, k, kBD, (uint64_t)sh.B * sh.hkv * sh.L, 64) || !b_map(&mv, v, kBD, (uint64_t)sh.B * sh.hkv * sh.L, 64))
-        return cudaErrorInvalidValue;
-    const size_t smem = BSmem::ALLOC;
-    cudaError_t e = set_smem_once((const void *)bwd_tc_kernel<G>, smem);
+    const uint64_t qrows = (uint64_t)sh.B * sh.L * sh.hq, krows = (uint64_t)sh.B * sh.hkv * sh.L;
+    // query / output-gradient rows: d = 128, the 3D view (8 rows x both halves per box);
+    // d = 64, 2D boxes of 8 rows x 64 columns
+    const bool qok = (D == 128) ? (b_map_q3(&mq, q, qrows) && b_map_q3(&mo, dO, qrows))
+                                : (b_map(&mq, q, 64, qrows, 8) && b_map(&mo, dO, 64, qrows, 8));
+    if (!qok || !b_map(&mk, k, D, krows, 64) || !b_map(&mv, v, D, krows, 64)) return cudaErrorInvalidValue;
+    const size_t smem = BSmem<D>::ALLOC;
+    cudaError_t e = set_smem_once((const void *)bwd_tc_kernel<G, D>, smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 0;
     if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    bwd_tc_kernel<G><<<sms, kBThreads, smem, st>>>(mq, mo, mk, mv, plan, inv.entries, inv.entw, lse, dw, acc,
+    bwd_tc_kernel<G, D><<<sms, kBThreads, smem, st>>>(mq, mo, mk, mv, plan, inv.entries, inv.entw, lse, dw, acc,
                                                    (__nv_bfloat16 *)dq, dk_acc, dv_acc, ds, wait_limit_ns());
     return cudaGetLastError();
 }
 }  // namespace
 
 bool bwd_tc_supported(const Shape &sh) {
-    return sh.bf16 && sh.d == kBD && (sh.G == 8 || sh.G == 16) && sh.K <= 16 && b_encode() != nullptr;
+    return sh.bf16 && (sh.d == 64 || sh.d == 128) && (sh.G == 8 || sh.G == 16) && sh.K <= 16 &&
+           b_encode() != nullptr;
 }
 
 cudaError_t launch_bwd_tc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv, const void *q, const void *k,
                           const void *v, const void *dO, const float *lse, float *dw, __half *acc, void *dq,
                           float *dk_acc, float *dv_acc, DevStatus *ds, cudaStream_t st) {
-    if (sh.G == 8) return launch_btc<8>(sh, plan, inv, q, k, v, dO, lse, dw, acc, dq, dk_acc, dv_acc, ds, st);
-    if (sh.G == 16) return launch_btc<16>(sh, plan, inv, q, k, v, dO, lse, dw, acc, dq, dk_acc, dv_acc, ds, st);
+    if (sh.d == 128) {
+        if (sh.G == 8) return launch_btc<8, 128>(sh, plan, inv, q, k, v, dO, lse, dw, acc, dq, dk_acc, dv_acc, ds, st);
+        if (sh.G == 16) return launch_btc<16, 128>(sh, plan, inv, q, k, v, dO, lse, dw, acc, dq, dk_acc, dv_acc, ds, st);
+    } else if (sh.d == 64) {
+        if (sh.G == 8) return launch_btc<8, 64>(sh, plan, inv, q, k, v, dO, lse, dw, acc, dq, dk_acc, dv_acc, ds, st);
+        if (sh.G == 16) return launch_btc<16, 64>(sh, plan, inv, q, k, v, dO, lse, dw, acc, dq, dk_acc, dv_acc, ds, st);
+    }
     return cudaErrorInvalidValue;
 }
 
@@ -989,15 +1065,25 @@ cudaError_t launch_bwd_select(const Shape &sh, const void *q_slc, const int32_t 
                               const float *kbar, void *dq_slc, float *dkbar, const BwdWs &inv, cudaStream_t st) {
     const int64_t rows = (int64_t)sh.B * sh.L * sh.hkv;
     if (rows == 0) return cudaSuccess;
-    bwd_select_kernel<<<(unsigned)ceil_div(rows, 8), 256, 0, st>>>((const __nv_bfloat16 *)q_slc, idx, w, dw, kbar,
-                                                                   (__nv_bfloat16 *)dq_slc, rows, sh.L, sh.hkv,
-                                                                   std::max(sh.nc, 1), sh.K);
+    if (sh.d == 128)
+        bwd_select_kernel<128><<<(unsigned)ceil_div(rows, 8), 256, 0, st>>>(
+            (const __nv_bfloat16 *)q_slc, idx, w, dw, kbar, (__nv_bfloat16 *)dq_slc, rows, sh.L, sh.hkv,
+            std::max(sh.nc, 1), sh.K);
+    else
+        bwd_select_kernel<64><<<(unsigned)ceil_div(rows, 8), 256, 0, st>>>(
+            (const __nv_bfloat16 *)q_slc, idx, w, dw, kbar, (__nv_bfloat16 *)dq_slc, rows, sh.L, sh.hkv,
+            std::max(sh.nc, 1), sh.K);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess || sh.nc == 0) return e;
     // segments of kBwdSeg list entries: at most L*K/kBwdSeg + nc per (b, g); 8 per block
     const int64_t maxseg = ceil_div((int64_t)sh.L * sh.K, kBwdSeg) + sh.nc;
-    bwd_dkbar_kernel<<<dim3((unsigned)ceil_div(maxseg, 8), (unsigned)(sh.B * sh.hkv)), 256, 0, st>>>(
-        (const __nv_bfloat16 *)q_slc, dw, inv.chunk_off, inv.seg_off, inv.entries, dkbar, sh.L, sh.hkv, sh.nc, sh.K);
+    const dim3 grid((unsigned)ceil_div(maxseg, 8), (unsigned)(sh.B * sh.hkv));
+    if (sh.d == 128)
+        bwd_dkbar_kernel<128><<<grid, 256, 0, st>>>((const __nv_bfloat16 *)q_slc, dw, inv.chunk_off, inv.seg_off,
+                                                    inv.entries, dkbar, sh.L, sh.hkv, sh.nc, sh.K);
+    else
+        bwd_dkbar_kernel<64><<<grid, 256, 0, st>>>((const __nv_bfloat16 *)q_slc, dw, inv.chunk_off, inv.seg_off,
+                                                   inv.entries, dkbar, sh.L, sh.hkv, sh.nc, sh.K);
     return cudaGetLastError();
 }
 

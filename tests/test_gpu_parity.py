@@ -486,14 +486,18 @@ def test_bwd_small_full(wl):
         assert_out(f64(g), r, wl.dtype, name, grad=True)
 
 
-# chunk-major tensor-core backward: bf16, d = 128, G in {8, 16}
+# chunk-major tensor-core backward: bf16, d in {64, 128}, G in {8, 16}
 BWD_TC = [small(h_q=16, h_kv=1, K=4, L=64 * 45 + 3, B=1, kind="train"),
           small(h_q=16, h_kv=2, K=8, L=64 * 100 + 17, B=2, seed=9, kind="train"),
           small(h_q=16, h_kv=2, K=16, L=2048, kind="train"),
-          small(h_q=16, h_kv=2, K=1, L=777, B=3, kind="train")]
+          small(h_q=16, h_kv=2, K=1, L=777, B=3, kind="train"),
+          small(h_q=16, h_kv=1, d=64, K=4, L=64 * 45 + 3, B=1, seed=21, kind="train"),
+          small(h_q=16, h_kv=2, d=64, K=8, L=64 * 100 + 17, B=2, seed=22, kind="train"),
+          small(h_q=16, h_kv=2, d=64, K=16, L=2048, seed=23, kind="train")]
 
 
-@pytest.mark.parametrize("wl", BWD_TC, ids=["g16-ragged", "g8-multiwindow", "g8-k16", "g8-k1-b3"])
+@pytest.mark.parametrize("wl", BWD_TC, ids=["g16-ragged", "g8-multiwindow", "g8-k16", "g8-k1-b3",
+                                            "d64-g16-ragged", "d64-g8-b2", "d64-g8-k16"])
 def test_bwd_tensor_core_path_full(wl):
     x, kbar, sel = gap_ruled(wl)
     ref = oracle.bwd(x["q"], x["k"], x["v"], x["q_slc"], kbar, x["dO"], wl.S, wl.K)
@@ -507,13 +511,13 @@ def test_bwd_tensor_core_path_full(wl):
         assert_out(f64(g), r, "bf16", name, grad=True)
 
 
+@pytest.mark.parametrize("wl", [BWD_TC[0], BWD_TC[4]], ids=["d128", "d64"])
 @pytest.mark.parametrize("factor", [2.0 ** 12, 2.0 ** -12], ids=["dO-x4096", "dO-x1/4096"])
-def test_bwd_tensor_core_grad_scale(factor):
+def test_bwd_tensor_core_grad_scale(factor, wl):
     """The tensor-core backward sums dq in fp16 scaled by a power of two at or above a
     bound computed from max row norms of dO and v and max|k|.  Every gradient is
     linear in dO and scaling dO by a power of two is exact, so grads / factor must
     match the unscaled oracle at the same bar."""
-    wl = BWD_TC[0]
     x, kbar, sel = gap_ruled(wl)
     ref = oracle.bwd(x["q"], x["k"], x["v"], x["q_slc"], kbar, x["dO"], wl.S, wl.K)
     xs = dict(x)

@@ -26,7 +26,7 @@ hsa_status_t check_shape(const hsa_shape_t *s, bool decode) {
         return HSA_ERR_INVALID_ARG;
     if (s->h_q % s->h_kv != 0) return HSA_ERR_INVALID_ARG;
     if (s->dtype != HSA_F32 && s->dtype != HSA_BF16) return HSA_ERR_INVALID_ARG;
-    if (s->S != kChunk) return HSA_ERR_UNSUPPORTED;
+    if (s->S != 16 && s->S != 32 && s->S != 64 && s->S != 128) return HSA_ERR_UNSUPPORTED;
     if (s->d != 64 && s->d != 128) return HSA_ERR_UNSUPPORTED;
     if (s->K > kMaxK || s->h_q / s->h_kv > kMaxG) return HSA_ERR_UNSUPPORTED;
     // entries pack t * 16 + slot into int32; list offsets are int32

@@ -11,7 +11,8 @@
 
 namespace hsa {
 
-constexpr int kChunk = 64;     // S: the only chunk size built (fixed on the pages)
+constexpr int kChunk = 64;     // S of the tensor-core kernels (the pages' chunk size)
+constexpr int kMaxS = 128;     // chunk sizes 16, 32, 64 and 128 run on the CUDA-core kernels
 constexpr int kMaxK = 16;      // top-K bound
 constexpr int kMaxG = 16;      // query heads per KV group bound
 constexpr size_t kWsHeader = 256;

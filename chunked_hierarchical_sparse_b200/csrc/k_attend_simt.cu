@@ -16,26 +16,26 @@ namespace hsa {
 
 constexpr int kAttThreads = 128;
 
-// Shared-memory layout for one (token, group) block.
+// Shared-memory layout for one (token, group) block; S keys per chunk.
 struct AttSmem {
-    float *Ks;   // [64][d+1]
-    float *Vs;   // [64][d]
+    float *Ks;   // [S][d+1]
+    float *Vs;   // [S][d]
     float *Qs;   // [G][d]
-    float *P;    // [G][64]
+    float *P;    // [G][S]
     float *coef; // [G]
 };
 
-__host__ __device__ inline size_t att_smem_floats(int d, int G) {
-    return (size_t)kChunk * (d + 1) + (size_t)kChunk * d + (size_t)G * d + (size_t)G * kChunk + kMaxG;
+__host__ __device__ inline size_t att_smem_floats(int d, int G, int S) {
+    return (size_t)S * (d + 1) + (size_t)S * d + (size_t)G * d + (size_t)G * S + kMaxG;
 }
 
-__device__ inline AttSmem att_carve(float *sm, int d, int G) {
+__device__ inline AttSmem att_carve(float *sm, int d, int G, int S) {
     AttSmem s;
     s.Ks = sm;
-    s.Vs = s.Ks + kChunk * (d + 1);
-    s.Qs = s.Vs + kChunk * d;
+    s.Vs = s.Ks + S * (d + 1);
+    s.Qs = s.Vs + S * d;
     s.P = s.Qs + G * d;
-    s.coef = s.P + G * kChunk;
+    s.coef = s.P + G * S;
     return s;
 }
 
@@ -44,7 +44,7 @@ __device__ inline AttSmem att_carve(float *sm, int d, int G) {
 // o[h][j] for the thread's (h, j) pairs e = tid + 128 * i.
 // kv_base points at chunk 0 of this (b, g) in the [.., L, d] K/V layout.
 template <typename T, int MAXPER>
-__device__ void attend_group(const T *__restrict__ kbase, const T *__restrict__ vbase, int d, int G,
+__device__ void attend_group(const T *__restrict__ kbase, const T *__restrict__ vbase, int d, int G, int S,
                              int K, const int *slot_c, const float *slot_w, AttSmem s,
                              float (&oacc)[MAXPER], float *lse_out /* [G][K] or null, stride K */) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -58,16 +58,16 @@ __device__ void attend_group(const T *__restrict__ kbase, const T *__restrict__ 
         }
         const float wk = slot_w[kk];
         __syncthreads();
-        const T *kc = kbase + (int64_t)c * kChunk * d;
-        const T *vc = vbase + (int64_t)c * kChunk * d;
-        for (int e = tid; e < kChunk * d; e += kAttThreads) {
+        const T *kc = kbase + (int64_t)c * S * d;
+        const T *vc = vbase + (int64_t)c * S * d;
+        for (int e = tid; e < S * d; e += kAttThreads) {
             const int i = e / d, j = e % d;
             s.Ks[i * (d + 1) + j] = Elem<T>::load(kc + e);
             s.Vs[e] = Elem<T>::load(vc + e);
         }
         __syncthreads();
-        for (int e = tid; e < G * kChunk; e += kAttThreads) {
-            const int h = e / kChunk, i = e % kChunk;
+        for (int e = tid; e < G * S; e += kAttThreads) {
+            const int h = e / S, i = e % S;
             const float *qh = s.Qs + h * d;
             const float *ki = s.Ks + i * (d + 1);
             float acc = 0.f;
@@ -76,18 +76,31 @@ __device__ void attend_group(const T *__restrict__ kbase, const T *__restrict__ 
         }
         __syncthreads();
         // softmax-off-by-one per head: m = max(0, max x); Z = e^{-m} + sum e^{x-m}
+        // (lane takes keys lane, lane + 32, ...)
         for (int h = warp; h < G; h += kAttThreads / 32) {
-            float x0 = s.P[h * kChunk + lane], x1 = s.P[h * kChunk + lane + 32];
-            float m = fmaxf(0.f, fmaxf(x0, x1));
+            float xv[kMaxS / 32];
+            float m = 0.f;
+#pragma unroll
+            for (int u = 0; u < kMaxS / 32; ++u) {
+                const int i = lane + 32 * u;
+                xv[u] = (i < S) ? s.P[h * S + i] : -CUDART_INF_F;
+                m = fmaxf(m, xv[u]);
+            }
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
-            const float e0 = expf(x0 - m), e1 = expf(x1 - m);
-            float z = e0 + e1;
+            float z = 0.f;
+#pragma unroll
+            for (int u = 0; u < kMaxS / 32; ++u) {
+                const int i = lane + 32 * u;
+                if (i < S) {
+                    const float ev = expf(xv[u] - m);
+                    s.P[h * S + i] = ev;
+                    z += ev;
+                }
+            }
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
             z += expf(-m);
-            s.P[h * kChunk + lane] = e0;
-            s.P[h * kChunk + lane + 32] = e1;
             if (lane == 0) {
                 s.coef[h] = wk / z;
                 if (lse_out) lse_out[h * K + kk] = m + logf(z);
@@ -99,9 +112,9 @@ __device__ void attend_group(const T *__restrict__ kbase, const T *__restrict__ 
             const int e = tid + kAttThreads * i;
             if (e < G * d) {
                 const int h = e / d, j = e % d;
-                const float *ph = s.P + h * kChunk;
+                const float *ph = s.P + h * S;
                 float acc = 0.f;
-                for (int r = 0; r < kChunk; ++r) acc = fmaf(ph[r], s.Vs[r * d + j], acc);
+                for (int r = 0; r < S; ++r) acc = fmaf(ph[r], s.Vs[r * d + j], acc);
                 oacc[i] = fmaf(s.coef[h], acc, oacc[i]);
             }
         }
@@ -113,10 +126,10 @@ template <typename T, int MAXPER>
 __global__ void __launch_bounds__(kAttThreads) attend_simt_kernel(
     const T *__restrict__ q, const T *__restrict__ k, const T *__restrict__ v,
     const int32_t *__restrict__ idx, const float *__restrict__ w, T *__restrict__ o,
-    float *__restrict__ lse, int L, int hq, int hkv, int d, int nc, int K, int G, DevStatus *ds) {
+    float *__restrict__ lse, int L, int hq, int hkv, int d, int S, int nc, int K, int G, DevStatus *ds) {
     extern __shared__ float4 smem4[];
     float *sm = reinterpret_cast<float *>(smem4);
-    AttSmem s = att_carve(sm, d, G);
+    AttSmem s = att_carve(sm, d, G, S);
     __shared__ int slot_c[kMaxK];
     __shared__ float slot_w[kMaxK];
     const int t = blockIdx.x;
@@ -125,7 +138,7 @@ __global__ void __launch_bounds__(kAttThreads) attend_simt_kernel(
     const int64_t row = (int64_t)b * L + t;
     if (tid < K) {
         int c = idx[(row * hkv + g) * K + tid];
-        if (c >= 0 && (c >= nc || c >= t / kChunk)) {
+        if (c >= 0 && (c >= nc || c >= t / S)) {
             report(ds, HSA_ERR_DEVICE_CHECK, kKAttendSimt, (int)row, c);
             c = -1;
         }
@@ -140,7 +153,7 @@ __global__ void __launch_bounds__(kAttThreads) attend_simt_kernel(
     for (int i = 0; i < MAXPER; ++i) oacc[i] = 0.f;
     const T *kbase = k + (int64_t)bg * L * d;
     const T *vbase = v + (int64_t)bg * L * d;
-    attend_group<T, MAXPER>(kbase, vbase, d, G, K, slot_c, slot_w, s, oacc,
+    attend_group<T, MAXPER>(kbase, vbase, d, G, S, K, slot_c, slot_w, s, oacc,
                             lse ? lse + (row * hq + (int64_t)g * G) * K : nullptr);
 #pragma unroll
     for (int i = 0; i < MAXPER; ++i) {
@@ -154,7 +167,7 @@ static cudaError_t attend_dispatch(const Shape &sh, const void *q, const void *k
                                    const int32_t *idx, const float *w, void *o, float *lse,
                                    DevStatus *ds, cudaStream_t st) {
     dim3 grid((unsigned)sh.L, (unsigned)(sh.B * sh.hkv));
-    const size_t smem = att_smem_floats(sh.d, sh.G) * sizeof(float);
+    const size_t smem = att_smem_floats(sh.d, sh.G, sh.S) * sizeof(float);
     const int per = (int)ceil_div((int64_t)sh.G * sh.d, kAttThreads);
 #define HSA_ATT_CASE(N)                                                                          \
     if (per <= N) {                                                                              \
@@ -162,7 +175,7 @@ static cudaError_t attend_dispatch(const Shape &sh, const void *q, const void *k
         if (e != cudaSuccess) return e;                                                          \
         attend_simt_kernel<T, N><<<grid, kAttThreads, smem, st>>>(                               \
             (const T *)q, (const T *)k, (const T *)v, idx, w, (T *)o, lse, sh.L, sh.hq, sh.hkv,  \
-            sh.d, sh.nc, sh.K, sh.G, ds);                                                        \
+            sh.d, sh.S, sh.nc, sh.K, sh.G, ds);                                                  \
         return cudaGetLastError();                                                               \
     }
     HSA_ATT_CASE(2)
@@ -189,11 +202,11 @@ template <typename T, int MAXPER>
 __global__ void __launch_bounds__(kAttThreads) decode_simt_kernel(
     const T *__restrict__ q, const T *__restrict__ q_slc, const T *__restrict__ kc,
     const T *__restrict__ vc, const float *__restrict__ kbar, T *__restrict__ o,
-    int32_t *__restrict__ idx_out, float *__restrict__ w_out, int P, int hq, int hkv, int d, int nc,
+    int32_t *__restrict__ idx_out, float *__restrict__ w_out, int P, int hq, int hkv, int d, int S, int nc,
     int K, int G) {
     extern __shared__ float4 smem4[];
     float *sm = reinterpret_cast<float *>(smem4);
-    AttSmem s = att_carve(sm, d, G);
+    AttSmem s = att_carve(sm, d, G, S);
     float *scores = s.coef + kMaxG;  // [nc]
     float *qs = scores + nc;         // [d]
     __shared__ int slot_c[kMaxK];
@@ -236,7 +249,7 @@ __global__ void __launch_bounds__(kAttThreads) decode_simt_kernel(
     float oacc[MAXPER];
 #pragma unroll
     for (int i = 0; i < MAXPER; ++i) oacc[i] = 0.f;
-    attend_group<T, MAXPER>(kc + (int64_t)bg * P * d, vc + (int64_t)bg * P * d, d, G, K, slot_c,
+    attend_group<T, MAXPER>(kc + (int64_t)bg * P * d, vc + (int64_t)bg * P * d, d, G, S, K, slot_c,
                             slot_w, s, oacc, nullptr);
 #pragma unroll
     for (int i = 0; i < MAXPER; ++i) {
@@ -249,7 +262,7 @@ template <typename T>
 static cudaError_t decode_dispatch(const Shape &sh, const void *q, const void *q_slc, const void *kc,
                                    const void *vc, const float *kbar, void *o, int32_t *idx_out,
                                    float *w_out, cudaStream_t st) {
-    const size_t smem = (att_smem_floats(sh.d, sh.G) + (size_t)sh.nc + sh.d) * sizeof(float);
+    const size_t smem = (att_smem_floats(sh.d, sh.G, sh.S) + (size_t)sh.nc + sh.d) * sizeof(float);
     const int per = (int)ceil_div((int64_t)sh.G * sh.d, kAttThreads);
 #define HSA_DEC_CASE(N)                                                                           \
     if (per <= N) {                                                                               \
@@ -257,7 +270,7 @@ static cudaError_t decode_dispatch(const Shape &sh, const void *q, const void *q
         if (e != cudaSuccess) return e;                                                           \
         decode_simt_kernel<T, N><<<(unsigned)(sh.B * sh.hkv), kAttThreads, smem, st>>>(           \
             (const T *)q, (const T *)q_slc, (const T *)kc, (const T *)vc, kbar, (T *)o, idx_out,   \
-            w_out, sh.L, sh.hq, sh.hkv, sh.d, sh.nc, sh.K, sh.G);                                 \
+            w_out, sh.L, sh.hq, sh.hkv, sh.d, sh.S, sh.nc, sh.K, sh.G);                           \
         return cudaGetLastError();                                                                \
     }
     HSA_DEC_CASE(2)

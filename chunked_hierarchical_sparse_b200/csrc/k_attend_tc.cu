@@ -852,8 +852,8 @@ cudaError_t launch_wsum(const Shape &sh, const int32_t *idx, const float *w, int
 }
 
 bool attend_tc_supported(const Shape &sh) {
-    return sh.bf16 && (sh.d == 64 || sh.d == 128) && (sh.G == 8 || sh.G == 16) && sh.K <= 16 &&
-           get_encode() != nullptr;
+    return sh.bf16 && sh.S == kChunk && (sh.d == 64 || sh.d == 128) && (sh.G == 8 || sh.G == 16) &&
+           sh.K <= 16 && get_encode() != nullptr;
 }
 
 cudaError_t launch_attend_tc(const Shape &sh, const AttendPlan &plan, const int32_t *entries, const float *entw,

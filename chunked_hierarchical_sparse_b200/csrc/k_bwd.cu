@@ -32,16 +32,16 @@ __global__ void __launch_bounds__(kB1Threads) bwd_phase1_kernel(
     const T *__restrict__ v, const T *__restrict__ dO, const float *__restrict__ lse,
     const int32_t *__restrict__ idx, const float *__restrict__ w, const float *__restrict__ kbar,
     T *__restrict__ dq, T *__restrict__ dq_slc, float *__restrict__ dkbar, float *__restrict__ delta,
-    int L, int hq, int hkv, int d, int nc, int K, int G, DevStatus *ds) {
+    int L, int hq, int hkv, int d, int S, int nc, int K, int G, DevStatus *ds) {
     extern __shared__ float4 smem4[];
     float *sm = reinterpret_cast<float *>(smem4);
-    float *Ks = sm;                        // [64][d+1]
-    float *Vs = Ks + kChunk * (d + 1);     // [64][d+1]
-    float *Qs = Vs + kChunk * (d + 1);     // [G][d]
+    float *Ks = sm;                        // [S][d+1]
+    float *Vs = Ks + S * (d + 1);          // [S][d+1]
+    float *Qs = Vs + S * (d + 1);          // [G][d]
     float *dOs = Qs + G * d;               // [G][d]
-    float *Pm = dOs + G * d;               // [G][64]
-    float *dPm = Pm + G * kChunk;          // [G][64]
-    float *Dl = dPm + G * kChunk;          // [G]
+    float *Pm = dOs + G * d;               // [G][S]
+    float *dPm = Pm + G * S;               // [G][S]
+    float *Dl = dPm + G * S;               // [G]
     __shared__ int slot_c[kMaxK];
     __shared__ float slot_w[kMaxK];
     __shared__ float dw_s[kMaxK];
@@ -53,7 +53,7 @@ __global__ void __launch_bounds__(kB1Threads) bwd_phase1_kernel(
     const float scale = 1.0f / sqrtf((float)d);
     if (tid < K) {
         int c = idx[(row * hkv + g) * K + tid];
-        if (c >= 0 && (c >= nc || c >= t / kChunk)) {
+        if (c >= 0 && (c >= nc || c >= t / S)) {
             report(ds, HSA_ERR_DEVICE_CHECK, kKBwd1, (int)row, c);
             c = -1;
         }
@@ -79,14 +79,14 @@ __global__ void __launch_bounds__(kB1Threads) bwd_phase1_kernel(
         }
         const float wk = slot_w[kk];
         __syncthreads();
-        for (int e = tid; e < kChunk * d; e += kB1Threads) {
+        for (int e = tid; e < S * d; e += kB1Threads) {
             const int i = e / d, j = e % d;
-            Ks[i * (d + 1) + j] = Elem<T>::load(kb + (int64_t)c * kChunk * d + e);
-            Vs[i * (d + 1) + j] = Elem<T>::load(vb + (int64_t)c * kChunk * d + e);
+            Ks[i * (d + 1) + j] = Elem<T>::load(kb + (int64_t)c * S * d + e);
+            Vs[i * (d + 1) + j] = Elem<T>::load(vb + (int64_t)c * S * d + e);
         }
         __syncthreads();
-        for (int e = tid; e < G * kChunk; e += kB1Threads) {
-            const int h = e / kChunk, i = e % kChunk;
+        for (int e = tid; e < G * S; e += kB1Threads) {
+            const int h = e / S, i = e % S;
             float ax = 0.f, ap = 0.f;
             for (int j = 0; j < d; ++j) {
                 ax = fmaf(Qs[h * d + j], Ks[i * (d + 1) + j], ax);
@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(kB1Threads) bwd_phase1_kernel(
             float acc = 0.f;
             for (int j = lane; j < d; j += 32) {
                 float o = 0.f;
-                for (int i = 0; i < kChunk; ++i) o = fmaf(Pm[h * kChunk + i], Vs[i * (d + 1) + j], o);
+                for (int i = 0; i < S; ++i) o = fmaf(Pm[h * S + i], Vs[i * (d + 1) + j], o);
                 acc = fmaf(dOs[h * d + j], o, acc);
             }
 #pragma unroll
@@ -118,8 +118,8 @@ __global__ void __launch_bounds__(kB1Threads) bwd_phase1_kernel(
             for (int h = 0; h < G; ++h) sdl += Dl[h];
             dw_s[kk] = sdl;
         }
-        for (int e = tid; e < G * kChunk; e += kB1Threads) {
-            const int h = e / kChunk;
+        for (int e = tid; e < G * S; e += kB1Threads) {
+            const int h = e / S;
             dPm[e] = wk * Pm[e] * (dPm[e] - Dl[h]);  // dx
         }
         __syncthreads();
@@ -129,7 +129,7 @@ __global__ void __launch_bounds__(kB1Threads) bwd_phase1_kernel(
             if (e < G * d) {
                 const int h = e / d, j = e % d;
                 float acc = 0.f;
-                for (int r = 0; r < kChunk; ++r) acc = fmaf(dPm[h * kChunk + r], Ks[r * (d + 1) + j], acc);
+                for (int r = 0; r < S; ++r) acc = fmaf(dPm[h * S + r], Ks[r * (d + 1) + j], acc);
                 dqa[i] = fmaf(acc, scale, dqa[i]);
             }
         }
@@ -189,8 +189,8 @@ static cudaError_t phase1_dispatch(const Shape &sh, const void *q, const void *q
                                    const int32_t *idx, const float *w, const float *kbar, void *dq,
                                    void *dq_slc, const BwdWs &ws, DevStatus *ds, cudaStream_t st) {
     dim3 grid((unsigned)sh.L, (unsigned)(sh.B * sh.hkv));
-    const size_t smem = sizeof(float) * ((size_t)2 * kChunk * (sh.d + 1) + (size_t)2 * sh.G * sh.d +
-                                         (size_t)2 * sh.G * kChunk + kMaxG);
+    const size_t smem = sizeof(float) * ((size_t)2 * sh.S * (sh.d + 1) + (size_t)2 * sh.G * sh.d +
+                                         (size_t)2 * sh.G * sh.S + kMaxG);
     const int per = (int)ceil_div((int64_t)sh.G * sh.d, kB1Threads);
 #define HSA_B1_CASE(N)                                                                            \
     if (per <= N) {                                                                               \
@@ -198,8 +198,8 @@ static cudaError_t phase1_dispatch(const Shape &sh, const void *q, const void *q
         if (e != cudaSuccess) return e;                                                           \
         bwd_phase1_kernel<T, N><<<grid, kB1Threads, smem, st>>>(                                  \
             (const T *)q, (const T *)q_slc, (const T *)k, (const T *)v, (const T *)dO, lse, idx, w, \
-            kbar, (T *)dq, (T *)dq_slc, ws.dkbar, ws.delta, sh.L, sh.hq, sh.hkv, sh.d, sh.nc, sh.K, \
-            sh.G, ds);                                                                            \
+            kbar, (T *)dq, (T *)dq_slc, ws.dkbar, ws.delta, sh.L, sh.hq, sh.hkv, sh.d, sh.S, sh.nc, \
+            sh.K, sh.G, ds);                                                                      \
         return cudaGetLastError();                                                                \
     }
     HSA_B1_CASE(2)
@@ -224,11 +224,12 @@ cudaError_t launch_bwd_phase1(const Shape &sh, const void *q, const void *q_slc,
 // ------------------------------------------------------------------ phase 2
 // Grid (segment, b*hkv): segment z of (b, g) belongs to the chunk c with
 // seg_off[c] <= z < seg_off[c+1] and covers list entries
-// [off_c + (z - seg_off[c])*SEG, ... + SEG).  256 threads: key row i = tid/4, column
-// quarter jq = tid%4; the thread keeps its quarter of k_i, v_i and of the
-// dk_i, dv_i accumulators in registers.  Partial sums are added into fp32
+// [off_c + (z - seg_off[c])*SEG, ... + SEG).  A block takes min(S, 64) keys of the chunk
+// (blockIdx.z picks the 64-key half of a 128-key chunk), four threads per key: key row
+// i = tid/4, column quarter jq = tid%4; the thread keeps its quarter of k_i, v_i and of
+// the dk_i, dv_i accumulators in registers.  Partial sums are added into fp32
 // accumulators; a finishing kernel adds dkbar/S and rounds.
-constexpr int kB2Threads = 256;
+constexpr int kB2Threads = 256;  // the most threads a block takes (64 keys, 4 per key)
 constexpr int kB2Seg = kBwdSeg;
 
 template <typename T, int DQ>
@@ -237,7 +238,7 @@ __global__ void __launch_bounds__(kB2Threads) bwd_phase2_kernel(
     const float *__restrict__ lse, const float *__restrict__ w, const float *__restrict__ delta,
     const int32_t *__restrict__ chunk_off, const int32_t *__restrict__ seg_off,
     const int32_t *__restrict__ entries, float *__restrict__ dk_acc, float *__restrict__ dv_acc,
-    int L, int hq, int hkv, int nc, int K, int G) {
+    int L, int hq, int hkv, int S, int nc, int K, int G) {
     constexpr int d = DQ * 4;
     __shared__ float qs[d], dos[d];
     const int z = blockIdx.x, bg = blockIdx.y, b = bg / hkv, g = bg % hkv;
@@ -253,9 +254,9 @@ __global__ void __launch_bounds__(kB2Threads) bwd_phase2_kernel(
     const int beg = off[c] + (z - so[c]) * kB2Seg;
     const int end = min(off[c + 1], beg + kB2Seg);
     if (beg >= end) return;
-    const int tid = threadIdx.x, i = tid >> 2, jq = tid & 3;
+    const int tid = threadIdx.x, i = (tid >> 2) + 64 * (int)blockIdx.z, jq = tid & 3;
     const float scale = 1.0f / sqrtf((float)d);
-    const int64_t krow = ((int64_t)bg * L + (int64_t)c * kChunk + i) * d + jq * DQ;
+    const int64_t krow = ((int64_t)bg * L + (int64_t)c * S + i) * d + jq * DQ;
     float kr[DQ], vr[DQ], dka[DQ], dva[DQ];
 #pragma unroll
     for (int e = 0; e < DQ; ++e) {
@@ -272,7 +273,7 @@ __global__ void __launch_bounds__(kB2Threads) bwd_phase2_kernel(
         const float wk = w[(row * hkv + g) * K + kk];
         for (int h = g * G; h < (g + 1) * G; ++h) {
             __syncthreads();
-            for (int j = tid; j < d; j += kB2Threads) {
+            for (int j = tid; j < d; j += blockDim.x) {
                 qs[j] = Elem<T>::load(q + (row * hq + h) * d + j);
                 dos[j] = Elem<T>::load(dO + (row * hq + h) * d + j);
             }
@@ -308,17 +309,17 @@ __global__ void __launch_bounds__(kB2Threads) bwd_phase2_kernel(
 template <typename T>
 __global__ void bwd_finish_kernel(const float *__restrict__ dk_acc, const float *__restrict__ dv_acc,
                                   const float *__restrict__ dkbar, T *__restrict__ dk, T *__restrict__ dv,
-                                  int L, int d, int nc, int64_t total) {
+                                  int L, int d, int S, int nc, int64_t total) {
     for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
          e += (int64_t)gridDim.x * blockDim.x) {
         const int j = (int)(e % d);
         const int64_t r = e / d;
         const int t = (int)(r % L);
         const int64_t bg = r / L;
-        const int c = t / kChunk;
+        const int c = t / S;
         float a = 0.f, bv = 0.f;
         if (c < nc) {
-            a = dk_acc[e] + dkbar[(bg * nc + c) * d + j] / kChunk;
+            a = dk_acc[e] + dkbar[(bg * nc + c) * d + j] / S;
             bv = dv_acc[e];
         }
         Elem<T>::store(dk + e, a);
@@ -334,22 +335,23 @@ static cudaError_t phase2_dispatch(const Shape &sh, const void *q, const void *k
     if (sh.nc > 0) {
         // a (b, g) has at most L*K/SEG + nc segments
         const int maxseg = (int)(ceil_div((int64_t)sh.L * sh.K, kB2Seg) + sh.nc);
-        dim3 grid(maxseg, sh.B * sh.hkv);
+        dim3 grid(maxseg, sh.B * sh.hkv, sh.S > 64 ? sh.S / 64 : 1);
+        const unsigned nthr = 4 * (unsigned)std::min(sh.S, 64);  // one thread per (key, column quarter)
         if (sh.d == 128)
-            bwd_phase2_kernel<T, 32><<<grid, kB2Threads, 0, st>>>(
+            bwd_phase2_kernel<T, 32><<<grid, nthr, 0, st>>>(
                 (const T *)q, (const T *)k, (const T *)v, (const T *)dO, lse, w, ws.delta, ws.chunk_off,
-                ws.seg_off, ws.entries, ws.dk_acc, ws.dv_acc, sh.L, sh.hq, sh.hkv, sh.nc, sh.K, sh.G);
+                ws.seg_off, ws.entries, ws.dk_acc, ws.dv_acc, sh.L, sh.hq, sh.hkv, sh.S, sh.nc, sh.K, sh.G);
         else
-            bwd_phase2_kernel<T, 16><<<grid, kB2Threads, 0, st>>>(
+            bwd_phase2_kernel<T, 16><<<grid, nthr, 0, st>>>(
                 (const T *)q, (const T *)k, (const T *)v, (const T *)dO, lse, w, ws.delta, ws.chunk_off,
-                ws.seg_off, ws.entries, ws.dk_acc, ws.dv_acc, sh.L, sh.hq, sh.hkv, sh.nc, sh.K, sh.G);
+                ws.seg_off, ws.entries, ws.dk_acc, ws.dv_acc, sh.L, sh.hq, sh.hkv, sh.S, sh.nc, sh.K, sh.G);
         cudaError_t e = cudaGetLastError();
         if (e != cudaSuccess) return e;
     }
     const int64_t total = (int64_t)sh.B * sh.hkv * sh.L * sh.d;
     const int blocks = (int)std::min<int64_t>(ceil_div(total, 256), 148 * 16);
     bwd_finish_kernel<T><<<blocks, 256, 0, st>>>(ws.dk_acc, ws.dv_acc, ws.dkbar, (T *)dk, (T *)dv,
-                                                  sh.L, sh.d, sh.nc, total);
+                                                  sh.L, sh.d, sh.S, sh.nc, total);
     return cudaGetLastError();
 }
 
@@ -359,7 +361,7 @@ static cudaError_t finish_dispatch(const Shape &sh, const BwdWs &ws, void *dk, v
     if (total == 0) return cudaSuccess;
     const int blocks = (int)std::min<int64_t>(ceil_div(total, 256), 148 * 16);
     bwd_finish_kernel<T><<<blocks, 256, 0, st>>>(ws.dk_acc, ws.dv_acc, ws.dkbar, (T *)dk, (T *)dv, sh.L, sh.d,
-                                                  sh.nc, total);
+                                                  sh.S, sh.nc, total);
     return cudaGetLastError();
 }
 

@@ -1044,8 +1044,8 @@ cudaError_t launch_btc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv
 }  // namespace
 
 bool bwd_tc_supported(const Shape &sh) {
-    return sh.bf16 && (sh.d == 64 || sh.d == 128) && (sh.G == 8 || sh.G == 16) && sh.K <= 16 &&
-           b_encode() != nullptr;
+    return sh.bf16 && sh.S == kChunk && (sh.d == 64 || sh.d == 128) && (sh.G == 8 || sh.G == 16) &&
+           sh.K <= 16 && b_encode() != nullptr;
 }
 
 cudaError_t launch_bwd_tc(const Shape &sh, const AttendPlan &plan, const BwdWs &inv, const void *q, const void *k,

@@ -580,7 +580,7 @@ static cudaError_t decode_launch(const Shape &sh, int NL, const void *q, const v
 }
 
 bool decode_cluster_supported(const Shape &sh, int NL) {
-    return (sh.d == 64 || sh.d == 128) && sh.G <= kMaxG && sh.K <= kMaxK && NL >= 1 &&
+    return sh.S == kChunk && (sh.d == 64 || sh.d == 128) && sh.G <= kMaxG && sh.K <= kMaxK && NL >= 1 &&
            decode_cluster_smem(sh.nc, sh.d, NL, sh.G) <= 200 * 1024;
 }
 

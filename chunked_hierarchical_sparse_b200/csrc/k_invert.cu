@@ -18,7 +18,7 @@ namespace hsa {
 
 __global__ void __launch_bounds__(256) inv_hist_kernel(const int32_t *__restrict__ idx,
                                                        int32_t *__restrict__ hist, int L, int hkv,
-                                                       int nc, int K, int ntb, DevStatus *ds) {
+                                                       int nc, int K, int S, int ntb, DevStatus *ds) {
     extern __shared__ int h_s[];
     const int tb = blockIdx.x, bg = blockIdx.y, b = bg / hkv, g = bg % hkv;
     for (int c = threadIdx.x; c < nc; c += blockDim.x) h_s[c] = 0;
@@ -29,7 +29,7 @@ __global__ void __launch_bounds__(256) inv_hist_kernel(const int32_t *__restrict
         if (t >= L) break;
         const int c = idx[(((int64_t)b * L + t) * hkv + g) * K + kk];
         if (c < 0) continue;
-        if (c >= nc || c >= t / kChunk) {
+        if (c >= nc || c >= t / S) {
             report(ds, HSA_ERR_DEVICE_CHECK, kKInvert, t, c);
             continue;
         }
@@ -141,7 +141,7 @@ __global__ void __launch_bounds__(32) inv_scatter_kernel(const int32_t *__restri
                                                          const int32_t *__restrict__ chunk_off,
                                                          int32_t *__restrict__ entries,
                                                          float *__restrict__ entw, int L,
-                                                         int hkv, int nc, int K, int ntb) {
+                                                         int hkv, int nc, int K, int S, int ntb) {
     extern __shared__ int cur[];  // [nc] cursors, [kInvTokBlock * K] the block's selections and weights
     int *sel = cur + nc;
     float *selw = reinterpret_cast<float *>(sel + kInvTokBlock * K);
@@ -168,7 +168,7 @@ __global__ void __launch_bounds__(32) inv_scatter_kernel(const int32_t *__restri
         const int t = tb + lane / K, kk = lane % K;
         int c = -1;
         if (lane < tpi * K && t < t1) c = sel[(t - t0) * K + kk];
-        const bool ok = c >= 0 && c < nc && c < t / kChunk;
+        const bool ok = c >= 0 && c < nc && c < t / S;
         const unsigned peers = __match_any_sync(0xffffffffu, ok ? c : -1 - lane);
         if (ok) {
             const int pos = cur[c] + __popc(peers & ((1u << lane) - 1u));
@@ -197,7 +197,7 @@ cudaError_t launch_invert(const Shape &sh, const int32_t *idx, const float *w, c
         if (e != cudaSuccess) return e;
     }
     dim3 grid(ntb, sh.B * sh.hkv);
-    inv_hist_kernel<<<grid, 256, smem, st>>>(idx, ws.hist, sh.L, sh.hkv, sh.nc, sh.K, ntb, ds);
+    inv_hist_kernel<<<grid, 256, smem, st>>>(idx, ws.hist, sh.L, sh.hkv, sh.nc, sh.K, sh.S, ntb, ds);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     inv_colscan_kernel<<<dim3((unsigned)ceil_div(sh.nc, 32), sh.B * sh.hkv), dim3(32, 32), 0, st>>>(
         ws.hist, ws.chunk_off, sh.nc, ntb);
@@ -205,7 +205,7 @@ cudaError_t launch_invert(const Shape &sh, const int32_t *idx, const float *w, c
     inv_scan_kernel<<<sh.B * sh.hkv, 1024, 2 * smem, st>>>(ws.chunk_off, ws.seg_off, sh.nc, kBwdSeg);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     inv_scatter_kernel<<<grid, 32, ssmem, st>>>(idx, w, ws.hist, ws.chunk_off, ws.entries, w ? ws.entw : nullptr,
-                                                 sh.L, sh.hkv, sh.nc, sh.K, ntb);
+                                                 sh.L, sh.hkv, sh.nc, sh.K, sh.S, ntb);
     return cudaGetLastError();
 }
 

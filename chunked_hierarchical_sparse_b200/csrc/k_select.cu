@@ -27,7 +27,8 @@ namespace hsa {
 // accumulators, which only ever sum values of complete chunks.
 template <typename T>
 __global__ void __launch_bounds__(128, 4) pool_kernel(const T *__restrict__ k, float *__restrict__ kbar,
-                                                   int L, int d, int nc, int64_t nchunks, PoolExtras x) {
+                                                   int L, int d, int S, int nc, int64_t nchunks,
+                                                   PoolExtras x) {
     constexpr int VEC = 16 / sizeof(T);
     constexpr int NB = 8;  // rows in flight per lane and tensor (4 blocks per SM stay resident)
     const int lane = threadIdx.x & 31;
@@ -36,10 +37,10 @@ __global__ void __launch_bounds__(128, 4) pool_kernel(const T *__restrict__ k, f
     const int tpc = d / VEC;      // lanes per row (8, 16 or 32)
     const int rs = 32 / tpc;      // row parts
     const int lr = lane % tpc, part = lane / tpc;
-    const int rows = kChunk / rs;  // 16, 32 or 64: a multiple of NB
+    const int rows = S / rs;       // rows of the chunk per row part
     const int c = (int)(bgc % nc);
     const int64_t bg = bgc / nc;
-    const int64_t off = ((bg * L + (int64_t)c * kChunk + (int64_t)part * rows) * d) + lr * VEC;
+    const int64_t off = ((bg * L + (int64_t)c * S + (int64_t)part * rows) * d) + lr * VEC;
     const T *src = k + off;
     double acc[VEC];
 #pragma unroll
@@ -48,12 +49,17 @@ __global__ void __launch_bounds__(128, 4) pool_kernel(const T *__restrict__ k, f
     float m = 0.f;
     for (int r0 = 0; r0 < rows; r0 += NB) {
         // the round's key rows and value rows are all in flight together
+        // a part shorter than NB rows (S = 16 with 4 row parts) loads zeros past its end
         uint4 raw[NB], rv[NB];
 #pragma unroll
-        for (int u = 0; u < NB; ++u) raw[u] = __ldcs(reinterpret_cast<const uint4 *>(src + (int64_t)(r0 + u) * d));
+        for (int u = 0; u < NB; ++u)
+            raw[u] = (r0 + u < rows) ? __ldcs(reinterpret_cast<const uint4 *>(src + (int64_t)(r0 + u) * d))
+                                     : make_uint4(0, 0, 0, 0);
         if (vsrc) {
 #pragma unroll
-            for (int u = 0; u < NB; ++u) rv[u] = __ldcs(reinterpret_cast<const uint4 *>(vsrc + (int64_t)(r0 + u) * d));
+            for (int u = 0; u < NB; ++u)
+                rv[u] = (r0 + u < rows) ? __ldcs(reinterpret_cast<const uint4 *>(vsrc + (int64_t)(r0 + u) * d))
+                                        : make_uint4(0, 0, 0, 0);
         }
 #pragma unroll
         for (int u = 0; u < NB; ++u) {
@@ -81,7 +87,7 @@ __global__ void __launch_bounds__(128, 4) pool_kernel(const T *__restrict__ k, f
     if (part == 0) {
         float out[VEC];
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) out[e] = (float)(acc[e] / kChunk);
+        for (int e = 0; e < VEC; ++e) out[e] = (float)(acc[e] / S);
         float4 *dst = reinterpret_cast<float4 *>(kbar + bgc * d + lr * VEC);
 #pragma unroll
         for (int e = 0; e < VEC / 4; ++e) dst[e] = make_float4(out[4 * e], out[4 * e + 1], out[4 * e + 2], out[4 * e + 3]);
@@ -108,9 +114,10 @@ cudaError_t launch_pool(const Shape &sh, const void *k, float *kbar, DevStatus *
     if (chunks == 0) return cudaSuccess;
     const unsigned blocks = (unsigned)ceil_div(chunks, 4);  // 4 warps = 4 chunks per block
     if (sh.bf16)
-        pool_kernel<__nv_bfloat16><<<blocks, 128, 0, st>>>((const __nv_bfloat16 *)k, kbar, sh.L, sh.d, sh.nc, chunks, x);
+        pool_kernel<__nv_bfloat16><<<blocks, 128, 0, st>>>((const __nv_bfloat16 *)k, kbar, sh.L, sh.d, sh.S, sh.nc,
+                                                            chunks, x);
     else
-        pool_kernel<float><<<blocks, 128, 0, st>>>((const float *)k, kbar, sh.L, sh.d, sh.nc, chunks,
+        pool_kernel<float><<<blocks, 128, 0, st>>>((const float *)k, kbar, sh.L, sh.d, sh.S, sh.nc, chunks,
                                                    PoolExtras{});  // split and max|v| serve bf16 paths only
     return cudaGetLastError();
 }
@@ -125,7 +132,7 @@ constexpr int kSelCh = 64;
 template <typename T>
 __global__ void __launch_bounds__(256) select_simt_kernel(
     const T *__restrict__ q_slc, const float *__restrict__ kbar, int32_t *__restrict__ idx,
-    float *__restrict__ w, int L, int hkv, int d, int nc, int K) {
+    float *__restrict__ w, int L, int hkv, int d, int S, int nc, int K) {
     extern __shared__ float4 smem4[];
     float *sm = reinterpret_cast<float *>(smem4);
     float *qT = sm;                                 // [d][64]
@@ -149,7 +156,7 @@ __global__ void __launch_bounds__(256) select_simt_kernel(
         best_c[e] = -1;
     }
     const int tlast = min(t0 + kSelTok, L) - 1;
-    const int ne_max = min(tlast / kChunk, nc);
+    const int ne_max = min(tlast / S, nc);
     const int ty = tid / 16, tx = tid % 16;
     const float *kb = kbar + (int64_t)bg * nc * d;
 
@@ -183,7 +190,7 @@ __global__ void __launch_bounds__(256) select_simt_kernel(
         for (int tt = warp * 8; tt < warp * 8 + 8; ++tt) {
             const int t = t0 + tt;
             if (t >= L) break;
-            const int ne = min(t / kChunk, nc);
+            const int ne = min(t / S, nc);
             const int ca = c0 + lane, cb = c0 + lane + 32;
             const float sa = sc[tt * (kSelCh + 1) + lane];
             const float sb = sc[tt * (kSelCh + 1) + lane + 32];
@@ -227,12 +234,12 @@ cudaError_t launch_select_simt(const Shape &sh, const void *q_slc, const float *
         e = set_smem_once((const void *)select_simt_kernel<__nv_bfloat16>, (size_t)(smem));
         if (e != cudaSuccess) return e;
         select_simt_kernel<__nv_bfloat16><<<grid, 256, smem, st>>>(
-            (const __nv_bfloat16 *)q_slc, kbar, idx, w, sh.L, sh.hkv, sh.d, sh.nc, sh.K);
+            (const __nv_bfloat16 *)q_slc, kbar, idx, w, sh.L, sh.hkv, sh.d, sh.S, sh.nc, sh.K);
     } else {
         e = set_smem_once((const void *)select_simt_kernel<float>, (size_t)(smem));
         if (e != cudaSuccess) return e;
         select_simt_kernel<float><<<grid, 256, smem, st>>>((const float *)q_slc, kbar, idx, w, sh.L,
-                                                           sh.hkv, sh.d, sh.nc, sh.K);
+                                                           sh.hkv, sh.d, sh.S, sh.nc, sh.K);
     }
     return cudaGetLastError();
 }

@@ -417,7 +417,7 @@ cudaError_t launch_sel(const Shape &sh, const void *q_slc, const float *kbar, __
 }  // namespace
 
 bool select_tc_supported(const Shape &sh) {
-    return sh.bf16 && (sh.d == 64 || sh.d == 128) && sel_encode() != nullptr;
+    return sh.bf16 && sh.S == kChunk && (sh.d == 64 || sh.d == 128) && sel_encode() != nullptr;
 }
 
 cudaError_t launch_select_tc(const Shape &sh, const void *q_slc, const float *kbar, __nv_bfloat16 *hi,

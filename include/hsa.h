@@ -48,8 +48,10 @@
  * k, v, q_slc, o, dO, dq, dk, dv, dq_slc.  Arithmetic is fp32 (bf16 tensor-core
  * products accumulate in fp32); outputs are rounded once, to nearest even.
  *
- * Supported shapes: S = 64; d in {64, 128}; 1 <= K <= 16; h_q % h_kv == 0 and
- * h_q/h_kv <= 16; B >= 1, L >= 0; every pointer 16-byte aligned.
+ * Supported shapes: S in {16, 32, 64, 128}; d in {64, 128}; 1 <= K <= 16;
+ * h_q % h_kv == 0 and h_q/h_kv <= 16; B >= 1, L >= 0; every pointer 16-byte
+ * aligned.  The tensor-core kernels take S = 64 (the pages' chunk size); the
+ * other chunk sizes run on the CUDA-core kernels.
  *
  * Ownership: the caller owns every buffer (inputs, outputs, workspace); the
  * library never allocates, frees or synchronises -- each call only enqueues
@@ -83,7 +85,7 @@ extern "C" {
 typedef enum {
     HSA_OK = 0,
     HSA_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, inconsistent shape      */
-    HSA_ERR_UNSUPPORTED = 2,  /* valid but not built: S != 64, d not in {64,128}  */
+    HSA_ERR_UNSUPPORTED = 2,  /* valid but not built: S or d outside the above    */
     HSA_ERR_WORKSPACE = 3,    /* ws_bytes < hsa_workspace_size(shape, op)         */
     HSA_ERR_CUDA = 4,         /* a CUDA launch or API call failed                 */
     HSA_ERR_TIMEOUT = 5,      /* device status: a bounded wait ran out            */
@@ -98,7 +100,7 @@ typedef struct {
     int32_t h_q;   /* query heads                                            */
     int32_t h_kv;  /* KV heads = query groups                                */
     int32_t d;     /* head dimension                                         */
-    int32_t S;     /* chunk size (64, [P1 §limitations])                     */
+    int32_t S;     /* chunk size: 16, 32, 64 or 128 ([P1 §limitations] fixes 64) */
     int32_t K;     /* chunks selected per (token, group)                     */
     int32_t dtype; /* hsa_dtype_t of the token tensors                       */
 } hsa_shape_t;

@@ -58,8 +58,10 @@ def test_workspace_size_host_only(lib):
     fwd = lib.hsa_workspace_size(ctypes.byref(sh), OP_FWD)
     assert fwd >= 256 + 1 * 2 * 16 * 128 * 4 + 2 * 1024 * 2 * 8 * 4
     assert lib.hsa_workspace_size(ctypes.byref(sh), OP_BWD) > fwd
-    for bad in (dict(S=32), dict(d=96), dict(K=17), dict(h_q=15), dict(h_kv=0), dict(dtype=7)):
+    for bad in (dict(S=48), dict(S=8), dict(d=96), dict(K=17), dict(h_q=15), dict(h_kv=0), dict(dtype=7)):
         assert lib.hsa_workspace_size(ctypes.byref(_shape(**bad)), OP_FWD) == 0, bad
+    for S in (16, 32, 128):  # other chunk sizes run on the CUDA-core kernels
+        assert lib.hsa_workspace_size(ctypes.byref(_shape(S=S)), OP_FWD) > 256, S
     assert lib.hsa_workspace_size(ctypes.byref(sh), 99) == 0
 
 
@@ -75,7 +77,7 @@ def test_host_validation_without_gpu(lib):
     # misaligned input
     assert lib.hsa_pool(ctypes.byref(sh), odd, good, ws, 1 << 20, None) == 1
     # unsupported chunk size / head dim
-    assert lib.hsa_pool(ctypes.byref(_shape(S=32)), good, good, ws, 1 << 20, None) == 2
+    assert lib.hsa_pool(ctypes.byref(_shape(S=48)), good, good, ws, 1 << 20, None) == 2
     assert lib.hsa_fwd(ctypes.byref(_shape(d=80)), good, good, good, good, good, None, None, None,
                        None, ws, 1 << 30, None) == 2
     # h_q not a multiple of h_kv

@@ -537,6 +537,53 @@ def test_bwd_train_workload_full():
         assert_out(f64(g), r, "bf16", f"{name}[train16k]", grad=True)
 
 
+# --------------------------------------------------------------------------- other chunk sizes
+# The tensor-core kernels are built around the pages' 64-key chunk; S in {16, 32, 128}
+# runs on the CUDA-core kernels (pooling, selection, token-major attention, the decode
+# step and the two-phase backward).  (S, dtype, d, h_q, h_kv)
+S_CASES = [(16, "f32", 64, 8, 2), (32, "bf16", 128, 16, 2), (128, "bf16", 64, 8, 2),
+           (16, "bf16", 128, 4, 1), (128, "f32", 128, 8, 4)]
+
+
+@pytest.mark.parametrize("S,dtype,d,h_q,h_kv", S_CASES, ids=[f"S{c[0]}-{c[1]}-d{c[2]}" for c in S_CASES])
+def test_other_chunk_sizes_fwd_bwd(S, dtype, d, h_q, h_kv):
+    K = 4
+    wl = synth.Workload(f"s{S}", 2, S * 21 + 5, h_q, h_kv, d, S, K, dtype, "iid", "train", 300 + S + d)
+    x, kbar, sel = gap_ruled(wl)
+    m = hsa()
+    q, k, v, qs, dO = (to_dev(x[n], dtype) for n in ("q", "k", "v", "q_slc", "dO"))
+    assert np.array_equal(m.hsa_pool(k, S=S).cpu().numpy(), kbar)
+    o_ref, lse_ref, idx_ref, w_ref = oracle.fwd(x["q"], x["k"], x["v"], x["q_slc"], kbar, S, K)
+    o, lse, idx, w, kb = m.hsa_fwd(q, k, v, qs, K, S=S)
+    torch.cuda.synchronize()
+    assert np.array_equal(kb.cpu().numpy(), kbar)
+    assert np.array_equal(idx.cpu().numpy().reshape(idx_ref.shape), idx_ref)
+    assert np.abs(w.cpu().numpy().reshape(w_ref.shape) - w_ref).max() <= 1e-5
+    assert_out(f64(o).reshape(o_ref.shape), o_ref, dtype, f"o (S={S})")
+    assert np.abs(f64(lse).reshape(lse_ref.shape) - lse_ref).max() <= (1e-5 if dtype == "f32" else 2e-3)
+    assert not f64(o)[:, :S].any()
+    ref = oracle.bwd(x["q"], x["k"], x["v"], x["q_slc"], kbar, x["dO"], S, K)
+    got = m.hsa_bwd(q, k, v, qs, dO, lse, idx, w, kb, K, S=S)
+    torch.cuda.synchronize()
+    for name, g, r in zip(("dq", "dk", "dv", "dq_slc"), got, ref[:4]):
+        assert_out(f64(g), r, dtype, f"{name} (S={S})", grad=True)
+
+
+@pytest.mark.parametrize("S", [16, 32, 128])
+def test_decode_other_chunk_sizes(S):
+    wl = synth.Workload("dec", 3, S * 20 + 3, 8, 2, 64, S, 4, "bf16", "iid", "decode", 90 + S)
+    x, kbar, (o_ref, idx_ref, w_ref, gap) = gap_ruled(wl)
+    m = hsa()
+    kc, vc = to_dev(x["k"], "bf16"), to_dev(x["v"], "bf16")
+    kb = m.hsa_pool(kc, S=S)
+    assert np.array_equal(kb.cpu().numpy(), kbar)
+    o, idx, w = m.hsa_decode(to_dev(x["q"], "bf16"), to_dev(x["q_slc"], "bf16"), kc, vc, kb, wl.K, S=S)
+    torch.cuda.synchronize()
+    assert np.array_equal(idx.cpu().numpy(), idx_ref)
+    assert np.abs(w.cpu().numpy() - w_ref).max() <= 1e-5
+    assert_out(f64(o), o_ref, "bf16", f"decode o (S={S})")
+
+
 # --------------------------------------------------------------------------- status / errors
 def test_device_status_clean_and_bad_index_reported():
     """A corrupted chunk index (one that is not causally eligible) is caught on

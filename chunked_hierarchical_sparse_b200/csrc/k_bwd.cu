@@ -17,6 +17,7 @@
 //   dk (keys of chunk c) += dkbar_c / S        (mean pooling)
 // p is recomputed from the forward's lse: p_i = exp(x_i - lse).
 #include <algorithm>
+#include <type_traits>
 
 #include "hsa_internal.cuh"
 
@@ -306,24 +307,43 @@ __global__ void __launch_bounds__(kB2Threads) bwd_phase2_kernel(
 }
 
 // dk = dk_acc + dkbar_c / S; dv = dv_acc; rows of the trailing partial chunk = 0.
+// One thread per 4 consecutive values of a row (d is a multiple of 4); 1/S is exact
+// (S is a power of two), so the product equals the quotient.
+template <typename T>
+__device__ __forceinline__ void store4(T *p, float4 v) {
+    if constexpr (std::is_same<T, float>::value) {
+        *reinterpret_cast<float4 *>(p) = v;
+    } else {
+        __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+        uint2 u;
+        u.x = *reinterpret_cast<uint32_t *>(&a);
+        u.y = *reinterpret_cast<uint32_t *>(&b);
+        *reinterpret_cast<uint2 *>(p) = u;
+    }
+}
+
 template <typename T>
 __global__ void bwd_finish_kernel(const float *__restrict__ dk_acc, const float *__restrict__ dv_acc,
                                   const float *__restrict__ dkbar, T *__restrict__ dk, T *__restrict__ dv,
                                   int L, int d, int S, int nc, int64_t total) {
-    for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
-         e += (int64_t)gridDim.x * blockDim.x) {
-        const int j = (int)(e % d);
-        const int64_t r = e / d;
+    const int d4 = d / 4;
+    const float inv_s = 1.0f / (float)S;
+    for (int64_t e4 = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e4 < total / 4;
+         e4 += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = e4 / d4;  // row (b, g, t)
+        const int j = (int)(e4 - r * d4) * 4;
         const int t = (int)(r % L);
         const int64_t bg = r / L;
         const int c = t / S;
-        float a = 0.f, bv = 0.f;
+        float4 a = make_float4(0.f, 0.f, 0.f, 0.f), bv = a;
         if (c < nc) {
-            a = dk_acc[e] + dkbar[(bg * nc + c) * d + j] / S;
-            bv = dv_acc[e];
+            a = *reinterpret_cast<const float4 *>(dk_acc + e4 * 4);
+            const float4 kb = *reinterpret_cast<const float4 *>(dkbar + (bg * nc + c) * d + j);
+            a.x += kb.x * inv_s; a.y += kb.y * inv_s; a.z += kb.z * inv_s; a.w += kb.w * inv_s;
+            bv = *reinterpret_cast<const float4 *>(dv_acc + e4 * 4);
         }
-        Elem<T>::store(dk + e, a);
-        Elem<T>::store(dv + e, bv);
+        store4<T>(dk + e4 * 4, a);
+        store4<T>(dv + e4 * 4, bv);
     }
 }
 
@@ -349,7 +369,7 @@ static cudaError_t phase2_dispatch(const Shape &sh, const void *q, const void *k
         if (e != cudaSuccess) return e;
     }
     const int64_t total = (int64_t)sh.B * sh.hkv * sh.L * sh.d;
-    const int blocks = (int)std::min<int64_t>(ceil_div(total, 256), 148 * 16);
+    const int blocks = (int)std::min<int64_t>(ceil_div(total / 4, 256), 148 * 16);
     bwd_finish_kernel<T><<<blocks, 256, 0, st>>>(ws.dk_acc, ws.dv_acc, ws.dkbar, (T *)dk, (T *)dv,
                                                   sh.L, sh.d, sh.S, sh.nc, total);
     return cudaGetLastError();
@@ -359,7 +379,7 @@ template <typename T>
 static cudaError_t finish_dispatch(const Shape &sh, const BwdWs &ws, void *dk, void *dv, cudaStream_t st) {
     const int64_t total = (int64_t)sh.B * sh.hkv * sh.L * sh.d;
     if (total == 0) return cudaSuccess;
-    const int blocks = (int)std::min<int64_t>(ceil_div(total, 256), 148 * 16);
+    const int blocks = (int)std::min<int64_t>(ceil_div(total / 4, 256), 148 * 16);
     bwd_finish_kernel<T><<<blocks, 256, 0, st>>>(ws.dk_acc, ws.dv_acc, ws.dkbar, (T *)dk, (T *)dv, sh.L, sh.d,
                                                   sh.S, sh.nc, total);
     return cudaGetLastError();

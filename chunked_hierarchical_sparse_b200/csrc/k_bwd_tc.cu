@@ -781,6 +781,18 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
 }
 
 // ------------------------------------------------------------------ stick-breaking backward
+// The D / 32 consecutive fp32 values of lane `lane` of a d = D row (one vector load).
+template <int D>
+__device__ __forceinline__ void lane_cols_f32(const float *row, int lane, float (&f)[D / 32]) {
+    if constexpr (D == 128) {
+        const float4 v = *reinterpret_cast<const float4 *>(row + lane * 4);
+        f[0] = v.x; f[1] = v.y; f[2] = v.z; f[3] = v.w;
+    } else {
+        const float2 v = *reinterpret_cast<const float2 *>(row + lane * 2);
+        f[0] = v.x; f[1] = v.y;
+    }
+}
+
 // The D / 32 consecutive bf16 values of lane `lane` of a d = D row, as floats.
 template <int D>
 __device__ __forceinline__ void lane_cols(const __nv_bfloat16 *row, int lane, float (&f)[D / 32]) {
@@ -830,7 +842,8 @@ __global__ void __launch_bounds__(256) bwd_select_kernel(const __nv_bfloat16 *__
     for (int k = 0; k < K; ++k) {
         const int c = __shfl_sync(0xffffffffu, ck, k);
         if (c < 0) continue;  // an empty or ineligible slot: score and gradient stay 0
-        const float *kr = kbar + (bg * nc + c) * D + lane * NC;
+        float kr[NC];
+        lane_cols_f32<D>(kbar + (bg * nc + c) * D, lane, kr);
         float a = 0.f;
 #pragma unroll
         for (int e = 0; e < NC; ++e) a = fmaf(qv[e], kr[e], a);
@@ -855,7 +868,8 @@ __global__ void __launch_bounds__(256) bwd_select_kernel(const __nv_bfloat16 *__
         const int c = __shfl_sync(0xffffffffu, ck, k);
         if (c < 0) continue;
         const float dsj = __shfl_sync(0xffffffffu, dsk, k) * scale;
-        const float *kr = kbar + (bg * nc + c) * D + lane * NC;
+        float kr[NC];
+        lane_cols_f32<D>(kbar + (bg * nc + c) * D, lane, kr);
 #pragma unroll
         for (int e = 0; e < NC; ++e) dqv[e] = fmaf(dsj, kr[e], dqv[e]);
     }

@@ -517,7 +517,7 @@ def main():
     sets = [dict(q=q, k=k, v=v, q_slc=qs, o=o, ws=ws)]
     sets.append({n: torch.empty_like(t_) for n, t_ in sets[0].items()})
     s_up, s_fw, s_dn = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
-    n_e2e = 6
+    n_e2e = 12  # the pipeline's fill (first upload) and drain (last read-back) spread over 12 steps
 
     def pipeline(n):
         ev = lambda: torch.cuda.Event(enable_timing=True)

@@ -404,6 +404,8 @@ def main():
     ap.add_argument("--no-cpu", action="store_true", help="skip the oracle CPU baseline")
     ap.add_argument("--decode-only", action="store_true",
                     help="time only the decode16k step (one GPU; the case used for ncu captures of the decode kernel)")
+    ap.add_argument("--train-only", action="store_true",
+                    help="time only the train16k step (one GPU; the case used for ncu captures of the backward)")
     ap.add_argument("--workload", default="fwd64k", choices=["fwd64k", "fwd16k"],
                     help="forward workload (fwd16k: the smaller case used for ncu captures)")
     args = ap.parse_args()
@@ -426,9 +428,10 @@ def main():
     dev = torch.device("cuda", local if world > 1 else 0)
     torch.cuda.set_device(dev)
     hsa.load_library()
-    if args.decode_only:
+    if args.decode_only or args.train_only:
         if rank == 0:
-            print(json.dumps({"decode": bench_decode(hsa, dev)}), flush=True)
+            key, fn = ("decode", bench_decode) if args.decode_only else ("train", bench_train)
+            print(json.dumps({key: fn(hsa, dev)}), flush=True)
         dist_util.finish(world)
         return
 

@@ -202,7 +202,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_tc_kernel(
         acc_inv = __int_as_float((127 - ev) << 23);
     }
 
-    // every lane waits (converged, sleeping in try_wait); the warp's verdict is a vote
+    // every lane waits (converged, sleeping in try_wait); the warp decides by a vote
     auto warp_wait = [&](uint64_t *b, uint32_t par) -> bool {
         return __all_sync(0xffffffffu, mbar_wait(b, par, wait_ns));
     };

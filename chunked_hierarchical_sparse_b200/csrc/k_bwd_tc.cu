@@ -221,7 +221,7 @@ __global__ void __launch_bounds__(kBThreads, 1) bwd_tc_kernel(
         acc_inv = __int_as_float((127 - ev) << 23);
     }
 
-    auto warp_wait = [&](uint64_t *b, uint32_t par) -> bool {  // every lane waits; the verdict is a vote
+    auto warp_wait = [&](uint64_t *b, uint32_t par) -> bool {  // every lane waits; the warp decides by a vote
         return __all_sync(0xffffffffu, mbar_wait(b, par, wait_ns));
     };
 

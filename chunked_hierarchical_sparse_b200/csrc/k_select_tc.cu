@@ -169,7 +169,7 @@ __global__ void __launch_bounds__(kSelThreads, 2) select_tc_kernel(
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
 
-    // every lane waits (converged, sleeping in try_wait); the warp's verdict is a vote
+    // every lane waits (converged, sleeping in try_wait); the warp decides by a vote
     auto warp_wait = [&](uint64_t *bb, uint32_t par) -> bool {
         return __all_sync(0xffffffffu, mbar_wait(bb, par, wait_ns));
     };

@@ -366,6 +366,36 @@ def test_decode_small_edges(P):
     assert_out(f64(o), o_ref, "f32", "o")
 
 
+# the cluster kernel's other shapes: bf16 d = 64 (tensor-core chunk attention at d = 64),
+# 16 query heads per group (the MMA's 16 rows all used), fp32 with 16 heads; one and two layers
+DEC_SHAPES = [("bf16", 64, 16, 2), ("bf16", 128, 16, 1), ("f32", 128, 16, 1), ("bf16", 64, 8, 1)]
+
+
+@pytest.mark.parametrize("dtype,d,h_q,h_kv", DEC_SHAPES, ids=["bf16-d64-g8", "bf16-d128-g16", "f32-d128-g16",
+                                                             "bf16-d64-g8-hkv1"])
+@pytest.mark.parametrize("NL", [1, 2])
+def test_decode_cluster_shapes(dtype, d, h_q, h_kv, NL):
+    wl = synth.Workload("decs", 3, 64 * 57 + 21, h_q, h_kv, d, 64, 8, dtype, "iid", "decode", 60 + d + h_q)
+    x, kbar, (o_ref, idx_ref, w_ref, gap) = gap_ruled(wl)
+    m = hsa()
+    kc, vc = to_dev(x["k"], dtype), to_dev(x["v"], dtype)
+    kb = torch.from_numpy(kbar).to(DEV)
+    qsl = to_dev(x["q_slc"], dtype)
+    qs_np = synth.layer_queries(wl, NL)
+    m.hsa_timing_enable(True)
+    o, idx, w = m.hsa_decode_multi(to_dev(qs_np, dtype), qsl, kc, vc, kb, wl.K)
+    _, n_launch = m.hsa_timing_read("decode")
+    m.hsa_timing_enable(False)
+    torch.cuda.synchronize()
+    assert n_launch == 1, "the cluster kernel did not take the call"
+    assert np.array_equal(idx.cpu().numpy(), idx_ref)
+    assert np.abs(w.cpu().numpy() - w_ref).max() <= 1e-5
+    for l in range(NL):
+        o_l, i_l, _, _ = oracle.decode(qs_np[l], x["q_slc"], x["k"], x["v"], kbar, wl.S, wl.K)
+        assert np.array_equal(i_l, idx_ref)
+        assert_out(f64(o[l]), o_l, dtype, f"decode o[layer {l}] ({dtype} d={d} G={h_q // h_kv})")
+
+
 def test_decode_offloaded_cache_workload():
     """KV cache in page-locked host memory: only the selected chunks cross the host
     link.  Same kernel and data as the device-cache run, so the same bits."""

@@ -160,12 +160,9 @@ cudaError_t launch_bwd_phase2(const Shape &sh, const void *q, const void *k, con
                               const void *dO, const float *lse, const float *w, void *dk, void *dv,
                               const BwdWs &ws, DevStatus *ds, cudaStream_t st);
 
-#ifndef HSA_INV_BLOCK
-#define HSA_INV_BLOCK 128
-#endif
 // tokens per histogram block of the inversion: the scatter walks a block's tokens
 // in order (one warp); the histogram holds ceil(L / block) x n_c counts per (b, g)
-constexpr int kInvTokBlock = HSA_INV_BLOCK;
+constexpr int kInvTokBlock = 128;
 constexpr int kBwdSeg = 32;        // list entries per phase-2 block
 
 // ---------------------------------------------------------------- chunk-major forward plan
@@ -174,19 +171,11 @@ constexpr int kCombTokens = 16;    // tokens per combine item
 // Accumulators of the chunk-major passes: a ring of kRing window slots, each
 // a [W tokens][G heads][d] block of scaled fp16 sums that the tiles of one
 // window reduce their weighted outputs (forward) or dq rows (backward) into
-// (compile-time tunables; the ring stays resident in L2 next to the K/V and
-// query working set).
-#ifndef HSA_ACC_RING
-#define HSA_ACC_RING 2
-#endif
-#ifndef HSA_ACC_SLOT_MB
-#define HSA_ACC_SLOT_MB 32
-#endif
-#ifndef HSA_MAX_WINDOW
-#define HSA_MAX_WINDOW 16384
-#endif
-constexpr int kRing = HSA_ACC_RING;
-constexpr size_t kAccSlotBudget = size_t(HSA_ACC_SLOT_MB) << 20;
+// (two 32 MiB slots: the ring stays resident in L2 next to the K/V and query
+// working set; smaller slots and a third slot were measured slower at 64K).
+constexpr int kRing = 2;
+constexpr size_t kAccSlotBudget = size_t(32) << 20;
+constexpr int kMaxWindow = 16384;  // tokens per window at most
 
 struct AttendPlan {
     int B, L, hq, hkv, D, K, G, nc, ntb, W, nW, J, TT;
@@ -230,7 +219,7 @@ inline int attend_window(int G, int d, int esize) {
     const int64_t per_tok = (int64_t)G * d * esize;
     int64_t w = (int64_t)(kAccSlotBudget / per_tok) / kInvTokBlock * kInvTokBlock;
     if (w < kInvTokBlock) w = kInvTokBlock;
-    if (w > HSA_MAX_WINDOW) w = HSA_MAX_WINDOW;
+    if (w > kMaxWindow) w = kMaxWindow;
     return (int)w;
 }
 

@@ -45,11 +45,8 @@ using namespace sm100;
 namespace {
 
 
-#ifndef HSA_BEPI_UNROLL
-#define HSA_BEPI_UNROLL 1
-#endif
 // unrolling of the epilogue's column loops: rolled, the roles' hot code fits the instruction cache
-constexpr int kBEpiUnroll = HSA_BEPI_UNROLL;
+constexpr int kBEpiUnroll = 1;
 
 constexpr int kBThreads = 384;
 constexpr int kBWarpEpi = 4, kBWarpConv = 8, kBWarpProd = 10, kBWarpMma = 11;
